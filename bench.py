@@ -1,0 +1,382 @@
+"""DCKV codec benchmark on B200: encode + decode throughput of a 4,096-token prompt.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--impl dckv|reference] [--config c2|c1|c3|c3b|c4|c5]
+
+A step is one pass of the whole codec hot path over one batch: encode (transform GEMMs,
+quantiser, mean models, rANS, compaction) then decode (two rANS passes, odd mean model,
+inverse GEMM with RoPE and scatter).  value = prompt tokens per second through that
+round trip, inputs resident in HBM.  Per-stage device times come from CUDA events the
+library records on its launch stream.  Under torchrun each rank codes its own prompt
+(replicas, weak scaling; no data-path collective) and the slowest rank's time is used.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+CONFIGS = {
+    # name: (prompt lengths, target bytes/token (None = literal small codec), student-t fraction, description)
+    "c1": ([256], None, 0.0, "1 x 256-token prompt (124 coded rows), literal codec b = 0.6 Delta"),
+    "c2": ([4096], 220.0, 0.0, "1 x 4096-token prompt, 6144-dim bf16 rows, step scale for ~220 B/token"),
+    "c3": ([32768], 220.0, 0.0, "1 x 32768-token prompt, ~220 B/token"),
+    "c3b": ([32768], 110.0, 0.0, "1 x 32768-token prompt, ~110 B/token (many components dropped)"),
+    "c4": ([131072], 220.0, 0.0, "1 x 131072-token prompt, ~220 B/token"),
+    "c5": ([4096] * 64, 220.0, 0.01, "64 x 4096-token prompts, 1% Student-t (nu=2) rows, ~220 B/token"),
+}
+
+GEMM_STAGES = {"gemm_hidden", "gemm_transform", "gemm_mean_odd", "gemm_inverse"}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+class ClockSampler:
+    def __init__(self, index=0):
+        self.proc = None
+        self.path = None
+        self.index = index
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for name, val in zip(names, r[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def make_inputs(cfg_name, rank, device):
+    import dckv_synth as S
+
+    lens, target, st, _ = CONFIGS[cfg_name]
+    src = S.source(0)
+    if target is None:
+        cod = S.codec(src, step_scale=1.0, literal_b=True)
+    else:
+        cod = S.codec(src, step_scale=None, target_bytes=target)
+    seeds = [1000 * rank + i for i in range(len(lens))]
+    x, tok, offs = S.batch(src, lens, seeds, student_t_frac=st, device=device)
+    return src, cod, x, tok, offs
+
+
+def oracle_sample(cod, x_cpu_bits, tok_cpu, n_rows):
+    """Oracle encode + decode of the first n_rows coded rows of the prompt (plus its kept
+    rows), timed on the host cores.  Returns (seconds, tokens processed)."""
+    import oracle as O
+
+    N = min(x_cpu_bits.shape[0], n_rows + 132)
+    xs = x_cpu_bits[:N]
+    ts = tok_cpu[:N]
+    offs = np.array([0, N], np.int64)
+    t0 = time.perf_counter()
+    blob = O.encode(xs, ts, offs, cod)
+    O.decode(blob, ts, offs, cod)
+    return time.perf_counter() - t0, N
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+def run_reference(args):
+    """The oracle, as it stands, on the host cores: the reference arm of this benchmark."""
+    ws, rank, local = dist_env()
+    if rank != 0:
+        return 0
+    import torch
+
+    _, cod, x, tok, offs = make_inputs(args.config, 0, "cpu")
+    xb = x.view(torch.int16).numpy().view(np.uint16)
+    tk = tok.numpy()
+    rows = args.reference_rows
+    for _ in range(args.warmup if args.warmup < 1 else 1):
+        oracle_sample(cod, xb, tk, min(rows, 32))
+    times = []
+    toks = 0
+    for _ in range(args.steps):
+        dt, n = oracle_sample(cod, xb, tk, rows)
+        times.append(dt)
+        toks = n
+    mean = statistics.mean(times)
+    value = toks / mean
+    lens, _, _, desc = CONFIGS[args.config]
+    line = {
+        "metric": "decode & encode tokens/s (6144-dim rows) at 1 B200; bytes/token; % roofline",
+        "impl": "reference", "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": mean * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": desc, "sample": f"first {toks} tokens of the prompt ({toks - 132} coded rows)"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": host_cores(), "kind": "oracle",
+                         "sample": f"encode+decode of {toks} tokens per step"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_gpu(args):
+    import torch
+
+    import learned_kv_cache_dckv_b200 as D
+
+    ws, rank, local = dist_env()
+    dist = None
+    if ws > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    _, cod, x, tok, offs = make_inputs(args.config, rank, dev)
+    n_tok = int(offs[-1])
+    n_rows = sum(max(0, int(n) - 132) for n in np.diff(offs))
+    gc = D.Codec(D.upload_params(cod, dev), dev.index)
+    stream = torch.cuda.current_stream()
+    blob = torch.empty(D.dckv_blob_bound(gc.handle, offs), dtype=torch.uint8, device=dev)
+    k_out = torch.empty((6, n_tok, 2, 256), dtype=torch.bfloat16, device=dev)
+    v_out = torch.empty_like(k_out)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    # warm-up (also learns the blob size once)
+    for _ in range(max(1, args.warmup)):
+        gc.encode(x, tok, offs, blob=blob)
+        torch.cuda.synchronize()
+        size = int(gc.blob_size.item())
+        gc.decode(blob, size, tok, offs, k_out, v_out)
+    torch.cuda.synchronize()
+    st = int(gc.status.item())
+    if st != D.DCKV_OK:
+        raise RuntimeError(f"codec status {D.STATUS_NAMES[st]}")
+    size = int(gc.blob_size.item())
+
+    # timed region: K steps, per-step events, L2 flushed between steps (outside the events)
+    stage_ms = {}
+    step_ms, enc_ms, dec_ms = [], [], []
+    sampler = ClockSampler(dev.index)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    wall0 = time.perf_counter()
+    for it in range(args.steps):
+        flush.fill_(it & 0xFF)
+        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        D.dckv_set_timing(gc.handle, True)
+        e0.record(stream)
+        gc.encode(x, tok, offs, blob=blob)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        for name, ms in D.dckv_get_timing(gc.handle):
+            stage_ms.setdefault("enc:" + name, []).append(ms)
+        flush.fill_((it + 1) & 0xFF)
+        e1b = torch.cuda.Event(enable_timing=True)
+        e1b.record(stream)
+        gc.decode(blob, size, tok, offs, k_out, v_out)
+        e2.record(stream)
+        torch.cuda.synchronize()
+        for name, ms in D.dckv_get_timing(gc.handle):
+            stage_ms.setdefault("dec:" + name, []).append(ms)
+        enc_ms.append(e0.elapsed_time(e1))
+        dec_ms.append(e1b.elapsed_time(e2))
+        step_ms.append(enc_ms[-1] + dec_ms[-1])
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - wall0
+    clocks = sampler.stop()
+    D.dckv_set_timing(gc.handle, False)
+    st = int(gc.status.item())
+    if st != D.DCKV_OK:
+        raise RuntimeError(f"codec status {D.STATUS_NAMES[st]}")
+
+    ms_step = statistics.mean(step_ms)
+    ms_enc = statistics.mean(enc_ms)
+    ms_dec = statistics.mean(dec_ms)
+    if dist:
+        t = torch.tensor([ms_step, ms_enc, ms_dec], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step, ms_enc, ms_dec = t.tolist()
+
+    # end to end through the public API with host buffers: H2D rows + ids, encode,
+    # D2H blob; H2D blob, decode, D2H K and V -- all inside the timed region
+    x_h = x.cpu().pin_memory()
+    tok_h = tok.cpu().pin_memory()
+    blob_h = torch.empty(size, dtype=torch.uint8).pin_memory()
+    k_h = torch.empty(k_out.shape, dtype=torch.bfloat16).pin_memory()
+    v_h = torch.empty_like(k_h).pin_memory()
+    x_d = torch.empty_like(x)
+    tok_d = torch.empty_like(tok)
+    blob_d2 = torch.empty_like(blob)
+    e2e_ms = []
+    for it in range(max(2, args.steps // 2) + 1):
+        flush.fill_(it & 0xFF)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        x_d.copy_(x_h, non_blocking=True)
+        tok_d.copy_(tok_h, non_blocking=True)
+        gc.encode(x_d, tok_d, offs, blob=blob)
+        blob_h.copy_(blob[:size], non_blocking=True)
+        blob_d2[:size].copy_(blob_h, non_blocking=True)
+        gc.decode(blob_d2, size, tok_d, offs, k_out, v_out)
+        k_h.copy_(k_out, non_blocking=True)
+        v_h.copy_(v_out, non_blocking=True)
+        b.record(stream)
+        torch.cuda.synchronize()
+        if it > 0:
+            e2e_ms.append(a.elapsed_time(b))
+    h2d = x.numel() * 2 + tok.numel() * 4 + size
+    d2h = size + 2 * k_out.numel() * 2
+    ms_e2e = statistics.mean(e2e_ms)
+    if dist:
+        t = torch.tensor([ms_e2e], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_e2e = t.item()
+
+    # roofline of the dominant kernel (largest mean stage time among the GEMMs)
+    peaks, peak_kind = load_peaks()
+    means = {k: statistics.mean(v) for k, v in stage_ms.items()}
+    n_even = sum((max(0, int(n) - 132) + 1) // 2 for n in np.diff(offs))
+    n_odd = n_rows - n_even
+    k_eff = gc.k_eff
+    algo_flops = {  # algorithmic (unsplit) FLOPs per launch
+        "enc:gemm_hidden": 2.0 * n_rows * 6144 * 256,
+        "enc:gemm_transform": 2.0 * n_rows * (6144 * 2048 + 256 * 2048),
+        "enc:gemm_mean_odd": 2.0 * n_odd * 4096 * 2048,
+        "dec:gemm_mean_odd": 2.0 * n_odd * 4096 * 2048,
+        "dec:gemm_inverse": 2.0 * n_rows * 2048 * 6144,
+    }
+    issued_flops = {  # what the tensor pipe executes (split operands, padded tiles)
+        "enc:gemm_hidden": 2.0 * 2 * (-(-n_rows // 128) * 128) * 6144 * 256,
+        "enc:gemm_transform": 2.0 * (-(-n_rows // 256) * 256) * (2 * 6144 * 2048 + 4 * 256 * 2048),
+        "enc:gemm_mean_odd": 2.0 * (-(-(n_even + len(offs) - 1) // 256) * 256) * 4096 * 2048,
+        "dec:gemm_mean_odd": 2.0 * (-(-(n_even + len(offs) - 1) // 256) * 256) * 4096 * 2048,
+        "dec:gemm_inverse": 2.0 * 2 * (-(-n_rows // 256) * 256) * 2048 * 6144,
+    }
+    dom = max(algo_flops, key=lambda k: means.get(k, 0.0))
+    peak = float(peaks.get("bf16_tflops", 1590.0))
+    achieved = algo_flops[dom] / (means[dom] * 1e-3) / 1e12
+    roofline = {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "peak_source": f"{peak_kind} dense bf16 (fp16 operands run at the same rate)",
+                "issued_frac": issued_flops[dom] / (means[dom] * 1e-3) / 1e12 / peak,
+                "traffic": None}
+
+    tokens = n_tok
+    value = tokens * ws / (ms_step * 1e-3)
+    lens, target, stf, desc = CONFIGS[args.config]
+    payload = size - sum(min(int(n), 132) for n in np.diff(offs)) * 12288
+    line = {
+        "metric": "decode & encode tokens/s (6144-dim rows) at 1 B200; bytes/token; % roofline",
+        "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp16", "data": "synthetic",
+        "config": {"workload": desc, "prompts": len(lens), "seq_len": lens[0], "tokens_per_step": tokens,
+                   "coded_rows": n_rows, "step_scale": cod.step_scale, "k_eff": k_eff,
+                   "l2": "256 MiB buffer written between encode and decode and between steps (outside the events)",
+                   "arith": "fp16 split operands, fp32 TMEM accumulation; rANS in u32",
+                   "parallelism": f"replicas x{ws}"},
+        "encode_tokens_per_s": tokens * ws / (ms_enc * 1e-3),
+        "decode_tokens_per_s": tokens * ws / (ms_dec * 1e-3),
+        "encode_ms": ms_enc, "decode_ms": ms_dec,
+        "bytes_per_token": payload / max(n_rows, 1),
+        "compression_vs_bf16": 12288.0 * n_rows / max(payload, 1),
+        "stage_ms": {k: round(v, 5) for k, v in sorted(means.items())},
+        "roofline": roofline,
+        "e2e": {"value": tokens * ws / (ms_e2e * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": 16 * args.steps,
+        "wall_s_timed_region": wall,
+        "clocks": clocks,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        xb = x.cpu().view(torch.int16).numpy().view(np.uint16)
+        dt, ntok = oracle_sample(cod, xb, tok.cpu().numpy(), args.reference_rows)
+        line["cpu_baseline"] = {"value": ntok / dt, "unit": "tokens/s", "cores": host_cores(), "kind": "oracle",
+                                "sample": f"oracle encode+decode of the first {ntok} tokens ({ntok - 132} coded rows)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    gc.close()
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="dckv", choices=["dckv", "reference"])
+    ap.add_argument("--config", default="c2", choices=sorted(CONFIGS))
+    ap.add_argument("--reference-rows", type=int, default=1024)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,61 @@
+/*
+ * dckv_inspect.h -- inspection and self-test entry points of the DCKV library.
+ *
+ * These calls expose intermediates (workspace layout, derived tables, per-stage device
+ * times) and the raw tcgen05 GEMM, so that tests can compare each stage with an
+ * independent reference and benchmarks can attribute time to kernels.  They are not
+ * needed to encode or decode.  Same conventions as dckv.h: device pointers are
+ * caller-owned, calls are ordered on the given stream.
+ */
+#ifndef DCKV_INSPECT_H_
+#define DCKV_INSPECT_H_
+
+#include "dckv.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Byte offsets (from the workspace base) of the intermediates of one call shape.
+ * which = 0: encode layout, 1: decode layout.  After dckv_encode on a stream:
+ *   q32  int32 [n_rows][2048] codes q = round(y / Delta) (0 for dropped components),
+ *        rows in prompt order, coded rows only (positions 4 .. N-129 of each prompt);
+ *   qe   bf16 [ne_pad][2048] even-row codes, one extra zero row after each prompt;
+ *   c_odd int8 [ne_pad][2048] centres of the odd row whose left neighbour is that row.
+ * After dckv_decode: q16 fp16 [n_rows][2048] decoded codes (exact below 2048), qe, c_odd. */
+typedef struct {
+  uint64_t q32, qe, c_odd, q16, x16, g16;
+  int64_t n_rows, ne_pad;
+  int32_t n_chunks;
+  uint64_t total;
+} dckv_ws_view;
+
+int dckv_ws_offsets(const dckv_codec *codec, const int64_t *seq_offsets, int batch, int which, dckv_ws_view *out);
+
+/* Copy the derived tables to host memory (any pointer may be NULL):
+ *   cdf   uint16 [64][510] cumulative frequencies per scale index (cdf[510] = 65536);
+ *   scale uint8 [2048] scale index s_c;  keep uint8 [2048] 1 = coded;
+ *   exps  int32 [3] power-of-two operand scales (transform, correction, inverse).
+ * Synchronises the device. */
+int dckv_codec_export(const dckv_codec *codec, uint16_t *cdf, uint8_t *scale, uint8_t *keep, int32_t *exps);
+
+/* Device pointers of the per-vocabulary mean tables (fp32 [vocab][2048]):
+ * t_even = embed @ w_even, t_odd = embed @ w_odd[0:2048]. */
+int dckv_codec_tables(const dckv_codec *codec, const void **t_even, const void **t_odd);
+
+/* Per-stage device times of the last encode / decode issued with timing enabled.
+ * Events are recorded on the call's stream; read after synchronising it.  Returns the
+ * number of stages written to ms / names (at most max). */
+int dckv_set_timing(dckv_codec *codec, int enable);
+int dckv_get_timing(const dckv_codec *codec, float *ms, const char **names, int max);
+
+/* Self-test of the tcgen05 GEMM core: D[n][m] = sum_s sum_k A[s][m][k] * B[n][k]
+ * (fp32 accumulate).  A: device fp16/bf16 [slabs][M][K]; B: device [N][K]; D: device
+ * fp32 [N][M].  M % 128 == 0, K % 64 == 0, slabs in {1, 2}, bn (N tile) in 16..256 step 16. */
+int dckv_debug_gemm(int bf16, const void *A, int slabs, const void *B, int M, int N, int K, float *D, int bn,
+                    void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DCKV_INSPECT_H_ */

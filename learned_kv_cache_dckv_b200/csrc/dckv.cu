@@ -1,0 +1,1153 @@
+// dckv.cu -- the DCKV codec library for B200 (sm_100a): codec setup, encode, decode,
+// byte accounting, behind the C ABI declared in include/dckv.h.
+//
+// Method: "DCKV: Learned Transform Coding of the Prompt KV Cache in Hybrid Language
+// Models" (trove.briskstack.com summary), section "How it works" -- row assembly and
+// kept rows (first paragraph), transform / drop rule ("Transform"), rANS under Laplace
+// with 64-bit escapes ("Coding"), checkerboard conditional means ("Conditional entropy
+// models"), RoPE reapplied after decoding (first paragraph).
+//
+// Encode:  rows --convert--> fp16 coded rows (+ kept rows into the blob)
+//          --GEMM H (tcgen05, GELU epilogue)--> correction hidden units (fp16 hi/lo)
+//          --GEMM Y (tcgen05, quantise epilogue)--> int32 codes, bf16 even codes
+//          --GEMM odd mean (tcgen05, centre epilogue)--> odd centres
+//          --rANS encode (one warp per chunk)--> words --scan--> chunk table, header
+//          --compaction--> chunk sections
+// Decode:  header check --rANS even--> even codes --GEMM odd mean--> odd centres
+//          --rANS odd--> odd codes --GEMM inverse (RoPE + scatter epilogue)--> K, V
+//          (+ kept rows with RoPE, + exact fix-up of rows holding codes beyond +-2047)
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "../../include/dckv_inspect.h"
+#include "dckv_epilogues.cuh"
+#include "dckv_gemm.cuh"
+#include "dckv_internal.cuh"
+#include "dckv_rans.cuh"
+
+using namespace dckv;
+
+// ============================================================================ errors
+static thread_local char g_err[512] = "";
+
+static int fail(int code, const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+#define CK(x)                                                                           \
+  do {                                                                                  \
+    cudaError_t e_ = (x);                                                               \
+    if (e_ != cudaSuccess) return fail(DCKV_ECUDA, "%s: %s", #x, cudaGetErrorString(e_)); \
+  } while (0)
+
+#define RET(x)                   \
+  do {                           \
+    int r_ = (x);                \
+    if (r_ != DCKV_OK) return r_; \
+  } while (0)
+
+extern "C" const char *dckv_last_error(void) { return g_err; }
+
+// ============================================================================ tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// A operand: [slabs][M][K] (K contiguous), box {64, 128, box_slabs}, 128-byte swizzle.
+static int map_a(CUtensorMap *m, const void *ptr, bool bf16, uint64_t K, uint64_t M, uint64_t slabs, int box_slabs) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(DCKV_ECUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[3] = {K, M, slabs};
+  cuuint64_t strides[2] = {K * 2, K * M * 2};
+  cuuint32_t box[3] = {(cuuint32_t)GEMM_BK, (cuuint32_t)GEMM_BM, (cuuint32_t)box_slabs};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+                  const_cast<void *>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(DCKV_ECUDA, "tensor map (A) encode failed: %d", (int)r);
+  return DCKV_OK;
+}
+
+// B operand: [rows][K] (K contiguous), box {64, bn}, 128-byte swizzle, zero fill past the end.
+static int map_b(CUtensorMap *m, const void *ptr, bool bf16, uint64_t K, uint64_t rows, int bn) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(DCKV_ECUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[2] = {K, rows};
+  cuuint64_t strides[1] = {K * 2};
+  cuuint32_t box[2] = {(cuuint32_t)GEMM_BK, (cuuint32_t)bn};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                  const_cast<void *>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(DCKV_ECUDA, "tensor map (B) encode failed: %d", (int)r);
+  return DCKV_OK;
+}
+
+// ============================================================================ GEMM launch
+template <class Epi, int STAGES, int MAX_SLABS>
+static int run_gemm(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &b0, const CUtensorMap &b1,
+                    const GemmProblem &prob, const typename Epi::Params &ep, int num_sms, cudaStream_t st) {
+  constexpr int smem = gemm_smem_bytes<Epi, STAGES, MAX_SLABS>();
+  static_assert(smem <= 232448, "GEMM shared memory above the sm_100 limit");
+  auto kern = gemm_kernel<Epi, STAGES, MAX_SLABS>;
+  CK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  const int tiles = prob.m_tiles * prob.n_tiles;
+  if (tiles <= 0) return DCKV_OK;
+  for (int i = 0; i < prob.n_seg; ++i)
+    if (prob.seg[i].n_slab < 1 || prob.seg[i].n_slab > MAX_SLABS) return fail(DCKV_EINVAL, "bad slab count");
+  const int grid = std::min(tiles, num_sms);
+  kern<<<grid, GEMM_THREADS, smem, st>>>(a0, a1, b0, b1, prob, ep);
+  CK(cudaGetLastError());
+  return DCKV_OK;
+}
+
+template <class Epi, int STAGES, int MAX_SLABS, int CHUNK_STEPS>
+static int run_gemm_chunked(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &b0,
+                            const CUtensorMap &b1, const GemmProblem &prob, const typename Epi::Params &ep,
+                            int num_sms, cudaStream_t st) {
+  constexpr int smem = gemm_chunked_smem_bytes<STAGES, MAX_SLABS>();
+  static_assert(smem <= 232448, "GEMM shared memory above the sm_100 limit");
+  auto kern = gemm_chunked_kernel<Epi, STAGES, MAX_SLABS, CHUNK_STEPS>;
+  CK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  const int tiles = prob.m_tiles * prob.n_tiles;
+  if (tiles <= 0) return DCKV_OK;
+  if (prob.bn != GEMM_MAX_BN) return fail(DCKV_EINVAL, "chunked GEMM needs bn = 256");
+  for (int i = 0; i < prob.n_seg; ++i)
+    if (prob.seg[i].n_slab < 1 || prob.seg[i].n_slab > MAX_SLABS) return fail(DCKV_EINVAL, "bad slab count");
+  const int grid = std::min(tiles, num_sms);
+  kern<<<grid, GEMMC_THREADS, smem, st>>>(a0, a1, b0, b1, prob, ep);
+  CK(cudaGetLastError());
+  return DCKV_OK;
+}
+
+static GemmProblem make_problem(int m_tiles, int64_t n_rows, int bn, bool bf16, int32_t *status) {
+  GemmProblem p;
+  memset(&p, 0, sizeof(p));
+  p.m_tiles = m_tiles;
+  p.n_rows = (int)n_rows;
+  p.bn = bn;
+  p.n_tiles = (int)((n_rows + bn - 1) / bn);
+  p.idesc = idesc_f16(bf16 ? 1 : 0, GEMM_BM, bn);
+  p.status = status;
+  return p;
+}
+
+static void add_seg(GemmProblem &p, int a_map, int a_slab0, int n_slab, int a_k0, int b_map, int b_row_shift, int b_k0,
+                    int k_steps) {
+  GemmSeg &s = p.seg[p.n_seg++];
+  s.a_map = a_map;
+  s.a_slab0 = a_slab0;
+  s.n_slab = n_slab;
+  s.a_k0 = a_k0;
+  s.b_map = b_map;
+  s.b_row_shift = b_row_shift;
+  s.b_k0 = b_k0;
+  s.k_steps = k_steps;
+}
+
+// ============================================================================ setup kernels
+// Drop mask and scale index per component: beta = b / Delta (steps); kept iff beta >= 0.05;
+// s = clamp(round(8 log2(beta / 0.05)), 0, 63)  ("Transform": drop below 0.05 steps).
+__global__ void k_scale_keep(const float *b, const float *delta, uint8_t *scale, uint8_t *keep, int32_t *bad) {
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= N_COEF) return;
+  const double d = (double)delta[c];
+  const double beta = (double)b[c] / d;
+  if (!(d > 0.0) || !isfinite(d) || !isfinite(beta) || beta < 0.0) atomicExch(bad, 1);
+  const bool kp = beta >= B0_STEPS;
+  int s = 0;
+  if (kp) {
+    const double v = rint(8.0 * log2(beta / B0_STEPS));
+    s = (int)fmin(fmax(v, 0.0), (double)(N_SCALES - 1));
+  }
+  keep[c] = kp ? 1 : 0;
+  scale[c] = (uint8_t)s;
+}
+
+// Integer Laplace tables ("Coding"): beta_s = 0.05 * 2^(s/8) steps; p(r) = Laplace(0, beta)
+// mass of [r - 1/2, r + 1/2] for r in [-254, 254], ESC = mass beyond +-254.5;
+// freq = 1 + floor(p * (2^16 - 510)), the remainder of 2^16 to r = 0; cdf in symbol order.
+__global__ void k_tables(uint16_t *cdf_out) {
+  __shared__ int64_t fr[N_SYM];
+  const int s = blockIdx.x;
+  const double beta = B0_STEPS * pow(2.0, (double)s / 8.0);
+  for (int k = threadIdx.x; k < N_SYM; k += blockDim.x) {
+    double p;
+    if (k == ESC_SYM) {
+      p = exp(-(R_MAX + 0.5) / beta);
+    } else {
+      const double ar = fabs((double)(k - R_MAX));
+      p = ar == 0.0 ? -expm1(-0.5 / beta) : 0.5 * exp(-(ar - 0.5) / beta) * -expm1(-1.0 / beta);
+    }
+    fr[k] = 1 + (int64_t)floor(p * (double)(PREC_TOTAL - N_SYM));
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int64_t sum = 0;
+    for (int k = 0; k < N_SYM; ++k) sum += fr[k];
+    fr[R_MAX] += (int64_t)PREC_TOTAL - sum;
+    int64_t c = 0;
+    for (int k = 0; k < N_SYM; ++k) {
+      cdf_out[s * N_SYM + k] = (uint16_t)c;
+      c += fr[k];
+    }
+  }
+}
+
+// out[c] = sum_r v[r] * mat[r][c] in fp64, one thread per column, sequential in r.
+__global__ void k_vec_mat(const float *v, const float *mat, int rows, int cols, float *out) {
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= cols) return;
+  double acc = 0.0;
+  for (int r = 0; r < rows; ++r) acc += (double)v[r] * (double)mat[(int64_t)r * cols + c];
+  out[c] = (float)acc;
+}
+
+// max |mat| (optionally times delta[column]) via integer atomicMax on non-negative floats.
+__global__ void k_absmax(const float *mat, int64_t n, int cols, const float *delta, int *out) {
+  float m = 0.f;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    float v = fabsf(mat[i]);
+    if (delta) v *= fabsf(delta[i % cols]);
+    m = fmaxf(m, v);
+  }
+  for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) atomicMax(out, __float_as_int(m));
+}
+
+// Split operand: out[0][m][k] = fp16(v), out[1][m][k] = fp16(v - fp16(v)), v = in(m, k) * 2^p.
+//   mode 0: in(m, k) = src[k * M + m]   (transpose of a row-major [K][M] matrix)
+//   mode 1: in(m, k) = src[dim(m) * K + k] * delta[k]   (inverse operand, permuted rows)
+__global__ void k_split(const float *src, int M, int K, int mode, const float *delta, double scale, __half *out) {
+  __shared__ float tile[32][33];
+  const int k0 = blockIdx.x * 32, m0 = blockIdx.y * 32;
+  const int tx = threadIdx.x, ty = threadIdx.y;  // 32 x 8
+  if (mode == 0) {
+    for (int y = ty; y < 32; y += 8) {
+      const int k = k0 + y, m = m0 + tx;
+      tile[y][tx] = (k < K && m < M) ? src[(int64_t)k * M + m] : 0.f;
+    }
+    __syncthreads();
+    for (int y = ty; y < 32; y += 8) {
+      const int m = m0 + y, k = k0 + tx;
+      if (m < M && k < K) {
+        const double v = (double)tile[tx][y] * scale;
+        const __half hi = __double2half(v);
+        const __half lo = __double2half(v - (double)__half2float(hi));
+        out[(int64_t)m * K + k] = hi;
+        out[(int64_t)M * K + (int64_t)m * K + k] = lo;
+      }
+    }
+  } else {
+    for (int y = ty; y < 32; y += 8) {
+      const int m = m0 + y, k = k0 + tx;
+      if (m < M && k < K) {
+        const double v = (double)src[(int64_t)inv_row_to_dim(m) * K + k] * (double)delta[k] * scale;
+        const __half hi = __double2half(v);
+        const __half lo = __double2half(v - (double)__half2float(hi));
+        out[(int64_t)m * K + k] = hi;
+        out[(int64_t)M * K + (int64_t)m * K + k] = lo;
+      }
+    }
+  }
+}
+
+// out[o][k] = src[(k + k_off) * ld + o], o < O, k < K  (bf16 bits)
+__global__ void k_transpose16(const uint16_t *src, int ld, int k_off, int O, int K, uint16_t *out) {
+  __shared__ uint16_t tile[32][33];
+  const int k0 = blockIdx.x * 32, o0 = blockIdx.y * 32;
+  const int tx = threadIdx.x, ty = threadIdx.y;
+  for (int y = ty; y < 32; y += 8) {
+    const int k = k0 + y, o = o0 + tx;
+    tile[y][tx] = (k < K && o < O) ? src[(int64_t)(k + k_off) * ld + o] : 0;
+  }
+  __syncthreads();
+  for (int y = ty; y < 32; y += 8) {
+    const int o = o0 + y, k = k0 + tx;
+    if (o < O && k < K) out[(int64_t)o * K + k] = tile[tx][y];
+  }
+}
+
+__global__ void k_permute_mu(const float *mu, float *mu_perm) {
+  const int p = blockIdx.x * blockDim.x + threadIdx.x;
+  if (p < ROW_DIM) mu_perm[p] = mu[inv_row_to_dim(p)];
+}
+
+// ============================================================================ per-call kernels
+// Row tables of one prompt per block: coded row r = row_base + i holds position 4 + i.
+__global__ void k_layout(const PromptInfo *prompts, int32_t *row_tok, int32_t *row_pos, int32_t *row_edst,
+                         int32_t *e_tok, __nv_bfloat16 *qe_zero_pad) {
+  const PromptInfo pi = prompts[blockIdx.x];
+  for (int i = threadIdx.x; i < pi.n; i += blockDim.x) {
+    const int r = pi.row_base + i;
+    row_tok[r] = (int32_t)(pi.tok_base + HEAD_KEPT + i);
+    row_pos[r] = HEAD_KEPT + i;
+    row_edst[r] = (i & 1) ? -1 : pi.ebase + (i >> 1);
+  }
+  for (int e = threadIdx.x; e <= pi.n_e; e += blockDim.x)
+    e_tok[pi.ebase + e] = e < pi.n_o ? (int32_t)(pi.tok_base + HEAD_KEPT + 2 * e + 1) : -1;
+  if (qe_zero_pad)  // the row after a prompt's last even row is its odd rows' zero right neighbour
+    for (int k = threadIdx.x; k < N_COEF; k += blockDim.x)
+      qe_zero_pad[(int64_t)(pi.ebase + pi.n_e) * N_COEF + k] = __float2bfloat16_rn(0.f);
+}
+
+__device__ __forceinline__ int find_prompt(const PromptInfo *p, int batch, int64_t tok) {
+  int lo = 0, hi = batch;  // last prompt with tok_base <= tok
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (p[mid].tok_base <= tok) lo = mid; else hi = mid;
+  }
+  return lo;
+}
+
+// One block per token row: coded rows -> fp16 copy (clamped to +-65504, reported as
+// DCKV_ERANGE), kept rows -> the blob's kept section verbatim.
+__global__ void __launch_bounds__(192) k_convert(const __nv_bfloat16 *rows, const PromptInfo *prompts, int batch,
+                                                 __half *x16, uint8_t *blob, uint64_t blob_cap, uint64_t off_kept,
+                                                 int32_t *status) {
+  const int64_t t = blockIdx.x;
+  const int b = find_prompt(prompts, batch, t);
+  const PromptInfo pi = prompts[b];
+  const int p = (int)(t - pi.tok_base);
+  const uint4 *src = reinterpret_cast<const uint4 *>(rows + t * ROW_DIM);
+  const bool coded = pi.n > 0 && p >= HEAD_KEPT && p < pi.N - TAIL_KEPT;
+  if (coded) {
+    uint4 *dst = reinterpret_cast<uint4 *>(x16 + (int64_t)(pi.row_base + p - HEAD_KEPT) * ROW_DIM);
+    bool clamped = false;
+    for (int v = threadIdx.x; v < ROW_DIM / 8; v += blockDim.x) {
+      uint4 in = src[v];
+      const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&in);
+      uint4 o;
+      __half2 *oh = reinterpret_cast<__half2 *>(&o);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float2 f = __bfloat1622float2(h[q]);
+        const float lim = 65504.f;
+        if (!(fabsf(f.x) <= lim) || !(fabsf(f.y) <= lim)) clamped = true;
+        f.x = fminf(fmaxf(f.x, -lim), lim);
+        f.y = fminf(fmaxf(f.y, -lim), lim);
+        oh[q] = __floats2half2_rn(f.x, f.y);
+      }
+      dst[v] = o;
+    }
+    if (clamped) atomicExch(status, DCKV_ERANGE);
+  } else {
+    const int kidx = (pi.n == 0 || p < HEAD_KEPT) ? p : HEAD_KEPT + (p - (pi.N - TAIL_KEPT));
+    const uint64_t off = off_kept + (uint64_t)(pi.kept_base + kidx) * (ROW_DIM * 2);
+    if (off + ROW_DIM * 2 > blob_cap) return;
+    uint4 *dst = reinterpret_cast<uint4 *>(blob + off);
+    for (int v = threadIdx.x; v < ROW_DIM / 8; v += blockDim.x) dst[v] = src[v];
+  }
+}
+
+// Decode-side check of the blob header and tables against the expected batch shape.
+struct HeaderCheck {
+  const uint8_t *blob;
+  uint64_t blob_bytes;
+  const PromptInfo *prompts;
+  int batch, chunk_rows, k_eff, n_chunks_e, n_chunks_o;
+  int64_t n_kept;
+  uint64_t off_kept, off_streams;
+  int32_t *valid;
+  int32_t *status;
+};
+
+__global__ void k_check_header(HeaderCheck h) {
+  __shared__ int bad;
+  if (threadIdx.x == 0) bad = 0;
+  __syncthreads();
+  const int n_ch = h.n_chunks_e + h.n_chunks_o;
+  const uint64_t tab_end = HEADER_BYTES + 4ull * (h.batch + n_ch + 1);
+  if (h.blob_bytes < tab_end || h.blob_bytes < h.off_streams) {
+    if (threadIdx.x == 0) bad = 1;
+  } else {
+    if (threadIdx.x == 0) {
+      const uint32_t *h32 = reinterpret_cast<const uint32_t *>(h.blob);
+      const uint16_t *h16 = reinterpret_cast<const uint16_t *>(h.blob);
+      const uint64_t *h64 = reinterpret_cast<const uint64_t *>(h.blob + 32);
+      if (h32[0] != MAGIC || h16[2] != VERSION || h16[3] != (uint16_t)h.chunk_rows || h32[2] != (uint32_t)h.batch ||
+          h32[3] != (uint32_t)N_COEF || h32[4] != (uint32_t)h.k_eff || h32[5] != (uint32_t)h.n_chunks_e ||
+          h32[6] != (uint32_t)h.n_chunks_o || h32[7] != (uint32_t)h.n_kept || h64[1] != h.off_streams ||
+          h64[2] != h.off_kept || h64[0] > h.blob_bytes)
+        bad = 1;
+      const uint32_t *ct = h32 + HEADER_BYTES / 4 + h.batch;
+      if (ct[0] != 0 || h.off_streams + ct[n_ch] != h64[0]) bad = 1;
+    }
+    __syncthreads();
+    const uint32_t *pt = reinterpret_cast<const uint32_t *>(h.blob + HEADER_BYTES);
+    for (int b = threadIdx.x; b < h.batch; b += blockDim.x)
+      if (pt[b] != (uint32_t)h.prompts[b].N) bad = 1;
+    const uint32_t *ct = pt + h.batch;
+    for (int c = threadIdx.x; c < n_ch; c += blockDim.x)
+      if (ct[c + 1] < ct[c] || ct[c + 1] - ct[c] < (uint32_t)CHUNK_FIXED_BYTES || (ct[c] & 3u)) bad = 1;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    *h.valid = bad ? 0 : 1;
+    if (bad) atomicExch(h.status, DCKV_ECORRUPT);
+  }
+}
+
+// Kept rows: bf16 from the blob, RoPE on keys (same rotation as the inverse epilogue), bf16.
+__global__ void __launch_bounds__(256) k_kept(const uint8_t *blob, uint64_t off_kept, const PromptInfo *prompts,
+                                              int batch, const double *theta, __nv_bfloat16 *k_out,
+                                              __nv_bfloat16 *v_out, int64_t n_tokens, const int32_t *valid) {
+  if (*valid != 1) return;
+  const int64_t kr = blockIdx.x;  // kept row index in the blob
+  int lo = 0, hi = batch;         // last prompt with kept_base <= kr
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (prompts[mid].kept_base <= kr) lo = mid; else hi = mid;
+  }
+  const PromptInfo pi = prompts[lo];
+  const int kidx = (int)(kr - pi.kept_base);
+  const int pos = (pi.n == 0 || kidx < HEAD_KEPT) ? kidx : pi.N - TAIL_KEPT + (kidx - HEAD_KEPT);
+  const int64_t tok = pi.tok_base + pos;
+  const __nv_bfloat16 *row = reinterpret_cast<const __nv_bfloat16 *>(blob + off_kept + (uint64_t)kr * ROW_DIM * 2);
+  // 24 head vectors x 128 pairs
+  for (int idx = threadIdx.x; idx < 24 * 128; idx += blockDim.x) {
+    const int hv = idx >> 7, i = idx & 127;
+    const int layer = hv >> 2, kv = (hv >> 1) & 1, head = hv & 1;
+    float a = __bfloat162float(row[hv * HEAD_DIM + i]);
+    float b = __bfloat162float(row[hv * HEAD_DIM + 128 + i]);
+    if (kv == 0) {
+      float cs, sn;
+      rope_cs(pos, i, theta, cs, sn);
+      const float a2 = a * cs - b * sn, b2 = b * cs + a * sn;
+      a = a2;
+      b = b2;
+    }
+    __nv_bfloat16 *dst = (kv == 0 ? k_out : v_out) + ((layer * n_tokens + tok) * 2 + head) * HEAD_DIM;
+    dst[i] = __float2bfloat16_rn(a);
+    dst[128 + i] = __float2bfloat16_rn(b);
+  }
+}
+
+__host__ __device__ __forceinline__ int dim_to_inv_row(int d) {
+  const int hv = d / HEAD_DIM, dd = d % HEAD_DIM;
+  const int half = dd < 128 ? dd / 64 : (dd - 128) / 64;
+  const int r = dd < 128 ? dd % 64 : 64 + (dd - 128) % 64;
+  return (2 * hv + half) * GEMM_BM + r;
+}
+
+// Rows holding a code with |q| >= 2048 (not exact in the fp16 operand) are recomputed
+// here in fp32 from the exact codes, after the inverse GEMM wrote them.
+__global__ void __launch_bounds__(256) k_fixup(const int32_t *biglist, const uint32_t *bigcount, const __half *q16,
+                                               const int32_t *qbig, const __half *a_inv, float inv_scale,
+                                               const float *mu_perm, const double *theta, const int32_t *row_tok,
+                                               const int32_t *row_pos, __nv_bfloat16 *k_out, __nv_bfloat16 *v_out,
+                                               int64_t n_tokens) {
+  __shared__ float qs[N_COEF];
+  __shared__ float xs[ROW_DIM];
+  const uint32_t n = *bigcount;
+  for (uint32_t li = blockIdx.x; li < n; li += gridDim.x) {
+    const int64_t r = biglist[li];
+    for (int c = threadIdx.x; c < N_COEF; c += blockDim.x) {
+      float v = __half2float(q16[r * N_COEF + c]);
+      if (fabsf(v) >= (float)BIG_CODE) v = (float)qbig[r * N_COEF + c];
+      qs[c] = v;
+    }
+    __syncthreads();
+    const __half *lo = a_inv + (int64_t)ROW_DIM * N_COEF;
+    for (int d = threadIdx.x; d < ROW_DIM; d += blockDim.x) {
+      const int64_t p = dim_to_inv_row(d);
+      float acc = 0.f;
+      for (int c = 0; c < N_COEF; ++c)
+        acc = fmaf(qs[c], __half2float(a_inv[p * N_COEF + c]) + __half2float(lo[p * N_COEF + c]), acc);
+      xs[d] = acc * inv_scale + mu_perm[p];
+    }
+    __syncthreads();
+    const int pos = row_pos[r];
+    const int64_t tok = row_tok[r];
+    for (int idx = threadIdx.x; idx < 24 * 128; idx += blockDim.x) {
+      const int hv = idx >> 7, i = idx & 127;
+      const int layer = hv >> 2, kv = (hv >> 1) & 1, head = hv & 1;
+      float a = xs[hv * HEAD_DIM + i], b = xs[hv * HEAD_DIM + 128 + i];
+      if (kv == 0) {
+        float cs, sn;
+        rope_cs(pos, i, theta, cs, sn);
+        const float a2 = a * cs - b * sn, b2 = b * cs + a * sn;
+        a = a2;
+        b = b2;
+      }
+      __nv_bfloat16 *dst = (kv == 0 ? k_out : v_out) + ((layer * n_tokens + tok) * 2 + head) * HEAD_DIM;
+      dst[i] = __float2bfloat16_rn(a);
+      dst[128 + i] = __float2bfloat16_rn(b);
+    }
+    __syncthreads();
+  }
+}
+
+// ============================================================================ host layout
+static inline uint64_t align_up(uint64_t v, uint64_t a) { return (v + a - 1) / a * a; }
+
+static int build_layout(const dckv_codec *c, const int64_t *offs, int batch, Layout &L) {
+  if (!offs) return fail(DCKV_EINVAL, "seq_offsets is NULL");
+  if (batch < 1 || batch > DCKV_MAX_PROMPTS) return fail(DCKV_EINVAL, "batch %d out of range", batch);
+  if (offs[0] != 0) return fail(DCKV_EINVAL, "seq_offsets[0] must be 0");
+  L = Layout();
+  L.batch = batch;
+  const int G = c->chunk_rows;
+  int64_t rows = 0, ne = 0, kept = 0;
+  int ce = 0, co = 0;
+  L.prompts.resize(batch);
+  for (int b = 0; b < batch; ++b) {
+    const int64_t N = offs[b + 1] - offs[b];
+    if (N < 0 || N > (int64_t)1 << 30) return fail(DCKV_EINVAL, "prompt %d has a bad length", b);
+    PromptInfo &p = L.prompts[b];
+    p.tok_base = offs[b];
+    p.N = (int32_t)N;
+    p.n = (int32_t)std::max<int64_t>(0, N - HEAD_KEPT - TAIL_KEPT);
+    p.n_e = (p.n + 1) / 2;
+    p.n_o = p.n / 2;
+    p.row_base = (int32_t)rows;
+    p.ebase = (int32_t)ne;
+    p.kept_base = (int32_t)kept;
+    p.n_kept = (int32_t)(N - p.n);
+    p.chunk_e0 = ce;
+    ce += (p.n_e + G - 1) / G;
+    rows += p.n;
+    ne += p.n_e + 1;
+    kept += p.n_kept;
+  }
+  for (int b = 0; b < batch; ++b) {
+    L.prompts[b].chunk_o0 = ce + co;
+    co += (L.prompts[b].n_o + G - 1) / G;
+  }
+  L.n_tokens = offs[batch];
+  if (L.n_tokens >= ((int64_t)1 << 31)) return fail(DCKV_EINVAL, "too many tokens");
+  if (rows > DCKV_MAX_ROWS) return fail(DCKV_EINVAL, "too many coded rows (%lld)", (long long)rows);
+  L.n_rows = rows;
+  L.ne_pad = ne;
+  L.n_kept = kept;
+  L.n_chunks_e = ce;
+  L.n_chunks_o = co;
+  L.n_chunks = ce + co;
+  L.chunks.resize(L.n_chunks);
+  int64_t slot = 0;
+  int ci = 0;
+  for (int par = 0; par < 2; ++par)
+    for (int b = 0; b < batch; ++b) {
+      const PromptInfo &p = L.prompts[b];
+      const int nr = par ? p.n_o : p.n_e;
+      for (int j0 = 0; j0 < nr; j0 += G) {
+        ChunkDesc &d = L.chunks[ci++];
+        d.prompt = b;
+        d.parity = par;
+        d.j0 = j0;
+        d.nrows = std::min(G, nr - j0);
+        d.sym_base = slot * c->k_eff;
+        slot += d.nrows;
+      }
+    }
+  L.n_symbols = rows * (int64_t)c->k_eff;
+  L.off_kept = align_up(HEADER_BYTES + 4ull * (batch + L.n_chunks + 1), 16);
+  L.off_streams = L.off_kept + (uint64_t)kept * ROW_DIM * 2;
+  return DCKV_OK;
+}
+
+static WsPlan plan_ws(const Layout &L, int which /*0 encode, 1 decode*/) {
+  WsPlan w;
+  memset(&w, 0, sizeof(w));
+  uint64_t o = 0;
+  auto take = [&](uint64_t bytes) {
+    const uint64_t at = o;
+    o = align_up(o + std::max<uint64_t>(bytes, 1), 256);
+    return (size_t)at;
+  };
+  w.prompts = take(sizeof(PromptInfo) * L.batch);
+  w.chunks = take(sizeof(ChunkDesc) * std::max(L.n_chunks, 1));
+  w.row_tok = take(4ull * L.n_rows);
+  w.row_pos = take(4ull * L.n_rows);
+  w.row_edst = take(4ull * L.n_rows);
+  w.e_tok = take(4ull * L.ne_pad);
+  w.qe = take(2ull * L.ne_pad * N_COEF);
+  w.c_odd = take(1ull * L.ne_pad * N_COEF);
+  w.counters = take(256);
+  if (which == 0) {
+    w.x16 = take(2ull * L.n_rows * ROW_DIM);
+    w.g16 = take(2ull * L.n_rows * 2 * N_HIDDEN);
+    w.q32 = take(4ull * L.n_rows * N_COEF);
+    w.words = take(2ull * L.n_symbols);
+    w.states = take(128ull * L.n_chunks);
+    w.nwords = take(4ull * L.n_chunks);
+    w.nesc = take(4ull * L.n_chunks);
+    w.offs = take(4ull * (L.n_chunks + 1));
+  } else {
+    w.q16 = take(2ull * L.n_rows * N_COEF);
+    w.qbig = take(4ull * L.n_rows * N_COEF);
+    w.bigflag = take(4ull * L.n_rows);
+    w.biglist = take(4ull * L.n_rows);
+  }
+  w.total = o;
+  return w;
+}
+
+static void stage_mark(const dckv_codec *cc, cudaStream_t st, const char *name) {
+  dckv_codec *c = const_cast<dckv_codec *>(cc);
+  if (!c->timing || c->n_ev >= 24) return;
+  c->ev_names[c->n_ev] = name;
+  cudaEventRecord(c->ev[c->n_ev++], st);
+}
+
+// ============================================================================ codec create
+extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_rows, dckv_codec **out) {
+  if (!out) return fail(DCKV_EINVAL, "out is NULL");
+  *out = nullptr;
+  if (!prm || !prm->mu || !prm->basis || !prm->w1 || !prm->w2 || !prm->delta || !prm->laplace_b || !prm->embed ||
+      !prm->w_even || !prm->w_odd)
+    return fail(DCKV_EINVAL, "a parameter pointer is NULL");
+  if (prm->vocab < 1 || prm->vocab > (1 << 20)) return fail(DCKV_EINVAL, "vocab out of range");
+  if (chunk_rows == 0) chunk_rows = 32;
+  if (chunk_rows < 1 || chunk_rows > 256) return fail(DCKV_EINVAL, "chunk_rows out of range");
+  if (((uintptr_t)prm->embed | (uintptr_t)prm->w_even | (uintptr_t)prm->w_odd) & 15)
+    return fail(DCKV_EINVAL, "bf16 parameters must be 16-byte aligned");
+  CK(cudaSetDevice(device));
+  cudaDeviceProp prop;
+  CK(cudaGetDeviceProperties(&prop, device));
+  if (prop.major != 10) return fail(DCKV_EINVAL, "needs an sm_100 device (found sm_%d%d)", prop.major, prop.minor);
+  if (!encode_fn()) return fail(DCKV_ECUDA, "cuTensorMapEncodeTiled unavailable");
+
+  dckv_codec *c = new dckv_codec();
+  c->device = device;
+  c->num_sms = prop.multiProcessorCount;
+  c->chunk_rows = chunk_rows;
+  c->vocab = prm->vocab;
+  c->p = *prm;
+  for (int i = 0; i < 24; ++i) cudaEventCreate(&c->ev[i]);
+
+  auto cleanup = [&](int code) {
+    dckv_codec_destroy(c);
+    return code;
+  };
+
+  // one device block for every derived tensor
+  const uint64_t V = (uint64_t)prm->vocab;
+  uint64_t o = 0;
+  auto take = [&](uint64_t bytes) {
+    const uint64_t at = o;
+    o = align_up(o + bytes, 1024);
+    return at;
+  };
+  const uint64_t o_ay = take(2ull * 2 * N_COEF * ROW_DIM);
+  const uint64_t o_aw2 = take(2ull * 2 * N_COEF * N_HIDDEN);
+  const uint64_t o_ah = take(2ull * 2 * N_HIDDEN * ROW_DIM);
+  const uint64_t o_ainv = take(2ull * 2 * ROW_DIM * N_COEF);
+  const uint64_t o_aon = take(2ull * N_COEF * 2 * N_COEF);
+  const uint64_t o_te = take(4ull * V * N_COEF);
+  const uint64_t o_to = take(4ull * V * N_COEF);
+  const uint64_t o_mub = take(4ull * N_COEF);
+  const uint64_t o_muw1 = take(4ull * N_HIDDEN);
+  const uint64_t o_mup = take(4ull * ROW_DIM);
+  const uint64_t o_delta = take(4ull * N_COEF);
+  const uint64_t o_keep = take(N_COEF);
+  const uint64_t o_scale = take(N_COEF);
+  const uint64_t o_kl = take(2ull * N_COEF);
+  const uint64_t o_ks = take(N_COEF);
+  const uint64_t o_cdf = take(2ull * N_SCALES * N_SYM);
+  const uint64_t o_theta = take(8ull * 128);
+  const uint64_t o_tmp = take(2ull * 2 * N_COEF * N_COEF);  // W_e^T and W_oE^T (setup only)
+  const uint64_t o_scr = take(64);
+  if (cudaMalloc(&c->blk, o) != cudaSuccess) return cleanup(fail(DCKV_ECUDA, "cudaMalloc(%llu) failed", (unsigned long long)o));
+  uint8_t *B = (uint8_t *)c->blk;
+  c->a_y = (__half *)(B + o_ay);
+  c->a_w2 = (__half *)(B + o_aw2);
+  c->a_h = (__half *)(B + o_ah);
+  c->a_inv = (__half *)(B + o_ainv);
+  c->a_on = (__nv_bfloat16 *)(B + o_aon);
+  c->t_even = (float *)(B + o_te);
+  c->t_odd = (float *)(B + o_to);
+  c->mub = (float *)(B + o_mub);
+  c->muw1 = (float *)(B + o_muw1);
+  c->mu_perm = (float *)(B + o_mup);
+  c->delta = (float *)(B + o_delta);
+  c->keep = B + o_keep;
+  c->scale = B + o_scale;
+  c->kept_list = (int16_t *)(B + o_kl);
+  c->kept_scale = B + o_ks;
+  c->cdf = (uint16_t *)(B + o_cdf);
+  c->theta = (double *)(B + o_theta);
+  uint16_t *tmp_e = (uint16_t *)(B + o_tmp);
+  uint16_t *tmp_oe = tmp_e + (size_t)N_COEF * N_COEF;
+  int32_t *scr = (int32_t *)(B + o_scr);
+  cudaStream_t st = 0;
+
+  if (cudaMemset(scr, 0, 64) != cudaSuccess) return cleanup(fail(DCKV_ECUDA, "memset"));
+  // drop mask, scale index, tables
+  k_scale_keep<<<(N_COEF + 255) / 256, 256, 0, st>>>(prm->laplace_b, prm->delta, c->scale, c->keep, scr);
+  k_tables<<<N_SCALES, 512, 0, st>>>(c->cdf);
+  cudaMemcpyAsync(c->delta, prm->delta, 4ull * N_COEF, cudaMemcpyDeviceToDevice, st);
+  // scale exponents: largest |value| of each split operand brought to about 2^12
+  k_absmax<<<256, 256, 0, st>>>(prm->basis, (int64_t)ROW_DIM * N_COEF, N_COEF, nullptr, scr + 1);
+  k_absmax<<<64, 256, 0, st>>>(prm->w2, (int64_t)N_HIDDEN * N_COEF, N_COEF, nullptr, scr + 2);
+  k_absmax<<<256, 256, 0, st>>>(prm->w1, (int64_t)ROW_DIM * N_HIDDEN, N_HIDDEN, nullptr, scr + 3);
+  k_absmax<<<256, 256, 0, st>>>(prm->basis, (int64_t)ROW_DIM * N_COEF, N_COEF, prm->delta, scr + 4);
+  int32_t host_scr[8];
+  uint8_t keep_h[N_COEF], scale_h[N_COEF];
+  if (cudaMemcpy(host_scr, scr, 32, cudaMemcpyDeviceToHost) != cudaSuccess ||
+      cudaMemcpy(keep_h, c->keep, N_COEF, cudaMemcpyDeviceToHost) != cudaSuccess ||
+      cudaMemcpy(scale_h, c->scale, N_COEF, cudaMemcpyDeviceToHost) != cudaSuccess)
+    return cleanup(fail(DCKV_ECUDA, "setup readback failed: %s", cudaGetErrorString(cudaGetLastError())));
+  if (host_scr[0]) return cleanup(fail(DCKV_EINVAL, "delta must be positive and laplace_b finite"));
+  auto exp_for = [](int32_t bits) {
+    float m;
+    memcpy(&m, &bits, 4);
+    if (!(m > 0.f) || !std::isfinite(m)) return 0;
+    int e = (int)std::floor(std::log2(4096.0 / (double)m));
+    return std::min(40, std::max(-40, e));
+  };
+  float mb, mw2;
+  memcpy(&mb, &host_scr[1], 4);
+  memcpy(&mw2, &host_scr[2], 4);
+  int32_t mboth;
+  const float mmax = std::max(mb, mw2);
+  memcpy(&mboth, &mmax, 4);
+  c->p_y = exp_for(mboth);
+  c->p_h = exp_for(host_scr[3]);
+  c->p_inv = exp_for(host_scr[4]);
+  // kept components
+  std::vector<int16_t> kl;
+  std::vector<uint8_t> ks;
+  for (int i = 0; i < N_COEF; ++i)
+    if (keep_h[i]) {
+      kl.push_back((int16_t)i);
+      ks.push_back(scale_h[i]);
+    }
+  c->k_eff = (int)kl.size();
+  kl.resize(N_COEF, 0);
+  ks.resize(N_COEF, 0);
+  double theta_h[128];
+  for (int i = 0; i < 128; ++i) theta_h[i] = std::pow(ROPE_BASE, -2.0 * i / HEAD_DIM);
+  if (cudaMemcpy(c->kept_list, kl.data(), 2 * N_COEF, cudaMemcpyHostToDevice) != cudaSuccess ||
+      cudaMemcpy(c->kept_scale, ks.data(), N_COEF, cudaMemcpyHostToDevice) != cudaSuccess ||
+      cudaMemcpy(c->theta, theta_h, sizeof(theta_h), cudaMemcpyHostToDevice) != cudaSuccess)
+    return cleanup(fail(DCKV_ECUDA, "setup upload failed"));
+  // mean projections in fp64
+  k_vec_mat<<<(N_COEF + 255) / 256, 256, 0, st>>>(prm->mu, prm->basis, ROW_DIM, N_COEF, c->mub);
+  k_vec_mat<<<1, 256, 0, st>>>(prm->mu, prm->w1, ROW_DIM, N_HIDDEN, c->muw1);
+  k_permute_mu<<<(ROW_DIM + 255) / 256, 256, 0, st>>>(prm->mu, c->mu_perm);
+  // split operands (hi/lo fp16, power-of-two scaled)
+  dim3 tb(32, 8);
+  k_split<<<dim3(ROW_DIM / 32, N_COEF / 32), tb, 0, st>>>(prm->basis, N_COEF, ROW_DIM, 0, nullptr, std::ldexp(1.0, c->p_y), c->a_y);
+  k_split<<<dim3(N_HIDDEN / 32, N_COEF / 32), tb, 0, st>>>(prm->w2, N_COEF, N_HIDDEN, 0, nullptr, std::ldexp(1.0, c->p_y), c->a_w2);
+  k_split<<<dim3(ROW_DIM / 32, N_HIDDEN / 32), tb, 0, st>>>(prm->w1, N_HIDDEN, ROW_DIM, 0, nullptr, std::ldexp(1.0, c->p_h), c->a_h);
+  k_split<<<dim3(N_COEF / 32, ROW_DIM / 32), tb, 0, st>>>(prm->basis, ROW_DIM, N_COEF, 1, prm->delta, std::ldexp(1.0, c->p_inv), c->a_inv);
+  // mean-model weights, K-major
+  k_transpose16<<<dim3(2 * N_COEF / 32, N_COEF / 32), tb, 0, st>>>(prm->w_odd, N_COEF, N_COEF, N_COEF, 2 * N_COEF,
+                                                                   (uint16_t *)c->a_on);
+  k_transpose16<<<dim3(N_COEF / 32, N_COEF / 32), tb, 0, st>>>(prm->w_even, N_COEF, 0, N_COEF, N_COEF, tmp_e);
+  k_transpose16<<<dim3(N_COEF / 32, N_COEF / 32), tb, 0, st>>>(prm->w_odd, N_COEF, 0, N_COEF, N_COEF, tmp_oe);
+  if (cudaGetLastError() != cudaSuccess) return cleanup(fail(DCKV_ECUDA, "setup kernels failed to launch"));
+  // tensor maps of the static operands
+  int r = DCKV_OK;
+  if ((r = map_a(&c->map_ay2, c->a_y, false, ROW_DIM, N_COEF, 2, 2)) ||
+      (r = map_a(&c->map_aw2_2, c->a_w2, false, N_HIDDEN, N_COEF, 2, 2)) ||
+      (r = map_a(&c->map_aw2_1, c->a_w2, false, N_HIDDEN, N_COEF, 2, 1)) ||
+      (r = map_a(&c->map_ah2, c->a_h, false, ROW_DIM, N_HIDDEN, 2, 2)) ||
+      (r = map_a(&c->map_ainv2, c->a_inv, false, N_COEF, ROW_DIM, 2, 2)) ||
+      (r = map_a(&c->map_aon1, c->a_on, true, 2 * N_COEF, N_COEF, 1, 1)))
+    return cleanup(r);
+  // per-vocabulary mean tables: t_even = embed @ w_even, t_odd = embed @ w_odd[0:2048]
+  {
+    CUtensorMap ma_e, ma_o, mb_emb;
+    if ((r = map_a(&ma_e, tmp_e, true, N_COEF, N_COEF, 1, 1)) || (r = map_a(&ma_o, tmp_oe, true, N_COEF, N_COEF, 1, 1)) ||
+        (r = map_b(&mb_emb, prm->embed, true, N_COEF, V, 256)))
+      return cleanup(r);
+    for (int which = 0; which < 2; ++which) {
+      GemmProblem pr = make_problem(N_COEF / GEMM_BM, (int64_t)V, 256, true, scr + 5);
+      add_seg(pr, 0, 0, 1, 0, 0, 0, 0, N_COEF / GEMM_BK);
+      EpiStoreF32::Params ep{which ? c->t_odd : c->t_even, N_COEF, 1.0f};
+      if ((r = run_gemm<EpiStoreF32, 4, 1>(which ? ma_o : ma_e, ma_e, mb_emb, mb_emb, pr, ep, c->num_sms, st)))
+        return cleanup(r);
+    }
+  }
+  if (cudaDeviceSynchronize() != cudaSuccess)
+    return cleanup(fail(DCKV_ECUDA, "codec setup failed: %s", cudaGetErrorString(cudaGetLastError())));
+  int32_t tmo = 0;
+  cudaMemcpy(&tmo, scr + 5, 4, cudaMemcpyDeviceToHost);
+  if (tmo) return cleanup(fail(DCKV_ETIMEOUT, "setup GEMM timed out"));
+  *out = c;
+  return DCKV_OK;
+}
+
+extern "C" void dckv_codec_destroy(dckv_codec *c) {
+  if (!c) return;
+  cudaSetDevice(c->device);
+  if (c->blk) cudaFree(c->blk);
+  for (int i = 0; i < 24; ++i)
+    if (c->ev[i]) cudaEventDestroy(c->ev[i]);
+  delete c;
+}
+
+extern "C" int dckv_codec_k_eff(const dckv_codec *c) { return c ? c->k_eff : -1; }
+
+extern "C" size_t dckv_workspace_bytes(const dckv_codec *c, const int64_t *offs, int batch) {
+  if (!c) return 0;
+  Layout L;
+  if (build_layout(c, offs, batch, L) != DCKV_OK) return 0;
+  return std::max(plan_ws(L, 0).total, plan_ws(L, 1).total);
+}
+
+extern "C" size_t dckv_blob_bound(const dckv_codec *c, const int64_t *offs, int batch) {
+  if (!c) return 0;
+  Layout L;
+  if (build_layout(c, offs, batch, L) != DCKV_OK) return 0;
+  // every symbol escaped: 8 bytes of escape value + one word each, plus fixed parts
+  return L.off_streams + (uint64_t)L.n_chunks * (CHUNK_FIXED_BYTES + 4) + 10ull * L.n_symbols;
+}
+
+static int upload_tables(const Layout &L, uint8_t *ws, const WsPlan &w, cudaStream_t st) {
+  CK(cudaMemcpyAsync(ws + w.prompts, L.prompts.data(), sizeof(PromptInfo) * L.batch, cudaMemcpyHostToDevice, st));
+  if (L.n_chunks)
+    CK(cudaMemcpyAsync(ws + w.chunks, L.chunks.data(), sizeof(ChunkDesc) * L.n_chunks, cudaMemcpyHostToDevice, st));
+  return DCKV_OK;
+}
+
+// ============================================================================ encode
+extern "C" int dckv_encode(const dckv_codec *c, const void *rows, const int32_t *token_ids, const int64_t *seq_offsets,
+                           int batch, void *blob, size_t blob_cap, uint64_t *blob_size_dev, int32_t *status_dev,
+                           void *workspace, size_t ws_bytes, void *stream) {
+  if (!c || !rows || !token_ids || !blob || !blob_size_dev || !status_dev || !workspace)
+    return fail(DCKV_EINVAL, "a pointer argument is NULL");
+  if (((uintptr_t)rows & 15) || ((uintptr_t)blob & 15) || ((uintptr_t)workspace & 255))
+    return fail(DCKV_EINVAL, "rows/blob must be 16-byte and workspace 256-byte aligned");
+  Layout L;
+  RET(build_layout(c, seq_offsets, batch, L));
+  const WsPlan w = plan_ws(L, 0);
+  if (ws_bytes < w.total) return fail(DCKV_ECAPACITY, "workspace too small (%zu < %zu)", ws_bytes, w.total);
+  cudaStream_t st = (cudaStream_t)stream;
+  CK(cudaSetDevice(c->device));
+  dckv_codec *cm = const_cast<dckv_codec *>(c);
+  cm->n_ev = 0;
+  uint8_t *ws = (uint8_t *)workspace;
+  uint8_t *bl = (uint8_t *)blob;
+  PromptInfo *d_prompts = (PromptInfo *)(ws + w.prompts);
+  ChunkDesc *d_chunks = (ChunkDesc *)(ws + w.chunks);
+  int32_t *row_tok = (int32_t *)(ws + w.row_tok), *row_pos = (int32_t *)(ws + w.row_pos);
+  int32_t *row_edst = (int32_t *)(ws + w.row_edst), *e_tok = (int32_t *)(ws + w.e_tok);
+  __half *x16 = (__half *)(ws + w.x16);
+  __half *g16 = (__half *)(ws + w.g16);
+  int32_t *q32 = (int32_t *)(ws + w.q32);
+  __nv_bfloat16 *qe = (__nv_bfloat16 *)(ws + w.qe);
+  int8_t *c_odd = (int8_t *)(ws + w.c_odd);
+
+  stage_mark(c, st, "start");
+  CK(cudaMemsetAsync(status_dev, 0, 4, st));
+  RET(upload_tables(L, ws, w, st));
+  k_layout<<<L.batch, 256, 0, st>>>(d_prompts, row_tok, row_pos, row_edst, e_tok, qe);
+  if (L.n_tokens > 0)
+    k_convert<<<(unsigned)L.n_tokens, 192, 0, st>>>((const __nv_bfloat16 *)rows, d_prompts, L.batch, x16, bl, blob_cap,
+                                                    L.off_kept, status_dev);
+  CK(cudaGetLastError());
+  stage_mark(c, st, "layout+convert");
+  if (L.n_rows > 0) {
+    CUtensorMap mb_x128, mb_x256, mb_g, mb_qe;
+    RET(map_b(&mb_x128, x16, false, ROW_DIM, L.n_rows, 128));
+    RET(map_b(&mb_x256, x16, false, ROW_DIM, L.n_rows, 256));
+    RET(map_b(&mb_g, g16, false, 2 * N_HIDDEN, L.n_rows, 256));
+    RET(map_b(&mb_qe, qe, true, N_COEF, L.ne_pad, 256));
+    // correction hidden layer: h = x @ w1 - mu @ w1, GELU, fp16 hi/lo
+    {
+      GemmProblem pr = make_problem(N_HIDDEN / GEMM_BM, L.n_rows, 128, false, status_dev);
+      add_seg(pr, 0, 0, 2, 0, 0, 0, 0, ROW_DIM / GEMM_BK);
+      EpiGelu::Params ep{c->muw1, (float)std::ldexp(1.0, -c->p_h), g16};
+      RET((run_gemm<EpiGelu, 3, 2>(c->map_ah2, c->map_ah2, mb_x128, mb_x128, pr, ep, c->num_sms, st)));
+    }
+    stage_mark(c, st, "gemm_hidden");
+    // transform + quantiser: y = x @ B + g @ w2 - mu @ B
+    {
+      GemmProblem pr = make_problem(N_COEF / GEMM_BM, L.n_rows, 256, false, status_dev);
+      add_seg(pr, 0, 0, 2, 0, 0, 0, 0, ROW_DIM / GEMM_BK);
+      add_seg(pr, 1, 0, 2, 0, 1, 0, 0, N_HIDDEN / GEMM_BK);
+      add_seg(pr, 1, 0, 2, 0, 1, 0, N_HIDDEN, N_HIDDEN / GEMM_BK);
+      EpiQuant::Params ep{c->mub, c->delta, c->keep, (float)std::ldexp(1.0, -c->p_y), q32, qe, row_edst};
+      RET((run_gemm_chunked<EpiQuantTotals, 3, 2, 2>(c->map_ay2, c->map_aw2_2, mb_x256, mb_g, pr, ep, c->num_sms,
+                                                      st)));
+    }
+    stage_mark(c, st, "gemm_transform");
+    // odd mean model: [e, bf16(q_left), bf16(q_right)] @ w_odd -> centres
+    {
+      GemmProblem pr = make_problem(N_COEF / GEMM_BM, L.ne_pad, 256, true, status_dev);
+      add_seg(pr, 0, 0, 1, 0, 0, 0, 0, N_COEF / GEMM_BK);
+      add_seg(pr, 0, 0, 1, N_COEF, 0, 1, 0, N_COEF / GEMM_BK);
+      EpiMeanOdd::Params ep{c->t_odd, token_ids, e_tok, c_odd, c->vocab};
+      RET((run_gemm<EpiMeanOdd, 4, 1>(c->map_aon1, c->map_aon1, mb_qe, mb_qe, pr, ep, c->num_sms, st)));
+    }
+    stage_mark(c, st, "gemm_mean_odd");
+  }
+  uint32_t *states = (uint32_t *)(ws + w.states), *nwords = (uint32_t *)(ws + w.nwords);
+  uint32_t *nesc = (uint32_t *)(ws + w.nesc), *offs = (uint32_t *)(ws + w.offs);
+  if (L.n_chunks > 0) {
+    RansEncArgs a{d_chunks, d_prompts, L.n_chunks, c->k_eff, c->kept_list, c->kept_scale, c->cdf, q32,
+                  c->t_even, token_ids, c_odd, c->vocab, (uint16_t *)(ws + w.words), states, nwords, nesc};
+    CK(cudaFuncSetAttribute(rans_encode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, CDF_SMEM_BYTES));
+    rans_encode_kernel<<<(L.n_chunks + RANS_WARPS - 1) / RANS_WARPS, RANS_WARPS * 32, CDF_SMEM_BYTES, st>>>(a);
+    CK(cudaGetLastError());
+  }
+  stage_mark(c, st, "rans_encode");
+  {
+    ScanArgs a{L.n_chunks, nwords, nesc, offs, bl, blob_cap, L.off_kept, L.off_streams, d_prompts, L.batch,
+               c->chunk_rows, c->k_eff, L.n_chunks_e, L.n_chunks_o, L.n_kept, blob_size_dev, status_dev};
+    scan_kernel<<<1, 1024, 0, st>>>(a);
+    CK(cudaGetLastError());
+  }
+  if (L.n_chunks > 0) {
+    CompactArgs a{d_chunks, d_prompts, L.n_chunks, c->k_eff, c->kept_list, q32, (const uint16_t *)(ws + w.words),
+                  states, nwords, nesc, offs, bl, blob_cap, L.off_streams};
+    compact_kernel<<<(L.n_chunks + RANS_WARPS - 1) / RANS_WARPS, RANS_WARPS * 32, 0, st>>>(a);
+    CK(cudaGetLastError());
+  }
+  stage_mark(c, st, "scan+compact");
+  return DCKV_OK;
+}
+
+// ============================================================================ decode
+extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_bytes, const int32_t *token_ids,
+                           const int64_t *seq_offsets, int batch, void *k_out, void *v_out, int32_t *status_dev,
+                           void *workspace, size_t ws_bytes, void *stream) {
+  if (!c || !blob || !token_ids || !k_out || !v_out || !status_dev || !workspace)
+    return fail(DCKV_EINVAL, "a pointer argument is NULL");
+  if (((uintptr_t)blob & 15) || ((uintptr_t)k_out & 15) || ((uintptr_t)v_out & 15) || ((uintptr_t)workspace & 255))
+    return fail(DCKV_EINVAL, "blob/k_out/v_out must be 16-byte and workspace 256-byte aligned");
+  Layout L;
+  RET(build_layout(c, seq_offsets, batch, L));
+  const WsPlan w = plan_ws(L, 1);
+  if (ws_bytes < w.total) return fail(DCKV_ECAPACITY, "workspace too small (%zu < %zu)", ws_bytes, w.total);
+  cudaStream_t st = (cudaStream_t)stream;
+  CK(cudaSetDevice(c->device));
+  dckv_codec *cm = const_cast<dckv_codec *>(c);
+  cm->n_ev = 0;
+  uint8_t *ws = (uint8_t *)workspace;
+  const uint8_t *bl = (const uint8_t *)blob;
+  PromptInfo *d_prompts = (PromptInfo *)(ws + w.prompts);
+  ChunkDesc *d_chunks = (ChunkDesc *)(ws + w.chunks);
+  int32_t *row_tok = (int32_t *)(ws + w.row_tok), *row_pos = (int32_t *)(ws + w.row_pos);
+  int32_t *row_edst = (int32_t *)(ws + w.row_edst), *e_tok = (int32_t *)(ws + w.e_tok);
+  __nv_bfloat16 *qe = (__nv_bfloat16 *)(ws + w.qe);
+  int8_t *c_odd = (int8_t *)(ws + w.c_odd);
+  __half *q16 = (__half *)(ws + w.q16);
+  int32_t *qbig = (int32_t *)(ws + w.qbig);
+  uint32_t *bigflag = (uint32_t *)(ws + w.bigflag);
+  int32_t *biglist = (int32_t *)(ws + w.biglist);
+  uint32_t *counters = (uint32_t *)(ws + w.counters);  // [0] big-row count, [1] header valid
+  int32_t *valid = (int32_t *)(counters + 1);
+
+  stage_mark(c, st, "start");
+  CK(cudaMemsetAsync(status_dev, 0, 4, st));
+  CK(cudaMemsetAsync(counters, 0, 256, st));
+  RET(upload_tables(L, ws, w, st));
+  CK(cudaMemsetAsync(qe, 0, 2ull * L.ne_pad * N_COEF, st));
+  if (L.n_rows) {
+    CK(cudaMemsetAsync(q16, 0, 2ull * L.n_rows * N_COEF, st));
+    CK(cudaMemsetAsync(bigflag, 0, 4ull * L.n_rows, st));
+  }
+  k_layout<<<L.batch, 256, 0, st>>>(d_prompts, row_tok, row_pos, row_edst, e_tok, nullptr);
+  HeaderCheck hc{bl, blob_bytes, d_prompts, L.batch, c->chunk_rows, c->k_eff, L.n_chunks_e, L.n_chunks_o,
+                 L.n_kept, L.off_kept, L.off_streams, valid, status_dev};
+  k_check_header<<<1, 256, 0, st>>>(hc);
+  CK(cudaGetLastError());
+  stage_mark(c, st, "layout+check");
+  const uint32_t *offs = (const uint32_t *)(bl + HEADER_BYTES + 4ull * L.batch);
+  CK(cudaFuncSetAttribute(rans_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, CDF_SMEM_BYTES));
+  RansDecArgs da{d_chunks, d_prompts, 0, L.n_chunks_e, c->k_eff, c->kept_list, c->kept_scale, c->cdf, c->t_even,
+                 token_ids, c_odd, c->vocab, bl, L.off_streams, offs, q16, qe, qbig, bigflag, biglist, counters,
+                 valid, status_dev};
+  if (L.n_chunks_e > 0) {
+    rans_decode_kernel<<<(L.n_chunks_e + RANS_WARPS - 1) / RANS_WARPS, RANS_WARPS * 32, CDF_SMEM_BYTES, st>>>(da);
+    CK(cudaGetLastError());
+  }
+  stage_mark(c, st, "rans_even");
+  if (L.n_rows > 0) {
+    CUtensorMap mb_qe;
+    RET(map_b(&mb_qe, qe, true, N_COEF, L.ne_pad, 256));
+    GemmProblem pr = make_problem(N_COEF / GEMM_BM, L.ne_pad, 256, true, status_dev);
+    add_seg(pr, 0, 0, 1, 0, 0, 0, 0, N_COEF / GEMM_BK);
+    add_seg(pr, 0, 0, 1, N_COEF, 0, 1, 0, N_COEF / GEMM_BK);
+    EpiMeanOdd::Params ep{c->t_odd, token_ids, e_tok, c_odd, c->vocab};
+    RET((run_gemm<EpiMeanOdd, 4, 1>(c->map_aon1, c->map_aon1, mb_qe, mb_qe, pr, ep, c->num_sms, st)));
+  }
+  stage_mark(c, st, "gemm_mean_odd");
+  if (L.n_chunks_o > 0) {
+    da.chunk0 = L.n_chunks_e;
+    da.n_chunks = L.n_chunks_o;
+    rans_decode_kernel<<<(L.n_chunks_o + RANS_WARPS - 1) / RANS_WARPS, RANS_WARPS * 32, CDF_SMEM_BYTES, st>>>(da);
+    CK(cudaGetLastError());
+  }
+  stage_mark(c, st, "rans_odd");
+  if (L.n_rows > 0) {
+    CUtensorMap mb_q;
+    RET(map_b(&mb_q, q16, false, N_COEF, L.n_rows, 256));
+    GemmProblem pr = make_problem(ROW_DIM / GEMM_BM, L.n_rows, 256, false, status_dev);
+    add_seg(pr, 0, 0, 2, 0, 0, 0, 0, N_COEF / GEMM_BK);
+    EpiInverse::Params ep{c->mu_perm, (float)std::ldexp(1.0, -c->p_inv), c->theta, row_tok, row_pos,
+                          (__nv_bfloat16 *)k_out, (__nv_bfloat16 *)v_out, L.n_tokens};
+    RET((run_gemm<EpiInverse, 3, 2>(c->map_ainv2, c->map_ainv2, mb_q, mb_q, pr, ep, c->num_sms, st)));
+  }
+  stage_mark(c, st, "gemm_inverse");
+  if (L.n_kept > 0)
+    k_kept<<<(unsigned)L.n_kept, 256, 0, st>>>(bl, L.off_kept, d_prompts, L.batch, c->theta, (__nv_bfloat16 *)k_out,
+                                              (__nv_bfloat16 *)v_out, L.n_tokens, valid);
+  if (L.n_rows > 0)
+    k_fixup<<<c->num_sms, 256, 0, st>>>(biglist, counters, q16, qbig, c->a_inv, (float)std::ldexp(1.0, -c->p_inv),
+                                       c->mu_perm, c->theta, row_tok, row_pos, (__nv_bfloat16 *)k_out,
+                                       (__nv_bfloat16 *)v_out, L.n_tokens);
+  CK(cudaGetLastError());
+  stage_mark(c, st, "kept+fixup");
+  return DCKV_OK;
+}
+
+// ============================================================================ bytes
+extern "C" int dckv_bytes(const void *blob_host, size_t len, dckv_byte_report *out) {
+  if (!blob_host || !out) return fail(DCKV_EINVAL, "NULL argument");
+  memset(out, 0, sizeof(*out));
+  const uint8_t *b = (const uint8_t *)blob_host;
+  if (len < (size_t)HEADER_BYTES) return fail(DCKV_ECORRUPT, "blob shorter than its header");
+  uint32_t h32[8];
+  uint16_t h16[4];
+  uint64_t h64[4];
+  memcpy(h32, b, 32);
+  memcpy(h16, b, 8);
+  memcpy(h64, b + 32, 32);
+  if (h32[0] != MAGIC || h16[2] != VERSION || h32[3] != (uint32_t)N_COEF || h16[3] == 0)
+    return fail(DCKV_ECORRUPT, "bad header");
+  const uint64_t total = h64[0], off_s = h64[1], off_k = h64[2];
+  const uint32_t nb = h32[2], n_ch = h32[5] + h32[6], n_kept = h32[7];
+  if (total > len) return fail(DCKV_ECORRUPT, "blob truncated");
+  const uint64_t tab_end = HEADER_BYTES + 4ull * (nb + (uint64_t)n_ch + 1);
+  if (tab_end > total || off_k != align_up(tab_end, 16) || off_s != off_k + (uint64_t)n_kept * ROW_DIM * 2 ||
+      off_s > total)
+    return fail(DCKV_ECORRUPT, "bad offsets");
+  std::vector<uint32_t> lens(nb), offs(n_ch + 1);
+  memcpy(lens.data(), b + HEADER_BYTES, 4ull * nb);
+  memcpy(offs.data(), b + HEADER_BYTES + 4ull * nb, 4ull * (n_ch + 1));
+  if (off_s + offs[n_ch] != total) return fail(DCKV_ECORRUPT, "chunk table does not reach the end");
+  uint64_t rows = 0;
+  for (uint32_t n : lens) rows += n > (uint32_t)(HEAD_KEPT + TAIL_KEPT) ? n - HEAD_KEPT - TAIL_KEPT : 0;
+  for (uint32_t ci = 0; ci < n_ch; ++ci) {
+    if (offs[ci + 1] < offs[ci] || offs[ci + 1] - offs[ci] < (uint32_t)CHUNK_FIXED_BYTES)
+      return fail(DCKV_ECORRUPT, "bad chunk %u", ci);
+    uint32_t ne;
+    memcpy(&ne, b + off_s + offs[ci] + 4 * LANES, 4);
+    const uint64_t sz = offs[ci + 1] - offs[ci];
+    if (CHUNK_FIXED_BYTES + 8ull * ne > sz) return fail(DCKV_ECORRUPT, "bad escape count in chunk %u", ci);
+    out->states += 4 * LANES;
+    out->esc_counts += 4;
+    out->esc_values += 8ull * ne;
+    out->n_escapes += ne;
+    // words cannot be told from a trailing zero pad word without decoding; count both
+    out->words += sz - CHUNK_FIXED_BYTES - 8ull * ne;
+  }
+  out->total = total;
+  out->header_tables = off_k;
+  out->kept_rows = off_s - off_k;
+  out->payload = total - out->kept_rows;
+  out->padding = 0;
+  out->n_prompts = nb;
+  out->n_chunks = n_ch;
+  out->n_coded_rows = (uint32_t)rows;
+  out->chunk_rows = h16[3];
+  out->k_eff = h32[4];
+  return DCKV_OK;
+}
+
+// ============================================================================ inspection
+extern "C" int dckv_set_timing(dckv_codec *c, int enable) {
+  if (!c) return DCKV_EINVAL;
+  c->timing = enable ? 1 : 0;
+  c->n_ev = 0;
+  return DCKV_OK;
+}
+
+extern "C" int dckv_get_timing(const dckv_codec *c, float *ms, const char **names, int max) {
+  if (!c || !ms) return -1;
+  int n = 0;
+  for (int i = 1; i < c->n_ev && n < max; ++i, ++n) {
+    float t = 0.f;
+    cudaEventElapsedTime(&t, c->ev[i - 1], c->ev[i]);
+    ms[n] = t;
+    if (names) names[n] = c->ev_names[i];
+  }
+  return n;
+}
+
+extern "C" int dckv_codec_export(const dckv_codec *c, uint16_t *cdf_host, uint8_t *scale_host, uint8_t *keep_host,
+                                 int32_t *exps_host) {
+  if (!c) return fail(DCKV_EINVAL, "NULL codec");
+  CK(cudaSetDevice(c->device));
+  if (cdf_host) CK(cudaMemcpy(cdf_host, c->cdf, 2ull * N_SCALES * N_SYM, cudaMemcpyDeviceToHost));
+  if (scale_host) CK(cudaMemcpy(scale_host, c->scale, N_COEF, cudaMemcpyDeviceToHost));
+  if (keep_host) CK(cudaMemcpy(keep_host, c->keep, N_COEF, cudaMemcpyDeviceToHost));
+  if (exps_host) {
+    exps_host[0] = c->p_y;
+    exps_host[1] = c->p_h;
+    exps_host[2] = c->p_inv;
+  }
+  return DCKV_OK;
+}
+
+extern "C" int dckv_codec_tables(const dckv_codec *c, const void **t_even, const void **t_odd) {
+  if (!c) return fail(DCKV_EINVAL, "NULL codec");
+  if (t_even) *t_even = c->t_even;
+  if (t_odd) *t_odd = c->t_odd;
+  return DCKV_OK;
+}
+
+extern "C" int dckv_ws_offsets(const dckv_codec *c, const int64_t *offs, int batch, int which, dckv_ws_view *out) {
+  if (!c || !out) return fail(DCKV_EINVAL, "NULL argument");
+  Layout L;
+  RET(build_layout(c, offs, batch, L));
+  const WsPlan w = plan_ws(L, which);
+  out->q32 = w.q32;
+  out->qe = w.qe;
+  out->c_odd = w.c_odd;
+  out->q16 = w.q16;
+  out->x16 = w.x16;
+  out->g16 = w.g16;
+  out->n_rows = L.n_rows;
+  out->ne_pad = L.ne_pad;
+  out->n_chunks = L.n_chunks;
+  out->total = w.total;
+  return DCKV_OK;
+}
+
+// D[n][m] = sum_s sum_k A[s][m][k] * B[n][k] through the tcgen05 GEMM (self-test).
+extern "C" int dckv_debug_gemm(int bf16, const void *A, int slabs, const void *Bm, int M, int N, int K, float *D,
+                               int bn, void *stream) {
+  if (!A || !Bm || !D || M % GEMM_BM || K % GEMM_BK || N < 1 || slabs < 1 || slabs > 2 || bn < 16 || bn > 256 ||
+      bn % 16)
+    return fail(DCKV_EINVAL, "bad GEMM shape");
+  int dev;
+  CK(cudaGetDevice(&dev));
+  int sms;
+  CK(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  CUtensorMap ma, mb;
+  RET(map_a(&ma, A, bf16 != 0, K, M, slabs, slabs));
+  RET(map_b(&mb, Bm, bf16 != 0, K, N, bn));
+  GemmProblem pr = make_problem(M / GEMM_BM, N, bn, bf16 != 0, nullptr);
+  add_seg(pr, 0, 0, slabs, 0, 0, 0, 0, K / GEMM_BK);
+  EpiStoreF32::Params ep{D, M, 1.0f};
+  return run_gemm<EpiStoreF32, 3, 2>(ma, ma, mb, mb, pr, ep, sms, (cudaStream_t)stream);
+}

@@ -1,0 +1,113 @@
+// dckv_internal.cuh -- shared definitions of the DCKV library (host + device).
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <vector>
+
+#include "../../include/dckv.h"
+
+namespace dckv {
+
+constexpr int ROW_DIM = DCKV_ROW_DIM;     // 6144
+constexpr int N_COEF = DCKV_N_COEF;       // 2048
+constexpr int N_HIDDEN = DCKV_N_HIDDEN;   // 256
+constexpr int HEAD_DIM = DCKV_HEAD_DIM;   // 256
+constexpr int HEAD_KEPT = DCKV_HEAD_KEPT;
+constexpr int TAIL_KEPT = DCKV_TAIL_KEPT;
+constexpr int ESC_LIMIT = 127;            // codes beyond +-127 are escaped
+constexpr int R_MAX = 2 * ESC_LIMIT;      // residual q - centre in [-254, 254]
+constexpr int N_SYM = 2 * R_MAX + 2;      // 509 residual symbols + ESC
+constexpr int ESC_SYM = N_SYM - 1;        // 509
+constexpr int N_SCALES = 64;
+constexpr uint32_t PREC_TOTAL = 1u << 16; // 16-bit frequency precision
+constexpr uint32_t RANS_L = 1u << 16;     // lower bound of a 32-bit state
+constexpr int LANES = 32;                 // interleaved states per chunk
+constexpr double B0_STEPS = 0.05;         // drop threshold and scale-index origin (steps)
+constexpr double ROPE_BASE = 1.0e7;
+constexpr uint32_t MAGIC = 0x564B4344u;   // "DCKV"
+constexpr int VERSION = 1;
+constexpr int HEADER_BYTES = 64;
+constexpr int CHUNK_FIXED_BYTES = 4 * LANES + 4;  // states + escape count
+constexpr int BIG_CODE = 2048;            // |q| >= 2048 is not exact in the fp16 code operand
+
+struct PromptInfo {
+  int64_t tok_base;  // first row (token) of the prompt in the batch
+  int32_t N;         // tokens
+  int32_t n;         // coded rows = max(0, N - 132)
+  int32_t n_e, n_o;  // even / odd coded rows
+  int32_t row_base;  // first coded row, natural order over the batch
+  int32_t ebase;     // first padded even row (each prompt owns n_e + 1 rows, last one zero)
+  int32_t kept_base; // first kept row in the blob's kept section
+  int32_t n_kept;
+  int32_t chunk_e0, chunk_o0;  // first even / odd chunk (global chunk index)
+};
+
+struct ChunkDesc {
+  int32_t prompt, parity, j0, nrows;
+  int64_t sym_base;  // first symbol slot in the word scratch (rows before * K_eff)
+};
+
+// Host-side batch layout, derived from seq_offsets only.
+struct Layout {
+  int batch = 0;
+  int64_t n_tokens = 0;
+  int64_t n_rows = 0;     // coded rows
+  int64_t ne_pad = 0;     // padded even rows (sum of n_e + 1)
+  int64_t n_kept = 0;
+  int n_chunks = 0, n_chunks_e = 0, n_chunks_o = 0;
+  int64_t n_symbols = 0;  // n_rows * K_eff
+  std::vector<PromptInfo> prompts;
+  std::vector<ChunkDesc> chunks;
+  uint64_t off_kept = 0, off_streams = 0;  // blob offsets
+};
+
+// Workspace carving (byte offsets from the workspace base, each 256-aligned).
+struct WsPlan {
+  size_t prompts, chunks, row_tok, row_pos, row_edst, e_tok;  // tables
+  size_t x16, g16, q32, qe, c_odd, words, states, nwords, nesc, offs;  // encode
+  size_t q16, qbig, bigflag, biglist, counters, valid;                  // decode
+  size_t total;
+};
+
+}  // namespace dckv
+
+// the opaque codec
+struct dckv_codec {
+  int device = 0;
+  int num_sms = 0;
+  int chunk_rows = 32;
+  int vocab = 0;
+  int k_eff = 0;
+  // caller-owned parameter pointers (read at create)
+  dckv_params p{};
+  // derived, library-owned device buffers
+  void *blk = nullptr;  // one allocation holding everything below
+  __half *a_y = nullptr;     // [2][2048][6144]  basis^T * 2^p_y, split hi/lo
+  __half *a_w2 = nullptr;    // [2][2048][256]   w2^T * 2^p_y, split
+  __half *a_h = nullptr;     // [2][256][6144]   w1^T * 2^p_h, split
+  __half *a_inv = nullptr;   // [2][6144][2048]  (Delta_c basis[d][c]) * 2^p_inv, dims permuted
+  __nv_bfloat16 *a_on = nullptr;  // [2048][4096]  odd mean model, neighbour blocks, transposed
+  float *t_even = nullptr;   // [vocab][2048]  embed @ w_even
+  float *t_odd = nullptr;    // [vocab][2048]  embed @ w_odd[0:2048]
+  float *mub = nullptr;      // [2048]  mu @ basis
+  float *muw1 = nullptr;     // [256]   mu @ w1
+  float *mu_perm = nullptr;  // [6144]  mu in the inverse GEMM's row order
+  float *delta = nullptr;    // [2048]
+  uint8_t *keep = nullptr;   // [2048]
+  uint8_t *scale = nullptr;  // [2048]
+  int16_t *kept_list = nullptr;   // [2048] kept component indices (first k_eff valid)
+  uint8_t *kept_scale = nullptr;  // [2048]
+  uint16_t *cdf = nullptr;   // [64][510]  cumulative frequencies (cdf[510] = 65536 implied)
+  double *theta = nullptr;   // [128] RoPE frequencies
+  int p_y = 0, p_h = 0, p_inv = 0;  // power-of-two operand scales
+  CUtensorMap map_ay2, map_aw2_2, map_aw2_1, map_ah2, map_ainv2, map_aon1;
+  // stage timing (optional)
+  int timing = 0;
+  cudaEvent_t ev[24];
+  int n_ev = 0;
+  const char *ev_names[24];
+};

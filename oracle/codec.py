@@ -35,7 +35,8 @@ __all__ = [
     "VERSION", "HEADER_BYTES", "DEFAULT_CHUNK_ROWS",
     "bf16_to_f64", "f64_to_bf16", "gelu", "transform", "scale_index", "quantise",
     "laplace_tables", "prompt_layout", "chunk_list", "mean_even", "mean_odd", "centres",
-    "symbols", "rans_encode", "rans_decode", "encode", "decode", "parse_blob",
+    "symbols", "rans_encode", "rans_decode", "encode", "decode", "parse_blob", "analyse",
+    "assemble_blob",
     "byte_report", "model_code_length_bits", "rope", "reconstruct", "kept_positions",
     "output_rows",
 ]
@@ -378,27 +379,19 @@ def _pad(buf: bytearray, align: int):
         buf.append(0)
 
 
-def encode(x, tok, seq_offsets, codec, chunk_rows: int = DEFAULT_CHUNK_ROWS, aux: dict | None = None):
-    """Encode a batch of prompts into one blob (bytes).
+def analyse(x, tok, seq_offsets, codec):
+    """Codes and centres of every prompt (the arithmetic of encoding, before the coder).
 
-    x: [sum N, 6144] rows (bf16 bits as uint16, or floats); tok: [sum N] token ids;
-    seq_offsets: [B+1].  Steps: transform -> quantise -> drop -> even means from the
-    token embedding -> odd means from embedding + both even neighbours -> centres ->
-    symbols -> rANS per chunk -> blob.  If `aux` is a dict it receives the intermediates
-    (q, ratio, centres, symbols per prompt and parity)."""
+    Per prompt: transform -> quantise -> drop; even means from the token embedding; odd
+    means from the embedding and both even neighbours; centres.  Returns a list of dicts
+    with q, ratio (y / Delta), qe, qo, mu_e, mu_o, ce, co."""
     x = np.asarray(x)
     tok = np.asarray(tok, np.int64)
     offs = np.asarray(seq_offsets, np.int64)
-    lens = np.diff(offs)
-    layout = prompt_layout(lens)
+    layout = prompt_layout(np.diff(offs))
     s_idx, keep = scale_index(codec.laplace_b, codec.delta)
-    kept_c = np.nonzero(keep)[0]
-    k_eff = kept_c.size
-    freq, cdf = laplace_tables()
-    chunks, n_ev, n_od = chunk_list(layout, chunk_rows)
-
-    per_prompt = []
-    for b, L in enumerate(layout):
+    out = []
+    for L in layout:
         t0 = L["tok_base"]
         n = L["n"]
         rows = x[t0 + HEAD_KEPT: t0 + HEAD_KEPT + n]
@@ -409,35 +402,57 @@ def encode(x, tok, seq_offsets, codec, chunk_rows: int = DEFAULT_CHUNK_ROWS, aux
             q = np.zeros((0, N_COEF), np.int64)
             ratio = np.zeros((0, N_COEF))
         qe, qo = q[0::2], q[1::2]
-        te = tok[t0 + HEAD_KEPT + 0: t0 + HEAD_KEPT + n: 2]
+        te = tok[t0 + HEAD_KEPT: t0 + HEAD_KEPT + n: 2]
         to = tok[t0 + HEAD_KEPT + 1: t0 + HEAD_KEPT + n: 2]
         mu_e = mean_even(codec.embed[te], codec.w_even) if qe.shape[0] else np.zeros((0, N_COEF))
         q_right = np.concatenate([qe[1:], np.zeros((1, N_COEF), np.int64)], 0)[: qo.shape[0]]
         mu_o = (mean_odd(codec.embed[to], qe[: qo.shape[0]], q_right, codec.w_odd)
                 if qo.shape[0] else np.zeros((0, N_COEF)))
-        ce, co = centres(mu_e), centres(mu_o)
-        se, esc_e = symbols(qe, ce, keep)
-        so, esc_o = symbols(qo, co, keep)
-        per_prompt.append(dict(q=q, ratio=ratio, qe=qe, qo=qo, mu_e=mu_e, mu_o=mu_o,
-                               ce=ce, co=co, se=se, so=so, esc_e=esc_e, esc_o=esc_o))
+        out.append(dict(q=q, ratio=ratio, qe=qe, qo=qo, mu_e=mu_e, mu_o=mu_o, ce=centres(mu_e), co=centres(mu_o)))
+    return out
+
+
+def assemble_blob(x, seq_offsets, codes, laplace_b, delta, chunk_rows: int = DEFAULT_CHUNK_ROWS,
+                  aux: dict | None = None):
+    """The coder and the container: symbols from (q, centre), rANS per chunk, escapes,
+    kept rows, header and tables.  `codes` is a list (per prompt) of dicts with qe, qo,
+    ce, co (codes and centres of even / odd rows)."""
+    x = np.asarray(x)
+    offs = np.asarray(seq_offsets, np.int64)
+    lens = np.diff(offs)
+    layout = prompt_layout(lens)
+    s_idx, keep = scale_index(laplace_b, delta)
+    kept_c = np.nonzero(keep)[0]
+    k_eff = kept_c.size
+    freq, cdf = laplace_tables()
+    chunks, n_ev, n_od = chunk_list(layout, chunk_rows)
+    syms = []
+    for P in codes:
+        se, esc_e = symbols(P["qe"], P["ce"], keep)
+        so, esc_o = symbols(P["qo"], P["co"], keep)
+        syms.append((se, so))
 
     streams = bytearray()
     offsets = []
     n_esc_total = 0
     code_bits = 0.0
+    sections = []
     for (b, par, j0, nr) in chunks:
-        P = per_prompt[b]
-        sym = (P["se"] if par == 0 else P["so"])[j0:j0 + nr].reshape(-1)
+        P = codes[b]
+        sym = syms[b][par][j0:j0 + nr].reshape(-1)
         qk = ((P["qe"] if par == 0 else P["qo"])[j0:j0 + nr])[:, kept_c].reshape(-1)
         scl = np.tile(s_idx[kept_c], nr).astype(np.uint8)
         states, words = rans_encode(sym, scl, freq, cdf)
         escv = qk[sym == ESC_SYMBOL]
         offsets.append(len(streams))
-        streams += states.astype("<u4").tobytes()
-        streams += struct.pack("<I", escv.size)
-        streams += escv.astype("<i8").tobytes()
-        streams += words.astype("<u2").tobytes()
-        _pad(streams, 4)
+        sec = bytearray()
+        sec += states.astype("<u4").tobytes()
+        sec += struct.pack("<I", escv.size)
+        sec += escv.astype("<i8").tobytes()
+        sec += words.astype("<u2").tobytes()
+        _pad(sec, 4)
+        streams += sec
+        sections.append(bytes(sec))
         n_esc_total += escv.size
         code_bits += model_code_length_bits(sym, scl, freq, escv.size)
     offsets.append(len(streams))
@@ -450,26 +465,41 @@ def encode(x, tok, seq_offsets, codec, chunk_rows: int = DEFAULT_CHUNK_ROWS, aux
             kept_rows.append(L["tok_base"] + p)
     n_kept = len(kept_rows)
 
+    # layout: header | prompt lengths | chunk offsets | pad16 | kept rows | chunk sections
     blob = bytearray(HEADER_BYTES)
     blob += np.asarray(lens, "<u4").tobytes()
     blob += np.asarray(offsets, "<u4").tobytes()
-    _pad(blob, 16)
-    off_streams = len(blob)
-    blob += streams
     _pad(blob, 16)
     off_kept = len(blob)
     if n_kept:
         kr = x[np.asarray(kept_rows)]
         kr_bits = kr if kr.dtype == np.uint16 else f64_to_bf16(kr)
         blob += np.ascontiguousarray(kr_bits, "<u2").tobytes()
+    off_streams = len(blob)
+    blob += streams
     total = len(blob)
     struct.pack_into("<IHHIIIIII", blob, 0, MAGIC, VERSION, chunk_rows, len(lens), N_COEF,
                      k_eff, n_ev, n_od, n_kept)
     struct.pack_into("<QQQQ", blob, 32, total, off_streams, off_kept, 0)
     if aux is not None:
-        aux.update(per_prompt=per_prompt, layout=layout, chunks=chunks, keep=keep, s_idx=s_idx,
-                   n_esc=n_esc_total, code_bits=code_bits, freq=freq, cdf=cdf)
+        aux.update(layout=layout, chunks=chunks, keep=keep, s_idx=s_idx, n_esc=n_esc_total,
+                   code_bits=code_bits, freq=freq, cdf=cdf, sections=sections)
     return bytes(blob)
+
+
+def encode(x, tok, seq_offsets, codec, chunk_rows: int = DEFAULT_CHUNK_ROWS, aux: dict | None = None):
+    """Encode a batch of prompts into one blob (bytes).
+
+    x: [sum N, 6144] rows (bf16 bits as uint16, or floats); tok: [sum N] token ids;
+    seq_offsets: [B+1].  Steps: transform -> quantise -> drop -> even means from the
+    token embedding -> odd means from embedding + both even neighbours -> centres ->
+    symbols -> rANS per chunk -> blob.  If `aux` is a dict it receives the intermediates
+    (per_prompt: q, ratio, centres, means per prompt and parity)."""
+    per_prompt = analyse(x, tok, seq_offsets, codec)
+    blob = assemble_blob(x, seq_offsets, per_prompt, codec.laplace_b, codec.delta, chunk_rows, aux)
+    if aux is not None:
+        aux["per_prompt"] = per_prompt
+    return blob
 
 
 def parse_blob(blob):
@@ -484,10 +514,15 @@ def parse_blob(blob):
     if total > len(blob):
         raise ValueError("blob truncated")
     p = HEADER_BYTES
+    if p + 4 * (nb + n_ev + n_od + 1) > total:
+        raise ValueError("tables overrun the blob")
     lens = np.frombuffer(blob, "<u4", nb, p).astype(np.int64)
     p += 4 * nb
     offs = np.frombuffer(blob, "<u4", n_ev + n_od + 1, p).astype(np.int64)
-    if np.any(np.diff(offs) < 0) or off_s + offs[-1] > off_k or off_k > total:
+    p += 4 * (n_ev + n_od + 1)
+    p = (p + 15) // 16 * 16
+    if (off_k != p or off_s != off_k + n_kept * ROW_DIM * 2 or offs[0] != 0
+            or np.any(np.diff(offs) < 4 * LANES + 4) or off_s + offs[-1] != total):
         raise ValueError("bad chunk table")
     return dict(chunk_rows=G, n_prompts=nb, k_eff=k_eff, n_chunks_even=n_ev, n_chunks_odd=n_od,
                 n_kept=n_kept, total=total, off_streams=off_s, off_kept=off_k, lens=lens,
@@ -594,7 +629,15 @@ def decode(blob, tok, seq_offsets, codec, aux: dict | None = None):
 
 def byte_report(blob, aux: dict | None = None):
     """Byte breakdown: header+tables, states, escape counts, escape values, words,
-    padding, kept rows; payload = everything except the kept rows."""
+    padding, kept rows; payload = everything except the kept rows.
+
+    Blob layout (little endian): 64-byte header {u32 magic 'DCKV', u16 version, u16 chunk
+    rows, u32 prompts, u32 coefficients, u32 kept components, u32 even chunks, u32 odd
+    chunks, u32 kept rows, u64 total bytes, u64 stream offset, u64 kept-row offset, u64 0};
+    u32 prompt lengths; u32 chunk-section offsets (relative to the stream offset, one more
+    than the chunks); zero pad to 16; kept rows (bf16, prompt-major, ascending position);
+    chunk sections, each {u32 states[32], u32 escape count, i64 escape codes, u16 words in
+    decoder order, zero pad to 4}."""
     blob = bytes(blob)
     hdr = parse_blob(blob)
     n_ch = hdr["n_chunks_even"] + hdr["n_chunks_odd"]
@@ -605,7 +648,8 @@ def byte_report(blob, aux: dict | None = None):
         esc_cnt += 4
         esc_val += 8 * ev.size
         words += 2 * w.size
-    kept = hdr["total"] - hdr["off_kept"]
-    return dict(total=hdr["total"], header_tables=hdr["off_streams"], states=states,
+    kept = hdr["off_streams"] - hdr["off_kept"]
+    return dict(total=hdr["total"], header_tables=hdr["off_kept"], states=states,
                 esc_counts=esc_cnt, esc_values=esc_val, words=words, kept_rows=kept,
-                payload=hdr["off_kept"], padding=hdr["total"] - states - esc_cnt - esc_val - words - kept - hdr["off_streams"])
+                payload=hdr["total"] - kept,
+                padding=hdr["total"] - kept - hdr["off_kept"] - states - esc_cnt - esc_val - words)

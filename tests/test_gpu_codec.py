@@ -1,0 +1,316 @@
+"""GPU codec vs the CPU oracle, element by element, through the C ABI.
+
+Parity rules (one GPU, seeded synthetic inputs):
+  codes      bit-exact, except |dq| = 1 flips where the oracle's y / Delta lies within
+             1e-3 of a half-step boundary, and such flips are at most 0.1% of codes;
+  centres    equal to the oracle's centres computed from the same codes, except where the
+             oracle's mean lies within 1e-4 of a half-step boundary (fp32 vs fp64 sums);
+  bitstream  given the GPU's codes and centres, the oracle coder and container produce
+             the GPU's blob byte for byte;
+  rows       decoded K/V within 1e-3 relative Frobenius of the oracle's decode of the
+             same blob (both rounded to bf16), and GPU decode reproduces the GPU encoder's
+             codes exactly;
+  determinism  repeated calls give identical blobs and rows.
+"""
+import numpy as np
+import pytest
+import torch
+
+import dckv_synth as S
+import learned_kv_cache_dckv_b200 as D
+import oracle as O
+
+pytestmark = pytest.mark.gpu
+
+FLIP_WINDOW = 1e-3
+FLIP_MAX_FRAC = 1e-3
+CENTRE_WINDOW = 1e-4
+ROW_TOL = 1e-3
+
+
+class _CAI:
+    def __init__(self, ptr, shape, typestr):
+        self.__cuda_array_interface__ = dict(shape=shape, typestr=typestr, data=(ptr, False), version=3)
+
+
+def bits(x):
+    return x.detach().cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+_GPU_CODECS = {}
+
+
+def gpu_codec(np_codec, chunk_rows=0):
+    key = (id(np_codec), chunk_rows)
+    if key not in _GPU_CODECS:
+        _GPU_CODECS[key] = D.Codec(D.upload_params(np_codec), 0, chunk_rows)
+    return _GPU_CODECS[key]
+
+
+def make_batch(src, cod, lens, seeds, boost=(), boost_gain=60.0, student_t=0.0):
+    x, tok, offs = S.batch(src, lens, seeds, student_t_frac=student_t, device="cuda")
+    if boost:
+        mu = torch.from_numpy(cod.mu).cuda()
+        idx = torch.tensor(list(boost), device="cuda")
+        x[idx] = (mu + (x[idx].float() - mu) * boost_gain).to(torch.bfloat16)
+    return x, tok, offs
+
+
+def encode_gpu(gc, x, tok, offs):
+    blob = gc.encode(x, tok, offs)
+    torch.cuda.synchronize()
+    status = int(gc.status.item())
+    size = int(gc.blob_size.item())
+    v = D.dckv_ws_offsets(gc.handle, offs, 0)
+    ws = gc._ws
+    n, ne = v["n_rows"], v["ne_pad"]
+    q32 = ws[v["q32"]: v["q32"] + 4 * n * 2048].view(torch.int32).reshape(n, 2048).cpu().numpy()
+    c_odd = ws[v["c_odd"]: v["c_odd"] + ne * 2048].view(torch.int8).reshape(ne, 2048).cpu().numpy()
+    return dict(blob_dev=blob, blob=blob[:size].cpu().numpy().tobytes(), size=size, status=status, q32=q32,
+                c_odd=c_odd)
+
+
+def decode_gpu(gc, blob_dev, size, tok, offs):
+    k, v = gc.decode(blob_dev, size, tok, offs)
+    torch.cuda.synchronize()
+    w = D.dckv_ws_offsets(gc.handle, offs, 1)
+    n = w["n_rows"]
+    q16 = gc._ws[w["q16"]: w["q16"] + 2 * n * 2048].view(torch.float16).reshape(n, 2048).float().cpu().numpy()
+    return k, v, int(gc.status.item()), q16
+
+
+def gpu_even_centres(gc, np_codec, tok_rows):
+    te_ptr, _ = D.dckv_codec_tables(gc.handle)
+    te = torch.as_tensor(_CAI(te_ptr, (np_codec.embed.shape[0], 2048), "<f4"), device="cuda")
+    mu = te[torch.as_tensor(tok_rows, device="cuda", dtype=torch.long)]
+    return torch.clamp(torch.round(mu), -127, 127).to(torch.int64).cpu().numpy()
+
+
+def split_gpu_codes(gc, np_codec, res, tok, offs):
+    lay = O.prompt_layout(np.diff(offs))
+    out = []
+    ebase = 0
+    tok_np = tok.cpu().numpy().astype(np.int64)
+    for L in lay:
+        q = res["q32"][L["row_base"]: L["row_base"] + L["n"]].astype(np.int64)
+        t0 = L["tok_base"] + 4
+        te = tok_np[t0: t0 + L["n"]: 2]
+        ce = gpu_even_centres(gc, np_codec, te) if te.size else np.zeros((0, 2048), np.int64)
+        co = res["c_odd"][ebase: ebase + L["n_o"]].astype(np.int64)
+        out.append(dict(q=q, qe=q[0::2], qo=q[1::2], ce=ce, co=co))
+        ebase += L["n_e"] + 1
+    return out
+
+
+def near_half(v, window):
+    f = np.abs(v - np.floor(v) - 0.5)
+    return f < window
+
+
+def check_codes(gpu_q, ora):
+    d = gpu_q - ora["q"]
+    bad = d != 0
+    if bad.any():
+        assert np.all(np.abs(d[bad]) == 1), "code differs by more than one step"
+        assert np.all(near_half(ora["ratio"][bad], FLIP_WINDOW)), "flip away from a half-step boundary"
+    assert bad.sum() <= FLIP_MAX_FRAC * max(1, gpu_q.size)
+    return int(bad.sum())
+
+
+def check_centres(gc_codes, np_codec, tok, offs):
+    """Oracle centres from the GPU's own codes vs the GPU's centres."""
+    lay = O.prompt_layout(np.diff(offs))
+    tok_np = tok.cpu().numpy().astype(np.int64)
+    mism = 0
+    total = 0
+    for L, G in zip(lay, gc_codes):
+        t0 = L["tok_base"] + 4
+        te = tok_np[t0: t0 + L["n"]: 2]
+        to = tok_np[t0 + 1: t0 + L["n"]: 2]
+        for par, toks in ((0, te), (1, to)):
+            if toks.size == 0:
+                continue
+            if par == 0:
+                mu = O.mean_even(np_codec.embed[toks], np_codec.w_even)
+            else:
+                qe = G["qe"]
+                right = np.concatenate([qe[1:], np.zeros((1, 2048), np.int64)])[: toks.size]
+                mu = O.mean_odd(np_codec.embed[toks], qe[: toks.size], right, np_codec.w_odd)
+            ora_c = O.centres(mu)
+            gpu_c = G["ce"] if par == 0 else G["co"]
+            bad = ora_c != gpu_c
+            if bad.any():
+                assert np.all(np.abs(ora_c[bad] - gpu_c[bad]) == 1)
+                assert np.all(near_half(mu[bad], CENTRE_WINDOW)), "centre differs away from a boundary"
+            mism += int(bad.sum())
+            total += bad.size
+    assert mism <= 1e-4 * max(total, 1)
+    return mism
+
+
+def rel_frob(a, b):
+    a = a.astype(np.float64)
+    b = b.astype(np.float64)
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30))
+
+
+def full_check(src, np_codec, lens, seeds, chunk_rows=0, boost=(), boost_gain=60.0, student_t=0.0,
+               expect_escapes=False, expect_big=False):
+    gc = gpu_codec(np_codec, chunk_rows)
+    G = gc.handle
+    x, tok, offs = make_batch(src, np_codec, lens, seeds, boost, boost_gain, student_t)
+    res = encode_gpu(gc, x, tok, offs)
+    assert res["status"] == D.DCKV_OK, D.STATUS_NAMES[res["status"]]
+    xb = bits(x)
+    ora = O.analyse(xb, tok.cpu().numpy(), offs, np_codec)
+    codes = split_gpu_codes(gc, np_codec, res, tok, offs)
+    flips = sum(check_codes(c["q"], o) for c, o in zip(codes, ora))
+    mism = check_centres(codes, np_codec, tok, offs)
+    # bitstream: the oracle's coder and container on the GPU's codes and centres
+    aux = {}
+    ora_blob = O.assemble_blob(xb, offs, codes, np_codec.laplace_b, np_codec.delta,
+                               chunk_rows or 32, aux=aux)
+    assert len(ora_blob) == res["size"]
+    if ora_blob != res["blob"]:
+        hdr = O.parse_blob(ora_blob)
+        first = next(i for i in range(len(ora_blob)) if ora_blob[i] != res["blob"][i])
+        pytest.fail(f"blob differs first at byte {first} (streams start at {hdr['off_streams']})")
+    if expect_escapes:
+        assert aux["n_esc"] > 0
+    # decode on the GPU, and the oracle's decode of the same blob
+    k, v, st, q16 = decode_gpu(gc, res["blob_dev"], res["size"], tok, offs)
+    assert st == D.DCKV_OK, D.STATUS_NAMES[st]
+    small = np.abs(res["q32"]) < 2048
+    assert np.array_equal(q16[small], res["q32"][small].astype(np.float32))
+    if expect_big:
+        assert (~small).any()
+    k_o, v_o = O.decode(res["blob"], tok.cpu().numpy(), offs, np_codec)
+    kg, vg = bits(k), bits(v)
+    for g, o in ((kg, k_o), (vg, v_o)):
+        e = rel_frob(O.bf16_to_f64(g), O.bf16_to_f64(o))
+        assert e <= ROW_TOL, e
+    return dict(gc=gc, x=x, tok=tok, offs=offs, res=res, flips=flips, centre_mismatch=mism, k=k, v=v, aux=aux)
+
+
+# ------------------------------------------------------------------------------------ tests
+def test_tables_scale_and_mask_identical(codec_55, codec_literal):
+    freq, cdf = O.laplace_tables()
+    for cod in (codec_55, codec_literal):
+        gc = gpu_codec(cod)
+        g_cdf, g_scale, g_keep, exps = D.dckv_codec_export(gc.handle)
+        assert np.array_equal(g_cdf.astype(np.int64), cdf[:, :510].astype(np.int64))
+        s, keep = O.scale_index(cod.laplace_b, cod.delta)
+        assert np.array_equal(g_keep.astype(bool), keep)
+        assert np.array_equal(g_scale.astype(np.int64), s)
+        assert gc.k_eff == int(keep.sum())
+
+
+def test_parity_literal_small_config(src, codec_literal):
+    # one prompt of 256 tokens (124 coded rows) plus ragged neighbours and degenerate prompts
+    full_check(src, codec_literal, [256, 700, 50, 132, 133, 134], seeds=[0, 1, 2, 3, 4, 5])
+
+
+def test_parity_fitted_rate_several_tiles(src, codec_55):
+    r = full_check(src, codec_55, [132 + 600, 132 + 301], seeds=[7, 8])
+    assert r["flips"] <= 0.001 * 901 * 2048
+
+
+def test_parity_centres_escapes_and_big_codes(src, codec_centred):
+    # rows pushed far out: escapes beyond +-127 and codes beyond the fp16-exact 2048
+    full_check(src, codec_centred, [132 + 90, 132 + 41, 140], seeds=[11, 12, 13], chunk_rows=8,
+               boost=(4, 9, 30, 60, 223 + 4, 223 + 50), boost_gain=400.0, expect_escapes=True, expect_big=True)
+
+
+def test_parity_student_t_rows(src, codec_55):
+    full_check(src, codec_55, [132 + 256], seeds=[21], chunk_rows=16, student_t=0.25)
+
+
+def test_determinism(src, codec_55):
+    gc = gpu_codec(codec_55)
+    x, tok, offs = make_batch(src, codec_55, [132 + 500, 300], [31, 32])
+    a = encode_gpu(gc, x, tok, offs)
+    b = encode_gpu(gc, x, tok, offs)
+    assert a["blob"] == b["blob"]
+    k1, v1, _, _ = decode_gpu(gc, a["blob_dev"], a["size"], tok, offs)
+    k1, v1 = k1.clone(), v1.clone()
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        k2, v2 = gc.decode(a["blob_dev"], a["size"], tok, offs, stream=s)
+    s.synchronize()
+    assert torch.equal(k1, k2) and torch.equal(v1, v2)
+
+
+def test_corrupt_blobs_report_status(src, codec_55):
+    gc = gpu_codec(codec_55)
+    x, tok, offs = make_batch(src, codec_55, [132 + 200], [41])
+    res = encode_gpu(gc, x, tok, offs)
+    blob = res["blob_dev"]
+    hdr = O.parse_blob(res["blob"])
+    # 1: truncated blob
+    _, _, st, _ = decode_gpu(gc, blob, res["size"] - 10, tok, offs)
+    assert st == D.DCKV_ECORRUPT
+    # 2: wrong prompt length
+    _, _, st, _ = decode_gpu(gc, blob, res["size"], tok, np.array([0, 331]))
+    assert st in (D.DCKV_ECORRUPT,)
+    # 3: words of a chunk overwritten
+    bad = blob.clone()
+    p = hdr["off_streams"] + hdr["chunk_offsets"][0] + 140
+    bad[p: p + 64] = 0xA5
+    _, _, st, _ = decode_gpu(gc, bad, res["size"], tok, offs)
+    assert st == D.DCKV_ECORRUPT
+    # 4: escape count inflated
+    bad = blob.clone()
+    bad[hdr["off_streams"] + hdr["chunk_offsets"][1] + 128] = 200
+    _, _, st, _ = decode_gpu(gc, bad, res["size"], tok, offs)
+    assert st == D.DCKV_ECORRUPT
+    # a clean decode still works afterwards
+    _, _, st, _ = decode_gpu(gc, blob, res["size"], tok, offs)
+    assert st == D.DCKV_OK
+
+
+def test_capacity_error(src, codec_55):
+    gc = gpu_codec(codec_55)
+    x, tok, offs = make_batch(src, codec_55, [132 + 64], [51])
+    small = torch.empty(2 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+    gc.encode(x, tok, offs, blob=small)
+    torch.cuda.synchronize()
+    assert int(gc.status.item()) == D.DCKV_ECAPACITY
+    with pytest.raises(D.DckvError):
+        D.dckv_encode(gc.handle, x, tok, offs, small, gc.blob_size, gc.status,
+                      torch.empty(1024, dtype=torch.uint8, device="cuda"))
+
+
+def test_full_size_4k_prompt_sampled(src, codec_55):
+    """4,096-token prompt at about 220 B/token, in the configuration the benchmark times:
+    sampled rows against the oracle, every chunk's section re-coded by the oracle coder,
+    and the payload against the model code length."""
+    gc = gpu_codec(codec_55)
+    x, tok, offs = make_batch(src, codec_55, [4096], [100])
+    res = encode_gpu(gc, x, tok, offs)
+    assert res["status"] == D.DCKV_OK
+    n = 4096 - 132
+    rng = np.random.default_rng(0)
+    rows = np.sort(rng.choice(n, 48, replace=False))
+    xb = bits(x)
+    y = O.transform(xb[4 + rows], codec_55)
+    q_o, ratio = O.quantise(y, codec_55.delta, O.scale_index(codec_55.laplace_b, codec_55.delta)[1])
+    check_codes(res["q32"][rows].astype(np.int64), dict(q=q_o, ratio=ratio))
+    codes = split_gpu_codes(gc, codec_55, res, tok, offs)
+    # the whole blob from the GPU's codes and centres through the oracle coder
+    aux = {}
+    ora_blob = O.assemble_blob(xb, offs, codes, codec_55.laplace_b, codec_55.delta, 32, aux=aux)
+    assert ora_blob == res["blob"]
+    payload = res["size"] - 132 * 12288
+    model_bytes = aux["code_bits"] / 8
+    assert payload <= 1.05 * model_bytes, (payload, model_bytes)
+    assert 150 <= payload / n <= 300
+    k, v, st, q16 = decode_gpu(gc, res["blob_dev"], res["size"], tok, offs)
+    assert st == D.DCKV_OK
+    assert np.array_equal(q16, res["q32"].astype(np.float32))
+    # sampled decoded rows against the oracle's reconstruction of the same codes
+    xh = O.reconstruct(res["q32"][rows].astype(np.int64), codec_55)
+    want = O.f64_to_bf16(O.output_rows(xh, 4 + rows)).reshape(-1, 6, 2, 2, 256)
+    kg = bits(k)[:, 4 + rows].transpose(1, 0, 2, 3)
+    vg = bits(v)[:, 4 + rows].transpose(1, 0, 2, 3)
+    assert rel_frob(O.bf16_to_f64(kg), O.bf16_to_f64(want[:, :, 0])) <= ROW_TOL
+    assert rel_frob(O.bf16_to_f64(vg), O.bf16_to_f64(want[:, :, 1])) <= ROW_TOL
