@@ -60,8 +60,8 @@ class ClockSampler:
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={q}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
@@ -83,6 +83,9 @@ class ClockSampler:
         os.unlink(self.path)
         if not rows:
             return None
+        if self.index is not None:
+            mine = [r for r in rows if r[0] == str(self.index)]
+            rows = mine or rows
         sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
         mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
         reasons = set()
@@ -216,11 +219,14 @@ def run_gpu(args):
     # timed region: K steps, per-step events, L2 flushed between steps (outside the events)
     stage_ms = {}
     step_ms, enc_ms, dec_ms = [], [], []
-    sampler = ClockSampler(dev.index)
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    phys = vis.split(",")[dev.index] if vis and vis.split(",")[dev.index].strip().isdigit() else str(dev.index)
+    sampler = ClockSampler(phys)
+    sampler.start()
+    time.sleep(0.5)  # let the sampler produce its first lines before the timed region
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
-    sampler.start()
     wall0 = time.perf_counter()
     for it in range(args.steps):
         flush.fill_(it & 0xFF)
@@ -366,7 +372,7 @@ def run_gpu(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="dckv", choices=["dckv", "reference"])
     ap.add_argument("--config", default="c2", choices=sorted(CONFIGS))

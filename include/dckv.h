@@ -100,8 +100,10 @@ typedef struct {
  * s = clamp(round(8 log2(beta/0.05)), 0, 63)), the 64 integer Laplace tables (16-bit
  * precision, 509 residuals + ESC), the split fp16 operands of the transform, correction
  * and inverse GEMMs, and the per-vocabulary mean tables embed @ w_even and
- * embed @ w_odd[0:2048] (fp32).  chunk_rows (1..256, 0 = default 32) is the number of
- * same-parity rows per rANS chunk.  Allocates device memory (about
+ * embed @ w_odd[0:2048] (fp32).  chunk_rows (1..256) is the number of same-parity rows
+ * per rANS chunk; 0 selects 16; -1 selects the smallest count whose fixed per-chunk bytes
+ * (states, escape count, offset) stay within 3.5% of the tables' own entropy per row.
+ * Fewer rows per chunk give more independent streams (faster decode) and more bytes.  Allocates device memory (about
  * 2 * vocab * 8 KiB + 230 MiB).  Synchronises the device.  Returns DCKV_OK or an error;
  * *out is NULL on error. */
 int dckv_codec_create(const dckv_params *params, int device, int chunk_rows, dckv_codec **out);

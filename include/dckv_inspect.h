@@ -21,10 +21,18 @@ extern "C" {
  *   q32  int32 [n_rows][2048] codes q = round(y / Delta) (0 for dropped components),
  *        rows in prompt order, coded rows only (positions 4 .. N-129 of each prompt);
  *   qe   bf16 [ne_pad][2048] even-row codes, one extra zero row after each prompt;
- *   c_odd int8 [ne_pad][2048] centres of the odd row whose left neighbour is that row.
- * After dckv_decode: q16 fp16 [n_rows][2048] decoded codes (exact below 2048), qe, c_odd. */
+ *   cen8 int8 [n_rows][K_eff] centres in slot order: slot row row_slot[r] of coded row r
+ *        (chunk order: every even row of every prompt, then every odd row), kept
+ *        components in ascending order;
+ *   sym16 uint16 [n_rows][K_eff] symbols in the same order;
+ *   row_slot int32 [n_rows].
+ * After dckv_decode: q16 fp16 [n_rows][2048] decoded codes (exact below 2048), qe, cen8.
+ * Encode recomputes in fp64 every code whose fp32 ratio y / Delta lies in a guard band
+ * around a half-step boundary (whole rows when the row's norm is large). */
 typedef struct {
-  uint64_t q32, qe, c_odd, q16, x16, g16;
+  uint64_t q32, qe, cen8, row_slot, sym16, q16, x16, g16;
+  uint64_t counters; /* uint32[64]; encode: [0] codes recomputed exactly, [1] rows recomputed whole;
+                        decode: [0] rows holding codes beyond +-2047 */
   int64_t n_rows, ne_pad;
   int32_t n_chunks;
   uint64_t total;
@@ -42,6 +50,15 @@ int dckv_codec_export(const dckv_codec *codec, uint16_t *cdf, uint8_t *scale, ui
 /* Device pointers of the per-vocabulary mean tables (fp32 [vocab][2048]):
  * t_even = embed @ w_even, t_odd = embed @ w_odd[0:2048]. */
 int dckv_codec_tables(const dckv_codec *codec, const void **t_even, const void **t_odd);
+
+/* Chunk rows G in use (chosen at creation when 0 was passed) and the entropy of the kept
+ * components' tables in bits per coded row (the rate the codec's own model expects). */
+int dckv_codec_info(const dckv_codec *codec, int32_t *chunk_rows, double *model_bits_per_row);
+
+/* Self-test hook: when ratio_dev (device fp32 [n_rows][2048]) is not NULL, later encodes
+ * also write the fp32 transform ratios y / Delta there, before any exact recomputation.
+ * Pass NULL to stop.  The buffer must cover the largest call's coded rows. */
+int dckv_debug_ratio(dckv_codec *codec, void *ratio_dev);
 
 /* Per-stage device times of the last encode / decode issued with timing enabled.
  * Events are recorded on the call's stream; read after synchronising it.  Returns the

@@ -53,7 +53,7 @@ class ByteReport(ctypes.Structure):
 
 
 class WsView(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_uint64) for n in ("q32", "qe", "c_odd", "q16", "x16", "g16")] + [
+    _fields_ = [(n, ctypes.c_uint64) for n in ("q32", "qe", "cen8", "row_slot", "sym16", "q16", "x16", "g16", "counters")] + [
         ("n_rows", ctypes.c_int64), ("ne_pad", ctypes.c_int64), ("n_chunks", ctypes.c_int32),
         ("total", ctypes.c_uint64)]
 
@@ -83,6 +83,8 @@ def lib():
         "dckv_set_timing": (I, [P, I]),
         "dckv_get_timing": (I, [P, P, P, I]),
         "dckv_debug_gemm": (I, [I, P, I, P, I, I, I, P, I, P]),
+        "dckv_debug_ratio": (I, [P, P]),
+        "dckv_codec_info": (I, [P, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -203,6 +205,17 @@ def dckv_codec_tables(handle):
     te, to = ctypes.c_void_p(), ctypes.c_void_p()
     _check(lib().dckv_codec_tables(handle, ctypes.byref(te), ctypes.byref(to)), "dckv_codec_tables")
     return te.value, to.value
+
+
+def dckv_debug_ratio(handle, ratio_dev):
+    _check(lib().dckv_debug_ratio(handle, None if ratio_dev is None else ratio_dev.data_ptr()), "dckv_debug_ratio")
+
+
+def dckv_codec_info(handle):
+    g = ctypes.c_int32()
+    bits = ctypes.c_double()
+    _check(lib().dckv_codec_info(handle, ctypes.byref(g), ctypes.byref(bits)), "dckv_codec_info")
+    return {"chunk_rows": int(g.value), "model_bits_per_row": float(bits.value)}
 
 
 def dckv_set_timing(handle, enable: bool):

@@ -128,13 +128,13 @@ template <class Epi, int STAGES, int MAX_SLABS, int CHUNK_STEPS>
 static int run_gemm_chunked(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &b0,
                             const CUtensorMap &b1, const GemmProblem &prob, const typename Epi::Params &ep,
                             int num_sms, cudaStream_t st) {
-  constexpr int smem = gemm_chunked_smem_bytes<STAGES, MAX_SLABS>();
+  constexpr int smem = gemm_chunked_smem_bytes<Epi, STAGES, MAX_SLABS>();
   static_assert(smem <= 232448, "GEMM shared memory above the sm_100 limit");
   auto kern = gemm_chunked_kernel<Epi, STAGES, MAX_SLABS, CHUNK_STEPS>;
   CK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   const int tiles = prob.m_tiles * prob.n_tiles;
   if (tiles <= 0) return DCKV_OK;
-  if (prob.bn != GEMM_MAX_BN) return fail(DCKV_EINVAL, "chunked GEMM needs bn = 256");
+  if (prob.bn != GEMMC_BN) return fail(DCKV_EINVAL, "chunked GEMM tile width mismatch");
   for (int i = 0; i < prob.n_seg; ++i)
     if (prob.seg[i].n_slab < 1 || prob.seg[i].n_slab > MAX_SLABS) return fail(DCKV_EINVAL, "bad slab count");
   const int grid = std::min(tiles, num_sms);
@@ -299,16 +299,20 @@ __global__ void k_permute_mu(const float *mu, float *mu_perm) {
 // ============================================================================ per-call kernels
 // Row tables of one prompt per block: coded row r = row_base + i holds position 4 + i.
 __global__ void k_layout(const PromptInfo *prompts, int32_t *row_tok, int32_t *row_pos, int32_t *row_edst,
-                         int32_t *e_tok, __nv_bfloat16 *qe_zero_pad) {
+                         int32_t *row_slot, int32_t *e_tok, int32_t *e_slot, __nv_bfloat16 *qe_zero_pad) {
   const PromptInfo pi = prompts[blockIdx.x];
   for (int i = threadIdx.x; i < pi.n; i += blockDim.x) {
     const int r = pi.row_base + i;
     row_tok[r] = (int32_t)(pi.tok_base + HEAD_KEPT + i);
     row_pos[r] = HEAD_KEPT + i;
     row_edst[r] = (i & 1) ? -1 : pi.ebase + (i >> 1);
+    row_slot[r] = (i & 1) ? pi.slot_o0 + (i >> 1) : pi.slot_e0 + (i >> 1);
   }
-  for (int e = threadIdx.x; e <= pi.n_e; e += blockDim.x)
-    e_tok[pi.ebase + e] = e < pi.n_o ? (int32_t)(pi.tok_base + HEAD_KEPT + 2 * e + 1) : -1;
+  for (int e = threadIdx.x; e <= pi.n_e; e += blockDim.x) {
+    const bool odd = e < pi.n_o;
+    e_tok[pi.ebase + e] = odd ? (int32_t)(pi.tok_base + HEAD_KEPT + 2 * e + 1) : -1;
+    e_slot[pi.ebase + e] = odd ? pi.slot_o0 + e : 0;
+  }
   if (qe_zero_pad)  // the row after a prompt's last even row is its odd rows' zero right neighbour
     for (int k = threadIdx.x; k < N_COEF; k += blockDim.x)
       qe_zero_pad[(int64_t)(pi.ebase + pi.n_e) * N_COEF + k] = __float2bfloat16_rn(0.f);
@@ -327,7 +331,8 @@ __device__ __forceinline__ int find_prompt(const PromptInfo *p, int batch, int64
 // DCKV_ERANGE), kept rows -> the blob's kept section verbatim.
 __global__ void __launch_bounds__(192) k_convert(const __nv_bfloat16 *rows, const PromptInfo *prompts, int batch,
                                                  __half *x16, uint8_t *blob, uint64_t blob_cap, uint64_t off_kept,
-                                                 int32_t *status) {
+                                                 float *row_norm, int32_t *status) {
+  __shared__ float red[6];
   const int64_t t = blockIdx.x;
   const int b = find_prompt(prompts, batch, t);
   const PromptInfo pi = prompts[b];
@@ -337,6 +342,7 @@ __global__ void __launch_bounds__(192) k_convert(const __nv_bfloat16 *rows, cons
   if (coded) {
     uint4 *dst = reinterpret_cast<uint4 *>(x16 + (int64_t)(pi.row_base + p - HEAD_KEPT) * ROW_DIM);
     bool clamped = false;
+    float ss = 0.f;
     for (int v = threadIdx.x; v < ROW_DIM / 8; v += blockDim.x) {
       uint4 in = src[v];
       const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&in);
@@ -345,6 +351,7 @@ __global__ void __launch_bounds__(192) k_convert(const __nv_bfloat16 *rows, cons
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         float2 f = __bfloat1622float2(h[q]);
+        ss = fmaf(f.x, f.x, fmaf(f.y, f.y, ss));
         const float lim = 65504.f;
         if (!(fabsf(f.x) <= lim) || !(fabsf(f.y) <= lim)) clamped = true;
         f.x = fminf(fmaxf(f.x, -lim), lim);
@@ -354,6 +361,14 @@ __global__ void __launch_bounds__(192) k_convert(const __nv_bfloat16 *rows, cons
       dst[v] = o;
     }
     if (clamped) atomicExch(status, DCKV_ERANGE);
+    for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float t = 0.f;
+      for (int w = 0; w < 6; ++w) t += red[w];
+      row_norm[pi.row_base + p - HEAD_KEPT] = isfinite(t) ? sqrtf(t) : 3.0e38f;
+    }
   } else {
     const int kidx = (pi.n == 0 || p < HEAD_KEPT) ? p : HEAD_KEPT + (p - (pi.N - TAIL_KEPT));
     const uint64_t off = off_kept + (uint64_t)(pi.kept_base + kidx) * (ROW_DIM * 2);
@@ -501,6 +516,101 @@ __global__ void __launch_bounds__(256) k_fixup(const int32_t *biglist, const uin
   }
 }
 
+// out[o][k] = src[k * O + o] (fp32 transpose of a row-major [K][O] matrix)
+__global__ void k_transpose32(const float *src, int K, int O, float *out) {
+  __shared__ float tile[32][33];
+  const int k0 = blockIdx.x * 32, o0 = blockIdx.y * 32;
+  const int tx = threadIdx.x, ty = threadIdx.y;
+  for (int y = ty; y < 32; y += 8) {
+    const int k = k0 + y, o = o0 + tx;
+    tile[y][tx] = (k < K && o < O) ? src[(int64_t)k * O + o] : 0.f;
+  }
+  __syncthreads();
+  for (int y = ty; y < 32; y += 8) {
+    const int o = o0 + y, k = k0 + tx;
+    if (o < O && k < K) out[(int64_t)o * K + k] = tile[tx][y];
+  }
+}
+
+__device__ __forceinline__ double warp_sum(double v) {
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ void store_code(int64_t row, int c, double ratio, int32_t *q32, __nv_bfloat16 *qe,
+                                           const int32_t *row_edst) {
+  const double qd = fmin(fmax(rint(ratio), -2147483648.0), 2147483647.0);
+  const int q = (int)qd;
+  q32[row * N_COEF + c] = q;
+  const int e = row_edst[row];
+  if (e >= 0) qe[(int64_t)e * N_COEF + c] = __float2bfloat16_rn((float)q);
+}
+
+// Exact recomputation of listed codes near a half-step boundary, one warp per code:
+// y = (x - mu) . basis[:, c] + g . w2[:, c] in fp64 (x from the caller's bf16 rows, g the
+// correction's hidden units from the chunk-accumulated GEMM), q = round(y / Delta_c).
+__global__ void __launch_bounds__(256) k_refine_codes(const uint32_t *el_list, const uint32_t *counters,
+                                                      int64_t el_cap, const __nv_bfloat16 *rows,
+                                                      const int32_t *row_tok, const float *mu32, const float *bt32,
+                                                      const float *w2t32, const __half *g16, const float *delta,
+                                                      const uint32_t *rowflag, int32_t *q32, __nv_bfloat16 *qe,
+                                                      const int32_t *row_edst) {
+  const int lane = threadIdx.x & 31;
+  const int64_t n = min((int64_t)counters[0], el_cap);
+  const int64_t wpb = blockDim.x >> 5;
+  for (int64_t idx = blockIdx.x * wpb + (threadIdx.x >> 5); idx < n; idx += gridDim.x * wpb) {
+    const uint32_t code = el_list[idx];
+    const int64_t row = code >> 11;
+    const int c = (int)(code & 2047u);
+    if (rowflag[row]) continue;  // recomputed whole by k_refine_rows
+    const __nv_bfloat16 *xr = rows + (int64_t)row_tok[row] * ROW_DIM;
+    const float *bt = bt32 + (int64_t)c * ROW_DIM;
+    double acc = 0.0;
+    for (int i = lane; i < ROW_DIM; i += 32) acc += ((double)__bfloat162float(xr[i]) - (double)mu32[i]) * (double)bt[i];
+    const __half *g = g16 + row * (2 * N_HIDDEN);
+    for (int h = lane; h < N_HIDDEN; h += 32)
+      acc += ((double)__half2float(g[h]) + (double)__half2float(g[N_HIDDEN + h])) * (double)w2t32[c * N_HIDDEN + h];
+    acc = warp_sum(acc);
+    if (lane == 0) store_code(row, c, acc / (double)delta[c], q32, qe, row_edst);
+  }
+}
+
+// Whole-row exact recomputation (rows with a large norm), one block per listed row:
+// h = (x - mu) w1, g = GELU(h) (erf), y = (x - mu) basis + g w2, all in fp64.
+__global__ void __launch_bounds__(256) k_refine_rows(const uint32_t *full_list, const uint32_t *counters,
+                                                     const __nv_bfloat16 *rows, const int32_t *row_tok,
+                                                     const float *mu32, const float *bt32, const float *w1t32,
+                                                     const float *w2t32, const float *delta, const uint8_t *keep,
+                                                     int32_t *q32, __nv_bfloat16 *qe, const int32_t *row_edst) {
+  extern __shared__ __align__(16) double xc[];  // [6144] then g[256]
+  double *gs = xc + ROW_DIM;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const uint32_t n = counters[1];
+  for (uint32_t li = blockIdx.x; li < n; li += gridDim.x) {
+    const int64_t row = full_list[li];
+    const __nv_bfloat16 *xr = rows + (int64_t)row_tok[row] * ROW_DIM;
+    for (int i = threadIdx.x; i < ROW_DIM; i += blockDim.x) xc[i] = (double)__bfloat162float(xr[i]) - (double)mu32[i];
+    __syncthreads();
+    for (int h = warp; h < N_HIDDEN; h += nw) {
+      const float *w = w1t32 + (int64_t)h * ROW_DIM;
+      double acc = 0.0;
+      for (int i = lane; i < ROW_DIM; i += 32) acc += xc[i] * (double)w[i];
+      acc = warp_sum(acc);
+      if (lane == 0) gs[h] = 0.5 * acc * (1.0 + erf(acc * 0.70710678118654752440));
+    }
+    __syncthreads();
+    for (int c = warp; c < N_COEF; c += nw) {
+      const float *bt = bt32 + (int64_t)c * ROW_DIM;
+      double acc = 0.0;
+      for (int i = lane; i < ROW_DIM; i += 32) acc += xc[i] * (double)bt[i];
+      for (int h = lane; h < N_HIDDEN; h += 32) acc += gs[h] * (double)w2t32[c * N_HIDDEN + h];
+      acc = warp_sum(acc);
+      if (lane == 0) store_code(row, c, keep[c] ? acc / (double)delta[c] : 0.0, q32, qe, row_edst);
+    }
+    __syncthreads();
+  }
+}
+
 // ============================================================================ host layout
 static inline uint64_t align_up(uint64_t v, uint64_t a) { return (v + a - 1) / a * a; }
 
@@ -533,9 +643,16 @@ static int build_layout(const dckv_codec *c, const int64_t *offs, int batch, Lay
     ne += p.n_e + 1;
     kept += p.n_kept;
   }
+  int64_t se = 0, so = 0;
   for (int b = 0; b < batch; ++b) {
     L.prompts[b].chunk_o0 = ce + co;
     co += (L.prompts[b].n_o + G - 1) / G;
+    L.prompts[b].slot_e0 = (int32_t)se;
+    se += L.prompts[b].n_e;
+  }
+  for (int b = 0; b < batch; ++b) {
+    L.prompts[b].slot_o0 = (int32_t)(se + so);
+    so += L.prompts[b].n_o;
   }
   L.n_tokens = offs[batch];
   if (L.n_tokens >= ((int64_t)1 << 31)) return fail(DCKV_EINVAL, "too many tokens");
@@ -584,18 +701,26 @@ static WsPlan plan_ws(const Layout &L, int which /*0 encode, 1 decode*/) {
   w.row_pos = take(4ull * L.n_rows);
   w.row_edst = take(4ull * L.n_rows);
   w.e_tok = take(4ull * L.ne_pad);
+  w.row_slot = take(4ull * L.n_rows);
+  w.e_slot = take(4ull * L.ne_pad);
   w.qe = take(2ull * L.ne_pad * N_COEF);
-  w.c_odd = take(1ull * L.ne_pad * N_COEF);
+  w.cen8 = take(1ull * L.n_symbols);
   w.counters = take(256);
   if (which == 0) {
     w.x16 = take(2ull * L.n_rows * ROW_DIM);
     w.g16 = take(2ull * L.n_rows * 2 * N_HIDDEN);
     w.q32 = take(4ull * L.n_rows * N_COEF);
+    w.sym16 = take(2ull * L.n_symbols);
     w.words = take(2ull * L.n_symbols);
     w.states = take(128ull * L.n_chunks);
     w.nwords = take(4ull * L.n_chunks);
     w.nesc = take(4ull * L.n_chunks);
     w.offs = take(4ull * (L.n_chunks + 1));
+    w.row_norm = take(4ull * L.n_rows);
+    w.rowflag = take(4ull * L.n_rows);
+    w.el_cap = 64 * L.n_rows + 4096;
+    w.el_list = take(4ull * w.el_cap);
+    w.full_list = take(4ull * L.n_rows);
   } else {
     w.q16 = take(2ull * L.n_rows * N_COEF);
     w.qbig = take(4ull * L.n_rows * N_COEF);
@@ -621,10 +746,10 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
       !prm->w_even || !prm->w_odd)
     return fail(DCKV_EINVAL, "a parameter pointer is NULL");
   if (prm->vocab < 1 || prm->vocab > (1 << 20)) return fail(DCKV_EINVAL, "vocab out of range");
-  if (chunk_rows == 0) chunk_rows = 32;
-  if (chunk_rows < 1 || chunk_rows > 256) return fail(DCKV_EINVAL, "chunk_rows out of range");
+  if (chunk_rows < -1 || chunk_rows > 256) return fail(DCKV_EINVAL, "chunk_rows out of range");
   if (((uintptr_t)prm->embed | (uintptr_t)prm->w_even | (uintptr_t)prm->w_odd) & 15)
     return fail(DCKV_EINVAL, "bf16 parameters must be 16-byte aligned");
+  static_assert(RANS_DEC_SMEM <= 232448, "decoder tables exceed shared memory");
   CK(cudaSetDevice(device));
   cudaDeviceProp prop;
   CK(cudaGetDeviceProperties(&prop, device));
@@ -668,7 +793,13 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
   const uint64_t o_kl = take(2ull * N_COEF);
   const uint64_t o_ks = take(N_COEF);
   const uint64_t o_cdf = take(2ull * N_SCALES * N_SYM);
+  const uint64_t o_lut = take(2ull * N_SCALES * LUT_SIZE);
+  const uint64_t o_kidx = take(2ull * N_COEF);
   const uint64_t o_theta = take(8ull * 128);
+  const uint64_t o_bt32 = take(4ull * N_COEF * ROW_DIM);
+  const uint64_t o_w1t32 = take(4ull * N_HIDDEN * ROW_DIM);
+  const uint64_t o_w2t32 = take(4ull * N_COEF * N_HIDDEN);
+  const uint64_t o_mu32 = take(4ull * ROW_DIM);
   const uint64_t o_tmp = take(2ull * 2 * N_COEF * N_COEF);  // W_e^T and W_oE^T (setup only)
   const uint64_t o_scr = take(64);
   if (cudaMalloc(&c->blk, o) != cudaSuccess) return cleanup(fail(DCKV_ECUDA, "cudaMalloc(%llu) failed", (unsigned long long)o));
@@ -689,7 +820,13 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
   c->kept_list = (int16_t *)(B + o_kl);
   c->kept_scale = B + o_ks;
   c->cdf = (uint16_t *)(B + o_cdf);
+  c->lut = (uint16_t *)(B + o_lut);
+  c->kidx = (int16_t *)(B + o_kidx);
   c->theta = (double *)(B + o_theta);
+  c->bt32 = (float *)(B + o_bt32);
+  c->w1t32 = (float *)(B + o_w1t32);
+  c->w2t32 = (float *)(B + o_w2t32);
+  c->mu32 = (float *)(B + o_mu32);
   uint16_t *tmp_e = (uint16_t *)(B + o_tmp);
   uint16_t *tmp_oe = tmp_e + (size_t)N_COEF * N_COEF;
   int32_t *scr = (int32_t *)(B + o_scr);
@@ -699,6 +836,7 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
   // drop mask, scale index, tables
   k_scale_keep<<<(N_COEF + 255) / 256, 256, 0, st>>>(prm->laplace_b, prm->delta, c->scale, c->keep, scr);
   k_tables<<<N_SCALES, 512, 0, st>>>(c->cdf);
+  k_build_lut<<<N_SCALES, 256, 0, st>>>(c->cdf, c->lut);
   cudaMemcpyAsync(c->delta, prm->delta, 4ull * N_COEF, cudaMemcpyDeviceToDevice, st);
   // scale exponents: largest |value| of each split operand brought to about 2^12
   k_absmax<<<256, 256, 0, st>>>(prm->basis, (int64_t)ROW_DIM * N_COEF, N_COEF, nullptr, scr + 1);
@@ -737,12 +875,41 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
       ks.push_back(scale_h[i]);
     }
   c->k_eff = (int)kl.size();
+  std::vector<int16_t> kx(N_COEF, -1);
+  for (int i = 0; i < c->k_eff; ++i) kx[kl[i]] = (int16_t)i;
   kl.resize(N_COEF, 0);
   ks.resize(N_COEF, 0);
+  // entropy of the kept components' tables (bits per coded row): the chunk size is the
+  // smallest one whose fixed cost (states, escape count, offset, pad: ~137 B) stays
+  // within 3.5% of it, unless the caller fixed it
+  {
+    std::vector<uint16_t> cdf_h((size_t)N_SCALES * N_SYM);
+    if (cudaMemcpy(cdf_h.data(), c->cdf, 2ull * N_SCALES * N_SYM, cudaMemcpyDeviceToHost) != cudaSuccess)
+      return cleanup(fail(DCKV_ECUDA, "table readback failed"));
+    double hs[N_SCALES];
+    for (int s = 0; s < N_SCALES; ++s) {
+      double h = 0.0;
+      for (int k = 0; k < N_SYM; ++k) {
+        const double f = (double)((k + 1 < N_SYM ? cdf_h[s * N_SYM + k + 1] : PREC_TOTAL) - cdf_h[s * N_SYM + k]);
+        if (f > 0) h -= f / PREC_TOTAL * std::log2(f / PREC_TOTAL);
+      }
+      hs[s] = h;
+    }
+    double bits = 0.0;
+    for (int i = 0; i < c->k_eff; ++i) bits += hs[ks[i]];
+    c->model_bits_per_row = bits;
+    if (c->chunk_rows == 0) c->chunk_rows = 16;
+    if (c->chunk_rows < 0) {
+      const double per_row = 0.035 * bits / 8.0;
+      int g = per_row > 0 ? (int)std::ceil((CHUNK_FIXED_BYTES + 5) / per_row) : 256;
+      c->chunk_rows = std::min(256, std::max(8, g));
+    }
+  }
   double theta_h[128];
   for (int i = 0; i < 128; ++i) theta_h[i] = std::pow(ROPE_BASE, -2.0 * i / HEAD_DIM);
   if (cudaMemcpy(c->kept_list, kl.data(), 2 * N_COEF, cudaMemcpyHostToDevice) != cudaSuccess ||
       cudaMemcpy(c->kept_scale, ks.data(), N_COEF, cudaMemcpyHostToDevice) != cudaSuccess ||
+      cudaMemcpy(c->kidx, kx.data(), 2 * N_COEF, cudaMemcpyHostToDevice) != cudaSuccess ||
       cudaMemcpy(c->theta, theta_h, sizeof(theta_h), cudaMemcpyHostToDevice) != cudaSuccess)
     return cleanup(fail(DCKV_ECUDA, "setup upload failed"));
   // mean projections in fp64
@@ -755,6 +922,11 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
   k_split<<<dim3(N_HIDDEN / 32, N_COEF / 32), tb, 0, st>>>(prm->w2, N_COEF, N_HIDDEN, 0, nullptr, std::ldexp(1.0, c->p_y), c->a_w2);
   k_split<<<dim3(ROW_DIM / 32, N_HIDDEN / 32), tb, 0, st>>>(prm->w1, N_HIDDEN, ROW_DIM, 0, nullptr, std::ldexp(1.0, c->p_h), c->a_h);
   k_split<<<dim3(N_COEF / 32, ROW_DIM / 32), tb, 0, st>>>(prm->basis, ROW_DIM, N_COEF, 1, prm->delta, std::ldexp(1.0, c->p_inv), c->a_inv);
+  // fp32 copies for the exact refinement
+  k_transpose32<<<dim3(ROW_DIM / 32, N_COEF / 32), tb, 0, st>>>(prm->basis, ROW_DIM, N_COEF, c->bt32);
+  k_transpose32<<<dim3(ROW_DIM / 32, N_HIDDEN / 32), tb, 0, st>>>(prm->w1, ROW_DIM, N_HIDDEN, c->w1t32);
+  k_transpose32<<<dim3(N_HIDDEN / 32, N_COEF / 32), tb, 0, st>>>(prm->w2, N_HIDDEN, N_COEF, c->w2t32);
+  cudaMemcpyAsync(c->mu32, prm->mu, 4ull * ROW_DIM, cudaMemcpyDeviceToDevice, st);
   // mean-model weights, K-major
   k_transpose16<<<dim3(2 * N_COEF / 32, N_COEF / 32), tb, 0, st>>>(prm->w_odd, N_COEF, N_COEF, N_COEF, 2 * N_COEF,
                                                                    (uint16_t *)c->a_on);
@@ -852,59 +1024,86 @@ extern "C" int dckv_encode(const dckv_codec *c, const void *rows, const int32_t 
   __half *g16 = (__half *)(ws + w.g16);
   int32_t *q32 = (int32_t *)(ws + w.q32);
   __nv_bfloat16 *qe = (__nv_bfloat16 *)(ws + w.qe);
-  int8_t *c_odd = (int8_t *)(ws + w.c_odd);
+  int32_t *row_slot = (int32_t *)(ws + w.row_slot), *e_slot = (int32_t *)(ws + w.e_slot);
+  int8_t *cen8 = (int8_t *)(ws + w.cen8);
+  uint16_t *sym16 = (uint16_t *)(ws + w.sym16);
+
+  float *row_norm = (float *)(ws + w.row_norm);
+  uint32_t *rowflag = (uint32_t *)(ws + w.rowflag);
+  uint32_t *el_list = (uint32_t *)(ws + w.el_list), *full_list = (uint32_t *)(ws + w.full_list);
+  uint32_t *counters = (uint32_t *)(ws + w.counters);  // [0] codes to refine, [1] rows to refine
 
   stage_mark(c, st, "start");
   CK(cudaMemsetAsync(status_dev, 0, 4, st));
+  CK(cudaMemsetAsync(counters, 0, 256, st));
+  if (L.n_rows) CK(cudaMemsetAsync(rowflag, 0, 4ull * L.n_rows, st));
   RET(upload_tables(L, ws, w, st));
-  k_layout<<<L.batch, 256, 0, st>>>(d_prompts, row_tok, row_pos, row_edst, e_tok, qe);
+  k_layout<<<L.batch, 256, 0, st>>>(d_prompts, row_tok, row_pos, row_edst, row_slot, e_tok, e_slot, qe);
   if (L.n_tokens > 0)
     k_convert<<<(unsigned)L.n_tokens, 192, 0, st>>>((const __nv_bfloat16 *)rows, d_prompts, L.batch, x16, bl, blob_cap,
-                                                    L.off_kept, status_dev);
+                                                    L.off_kept, row_norm, status_dev);
   CK(cudaGetLastError());
   stage_mark(c, st, "layout+convert");
   if (L.n_rows > 0) {
-    CUtensorMap mb_x128, mb_x256, mb_g, mb_qe;
+    CUtensorMap mb_x128, mb_g128, mb_qe;
     RET(map_b(&mb_x128, x16, false, ROW_DIM, L.n_rows, 128));
-    RET(map_b(&mb_x256, x16, false, ROW_DIM, L.n_rows, 256));
-    RET(map_b(&mb_g, g16, false, 2 * N_HIDDEN, L.n_rows, 256));
+    RET(map_b(&mb_g128, g16, false, 2 * N_HIDDEN, L.n_rows, 128));
     RET(map_b(&mb_qe, qe, true, N_COEF, L.ne_pad, 256));
     // correction hidden layer: h = x @ w1 - mu @ w1, GELU, fp16 hi/lo
     {
       GemmProblem pr = make_problem(N_HIDDEN / GEMM_BM, L.n_rows, 128, false, status_dev);
       add_seg(pr, 0, 0, 2, 0, 0, 0, 0, ROW_DIM / GEMM_BK);
       EpiGelu::Params ep{c->muw1, (float)std::ldexp(1.0, -c->p_h), g16};
-      RET((run_gemm<EpiGelu, 3, 2>(c->map_ah2, c->map_ah2, mb_x128, mb_x128, pr, ep, c->num_sms, st)));
+      RET((run_gemm_chunked<EpiGeluTotals, 4, 2, 4>(c->map_ah2, c->map_ah2, mb_x128, mb_x128, pr, ep,
+                                                          c->num_sms, st)));
     }
     stage_mark(c, st, "gemm_hidden");
     // transform + quantiser: y = x @ B + g @ w2 - mu @ B
     {
-      GemmProblem pr = make_problem(N_COEF / GEMM_BM, L.n_rows, 256, false, status_dev);
+      GemmProblem pr = make_problem(N_COEF / GEMM_BM, L.n_rows, GEMMC_BN, false, status_dev);
       add_seg(pr, 0, 0, 2, 0, 0, 0, 0, ROW_DIM / GEMM_BK);
       add_seg(pr, 1, 0, 2, 0, 1, 0, 0, N_HIDDEN / GEMM_BK);
       add_seg(pr, 1, 0, 2, 0, 1, 0, N_HIDDEN, N_HIDDEN / GEMM_BK);
-      EpiQuant::Params ep{c->mub, c->delta, c->keep, (float)std::ldexp(1.0, -c->p_y), q32, qe, row_edst};
-      RET((run_gemm_chunked<EpiQuantTotals, 3, 2, 2>(c->map_ay2, c->map_aw2_2, mb_x256, mb_g, pr, ep, c->num_sms,
-                                                      st)));
+      EpiQuantTotals::Params ep{{c->mub, c->delta, c->keep, (float)std::ldexp(1.0, -c->p_y), q32, qe, row_edst},
+                                row_norm, rowflag, el_list, full_list, counters, w.el_cap, c->dbg_ratio};
+      RET((run_gemm_chunked<EpiQuantTotals, 4, 2, 4>(c->map_ay2, c->map_aw2_2, mb_x128, mb_g128, pr, ep,
+                                                      c->num_sms, st)));
     }
     stage_mark(c, st, "gemm_transform");
+    // codes whose fp32 ratio lies in the guard band around a half step: exact fp64 values
+    k_refine_codes<<<c->num_sms * 4, 256, 0, st>>>(el_list, counters, w.el_cap, (const __nv_bfloat16 *)rows, row_tok,
+                                                  c->mu32, c->bt32, c->w2t32, g16, c->delta, rowflag, q32, qe,
+                                                  row_edst);
+    const int rsmem = (ROW_DIM + N_HIDDEN) * 8;
+    CK(cudaFuncSetAttribute(k_refine_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, rsmem));
+    k_refine_rows<<<c->num_sms, 256, rsmem, st>>>(full_list, counters, (const __nv_bfloat16 *)rows, row_tok, c->mu32,
+                                                  c->bt32, c->w1t32, c->w2t32, c->delta, c->keep, q32, qe, row_edst);
+    CK(cudaGetLastError());
+    stage_mark(c, st, "refine");
     // odd mean model: [e, bf16(q_left), bf16(q_right)] @ w_odd -> centres
     {
       GemmProblem pr = make_problem(N_COEF / GEMM_BM, L.ne_pad, 256, true, status_dev);
       add_seg(pr, 0, 0, 1, 0, 0, 0, 0, N_COEF / GEMM_BK);
       add_seg(pr, 0, 0, 1, N_COEF, 0, 1, 0, N_COEF / GEMM_BK);
-      EpiMeanOdd::Params ep{c->t_odd, token_ids, e_tok, c_odd, c->vocab};
+      EpiMeanOdd::Params ep{c->t_odd, token_ids, e_tok, e_slot, c->kidx, cen8, c->k_eff, c->vocab};
       RET((run_gemm<EpiMeanOdd, 4, 1>(c->map_aon1, c->map_aon1, mb_qe, mb_qe, pr, ep, c->num_sms, st)));
     }
     stage_mark(c, st, "gemm_mean_odd");
+    // even centres from the vocabulary table, then every symbol, in slot order
+    const unsigned rg = (unsigned)std::min<int64_t>(L.n_rows, 65535);
+    k_centres_even<<<rg, 256, 0, st>>>(L.n_rows, row_slot, row_edst, row_tok, token_ids, c->t_even, c->vocab,
+                                       c->kept_list, c->k_eff, cen8, nullptr);
+    k_symbols<<<rg, 256, 0, st>>>(L.n_rows, row_slot, q32, cen8, c->kept_list, c->k_eff, sym16);
+    CK(cudaGetLastError());
+    stage_mark(c, st, "symbols");
   }
   uint32_t *states = (uint32_t *)(ws + w.states), *nwords = (uint32_t *)(ws + w.nwords);
   uint32_t *nesc = (uint32_t *)(ws + w.nesc), *offs = (uint32_t *)(ws + w.offs);
   if (L.n_chunks > 0) {
-    RansEncArgs a{d_chunks, d_prompts, L.n_chunks, c->k_eff, c->kept_list, c->kept_scale, c->cdf, q32,
-                  c->t_even, token_ids, c_odd, c->vocab, (uint16_t *)(ws + w.words), states, nwords, nesc};
-    CK(cudaFuncSetAttribute(rans_encode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, CDF_SMEM_BYTES));
-    rans_encode_kernel<<<(L.n_chunks + RANS_WARPS - 1) / RANS_WARPS, RANS_WARPS * 32, CDF_SMEM_BYTES, st>>>(a);
+    RansEncArgs a{d_chunks, L.n_chunks, c->k_eff, c->kept_scale, c->cdf, sym16, (uint16_t *)(ws + w.words),
+                  states, nwords, nesc};
+    CK(cudaFuncSetAttribute(rans_encode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, RANS_ENC_SMEM));
+    rans_encode_kernel<<<(L.n_chunks + RANS_WARPS - 1) / RANS_WARPS, RANS_WARPS * 32, RANS_ENC_SMEM, st>>>(a);
     CK(cudaGetLastError());
   }
   stage_mark(c, st, "rans_encode");
@@ -915,8 +1114,8 @@ extern "C" int dckv_encode(const dckv_codec *c, const void *rows, const int32_t 
     CK(cudaGetLastError());
   }
   if (L.n_chunks > 0) {
-    CompactArgs a{d_chunks, d_prompts, L.n_chunks, c->k_eff, c->kept_list, q32, (const uint16_t *)(ws + w.words),
-                  states, nwords, nesc, offs, bl, blob_cap, L.off_streams};
+    CompactArgs a{d_chunks, d_prompts, L.n_chunks, c->k_eff, c->kept_list, q32, sym16,
+                  (const uint16_t *)(ws + w.words), states, nwords, nesc, offs, bl, blob_cap, L.off_streams};
     compact_kernel<<<(L.n_chunks + RANS_WARPS - 1) / RANS_WARPS, RANS_WARPS * 32, 0, st>>>(a);
     CK(cudaGetLastError());
   }
@@ -947,7 +1146,8 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
   int32_t *row_tok = (int32_t *)(ws + w.row_tok), *row_pos = (int32_t *)(ws + w.row_pos);
   int32_t *row_edst = (int32_t *)(ws + w.row_edst), *e_tok = (int32_t *)(ws + w.e_tok);
   __nv_bfloat16 *qe = (__nv_bfloat16 *)(ws + w.qe);
-  int8_t *c_odd = (int8_t *)(ws + w.c_odd);
+  int32_t *row_slot = (int32_t *)(ws + w.row_slot), *e_slot = (int32_t *)(ws + w.e_slot);
+  int8_t *cen8 = (int8_t *)(ws + w.cen8);
   __half *q16 = (__half *)(ws + w.q16);
   int32_t *qbig = (int32_t *)(ws + w.qbig);
   uint32_t *bigflag = (uint32_t *)(ws + w.bigflag);
@@ -964,19 +1164,21 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
     CK(cudaMemsetAsync(q16, 0, 2ull * L.n_rows * N_COEF, st));
     CK(cudaMemsetAsync(bigflag, 0, 4ull * L.n_rows, st));
   }
-  k_layout<<<L.batch, 256, 0, st>>>(d_prompts, row_tok, row_pos, row_edst, e_tok, nullptr);
+  k_layout<<<L.batch, 256, 0, st>>>(d_prompts, row_tok, row_pos, row_edst, row_slot, e_tok, e_slot, nullptr);
   HeaderCheck hc{bl, blob_bytes, d_prompts, L.batch, c->chunk_rows, c->k_eff, L.n_chunks_e, L.n_chunks_o,
                  L.n_kept, L.off_kept, L.off_streams, valid, status_dev};
   k_check_header<<<1, 256, 0, st>>>(hc);
   CK(cudaGetLastError());
   stage_mark(c, st, "layout+check");
   const uint32_t *offs = (const uint32_t *)(bl + HEADER_BYTES + 4ull * L.batch);
-  CK(cudaFuncSetAttribute(rans_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, CDF_SMEM_BYTES));
-  RansDecArgs da{d_chunks, d_prompts, 0, L.n_chunks_e, c->k_eff, c->kept_list, c->kept_scale, c->cdf, c->t_even,
-                 token_ids, c_odd, c->vocab, bl, L.off_streams, offs, q16, qe, qbig, bigflag, biglist, counters,
-                 valid, status_dev};
+  if (L.n_rows > 0)
+    k_centres_even<<<(unsigned)std::min<int64_t>(L.n_rows, 65535), 256, 0, st>>>(
+        L.n_rows, row_slot, row_edst, row_tok, token_ids, c->t_even, c->vocab, c->kept_list, c->k_eff, cen8, valid);
+  CK(cudaFuncSetAttribute(rans_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, RANS_DEC_SMEM));
+  RansDecArgs da{d_chunks, d_prompts, 0, L.n_chunks_e, c->k_eff, c->kept_list, c->kept_scale, c->cdf, c->lut,
+                 cen8, bl, L.off_streams, offs, q16, qe, qbig, bigflag, biglist, counters, valid, status_dev};
   if (L.n_chunks_e > 0) {
-    rans_decode_kernel<<<(L.n_chunks_e + RANS_WARPS - 1) / RANS_WARPS, RANS_WARPS * 32, CDF_SMEM_BYTES, st>>>(da);
+    rans_decode_kernel<<<(L.n_chunks_e + RANS_WARPS - 1) / RANS_WARPS, RANS_WARPS * 32, RANS_DEC_SMEM, st>>>(da);
     CK(cudaGetLastError());
   }
   stage_mark(c, st, "rans_even");
@@ -986,14 +1188,14 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
     GemmProblem pr = make_problem(N_COEF / GEMM_BM, L.ne_pad, 256, true, status_dev);
     add_seg(pr, 0, 0, 1, 0, 0, 0, 0, N_COEF / GEMM_BK);
     add_seg(pr, 0, 0, 1, N_COEF, 0, 1, 0, N_COEF / GEMM_BK);
-    EpiMeanOdd::Params ep{c->t_odd, token_ids, e_tok, c_odd, c->vocab};
+    EpiMeanOdd::Params ep{c->t_odd, token_ids, e_tok, e_slot, c->kidx, cen8, c->k_eff, c->vocab};
     RET((run_gemm<EpiMeanOdd, 4, 1>(c->map_aon1, c->map_aon1, mb_qe, mb_qe, pr, ep, c->num_sms, st)));
   }
   stage_mark(c, st, "gemm_mean_odd");
   if (L.n_chunks_o > 0) {
     da.chunk0 = L.n_chunks_e;
     da.n_chunks = L.n_chunks_o;
-    rans_decode_kernel<<<(L.n_chunks_o + RANS_WARPS - 1) / RANS_WARPS, RANS_WARPS * 32, CDF_SMEM_BYTES, st>>>(da);
+    rans_decode_kernel<<<(L.n_chunks_o + RANS_WARPS - 1) / RANS_WARPS, RANS_WARPS * 32, RANS_DEC_SMEM, st>>>(da);
     CK(cudaGetLastError());
   }
   stage_mark(c, st, "rans_odd");
@@ -1108,6 +1310,19 @@ extern "C" int dckv_codec_export(const dckv_codec *c, uint16_t *cdf_host, uint8_
   return DCKV_OK;
 }
 
+extern "C" int dckv_debug_ratio(dckv_codec *c, void *ratio_dev) {
+  if (!c) return fail(DCKV_EINVAL, "NULL codec");
+  c->dbg_ratio = (float *)ratio_dev;
+  return DCKV_OK;
+}
+
+extern "C" int dckv_codec_info(const dckv_codec *c, int32_t *chunk_rows, double *model_bits_per_row) {
+  if (!c) return fail(DCKV_EINVAL, "NULL codec");
+  if (chunk_rows) *chunk_rows = c->chunk_rows;
+  if (model_bits_per_row) *model_bits_per_row = c->model_bits_per_row;
+  return DCKV_OK;
+}
+
 extern "C" int dckv_codec_tables(const dckv_codec *c, const void **t_even, const void **t_odd) {
   if (!c) return fail(DCKV_EINVAL, "NULL codec");
   if (t_even) *t_even = c->t_even;
@@ -1122,10 +1337,13 @@ extern "C" int dckv_ws_offsets(const dckv_codec *c, const int64_t *offs, int bat
   const WsPlan w = plan_ws(L, which);
   out->q32 = w.q32;
   out->qe = w.qe;
-  out->c_odd = w.c_odd;
+  out->cen8 = w.cen8;
+  out->row_slot = w.row_slot;
+  out->sym16 = w.sym16;
   out->q16 = w.q16;
   out->x16 = w.x16;
   out->g16 = w.g16;
+  out->counters = w.counters;
   out->n_rows = L.n_rows;
   out->ne_pad = L.ne_pad;
   out->n_chunks = L.n_chunks;

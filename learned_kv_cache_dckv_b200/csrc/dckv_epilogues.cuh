@@ -78,6 +78,38 @@ struct EpiGelu {
   }
 };
 
+// Chunk-accumulated form of EpiGelu (the hidden units feed the exact refinement too):
+// reads this thread's totals (columns c_begin .. c_begin + 63) from TMEM.
+struct EpiGeluTotals {
+  using Params = EpiGelu::Params;
+  static constexpr int SMEM_BYTES = 0;
+  __device__ static void tile(const Params &p, char *, int mt, int n0, int n_valid, int c_begin, uint32_t ttot,
+                              int ew, int lane, int) {
+    const int m = mt * GEMM_BM + ew * 32 + lane;
+    const float mw = p.muw1[m];
+#pragma unroll 1
+    for (int g = 0; g < 2; ++g) {
+      const int col0 = c_begin + g * 32;
+      if (col0 >= n_valid) break;
+      uint32_t r[32];
+      tmem_ld_32x32b_x32(ttot + (uint32_t)(g * 32), r);
+      tmem_ld_wait();
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        if (col0 + j < n_valid) {
+          const float h = u2f(r[j]) * p.scale - mw;
+          const float gl = 0.5f * h * (1.0f + erff(h * 0.70710678118654752f));
+          const __half hi = __float2half_rn(gl);
+          const __half lo = __float2half_rn(gl - __half2float(hi));
+          __half *row = p.g + (int64_t)(n0 + col0 + j) * (2 * N_HIDDEN);
+          row[m] = hi;
+          row[N_HIDDEN + m] = lo;
+        }
+      }
+    }
+  }
+};
+
 // ------------------------------------------------------------------ transform + quantiser
 // y = D * 2^-p_y - (mu @ basis)[c];  q = round_half_even(y / Delta_c), 0 if dropped;
 // q32[row][c] = q; even rows also write bf16(q) to their padded even row (the odd mean
@@ -118,26 +150,65 @@ struct EpiQuant {
   }
 };
 
-// Chunk-accumulated form of the same epilogue: the thread's 128 totals (columns
-// c_begin .. c_begin + 127 of the tile) are already summed in fp32 registers.
+// Chunk-accumulated transform + quantiser: reads this thread's totals (columns
+// c_begin .. c_begin + 63) from TMEM; codes whose fp32 ratio lies in the guard band around
+// a half step are listed for exact fp64 recomputation (whole rows when the row is large).
 struct EpiQuantTotals {
-  using Params = EpiQuant::Params;
-  __device__ static void finish(const Params &p, int mt, int n0, int n_valid, int c_begin, const float (&tot)[128],
-                                int ew, int lane) {
+  struct Params {
+    EpiQuant::Params q;
+    const float *row_norm;   // [rows] |x|_2 of the coded row
+    uint32_t *rowflag;       // [rows] 1 once the row is listed for full refinement
+    uint32_t *el_list;       // codes to refine: row * 2048 + c
+    uint32_t *full_list;     // rows to refine whole
+    uint32_t *counters;      // [0] listed codes, [1] listed rows
+    int64_t el_cap;
+    float *dbg_ratio;        // optional export of the fp32 ratios (self-test)
+  };
+  static constexpr int SMEM_BYTES = 0;
+  __device__ static void list_row(const Params &p, int row) {
+    if (atomicExch(&p.rowflag[row], 1u) == 0u) p.full_list[atomicAdd(&p.counters[1], 1u)] = (uint32_t)row;
+  }
+  __device__ static __noinline__ void flag(const Params &pp, int row, int c) {
+    if (pp.row_norm[row] > REFINE_NORM_FULL) {
+      list_row(pp, row);
+    } else {
+      const uint32_t idx = atomicAdd(&pp.counters[0], 1u);
+      if ((int64_t)idx < pp.el_cap) pp.el_list[idx] = (uint32_t)row * N_COEF + (uint32_t)c;
+      else list_row(pp, row);
+    }
+  }
+  __device__ static void tile(const Params &pp, char *, int mt, int n0, int n_valid, int c_begin, uint32_t ttot,
+                              int ew, int lane, int) {
+    const EpiQuant::Params &p = pp.q;
     const int c = mt * GEMM_BM + ew * 32 + lane;
     const float mb = p.mub[c];
     const float dl = p.delta[c];
     const bool kp = p.keep[c] != 0;
-#pragma unroll
-    for (int j = 0; j < 128; ++j) {
-      const int col = c_begin + j;
-      if (col < n_valid) {
-        const int row = n0 + col;
-        const float y = tot[j] * p.scale - mb;
-        const int q = kp ? __float2int_rn(__fdiv_rn(y, dl)) : 0;
-        p.q32[(int64_t)row * N_COEF + c] = q;
-        const int e = p.row_edst[row];
-        if (e >= 0) p.qe[(int64_t)e * N_COEF + c] = __float2bfloat16_rn((float)q);
+    const float wk = REFINE_KAPPA / dl;
+#pragma unroll 1
+    for (int g = 0; g < 2; ++g) {
+      const int col0 = c_begin + g * 32;
+      if (col0 >= n_valid) break;
+      uint32_t r[32];
+      tmem_ld_32x32b_x32(ttot + (uint32_t)(g * 32), r);
+      tmem_ld_wait();
+#pragma unroll 8
+      for (int j = 0; j < 32; ++j) {
+        const int col = col0 + j;
+        if (col < n_valid) {
+          const int row = n0 + col;
+          const float y = u2f(r[j]) * p.scale - mb;
+          const float ratio = __fdiv_rn(y, dl);
+          const int q = kp ? __float2int_rn(ratio) : 0;
+          p.q32[(int64_t)row * N_COEF + c] = q;
+          const int e = p.row_edst[row];
+          if (e >= 0) p.qe[(int64_t)e * N_COEF + c] = __float2bfloat16_rn((float)q);
+          if (pp.dbg_ratio) pp.dbg_ratio[(int64_t)row * N_COEF + c] = ratio;
+          if (kp) {
+            const float w = wk * pp.row_norm[row] + REFINE_W0;
+            if (0.5f - fabsf(ratio - rintf(ratio)) < w || !(fabsf(ratio) < 1.0e6f)) flag(pp, row, c);
+          }
+        }
       }
     }
   }
@@ -151,33 +222,53 @@ struct EpiMeanOdd {
   struct Params {
     const float *t_odd;      // [vocab][2048]
     const int32_t *tok_ids;  // [tokens]
-    const int32_t *e_tok;    // [ne_pad]
-    int8_t *c_odd;           // [ne_pad][2048]
+    const int32_t *e_tok;    // [ne_pad] token row of the odd row, -1 if none
+    const int32_t *e_slot;   // [ne_pad] slot row of that odd row
+    const int16_t *kidx;     // [2048] kept index, -1 if dropped
+    int8_t *cen8;            // [slots][k_eff]
+    int k_eff;
     int vocab;
   };
-  static constexpr int SMEM_BYTES = 0;
-  __device__ static void tile(const Params &p, char *, int mt, int n0, int n_valid, int bn, uint32_t tacc, int ew,
-                              int lane, int) {
+  // per tile column: t_odd row offset (or -1) and the slot row
+  static constexpr int SMEM_BYTES = 256 * 16;
+  __device__ static void tile(const Params &p, char *scratch, int mt, int n0, int n_valid, int bn, uint32_t tacc,
+                              int ew, int lane, int et) {
+    int64_t *s_row = reinterpret_cast<int64_t *>(scratch);
+    int32_t *s_slot = reinterpret_cast<int32_t *>(scratch + 256 * 8);
+    for (int j = et; j < n_valid; j += 128) {
+      const int ti = p.e_tok[n0 + j];
+      int64_t off = -1;
+      if (ti >= 0) {
+        const int tok = min(max(p.tok_ids[ti], 0), p.vocab - 1);
+        off = (int64_t)tok * N_COEF;
+      }
+      s_row[j] = off;
+      s_slot[j] = p.e_slot[n0 + j];
+    }
+    named_bar_sync(1, 128);
     const int c = mt * GEMM_BM + ew * 32 + lane;
+    const int kc = p.kidx[c];
     for (int c0 = 0; c0 < n_valid; c0 += 32) {
       uint32_t r[32];
       tmem_ld_32x32b_x32(tacc + (uint32_t)c0, r);
+      float tv[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {  // independent loads, issued together
+        const int64_t off = (kc >= 0 && c0 + j < n_valid) ? s_row[c0 + j] : -1;
+        tv[j] = off >= 0 ? __ldg(p.t_odd + off + c) : 0.f;
+      }
       tmem_ld_wait();
+      if (kc < 0) continue;
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
-        if (c0 + j < n_valid) {
-          const int e = n0 + c0 + j;
-          const int ti = p.e_tok[e];
-          if (ti >= 0) {
-            int tok = p.tok_ids[ti];
-            tok = min(max(tok, 0), p.vocab - 1);
-            const float mu = u2f(r[j]) + p.t_odd[(int64_t)tok * N_COEF + c];
-            const float cen = fminf(fmaxf(rintf(mu), -(float)ESC_LIMIT), (float)ESC_LIMIT);
-            p.c_odd[(int64_t)e * N_COEF + c] = (int8_t)cen;
-          }
+        if (c0 + j < n_valid && s_row[c0 + j] >= 0) {
+          const float mu = u2f(r[j]) + tv[j];
+          const float cen = fminf(fmaxf(rintf(mu), -(float)ESC_LIMIT), (float)ESC_LIMIT);
+          p.cen8[(int64_t)s_slot[c0 + j] * p.k_eff + kc] = (int8_t)cen;
         }
       }
     }
+    named_bar_sync(1, 128);  // the metadata is rewritten by the next tile
   }
 };
 

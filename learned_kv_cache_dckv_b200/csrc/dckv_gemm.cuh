@@ -49,9 +49,9 @@ struct GemmProblem {
   int *status;  // device int32; DCKV_ETIMEOUT (5) is written on a timed-out wait
 };
 
-template <int MAX_SLABS>
+template <int MAX_SLABS, int BN_MAX = GEMM_MAX_BN>
 struct GemmSmem {
-  static constexpr int STAGE_BYTES = MAX_SLABS * GEMM_SLAB_BYTES + GEMM_B_BYTES;
+  static constexpr int STAGE_BYTES = MAX_SLABS * GEMM_SLAB_BYTES + BN_MAX * GEMM_BK * 2;
 };
 
 // Epi must provide:
@@ -224,13 +224,16 @@ constexpr int gemm_smem_bytes() {
 }
 
 // ------------------------------------------------------------------------------------------
-// Chunk-accumulated variant (bn = 256).  The tensor core sums each MMA's products into the
+// Chunk-accumulated variant (bn = 128).  The tensor core sums each MMA's products into the
 // fp32 accumulator with truncation, so over a long K the error grows with the number of
 // MMA steps times the accumulator's ulp.  Here every CHUNK_STEPS * 64 elements of K go into
-// a fresh TMEM partial (two partials alternate), and 8 epilogue warps add each partial into
-// fp32 register totals with round-to-nearest; Epi::finish then works on the totals.
-// Thread (warp w >= 2): TMEM lane quarter w % 4, column half (w - 2) / 4.
+// a fresh TMEM partial P (two alternate, columns 0-127 and 128-255), and the epilogue warps
+// add each partial into a TMEM running total T (two alternate per tile, columns 256-383
+// and 384-511) with fp32 round-to-nearest adds.  After a tile's last chunk, Epi::tile reads
+// its totals from T.  Eight epilogue warps: warp w >= 2 owns TMEM lane quarter w % 4 and
+// column half (w - 2) / 4 (64 columns).
 constexpr int GEMMC_THREADS = 320;
+constexpr int GEMMC_BN = 128;
 
 template <class Epi, int STAGES, int MAX_SLABS, int CHUNK_STEPS>
 __global__ void __launch_bounds__(GEMMC_THREADS, 1)
@@ -238,7 +241,7 @@ __global__ void __launch_bounds__(GEMMC_THREADS, 1)
                         const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
                         const GemmProblem prob, const typename Epi::Params ep) {
   extern __shared__ __align__(1024) uint8_t dyn_smem[];
-  constexpr int STAGE_BYTES = GemmSmem<MAX_SLABS>::STAGE_BYTES;
+  constexpr int STAGE_BYTES = GemmSmem<MAX_SLABS, GEMMC_BN>::STAGE_BYTES;
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
   uint8_t *stages = base;
   uint64_t *full_bar = reinterpret_cast<uint64_t *>(base + STAGES * STAGE_BYTES);
@@ -247,6 +250,7 @@ __global__ void __launch_bounds__(GEMMC_THREADS, 1)
   uint64_t *part_empty = part_full + 2;
   uint32_t *tmem_base_smem = reinterpret_cast<uint32_t *>(part_empty + 2);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_base_smem + 1);
+  char *epi_scratch = reinterpret_cast<char *>(base + STAGES * STAGE_BYTES + 1024);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -329,7 +333,7 @@ __global__ void __launch_bounds__(GEMMC_THREADS, 1)
                 break;
               }
               tc_fence_after();
-              d_tmem = tmem_base + (uint32_t)(pb * GEMM_MAX_BN);
+              d_tmem = tmem_base + (uint32_t)(pb * GEMMC_BN);
               accumulate = 0;
             }
             if (!mbar_wait(&full_bar[stage], phase, abort_flag)) {
@@ -369,34 +373,38 @@ __global__ void __launch_bounds__(GEMMC_THREADS, 1)
     const int et = threadIdx.x - 64;  // 0..255
     const int ew = warp & 3;
     const int half = (warp - 2) >> 2;
-    const int c_begin = half * 128;
-    int pb = 0;
+    const uint32_t lane_base = (uint32_t)(ew * 32) << 16;
+    int pb = 0, tbuf = 0;
     uint32_t pph = 0;
     bool stop = false;
     for (int t = blockIdx.x; t < total_tiles && !stop; t += gridDim.x) {
       const int mt = t % prob.m_tiles;
       const int n0 = (t / prob.m_tiles) * prob.bn;
       const int n_valid = min(prob.bn, prob.n_rows - n0);
-      float tot[128];
-#pragma unroll
-      for (int j = 0; j < 128; ++j) tot[j] = 0.f;
+      const uint32_t tot = tmem_base + lane_base + (uint32_t)(2 * GEMMC_BN + tbuf * GEMMC_BN + half * 64);
       for (int ch = 0; ch < n_chunks; ++ch) {
-        if (et == 0) mbar_wait(&part_full[pb], pph, abort_flag);
-        named_bar_sync(1, 256);
-        if (*abort_flag) {
+        if (!mbar_wait(&part_full[pb], pph, abort_flag)) {
           stop = true;
           break;
         }
         tc_fence_after();
-        const uint32_t tb = tmem_base + ((uint32_t)(ew * 32) << 16) + (uint32_t)(pb * GEMM_MAX_BN + c_begin);
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
+        const uint32_t part = tmem_base + lane_base + (uint32_t)(pb * GEMMC_BN + half * 64);
+#pragma unroll 1
+        for (int g = 0; g < 2; ++g) {
           uint32_t r[32];
-          tmem_ld_32x32b_x32(tb + (uint32_t)(g * 32), r);
-          tmem_ld_wait();
+          tmem_ld_32x32b_x32(part + g * 32, r);
+          if (ch > 0) {
+            uint32_t s[32];
+            tmem_ld_32x32b_x32(tot + g * 32, s);
+            tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) tot[g * 32 + j] += __uint_as_float(r[j]);
+            for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) + __uint_as_float(s[j]));
+          } else {
+            tmem_ld_wait();
+          }
+          tmem_st_32x32b_x32(tot + g * 32, r);
         }
+        tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&part_empty[pb]);
         if (++pb == 2) {
@@ -405,7 +413,9 @@ __global__ void __launch_bounds__(GEMMC_THREADS, 1)
         }
       }
       if (stop) break;
-      Epi::finish(ep, mt, n0, n_valid, c_begin, tot, ew, lane);
+      tc_fence_after();
+      Epi::tile(ep, epi_scratch, mt, n0, n_valid, half * 64, tot, ew, lane, et);
+      tbuf ^= 1;
     }
   }
 
@@ -417,9 +427,9 @@ __global__ void __launch_bounds__(GEMMC_THREADS, 1)
   }
 }
 
-template <int STAGES, int MAX_SLABS>
+template <class Epi, int STAGES, int MAX_SLABS>
 constexpr int gemm_chunked_smem_bytes() {
-  return 1024 + STAGES * GemmSmem<MAX_SLABS>::STAGE_BYTES + 1024;
+  return 1024 + STAGES * GemmSmem<MAX_SLABS, GEMMC_BN>::STAGE_BYTES + 1024 + Epi::SMEM_BYTES;
 }
 
 }  // namespace dckv

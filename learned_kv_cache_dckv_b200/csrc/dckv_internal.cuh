@@ -33,6 +33,13 @@ constexpr int VERSION = 1;
 constexpr int HEADER_BYTES = 64;
 constexpr int CHUNK_FIXED_BYTES = 4 * LANES + 4;  // states + escape count
 constexpr int BIG_CODE = 2048;            // |q| >= 2048 is not exact in the fp16 code operand
+// Guard band of the transform: a code is recomputed in fp64 when its fp32 ratio y / Delta
+// lies within REFINE_KAPPA * |x|_2 / Delta + REFINE_W0 of a half-step boundary (the fp32
+// path's error grows with the row's norm); rows with |x|_2 > REFINE_NORM_FULL are
+// recomputed whole, correction layer included.
+constexpr float REFINE_KAPPA = 5.0e-7f;  // measured fp32 error on B200: <= 1.7e-7 * |x|_2
+constexpr float REFINE_W0 = 2.0e-5f;
+constexpr float REFINE_NORM_FULL = 32.0f;
 
 struct PromptInfo {
   int64_t tok_base;  // first row (token) of the prompt in the batch
@@ -44,6 +51,7 @@ struct PromptInfo {
   int32_t kept_base; // first kept row in the blob's kept section
   int32_t n_kept;
   int32_t chunk_e0, chunk_o0;  // first even / odd chunk (global chunk index)
+  int32_t slot_e0, slot_o0;    // slot row of the first even / odd row (chunk order)
 };
 
 struct ChunkDesc {
@@ -67,8 +75,11 @@ struct Layout {
 
 // Workspace carving (byte offsets from the workspace base, each 256-aligned).
 struct WsPlan {
-  size_t prompts, chunks, row_tok, row_pos, row_edst, e_tok;  // tables
-  size_t x16, g16, q32, qe, c_odd, words, states, nwords, nesc, offs;  // encode
+  size_t prompts, chunks, row_tok, row_pos, row_edst, e_tok, row_slot, e_slot;  // tables
+  size_t qe, cen8;                                                               // both
+  size_t x16, g16, q32, sym16, words, states, nwords, nesc, offs;                 // encode
+  size_t row_norm, rowflag, el_list, full_list;                         // encode refinement
+  int64_t el_cap;
   size_t q16, qbig, bigflag, biglist, counters, valid;                  // decode
   size_t total;
 };
@@ -102,7 +113,16 @@ struct dckv_codec {
   int16_t *kept_list = nullptr;   // [2048] kept component indices (first k_eff valid)
   uint8_t *kept_scale = nullptr;  // [2048]
   uint16_t *cdf = nullptr;   // [64][510]  cumulative frequencies (cdf[510] = 65536 implied)
+  uint16_t *lut = nullptr;   // [64][1024] decoder lookup (symbol holding slot b * 64)
+  int16_t *kidx = nullptr;   // [2048] kept index of a component, -1 if dropped
+  double model_bits_per_row = 0.0;  // entropy of the kept components' tables
+  float *dbg_ratio = nullptr;       // optional [rows][2048] export of the fp32 ratios y / Delta
   double *theta = nullptr;   // [128] RoPE frequencies
+  // exact (fp64) refinement of codes near a half-step boundary: fp32 copies, c-major
+  float *bt32 = nullptr;     // [2048][6144] basis^T
+  float *w1t32 = nullptr;    // [256][6144]  w1^T
+  float *w2t32 = nullptr;    // [2048][256]  w2^T
+  float *mu32 = nullptr;     // [6144]
   int p_y = 0, p_h = 0, p_inv = 0;  // power-of-two operand scales
   CUtensorMap map_ay2, map_aw2_2, map_aw2_1, map_ah2, map_ainv2, map_aon1;
   // stage timing (optional)

@@ -1,5 +1,5 @@
-// dckv_rans.cuh -- warp-interleaved rANS encode / decode, escape handling, scan and
-// compaction kernels of the DCKV codec.
+// dckv_rans.cuh -- warp-interleaved rANS encode / decode, parameter-to-symbol kernels,
+// scan and compaction of the DCKV codec.
 //
 // Coder (per chunk, one warp): 32 interleaved 32-bit states (lane j codes symbols
 // i = 32 t + j), 16-bit frequency precision, 16-bit renormalisation words, states in
@@ -8,108 +8,148 @@
 // t = T-1..0; at each step the lanes that must renormalise emit one word each, placed
 // with a ballot / popcount so that the decoder, walking t = 0..T-1 and reading words in
 // lane order, consumes exactly what was emitted.
+//
+// Everything a sequential step needs that does not depend on the state (symbols for the
+// encoder, centres for the decoder) is computed beforehand by fully parallel kernels and
+// laid out in "slot" order -- chunk by chunk, row by row, kept component by kept
+// component -- so the sequential loops read contiguous data one step ahead.
 #pragma once
 #include "dckv_internal.cuh"
 #include "dckv_ptx.cuh"
 
 namespace dckv {
 
-constexpr int RANS_WARPS = 8;  // chunks per block
-constexpr int CDF_SMEM_BYTES = N_SCALES * (N_SYM) * 2;
+constexpr int RANS_WARPS = 4;                            // chunks per block
+constexpr int PF = 16;                                   // steps of look-ahead for state-free data
+constexpr int CDF_SMEM_BYTES = N_SCALES * N_SYM * 2;     // 65,280
+constexpr int LUT_BITS = 10;                             // decoder lookup on slot >> 6
+constexpr int LUT_SIZE = 1 << LUT_BITS;
+constexpr int LUT_SMEM_BYTES = N_SCALES * LUT_SIZE * 2;  // 131,072
+constexpr int RANS_ENC_SMEM = CDF_SMEM_BYTES + N_COEF;
+constexpr int RANS_DEC_SMEM = CDF_SMEM_BYTES + LUT_SMEM_BYTES + N_COEF + 2 * N_COEF;
 
-__device__ __forceinline__ void load_cdf_smem(uint16_t *s_cdf, const uint16_t *g_cdf) {
-  const uint4 *src = reinterpret_cast<const uint4 *>(g_cdf);
-  uint4 *dst = reinterpret_cast<uint4 *>(s_cdf);
-  for (int i = threadIdx.x; i < CDF_SMEM_BYTES / 16; i += blockDim.x) dst[i] = src[i];
-  __syncthreads();
+__device__ __forceinline__ void copy_smem16(void *dst, const void *src, int bytes) {
+  const uint4 *s = reinterpret_cast<const uint4 *>(src);
+  uint4 *d = reinterpret_cast<uint4 *>(dst);
+  for (int i = threadIdx.x; i < bytes / 16; i += blockDim.x) d[i] = s[i];
 }
 
 __device__ __forceinline__ uint32_t cdf_at(const uint16_t *tab, int k) { return k < N_SYM ? tab[k] : PREC_TOTAL; }
 
-// centre of an even row: clamp(round(T_even[token][c]), +-127)
-__device__ __forceinline__ int even_centre(const float *t_even, int tok, int c) {
-  const float mu = t_even[(int64_t)tok * N_COEF + c];
-  return (int)fminf(fmaxf(rintf(mu), -(float)ESC_LIMIT), (float)ESC_LIMIT);
+// ------------------------------------------------------------------------------ symbols
+// Centres of even rows, clamp(round(T_even[token][c]), +-127), in slot order.
+__global__ void __launch_bounds__(256) k_centres_even(int64_t n_rows, const int32_t *row_slot,
+                                                      const int32_t *row_edst, const int32_t *row_tok,
+                                                      const int32_t *tok_ids, const float *t_even, int vocab,
+                                                      const int16_t *kept_list, int k_eff, int8_t *cen8,
+                                                      const int32_t *valid) {
+  if (valid && *valid != 1) return;
+  for (int64_t row = blockIdx.x; row < n_rows; row += gridDim.x) {
+    if (row_edst[row] < 0) continue;
+    int tok = tok_ids[row_tok[row]];
+    tok = min(max(tok, 0), vocab - 1);
+    const float *te = t_even + (int64_t)tok * N_COEF;
+    int8_t *dst = cen8 + (int64_t)row_slot[row] * k_eff;
+    for (int k = threadIdx.x; k < k_eff; k += blockDim.x) {
+      const float mu = te[kept_list[k]];
+      dst[k] = (int8_t)fminf(fmaxf(rintf(mu), -(float)ESC_LIMIT), (float)ESC_LIMIT);
+    }
+  }
 }
 
+// Encoder symbols in slot order: ESC if |q| > 127 else q - centre + 254.
+__global__ void __launch_bounds__(256) k_symbols(int64_t n_rows, const int32_t *row_slot, const int32_t *q32,
+                                                 const int8_t *cen8, const int16_t *kept_list, int k_eff,
+                                                 uint16_t *sym16) {
+  for (int64_t row = blockIdx.x; row < n_rows; row += gridDim.x) {
+    const int64_t base = (int64_t)row_slot[row] * k_eff;
+    const int32_t *q = q32 + row * N_COEF;
+    for (int k = threadIdx.x; k < k_eff; k += blockDim.x) {
+      const int v = q[kept_list[k]];
+      sym16[base + k] =
+          (v > ESC_LIMIT || v < -ESC_LIMIT) ? (uint16_t)ESC_SYM : (uint16_t)(v - cen8[base + k] + R_MAX);
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------ encode
 struct RansEncArgs {
   const ChunkDesc *chunks;
-  const PromptInfo *prompts;
   int n_chunks;
   int k_eff;
-  const int16_t *kept_list;
   const uint8_t *kept_scale;
   const uint16_t *cdf;
-  const int32_t *q32;       // [rows][2048]
-  const float *t_even;      // [vocab][2048]
-  const int32_t *tok_ids;   // [tokens]
-  const int8_t *c_odd;      // [ne_pad][2048]
-  int vocab;
-  uint16_t *words;          // word scratch: chunk c owns [sym_base, sym_base + S)
-  uint32_t *states;         // [chunks][32]
-  uint32_t *nwords;         // [chunks] words emitted
-  uint32_t *nesc;           // [chunks] escapes
+  const uint16_t *sym16;  // slot order
+  uint16_t *words;        // word scratch: chunk c owns [sym_base, sym_base + S)
+  uint32_t *states;       // [chunks][32]
+  uint32_t *nwords;       // [chunks] words emitted
+  uint32_t *nesc;         // [chunks] escapes
 };
 
 __global__ void __launch_bounds__(RANS_WARPS * 32) rans_encode_kernel(RansEncArgs a) {
   extern __shared__ __align__(16) uint8_t sm[];
   uint16_t *s_cdf = reinterpret_cast<uint16_t *>(sm);
-  load_cdf_smem(s_cdf, a.cdf);
+  uint8_t *s_scale = sm + CDF_SMEM_BYTES;
+  copy_smem16(s_cdf, a.cdf, CDF_SMEM_BYTES);
+  copy_smem16(s_scale, a.kept_scale, N_COEF);
+  __syncthreads();
   const int lane = threadIdx.x & 31;
   const int ci = blockIdx.x * RANS_WARPS + (threadIdx.x >> 5);
   if (ci >= a.n_chunks) return;
   const ChunkDesc cd = a.chunks[ci];
-  const PromptInfo pi = a.prompts[cd.prompt];
   const int K = a.k_eff;
   const int64_t S = (int64_t)cd.nrows * K;
   const int64_t T = (S + 31) / 32;
+  const uint16_t *syms = a.sym16 + cd.sym_base;
   uint16_t *wslot = a.words + cd.sym_base;
   int64_t pos = S;  // words are placed downwards from the end of the slot
   uint32_t x = RANS_L;
   uint32_t n_esc = 0;
   const uint32_t lt_mask = (1u << lane) - 1u;
-  for (int64_t t = T - 1; t >= 0; --t) {
-    const int64_t i = t * 32 + lane;
-    const bool valid = i < S;
-    uint32_t f = 1, c = 0;
-    bool is_esc = false;
-    if (valid) {
-      const int rl = (int)(i / K);
-      const int k = (int)(i - (int64_t)rl * K);
-      const int comp = a.kept_list[k];
-      const int s = a.kept_scale[k];
-      const int j = cd.j0 + rl;
-      const int64_t row = (int64_t)pi.row_base + 2 * j + cd.parity;
-      const int q = a.q32[row * N_COEF + comp];
-      int sym;
-      if (q > ESC_LIMIT || q < -ESC_LIMIT) {
-        sym = ESC_SYM;
-        is_esc = true;
-      } else {
-        int cen;
-        if (cd.parity == 0) {
-          int tok = a.tok_ids[pi.tok_base + HEAD_KEPT + 2 * j];
-          tok = min(max(tok, 0), a.vocab - 1);
-          cen = even_centre(a.t_even, tok, comp);
-        } else {
-          cen = a.c_odd[(int64_t)(pi.ebase + j) * N_COEF + comp];
-        }
-        sym = q - cen + R_MAX;
+  // symbol i = 32 t + lane, kept-component index k = i mod K, walked downwards; symbols
+  // are fetched PF steps ahead through a register ring (independent of the state)
+  int k = (K > 0 && T > 0) ? (int)(((T - 1) * 32 + lane) % K) : 0;
+  uint16_t ring[PF];
+#pragma unroll
+  for (int u = 0; u < PF; ++u) {
+    const int64_t iu = (T - 1 - u) * 32 + lane;
+    ring[u] = (T - 1 - u >= 0 && iu < S) ? syms[iu] : (uint16_t)0;
+  }
+  for (int64_t t0 = T - 1; t0 >= 0; t0 -= PF) {
+#pragma unroll
+    for (int u = 0; u < PF; ++u) {
+      const int64_t t = t0 - u;
+      if (t < 0) break;
+      const int64_t i = t * 32 + lane;
+      const bool valid = i < S;
+      const int sym = ring[u];
+      const int64_t tn = t - PF;
+      ring[u] = (tn >= 0 && tn * 32 + lane < S) ? syms[tn * 32 + lane] : (uint16_t)0;
+      const int kk = k;
+      if (K > 0) {
+        k -= 32;
+        while (k < 0) k += K;
       }
-      const uint16_t *tab = s_cdf + s * N_SYM;
-      c = tab[sym];
-      f = cdf_at(tab, sym + 1) - c;
+      uint32_t f = 1, c = 0;
+      if (valid) {
+        const uint16_t *tab = s_cdf + s_scale[kk] * N_SYM;
+        c = tab[sym];
+        f = cdf_at(tab, sym + 1) - c;
+      }
+      const bool emit = valid && x >= (f << 16);
+      const uint32_t m = __ballot_sync(0xffffffffu, emit);
+      const int nm = __popc(m);
+      if (emit) {
+        wslot[pos - nm + __popc(m & lt_mask)] = (uint16_t)(x & 0xFFFFu);
+        x >>= 16;
+      }
+      pos -= nm;
+      if (valid) {
+        const uint32_t qf = x / f;
+        x = (qf << 16) + (x - qf * f) + c;
+      }
+      n_esc += __popc(__ballot_sync(0xffffffffu, valid && sym == ESC_SYM));
     }
-    const bool emit = valid && x >= (f << 16);
-    const uint32_t m = __ballot_sync(0xffffffffu, emit);
-    const int nm = __popc(m);
-    if (emit) {
-      wslot[pos - nm + __popc(m & lt_mask)] = (uint16_t)(x & 0xFFFFu);
-      x >>= 16;
-    }
-    pos -= nm;
-    if (valid) x = ((x / f) << 16) + (x % f) + c;
-    n_esc += __popc(__ballot_sync(0xffffffffu, is_esc));
   }
   a.states[(int64_t)ci * 32 + lane] = x;
   if (lane == 0) {
@@ -178,7 +218,6 @@ __global__ void __launch_bounds__(1024) scan_kernel(ScanArgs a) {
   }
   __syncthreads();
   if (a.off_kept > a.blob_cap) return;
-  // header
   if (tid == 0) {
     uint8_t *h = a.blob;
     uint32_t *h32 = reinterpret_cast<uint32_t *>(h);
@@ -201,7 +240,6 @@ __global__ void __launch_bounds__(1024) scan_kernel(ScanArgs a) {
   for (int b = tid; b < a.batch; b += 1024) pt[b] = (uint32_t)a.prompts[b].N;
   uint32_t *ct = pt + a.batch;
   for (int c = tid; c <= a.n_chunks; c += 1024) ct[c] = a.offs[c];
-  // zero pad up to the kept rows
   const uint64_t tab_end = HEADER_BYTES + 4ull * (a.batch + a.n_chunks + 1);
   for (uint64_t o = tab_end + tid; o < a.off_kept; o += 1024) a.blob[o] = 0;
 }
@@ -214,6 +252,7 @@ struct CompactArgs {
   int k_eff;
   const int16_t *kept_list;
   const int32_t *q32;
+  const uint16_t *sym16;
   const uint16_t *words;
   const uint32_t *states, *nwords, *nesc, *offs;
   uint8_t *blob;
@@ -240,21 +279,17 @@ __global__ void __launch_bounds__(RANS_WARPS * 32) compact_kernel(CompactArgs a)
     uint32_t *ev = reinterpret_cast<uint32_t *>(sec + CHUNK_FIXED_BYTES);
     uint32_t ep = 0;
     const uint32_t lt_mask = (1u << lane) - 1u;
+    const uint16_t *syms = a.sym16 + cd.sym_base;
     for (int64_t i0 = 0; i0 < S && ep < ne; i0 += 32) {
       const int64_t i = i0 + lane;
-      int q = 0;
-      bool esc = false;
-      if (i < S) {
+      const bool esc = i < S && syms[i] == ESC_SYM;
+      const uint32_t m = __ballot_sync(0xffffffffu, esc);
+      if (esc) {
         const int rl = (int)(i / K);
         const int k = (int)(i - (int64_t)rl * K);
         const int64_t row = (int64_t)pi.row_base + 2 * (cd.j0 + rl) + cd.parity;
-        q = a.q32[row * N_COEF + a.kept_list[k]];
-        esc = q > ESC_LIMIT || q < -ESC_LIMIT;
-      }
-      const uint32_t m = __ballot_sync(0xffffffffu, esc);
-      if (esc) {
+        const int64_t v = (int64_t)a.q32[row * N_COEF + a.kept_list[k]];
         const uint32_t slot = ep + __popc(m & lt_mask);
-        const int64_t v = (int64_t)q;
         ev[2 * slot] = (uint32_t)(uint64_t)v;
         ev[2 * slot + 1] = (uint32_t)((uint64_t)v >> 32);
       }
@@ -269,7 +304,23 @@ __global__ void __launch_bounds__(RANS_WARPS * 32) compact_kernel(CompactArgs a)
   if (lane == 0 && (end - beg) > used) wd[nw] = 0;
 }
 
-// Decodes one pass (parity) of chunks: one warp per chunk.  Writes q as fp16 (exact for
+// ------------------------------------------------------------------------------ decode
+// Decoder lookup: lut[s][b] = the symbol whose slot range holds slot b * 64.
+__global__ void k_build_lut(const uint16_t *cdf, uint16_t *lut) {
+  const int s = blockIdx.x;
+  const uint16_t *tab = cdf + s * N_SYM;
+  for (int b = threadIdx.x; b < LUT_SIZE; b += blockDim.x) {
+    const uint32_t slot = (uint32_t)b << (16 - LUT_BITS);
+    int lo = 0, hi = N_SYM;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (tab[mid] <= slot) lo = mid; else hi = mid;
+    }
+    lut[s * LUT_SIZE + b] = (uint16_t)lo;
+  }
+}
+
+// Decodes one pass (parity) of chunks, one warp per chunk.  Writes q as fp16 (exact for
 // |q| < 2048) for the inverse GEMM, bf16(q) into padded even rows for the odd mean model,
 // and exact int32 values of codes with |q| >= 2048 (their rows are listed for a fix-up).
 struct RansDecArgs {
@@ -280,10 +331,8 @@ struct RansDecArgs {
   const int16_t *kept_list;
   const uint8_t *kept_scale;
   const uint16_t *cdf;
-  const float *t_even;
-  const int32_t *tok_ids;
-  const int8_t *c_odd;
-  int vocab;
+  const uint16_t *lut;
+  const int8_t *cen8;    // slot order
   const uint8_t *blob;
   uint64_t off_streams;
   const uint32_t *offs;  // chunk table inside the blob
@@ -300,8 +349,15 @@ struct RansDecArgs {
 __global__ void __launch_bounds__(RANS_WARPS * 32) rans_decode_kernel(RansDecArgs a) {
   extern __shared__ __align__(16) uint8_t sm[];
   uint16_t *s_cdf = reinterpret_cast<uint16_t *>(sm);
+  uint16_t *s_lut = reinterpret_cast<uint16_t *>(sm + CDF_SMEM_BYTES);
+  uint8_t *s_scale = sm + CDF_SMEM_BYTES + LUT_SMEM_BYTES;
+  int16_t *s_kept = reinterpret_cast<int16_t *>(sm + CDF_SMEM_BYTES + LUT_SMEM_BYTES + N_COEF);
   if (*a.valid != 1) return;
-  load_cdf_smem(s_cdf, a.cdf);
+  copy_smem16(s_cdf, a.cdf, CDF_SMEM_BYTES);
+  copy_smem16(s_lut, a.lut, LUT_SMEM_BYTES);
+  copy_smem16(s_scale, a.kept_scale, N_COEF);
+  copy_smem16(s_kept, a.kept_list, 2 * N_COEF);
+  __syncthreads();
   const int lane = threadIdx.x & 31;
   const int wi = blockIdx.x * RANS_WARPS + (threadIdx.x >> 5);
   if (wi >= a.n_chunks) return;
@@ -324,79 +380,107 @@ __global__ void __launch_bounds__(RANS_WARPS * 32) rans_decode_kernel(RansDecArg
   const uint32_t *ev = reinterpret_cast<const uint32_t *>(sec + CHUNK_FIXED_BYTES);
   const uint16_t *wd = reinterpret_cast<const uint16_t *>(sec + CHUNK_FIXED_BYTES + 8ull * ne);
   const int64_t n_wd = (int64_t)((end - beg) - CHUNK_FIXED_BYTES - 8ull * ne) / 2;
-  int64_t wp = 0;
+  const int8_t *cens = a.cen8 + cd.sym_base;
+  // words pass through a 64-word register window: lane j holds words wb + j and wb + 32 + j
+  int64_t wb = 0, wp = 0;
+  uint32_t w0 = lane < n_wd ? wd[lane] : 0u;
+  uint32_t w1 = 32 + lane < n_wd ? wd[32 + lane] : 0u;
   uint32_t ep = 0;
   const uint32_t lt_mask = (1u << lane) - 1u;
   if (x < RANS_L) bad = true;
-  for (int64_t t = 0; t < T; ++t) {
-    const int64_t i = t * 32 + lane;
-    const bool valid = i < S;
-    int q = 0, comp = 0;
-    int64_t row = 0;
-    bool need = false, is_esc = false;
-    if (valid) {
-      const int rl = (int)(i / K);
-      const int k = (int)(i - (int64_t)rl * K);
-      comp = a.kept_list[k];
-      const int s = a.kept_scale[k];
-      const int j = cd.j0 + rl;
-      row = (int64_t)pi.row_base + 2 * j + cd.parity;
-      const uint16_t *tab = s_cdf + s * N_SYM;
-      const uint32_t slot = x & 0xFFFFu;
-      int lo = 0, hi = N_SYM;  // invariant: tab[lo] <= slot < cdf(hi); 9 halvings
-      while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (tab[mid] <= slot) lo = mid; else hi = mid;
-      }
-      const uint32_t c = tab[lo];
-      const uint32_t f = cdf_at(tab, lo + 1) - c;
-      x = f * (x >> 16) + slot - c;
-      need = x < RANS_L;
-      if (lo == ESC_SYM) {
-        is_esc = true;
-      } else {
-        int cen;
-        if (cd.parity == 0) {
-          int tok = a.tok_ids[pi.tok_base + HEAD_KEPT + 2 * j];
-          tok = min(max(tok, 0), a.vocab - 1);
-          cen = even_centre(a.t_even, tok, comp);
-        } else {
-          cen = a.c_odd[(int64_t)(pi.ebase + j) * N_COEF + comp];
+  int rl = 0, k = lane;
+  if (K > 0)
+    while (k >= K) {
+      k -= K;
+      ++rl;
+    }
+  // centres are fetched PF steps ahead through a register ring (independent of the state)
+  int8_t ring[PF];
+#pragma unroll
+  for (int u = 0; u < PF; ++u) {
+    const int64_t iu = (int64_t)u * 32 + lane;
+    ring[u] = iu < S ? cens[iu] : (int8_t)0;
+  }
+  for (int64_t t0 = 0; t0 < T; t0 += PF) {
+#pragma unroll
+    for (int u = 0; u < PF; ++u) {
+      const int64_t t = t0 + u;
+      if (t >= T || bad) break;
+      const int64_t i = t * 32 + lane;
+      const bool valid = i < S;
+      const int cen = ring[u];
+      const int64_t inext = i + (int64_t)PF * 32;
+      ring[u] = inext < S ? cens[inext] : (int8_t)0;
+      const int kk = k, rr = rl;
+      int q = 0, comp = 0;
+      bool need = false, is_esc = false;
+      if (valid) {
+        comp = s_kept[kk];
+        const int s = s_scale[kk];
+        const uint16_t *tab = s_cdf + s * N_SYM;
+        const uint32_t slot = x & 0xFFFFu;
+        const int b = (int)(slot >> (16 - LUT_BITS));
+        int lo = s_lut[s * LUT_SIZE + b];
+        int hi = b + 1 < LUT_SIZE ? s_lut[s * LUT_SIZE + b + 1] : N_SYM - 1;  // answer in [lo, hi]
+        while (hi > lo) {
+          const int mid = (lo + hi + 1) >> 1;
+          if (tab[mid] <= slot) lo = mid; else hi = mid - 1;
         }
-        q = lo - R_MAX + cen;
+        const uint32_t c = tab[lo];
+        const uint32_t f = cdf_at(tab, lo + 1) - c;
+        x = f * (x >> 16) + slot - c;
+        need = x < RANS_L;
+        if (lo == ESC_SYM) is_esc = true;
+        else q = lo - R_MAX + cen;
+      }
+      const uint32_t m = __ballot_sync(0xffffffffu, need);
+      const int rank = __popc(m & lt_mask);
+      const int p = (int)(wp - wb) + rank;  // position in the window, < 64 by construction
+      const uint32_t v0 = __shfl_sync(0xffffffffu, w0, p & 31);
+      const uint32_t v1 = __shfl_sync(0xffffffffu, w1, p & 31);
+      if (need) {
+        if (wp + rank < n_wd) x = (x << 16) | (p < 32 ? v0 : v1);
+        else bad = true;
+      }
+      wp += __popc(m);
+      if (wp - wb >= 32) {  // slide the window by 32 words
+        w0 = w1;
+        wb += 32;
+        w1 = wb + 32 + lane < n_wd ? wd[wb + 32 + lane] : 0u;
+      }
+      const uint32_t me = __ballot_sync(0xffffffffu, is_esc);
+      if (is_esc) {
+        const uint32_t e = ep + __popc(me & lt_mask);
+        if (e < ne) {
+          const uint64_t v = (uint64_t)ev[2 * e] | ((uint64_t)ev[2 * e + 1] << 32);
+          const int64_t sv = (int64_t)v;
+          q = (int)max(min(sv, (int64_t)INT32_MAX), (int64_t)INT32_MIN);
+          if (sv >= -ESC_LIMIT && sv <= ESC_LIMIT) bad = true;  // not an escape value
+        } else {
+          bad = true;
+        }
+      }
+      ep += __popc(me);
+      bad = __any_sync(0xffffffffu, bad);
+      if (valid && !bad) {
+        const int j = cd.j0 + rr;
+        const int64_t row = (int64_t)pi.row_base + 2 * j + cd.parity;
+        a.q16[row * N_COEF + comp] = __float2half_rn((float)q);
+        if (cd.parity == 0) a.qe[(int64_t)(pi.ebase + j) * N_COEF + comp] = __float2bfloat16_rn((float)q);
+        if (q >= BIG_CODE || q <= -BIG_CODE) {
+          a.qbig[row * N_COEF + comp] = q;
+          if (atomicExch(&a.bigflag[row], 1u) == 0u) a.biglist[atomicAdd(a.bigcount, 1u)] = (int32_t)row;
+        }
+      }
+      if (K > 0) {
+        k += 32;
+        while (k >= K) {
+          k -= K;
+          ++rl;
+        }
       }
     }
-    const uint32_t m = __ballot_sync(0xffffffffu, need);
-    if (need) {
-      const int64_t w = wp + __popc(m & lt_mask);
-      if (w < n_wd) x = (x << 16) | wd[w]; else bad = true;
-    }
-    wp += __popc(m);
-    const uint32_t me = __ballot_sync(0xffffffffu, is_esc);
-    if (is_esc) {
-      const uint32_t e = ep + __popc(me & lt_mask);
-      if (e < ne) {
-        const uint64_t v = (uint64_t)ev[2 * e] | ((uint64_t)ev[2 * e + 1] << 32);
-        const int64_t sv = (int64_t)v;
-        q = (int)max(min(sv, (int64_t)INT32_MAX), (int64_t)INT32_MIN);
-        if (sv >= -ESC_LIMIT && sv <= ESC_LIMIT) bad = true;  // not an escape value
-      } else {
-        bad = true;
-      }
-    }
-    ep += __popc(me);
-    if (__any_sync(0xffffffffu, bad)) break;
-    if (valid) {
-      a.q16[row * N_COEF + comp] = __float2half_rn((float)q);
-      if (cd.parity == 0) {
-        const int j = (int)((row - pi.row_base) >> 1);
-        a.qe[(int64_t)(pi.ebase + j) * N_COEF + comp] = __float2bfloat16_rn((float)q);
-      }
-      if (q >= BIG_CODE || q <= -BIG_CODE) {
-        a.qbig[row * N_COEF + comp] = q;
-        if (atomicExch(&a.bigflag[row], 1u) == 0u) a.biglist[atomicAdd(a.bigcount, 1u)] = (int32_t)row;
-      }
-    }
+    if (bad) break;
   }
   // the stream must be consumed exactly: every state back at L, all escapes used, at
   // most one zero pad word left

@@ -65,9 +65,12 @@ def encode_gpu(gc, x, tok, offs):
     ws = gc._ws
     n, ne = v["n_rows"], v["ne_pad"]
     q32 = ws[v["q32"]: v["q32"] + 4 * n * 2048].view(torch.int32).reshape(n, 2048).cpu().numpy()
-    c_odd = ws[v["c_odd"]: v["c_odd"] + ne * 2048].view(torch.int8).reshape(ne, 2048).cpu().numpy()
+    K = gc.k_eff
+    cen8 = ws[v["cen8"]: v["cen8"] + n * K].view(torch.int8).reshape(n, K).cpu().numpy()
+    row_slot = ws[v["row_slot"]: v["row_slot"] + 4 * n].view(torch.int32).cpu().numpy()
+    cnt = ws[v["counters"]: v["counters"] + 8].view(torch.int32).cpu().numpy()
     return dict(blob_dev=blob, blob=blob[:size].cpu().numpy().tobytes(), size=size, status=status, q32=q32,
-                c_odd=c_odd)
+                cen=cen8[row_slot] if n else cen8, refined_codes=int(cnt[0]), refined_rows=int(cnt[1]))
 
 
 def decode_gpu(gc, blob_dev, size, tok, offs):
@@ -79,26 +82,17 @@ def decode_gpu(gc, blob_dev, size, tok, offs):
     return k, v, int(gc.status.item()), q16
 
 
-def gpu_even_centres(gc, np_codec, tok_rows):
-    te_ptr, _ = D.dckv_codec_tables(gc.handle)
-    te = torch.as_tensor(_CAI(te_ptr, (np_codec.embed.shape[0], 2048), "<f4"), device="cuda")
-    mu = te[torch.as_tensor(tok_rows, device="cuda", dtype=torch.long)]
-    return torch.clamp(torch.round(mu), -127, 127).to(torch.int64).cpu().numpy()
-
-
 def split_gpu_codes(gc, np_codec, res, tok, offs):
+    """Per prompt: the GPU's codes and centres (centres of dropped components are 0; they
+    are never used)."""
     lay = O.prompt_layout(np.diff(offs))
+    keep = O.scale_index(np_codec.laplace_b, np_codec.delta)[1]
     out = []
-    ebase = 0
-    tok_np = tok.cpu().numpy().astype(np.int64)
     for L in lay:
         q = res["q32"][L["row_base"]: L["row_base"] + L["n"]].astype(np.int64)
-        t0 = L["tok_base"] + 4
-        te = tok_np[t0: t0 + L["n"]: 2]
-        ce = gpu_even_centres(gc, np_codec, te) if te.size else np.zeros((0, 2048), np.int64)
-        co = res["c_odd"][ebase: ebase + L["n_o"]].astype(np.int64)
-        out.append(dict(q=q, qe=q[0::2], qo=q[1::2], ce=ce, co=co))
-        ebase += L["n_e"] + 1
+        cen = np.zeros((L["n"], 2048), np.int64)
+        cen[:, keep] = res["cen"][L["row_base"]: L["row_base"] + L["n"]]
+        out.append(dict(q=q, qe=q[0::2], qo=q[1::2], ce=cen[0::2], co=cen[1::2]))
     return out
 
 
@@ -136,8 +130,10 @@ def check_centres(gc_codes, np_codec, tok, offs):
                 qe = G["qe"]
                 right = np.concatenate([qe[1:], np.zeros((1, 2048), np.int64)])[: toks.size]
                 mu = O.mean_odd(np_codec.embed[toks], qe[: toks.size], right, np_codec.w_odd)
-            ora_c = O.centres(mu)
-            gpu_c = G["ce"] if par == 0 else G["co"]
+            keep = O.scale_index(np_codec.laplace_b, np_codec.delta)[1]
+            ora_c = O.centres(mu)[:, keep]
+            gpu_c = (G["ce"] if par == 0 else G["co"])[:, keep]
+            mu = mu[:, keep]
             bad = ora_c != gpu_c
             if bad.any():
                 assert np.all(np.abs(ora_c[bad] - gpu_c[bad]) == 1)
@@ -168,8 +164,9 @@ def full_check(src, np_codec, lens, seeds, chunk_rows=0, boost=(), boost_gain=60
     mism = check_centres(codes, np_codec, tok, offs)
     # bitstream: the oracle's coder and container on the GPU's codes and centres
     aux = {}
-    ora_blob = O.assemble_blob(xb, offs, codes, np_codec.laplace_b, np_codec.delta,
-                               chunk_rows or 32, aux=aux)
+    G = D.dckv_codec_info(gc.handle)["chunk_rows"]
+    assert G == (chunk_rows or 16)
+    ora_blob = O.assemble_blob(xb, offs, codes, np_codec.laplace_b, np_codec.delta, G, aux=aux)
     assert len(ora_blob) == res["size"]
     if ora_blob != res["blob"]:
         hdr = O.parse_blob(ora_blob)
@@ -177,6 +174,8 @@ def full_check(src, np_codec, lens, seeds, chunk_rows=0, boost=(), boost_gain=60
         pytest.fail(f"blob differs first at byte {first} (streams start at {hdr['off_streams']})")
     if expect_escapes:
         assert aux["n_esc"] > 0
+    if boost:
+        assert res["refined_rows"] >= 1  # far-out rows are recomputed whole
     # decode on the GPU, and the oracle's decode of the same blob
     k, v, st, q16 = decode_gpu(gc, res["blob_dev"], res["size"], tok, offs)
     assert st == D.DCKV_OK, D.STATUS_NAMES[st]
@@ -271,7 +270,7 @@ def test_corrupt_blobs_report_status(src, codec_55):
 def test_capacity_error(src, codec_55):
     gc = gpu_codec(codec_55)
     x, tok, offs = make_batch(src, codec_55, [132 + 64], [51])
-    small = torch.empty(2 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+    small = torch.empty(1024 * 1024, dtype=torch.uint8, device="cuda")  # below the kept rows' 1.55 MiB
     gc.encode(x, tok, offs, blob=small)
     torch.cuda.synchronize()
     assert int(gc.status.item()) == D.DCKV_ECAPACITY
@@ -298,7 +297,8 @@ def test_full_size_4k_prompt_sampled(src, codec_55):
     codes = split_gpu_codes(gc, codec_55, res, tok, offs)
     # the whole blob from the GPU's codes and centres through the oracle coder
     aux = {}
-    ora_blob = O.assemble_blob(xb, offs, codes, codec_55.laplace_b, codec_55.delta, 32, aux=aux)
+    G = D.dckv_codec_info(gc.handle)["chunk_rows"]
+    ora_blob = O.assemble_blob(xb, offs, codes, codec_55.laplace_b, codec_55.delta, G, aux=aux)
     assert ora_blob == res["blob"]
     payload = res["size"] - 132 * 12288
     model_bytes = aux["code_bits"] / 8
@@ -314,3 +314,35 @@ def test_full_size_4k_prompt_sampled(src, codec_55):
     vg = bits(v)[:, 4 + rows].transpose(1, 0, 2, 3)
     assert rel_frob(O.bf16_to_f64(kg), O.bf16_to_f64(want[:, :, 0])) <= ROW_TOL
     assert rel_frob(O.bf16_to_f64(vg), O.bf16_to_f64(want[:, :, 1])) <= ROW_TOL
+
+
+@pytest.mark.parametrize("which", ["literal", "fitted"])
+def test_guard_band_bounds_fp32_error(src, codec_literal, codec_55, which):
+    """The fp32 transform ratio y / Delta (before exact recomputation) stays within the
+    guard band the encoder uses to pick codes for fp64 recomputation,
+    5e-7 * |x|_2 / Delta + 2e-5, so every code outside the band is decided correctly."""
+    cod = codec_literal if which == "literal" else codec_55
+    gc = gpu_codec(cod)
+    lens = [132 + 400, 300] if which == "literal" else [132 + 700]
+    x, tok, offs = make_batch(src, cod, lens, seeds=[61, 62][: len(lens)])
+    n = sum(max(0, L - 132) for L in lens)
+    ratio = torch.full((n, 2048), float("nan"), dtype=torch.float32, device="cuda")
+    D.dckv_debug_ratio(gc.handle, ratio)
+    try:
+        encode_gpu(gc, x, tok, offs)
+    finally:
+        D.dckv_debug_ratio(gc.handle, None)
+    g = ratio.cpu().numpy().astype(np.float64)
+    xb = bits(x)
+    ora = O.analyse(xb, tok.cpu().numpy(), offs, cod)
+    r_o = np.concatenate([P["ratio"] for P in ora])
+    lay = O.prompt_layout(np.diff(offs))
+    rows = np.concatenate([np.arange(L["tok_base"] + 4, L["tok_base"] + 4 + L["n"]) for L in lay])
+    xn = np.linalg.norm(O.bf16_to_f64(xb[rows]), axis=1)
+    keep = O.scale_index(cod.laplace_b, cod.delta)[1]
+    d = cod.delta.astype(np.float64)
+    err = np.abs(g - r_o)[:, keep]
+    band = (5e-7 * xn[:, None] / d[None, keep]) + 2e-5
+    kappa = np.max(err * d[None, keep] / xn[:, None])
+    print(f"{which}: max fp32 ratio error {err.max():.3e} steps, effective kappa {kappa:.3e}")
+    assert np.all(err < band), (err.max(), kappa)
