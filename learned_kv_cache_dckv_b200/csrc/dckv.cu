@@ -299,8 +299,11 @@ __global__ void k_permute_mu(const float *mu, float *mu_perm) {
 // ============================================================================ per-call kernels
 // Row tables of one prompt per block: coded row r = row_base + i holds position 4 + i.
 __global__ void k_layout(const PromptInfo *prompts, int32_t *row_tok, int32_t *row_pos, int32_t *row_edst,
-                         int32_t *row_slot, int32_t *e_tok, int32_t *e_slot, __nv_bfloat16 *qe_zero_pad) {
+                         int32_t *row_slot, int32_t *e_tok, int32_t *e_slot, int32_t *slot_chunk, int chunk_rows,
+                         __nv_bfloat16 *qe_zero_pad) {
   const PromptInfo pi = prompts[blockIdx.x];
+  for (int j = threadIdx.x; j < pi.n_e; j += blockDim.x) slot_chunk[pi.slot_e0 + j] = pi.chunk_e0 + j / chunk_rows;
+  for (int j = threadIdx.x; j < pi.n_o; j += blockDim.x) slot_chunk[pi.slot_o0 + j] = pi.chunk_o0 + j / chunk_rows;
   for (int i = threadIdx.x; i < pi.n; i += blockDim.x) {
     const int r = pi.row_base + i;
     row_tok[r] = (int32_t)(pi.tok_base + HEAD_KEPT + i);
@@ -703,6 +706,7 @@ static WsPlan plan_ws(const Layout &L, int which /*0 encode, 1 decode*/) {
   w.e_tok = take(4ull * L.ne_pad);
   w.row_slot = take(4ull * L.n_rows);
   w.e_slot = take(4ull * L.ne_pad);
+  w.slot_chunk = take(4ull * L.n_rows);
   w.qe = take(2ull * L.ne_pad * N_COEF);
   w.cen8 = take(1ull * L.n_symbols);
   w.counters = take(256);
@@ -711,6 +715,7 @@ static WsPlan plan_ws(const Layout &L, int which /*0 encode, 1 decode*/) {
     w.g16 = take(2ull * L.n_rows * 2 * N_HIDDEN);
     w.q32 = take(4ull * L.n_rows * N_COEF);
     w.sym16 = take(2ull * L.n_symbols);
+    w.cf32 = take(4ull * L.n_symbols);
     w.words = take(2ull * L.n_symbols);
     w.states = take(128ull * L.n_chunks);
     w.nwords = take(4ull * L.n_chunks);
@@ -722,6 +727,8 @@ static WsPlan plan_ws(const Layout &L, int which /*0 encode, 1 decode*/) {
     w.el_list = take(4ull * w.el_cap);
     w.full_list = take(4ull * L.n_rows);
   } else {
+    w.slots16 = take(2ull * L.n_symbols);
+    w.row_esc = take(4ull * L.n_rows);
     w.q16 = take(2ull * L.n_rows * N_COEF);
     w.qbig = take(4ull * L.n_rows * N_COEF);
     w.bigflag = take(4ull * L.n_rows);
@@ -1027,6 +1034,9 @@ extern "C" int dckv_encode(const dckv_codec *c, const void *rows, const int32_t 
   int32_t *row_slot = (int32_t *)(ws + w.row_slot), *e_slot = (int32_t *)(ws + w.e_slot);
   int8_t *cen8 = (int8_t *)(ws + w.cen8);
   uint16_t *sym16 = (uint16_t *)(ws + w.sym16);
+  uint32_t *cf32 = (uint32_t *)(ws + w.cf32);
+  int32_t *slot_chunk = (int32_t *)(ws + w.slot_chunk);
+  uint32_t *nesc_w = (uint32_t *)(ws + w.nesc);
 
   float *row_norm = (float *)(ws + w.row_norm);
   uint32_t *rowflag = (uint32_t *)(ws + w.rowflag);
@@ -1037,8 +1047,10 @@ extern "C" int dckv_encode(const dckv_codec *c, const void *rows, const int32_t 
   CK(cudaMemsetAsync(status_dev, 0, 4, st));
   CK(cudaMemsetAsync(counters, 0, 256, st));
   if (L.n_rows) CK(cudaMemsetAsync(rowflag, 0, 4ull * L.n_rows, st));
+  if (L.n_chunks) CK(cudaMemsetAsync(nesc_w, 0, 4ull * L.n_chunks, st));
   RET(upload_tables(L, ws, w, st));
-  k_layout<<<L.batch, 256, 0, st>>>(d_prompts, row_tok, row_pos, row_edst, row_slot, e_tok, e_slot, qe);
+  k_layout<<<L.batch, 256, 0, st>>>(d_prompts, row_tok, row_pos, row_edst, row_slot, e_tok, e_slot, slot_chunk,
+                                    c->chunk_rows, qe);
   if (L.n_tokens > 0)
     k_convert<<<(unsigned)L.n_tokens, 192, 0, st>>>((const __nv_bfloat16 *)rows, d_prompts, L.batch, x16, bl, blob_cap,
                                                     L.off_kept, row_norm, status_dev);
@@ -1093,17 +1105,16 @@ extern "C" int dckv_encode(const dckv_codec *c, const void *rows, const int32_t 
     const unsigned rg = (unsigned)std::min<int64_t>(L.n_rows, 65535);
     k_centres_even<<<rg, 256, 0, st>>>(L.n_rows, row_slot, row_edst, row_tok, token_ids, c->t_even, c->vocab,
                                        c->kept_list, c->k_eff, cen8, nullptr);
-    k_symbols<<<rg, 256, 0, st>>>(L.n_rows, row_slot, q32, cen8, c->kept_list, c->k_eff, sym16);
+    k_symbols<<<rg, 256, 0, st>>>(L.n_rows, row_slot, slot_chunk, q32, cen8, c->kept_list, c->kept_scale, c->cdf,
+                                  c->k_eff, sym16, cf32, nesc_w);
     CK(cudaGetLastError());
     stage_mark(c, st, "symbols");
   }
   uint32_t *states = (uint32_t *)(ws + w.states), *nwords = (uint32_t *)(ws + w.nwords);
   uint32_t *nesc = (uint32_t *)(ws + w.nesc), *offs = (uint32_t *)(ws + w.offs);
   if (L.n_chunks > 0) {
-    RansEncArgs a{d_chunks, L.n_chunks, c->k_eff, c->kept_scale, c->cdf, sym16, (uint16_t *)(ws + w.words),
-                  states, nwords, nesc};
-    CK(cudaFuncSetAttribute(rans_encode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, RANS_ENC_SMEM));
-    rans_encode_kernel<<<(L.n_chunks + RANS_WARPS - 1) / RANS_WARPS, RANS_WARPS * 32, RANS_ENC_SMEM, st>>>(a);
+    RansEncArgs a{d_chunks, L.n_chunks, c->k_eff, cf32, (uint16_t *)(ws + w.words), states, nwords};
+    rans_encode_kernel<<<(L.n_chunks + RANS_WARPS - 1) / RANS_WARPS, RANS_WARPS * 32, 0, st>>>(a);
     CK(cudaGetLastError());
   }
   stage_mark(c, st, "rans_encode");
@@ -1148,6 +1159,9 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
   __nv_bfloat16 *qe = (__nv_bfloat16 *)(ws + w.qe);
   int32_t *row_slot = (int32_t *)(ws + w.row_slot), *e_slot = (int32_t *)(ws + w.e_slot);
   int8_t *cen8 = (int8_t *)(ws + w.cen8);
+  int32_t *slot_chunk = (int32_t *)(ws + w.slot_chunk);
+  uint16_t *slots16 = (uint16_t *)(ws + w.slots16);
+  uint32_t *row_esc = (uint32_t *)(ws + w.row_esc);
   __half *q16 = (__half *)(ws + w.q16);
   int32_t *qbig = (int32_t *)(ws + w.qbig);
   uint32_t *bigflag = (uint32_t *)(ws + w.bigflag);
@@ -1164,7 +1178,8 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
     CK(cudaMemsetAsync(q16, 0, 2ull * L.n_rows * N_COEF, st));
     CK(cudaMemsetAsync(bigflag, 0, 4ull * L.n_rows, st));
   }
-  k_layout<<<L.batch, 256, 0, st>>>(d_prompts, row_tok, row_pos, row_edst, row_slot, e_tok, e_slot, nullptr);
+  k_layout<<<L.batch, 256, 0, st>>>(d_prompts, row_tok, row_pos, row_edst, row_slot, e_tok, e_slot, slot_chunk,
+                                    c->chunk_rows, nullptr);
   HeaderCheck hc{bl, blob_bytes, d_prompts, L.batch, c->chunk_rows, c->k_eff, L.n_chunks_e, L.n_chunks_o,
                  L.n_kept, L.off_kept, L.off_streams, valid, status_dev};
   k_check_header<<<1, 256, 0, st>>>(hc);
@@ -1175,10 +1190,20 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
     k_centres_even<<<(unsigned)std::min<int64_t>(L.n_rows, 65535), 256, 0, st>>>(
         L.n_rows, row_slot, row_edst, row_tok, token_ids, c->t_even, c->vocab, c->kept_list, c->k_eff, cen8, valid);
   CK(cudaFuncSetAttribute(rans_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, RANS_DEC_SMEM));
-  RansDecArgs da{d_chunks, d_prompts, 0, L.n_chunks_e, c->k_eff, c->kept_list, c->kept_scale, c->cdf, c->lut,
-                 cen8, bl, L.off_streams, offs, q16, qe, qbig, bigflag, biglist, counters, valid, status_dev};
+  CK(cudaFuncSetAttribute(k_decode_symbols, cudaFuncAttributeMaxDynamicSharedMemorySize, DEC_FINISH_SMEM));
+  RansDecArgs da{d_chunks, 0, L.n_chunks_e, c->k_eff, c->kept_scale, c->cdf, c->lut, bl, L.off_streams, offs,
+                 slots16, valid, status_dev};
+  DecCodesArgs fa{d_chunks, d_prompts, 0, L.n_chunks_e, c->chunk_rows, c->k_eff, c->kept_list, cen8, slots16,
+                  row_esc, bl, L.off_streams, offs, q16, qe, qbig, bigflag, biglist, counters, valid, status_dev};
+  int64_t ne_rows = 0;
+  for (const PromptInfo &p : L.prompts) ne_rows += p.n_e;
+  const unsigned sym_blocks = (unsigned)std::max<int64_t>(1, std::min<int64_t>(L.n_rows, 4 * c->num_sms));
   if (L.n_chunks_e > 0) {
     rans_decode_kernel<<<(L.n_chunks_e + RANS_WARPS - 1) / RANS_WARPS, RANS_WARPS * 32, RANS_DEC_SMEM, st>>>(da);
+    stage_mark(c, st, "rans_even_loop");
+    k_decode_symbols<<<sym_blocks, 256, DEC_FINISH_SMEM, st>>>(0, ne_rows, c->k_eff, c->kept_scale, c->cdf, c->lut,
+                                                              slots16, row_esc, valid);
+    k_decode_codes<<<(unsigned)((L.n_chunks_e * c->chunk_rows + 7) / 8), 256, 0, st>>>(fa);
     CK(cudaGetLastError());
   }
   stage_mark(c, st, "rans_even");
@@ -1195,7 +1220,13 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
   if (L.n_chunks_o > 0) {
     da.chunk0 = L.n_chunks_e;
     da.n_chunks = L.n_chunks_o;
+    fa.chunk0 = L.n_chunks_e;
+    fa.n_chunks = L.n_chunks_o;
     rans_decode_kernel<<<(L.n_chunks_o + RANS_WARPS - 1) / RANS_WARPS, RANS_WARPS * 32, RANS_DEC_SMEM, st>>>(da);
+    stage_mark(c, st, "rans_odd_loop");
+    k_decode_symbols<<<sym_blocks, 256, DEC_FINISH_SMEM, st>>>(ne_rows, L.n_rows - ne_rows, c->k_eff, c->kept_scale,
+                                                              c->cdf, c->lut, slots16, row_esc, valid);
+    k_decode_codes<<<(unsigned)((L.n_chunks_o * c->chunk_rows + 7) / 8), 256, 0, st>>>(fa);
     CK(cudaGetLastError());
   }
   stage_mark(c, st, "rans_odd");

@@ -75,9 +75,10 @@ struct Layout {
 
 // Workspace carving (byte offsets from the workspace base, each 256-aligned).
 struct WsPlan {
-  size_t prompts, chunks, row_tok, row_pos, row_edst, e_tok, row_slot, e_slot;  // tables
+  size_t prompts, chunks, row_tok, row_pos, row_edst, e_tok, row_slot, e_slot, slot_chunk;  // tables
   size_t qe, cen8;                                                               // both
-  size_t x16, g16, q32, sym16, words, states, nwords, nesc, offs;                 // encode
+  size_t x16, g16, q32, sym16, cf32, words, states, nwords, nesc, offs;           // encode
+  size_t slots16, row_esc;                                                        // decode
   size_t row_norm, rowflag, el_list, full_list;                         // encode refinement
   int64_t el_cap;
   size_t q16, qbig, bigflag, biglist, counters, valid;                  // decode

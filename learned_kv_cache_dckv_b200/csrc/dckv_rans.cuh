@@ -25,8 +25,8 @@ constexpr int CDF_SMEM_BYTES = N_SCALES * N_SYM * 2;     // 65,280
 constexpr int LUT_BITS = 10;                             // decoder lookup on slot >> 6
 constexpr int LUT_SIZE = 1 << LUT_BITS;
 constexpr int LUT_SMEM_BYTES = N_SCALES * LUT_SIZE * 2;  // 131,072
-constexpr int RANS_ENC_SMEM = CDF_SMEM_BYTES + N_COEF;
-constexpr int RANS_DEC_SMEM = CDF_SMEM_BYTES + LUT_SMEM_BYTES + N_COEF + 2 * N_COEF;
+constexpr int RANS_DEC_SMEM = CDF_SMEM_BYTES + LUT_SMEM_BYTES + N_COEF;
+constexpr int DEC_FINISH_SMEM = CDF_SMEM_BYTES + LUT_SMEM_BYTES;
 
 __device__ __forceinline__ void copy_smem16(void *dst, const void *src, int bytes) {
   const uint4 *s = reinterpret_cast<const uint4 *>(src);
@@ -57,18 +57,35 @@ __global__ void __launch_bounds__(256) k_centres_even(int64_t n_rows, const int3
   }
 }
 
-// Encoder symbols in slot order: ESC if |q| > 127 else q - centre + 254.
-__global__ void __launch_bounds__(256) k_symbols(int64_t n_rows, const int32_t *row_slot, const int32_t *q32,
-                                                 const int8_t *cen8, const int16_t *kept_list, int k_eff,
-                                                 uint16_t *sym16) {
+// Encoder inputs in slot order: the symbol (ESC if |q| > 127 else q - centre + 254), its
+// table entry packed as cdf | (freq - 1) << 16, and the escape count of each chunk.
+__global__ void __launch_bounds__(256) k_symbols(int64_t n_rows, const int32_t *row_slot, const int32_t *slot_chunk,
+                                                 const int32_t *q32, const int8_t *cen8, const int16_t *kept_list,
+                                                 const uint8_t *kept_scale, const uint16_t *cdf, int k_eff,
+                                                 uint16_t *sym16, uint32_t *cf32, uint32_t *nesc) {
+  __shared__ int esc_count;
   for (int64_t row = blockIdx.x; row < n_rows; row += gridDim.x) {
-    const int64_t base = (int64_t)row_slot[row] * k_eff;
+    if (threadIdx.x == 0) esc_count = 0;
+    __syncthreads();
+    const int slot = row_slot[row];
+    const int64_t base = (int64_t)slot * k_eff;
     const int32_t *q = q32 + row * N_COEF;
+    int esc = 0;
     for (int k = threadIdx.x; k < k_eff; k += blockDim.x) {
       const int v = q[kept_list[k]];
-      sym16[base + k] =
-          (v > ESC_LIMIT || v < -ESC_LIMIT) ? (uint16_t)ESC_SYM : (uint16_t)(v - cen8[base + k] + R_MAX);
+      const bool is_esc = v > ESC_LIMIT || v < -ESC_LIMIT;
+      const int sym = is_esc ? ESC_SYM : v - cen8[base + k] + R_MAX;
+      esc += is_esc;
+      const uint16_t *tab = cdf + kept_scale[k] * N_SYM;
+      const uint32_t c = tab[sym];
+      const uint32_t f = cdf_at(tab, sym + 1) - c;
+      sym16[base + k] = (uint16_t)sym;
+      cf32[base + k] = c | ((f - 1u) << 16);
     }
+    if (esc) atomicAdd(&esc_count, esc);
+    __syncthreads();
+    if (threadIdx.x == 0 && esc_count) atomicAdd(&nesc[slot_chunk[slot]], (uint32_t)esc_count);
+    __syncthreads();
   }
 }
 
@@ -77,85 +94,60 @@ struct RansEncArgs {
   const ChunkDesc *chunks;
   int n_chunks;
   int k_eff;
-  const uint8_t *kept_scale;
-  const uint16_t *cdf;
-  const uint16_t *sym16;  // slot order
-  uint16_t *words;        // word scratch: chunk c owns [sym_base, sym_base + S)
-  uint32_t *states;       // [chunks][32]
-  uint32_t *nwords;       // [chunks] words emitted
-  uint32_t *nesc;         // [chunks] escapes
+  const uint32_t *cf32;  // slot order: cdf | (freq - 1) << 16
+  uint16_t *words;       // word scratch: chunk c owns [sym_base, sym_base + S)
+  uint32_t *states;      // [chunks][32]
+  uint32_t *nwords;      // [chunks] words emitted
 };
 
 __global__ void __launch_bounds__(RANS_WARPS * 32) rans_encode_kernel(RansEncArgs a) {
-  extern __shared__ __align__(16) uint8_t sm[];
-  uint16_t *s_cdf = reinterpret_cast<uint16_t *>(sm);
-  uint8_t *s_scale = sm + CDF_SMEM_BYTES;
-  copy_smem16(s_cdf, a.cdf, CDF_SMEM_BYTES);
-  copy_smem16(s_scale, a.kept_scale, N_COEF);
-  __syncthreads();
   const int lane = threadIdx.x & 31;
   const int ci = blockIdx.x * RANS_WARPS + (threadIdx.x >> 5);
   if (ci >= a.n_chunks) return;
   const ChunkDesc cd = a.chunks[ci];
-  const int K = a.k_eff;
-  const int64_t S = (int64_t)cd.nrows * K;
-  const int64_t T = (S + 31) / 32;
-  const uint16_t *syms = a.sym16 + cd.sym_base;
+  const uint32_t S = (uint32_t)cd.nrows * (uint32_t)a.k_eff;  // < 2^20
+  const int T = (int)((S + 31) / 32);
+  const uint32_t *cfs = a.cf32 + cd.sym_base;
   uint16_t *wslot = a.words + cd.sym_base;
-  int64_t pos = S;  // words are placed downwards from the end of the slot
+  uint32_t pos = S;  // words are placed downwards from the end of the slot
   uint32_t x = RANS_L;
-  uint32_t n_esc = 0;
   const uint32_t lt_mask = (1u << lane) - 1u;
-  // symbol i = 32 t + lane, kept-component index k = i mod K, walked downwards; symbols
-  // are fetched PF steps ahead through a register ring (independent of the state)
-  int k = (K > 0 && T > 0) ? (int)(((T - 1) * 32 + lane) % K) : 0;
-  uint16_t ring[PF];
+  // table entries are fetched PF steps ahead through a register ring (independent of x)
+  uint32_t ring[PF];
 #pragma unroll
   for (int u = 0; u < PF; ++u) {
-    const int64_t iu = (T - 1 - u) * 32 + lane;
-    ring[u] = (T - 1 - u >= 0 && iu < S) ? syms[iu] : (uint16_t)0;
+    const int t = T - 1 - u;
+    const uint32_t iu = (uint32_t)t * 32u + lane;
+    ring[u] = (t >= 0 && iu < S) ? cfs[iu] : 0u;
   }
-  for (int64_t t0 = T - 1; t0 >= 0; t0 -= PF) {
+  for (int t0 = T - 1; t0 >= 0; t0 -= PF) {
 #pragma unroll
     for (int u = 0; u < PF; ++u) {
-      const int64_t t = t0 - u;
+      const int t = t0 - u;
       if (t < 0) break;
-      const int64_t i = t * 32 + lane;
+      const uint32_t i = (uint32_t)t * 32u + lane;
       const bool valid = i < S;
-      const int sym = ring[u];
-      const int64_t tn = t - PF;
-      ring[u] = (tn >= 0 && tn * 32 + lane < S) ? syms[tn * 32 + lane] : (uint16_t)0;
-      const int kk = k;
-      if (K > 0) {
-        k -= 32;
-        while (k < 0) k += K;
-      }
-      uint32_t f = 1, c = 0;
-      if (valid) {
-        const uint16_t *tab = s_cdf + s_scale[kk] * N_SYM;
-        c = tab[sym];
-        f = cdf_at(tab, sym + 1) - c;
-      }
+      const uint32_t cf = ring[u];
+      const int tn = t - PF;
+      const uint32_t in = (uint32_t)tn * 32u + lane;
+      ring[u] = (tn >= 0 && in < S) ? cfs[in] : 0u;
+      const uint32_t c = cf & 0xFFFFu;
+      const uint32_t f = valid ? (cf >> 16) + 1u : 1u;
       const bool emit = valid && x >= (f << 16);
       const uint32_t m = __ballot_sync(0xffffffffu, emit);
-      const int nm = __popc(m);
       if (emit) {
-        wslot[pos - nm + __popc(m & lt_mask)] = (uint16_t)(x & 0xFFFFu);
+        wslot[pos - __popc(m) + __popc(m & lt_mask)] = (uint16_t)(x & 0xFFFFu);
         x >>= 16;
       }
-      pos -= nm;
+      pos -= __popc(m);
       if (valid) {
         const uint32_t qf = x / f;
         x = (qf << 16) + (x - qf * f) + c;
       }
-      n_esc += __popc(__ballot_sync(0xffffffffu, valid && sym == ESC_SYM));
     }
   }
   a.states[(int64_t)ci * 32 + lane] = x;
-  if (lane == 0) {
-    a.nwords[ci] = (uint32_t)(S - pos);
-    a.nesc[ci] = n_esc;
-  }
+  if (lane == 0) a.nwords[ci] = S - pos;
 }
 
 // Exclusive scan of chunk section sizes (one block); writes the chunk table and header.
@@ -320,28 +312,20 @@ __global__ void k_build_lut(const uint16_t *cdf, uint16_t *lut) {
   }
 }
 
-// Decodes one pass (parity) of chunks, one warp per chunk.  Writes q as fp16 (exact for
-// |q| < 2048) for the inverse GEMM, bf16(q) into padded even rows for the odd mean model,
-// and exact int32 values of codes with |q| >= 2048 (their rows are listed for a fix-up).
+// Decodes one pass (parity) of chunks, one warp per chunk.  The loop carries only the
+// rANS states: for each symbol it finds the table entry holding the state's slot, updates
+// the state, renormalises, and writes the slot (slot order) for the finishing kernel.
 struct RansDecArgs {
   const ChunkDesc *chunks;
-  const PromptInfo *prompts;
   int chunk0, n_chunks;  // this pass: chunks [chunk0, chunk0 + n_chunks)
   int k_eff;
-  const int16_t *kept_list;
   const uint8_t *kept_scale;
   const uint16_t *cdf;
   const uint16_t *lut;
-  const int8_t *cen8;    // slot order
   const uint8_t *blob;
   uint64_t off_streams;
   const uint32_t *offs;  // chunk table inside the blob
-  __half *q16;           // [rows][2048]
-  __nv_bfloat16 *qe;     // [ne_pad][2048]
-  int32_t *qbig;         // [rows][2048], written only where |q| >= 2048
-  uint32_t *bigflag;     // [rows]
-  int32_t *biglist;      // [rows]
-  uint32_t *bigcount;
+  uint16_t *slots;       // slot order: the decoded slot of every symbol
   const int32_t *valid;  // header check result (1 = ok)
   int32_t *status;
 };
@@ -351,72 +335,50 @@ __global__ void __launch_bounds__(RANS_WARPS * 32) rans_decode_kernel(RansDecArg
   uint16_t *s_cdf = reinterpret_cast<uint16_t *>(sm);
   uint16_t *s_lut = reinterpret_cast<uint16_t *>(sm + CDF_SMEM_BYTES);
   uint8_t *s_scale = sm + CDF_SMEM_BYTES + LUT_SMEM_BYTES;
-  int16_t *s_kept = reinterpret_cast<int16_t *>(sm + CDF_SMEM_BYTES + LUT_SMEM_BYTES + N_COEF);
   if (*a.valid != 1) return;
   copy_smem16(s_cdf, a.cdf, CDF_SMEM_BYTES);
   copy_smem16(s_lut, a.lut, LUT_SMEM_BYTES);
   copy_smem16(s_scale, a.kept_scale, N_COEF);
-  copy_smem16(s_kept, a.kept_list, 2 * N_COEF);
   __syncthreads();
   const int lane = threadIdx.x & 31;
   const int wi = blockIdx.x * RANS_WARPS + (threadIdx.x >> 5);
   if (wi >= a.n_chunks) return;
   const int ci = a.chunk0 + wi;
   const ChunkDesc cd = a.chunks[ci];
-  const PromptInfo pi = a.prompts[cd.prompt];
   const int K = a.k_eff;
-  const int64_t S = (int64_t)cd.nrows * K;
-  const int64_t T = (S + 31) / 32;
+  const uint32_t S = (uint32_t)cd.nrows * (uint32_t)K;  // < 2^20
+  const int T = (int)((S + 31) / 32);
   const uint64_t beg = a.off_streams + a.offs[ci];
   const uint64_t end = a.off_streams + a.offs[ci + 1];
   const uint8_t *sec = a.blob + beg;
   const uint32_t ne = reinterpret_cast<const uint32_t *>(sec)[32];
-  bool bad = (end - beg) < CHUNK_FIXED_BYTES || (uint64_t)CHUNK_FIXED_BYTES + 8ull * ne > (end - beg);
-  if (__any_sync(0xffffffffu, bad)) {
+  if ((end - beg) < CHUNK_FIXED_BYTES || (uint64_t)CHUNK_FIXED_BYTES + 8ull * ne > (end - beg)) {
     if (lane == 0) atomicExch(a.status, DCKV_ECORRUPT);
     return;
   }
   uint32_t x = reinterpret_cast<const uint32_t *>(sec)[lane];
-  const uint32_t *ev = reinterpret_cast<const uint32_t *>(sec + CHUNK_FIXED_BYTES);
   const uint16_t *wd = reinterpret_cast<const uint16_t *>(sec + CHUNK_FIXED_BYTES + 8ull * ne);
-  const int64_t n_wd = (int64_t)((end - beg) - CHUNK_FIXED_BYTES - 8ull * ne) / 2;
-  const int8_t *cens = a.cen8 + cd.sym_base;
-  // words pass through a 64-word register window: lane j holds words wb + j and wb + 32 + j
-  int64_t wb = 0, wp = 0;
+  const uint32_t n_wd = (uint32_t)(((end - beg) - CHUNK_FIXED_BYTES - 8ull * ne) / 2);
+  uint16_t *out = a.slots + cd.sym_base;
+  // words pass through a 96-word register ring: lane j holds words wb + j, wb + 32 + j and
+  // (prefetched) wb + 64 + j
+  uint32_t wb = 0, wp = 0;
   uint32_t w0 = lane < n_wd ? wd[lane] : 0u;
   uint32_t w1 = 32 + lane < n_wd ? wd[32 + lane] : 0u;
-  uint32_t ep = 0;
+  uint32_t w2 = 64 + lane < n_wd ? wd[64 + lane] : 0u;
   const uint32_t lt_mask = (1u << lane) - 1u;
-  if (x < RANS_L) bad = true;
-  int rl = 0, k = lane;
-  if (K > 0)
-    while (k >= K) {
-      k -= K;
-      ++rl;
-    }
-  // centres are fetched PF steps ahead through a register ring (independent of the state)
-  int8_t ring[PF];
-#pragma unroll
-  for (int u = 0; u < PF; ++u) {
-    const int64_t iu = (int64_t)u * 32 + lane;
-    ring[u] = iu < S ? cens[iu] : (int8_t)0;
-  }
-  for (int64_t t0 = 0; t0 < T; t0 += PF) {
-#pragma unroll
-    for (int u = 0; u < PF; ++u) {
-      const int64_t t = t0 + u;
-      if (t >= T || bad) break;
-      const int64_t i = t * 32 + lane;
+  bool bad = x < RANS_L;
+  int k = K > 0 ? lane % K : 0;
+  for (int t0 = 0; t0 < T && !bad; t0 += 16) {
+#pragma unroll 4
+    for (int u = 0; u < 16; ++u) {
+      const int t = t0 + u;
+      if (t >= T) break;
+      const uint32_t i = (uint32_t)t * 32u + lane;
       const bool valid = i < S;
-      const int cen = ring[u];
-      const int64_t inext = i + (int64_t)PF * 32;
-      ring[u] = inext < S ? cens[inext] : (int8_t)0;
-      const int kk = k, rr = rl;
-      int q = 0, comp = 0;
-      bool need = false, is_esc = false;
+      bool need = false;
       if (valid) {
-        comp = s_kept[kk];
-        const int s = s_scale[kk];
+        const int s = s_scale[k];
         const uint16_t *tab = s_cdf + s * N_SYM;
         const uint32_t slot = x & 0xFFFFu;
         const int b = (int)(slot >> (16 - LUT_BITS));
@@ -430,30 +392,141 @@ __global__ void __launch_bounds__(RANS_WARPS * 32) rans_decode_kernel(RansDecArg
         const uint32_t f = cdf_at(tab, lo + 1) - c;
         x = f * (x >> 16) + slot - c;
         need = x < RANS_L;
-        if (lo == ESC_SYM) is_esc = true;
-        else q = lo - R_MAX + cen;
+        out[i] = (uint16_t)slot;
       }
       const uint32_t m = __ballot_sync(0xffffffffu, need);
-      const int rank = __popc(m & lt_mask);
-      const int p = (int)(wp - wb) + rank;  // position in the window, < 64 by construction
+      const uint32_t p = (wp - wb) + __popc(m & lt_mask);  // < 64 by construction
       const uint32_t v0 = __shfl_sync(0xffffffffu, w0, p & 31);
       const uint32_t v1 = __shfl_sync(0xffffffffu, w1, p & 31);
-      if (need) {
-        if (wp + rank < n_wd) x = (x << 16) | (p < 32 ? v0 : v1);
-        else bad = true;
-      }
+      if (need) x = (x << 16) | (p < 32 ? v0 : v1);
       wp += __popc(m);
-      if (wp - wb >= 32) {  // slide the window by 32 words
+      if (wp - wb >= 32) {  // slide the ring by 32 words
         w0 = w1;
+        w1 = w2;
         wb += 32;
-        w1 = wb + 32 + lane < n_wd ? wd[wb + 32 + lane] : 0u;
+        w2 = wb + 64 + lane < n_wd ? wd[wb + 64 + lane] : 0u;
       }
+      k += 32;
+      if (K > 0)
+        while (k >= K) k -= K;
+    }
+    bad = __any_sync(0xffffffffu, bad || wp > n_wd);
+  }
+  // the stream must be consumed exactly: every state back at L, at most one zero pad
+  // word left (escape values are checked by the finishing kernel)
+  if (!bad) {
+    if (x != RANS_L) bad = true;
+    if (!(wp == n_wd || (wp + 1 == n_wd && wd[n_wd - 1] == 0))) bad = true;
+  }
+  if (__any_sync(0xffffffffu, bad) && lane == 0) atomicExch(a.status, DCKV_ECORRUPT);
+}
+
+// Finishing a decoded pass, parallel over rows.  Step 1 (one block per row): symbol from
+// (scale, slot) through the lookup table, written back over the slot; escapes counted per
+// row.  Step 2 (one warp per row): the row's first escape index is the escape count of
+// the chunk's earlier rows; escapes are matched in symbol order to the chunk's 64-bit
+// values; q = symbol - 254 + centre is written as fp16 (exact below 2048) for the inverse
+// GEMM, bf16(q) into padded even rows for the odd mean model, and exact int32 values of
+// codes with |q| >= 2048 (their rows are listed for a fix-up).
+__global__ void __launch_bounds__(256) k_decode_symbols(int64_t slot0, int64_t n_slots, int k_eff,
+                                                        const uint8_t *kept_scale, const uint16_t *cdf,
+                                                        const uint16_t *lut, uint16_t *slots, uint32_t *row_esc,
+                                                        const int32_t *valid) {
+  extern __shared__ __align__(16) uint8_t sm[];
+  uint16_t *s_cdf = reinterpret_cast<uint16_t *>(sm);
+  uint16_t *s_lut = reinterpret_cast<uint16_t *>(sm + CDF_SMEM_BYTES);
+  __shared__ uint32_t cnt;
+  if (*valid != 1) return;
+  copy_smem16(s_cdf, cdf, CDF_SMEM_BYTES);
+  copy_smem16(s_lut, lut, LUT_SMEM_BYTES);
+  __syncthreads();
+  for (int64_t r = blockIdx.x; r < n_slots; r += gridDim.x) {
+    if (threadIdx.x == 0) cnt = 0;
+    __syncthreads();
+    uint16_t *sl = slots + (slot0 + r) * k_eff;
+    uint32_t esc = 0;
+    for (int k = threadIdx.x; k < k_eff; k += blockDim.x) {
+      const int s = kept_scale[k];
+      const uint16_t *tab = s_cdf + s * N_SYM;
+      const uint32_t slot = sl[k];
+      const int b = (int)(slot >> (16 - LUT_BITS));
+      int lo = s_lut[s * LUT_SIZE + b];
+      int hi = b + 1 < LUT_SIZE ? s_lut[s * LUT_SIZE + b + 1] : N_SYM - 1;
+      while (hi > lo) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (tab[mid] <= slot) lo = mid; else hi = mid - 1;
+      }
+      sl[k] = (uint16_t)lo;
+      esc += (lo == ESC_SYM);
+    }
+    for (int o = 16; o; o >>= 1) esc += __shfl_xor_sync(0xffffffffu, esc, o);
+    if ((threadIdx.x & 31) == 0 && esc) atomicAdd(&cnt, esc);
+    __syncthreads();
+    if (threadIdx.x == 0) row_esc[slot0 + r] = cnt;
+    __syncthreads();
+  }
+}
+
+struct DecCodesArgs {
+  const ChunkDesc *chunks;
+  const PromptInfo *prompts;
+  int chunk0, n_chunks;
+  int chunk_rows;
+  int k_eff;
+  const int16_t *kept_list;
+  const int8_t *cen8;
+  const uint16_t *syms;     // slot order
+  const uint32_t *row_esc;  // per slot row
+  const uint8_t *blob;
+  uint64_t off_streams;
+  const uint32_t *offs;
+  __half *q16;
+  __nv_bfloat16 *qe;
+  int32_t *qbig;
+  uint32_t *bigflag;
+  int32_t *biglist;
+  uint32_t *bigcount;
+  const int32_t *valid;
+  int32_t *status;
+};
+
+__global__ void __launch_bounds__(256) k_decode_codes(DecCodesArgs a) {
+  if (*a.valid != 1) return;
+  const int lane = threadIdx.x & 31;
+  const int nw = blockDim.x >> 5;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  const int total_rows = a.n_chunks * a.chunk_rows;  // rows of the pass, chunk-major (some absent)
+  for (int wr = blockIdx.x * nw + (threadIdx.x >> 5); wr < total_rows; wr += gridDim.x * nw) {
+    const int ci = a.chunk0 + wr / a.chunk_rows;
+    const int rl = wr % a.chunk_rows;
+    const ChunkDesc cd = a.chunks[ci];
+    if (rl >= cd.nrows) continue;
+    const PromptInfo pi = a.prompts[cd.prompt];
+    const int K = a.k_eff;
+    const int64_t slot_row = cd.sym_base / (K > 0 ? K : 1) + rl;
+    const uint8_t *sec = a.blob + a.off_streams + a.offs[ci];
+    const uint32_t ne = reinterpret_cast<const uint32_t *>(sec)[32];
+    const uint32_t *ev = reinterpret_cast<const uint32_t *>(sec + CHUNK_FIXED_BYTES);
+    uint32_t ep = 0;
+    for (int r = 0; r < rl; ++r) ep += a.row_esc[slot_row - rl + r];
+    const uint16_t *sy = a.syms + slot_row * K;
+    const int8_t *ce = a.cen8 + slot_row * K;
+    const int j = cd.j0 + rl;
+    const int64_t row = (int64_t)pi.row_base + 2 * j + cd.parity;
+    __half *q16 = a.q16 + row * N_COEF;
+    __nv_bfloat16 *qe = cd.parity == 0 ? a.qe + (int64_t)(pi.ebase + j) * N_COEF : nullptr;
+    bool bad = false;
+    for (int k0 = 0; k0 < K; k0 += 32) {
+      const int k = k0 + lane;
+      const bool valid = k < K;
+      const int sym = valid ? sy[k] : 0;
+      const bool is_esc = valid && sym == ESC_SYM;
       const uint32_t me = __ballot_sync(0xffffffffu, is_esc);
+      int q = valid ? sym - R_MAX + ce[k] : 0;
       if (is_esc) {
         const uint32_t e = ep + __popc(me & lt_mask);
         if (e < ne) {
-          const uint64_t v = (uint64_t)ev[2 * e] | ((uint64_t)ev[2 * e + 1] << 32);
-          const int64_t sv = (int64_t)v;
+          const int64_t sv = (int64_t)((uint64_t)ev[2 * e] | ((uint64_t)ev[2 * e + 1] << 32));
           q = (int)max(min(sv, (int64_t)INT32_MAX), (int64_t)INT32_MIN);
           if (sv >= -ESC_LIMIT && sv <= ESC_LIMIT) bad = true;  // not an escape value
         } else {
@@ -461,35 +534,20 @@ __global__ void __launch_bounds__(RANS_WARPS * 32) rans_decode_kernel(RansDecArg
         }
       }
       ep += __popc(me);
-      bad = __any_sync(0xffffffffu, bad);
-      if (valid && !bad) {
-        const int j = cd.j0 + rr;
-        const int64_t row = (int64_t)pi.row_base + 2 * j + cd.parity;
-        a.q16[row * N_COEF + comp] = __float2half_rn((float)q);
-        if (cd.parity == 0) a.qe[(int64_t)(pi.ebase + j) * N_COEF + comp] = __float2bfloat16_rn((float)q);
+      if (valid) {
+        const int comp = a.kept_list[k];
+        q16[comp] = __float2half_rn((float)q);
+        if (qe) qe[comp] = __float2bfloat16_rn((float)q);
         if (q >= BIG_CODE || q <= -BIG_CODE) {
           a.qbig[row * N_COEF + comp] = q;
           if (atomicExch(&a.bigflag[row], 1u) == 0u) a.biglist[atomicAdd(a.bigcount, 1u)] = (int32_t)row;
         }
       }
-      if (K > 0) {
-        k += 32;
-        while (k >= K) {
-          k -= K;
-          ++rl;
-        }
-      }
     }
-    if (bad) break;
+    // the chunk's last row checks that every escape value was used
+    if (rl == cd.nrows - 1 && ep != ne) bad = true;
+    if (__any_sync(0xffffffffu, bad) && lane == 0) atomicExch(a.status, DCKV_ECORRUPT);
   }
-  // the stream must be consumed exactly: every state back at L, all escapes used, at
-  // most one zero pad word left
-  if (!bad) {
-    if (x != RANS_L) bad = true;
-    if (ep != ne) bad = true;
-    if (!(wp == n_wd || (wp == n_wd - 1 && wd[n_wd - 1] == 0))) bad = true;
-  }
-  if (__any_sync(0xffffffffu, bad) && lane == 0) atomicExch(a.status, DCKV_ECORRUPT);
 }
 
 }  // namespace dckv
