@@ -715,7 +715,7 @@ static WsPlan plan_ws(const Layout &L, int which /*0 encode, 1 decode*/) {
     w.g16 = take(2ull * L.n_rows * 2 * N_HIDDEN);
     w.q32 = take(4ull * L.n_rows * N_COEF);
     w.sym16 = take(2ull * L.n_symbols);
-    w.cf32 = take(4ull * L.n_symbols);
+    w.cf32 = take(8ull * L.n_symbols);
     w.words = take(2ull * L.n_symbols);
     w.states = take(128ull * L.n_chunks);
     w.nwords = take(4ull * L.n_chunks);
@@ -728,7 +728,6 @@ static WsPlan plan_ws(const Layout &L, int which /*0 encode, 1 decode*/) {
     w.full_list = take(4ull * L.n_rows);
   } else {
     w.slots16 = take(2ull * L.n_symbols);
-    w.row_esc = take(4ull * L.n_rows);
     w.q16 = take(2ull * L.n_rows * N_COEF);
     w.qbig = take(4ull * L.n_rows * N_COEF);
     w.bigflag = take(4ull * L.n_rows);
@@ -801,6 +800,9 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
   const uint64_t o_ks = take(N_COEF);
   const uint64_t o_cdf = take(2ull * N_SCALES * N_SYM);
   const uint64_t o_lut = take(2ull * N_SCALES * LUT_SIZE);
+  const uint64_t o_tail = take(4ull * N_SCALES);
+  const uint64_t o_dcdf = take(2ull * N_SCALES * DEC_CDF_STRIDE);
+  const uint64_t o_rcp = take(4ull * N_SCALES * N_SYM);
   const uint64_t o_kidx = take(2ull * N_COEF);
   const uint64_t o_theta = take(8ull * 128);
   const uint64_t o_bt32 = take(4ull * N_COEF * ROW_DIM);
@@ -828,6 +830,9 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
   c->kept_scale = B + o_ks;
   c->cdf = (uint16_t *)(B + o_cdf);
   c->lut = (uint16_t *)(B + o_lut);
+  c->tail = (uint32_t *)(B + o_tail);
+  c->dcdf = (uint16_t *)(B + o_dcdf);
+  c->rcp = (uint32_t *)(B + o_rcp);
   c->kidx = (int16_t *)(B + o_kidx);
   c->theta = (double *)(B + o_theta);
   c->bt32 = (float *)(B + o_bt32);
@@ -843,7 +848,7 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
   // drop mask, scale index, tables
   k_scale_keep<<<(N_COEF + 255) / 256, 256, 0, st>>>(prm->laplace_b, prm->delta, c->scale, c->keep, scr);
   k_tables<<<N_SCALES, 512, 0, st>>>(c->cdf);
-  k_build_lut<<<N_SCALES, 256, 0, st>>>(c->cdf, c->lut);
+  k_build_lut<<<N_SCALES, 256, 0, st>>>(c->cdf, c->dcdf, c->lut, c->tail, c->rcp);
   cudaMemcpyAsync(c->delta, prm->delta, 4ull * N_COEF, cudaMemcpyDeviceToDevice, st);
   // scale exponents: largest |value| of each split operand brought to about 2^12
   k_absmax<<<256, 256, 0, st>>>(prm->basis, (int64_t)ROW_DIM * N_COEF, N_COEF, nullptr, scr + 1);
@@ -1034,7 +1039,7 @@ extern "C" int dckv_encode(const dckv_codec *c, const void *rows, const int32_t 
   int32_t *row_slot = (int32_t *)(ws + w.row_slot), *e_slot = (int32_t *)(ws + w.e_slot);
   int8_t *cen8 = (int8_t *)(ws + w.cen8);
   uint16_t *sym16 = (uint16_t *)(ws + w.sym16);
-  uint32_t *cf32 = (uint32_t *)(ws + w.cf32);
+  uint2 *cfm = (uint2 *)(ws + w.cf32);
   int32_t *slot_chunk = (int32_t *)(ws + w.slot_chunk);
   uint32_t *nesc_w = (uint32_t *)(ws + w.nesc);
 
@@ -1106,14 +1111,14 @@ extern "C" int dckv_encode(const dckv_codec *c, const void *rows, const int32_t 
     k_centres_even<<<rg, 256, 0, st>>>(L.n_rows, row_slot, row_edst, row_tok, token_ids, c->t_even, c->vocab,
                                        c->kept_list, c->k_eff, cen8, nullptr);
     k_symbols<<<rg, 256, 0, st>>>(L.n_rows, row_slot, slot_chunk, q32, cen8, c->kept_list, c->kept_scale, c->cdf,
-                                  c->k_eff, sym16, cf32, nesc_w);
+                                  c->rcp, c->k_eff, sym16, cfm, nesc_w);
     CK(cudaGetLastError());
     stage_mark(c, st, "symbols");
   }
   uint32_t *states = (uint32_t *)(ws + w.states), *nwords = (uint32_t *)(ws + w.nwords);
   uint32_t *nesc = (uint32_t *)(ws + w.nesc), *offs = (uint32_t *)(ws + w.offs);
   if (L.n_chunks > 0) {
-    RansEncArgs a{d_chunks, L.n_chunks, c->k_eff, cf32, (uint16_t *)(ws + w.words), states, nwords};
+    RansEncArgs a{d_chunks, L.n_chunks, c->k_eff, cfm, (uint16_t *)(ws + w.words), states, nwords};
     rans_encode_kernel<<<(L.n_chunks + RANS_WARPS - 1) / RANS_WARPS, RANS_WARPS * 32, 0, st>>>(a);
     CK(cudaGetLastError());
   }
@@ -1160,8 +1165,7 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
   int32_t *row_slot = (int32_t *)(ws + w.row_slot), *e_slot = (int32_t *)(ws + w.e_slot);
   int8_t *cen8 = (int8_t *)(ws + w.cen8);
   int32_t *slot_chunk = (int32_t *)(ws + w.slot_chunk);
-  uint16_t *slots16 = (uint16_t *)(ws + w.slots16);
-  uint32_t *row_esc = (uint32_t *)(ws + w.row_esc);
+  uint16_t *syms16 = (uint16_t *)(ws + w.slots16);
   __half *q16 = (__half *)(ws + w.q16);
   int32_t *qbig = (int32_t *)(ws + w.qbig);
   uint32_t *bigflag = (uint32_t *)(ws + w.bigflag);
@@ -1189,24 +1193,25 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
   if (L.n_rows > 0)
     k_centres_even<<<(unsigned)std::min<int64_t>(L.n_rows, 65535), 256, 0, st>>>(
         L.n_rows, row_slot, row_edst, row_tok, token_ids, c->t_even, c->vocab, c->kept_list, c->k_eff, cen8, valid);
-  CK(cudaFuncSetAttribute(rans_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, RANS_DEC_SMEM));
-  CK(cudaFuncSetAttribute(k_decode_symbols, cudaFuncAttributeMaxDynamicSharedMemorySize, DEC_FINISH_SMEM));
-  RansDecArgs da{d_chunks, 0, L.n_chunks_e, c->k_eff, c->kept_scale, c->cdf, c->lut, bl, L.off_streams, offs,
-                 slots16, valid, status_dev};
-  DecCodesArgs fa{d_chunks, d_prompts, 0, L.n_chunks_e, c->chunk_rows, c->k_eff, c->kept_list, cen8, slots16,
-                  row_esc, bl, L.off_streams, offs, q16, qe, qbig, bigflag, biglist, counters, valid, status_dev};
-  int64_t ne_rows = 0;
-  for (const PromptInfo &p : L.prompts) ne_rows += p.n_e;
-  const unsigned sym_blocks = (unsigned)std::max<int64_t>(1, std::min<int64_t>(L.n_rows, 4 * c->num_sms));
-  if (L.n_chunks_e > 0) {
-    rans_decode_kernel<<<(L.n_chunks_e + RANS_WARPS - 1) / RANS_WARPS, RANS_WARPS * 32, RANS_DEC_SMEM, st>>>(da);
-    stage_mark(c, st, "rans_even_loop");
-    k_decode_symbols<<<sym_blocks, 256, DEC_FINISH_SMEM, st>>>(0, ne_rows, c->k_eff, c->kept_scale, c->cdf, c->lut,
-                                                              slots16, row_esc, valid);
-    k_decode_codes<<<(unsigned)((L.n_chunks_e * c->chunk_rows + 7) / 8), 256, 0, st>>>(fa);
-    CK(cudaGetLastError());
+  CK(cudaFuncSetAttribute(rans_decode_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, RANS_DEC_SMEM));
+  CK(cudaFuncSetAttribute(rans_decode_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, RANS_DEC_SMEM));
+  RansDecArgs da{d_chunks, 0, L.n_chunks, c->k_eff, c->kept_scale, c->dcdf, c->lut, c->tail, bl, L.off_streams,
+                 offs, syms16, valid, status_dev};
+  DecCodesArgs fa{d_chunks, d_prompts, 0, L.n_chunks_e, c->k_eff, c->kept_list, cen8, syms16, bl, L.off_streams,
+                  offs, q16, qe, qbig, bigflag, biglist, counters, valid, status_dev};
+  if (L.n_chunks > 0) {
+    const unsigned g = (L.n_chunks + RANS_WARPS - 1) / RANS_WARPS;
+    if (c->k_eff >= 32)
+      rans_decode_kernel<true><<<g, RANS_WARPS * 32, RANS_DEC_SMEM, st>>>(da);
+    else
+      rans_decode_kernel<false><<<g, RANS_WARPS * 32, RANS_DEC_SMEM, st>>>(da);
   }
-  stage_mark(c, st, "rans_even");
+  CK(cudaGetLastError());
+  stage_mark(c, st, "rans_loop");
+  if (L.n_chunks_e > 0)
+    k_decode_codes<<<(unsigned)L.n_chunks_e, DEC_CODES_THREADS, 0, st>>>(fa);
+  CK(cudaGetLastError());
+  stage_mark(c, st, "codes_even");
   if (L.n_rows > 0) {
     CUtensorMap mb_qe;
     RET(map_b(&mb_qe, qe, true, N_COEF, L.ne_pad, 256));
@@ -1218,18 +1223,12 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
   }
   stage_mark(c, st, "gemm_mean_odd");
   if (L.n_chunks_o > 0) {
-    da.chunk0 = L.n_chunks_e;
-    da.n_chunks = L.n_chunks_o;
     fa.chunk0 = L.n_chunks_e;
     fa.n_chunks = L.n_chunks_o;
-    rans_decode_kernel<<<(L.n_chunks_o + RANS_WARPS - 1) / RANS_WARPS, RANS_WARPS * 32, RANS_DEC_SMEM, st>>>(da);
-    stage_mark(c, st, "rans_odd_loop");
-    k_decode_symbols<<<sym_blocks, 256, DEC_FINISH_SMEM, st>>>(ne_rows, L.n_rows - ne_rows, c->k_eff, c->kept_scale,
-                                                              c->cdf, c->lut, slots16, row_esc, valid);
-    k_decode_codes<<<(unsigned)((L.n_chunks_o * c->chunk_rows + 7) / 8), 256, 0, st>>>(fa);
+    k_decode_codes<<<(unsigned)L.n_chunks_o, DEC_CODES_THREADS, 0, st>>>(fa);
     CK(cudaGetLastError());
   }
-  stage_mark(c, st, "rans_odd");
+  stage_mark(c, st, "codes_odd");
   if (L.n_rows > 0) {
     CUtensorMap mb_q;
     RET(map_b(&mb_q, q16, false, N_COEF, L.n_rows, 256));

@@ -78,7 +78,7 @@ struct WsPlan {
   size_t prompts, chunks, row_tok, row_pos, row_edst, e_tok, row_slot, e_slot, slot_chunk;  // tables
   size_t qe, cen8;                                                               // both
   size_t x16, g16, q32, sym16, cf32, words, states, nwords, nesc, offs;           // encode
-  size_t slots16, row_esc;                                                        // decode
+  size_t slots16;  // decode: decoded symbols (slot order)
   size_t row_norm, rowflag, el_list, full_list;                         // encode refinement
   int64_t el_cap;
   size_t q16, qbig, bigflag, biglist, counters, valid;                  // decode
@@ -115,6 +115,9 @@ struct dckv_codec {
   uint8_t *kept_scale = nullptr;  // [2048]
   uint16_t *cdf = nullptr;   // [64][510]  cumulative frequencies (cdf[510] = 65536 implied)
   uint16_t *lut = nullptr;   // [64][1024] decoder lookup (symbol holding slot b * 64)
+  uint32_t *tail = nullptr;  // [64] lengths of the frequency-1 runs at both ends
+  uint16_t *dcdf = nullptr;  // [64][512] cdf, padded with two zero entries (decoder)
+  uint32_t *rcp = nullptr;   // [64][510] division multiplier of each frequency (encoder)
   int16_t *kidx = nullptr;   // [2048] kept index of a component, -1 if dropped
   double model_bits_per_row = 0.0;  // entropy of the kept components' tables
   float *dbg_ratio = nullptr;       // optional [rows][2048] export of the fp32 ratios y / Delta

@@ -21,12 +21,17 @@ namespace dckv {
 
 constexpr int RANS_WARPS = 4;                            // chunks per block
 constexpr int PF = 16;                                   // steps of look-ahead for state-free data
-constexpr int CDF_SMEM_BYTES = N_SCALES * N_SYM * 2;     // 65,280
+constexpr int DEC_CDF_STRIDE = 512;                     // decoder cdf rows: 510 entries, then 0, 0
+constexpr int CDF_SMEM_BYTES = N_SCALES * DEC_CDF_STRIDE * 2;  // 65,536
 constexpr int LUT_BITS = 10;                             // decoder lookup on slot >> 6
 constexpr int LUT_SIZE = 1 << LUT_BITS;
 constexpr int LUT_SMEM_BYTES = N_SCALES * LUT_SIZE * 2;  // 131,072
-constexpr int RANS_DEC_SMEM = CDF_SMEM_BYTES + LUT_SMEM_BYTES + N_COEF;
-constexpr int DEC_FINISH_SMEM = CDF_SMEM_BYTES + LUT_SMEM_BYTES;
+constexpr int TAIL_SMEM_BYTES = N_SCALES * 4;
+constexpr int RANS_DEC_SMEM = CDF_SMEM_BYTES + LUT_SMEM_BYTES + TAIL_SMEM_BYTES + N_COEF;
+constexpr uint32_t CF_INVALID = 0xFFFFFFFFu;  // no table entry has cdf 65535 and freq 65536
+constexpr uint16_t LUT_SINGLE = 0x4000;       // the bucket lies inside one symbol's range
+constexpr uint16_t LUT_MULTI = 0x8000;        // two or more symbol boundaries in the bucket
+constexpr uint16_t LUT_SYM = 0x03FF;
 
 __device__ __forceinline__ void copy_smem16(void *dst, const void *src, int bytes) {
   const uint4 *s = reinterpret_cast<const uint4 *>(src);
@@ -58,11 +63,12 @@ __global__ void __launch_bounds__(256) k_centres_even(int64_t n_rows, const int3
 }
 
 // Encoder inputs in slot order: the symbol (ESC if |q| > 127 else q - centre + 254), its
-// table entry packed as cdf | (freq - 1) << 16, and the escape count of each chunk.
+// table entry {cdf | (freq - 1) << 16, division multiplier of freq}, and the escape count
+// of each chunk.
 __global__ void __launch_bounds__(256) k_symbols(int64_t n_rows, const int32_t *row_slot, const int32_t *slot_chunk,
                                                  const int32_t *q32, const int8_t *cen8, const int16_t *kept_list,
-                                                 const uint8_t *kept_scale, const uint16_t *cdf, int k_eff,
-                                                 uint16_t *sym16, uint32_t *cf32, uint32_t *nesc) {
+                                                 const uint8_t *kept_scale, const uint16_t *cdf, const uint32_t *rcp,
+                                                 int k_eff, uint16_t *sym16, uint2 *cfm, uint32_t *nesc) {
   __shared__ int esc_count;
   for (int64_t row = blockIdx.x; row < n_rows; row += gridDim.x) {
     if (threadIdx.x == 0) esc_count = 0;
@@ -76,11 +82,11 @@ __global__ void __launch_bounds__(256) k_symbols(int64_t n_rows, const int32_t *
       const bool is_esc = v > ESC_LIMIT || v < -ESC_LIMIT;
       const int sym = is_esc ? ESC_SYM : v - cen8[base + k] + R_MAX;
       esc += is_esc;
-      const uint16_t *tab = cdf + kept_scale[k] * N_SYM;
-      const uint32_t c = tab[sym];
-      const uint32_t f = cdf_at(tab, sym + 1) - c;
+      const int ti = kept_scale[k] * N_SYM + sym;
+      const uint32_t c = cdf[ti];
+      const uint32_t f = cdf_at(cdf + (ti - sym), sym + 1) - c;
       sym16[base + k] = (uint16_t)sym;
-      cf32[base + k] = c | ((f - 1u) << 16);
+      cfm[base + k] = make_uint2(c | ((f - 1u) << 16), rcp[ti]);
     }
     if (esc) atomicAdd(&esc_count, esc);
     __syncthreads();
@@ -90,14 +96,32 @@ __global__ void __launch_bounds__(256) k_symbols(int64_t n_rows, const int32_t *
 }
 
 // ------------------------------------------------------------------------------ encode
+// Division of the state by a symbol's frequency f uses the multiplier of Granlund and
+// Montgomery, "Division by invariant integers using multiplication" (1994), unsigned
+// case: with l = ceil(log2 f) and m = floor(2^32 (2^l - f) / f) + 1, every 32-bit x has
+// floor(x / f) = (t + ((x - t) >> 1)) >> (l - 1), t = high word of m x.  f = 1 is x itself.
+__host__ __device__ inline uint32_t div_multiplier(uint32_t f) {
+  if (f < 2) return 0;
+  uint32_t l = 0;
+  while ((1u << l) < f) ++l;
+  return (uint32_t)((((uint64_t)1 << 32) * (((uint64_t)1 << l) - f)) / f + 1);
+}
+
+// 16-bit store under a predicate, without a branch.
+__device__ __forceinline__ void st_u16_if(uint16_t *p, uint32_t v, bool pred) {
+  asm volatile("{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %2, 0;\n\t@q st.global.u16 [%0], %1;\n\t}" ::"l"(p),
+               "h"((unsigned short)(v & 0xFFFFu)), "r"((int)pred)
+               : "memory");
+}
+
 struct RansEncArgs {
   const ChunkDesc *chunks;
   int n_chunks;
   int k_eff;
-  const uint32_t *cf32;  // slot order: cdf | (freq - 1) << 16
-  uint16_t *words;       // word scratch: chunk c owns [sym_base, sym_base + S)
-  uint32_t *states;      // [chunks][32]
-  uint32_t *nwords;      // [chunks] words emitted
+  const uint2 *cfm;    // slot order: {cdf | (freq - 1) << 16, division multiplier}
+  uint16_t *words;     // word scratch: chunk c owns [sym_base, sym_base + S)
+  uint32_t *states;    // [chunks][32]
+  uint32_t *nwords;    // [chunks] words emitted
 };
 
 __global__ void __launch_bounds__(RANS_WARPS * 32) rans_encode_kernel(RansEncArgs a) {
@@ -107,44 +131,47 @@ __global__ void __launch_bounds__(RANS_WARPS * 32) rans_encode_kernel(RansEncArg
   const ChunkDesc cd = a.chunks[ci];
   const uint32_t S = (uint32_t)cd.nrows * (uint32_t)a.k_eff;  // < 2^20
   const int T = (int)((S + 31) / 32);
-  const uint32_t *cfs = a.cf32 + cd.sym_base;
+  const uint2 *cfs = a.cfm + cd.sym_base;
   uint16_t *wslot = a.words + cd.sym_base;
   uint32_t pos = S;  // words are placed downwards from the end of the slot
   uint32_t x = RANS_L;
   const uint32_t lt_mask = (1u << lane) - 1u;
-  // table entries are fetched PF steps ahead through a register ring (independent of x)
-  uint32_t ring[PF];
+  // steps run in groups of 16 from t = T-1 down; the next group's table entries are
+  // loaded while the current group is coded (they do not depend on the state)
+  uint2 cur[16], nxt[16];
 #pragma unroll
-  for (int u = 0; u < PF; ++u) {
+  for (int u = 0; u < 16; ++u) {
     const int t = T - 1 - u;
-    const uint32_t iu = (uint32_t)t * 32u + lane;
-    ring[u] = (t >= 0 && iu < S) ? cfs[iu] : 0u;
+    const uint32_t i = (uint32_t)t * 32u + lane;
+    cur[u] = (t >= 0 && i < S) ? cfs[i] : make_uint2(CF_INVALID, 0u);
   }
-  for (int t0 = T - 1; t0 >= 0; t0 -= PF) {
+  for (int t0 = T - 1; t0 >= 0; t0 -= 16) {
 #pragma unroll
-    for (int u = 0; u < PF; ++u) {
-      const int t = t0 - u;
-      if (t < 0) break;
+    for (int u = 0; u < 16; ++u) {
+      const int t = t0 - 16 - u;
       const uint32_t i = (uint32_t)t * 32u + lane;
-      const bool valid = i < S;
-      const uint32_t cf = ring[u];
-      const int tn = t - PF;
-      const uint32_t in = (uint32_t)tn * 32u + lane;
-      ring[u] = (tn >= 0 && in < S) ? cfs[in] : 0u;
+      nxt[u] = (t >= 0 && i < S) ? cfs[i] : make_uint2(CF_INVALID, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const uint32_t cf = cur[u].x;
+      const bool valid = cf != CF_INVALID;
       const uint32_t c = cf & 0xFFFFu;
       const uint32_t f = valid ? (cf >> 16) + 1u : 1u;
       const bool emit = valid && x >= (f << 16);
       const uint32_t m = __ballot_sync(0xffffffffu, emit);
-      if (emit) {
-        wslot[pos - __popc(m) + __popc(m & lt_mask)] = (uint16_t)(x & 0xFFFFu);
-        x >>= 16;
-      }
-      pos -= __popc(m);
-      if (valid) {
-        const uint32_t qf = x / f;
-        x = (qf << 16) + (x - qf * f) + c;
-      }
+      const uint32_t nm = __popc(m);
+      st_u16_if(wslot + (pos - nm + __popc(m & lt_mask)), x, emit);
+      pos -= nm;
+      const uint32_t xr = emit ? x >> 16 : x;
+      const uint32_t th = __umulhi(cur[u].y, xr);
+      const int sh = max(31 - __clz((int)(f - 1u)), 0);
+      const uint32_t qf = f == 1u ? xr : (th + ((xr - th) >> 1)) >> sh;
+      const uint32_t xn = xr + c + qf * (PREC_TOTAL - f);  // = (qf << 16) + xr mod f + c
+      x = valid ? xn : x;
     }
+#pragma unroll
+    for (int u = 0; u < 16; ++u) cur[u] = nxt[u];
   }
   a.states[(int64_t)ci * 32 + lane] = x;
   if (lane == 0) a.nwords[ci] = S - pos;
@@ -297,47 +324,167 @@ __global__ void __launch_bounds__(RANS_WARPS * 32) compact_kernel(CompactArgs a)
 }
 
 // ------------------------------------------------------------------------------ decode
-// Decoder lookup: lut[s][b] = the symbol whose slot range holds slot b * 64.
-__global__ void k_build_lut(const uint16_t *cdf, uint16_t *lut) {
+// Decoder tables, per scale s:
+//   dcdf[s][0..509] = cdf, dcdf[s][510] = dcdf[s][511] = 0 (65536 mod 2^16, so that
+//     freq = (dcdf[sym + 1] - dcdf[sym]) mod 2^16 for every symbol);
+//   lut[s][b] for the 64 slots b * 64 .. b * 64 + 63: bits 0-9 the symbol holding the
+//     first of them, LUT_SINGLE if one symbol holds all of them, LUT_MULTI if two or more
+//     symbol ranges start inside the bucket (else exactly one does);
+//   tail[s] = length of the leading run of frequency-1 symbols (cdf[sym] = sym) in bits
+//     0-15 and length n of the trailing run (cdf[sym] = 65536 - 510 + sym, ESC last;
+//     slots 65536 - n .. 65535) in bits 16-31; slots in a run decode by arithmetic;
+//   rcp[s][sym] = division multiplier of the symbol's frequency (encoder).
+__global__ void k_build_lut(const uint16_t *cdf, uint16_t *dcdf, uint16_t *lut, uint32_t *tail, uint32_t *rcp) {
   const int s = blockIdx.x;
   const uint16_t *tab = cdf + s * N_SYM;
-  for (int b = threadIdx.x; b < LUT_SIZE; b += blockDim.x) {
-    const uint32_t slot = (uint32_t)b << (16 - LUT_BITS);
+  auto holder = [&](uint32_t slot) {
     int lo = 0, hi = N_SYM;
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;
       if (tab[mid] <= slot) lo = mid; else hi = mid;
     }
-    lut[s * LUT_SIZE + b] = (uint16_t)lo;
+    return lo;
+  };
+  for (int b = threadIdx.x; b < LUT_SIZE; b += blockDim.x) {
+    const uint32_t slot = (uint32_t)b << (16 - LUT_BITS);
+    const int lo = holder(slot);
+    const int hi = holder(slot + (1u << (16 - LUT_BITS)) - 1u);
+    lut[s * LUT_SIZE + b] = (uint16_t)(lo | (hi == lo ? LUT_SINGLE : 0) | (hi >= lo + 2 ? LUT_MULTI : 0));
+  }
+  for (int k = threadIdx.x; k < DEC_CDF_STRIDE; k += blockDim.x) {
+    dcdf[s * DEC_CDF_STRIDE + k] = k < N_SYM ? tab[k] : (uint16_t)0;
+    if (k < N_SYM) rcp[s * N_SYM + k] = div_multiplier(cdf_at(tab, k + 1) - tab[k]);
+  }
+  if (threadIdx.x == 0) {
+    int lead = 0;  // symbols 0 .. lead-1 have frequency 1
+    while (lead < N_SYM && cdf_at(tab, lead + 1) - tab[lead] == 1u) ++lead;
+    int trail = N_SYM;  // symbols trail .. 509 have frequency 1
+    while (trail > lead && cdf_at(tab, trail) - tab[trail - 1] == 1u) --trail;
+    tail[s] = (uint32_t)lead | ((uint32_t)(N_SYM - trail) << 16);
   }
 }
 
-// Decodes one pass (parity) of chunks, one warp per chunk.  The loop carries only the
-// rANS states: for each symbol it finds the table entry holding the state's slot, updates
-// the state, renormalises, and writes the slot (slot order) for the finishing kernel.
+// Symbol holding `slot` under scale s, with its cumulative frequency c and frequency f.
+// Buckets with at most one boundary resolve without branches; the rest (frequency-1 runs
+// at the tails, several boundaries) take the second path.
+__device__ __forceinline__ int find_symbol(uint32_t slot, int s, const uint16_t *s_cdf, const uint16_t *s_lut,
+                                           const uint32_t *s_tail, uint32_t &c, uint32_t &f) {
+  const uint16_t *tab = s_cdf + s * DEC_CDF_STRIDE;
+  const uint32_t b = slot >> (16 - LUT_BITS);
+  const uint32_t e = s_lut[s * LUT_SIZE + b];
+  int sym = (int)(e & LUT_SYM);
+  if (!(e & LUT_MULTI)) {
+    const uint32_t c0 = tab[sym], c1 = tab[sym + 1], c2 = tab[sym + 2];
+    const bool up = !(e & LUT_SINGLE) && slot >= c1;
+    sym += up;
+    c = up ? c1 : c0;
+    f = ((up ? c2 : c1) - c) & 0xFFFFu;
+    return sym;
+  }
+  const uint32_t tl = s_tail[s];
+  const uint32_t n_lead = tl & 0xFFFFu, n_trail = tl >> 16;
+  if (slot < n_lead) {
+    c = slot;
+    f = 1;
+    return (int)slot;
+  }
+  if (slot + n_trail >= PREC_TOTAL) {
+    c = slot;
+    f = 1;
+    return (int)(slot - (PREC_TOTAL - (uint32_t)N_SYM));
+  }
+  int hi = b + 1 < (uint32_t)LUT_SIZE ? (int)(s_lut[s * LUT_SIZE + b + 1] & LUT_SYM) : N_SYM - 1;  // in [sym, hi]
+  while (hi > sym) {
+    const int mid = (sym + hi + 1) >> 1;
+    if (tab[mid] <= slot) sym = mid; else hi = mid - 1;
+  }
+  c = tab[sym];
+  f = ((uint32_t)tab[sym + 1] - c) & 0xFFFFu;
+  return sym;
+}
+
 struct RansDecArgs {
   const ChunkDesc *chunks;
-  int chunk0, n_chunks;  // this pass: chunks [chunk0, chunk0 + n_chunks)
+  int chunk0, n_chunks;  // chunks [chunk0, chunk0 + n_chunks)
   int k_eff;
   const uint8_t *kept_scale;
-  const uint16_t *cdf;
+  const uint16_t *dcdf;
   const uint16_t *lut;
+  const uint32_t *tail;
   const uint8_t *blob;
   uint64_t off_streams;
   const uint32_t *offs;  // chunk table inside the blob
-  uint16_t *slots;       // slot order: the decoded slot of every symbol
+  uint16_t *syms;        // slot order: the decoded symbol of every position
   const int32_t *valid;  // header check result (1 = ok)
   int32_t *status;
 };
 
+__device__ __forceinline__ void load_tables(uint8_t *sm, const uint16_t *dcdf, const uint16_t *lut,
+                                            const uint32_t *tail) {
+  copy_smem16(sm, dcdf, CDF_SMEM_BYTES);
+  copy_smem16(sm + CDF_SMEM_BYTES, lut, LUT_SMEM_BYTES);
+  copy_smem16(sm + CDF_SMEM_BYTES + LUT_SMEM_BYTES, tail, TAIL_SMEM_BYTES);
+}
+
+// State of one warp decoding one chunk.
+struct DecLane {
+  uint32_t x;           // rANS state
+  uint32_t w0, w1, w2;  // word ring: lane j holds words wb + j, wb + 32 + j, wb + 64 + j
+  uint32_t wb, wp;      // ring base, words consumed
+  int k;                // kept component of this lane's next symbol
+};
+
+// One decode step of all 32 lanes: symbol i = 32 t + lane.  CHECK: some lanes may lie
+// beyond the chunk's last symbol.  BIG_K: K >= 32 (the component advances by at most one
+// wrap per step).
+template <bool CHECK, bool BIG_K>
+__device__ __forceinline__ void dec_step(DecLane &d, uint32_t i, uint32_t S, int K, uint32_t lt_mask,
+                                         const uint8_t *s_scale, const uint16_t *s_cdf, const uint16_t *s_lut,
+                                         const uint32_t *s_tail, const uint16_t *wd, uint32_t n_wd, uint16_t *out) {
+  const bool valid = !CHECK || i < S;
+  bool need = false;
+  if (valid) {
+    const uint32_t slot = d.x & 0xFFFFu;
+    uint32_t c, f;
+    const int sym = find_symbol(slot, s_scale[d.k], s_cdf, s_lut, s_tail, c, f);
+    d.x = f * (d.x >> 16) + slot - c;
+    need = d.x < RANS_L;
+    out[i] = (uint16_t)sym;
+  }
+  const uint32_t m = __ballot_sync(0xffffffffu, need);
+  const uint32_t p = (d.wp - d.wb) + __popc(m & lt_mask);  // < 64: wp - wb < 32 before the step
+  const uint32_t v0 = __shfl_sync(0xffffffffu, d.w0, p & 31);
+  const uint32_t v1 = __shfl_sync(0xffffffffu, d.w1, p & 31);
+  d.x = need ? (d.x << 16) | (p < 32 ? v0 : v1) : d.x;
+  d.wp += __popc(m);
+  if (d.wp - d.wb >= 32) {  // warp-uniform: slide the ring by 32 words
+    d.w0 = d.w1;
+    d.w1 = d.w2;
+    d.wb += 32;
+    const uint32_t wi = d.wb + 64 + __popc(lt_mask);  // lane index
+    d.w2 = wi < n_wd ? wd[wi] : 0u;
+  }
+  if (BIG_K) {
+    d.k += 32;
+    d.k = d.k >= K ? d.k - K : d.k;
+  } else {
+    d.k += 32;
+    while (d.k >= K) d.k -= K;
+  }
+}
+
+// The rANS arithmetic needs only the table (scale) of each component, never the code
+// means, so every chunk of both parities decodes in one launch; centres are applied
+// afterwards by the finishing kernel, pass by pass.
+template <bool BIG_K>
 __global__ void __launch_bounds__(RANS_WARPS * 32) rans_decode_kernel(RansDecArgs a) {
   extern __shared__ __align__(16) uint8_t sm[];
-  uint16_t *s_cdf = reinterpret_cast<uint16_t *>(sm);
-  uint16_t *s_lut = reinterpret_cast<uint16_t *>(sm + CDF_SMEM_BYTES);
-  uint8_t *s_scale = sm + CDF_SMEM_BYTES + LUT_SMEM_BYTES;
+  const uint16_t *s_cdf = reinterpret_cast<const uint16_t *>(sm);
+  const uint16_t *s_lut = reinterpret_cast<const uint16_t *>(sm + CDF_SMEM_BYTES);
+  const uint32_t *s_tail = reinterpret_cast<const uint32_t *>(sm + CDF_SMEM_BYTES + LUT_SMEM_BYTES);
+  uint8_t *s_scale = sm + CDF_SMEM_BYTES + LUT_SMEM_BYTES + TAIL_SMEM_BYTES;
   if (*a.valid != 1) return;
-  copy_smem16(s_cdf, a.cdf, CDF_SMEM_BYTES);
-  copy_smem16(s_lut, a.lut, LUT_SMEM_BYTES);
+  load_tables(sm, a.dcdf, a.lut, a.tail);
   copy_smem16(s_scale, a.kept_scale, N_COEF);
   __syncthreads();
   const int lane = threadIdx.x & 31;
@@ -348,6 +495,7 @@ __global__ void __launch_bounds__(RANS_WARPS * 32) rans_decode_kernel(RansDecArg
   const int K = a.k_eff;
   const uint32_t S = (uint32_t)cd.nrows * (uint32_t)K;  // < 2^20
   const int T = (int)((S + 31) / 32);
+  const int T_full = (int)(S / 32);  // steps where every lane holds a symbol
   const uint64_t beg = a.off_streams + a.offs[ci];
   const uint64_t end = a.off_streams + a.offs[ci + 1];
   const uint8_t *sec = a.blob + beg;
@@ -356,127 +504,53 @@ __global__ void __launch_bounds__(RANS_WARPS * 32) rans_decode_kernel(RansDecArg
     if (lane == 0) atomicExch(a.status, DCKV_ECORRUPT);
     return;
   }
-  uint32_t x = reinterpret_cast<const uint32_t *>(sec)[lane];
   const uint16_t *wd = reinterpret_cast<const uint16_t *>(sec + CHUNK_FIXED_BYTES + 8ull * ne);
   const uint32_t n_wd = (uint32_t)(((end - beg) - CHUNK_FIXED_BYTES - 8ull * ne) / 2);
-  uint16_t *out = a.slots + cd.sym_base;
-  // words pass through a 96-word register ring: lane j holds words wb + j, wb + 32 + j and
-  // (prefetched) wb + 64 + j
-  uint32_t wb = 0, wp = 0;
-  uint32_t w0 = lane < n_wd ? wd[lane] : 0u;
-  uint32_t w1 = 32 + lane < n_wd ? wd[32 + lane] : 0u;
-  uint32_t w2 = 64 + lane < n_wd ? wd[64 + lane] : 0u;
+  uint16_t *out = a.syms + cd.sym_base;
   const uint32_t lt_mask = (1u << lane) - 1u;
-  bool bad = x < RANS_L;
-  int k = K > 0 ? lane % K : 0;
-  for (int t0 = 0; t0 < T && !bad; t0 += 16) {
-#pragma unroll 4
-    for (int u = 0; u < 16; ++u) {
-      const int t = t0 + u;
-      if (t >= T) break;
-      const uint32_t i = (uint32_t)t * 32u + lane;
-      const bool valid = i < S;
-      bool need = false;
-      if (valid) {
-        const int s = s_scale[k];
-        const uint16_t *tab = s_cdf + s * N_SYM;
-        const uint32_t slot = x & 0xFFFFu;
-        const int b = (int)(slot >> (16 - LUT_BITS));
-        int lo = s_lut[s * LUT_SIZE + b];
-        int hi = b + 1 < LUT_SIZE ? s_lut[s * LUT_SIZE + b + 1] : N_SYM - 1;  // answer in [lo, hi]
-        while (hi > lo) {
-          const int mid = (lo + hi + 1) >> 1;
-          if (tab[mid] <= slot) lo = mid; else hi = mid - 1;
-        }
-        const uint32_t c = tab[lo];
-        const uint32_t f = cdf_at(tab, lo + 1) - c;
-        x = f * (x >> 16) + slot - c;
-        need = x < RANS_L;
-        out[i] = (uint16_t)slot;
-      }
-      const uint32_t m = __ballot_sync(0xffffffffu, need);
-      const uint32_t p = (wp - wb) + __popc(m & lt_mask);  // < 64 by construction
-      const uint32_t v0 = __shfl_sync(0xffffffffu, w0, p & 31);
-      const uint32_t v1 = __shfl_sync(0xffffffffu, w1, p & 31);
-      if (need) x = (x << 16) | (p < 32 ? v0 : v1);
-      wp += __popc(m);
-      if (wp - wb >= 32) {  // slide the ring by 32 words
-        w0 = w1;
-        w1 = w2;
-        wb += 32;
-        w2 = wb + 64 + lane < n_wd ? wd[wb + 64 + lane] : 0u;
-      }
-      k += 32;
-      if (K > 0)
-        while (k >= K) k -= K;
-    }
-    bad = __any_sync(0xffffffffu, bad || wp > n_wd);
+  DecLane d;
+  d.x = reinterpret_cast<const uint32_t *>(sec)[lane];
+  d.wb = 0;
+  d.wp = 0;
+  d.w0 = (uint32_t)lane < n_wd ? wd[lane] : 0u;
+  d.w1 = 32u + lane < n_wd ? wd[32 + lane] : 0u;
+  d.w2 = 64u + lane < n_wd ? wd[64 + lane] : 0u;
+  d.k = K > 0 ? lane % K : 0;
+  bool bad = d.x < RANS_L;
+  int t = 0;
+  for (; t + 16 <= T_full && !bad; t += 16) {
+#pragma unroll
+    for (int u = 0; u < 16; ++u)
+      dec_step<false, BIG_K>(d, (uint32_t)(t + u) * 32u + lane, S, K, lt_mask, s_scale, s_cdf, s_lut, s_tail, wd,
+                             n_wd, out);
+    bad = __any_sync(0xffffffffu, bad || d.wp > n_wd);
   }
+  for (; t < T && !bad; ++t)
+    dec_step<true, BIG_K>(d, (uint32_t)t * 32u + lane, S, K, lt_mask, s_scale, s_cdf, s_lut, s_tail, wd, n_wd, out);
+  bad = __any_sync(0xffffffffu, bad || d.wp > n_wd);
   // the stream must be consumed exactly: every state back at L, at most one zero pad
   // word left (escape values are checked by the finishing kernel)
   if (!bad) {
-    if (x != RANS_L) bad = true;
-    if (!(wp == n_wd || (wp + 1 == n_wd && wd[n_wd - 1] == 0))) bad = true;
+    if (d.x != RANS_L) bad = true;
+    if (!(d.wp == n_wd || (d.wp + 1 == n_wd && wd[n_wd - 1] == 0))) bad = true;
   }
   if (__any_sync(0xffffffffu, bad) && lane == 0) atomicExch(a.status, DCKV_ECORRUPT);
 }
 
-// Finishing a decoded pass, parallel over rows.  Step 1 (one block per row): symbol from
-// (scale, slot) through the lookup table, written back over the slot; escapes counted per
-// row.  Step 2 (one warp per row): the row's first escape index is the escape count of
-// the chunk's earlier rows; escapes are matched in symbol order to the chunk's 64-bit
-// values; q = symbol - 254 + centre is written as fp16 (exact below 2048) for the inverse
-// GEMM, bf16(q) into padded even rows for the odd mean model, and exact int32 values of
-// codes with |q| >= 2048 (their rows are listed for a fix-up).
-__global__ void __launch_bounds__(256) k_decode_symbols(int64_t slot0, int64_t n_slots, int k_eff,
-                                                        const uint8_t *kept_scale, const uint16_t *cdf,
-                                                        const uint16_t *lut, uint16_t *slots, uint32_t *row_esc,
-                                                        const int32_t *valid) {
-  extern __shared__ __align__(16) uint8_t sm[];
-  uint16_t *s_cdf = reinterpret_cast<uint16_t *>(sm);
-  uint16_t *s_lut = reinterpret_cast<uint16_t *>(sm + CDF_SMEM_BYTES);
-  __shared__ uint32_t cnt;
-  if (*valid != 1) return;
-  copy_smem16(s_cdf, cdf, CDF_SMEM_BYTES);
-  copy_smem16(s_lut, lut, LUT_SMEM_BYTES);
-  __syncthreads();
-  for (int64_t r = blockIdx.x; r < n_slots; r += gridDim.x) {
-    if (threadIdx.x == 0) cnt = 0;
-    __syncthreads();
-    uint16_t *sl = slots + (slot0 + r) * k_eff;
-    uint32_t esc = 0;
-    for (int k = threadIdx.x; k < k_eff; k += blockDim.x) {
-      const int s = kept_scale[k];
-      const uint16_t *tab = s_cdf + s * N_SYM;
-      const uint32_t slot = sl[k];
-      const int b = (int)(slot >> (16 - LUT_BITS));
-      int lo = s_lut[s * LUT_SIZE + b];
-      int hi = b + 1 < LUT_SIZE ? s_lut[s * LUT_SIZE + b + 1] : N_SYM - 1;
-      while (hi > lo) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (tab[mid] <= slot) lo = mid; else hi = mid - 1;
-      }
-      sl[k] = (uint16_t)lo;
-      esc += (lo == ESC_SYM);
-    }
-    for (int o = 16; o; o >>= 1) esc += __shfl_xor_sync(0xffffffffu, esc, o);
-    if ((threadIdx.x & 31) == 0 && esc) atomicAdd(&cnt, esc);
-    __syncthreads();
-    if (threadIdx.x == 0) row_esc[slot0 + r] = cnt;
-    __syncthreads();
-  }
-}
-
+// Finishing a decoded pass, one block per chunk, one warp per row: code = centre +
+// symbol - 254, or the chunk's next escape value for ESC; codes go to q16 (fp16, exact
+// below 2048), even rows also to qe (bf16, the odd mean model's input), codes of 2048 or
+// more to qbig with the row listed for the exact fix-up.  Escape values are stored in
+// symbol order, so each row first counts its escapes and takes its base from the rows
+// before it.
 struct DecCodesArgs {
   const ChunkDesc *chunks;
   const PromptInfo *prompts;
   int chunk0, n_chunks;
-  int chunk_rows;
   int k_eff;
   const int16_t *kept_list;
   const int8_t *cen8;
   const uint16_t *syms;     // slot order
-  const uint32_t *row_esc;  // per slot row
   const uint8_t *blob;
   uint64_t off_streams;
   const uint32_t *offs;
@@ -490,63 +564,78 @@ struct DecCodesArgs {
   int32_t *status;
 };
 
-__global__ void __launch_bounds__(256) k_decode_codes(DecCodesArgs a) {
+constexpr int DEC_CODES_THREADS = 256;
+
+__global__ void __launch_bounds__(DEC_CODES_THREADS) k_decode_codes(DecCodesArgs a) {
+  __shared__ uint32_t s_esc[256];  // escapes per row of the chunk (at most 256 rows)
   if (*a.valid != 1) return;
   const int lane = threadIdx.x & 31;
-  const int nw = blockDim.x >> 5;
+  const int warp = threadIdx.x >> 5;
+  const int nw = DEC_CODES_THREADS / 32;
   const uint32_t lt_mask = (1u << lane) - 1u;
-  const int total_rows = a.n_chunks * a.chunk_rows;  // rows of the pass, chunk-major (some absent)
-  for (int wr = blockIdx.x * nw + (threadIdx.x >> 5); wr < total_rows; wr += gridDim.x * nw) {
-    const int ci = a.chunk0 + wr / a.chunk_rows;
-    const int rl = wr % a.chunk_rows;
+  const int K = a.k_eff;
+  for (int cb = blockIdx.x; cb < a.n_chunks; cb += gridDim.x) {
+    const int ci = a.chunk0 + cb;
     const ChunkDesc cd = a.chunks[ci];
-    if (rl >= cd.nrows) continue;
     const PromptInfo pi = a.prompts[cd.prompt];
-    const int K = a.k_eff;
-    const int64_t slot_row = cd.sym_base / (K > 0 ? K : 1) + rl;
+    const int64_t slot_row0 = cd.sym_base / (K > 0 ? K : 1);
     const uint8_t *sec = a.blob + a.off_streams + a.offs[ci];
     const uint32_t ne = reinterpret_cast<const uint32_t *>(sec)[32];
     const uint32_t *ev = reinterpret_cast<const uint32_t *>(sec + CHUNK_FIXED_BYTES);
-    uint32_t ep = 0;
-    for (int r = 0; r < rl; ++r) ep += a.row_esc[slot_row - rl + r];
-    const uint16_t *sy = a.syms + slot_row * K;
-    const int8_t *ce = a.cen8 + slot_row * K;
-    const int j = cd.j0 + rl;
-    const int64_t row = (int64_t)pi.row_base + 2 * j + cd.parity;
-    __half *q16 = a.q16 + row * N_COEF;
-    __nv_bfloat16 *qe = cd.parity == 0 ? a.qe + (int64_t)(pi.ebase + j) * N_COEF : nullptr;
-    bool bad = false;
-    for (int k0 = 0; k0 < K; k0 += 32) {
-      const int k = k0 + lane;
-      const bool valid = k < K;
-      const int sym = valid ? sy[k] : 0;
-      const bool is_esc = valid && sym == ESC_SYM;
-      const uint32_t me = __ballot_sync(0xffffffffu, is_esc);
-      int q = valid ? sym - R_MAX + ce[k] : 0;
-      if (is_esc) {
-        const uint32_t e = ep + __popc(me & lt_mask);
-        if (e < ne) {
-          const int64_t sv = (int64_t)((uint64_t)ev[2 * e] | ((uint64_t)ev[2 * e + 1] << 32));
-          q = (int)max(min(sv, (int64_t)INT32_MAX), (int64_t)INT32_MIN);
-          if (sv >= -ESC_LIMIT && sv <= ESC_LIMIT) bad = true;  // not an escape value
-        } else {
-          bad = true;
-        }
-      }
-      ep += __popc(me);
-      if (valid) {
-        const int comp = a.kept_list[k];
-        q16[comp] = __float2half_rn((float)q);
-        if (qe) qe[comp] = __float2bfloat16_rn((float)q);
-        if (q >= BIG_CODE || q <= -BIG_CODE) {
-          a.qbig[row * N_COEF + comp] = q;
-          if (atomicExch(&a.bigflag[row], 1u) == 0u) a.biglist[atomicAdd(a.bigcount, 1u)] = (int32_t)row;
-        }
-      }
+    for (int rl = warp; rl < cd.nrows; rl += nw) {
+      const uint16_t *sy = a.syms + (slot_row0 + rl) * K;
+      uint32_t n = 0;
+      for (int k = lane; k < K; k += 32) n += sy[k] == ESC_SYM;
+      for (int o = 16; o; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
+      if (lane == 0) s_esc[rl] = n;
     }
-    // the chunk's last row checks that every escape value was used
-    if (rl == cd.nrows - 1 && ep != ne) bad = true;
-    if (__any_sync(0xffffffffu, bad) && lane == 0) atomicExch(a.status, DCKV_ECORRUPT);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      uint32_t tot = 0;
+      for (int r = 0; r < cd.nrows; ++r) tot += s_esc[r];
+      if (tot != ne) atomicExch(a.status, DCKV_ECORRUPT);  // every escape value used exactly once
+    }
+    for (int rl = warp; rl < cd.nrows; rl += nw) {
+      uint32_t ep = 0;
+      for (int r = 0; r < rl; ++r) ep += s_esc[r];
+      const uint16_t *sy = a.syms + (slot_row0 + rl) * K;
+      const int8_t *ce = a.cen8 + (slot_row0 + rl) * K;
+      const int j = cd.j0 + rl;
+      const int64_t row = (int64_t)pi.row_base + 2 * j + cd.parity;
+      __half *q16 = a.q16 + row * N_COEF;
+      __nv_bfloat16 *qe = cd.parity == 0 ? a.qe + (int64_t)(pi.ebase + j) * N_COEF : nullptr;
+      bool bad = false;
+      for (int k0 = 0; k0 < K; k0 += 32) {
+        const int k = k0 + lane;
+        const bool valid = k < K;
+        const int sym = valid ? sy[k] : 0;
+        const bool is_esc = valid && sym == ESC_SYM;
+        const uint32_t me = __ballot_sync(0xffffffffu, is_esc);
+        int q = valid ? sym - R_MAX + ce[k] : 0;
+        if (is_esc) {
+          const uint32_t e = ep + __popc(me & lt_mask);
+          if (e < ne) {
+            const int64_t sv = (int64_t)((uint64_t)ev[2 * e] | ((uint64_t)ev[2 * e + 1] << 32));
+            q = (int)max(min(sv, (int64_t)INT32_MAX), (int64_t)INT32_MIN);
+            if (sv >= -ESC_LIMIT && sv <= ESC_LIMIT) bad = true;  // not an escape value
+          } else {
+            bad = true;
+          }
+        }
+        ep += __popc(me);
+        if (valid) {
+          const int comp = a.kept_list[k];
+          q16[comp] = __float2half_rn((float)q);
+          if (qe) qe[comp] = __float2bfloat16_rn((float)q);
+          if (q >= BIG_CODE || q <= -BIG_CODE) {
+            a.qbig[row * N_COEF + comp] = q;
+            if (atomicExch(&a.bigflag[row], 1u) == 0u) a.biglist[atomicAdd(a.bigcount, 1u)] = (int32_t)row;
+          }
+        }
+      }
+      if (__any_sync(0xffffffffu, bad) && lane == 0) atomicExch(a.status, DCKV_ECORRUPT);
+    }
+    __syncthreads();
   }
 }
 

@@ -224,6 +224,21 @@ def test_parity_student_t_rows(src, codec_55):
     full_check(src, codec_55, [132 + 256], seeds=[21], chunk_rows=16, student_t=0.25)
 
 
+_FEW_KEPT = {}
+
+
+@pytest.mark.parametrize("step_scale,chunk_rows,k_range", [(60.0, 0, (8, 31)), (120.0, 5, (1, 7)), (200.0, 0, (0, 0))])
+def test_parity_fewer_than_32_kept_components(src, step_scale, chunk_rows, k_range):
+    # coarse steps drop most components: a lane's component wraps several times per step,
+    # and with none kept the streams hold only their final states
+    if step_scale not in _FEW_KEPT:
+        _FEW_KEPT[step_scale] = S.codec(src, step_scale=step_scale)
+    cod = _FEW_KEPT[step_scale]
+    k = int(O.scale_index(cod.laplace_b, cod.delta)[1].sum())
+    assert k_range[0] <= k <= k_range[1]
+    full_check(src, cod, [132 + 200, 140, 132 + 37], seeds=[41, 42, 43], chunk_rows=chunk_rows)
+
+
 def test_determinism(src, codec_55):
     gc = gpu_codec(codec_55)
     x, tok, offs = make_batch(src, codec_55, [132 + 500, 300], [31, 32])
