@@ -150,6 +150,26 @@ int dckv_decode(const dckv_codec *codec, const void *blob, size_t blob_bytes,
                 void *v_out, int32_t *status_dev, void *workspace, size_t ws_bytes,
                 void *stream /* cudaStream_t */);
 
+/* dckv_decode without a caller workspace.  The DCKV method has no counterpart to this call;
+ * it serves callers that cannot hand over device memory (a serving engine whose KV-cache
+ * pool already holds all free device memory, a host program with no device allocator).
+ * Its scratch is one static device array of DCKV_STATIC_SCRATCH_BYTES per GPU that loads
+ * the library, held until the process exits; the call allocates nothing.
+ *   Limit: batches whose decode scratch (dckv_ws_offsets(..., 1, ...).total) exceeds
+ *   DCKV_STATIC_SCRATCH_BYTES -- about 800 coded rows at K_eff = 2048 -- are rejected with
+ *   DCKV_ECAPACITY before any device work.
+ *   Set-up: the first call on a device looks the array's device address up once (host-side
+ *   symbol lookup, under a lock); make that first call before any stream capture.
+ *   Sharing: every call on a device uses the same array, which keeps the last call's
+ *   contents; each call initialises (clears or overwrites) everything it reads before it
+ *   reads it.  Calls that overlap in time on one device -- different streams or host
+ *   threads without ordering between them -- race on the array; order them on one stream.
+ * Arguments, layouts, status and return values as dckv_decode. */
+#define DCKV_STATIC_SCRATCH_BYTES (16u << 20)
+int dckv_decode_static(const dckv_codec *codec, const void *blob, size_t blob_bytes,
+                       const int32_t *token_ids, const int64_t *seq_offsets, int batch, void *k_out,
+                       void *v_out, int32_t *status_dev, void *stream /* cudaStream_t */);
+
 /* Byte breakdown of a blob held in HOST memory (len bytes).  Blob layout, little endian:
  *   64-byte header {u32 magic 0x564B4344 "DCKV", u16 version 1, u16 chunk rows G,
  *     u32 prompts, u32 coefficients (2048), u32 K_eff, u32 even chunks, u32 odd chunks,

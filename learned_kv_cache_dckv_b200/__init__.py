@@ -75,6 +75,7 @@ def lib():
         "dckv_blob_bound": (Z, [P, P, I]),
         "dckv_encode": (I, [P, P, P, P, I, P, Z, P, P, P, Z, P]),
         "dckv_decode": (I, [P, P, Z, P, P, I, P, P, P, P, Z, P]),
+        "dckv_decode_static": (I, [P, P, Z, P, P, I, P, P, P, P]),
         "dckv_bytes": (I, [P, Z, ctypes.POINTER(ByteReport)]),
         "dckv_last_error": (ctypes.c_char_p, []),
         "dckv_ws_offsets": (I, [P, P, I, I, ctypes.POINTER(WsView)]),
@@ -174,6 +175,14 @@ def dckv_decode(handle, blob, blob_bytes, token_ids, seq_offsets, k_out, v_out, 
     _check(lib().dckv_decode(handle, blob.data_ptr(), int(blob_bytes), token_ids.data_ptr(), ptr, b,
                              k_out.data_ptr(), v_out.data_ptr(), status.data_ptr(), workspace.data_ptr(),
                              workspace.numel() * workspace.element_size(), _stream_ptr(stream)), "dckv_decode")
+
+
+def dckv_decode_static(handle, blob, blob_bytes, token_ids, seq_offsets, k_out, v_out, status, stream=None):
+    """dckv_decode on the library's static per-device scratch (no workspace argument)."""
+    a, ptr, b = _offs(seq_offsets)
+    _check(lib().dckv_decode_static(handle, blob.data_ptr(), int(blob_bytes), token_ids.data_ptr(), ptr, b,
+                                    k_out.data_ptr(), v_out.data_ptr(), status.data_ptr(), _stream_ptr(stream)),
+           "dckv_decode_static")
 
 
 def dckv_bytes(blob_host: bytes) -> dict:

@@ -1399,3 +1399,46 @@ extern "C" int dckv_debug_gemm(int bf16, const void *A, int slabs, const void *B
   EpiStoreF32::Params ep{D, M, 1.0f};
   return run_gemm<EpiStoreF32, 3, 2>(ma, ma, mb, mb, pr, ep, sms, (cudaStream_t)stream);
 }
+
+// ============================================================================ decode, static scratch
+// Scratch of dckv_decode_static: one file-scope device array per GPU that loads this
+// library, held until the process exits.  Callers that cannot hand over a workspace use it:
+// a serving engine that has reserved all free device memory for its KV-cache pool before
+// it restores cached prompts, or a host program without a device allocator of its own --
+// they have no spare device memory to offer, and allocating inside the call would
+// synchronise the device and could fail under memory pressure.
+static __device__ __align__(256) uint8_t g_static_scratch[DCKV_STATIC_SCRATCH_BYTES];
+
+namespace {
+constexpr int MAX_DEVICES = 64;
+std::mutex g_static_mu;
+void *g_static_ptr[MAX_DEVICES] = {};  // device address of g_static_scratch, per device
+}  // namespace
+
+extern "C" int dckv_decode_static(const dckv_codec *c, const void *blob, size_t blob_bytes,
+                                  const int32_t *token_ids, const int64_t *seq_offsets, int batch, void *k_out,
+                                  void *v_out, int32_t *status_dev, void *stream) {
+  if (!c) return fail(DCKV_EINVAL, "codec is NULL");
+  Layout L;
+  RET(build_layout(c, seq_offsets, batch, L));
+  const size_t need = plan_ws(L, 1).total;
+  if (need > (size_t)DCKV_STATIC_SCRATCH_BYTES)
+    return fail(DCKV_ECAPACITY, "batch needs %zu bytes of decode scratch; the static scratch holds %zu", need,
+                (size_t)DCKV_STATIC_SCRATCH_BYTES);
+  if (c->device < 0 || c->device >= MAX_DEVICES) return fail(DCKV_EINVAL, "device %d out of range", c->device);
+  CK(cudaSetDevice(c->device));
+  void *scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    if (!g_static_ptr[c->device]) {  // first call on this device: look the array up once
+      void *p = nullptr;
+      const cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
+      if (e != cudaSuccess || !p)
+        return fail(DCKV_ECUDA, "cudaGetSymbolAddress(static scratch) failed: %s", cudaGetErrorString(e));
+      g_static_ptr[c->device] = p;
+    }
+    scratch = g_static_ptr[c->device];
+  }
+  return dckv_decode(c, blob, blob_bytes, token_ids, seq_offsets, batch, k_out, v_out, status_dev, scratch,
+                     (size_t)DCKV_STATIC_SCRATCH_BYTES, stream);
+}
