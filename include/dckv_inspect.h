@@ -68,9 +68,10 @@ int dckv_get_timing(const dckv_codec *codec, float *ms, const char **names, int 
 
 /* Self-test of the tcgen05 GEMM core: D[n][m] = sum_s sum_k A[s][m][k] * B[n][k]
  * (fp32 accumulate).  A: device fp16/bf16 [slabs][M][K]; B: device [N][K]; D: device
- * fp32 [N][M].  M % 128 == 0, K % 64 == 0, slabs in {1, 2}, bn (N tile) in 16..256 step 16. */
+ * fp32 [N][M].  M % 128 == 0, K % 64 == 0, slabs in {1, 2}, bn (N tile) in 16..256 step 16.
+ * pair = 1 runs the CTA-pair kernel (cta_group::2, 256 x bn tiles; M % 256 == 0). */
 int dckv_debug_gemm(int bf16, const void *A, int slabs, const void *B, int M, int N, int K, float *D, int bn,
-                    void *stream);
+                    int pair, void *stream);
 
 #ifdef __cplusplus
 }

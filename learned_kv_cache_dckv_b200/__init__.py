@@ -83,7 +83,7 @@ def lib():
         "dckv_codec_tables": (I, [P, ctypes.POINTER(P), ctypes.POINTER(P)]),
         "dckv_set_timing": (I, [P, I]),
         "dckv_get_timing": (I, [P, P, P, I]),
-        "dckv_debug_gemm": (I, [I, P, I, P, I, I, I, P, I, P]),
+        "dckv_debug_gemm": (I, [I, P, I, P, I, I, I, P, I, I, P]),
         "dckv_debug_ratio": (I, [P, P]),
         "dckv_codec_info": (I, [P, P, P]),
     }
@@ -238,9 +238,10 @@ def dckv_get_timing(handle, max_stages: int = 24):
     return [(names[i].decode(), float(ms[i])) for i in range(max(0, n))]
 
 
-def dckv_debug_gemm(bf16: bool, A, slabs: int, B, M: int, N: int, K: int, D, bn: int = 256, stream=None):
+def dckv_debug_gemm(bf16: bool, A, slabs: int, B, M: int, N: int, K: int, D, bn: int = 256, pair: bool = False,
+                    stream=None):
     _check(lib().dckv_debug_gemm(1 if bf16 else 0, A.data_ptr(), int(slabs), B.data_ptr(), int(M), int(N), int(K),
-                                 D.data_ptr(), int(bn), _stream_ptr(stream)), "dckv_debug_gemm")
+                                 D.data_ptr(), int(bn), 1 if pair else 0, _stream_ptr(stream)), "dckv_debug_gemm")
 
 
 # ---------------------------------------------------------------------------------- helpers

@@ -124,6 +124,62 @@ static int run_gemm(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensor
   return DCKV_OK;
 }
 
+// CTA-pair launches: clusters of two, one pair per two SMs at most.
+static int launch_pairs(const void *kern, int tiles, int num_sms, int threads, int smem, cudaStream_t st,
+                        void **args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(2 * std::min(tiles, num_sms / 2)));
+  cfg.blockDim = dim3((unsigned)threads);
+  cfg.dynamicSmemBytes = (size_t)smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  CK(cudaLaunchKernelExC(&cfg, kern, args));
+  return DCKV_OK;
+}
+
+template <class Epi, int STAGES, int MAX_SLABS, int EPI_WARPS>
+static int run_gemm2(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &b0, const CUtensorMap &b1,
+                     GemmProblem prob, const typename Epi::Params &ep, int num_sms, bool bf16, cudaStream_t st) {
+  constexpr int smem = gemm2_smem_bytes<Epi, STAGES, MAX_SLABS, EPI_WARPS>();
+  static_assert(smem <= 232448, "GEMM shared memory above the sm_100 limit");
+  auto kern = gemm2_kernel<Epi, STAGES, MAX_SLABS, EPI_WARPS>;
+  CK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  if (prob.m_tiles % 2 || prob.bn % 16 || prob.bn > GEMM_MAX_BN) return fail(DCKV_EINVAL, "bad CTA-pair GEMM shape");
+  const int tiles = (prob.m_tiles / 2) * prob.n_tiles;
+  if (tiles <= 0) return DCKV_OK;
+  for (int i = 0; i < prob.n_seg; ++i)
+    if (prob.seg[i].n_slab < 1 || prob.seg[i].n_slab > MAX_SLABS) return fail(DCKV_EINVAL, "bad slab count");
+  prob.idesc = idesc_f16(bf16 ? 1 : 0, 2 * GEMM_BM, prob.bn);
+  typename Epi::Params epc = ep;
+  void *args[] = {(void *)&a0, (void *)&a1, (void *)&b0, (void *)&b1, (void *)&prob, (void *)&epc};
+  return launch_pairs((const void *)kern, tiles, num_sms, 64 + 32 * EPI_WARPS, smem, st, args);
+}
+
+template <class Epi, int STAGES, int MAX_SLABS, int CHUNK_STEPS, int BN>
+static int run_gemm2_chunked(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &b0,
+                             const CUtensorMap &b1, GemmProblem prob, const typename Epi::Params &ep, int num_sms,
+                             bool bf16, cudaStream_t st) {
+  constexpr int smem = gemm2_chunked_smem_bytes<STAGES, MAX_SLABS>();
+  static_assert(smem <= 232448, "GEMM shared memory above the sm_100 limit");
+  auto kern = gemm2_chunked_kernel<Epi, STAGES, MAX_SLABS, CHUNK_STEPS, BN>;
+  CK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  if (prob.m_tiles % 2 || prob.bn != BN) return fail(DCKV_EINVAL, "bad chunked CTA-pair GEMM shape");
+  const int tiles = (prob.m_tiles / 2) * prob.n_tiles;
+  if (tiles <= 0) return DCKV_OK;
+  for (int i = 0; i < prob.n_seg; ++i)
+    if (prob.seg[i].n_slab < 1 || prob.seg[i].n_slab > MAX_SLABS) return fail(DCKV_EINVAL, "bad slab count");
+  prob.idesc = idesc_f16(bf16 ? 1 : 0, 2 * GEMM_BM, BN);
+  typename Epi::Params epc = ep;
+  void *args[] = {(void *)&a0, (void *)&a1, (void *)&b0, (void *)&b1, (void *)&prob, (void *)&epc};
+  return launch_pairs((const void *)kern, tiles, num_sms, GEMM2C_THREADS, smem, st, args);
+}
+
 template <class Epi, int STAGES, int MAX_SLABS, int CHUNK_STEPS>
 static int run_gemm_chunked(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &b0,
                             const CUtensorMap &b1, const GemmProblem &prob, const typename Epi::Params &ep,
@@ -464,6 +520,18 @@ __global__ void __launch_bounds__(256) k_kept(const uint8_t *blob, uint64_t off_
   }
 }
 
+// RoPE table of a decode call: rope[pos][i] = (cos, sin) of pos * theta_i, the same values
+// rope_cs gives the kept-row and fix-up kernels.
+__global__ void __launch_bounds__(128) k_rope_table(float2 *rope, int64_t n_pos, const double *theta,
+                                                   const int32_t *valid) {
+  if (*valid != 1) return;
+  for (int64_t pos = blockIdx.x; pos < n_pos; pos += gridDim.x) {
+    float cs, sn;
+    rope_cs((int)pos, threadIdx.x, theta, cs, sn);
+    rope[pos * 128 + threadIdx.x] = make_float2(cs, sn);
+  }
+}
+
 __host__ __device__ __forceinline__ int dim_to_inv_row(int d) {
   const int hv = d / HEAD_DIM, dd = d % HEAD_DIM;
   const int half = dd < 128 ? dd / 64 : (dd - 128) / 64;
@@ -641,6 +709,7 @@ static int build_layout(const dckv_codec *c, const int64_t *offs, int batch, Lay
     p.kept_base = (int32_t)kept;
     p.n_kept = (int32_t)(N - p.n);
     p.chunk_e0 = ce;
+    L.max_len = std::max<int64_t>(L.max_len, N);
     ce += (p.n_e + G - 1) / G;
     rows += p.n;
     ne += p.n_e + 1;
@@ -728,6 +797,7 @@ static WsPlan plan_ws(const Layout &L, int which /*0 encode, 1 decode*/) {
     w.full_list = take(4ull * L.n_rows);
   } else {
     w.slots16 = take(2ull * L.n_symbols);
+    w.rope = take(8ull * 128 * std::max<int64_t>(L.max_len, 1));
     w.q16 = take(2ull * L.n_rows * N_COEF);
     w.qbig = take(4ull * L.n_rows * N_COEF);
     w.bigflag = take(4ull * L.n_rows);
@@ -1062,10 +1132,11 @@ extern "C" int dckv_encode(const dckv_codec *c, const void *rows, const int32_t 
   CK(cudaGetLastError());
   stage_mark(c, st, "layout+convert");
   if (L.n_rows > 0) {
-    CUtensorMap mb_x128, mb_g128, mb_qe;
+    CUtensorMap mb_x128, mb_xt, mb_gt, mb_qe;
     RET(map_b(&mb_x128, x16, false, ROW_DIM, L.n_rows, 128));
-    RET(map_b(&mb_g128, g16, false, 2 * N_HIDDEN, L.n_rows, 128));
-    RET(map_b(&mb_qe, qe, true, N_COEF, L.ne_pad, 256));
+    RET(map_b(&mb_xt, x16, false, ROW_DIM, L.n_rows, TRANSFORM_BN / 2));
+    RET(map_b(&mb_gt, g16, false, 2 * N_HIDDEN, L.n_rows, TRANSFORM_BN / 2));
+    RET(map_b(&mb_qe, qe, true, N_COEF, L.ne_pad, MEAN_ODD_BN / 2));
     // correction hidden layer: h = x @ w1 - mu @ w1, GELU, fp16 hi/lo
     {
       GemmProblem pr = make_problem(N_HIDDEN / GEMM_BM, L.n_rows, 128, false, status_dev);
@@ -1077,14 +1148,14 @@ extern "C" int dckv_encode(const dckv_codec *c, const void *rows, const int32_t 
     stage_mark(c, st, "gemm_hidden");
     // transform + quantiser: y = x @ B + g @ w2 - mu @ B
     {
-      GemmProblem pr = make_problem(N_COEF / GEMM_BM, L.n_rows, GEMMC_BN, false, status_dev);
+      GemmProblem pr = make_problem(N_COEF / GEMM_BM, L.n_rows, TRANSFORM_BN, false, status_dev);
       add_seg(pr, 0, 0, 2, 0, 0, 0, 0, ROW_DIM / GEMM_BK);
       add_seg(pr, 1, 0, 2, 0, 1, 0, 0, N_HIDDEN / GEMM_BK);
       add_seg(pr, 1, 0, 2, 0, 1, 0, N_HIDDEN, N_HIDDEN / GEMM_BK);
-      EpiQuantTotals::Params ep{{c->mub, c->delta, c->keep, (float)std::ldexp(1.0, -c->p_y), q32, qe, row_edst},
-                                row_norm, rowflag, el_list, full_list, counters, w.el_cap, c->dbg_ratio};
-      RET((run_gemm_chunked<EpiQuantTotals, 4, 2, 4>(c->map_ay2, c->map_aw2_2, mb_x128, mb_g128, pr, ep,
-                                                      c->num_sms, st)));
+      EpiQuantRegs::Params ep{{c->mub, c->delta, c->keep, (float)std::ldexp(1.0, -c->p_y), q32, qe, row_edst},
+                              row_norm, rowflag, el_list, full_list, counters, w.el_cap, c->dbg_ratio};
+      RET((run_gemm2_chunked<EpiQuantRegs, 4, 2, 4, TRANSFORM_BN>(c->map_ay2, c->map_aw2_2, mb_xt, mb_gt, pr, ep,
+                                                                   c->num_sms, false, st)));
     }
     stage_mark(c, st, "gemm_transform");
     // codes whose fp32 ratio lies in the guard band around a half step: exact fp64 values
@@ -1099,11 +1170,11 @@ extern "C" int dckv_encode(const dckv_codec *c, const void *rows, const int32_t 
     stage_mark(c, st, "refine");
     // odd mean model: [e, bf16(q_left), bf16(q_right)] @ w_odd -> centres
     {
-      GemmProblem pr = make_problem(N_COEF / GEMM_BM, L.ne_pad, 256, true, status_dev);
+      GemmProblem pr = make_problem(N_COEF / GEMM_BM, L.ne_pad, MEAN_ODD_BN, true, status_dev);
       add_seg(pr, 0, 0, 1, 0, 0, 0, 0, N_COEF / GEMM_BK);
       add_seg(pr, 0, 0, 1, N_COEF, 0, 1, 0, N_COEF / GEMM_BK);
       EpiMeanOdd::Params ep{c->t_odd, token_ids, e_tok, e_slot, c->kidx, cen8, c->k_eff, c->vocab};
-      RET((run_gemm<EpiMeanOdd, 4, 1>(c->map_aon1, c->map_aon1, mb_qe, mb_qe, pr, ep, c->num_sms, st)));
+      RET((run_gemm2<EpiMeanOdd, 6, 1, 8>(c->map_aon1, c->map_aon1, mb_qe, mb_qe, pr, ep, c->num_sms, true, st)));
     }
     stage_mark(c, st, "gemm_mean_odd");
     // even centres from the vocabulary table, then every symbol, in slot order
@@ -1166,6 +1237,7 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
   int8_t *cen8 = (int8_t *)(ws + w.cen8);
   int32_t *slot_chunk = (int32_t *)(ws + w.slot_chunk);
   uint16_t *syms16 = (uint16_t *)(ws + w.slots16);
+  float2 *rope = (float2 *)(ws + w.rope);
   __half *q16 = (__half *)(ws + w.q16);
   int32_t *qbig = (int32_t *)(ws + w.qbig);
   uint32_t *bigflag = (uint32_t *)(ws + w.bigflag);
@@ -1187,6 +1259,8 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
   HeaderCheck hc{bl, blob_bytes, d_prompts, L.batch, c->chunk_rows, c->k_eff, L.n_chunks_e, L.n_chunks_o,
                  L.n_kept, L.off_kept, L.off_streams, valid, status_dev};
   k_check_header<<<1, 256, 0, st>>>(hc);
+  if (L.n_rows > 0)
+    k_rope_table<<<(unsigned)std::min<int64_t>(L.max_len, 4096), 128, 0, st>>>(rope, L.max_len, c->theta, valid);
   CK(cudaGetLastError());
   stage_mark(c, st, "layout+check");
   const uint32_t *offs = (const uint32_t *)(bl + HEADER_BYTES + 4ull * L.batch);
@@ -1214,12 +1288,12 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
   stage_mark(c, st, "codes_even");
   if (L.n_rows > 0) {
     CUtensorMap mb_qe;
-    RET(map_b(&mb_qe, qe, true, N_COEF, L.ne_pad, 256));
-    GemmProblem pr = make_problem(N_COEF / GEMM_BM, L.ne_pad, 256, true, status_dev);
+    RET(map_b(&mb_qe, qe, true, N_COEF, L.ne_pad, MEAN_ODD_BN / 2));
+    GemmProblem pr = make_problem(N_COEF / GEMM_BM, L.ne_pad, MEAN_ODD_BN, true, status_dev);
     add_seg(pr, 0, 0, 1, 0, 0, 0, 0, N_COEF / GEMM_BK);
     add_seg(pr, 0, 0, 1, N_COEF, 0, 1, 0, N_COEF / GEMM_BK);
     EpiMeanOdd::Params ep{c->t_odd, token_ids, e_tok, e_slot, c->kidx, cen8, c->k_eff, c->vocab};
-    RET((run_gemm<EpiMeanOdd, 4, 1>(c->map_aon1, c->map_aon1, mb_qe, mb_qe, pr, ep, c->num_sms, st)));
+    RET((run_gemm2<EpiMeanOdd, 6, 1, 8>(c->map_aon1, c->map_aon1, mb_qe, mb_qe, pr, ep, c->num_sms, true, st)));
   }
   stage_mark(c, st, "gemm_mean_odd");
   if (L.n_chunks_o > 0) {
@@ -1231,12 +1305,12 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
   stage_mark(c, st, "codes_odd");
   if (L.n_rows > 0) {
     CUtensorMap mb_q;
-    RET(map_b(&mb_q, q16, false, N_COEF, L.n_rows, 256));
-    GemmProblem pr = make_problem(ROW_DIM / GEMM_BM, L.n_rows, 256, false, status_dev);
+    RET(map_b(&mb_q, q16, false, N_COEF, L.n_rows, INVERSE_BN / 2));
+    GemmProblem pr = make_problem(ROW_DIM / GEMM_BM, L.n_rows, INVERSE_BN, false, status_dev);
     add_seg(pr, 0, 0, 2, 0, 0, 0, 0, N_COEF / GEMM_BK);
-    EpiInverse::Params ep{c->mu_perm, (float)std::ldexp(1.0, -c->p_inv), c->theta, row_tok, row_pos,
+    EpiInverse::Params ep{c->mu_perm, (float)std::ldexp(1.0, -c->p_inv), rope, row_tok, row_pos,
                           (__nv_bfloat16 *)k_out, (__nv_bfloat16 *)v_out, L.n_tokens};
-    RET((run_gemm<EpiInverse, 3, 2>(c->map_ainv2, c->map_ainv2, mb_q, mb_q, pr, ep, c->num_sms, st)));
+    RET((run_gemm2<EpiInverse, 4, 2, 8>(c->map_ainv2, c->map_ainv2, mb_q, mb_q, pr, ep, c->num_sms, false, st)));
   }
   stage_mark(c, st, "gemm_inverse");
   if (L.n_kept > 0)
@@ -1383,9 +1457,9 @@ extern "C" int dckv_ws_offsets(const dckv_codec *c, const int64_t *offs, int bat
 
 // D[n][m] = sum_s sum_k A[s][m][k] * B[n][k] through the tcgen05 GEMM (self-test).
 extern "C" int dckv_debug_gemm(int bf16, const void *A, int slabs, const void *Bm, int M, int N, int K, float *D,
-                               int bn, void *stream) {
+                               int bn, int pair, void *stream) {
   if (!A || !Bm || !D || M % GEMM_BM || K % GEMM_BK || N < 1 || slabs < 1 || slabs > 2 || bn < 16 || bn > 256 ||
-      bn % 16)
+      bn % 16 || (pair && M % (2 * GEMM_BM)))
     return fail(DCKV_EINVAL, "bad GEMM shape");
   int dev;
   CK(cudaGetDevice(&dev));
@@ -1393,10 +1467,11 @@ extern "C" int dckv_debug_gemm(int bf16, const void *A, int slabs, const void *B
   CK(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
   CUtensorMap ma, mb;
   RET(map_a(&ma, A, bf16 != 0, K, M, slabs, slabs));
-  RET(map_b(&mb, Bm, bf16 != 0, K, N, bn));
+  RET(map_b(&mb, Bm, bf16 != 0, K, N, pair ? bn / 2 : bn));
   GemmProblem pr = make_problem(M / GEMM_BM, N, bn, bf16 != 0, nullptr);
   add_seg(pr, 0, 0, slabs, 0, 0, 0, 0, K / GEMM_BK);
   EpiStoreF32::Params ep{D, M, 1.0f};
+  if (pair) return run_gemm2<EpiStoreF32, 4, 2, 4>(ma, ma, mb, mb, pr, ep, sms, bf16 != 0, (cudaStream_t)stream);
   return run_gemm<EpiStoreF32, 3, 2>(ma, ma, mb, mb, pr, ep, sms, (cudaStream_t)stream);
 }
 

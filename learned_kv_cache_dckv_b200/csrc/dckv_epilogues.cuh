@@ -1,8 +1,8 @@
 // dckv_epilogues.cuh -- fused epilogues of the codec's tcgen05 GEMMs.
 //
-// Each epilogue runs on the 128 epilogue threads of gemm_kernel; thread (ew, lane) owns
-// output feature m = mt*128 + ew*32 + lane and walks the tile's token columns 32 at a
-// time with tcgen05.ld.
+// An epilogue runs on groups of 128 epilogue threads (EpiCtx); thread (ew, lane) owns
+// output feature m = mt*128 + ew*32 + lane and walks its group's token-column chunks
+// with tcgen05.ld.
 #pragma once
 #include "dckv_gemm.cuh"
 #include "dckv_internal.cuh"
@@ -30,16 +30,15 @@ struct EpiStoreF32 {
     float scale;
   };
   static constexpr int SMEM_BYTES = 0;
-  __device__ static void tile(const Params &p, char *, int mt, int n0, int n_valid, int bn, uint32_t tacc, int ew,
-                              int lane, int) {
-    const int m = mt * GEMM_BM + ew * 32 + lane;
-    for (int c0 = 0; c0 < n_valid; c0 += 32) {
+  __device__ static void tile(const Params &p, const EpiCtx &cx) {
+    const int m = cx.mt * GEMM_BM + cx.ew * 32 + cx.lane;
+    for (int c0 = cx.grp * 32; c0 < cx.n_valid; c0 += 32 * cx.n_grp) {
       uint32_t r[32];
-      tmem_ld_32x32b_x32(tacc + (uint32_t)c0, r);
+      tmem_ld_32x32b_x32(cx.tacc + (uint32_t)c0, r);
       tmem_ld_wait();
 #pragma unroll
       for (int j = 0; j < 32; ++j)
-        if (c0 + j < n_valid) p.out[(int64_t)(n0 + c0 + j) * p.ld + m] = u2f(r[j]) * p.scale;
+        if (c0 + j < cx.n_valid) p.out[(int64_t)(cx.n0 + c0 + j) * p.ld + m] = u2f(r[j]) * p.scale;
     }
   }
 };
@@ -53,29 +52,6 @@ struct EpiGelu {
     float scale;
     __half *g;  // [rows][512]
   };
-  static constexpr int SMEM_BYTES = 0;
-  __device__ static void tile(const Params &p, char *, int mt, int n0, int n_valid, int bn, uint32_t tacc, int ew,
-                              int lane, int) {
-    const int m = mt * GEMM_BM + ew * 32 + lane;
-    const float mw = p.muw1[m];
-    for (int c0 = 0; c0 < n_valid; c0 += 32) {
-      uint32_t r[32];
-      tmem_ld_32x32b_x32(tacc + (uint32_t)c0, r);
-      tmem_ld_wait();
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        if (c0 + j < n_valid) {
-          const float h = u2f(r[j]) * p.scale - mw;
-          const float g = 0.5f * h * (1.0f + erff(h * 0.70710678118654752f));
-          const __half hi = __float2half_rn(g);
-          const __half lo = __float2half_rn(g - __half2float(hi));
-          __half *row = p.g + (int64_t)(n0 + c0 + j) * (2 * N_HIDDEN);
-          row[m] = hi;
-          row[N_HIDDEN + m] = lo;
-        }
-      }
-    }
-  }
 };
 
 // Chunk-accumulated form of EpiGelu (the hidden units feed the exact refinement too):
@@ -124,36 +100,12 @@ struct EpiQuant {
     __nv_bfloat16 *qe;        // [ne_pad][2048]
     const int32_t *row_edst;  // [rows]: padded even row or -1
   };
-  static constexpr int SMEM_BYTES = 0;
-  __device__ static void tile(const Params &p, char *, int mt, int n0, int n_valid, int bn, uint32_t tacc, int ew,
-                              int lane, int) {
-    const int c = mt * GEMM_BM + ew * 32 + lane;
-    const float mb = p.mub[c];
-    const float dl = p.delta[c];
-    const bool kp = p.keep[c] != 0;
-    for (int c0 = 0; c0 < n_valid; c0 += 32) {
-      uint32_t r[32];
-      tmem_ld_32x32b_x32(tacc + (uint32_t)c0, r);
-      tmem_ld_wait();
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        if (c0 + j < n_valid) {
-          const int row = n0 + c0 + j;
-          const float y = u2f(r[j]) * p.scale - mb;
-          const int q = kp ? __float2int_rn(__fdiv_rn(y, dl)) : 0;
-          p.q32[(int64_t)row * N_COEF + c] = q;
-          const int e = p.row_edst[row];
-          if (e >= 0) p.qe[(int64_t)e * N_COEF + c] = __float2bfloat16_rn((float)q);
-        }
-      }
-    }
-  }
 };
 
-// Chunk-accumulated transform + quantiser: reads this thread's totals (columns
-// c_begin .. c_begin + 63) from TMEM; codes whose fp32 ratio lies in the guard band around
-// a half step are listed for exact fp64 recomputation (whole rows when the row is large).
-struct EpiQuantTotals {
+// Chunk-accumulated transform + quantiser: takes this thread's totals (NC columns from
+// col0) from registers; codes whose fp32 ratio lies in the guard band around a half step
+// are listed for exact fp64 recomputation (whole rows when the row is large).
+struct EpiQuantRegs {
   struct Params {
     EpiQuant::Params q;
     const float *row_norm;   // [rows] |x|_2 of the coded row
@@ -164,7 +116,6 @@ struct EpiQuantTotals {
     int64_t el_cap;
     float *dbg_ratio;        // optional export of the fp32 ratios (self-test)
   };
-  static constexpr int SMEM_BYTES = 0;
   __device__ static void list_row(const Params &p, int row) {
     if (atomicExch(&p.rowflag[row], 1u) == 0u) p.full_list[atomicAdd(&p.counters[1], 1u)] = (uint32_t)row;
   }
@@ -177,37 +128,30 @@ struct EpiQuantTotals {
       else list_row(pp, row);
     }
   }
-  __device__ static void tile(const Params &pp, char *, int mt, int n0, int n_valid, int c_begin, uint32_t ttot,
-                              int ew, int lane, int) {
+  template <int NC>
+  __device__ static void finish(const Params &pp, const float (&tot)[NC], int mt, int n0, int n_valid, int col0,
+                                int ew, int lane) {
     const EpiQuant::Params &p = pp.q;
     const int c = mt * GEMM_BM + ew * 32 + lane;
     const float mb = p.mub[c];
     const float dl = p.delta[c];
     const bool kp = p.keep[c] != 0;
     const float wk = REFINE_KAPPA / dl;
-#pragma unroll 1
-    for (int g = 0; g < 2; ++g) {
-      const int col0 = c_begin + g * 32;
-      if (col0 >= n_valid) break;
-      uint32_t r[32];
-      tmem_ld_32x32b_x32(ttot + (uint32_t)(g * 32), r);
-      tmem_ld_wait();
-#pragma unroll 8
-      for (int j = 0; j < 32; ++j) {
-        const int col = col0 + j;
-        if (col < n_valid) {
-          const int row = n0 + col;
-          const float y = u2f(r[j]) * p.scale - mb;
-          const float ratio = __fdiv_rn(y, dl);
-          const int q = kp ? __float2int_rn(ratio) : 0;
-          p.q32[(int64_t)row * N_COEF + c] = q;
-          const int e = p.row_edst[row];
-          if (e >= 0) p.qe[(int64_t)e * N_COEF + c] = __float2bfloat16_rn((float)q);
-          if (pp.dbg_ratio) pp.dbg_ratio[(int64_t)row * N_COEF + c] = ratio;
-          if (kp) {
-            const float w = wk * pp.row_norm[row] + REFINE_W0;
-            if (0.5f - fabsf(ratio - rintf(ratio)) < w || !(fabsf(ratio) < 1.0e6f)) flag(pp, row, c);
-          }
+#pragma unroll
+    for (int j = 0; j < NC; ++j) {
+      const int col = col0 + j;
+      if (col < n_valid) {
+        const int row = n0 + col;
+        const float y = tot[j] * p.scale - mb;
+        const float ratio = __fdiv_rn(y, dl);
+        const int q = kp ? __float2int_rn(ratio) : 0;
+        p.q32[(int64_t)row * N_COEF + c] = q;
+        const int e = p.row_edst[row];
+        if (e >= 0) p.qe[(int64_t)e * N_COEF + c] = __float2bfloat16_rn((float)q);
+        if (pp.dbg_ratio) pp.dbg_ratio[(int64_t)row * N_COEF + c] = ratio;
+        if (kp) {
+          const float w = wk * pp.row_norm[row] + REFINE_W0;
+          if (0.5f - fabsf(ratio - rintf(ratio)) < w || !(fabsf(ratio) < 1.0e6f)) flag(pp, row, c);
         }
       }
     }
@@ -229,28 +173,28 @@ struct EpiMeanOdd {
     int k_eff;
     int vocab;
   };
-  // per tile column: t_odd row offset (or -1) and the slot row
+  // per tile column: t_odd row offset (or -1) and the slot row (each group stages its own)
   static constexpr int SMEM_BYTES = 256 * 16;
-  __device__ static void tile(const Params &p, char *scratch, int mt, int n0, int n_valid, int bn, uint32_t tacc,
-                              int ew, int lane, int et) {
-    int64_t *s_row = reinterpret_cast<int64_t *>(scratch);
-    int32_t *s_slot = reinterpret_cast<int32_t *>(scratch + 256 * 8);
-    for (int j = et; j < n_valid; j += 128) {
-      const int ti = p.e_tok[n0 + j];
+  __device__ static void tile(const Params &p, const EpiCtx &cx) {
+    int64_t *s_row = reinterpret_cast<int64_t *>(cx.scratch);
+    int32_t *s_slot = reinterpret_cast<int32_t *>(cx.scratch + 256 * 8);
+    const int n_valid = cx.n_valid;
+    for (int j = cx.et; j < n_valid; j += 128) {
+      const int ti = p.e_tok[cx.n0 + j];
       int64_t off = -1;
       if (ti >= 0) {
         const int tok = min(max(p.tok_ids[ti], 0), p.vocab - 1);
         off = (int64_t)tok * N_COEF;
       }
       s_row[j] = off;
-      s_slot[j] = p.e_slot[n0 + j];
+      s_slot[j] = p.e_slot[cx.n0 + j];
     }
-    named_bar_sync(1, 128);
-    const int c = mt * GEMM_BM + ew * 32 + lane;
+    named_bar_sync(cx.bar, 128);
+    const int c = cx.mt * GEMM_BM + cx.ew * 32 + cx.lane;
     const int kc = p.kidx[c];
-    for (int c0 = 0; c0 < n_valid; c0 += 32) {
+    for (int c0 = cx.grp * 32; c0 < n_valid; c0 += 32 * cx.n_grp) {
       uint32_t r[32];
-      tmem_ld_32x32b_x32(tacc + (uint32_t)c0, r);
+      tmem_ld_32x32b_x32(cx.tacc + (uint32_t)c0, r);
       float tv[32];
 #pragma unroll
       for (int j = 0; j < 32; ++j) {  // independent loads, issued together
@@ -268,7 +212,7 @@ struct EpiMeanOdd {
         }
       }
     }
-    named_bar_sync(1, 128);  // the metadata is rewritten by the next tile
+    named_bar_sync(cx.bar, 128);  // the metadata is rewritten by the next tile
   }
 };
 
@@ -283,25 +227,28 @@ __host__ __device__ __forceinline__ int inv_row_to_dim(int p) {
 }
 
 // ------------------------------------------------------------------ inverse + RoPE + scatter
-// x = D * 2^-p_inv + mu[d]; keys get RoPE (rotate-half, base 1e7, position in prompt);
-// bf16 round-to-nearest-even; coalesced 16-byte stores into [6][tokens][2][256].
+// x = D * 2^-p_inv + mu[d]; keys get RoPE (rotate-half, base 1e7, position in prompt) with
+// cos / sin from a per-call table; bf16 round-to-nearest-even; coalesced 16-byte stores
+// into [6][tokens][2][256].  Chunks of 16 columns; the RoPE partner (row +-64) is read
+// through shared memory.
 struct EpiInverse {
   struct Params {
     const float *mu_perm;
     float scale;
-    const double *theta;
+    const float2 *rope;      // [positions][128] (cos, sin) of position * theta_i
     const int32_t *row_tok;  // [rows] token index in the batch
     const int32_t *row_pos;  // [rows] position within the prompt
     __nv_bfloat16 *k_out, *v_out;
     int64_t n_tokens;
   };
-  static constexpr int XCH_LD = 33;
-  static constexpr int SMEM_BYTES = 128 * XCH_LD * 4 + 32 * 128 * 2;
-  __device__ static void tile(const Params &p, char *scratch, int mt, int n0, int n_valid, int bn, uint32_t tacc,
-                              int ew, int lane, int et) {
-    float *xch = reinterpret_cast<float *>(scratch);
-    __nv_bfloat16 *ob = reinterpret_cast<__nv_bfloat16 *>(scratch + 128 * XCH_LD * 4);
-    const int ml = ew * 32 + lane;
+  static constexpr int CW = 16;
+  static constexpr int XCH_LD = CW + 1;
+  static constexpr int SMEM_BYTES = 128 * XCH_LD * 4 + CW * 128 * 2;
+  __device__ static void tile(const Params &p, const EpiCtx &cx) {
+    float *xch = reinterpret_cast<float *>(cx.scratch);
+    __nv_bfloat16 *ob = reinterpret_cast<__nv_bfloat16 *>(cx.scratch + 128 * XCH_LD * 4);
+    const int mt = cx.mt, n0 = cx.n0, n_valid = cx.n_valid, et = cx.et;
+    const int ml = cx.ew * 32 + cx.lane;
     const int hv = mt >> 1, half = mt & 1;
     const int layer = hv >> 2, kv = (hv >> 1) & 1, head = hv & 1;
     const bool first = ml < 64;
@@ -309,32 +256,34 @@ struct EpiInverse {
     const int fi = half * 64 + (ml & 63);  // frequency index of this row's pair
     const float mu = p.mu_perm[mt * GEMM_BM + ml];
     __nv_bfloat16 *dst_base = kv == 0 ? p.k_out : p.v_out;
-    for (int c0 = 0; c0 < n_valid; c0 += 32) {
-      uint32_t r[32];
-      tmem_ld_32x32b_x32(tacc + (uint32_t)c0, r);
+    for (int c0 = cx.grp * CW; c0 < n_valid; c0 += CW * cx.n_grp) {
+      uint32_t r[CW];
+      tmem_ld_32x32b_x16(cx.tacc + (uint32_t)c0, r);
       tmem_ld_wait();
-      float v[32];
+      float v[CW];
 #pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = u2f(r[j]) * p.scale + mu;
+      for (int j = 0; j < CW; ++j) v[j] = u2f(r[j]) * p.scale + mu;
       if (kv == 0) {
+        float2 cs[CW];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) xch[ml * XCH_LD + j] = v[j];
-        named_bar_sync(1, 128);
-#pragma unroll 4
-        for (int j = 0; j < 32; ++j) {
-          const float pv = xch[partner * XCH_LD + j];
+        for (int j = 0; j < CW; ++j) {
           const int row = min(n0 + c0 + j, n0 + n_valid - 1);
-          float cs, sn;
-          rope_cs(p.row_pos[row], fi, p.theta, cs, sn);
-          v[j] = first ? (v[j] * cs - pv * sn) : (v[j] * cs + pv * sn);
+          cs[j] = __ldg(p.rope + (int64_t)p.row_pos[row] * 128 + fi);
+          xch[ml * XCH_LD + j] = v[j];
+        }
+        named_bar_sync(cx.bar, 128);
+#pragma unroll
+        for (int j = 0; j < CW; ++j) {
+          const float pv = xch[partner * XCH_LD + j];
+          v[j] = first ? (v[j] * cs[j].x - pv * cs[j].y) : (v[j] * cs[j].x + pv * cs[j].y);
         }
       }
 #pragma unroll
-      for (int j = 0; j < 32; ++j) ob[j * 128 + ml] = __float2bfloat16_rn(v[j]);
-      named_bar_sync(1, 128);
-      // 32 tokens x 2 segments x 8 sixteen-byte chunks = 512 stores over 128 threads
+      for (int j = 0; j < CW; ++j) ob[j * 128 + ml] = __float2bfloat16_rn(v[j]);
+      named_bar_sync(cx.bar, 128);
+      // CW tokens x 2 segments x 8 sixteen-byte pieces over 128 threads
 #pragma unroll
-      for (int it = 0; it < 4; ++it) {
+      for (int it = 0; it < CW / 8; ++it) {
         const int qid = et + 128 * it;
         const int j = qid >> 4, sub = qid & 15, seg = sub >> 3, w = sub & 7;
         if (c0 + j < n_valid) {
@@ -344,7 +293,7 @@ struct EpiInverse {
           *reinterpret_cast<uint4 *>(dst_base + off) = *reinterpret_cast<const uint4 *>(ob + j * 128 + seg * 64 + w * 8);
         }
       }
-      named_bar_sync(1, 128);
+      named_bar_sync(cx.bar, 128);
     }
   }
 };

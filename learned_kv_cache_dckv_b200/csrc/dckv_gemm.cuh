@@ -49,6 +49,22 @@ struct GemmProblem {
   int *status;  // device int32; DCKV_ETIMEOUT (5) is written on a timed-out wait
 };
 
+// What an epilogue sees of one output tile.  The epilogue threads form groups of 128 (four
+// warps, one per TMEM lane quarter); group grp of n_grp takes the tile's column chunks k
+// with k % n_grp == grp (each epilogue fixes its chunk width), synchronises on named
+// barrier `bar` and owns `scratch` (Epi::SMEM_BYTES of shared memory).
+struct EpiCtx {
+  int mt;            // 128-row output-feature tile
+  int n0, n_valid;   // first token row of the tile, valid columns
+  int bn;            // tile width
+  uint32_t tacc;     // TMEM address of column 0 for this warp's lane quarter
+  int ew, lane;      // lane quarter (warp % 4), lane
+  int et;            // thread index in the group, 0..127
+  int grp, n_grp;
+  int bar;
+  char *scratch;
+};
+
 template <int MAX_SLABS, int BN_MAX = GEMM_MAX_BN>
 struct GemmSmem {
   static constexpr int STAGE_BYTES = MAX_SLABS * GEMM_SLAB_BYTES + BN_MAX * GEMM_BK * 2;
@@ -56,10 +72,9 @@ struct GemmSmem {
 
 // Epi must provide:
 //   struct Params;   static constexpr int SMEM_BYTES;
-//   __device__ static void tile(const Params&, char* scratch, int mt, int n0, int n_valid,
-//                               uint32_t tmem_acc, int ew, int lane, int et)
-// `tile` is called by all 128 epilogue threads (et = 0..127, ew = TMEM lane quarter) and
-// reads the accumulator for its rows with tcgen05.ld; it may use named barrier 1.
+//   __device__ static void tile(const Params&, const EpiCtx&)
+// `tile` is called by every thread of an epilogue group and reads the accumulator for its
+// rows with tcgen05.ld; here there is one group (named barrier 1).
 template <class Epi, int STAGES, int MAX_SLABS>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
@@ -200,7 +215,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       const int n0 = nt * prob.bn;
       const int n_valid = min(prob.bn, prob.n_rows - n0);
       const uint32_t tacc = tmem_base + ((uint32_t)(ew * 32) << 16) + (uint32_t)(acc * GEMM_MAX_BN);
-      Epi::tile(ep, epi_scratch, mt, n0, n_valid, prob.bn, tacc, ew, lane, et);
+      const EpiCtx cx{mt, n0, n_valid, prob.bn, tacc, ew, lane, et, 0, 1, 1, epi_scratch};
+      Epi::tile(ep, cx);
       tc_fence_before();
       mbar_arrive(&acc_empty[acc]);
       if (++acc == 2) {
@@ -221,6 +237,427 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 template <class Epi, int STAGES, int MAX_SLABS>
 constexpr int gemm_smem_bytes() {
   return 1024 /*align slack*/ + STAGES * GemmSmem<MAX_SLABS>::STAGE_BYTES + 1024 /*barriers*/ + Epi::SMEM_BYTES;
+}
+
+// ------------------------------------------------------------------------------------------
+// CTA-pair variant (cta_group::2).  A cluster of two CTAs owns a 256 x bn output tile: CTA
+// r holds A rows 128 r .. 128 r + 127 of the tile and B rows r bn/2 .. r bn/2 + bn/2 - 1, so
+// each SM stages half the B tile that a 1-CTA tile of the same width needs, and the pair
+// runs one M = 256 MMA per K step.  The leader (rank 0) waits for both halves on its own
+// full barrier, issues every MMA and commits to the barriers of both CTAs; each CTA drains
+// its own TMEM rows (feature tile 2 * pair_tile + r) with the same epilogue as above.
+// prob.m_tiles counts 128-row tiles and must be even; prob.bn <= 256, bn / 2 a multiple of 8.
+constexpr int GEMM_B_HALF_BYTES = (GEMM_MAX_BN / 2) * GEMM_BK * 2;  // 16 KiB
+
+template <int MAX_SLABS>
+struct Gemm2Smem {
+  static constexpr int STAGE_BYTES = MAX_SLABS * GEMM_SLAB_BYTES + GEMM_B_HALF_BYTES;
+};
+
+template <class Epi, int STAGES, int MAX_SLABS, int EPI_WARPS>
+__global__ void __launch_bounds__(64 + 32 * EPI_WARPS, 1)
+    gemm2_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
+                 const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
+                 const GemmProblem prob, const typename Epi::Params ep) {
+  extern __shared__ __align__(1024) uint8_t dyn_smem[];
+  constexpr int STAGE_BYTES = Gemm2Smem<MAX_SLABS>::STAGE_BYTES;
+  constexpr int N_GRP = EPI_WARPS / 4;
+  constexpr int EPI_SCRATCH = (Epi::SMEM_BYTES + 15) & ~15;
+  uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
+  uint8_t *stages = base;
+  uint64_t *full_bar = reinterpret_cast<uint64_t *>(base + STAGES * STAGE_BYTES);  // leader's counts both halves
+  uint64_t *empty_bar = full_bar + STAGES;
+  uint64_t *acc_full = empty_bar + STAGES;
+  uint64_t *acc_empty = acc_full + 2;  // leader's: one arrival per epilogue warp of either CTA
+  uint32_t *tmem_base_smem = reinterpret_cast<uint32_t *>(acc_empty + 2);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_base_smem + 1);
+  char *epi_scratch = reinterpret_cast<char *>(base + STAGES * STAGE_BYTES + 1024);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = blockIdx.x >> 1;
+  const int n_pairs = gridDim.x >> 1;
+  const int m_pairs = prob.m_tiles >> 1;
+  const int total_tiles = m_pairs * prob.n_tiles;
+  const int half_bn = prob.bn >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 2 * EPI_WARPS);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA0);
+    prefetch_tmap(&tmA1);
+    prefetch_tmap(&tmB0);
+    prefetch_tmap(&tmB1);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_base_smem, 512);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // both CTAs' barriers are initialised before any cross-CTA signal
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_base_smem;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer (both CTAs)
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = pair; t < total_tiles && ok; t += n_pairs) {
+        const int mp = t % m_pairs;
+        const int n0 = (t / m_pairs) * prob.bn;
+        for (int si = 0; si < prob.n_seg && ok; ++si) {
+          const GemmSeg sg = prob.seg[si];
+          const void *ta = sg.a_map ? (const void *)&tmA1 : (const void *)&tmA0;
+          const void *tb = sg.b_map ? (const void *)&tmB1 : (const void *)&tmB0;
+          const uint32_t bytes = (uint32_t)(sg.n_slab * GEMM_SLAB_BYTES + half_bn * GEMM_BK * 2);
+          for (int ks = 0; ks < sg.k_steps; ++ks) {
+            if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) {
+              ok = false;
+              break;
+            }
+            uint8_t *sa = stages + stage * STAGE_BYTES;
+            uint8_t *sb = sa + MAX_SLABS * GEMM_SLAB_BYTES;
+            const uint32_t fb = mapa_shared(smem_u32(&full_bar[stage]), 0);
+            if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * bytes);
+            tma_load_3d_pair(sa, ta, fb, sg.a_k0 + ks * GEMM_BK, (2 * mp + (int)rank) * GEMM_BM, sg.a_slab0);
+            tma_load_2d_pair(sb, tb, fb, sg.b_k0 + ks * GEMM_BK, n0 + (int)rank * half_bn + sg.b_row_shift);
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+        }
+      }
+      // wait until the leader has released every stage, so that no commit from it is
+      // still in flight towards this CTA's barriers when the CTA exits
+      for (int i = 0; i < STAGES && ok; ++i) {
+        if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) break;
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer (leader only)
+    if (lane == 0 && rank == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      for (int t = pair; t < total_tiles; t += n_pairs) {
+        if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * GEMM_MAX_BN);
+        uint32_t accumulate = 0;
+        bool ok = true;
+        for (int si = 0; si < prob.n_seg && ok; ++si) {
+          const GemmSeg sg = prob.seg[si];
+          for (int ks = 0; ks < sg.k_steps; ++ks) {
+            if (!mbar_wait(&full_bar[stage], phase, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t sa = smem_u32(stages + stage * STAGE_BYTES);
+            const uint32_t sb = sa + MAX_SLABS * GEMM_SLAB_BYTES;
+            for (int sl = 0; sl < sg.n_slab; ++sl) {
+#pragma unroll
+              for (int kk = 0; kk < GEMM_BK / 16; ++kk) {
+                umma_f16_pair(d_tmem, sw128_desc(sa + sl * GEMM_SLAB_BYTES + kk * 32), sw128_desc(sb + kk * 32),
+                              prob.idesc, accumulate);
+                accumulate = 1;
+              }
+            }
+            umma_commit_pair(&empty_bar[stage]);
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+        }
+        if (!ok) break;
+        umma_commit_pair(&acc_full[acc]);
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue (both CTAs)
+    const int grp = (warp - 2) >> 2;
+    const int et = threadIdx.x - 64 - 128 * grp;  // 0..127 within the group
+    const int ew = warp & 3;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = pair; t < total_tiles; t += n_pairs) {
+      if (et == 0) mbar_wait(&acc_full[acc], acc_phase, abort_flag);
+      named_bar_sync(1 + grp, 128);
+      if (*abort_flag) break;
+      tc_fence_after();
+      const int mp = t % m_pairs;
+      const int n0 = (t / m_pairs) * prob.bn;
+      const int n_valid = min(prob.bn, prob.n_rows - n0);
+      const uint32_t tacc = tmem_base + ((uint32_t)(ew * 32) << 16) + (uint32_t)(acc * GEMM_MAX_BN);
+      const EpiCtx cx{2 * mp + (int)rank, n0, n_valid, prob.bn, tacc, ew, lane, et, grp, N_GRP, 1 + grp,
+                      epi_scratch + grp * EPI_SCRATCH};
+      Epi::tile(ep, cx);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&acc_empty[acc]), 0));
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  }
+
+  __syncthreads();
+  cluster_sync();  // no CTA leaves while its peer may still signal its barriers or read TMEM
+  if (*abort_flag && threadIdx.x == 0 && prob.status) atomicExch(prob.status, 5);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, 512);
+  }
+}
+
+template <class Epi, int STAGES, int MAX_SLABS, int EPI_WARPS>
+constexpr int gemm2_smem_bytes() {
+  return 1024 + STAGES * Gemm2Smem<MAX_SLABS>::STAGE_BYTES + 1024 + (EPI_WARPS / 4) * ((Epi::SMEM_BYTES + 15) & ~15);
+}
+
+// ------------------------------------------------------------------------------------------
+// CTA-pair, chunk-accumulated variant (transform + quantiser).  Every CHUNK_STEPS * 64
+// elements of K go into a fresh TMEM partial P (two alternate, columns 0 and 256); the
+// eight epilogue warps of each CTA add each partial into running totals held in registers
+// (fp32 round-to-nearest adds, in chunk order) -- warp w >= 2 owns lane quarter w % 4 and
+// column half (w - 2) / 4, BN / 2 columns -- and after a tile's last chunk hand their totals
+// to Epi::finish.  Both P buffers stay free for the MMA while totals are finished.
+constexpr int GEMM2C_THREADS = 320;
+
+template <class Epi, int STAGES, int MAX_SLABS, int CHUNK_STEPS, int BN>
+__global__ void __launch_bounds__(GEMM2C_THREADS, 1)
+    gemm2_chunked_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
+                         const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
+                         const GemmProblem prob, const typename Epi::Params ep) {
+  static_assert(BN % 32 == 0 && BN <= GEMM_MAX_BN, "BN / 2 must be a multiple of 16");
+  constexpr int NC = BN / 2;  // columns per epilogue thread
+  extern __shared__ __align__(1024) uint8_t dyn_smem[];
+  constexpr int STAGE_BYTES = Gemm2Smem<MAX_SLABS>::STAGE_BYTES;
+  uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
+  uint8_t *stages = base;
+  uint64_t *full_bar = reinterpret_cast<uint64_t *>(base + STAGES * STAGE_BYTES);
+  uint64_t *empty_bar = full_bar + STAGES;
+  uint64_t *part_full = empty_bar + STAGES;
+  uint64_t *part_empty = part_full + 2;  // leader's: one arrival per epilogue warp of either CTA
+  uint32_t *tmem_base_smem = reinterpret_cast<uint32_t *>(part_empty + 2);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_base_smem + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = blockIdx.x >> 1;
+  const int n_pairs = gridDim.x >> 1;
+  const int m_pairs = prob.m_tiles >> 1;
+  const int total_tiles = m_pairs * prob.n_tiles;
+  constexpr int half_bn = BN / 2;
+  int ksteps = 0;
+  for (int si = 0; si < prob.n_seg; ++si) ksteps += prob.seg[si].k_steps;
+  const int n_chunks = (ksteps + CHUNK_STEPS - 1) / CHUNK_STEPS;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&part_full[a], 1);
+      mbar_init(&part_empty[a], 16);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA0);
+    prefetch_tmap(&tmA1);
+    prefetch_tmap(&tmB0);
+    prefetch_tmap(&tmB1);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_base_smem, 512);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_base_smem;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = pair; t < total_tiles && ok; t += n_pairs) {
+        const int mp = t % m_pairs;
+        const int n0 = (t / m_pairs) * BN;
+        for (int si = 0; si < prob.n_seg && ok; ++si) {
+          const GemmSeg sg = prob.seg[si];
+          const void *ta = sg.a_map ? (const void *)&tmA1 : (const void *)&tmA0;
+          const void *tb = sg.b_map ? (const void *)&tmB1 : (const void *)&tmB0;
+          const uint32_t bytes = (uint32_t)(sg.n_slab * GEMM_SLAB_BYTES + half_bn * GEMM_BK * 2);
+          for (int ks = 0; ks < sg.k_steps; ++ks) {
+            if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) {
+              ok = false;
+              break;
+            }
+            uint8_t *sa = stages + stage * STAGE_BYTES;
+            uint8_t *sb = sa + MAX_SLABS * GEMM_SLAB_BYTES;
+            const uint32_t fb = mapa_shared(smem_u32(&full_bar[stage]), 0);
+            if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * bytes);
+            tma_load_3d_pair(sa, ta, fb, sg.a_k0 + ks * GEMM_BK, (2 * mp + (int)rank) * GEMM_BM, sg.a_slab0);
+            tma_load_2d_pair(sb, tb, fb, sg.b_k0 + ks * GEMM_BK, n0 + (int)rank * half_bn + sg.b_row_shift);
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+        }
+      }
+      for (int i = 0; i < STAGES && ok; ++i) {
+        if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) break;
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int pb = 0;
+      uint32_t pph = 0;
+      bool ok = true;
+      for (int t = pair; t < total_tiles && ok; t += n_pairs) {
+        int in_chunk = 0, done = 0;
+        uint32_t d_tmem = 0, accumulate = 0;
+        for (int si = 0; si < prob.n_seg && ok; ++si) {
+          const GemmSeg sg = prob.seg[si];
+          for (int ks = 0; ks < sg.k_steps; ++ks) {
+            if (in_chunk == 0) {
+              if (!mbar_wait(&part_empty[pb], pph ^ 1u, abort_flag)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              d_tmem = tmem_base + (uint32_t)(pb * 256);
+              accumulate = 0;
+            }
+            if (!mbar_wait(&full_bar[stage], phase, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t sa = smem_u32(stages + stage * STAGE_BYTES);
+            const uint32_t sb = sa + MAX_SLABS * GEMM_SLAB_BYTES;
+            for (int sl = 0; sl < sg.n_slab; ++sl) {
+#pragma unroll
+              for (int kk = 0; kk < GEMM_BK / 16; ++kk) {
+                umma_f16_pair(d_tmem, sw128_desc(sa + sl * GEMM_SLAB_BYTES + kk * 32), sw128_desc(sb + kk * 32),
+                              prob.idesc, accumulate);
+                accumulate = 1;
+              }
+            }
+            umma_commit_pair(&empty_bar[stage]);
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+            ++done;
+            if (++in_chunk == CHUNK_STEPS || done == ksteps) {
+              umma_commit_pair(&part_full[pb]);
+              in_chunk = 0;
+              if (++pb == 2) {
+                pb = 0;
+                pph ^= 1u;
+              }
+            }
+          }
+        }
+      }
+    }
+  } else {
+    const int ew = warp & 3;
+    const int col0 = ((warp - 2) >> 2) * NC;
+    const uint32_t lane_base = (uint32_t)(ew * 32) << 16;
+    int pb = 0;
+    uint32_t pph = 0;
+    bool stop = false;
+    for (int t = pair; t < total_tiles && !stop; t += n_pairs) {
+      const int mp = t % m_pairs;
+      const int n0 = (t / m_pairs) * BN;
+      const int n_valid = min(BN, prob.n_rows - n0);
+      float tot[NC];
+#pragma unroll
+      for (int j = 0; j < NC; ++j) tot[j] = 0.f;
+      for (int ch = 0; ch < n_chunks; ++ch) {
+        if (!mbar_wait(&part_full[pb], pph, abort_flag)) {
+          stop = true;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t part = tmem_base + lane_base + (uint32_t)(pb * 256 + col0);
+#pragma unroll
+        for (int g = 0; g < NC / 16; g += 2) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x16(part + (uint32_t)(g * 16), r);
+          if (g + 1 < NC / 16) tmem_ld_32x32b_x16(part + (uint32_t)((g + 1) * 16), r + 16);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (g * 16 + j < NC) tot[g * 16 + j] += __uint_as_float(r[j]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&part_empty[pb]), 0));
+        if (++pb == 2) {
+          pb = 0;
+          pph ^= 1u;
+        }
+      }
+      if (stop) break;
+      Epi::template finish<NC>(ep, tot, 2 * mp + (int)rank, n0, n_valid, col0, ew, lane);
+    }
+  }
+
+  __syncthreads();
+  cluster_sync();
+  if (*abort_flag && threadIdx.x == 0 && prob.status) atomicExch(prob.status, 5);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, 512);
+  }
+}
+
+template <int STAGES, int MAX_SLABS>
+constexpr int gemm2_chunked_smem_bytes() {
+  return 1024 + STAGES * Gemm2Smem<MAX_SLABS>::STAGE_BYTES + 1024;
 }
 
 // ------------------------------------------------------------------------------------------

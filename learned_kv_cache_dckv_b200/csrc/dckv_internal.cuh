@@ -40,6 +40,11 @@ constexpr int BIG_CODE = 2048;            // |q| >= 2048 is not exact in the fp1
 constexpr float REFINE_KAPPA = 5.0e-7f;  // measured fp32 error on B200: <= 1.7e-7 * |x|_2
 constexpr float REFINE_W0 = 2.0e-5f;
 constexpr float REFINE_NORM_FULL = 32.0f;
+// GEMM tile widths (tokens per CTA-pair tile): 224 keeps the transform's 8 x ceil(n / 224)
+// pair tiles close to a whole number of waves over 74 pairs for 4K-token prompts.
+constexpr int TRANSFORM_BN = 224;
+constexpr int MEAN_ODD_BN = 224;
+constexpr int INVERSE_BN = 224;
 
 struct PromptInfo {
   int64_t tok_base;  // first row (token) of the prompt in the batch
@@ -66,6 +71,7 @@ struct Layout {
   int64_t n_rows = 0;     // coded rows
   int64_t ne_pad = 0;     // padded even rows (sum of n_e + 1)
   int64_t n_kept = 0;
+  int64_t max_len = 0;    // longest prompt (RoPE table positions)
   int n_chunks = 0, n_chunks_e = 0, n_chunks_o = 0;
   int64_t n_symbols = 0;  // n_rows * K_eff
   std::vector<PromptInfo> prompts;
@@ -79,6 +85,7 @@ struct WsPlan {
   size_t qe, cen8;                                                               // both
   size_t x16, g16, q32, sym16, cf32, words, states, nwords, nesc, offs;           // encode
   size_t slots16;  // decode: decoded symbols (slot order)
+  size_t rope;     // decode: float2 [max_len][128] RoPE (cos, sin)
   size_t row_norm, rowflag, el_list, full_list;                         // encode refinement
   int64_t el_cap;
   size_t q16, qbig, bigflag, biglist, counters, valid;                  // decode
