@@ -66,6 +66,10 @@ int dckv_debug_ratio(dckv_codec *codec, void *ratio_dev);
 int dckv_set_timing(dckv_codec *codec, int enable);
 int dckv_get_timing(const dckv_codec *codec, float *ms, const char **names, int max);
 
+/* Kernels this library has launched in this process so far (every codec and device;
+ * codec creation included).  Benchmarks read it before and after a timed region. */
+long long dckv_launch_count(void);
+
 /* Self-test of the tcgen05 GEMM core: D[n][m] = sum_s sum_k A[s][m][k] * B[n][k]
  * (fp32 accumulate).  A: device fp16/bf16 [slabs][M][K]; B: device [N][K]; D: device
  * fp32 [N][M].  M % 128 == 0, K % 64 == 0, slabs in {1, 2}, bn (N tile) in 16..256 step 16.

@@ -86,6 +86,7 @@ def lib():
         "dckv_debug_gemm": (I, [I, P, I, P, I, I, I, P, I, I, P]),
         "dckv_debug_ratio": (I, [P, P]),
         "dckv_codec_info": (I, [P, P, P]),
+        "dckv_launch_count": (ctypes.c_longlong, []),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -183,6 +184,10 @@ def dckv_decode_static(handle, blob, blob_bytes, token_ids, seq_offsets, k_out, 
     _check(lib().dckv_decode_static(handle, blob.data_ptr(), int(blob_bytes), token_ids.data_ptr(), ptr, b,
                                     k_out.data_ptr(), v_out.data_ptr(), status.data_ptr(), _stream_ptr(stream)),
            "dckv_decode_static")
+
+
+def dckv_launch_count() -> int:
+    return int(lib().dckv_launch_count())
 
 
 def dckv_bytes(blob_host: bytes) -> dict:

@@ -17,6 +17,7 @@
 //          --rANS odd--> odd codes --GEMM inverse (RoPE + scatter epilogue)--> K, V
 //          (+ kept rows with RoPE, + exact fix-up of rows holding codes beyond +-2047)
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -30,6 +31,9 @@
 #include "dckv_gemm.cuh"
 #include "dckv_internal.cuh"
 #include "dckv_rans.cuh"
+
+// Kernels launched by this library in this process (all codecs, all devices).
+static std::atomic<long long> g_launches{0};
 
 using namespace dckv;
 
@@ -119,7 +123,7 @@ static int run_gemm(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensor
   for (int i = 0; i < prob.n_seg; ++i)
     if (prob.seg[i].n_slab < 1 || prob.seg[i].n_slab > MAX_SLABS) return fail(DCKV_EINVAL, "bad slab count");
   const int grid = std::min(tiles, num_sms);
-  kern<<<grid, GEMM_THREADS, smem, st>>>(a0, a1, b0, b1, prob, ep);
+  { kern<<<grid, GEMM_THREADS, smem, st>>>(a0, a1, b0, b1, prob, ep); ++g_launches; }
   CK(cudaGetLastError());
   return DCKV_OK;
 }
@@ -140,6 +144,7 @@ static int launch_pairs(const void *kern, int tiles, int num_sms, int threads, i
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   CK(cudaLaunchKernelExC(&cfg, kern, args));
+  ++g_launches;
   return DCKV_OK;
 }
 
@@ -165,7 +170,7 @@ template <class Epi, int STAGES, int MAX_SLABS, int CHUNK_STEPS, int BN>
 static int run_gemm2_chunked(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &b0,
                              const CUtensorMap &b1, GemmProblem prob, const typename Epi::Params &ep, int num_sms,
                              bool bf16, cudaStream_t st) {
-  constexpr int smem = gemm2_chunked_smem_bytes<STAGES, MAX_SLABS>();
+  constexpr int smem = gemm2_chunked_smem_bytes<Epi, STAGES, MAX_SLABS>();
   static_assert(smem <= 232448, "GEMM shared memory above the sm_100 limit");
   auto kern = gemm2_chunked_kernel<Epi, STAGES, MAX_SLABS, CHUNK_STEPS, BN>;
   CK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
@@ -194,7 +199,7 @@ static int run_gemm_chunked(const CUtensorMap &a0, const CUtensorMap &a1, const 
   for (int i = 0; i < prob.n_seg; ++i)
     if (prob.seg[i].n_slab < 1 || prob.seg[i].n_slab > MAX_SLABS) return fail(DCKV_EINVAL, "bad slab count");
   const int grid = std::min(tiles, num_sms);
-  kern<<<grid, GEMMC_THREADS, smem, st>>>(a0, a1, b0, b1, prob, ep);
+  { kern<<<grid, GEMMC_THREADS, smem, st>>>(a0, a1, b0, b1, prob, ep); ++g_launches; }
   CK(cudaGetLastError());
   return DCKV_OK;
 }
@@ -354,26 +359,30 @@ __global__ void k_permute_mu(const float *mu, float *mu_perm) {
 
 // ============================================================================ per-call kernels
 // Row tables of one prompt per block: coded row r = row_base + i holds position 4 + i.
+// Grid (prompts, LAYOUT_SPLIT): the blocks of one prompt share its rows.
+constexpr int LAYOUT_SPLIT = 8;
+
 __global__ void k_layout(const PromptInfo *prompts, int32_t *row_tok, int32_t *row_pos, int32_t *row_edst,
                          int32_t *row_slot, int32_t *e_tok, int32_t *e_slot, int32_t *slot_chunk, int chunk_rows,
                          __nv_bfloat16 *qe_zero_pad) {
   const PromptInfo pi = prompts[blockIdx.x];
-  for (int j = threadIdx.x; j < pi.n_e; j += blockDim.x) slot_chunk[pi.slot_e0 + j] = pi.chunk_e0 + j / chunk_rows;
-  for (int j = threadIdx.x; j < pi.n_o; j += blockDim.x) slot_chunk[pi.slot_o0 + j] = pi.chunk_o0 + j / chunk_rows;
-  for (int i = threadIdx.x; i < pi.n; i += blockDim.x) {
+  const int t0 = blockIdx.y * blockDim.x + threadIdx.x, ts = gridDim.y * blockDim.x;
+  for (int j = t0; j < pi.n_e; j += ts) slot_chunk[pi.slot_e0 + j] = pi.chunk_e0 + j / chunk_rows;
+  for (int j = t0; j < pi.n_o; j += ts) slot_chunk[pi.slot_o0 + j] = pi.chunk_o0 + j / chunk_rows;
+  for (int i = t0; i < pi.n; i += ts) {
     const int r = pi.row_base + i;
     row_tok[r] = (int32_t)(pi.tok_base + HEAD_KEPT + i);
     row_pos[r] = HEAD_KEPT + i;
     row_edst[r] = (i & 1) ? -1 : pi.ebase + (i >> 1);
     row_slot[r] = (i & 1) ? pi.slot_o0 + (i >> 1) : pi.slot_e0 + (i >> 1);
   }
-  for (int e = threadIdx.x; e <= pi.n_e; e += blockDim.x) {
+  for (int e = t0; e <= pi.n_e; e += ts) {
     const bool odd = e < pi.n_o;
     e_tok[pi.ebase + e] = odd ? (int32_t)(pi.tok_base + HEAD_KEPT + 2 * e + 1) : -1;
     e_slot[pi.ebase + e] = odd ? pi.slot_o0 + e : 0;
   }
   if (qe_zero_pad)  // the row after a prompt's last even row is its odd rows' zero right neighbour
-    for (int k = threadIdx.x; k < N_COEF; k += blockDim.x)
+    for (int k = t0; k < N_COEF; k += ts)
       qe_zero_pad[(int64_t)(pi.ebase + pi.n_e) * N_COEF + k] = __float2bfloat16_rn(0.f);
 }
 
@@ -402,9 +411,14 @@ __global__ void __launch_bounds__(192) k_convert(const __nv_bfloat16 *rows, cons
     uint4 *dst = reinterpret_cast<uint4 *>(x16 + (int64_t)(pi.row_base + p - HEAD_KEPT) * ROW_DIM);
     bool clamped = false;
     float ss = 0.f;
-    for (int v = threadIdx.x; v < ROW_DIM / 8; v += blockDim.x) {
-      uint4 in = src[v];
-      const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&in);
+    constexpr int PER = ROW_DIM / 8 / 192;  // 4 sixteen-byte pieces per thread, loaded together
+    uint4 inb[PER];
+#pragma unroll
+    for (int u = 0; u < PER; ++u) inb[u] = __ldg(src + threadIdx.x + u * 192);
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+      const int v = threadIdx.x + u * 192;
+      const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&inb[u]);
       uint4 o;
       __half2 *oh = reinterpret_cast<__half2 *>(&o);
 #pragma unroll
@@ -433,7 +447,11 @@ __global__ void __launch_bounds__(192) k_convert(const __nv_bfloat16 *rows, cons
     const uint64_t off = off_kept + (uint64_t)(pi.kept_base + kidx) * (ROW_DIM * 2);
     if (off + ROW_DIM * 2 > blob_cap) return;
     uint4 *dst = reinterpret_cast<uint4 *>(blob + off);
-    for (int v = threadIdx.x; v < ROW_DIM / 8; v += blockDim.x) dst[v] = src[v];
+    uint4 inb[ROW_DIM / 8 / 192];
+#pragma unroll
+    for (int u = 0; u < ROW_DIM / 8 / 192; ++u) inb[u] = __ldg(src + threadIdx.x + u * 192);
+#pragma unroll
+    for (int u = 0; u < ROW_DIM / 8 / 192; ++u) dst[threadIdx.x + u * 192] = inb[u];
   }
 }
 
@@ -872,7 +890,7 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
   const uint64_t o_lut = take(2ull * N_SCALES * LUT_SIZE);
   const uint64_t o_tail = take(4ull * N_SCALES);
   const uint64_t o_dcdf = take(2ull * N_SCALES * DEC_CDF_STRIDE);
-  const uint64_t o_rcp = take(4ull * N_SCALES * N_SYM);
+  const uint64_t o_cfm = take(8ull * N_SCALES * N_SYM);
   const uint64_t o_kidx = take(2ull * N_COEF);
   const uint64_t o_theta = take(8ull * 128);
   const uint64_t o_bt32 = take(4ull * N_COEF * ROW_DIM);
@@ -902,7 +920,7 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
   c->lut = (uint16_t *)(B + o_lut);
   c->tail = (uint32_t *)(B + o_tail);
   c->dcdf = (uint16_t *)(B + o_dcdf);
-  c->rcp = (uint32_t *)(B + o_rcp);
+  c->cfm_tab = (uint2 *)(B + o_cfm);
   c->kidx = (int16_t *)(B + o_kidx);
   c->theta = (double *)(B + o_theta);
   c->bt32 = (float *)(B + o_bt32);
@@ -916,15 +934,15 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
 
   if (cudaMemset(scr, 0, 64) != cudaSuccess) return cleanup(fail(DCKV_ECUDA, "memset"));
   // drop mask, scale index, tables
-  k_scale_keep<<<(N_COEF + 255) / 256, 256, 0, st>>>(prm->laplace_b, prm->delta, c->scale, c->keep, scr);
-  k_tables<<<N_SCALES, 512, 0, st>>>(c->cdf);
-  k_build_lut<<<N_SCALES, 256, 0, st>>>(c->cdf, c->dcdf, c->lut, c->tail, c->rcp);
+  { k_scale_keep<<<(N_COEF + 255) / 256, 256, 0, st>>>(prm->laplace_b, prm->delta, c->scale, c->keep, scr); ++g_launches; }
+  { k_tables<<<N_SCALES, 512, 0, st>>>(c->cdf); ++g_launches; }
+  { k_build_lut<<<N_SCALES, 256, 0, st>>>(c->cdf, c->dcdf, c->lut, c->tail, c->cfm_tab); ++g_launches; }
   cudaMemcpyAsync(c->delta, prm->delta, 4ull * N_COEF, cudaMemcpyDeviceToDevice, st);
   // scale exponents: largest |value| of each split operand brought to about 2^12
-  k_absmax<<<256, 256, 0, st>>>(prm->basis, (int64_t)ROW_DIM * N_COEF, N_COEF, nullptr, scr + 1);
-  k_absmax<<<64, 256, 0, st>>>(prm->w2, (int64_t)N_HIDDEN * N_COEF, N_COEF, nullptr, scr + 2);
-  k_absmax<<<256, 256, 0, st>>>(prm->w1, (int64_t)ROW_DIM * N_HIDDEN, N_HIDDEN, nullptr, scr + 3);
-  k_absmax<<<256, 256, 0, st>>>(prm->basis, (int64_t)ROW_DIM * N_COEF, N_COEF, prm->delta, scr + 4);
+  { k_absmax<<<256, 256, 0, st>>>(prm->basis, (int64_t)ROW_DIM * N_COEF, N_COEF, nullptr, scr + 1); ++g_launches; }
+  { k_absmax<<<64, 256, 0, st>>>(prm->w2, (int64_t)N_HIDDEN * N_COEF, N_COEF, nullptr, scr + 2); ++g_launches; }
+  { k_absmax<<<256, 256, 0, st>>>(prm->w1, (int64_t)ROW_DIM * N_HIDDEN, N_HIDDEN, nullptr, scr + 3); ++g_launches; }
+  { k_absmax<<<256, 256, 0, st>>>(prm->basis, (int64_t)ROW_DIM * N_COEF, N_COEF, prm->delta, scr + 4); ++g_launches; }
   int32_t host_scr[8];
   uint8_t keep_h[N_COEF], scale_h[N_COEF];
   if (cudaMemcpy(host_scr, scr, 32, cudaMemcpyDeviceToHost) != cudaSuccess ||
@@ -995,25 +1013,25 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
       cudaMemcpy(c->theta, theta_h, sizeof(theta_h), cudaMemcpyHostToDevice) != cudaSuccess)
     return cleanup(fail(DCKV_ECUDA, "setup upload failed"));
   // mean projections in fp64
-  k_vec_mat<<<(N_COEF + 255) / 256, 256, 0, st>>>(prm->mu, prm->basis, ROW_DIM, N_COEF, c->mub);
-  k_vec_mat<<<1, 256, 0, st>>>(prm->mu, prm->w1, ROW_DIM, N_HIDDEN, c->muw1);
-  k_permute_mu<<<(ROW_DIM + 255) / 256, 256, 0, st>>>(prm->mu, c->mu_perm);
+  { k_vec_mat<<<(N_COEF + 255) / 256, 256, 0, st>>>(prm->mu, prm->basis, ROW_DIM, N_COEF, c->mub); ++g_launches; }
+  { k_vec_mat<<<1, 256, 0, st>>>(prm->mu, prm->w1, ROW_DIM, N_HIDDEN, c->muw1); ++g_launches; }
+  { k_permute_mu<<<(ROW_DIM + 255) / 256, 256, 0, st>>>(prm->mu, c->mu_perm); ++g_launches; }
   // split operands (hi/lo fp16, power-of-two scaled)
   dim3 tb(32, 8);
-  k_split<<<dim3(ROW_DIM / 32, N_COEF / 32), tb, 0, st>>>(prm->basis, N_COEF, ROW_DIM, 0, nullptr, std::ldexp(1.0, c->p_y), c->a_y);
-  k_split<<<dim3(N_HIDDEN / 32, N_COEF / 32), tb, 0, st>>>(prm->w2, N_COEF, N_HIDDEN, 0, nullptr, std::ldexp(1.0, c->p_y), c->a_w2);
-  k_split<<<dim3(ROW_DIM / 32, N_HIDDEN / 32), tb, 0, st>>>(prm->w1, N_HIDDEN, ROW_DIM, 0, nullptr, std::ldexp(1.0, c->p_h), c->a_h);
-  k_split<<<dim3(N_COEF / 32, ROW_DIM / 32), tb, 0, st>>>(prm->basis, ROW_DIM, N_COEF, 1, prm->delta, std::ldexp(1.0, c->p_inv), c->a_inv);
+  { k_split<<<dim3(ROW_DIM / 32, N_COEF / 32), tb, 0, st>>>(prm->basis, N_COEF, ROW_DIM, 0, nullptr, std::ldexp(1.0, c->p_y), c->a_y); ++g_launches; }
+  { k_split<<<dim3(N_HIDDEN / 32, N_COEF / 32), tb, 0, st>>>(prm->w2, N_COEF, N_HIDDEN, 0, nullptr, std::ldexp(1.0, c->p_y), c->a_w2); ++g_launches; }
+  { k_split<<<dim3(ROW_DIM / 32, N_HIDDEN / 32), tb, 0, st>>>(prm->w1, N_HIDDEN, ROW_DIM, 0, nullptr, std::ldexp(1.0, c->p_h), c->a_h); ++g_launches; }
+  { k_split<<<dim3(N_COEF / 32, ROW_DIM / 32), tb, 0, st>>>(prm->basis, ROW_DIM, N_COEF, 1, prm->delta, std::ldexp(1.0, c->p_inv), c->a_inv); ++g_launches; }
   // fp32 copies for the exact refinement
-  k_transpose32<<<dim3(ROW_DIM / 32, N_COEF / 32), tb, 0, st>>>(prm->basis, ROW_DIM, N_COEF, c->bt32);
-  k_transpose32<<<dim3(ROW_DIM / 32, N_HIDDEN / 32), tb, 0, st>>>(prm->w1, ROW_DIM, N_HIDDEN, c->w1t32);
-  k_transpose32<<<dim3(N_HIDDEN / 32, N_COEF / 32), tb, 0, st>>>(prm->w2, N_HIDDEN, N_COEF, c->w2t32);
+  { k_transpose32<<<dim3(ROW_DIM / 32, N_COEF / 32), tb, 0, st>>>(prm->basis, ROW_DIM, N_COEF, c->bt32); ++g_launches; }
+  { k_transpose32<<<dim3(ROW_DIM / 32, N_HIDDEN / 32), tb, 0, st>>>(prm->w1, ROW_DIM, N_HIDDEN, c->w1t32); ++g_launches; }
+  { k_transpose32<<<dim3(N_HIDDEN / 32, N_COEF / 32), tb, 0, st>>>(prm->w2, N_HIDDEN, N_COEF, c->w2t32); ++g_launches; }
   cudaMemcpyAsync(c->mu32, prm->mu, 4ull * ROW_DIM, cudaMemcpyDeviceToDevice, st);
   // mean-model weights, K-major
-  k_transpose16<<<dim3(2 * N_COEF / 32, N_COEF / 32), tb, 0, st>>>(prm->w_odd, N_COEF, N_COEF, N_COEF, 2 * N_COEF,
-                                                                   (uint16_t *)c->a_on);
-  k_transpose16<<<dim3(N_COEF / 32, N_COEF / 32), tb, 0, st>>>(prm->w_even, N_COEF, 0, N_COEF, N_COEF, tmp_e);
-  k_transpose16<<<dim3(N_COEF / 32, N_COEF / 32), tb, 0, st>>>(prm->w_odd, N_COEF, 0, N_COEF, N_COEF, tmp_oe);
+  { k_transpose16<<<dim3(2 * N_COEF / 32, N_COEF / 32), tb, 0, st>>>(prm->w_odd, N_COEF, N_COEF, N_COEF, 2 * N_COEF,
+                                                                   (uint16_t *)c->a_on); ++g_launches; }
+  { k_transpose16<<<dim3(N_COEF / 32, N_COEF / 32), tb, 0, st>>>(prm->w_even, N_COEF, 0, N_COEF, N_COEF, tmp_e); ++g_launches; }
+  { k_transpose16<<<dim3(N_COEF / 32, N_COEF / 32), tb, 0, st>>>(prm->w_odd, N_COEF, 0, N_COEF, N_COEF, tmp_oe); ++g_launches; }
   if (cudaGetLastError() != cudaSuccess) return cleanup(fail(DCKV_ECUDA, "setup kernels failed to launch"));
   // tensor maps of the static operands
   int r = DCKV_OK;
@@ -1124,11 +1142,11 @@ extern "C" int dckv_encode(const dckv_codec *c, const void *rows, const int32_t 
   if (L.n_rows) CK(cudaMemsetAsync(rowflag, 0, 4ull * L.n_rows, st));
   if (L.n_chunks) CK(cudaMemsetAsync(nesc_w, 0, 4ull * L.n_chunks, st));
   RET(upload_tables(L, ws, w, st));
-  k_layout<<<L.batch, 256, 0, st>>>(d_prompts, row_tok, row_pos, row_edst, row_slot, e_tok, e_slot, slot_chunk,
-                                    c->chunk_rows, qe);
+  { k_layout<<<dim3(L.batch, LAYOUT_SPLIT), 256, 0, st>>>(d_prompts, row_tok, row_pos, row_edst, row_slot, e_tok, e_slot, slot_chunk,
+                                    c->chunk_rows, qe); ++g_launches; }
   if (L.n_tokens > 0)
-    k_convert<<<(unsigned)L.n_tokens, 192, 0, st>>>((const __nv_bfloat16 *)rows, d_prompts, L.batch, x16, bl, blob_cap,
-                                                    L.off_kept, row_norm, status_dev);
+    { k_convert<<<(unsigned)L.n_tokens, 192, 0, st>>>((const __nv_bfloat16 *)rows, d_prompts, L.batch, x16, bl, blob_cap,
+                                                    L.off_kept, row_norm, status_dev); ++g_launches; }
   CK(cudaGetLastError());
   stage_mark(c, st, "layout+convert");
   if (L.n_rows > 0) {
@@ -1154,18 +1172,18 @@ extern "C" int dckv_encode(const dckv_codec *c, const void *rows, const int32_t 
       add_seg(pr, 1, 0, 2, 0, 1, 0, N_HIDDEN, N_HIDDEN / GEMM_BK);
       EpiQuantRegs::Params ep{{c->mub, c->delta, c->keep, (float)std::ldexp(1.0, -c->p_y), q32, qe, row_edst},
                               row_norm, rowflag, el_list, full_list, counters, w.el_cap, c->dbg_ratio};
-      RET((run_gemm2_chunked<EpiQuantRegs, 4, 2, 4, TRANSFORM_BN>(c->map_ay2, c->map_aw2_2, mb_xt, mb_gt, pr, ep,
+      RET((run_gemm2_chunked<EpiQuantRegs, 4, 2, TRANSFORM_CHUNK_STEPS, TRANSFORM_BN>(c->map_ay2, c->map_aw2_2, mb_xt, mb_gt, pr, ep,
                                                                    c->num_sms, false, st)));
     }
     stage_mark(c, st, "gemm_transform");
     // codes whose fp32 ratio lies in the guard band around a half step: exact fp64 values
-    k_refine_codes<<<c->num_sms * 4, 256, 0, st>>>(el_list, counters, w.el_cap, (const __nv_bfloat16 *)rows, row_tok,
+    { k_refine_codes<<<c->num_sms * 4, 256, 0, st>>>(el_list, counters, w.el_cap, (const __nv_bfloat16 *)rows, row_tok,
                                                   c->mu32, c->bt32, c->w2t32, g16, c->delta, rowflag, q32, qe,
-                                                  row_edst);
+                                                  row_edst); ++g_launches; }
     const int rsmem = (ROW_DIM + N_HIDDEN) * 8;
     CK(cudaFuncSetAttribute(k_refine_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, rsmem));
-    k_refine_rows<<<c->num_sms, 256, rsmem, st>>>(full_list, counters, (const __nv_bfloat16 *)rows, row_tok, c->mu32,
-                                                  c->bt32, c->w1t32, c->w2t32, c->delta, c->keep, q32, qe, row_edst);
+    { k_refine_rows<<<c->num_sms, 256, rsmem, st>>>(full_list, counters, (const __nv_bfloat16 *)rows, row_tok, c->mu32,
+                                                  c->bt32, c->w1t32, c->w2t32, c->delta, c->keep, q32, qe, row_edst); ++g_launches; }
     CK(cudaGetLastError());
     stage_mark(c, st, "refine");
     // odd mean model: [e, bf16(q_left), bf16(q_right)] @ w_odd -> centres
@@ -1179,10 +1197,10 @@ extern "C" int dckv_encode(const dckv_codec *c, const void *rows, const int32_t 
     stage_mark(c, st, "gemm_mean_odd");
     // even centres from the vocabulary table, then every symbol, in slot order
     const unsigned rg = (unsigned)std::min<int64_t>(L.n_rows, 65535);
-    k_centres_even<<<rg, 256, 0, st>>>(L.n_rows, row_slot, row_edst, row_tok, token_ids, c->t_even, c->vocab,
-                                       c->kept_list, c->k_eff, cen8, nullptr);
-    k_symbols<<<rg, 256, 0, st>>>(L.n_rows, row_slot, slot_chunk, q32, cen8, c->kept_list, c->kept_scale, c->cdf,
-                                  c->rcp, c->k_eff, sym16, cfm, nesc_w);
+    { k_centres_even<<<rg, 256, 0, st>>>(L.n_rows, row_slot, row_edst, row_tok, token_ids, c->t_even, c->vocab,
+                                       c->kept_list, c->k_eff, cen8, nullptr); ++g_launches; }
+    { k_symbols<<<rg, SYM_THREADS, 0, st>>>(L.n_rows, row_slot, slot_chunk, q32, cen8, c->kept_list, c->kept_scale,
+                                          c->cfm_tab, c->k_eff, sym16, cfm, nesc_w); ++g_launches; }
     CK(cudaGetLastError());
     stage_mark(c, st, "symbols");
   }
@@ -1190,20 +1208,20 @@ extern "C" int dckv_encode(const dckv_codec *c, const void *rows, const int32_t 
   uint32_t *nesc = (uint32_t *)(ws + w.nesc), *offs = (uint32_t *)(ws + w.offs);
   if (L.n_chunks > 0) {
     RansEncArgs a{d_chunks, L.n_chunks, c->k_eff, cfm, (uint16_t *)(ws + w.words), states, nwords};
-    rans_encode_kernel<<<(L.n_chunks + RANS_WARPS - 1) / RANS_WARPS, RANS_WARPS * 32, 0, st>>>(a);
+    { rans_encode_kernel<<<(L.n_chunks + RANS_WARPS - 1) / RANS_WARPS, RANS_WARPS * 32, 0, st>>>(a); ++g_launches; }
     CK(cudaGetLastError());
   }
   stage_mark(c, st, "rans_encode");
   {
     ScanArgs a{L.n_chunks, nwords, nesc, offs, bl, blob_cap, L.off_kept, L.off_streams, d_prompts, L.batch,
                c->chunk_rows, c->k_eff, L.n_chunks_e, L.n_chunks_o, L.n_kept, blob_size_dev, status_dev};
-    scan_kernel<<<1, 1024, 0, st>>>(a);
+    { scan_kernel<<<1, 1024, 0, st>>>(a); ++g_launches; }
     CK(cudaGetLastError());
   }
   if (L.n_chunks > 0) {
     CompactArgs a{d_chunks, d_prompts, L.n_chunks, c->k_eff, c->kept_list, q32, sym16,
                   (const uint16_t *)(ws + w.words), states, nwords, nesc, offs, bl, blob_cap, L.off_streams};
-    compact_kernel<<<(L.n_chunks + RANS_WARPS - 1) / RANS_WARPS, RANS_WARPS * 32, 0, st>>>(a);
+    { compact_kernel<<<L.n_chunks, COMPACT_THREADS, 0, st>>>(a); ++g_launches; }
     CK(cudaGetLastError());
   }
   stage_mark(c, st, "scan+compact");
@@ -1254,19 +1272,19 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
     CK(cudaMemsetAsync(q16, 0, 2ull * L.n_rows * N_COEF, st));
     CK(cudaMemsetAsync(bigflag, 0, 4ull * L.n_rows, st));
   }
-  k_layout<<<L.batch, 256, 0, st>>>(d_prompts, row_tok, row_pos, row_edst, row_slot, e_tok, e_slot, slot_chunk,
-                                    c->chunk_rows, nullptr);
+  { k_layout<<<dim3(L.batch, LAYOUT_SPLIT), 256, 0, st>>>(d_prompts, row_tok, row_pos, row_edst, row_slot, e_tok, e_slot, slot_chunk,
+                                    c->chunk_rows, nullptr); ++g_launches; }
   HeaderCheck hc{bl, blob_bytes, d_prompts, L.batch, c->chunk_rows, c->k_eff, L.n_chunks_e, L.n_chunks_o,
                  L.n_kept, L.off_kept, L.off_streams, valid, status_dev};
-  k_check_header<<<1, 256, 0, st>>>(hc);
+  { k_check_header<<<1, 256, 0, st>>>(hc); ++g_launches; }
   if (L.n_rows > 0)
-    k_rope_table<<<(unsigned)std::min<int64_t>(L.max_len, 4096), 128, 0, st>>>(rope, L.max_len, c->theta, valid);
+    { k_rope_table<<<(unsigned)std::min<int64_t>(L.max_len, 4096), 128, 0, st>>>(rope, L.max_len, c->theta, valid); ++g_launches; }
   CK(cudaGetLastError());
   stage_mark(c, st, "layout+check");
   const uint32_t *offs = (const uint32_t *)(bl + HEADER_BYTES + 4ull * L.batch);
   if (L.n_rows > 0)
-    k_centres_even<<<(unsigned)std::min<int64_t>(L.n_rows, 65535), 256, 0, st>>>(
-        L.n_rows, row_slot, row_edst, row_tok, token_ids, c->t_even, c->vocab, c->kept_list, c->k_eff, cen8, valid);
+    { k_centres_even<<<(unsigned)std::min<int64_t>(L.n_rows, 65535), 256, 0, st>>>(
+        L.n_rows, row_slot, row_edst, row_tok, token_ids, c->t_even, c->vocab, c->kept_list, c->k_eff, cen8, valid); ++g_launches; }
   CK(cudaFuncSetAttribute(rans_decode_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, RANS_DEC_SMEM));
   CK(cudaFuncSetAttribute(rans_decode_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, RANS_DEC_SMEM));
   RansDecArgs da{d_chunks, 0, L.n_chunks, c->k_eff, c->kept_scale, c->dcdf, c->lut, c->tail, bl, L.off_streams,
@@ -1276,14 +1294,14 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
   if (L.n_chunks > 0) {
     const unsigned g = (L.n_chunks + RANS_WARPS - 1) / RANS_WARPS;
     if (c->k_eff >= 32)
-      rans_decode_kernel<true><<<g, RANS_WARPS * 32, RANS_DEC_SMEM, st>>>(da);
+      { rans_decode_kernel<true><<<g, RANS_WARPS * 32, RANS_DEC_SMEM, st>>>(da); ++g_launches; }
     else
-      rans_decode_kernel<false><<<g, RANS_WARPS * 32, RANS_DEC_SMEM, st>>>(da);
+      { rans_decode_kernel<false><<<g, RANS_WARPS * 32, RANS_DEC_SMEM, st>>>(da); ++g_launches; }
   }
   CK(cudaGetLastError());
   stage_mark(c, st, "rans_loop");
   if (L.n_chunks_e > 0)
-    k_decode_codes<<<(unsigned)L.n_chunks_e, DEC_CODES_THREADS, 0, st>>>(fa);
+    { k_decode_codes<<<(unsigned)L.n_chunks_e, DEC_CODES_THREADS, 0, st>>>(fa); ++g_launches; }
   CK(cudaGetLastError());
   stage_mark(c, st, "codes_even");
   if (L.n_rows > 0) {
@@ -1299,7 +1317,7 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
   if (L.n_chunks_o > 0) {
     fa.chunk0 = L.n_chunks_e;
     fa.n_chunks = L.n_chunks_o;
-    k_decode_codes<<<(unsigned)L.n_chunks_o, DEC_CODES_THREADS, 0, st>>>(fa);
+    { k_decode_codes<<<(unsigned)L.n_chunks_o, DEC_CODES_THREADS, 0, st>>>(fa); ++g_launches; }
     CK(cudaGetLastError());
   }
   stage_mark(c, st, "codes_odd");
@@ -1314,12 +1332,12 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
   }
   stage_mark(c, st, "gemm_inverse");
   if (L.n_kept > 0)
-    k_kept<<<(unsigned)L.n_kept, 256, 0, st>>>(bl, L.off_kept, d_prompts, L.batch, c->theta, (__nv_bfloat16 *)k_out,
-                                              (__nv_bfloat16 *)v_out, L.n_tokens, valid);
+    { k_kept<<<(unsigned)L.n_kept, 256, 0, st>>>(bl, L.off_kept, d_prompts, L.batch, c->theta, (__nv_bfloat16 *)k_out,
+                                              (__nv_bfloat16 *)v_out, L.n_tokens, valid); ++g_launches; }
   if (L.n_rows > 0)
-    k_fixup<<<c->num_sms, 256, 0, st>>>(biglist, counters, q16, qbig, c->a_inv, (float)std::ldexp(1.0, -c->p_inv),
+    { k_fixup<<<c->num_sms, 256, 0, st>>>(biglist, counters, q16, qbig, c->a_inv, (float)std::ldexp(1.0, -c->p_inv),
                                        c->mu_perm, c->theta, row_tok, row_pos, (__nv_bfloat16 *)k_out,
-                                       (__nv_bfloat16 *)v_out, L.n_tokens);
+                                       (__nv_bfloat16 *)v_out, L.n_tokens); ++g_launches; }
   CK(cudaGetLastError());
   stage_mark(c, st, "kept+fixup");
   return DCKV_OK;
@@ -1419,6 +1437,8 @@ extern "C" int dckv_debug_ratio(dckv_codec *c, void *ratio_dev) {
   c->dbg_ratio = (float *)ratio_dev;
   return DCKV_OK;
 }
+
+extern "C" long long dckv_launch_count(void) { return g_launches.load(); }
 
 extern "C" int dckv_codec_info(const dckv_codec *c, int32_t *chunk_rows, double *model_bits_per_row) {
   if (!c) return fail(DCKV_EINVAL, "NULL codec");

@@ -30,7 +30,7 @@ struct EpiStoreF32 {
     float scale;
   };
   static constexpr int SMEM_BYTES = 0;
-  __device__ static void tile(const Params &p, const EpiCtx &cx) {
+  __device__ __forceinline__ static void tile(const Params &p, const EpiCtx &cx) {
     const int m = cx.mt * GEMM_BM + cx.ew * 32 + cx.lane;
     for (int c0 = cx.grp * 32; c0 < cx.n_valid; c0 += 32 * cx.n_grp) {
       uint32_t r[32];
@@ -59,7 +59,7 @@ struct EpiGelu {
 struct EpiGeluTotals {
   using Params = EpiGelu::Params;
   static constexpr int SMEM_BYTES = 0;
-  __device__ static void tile(const Params &p, char *, int mt, int n0, int n_valid, int c_begin, uint32_t ttot,
+  __device__ __forceinline__ static void tile(const Params &p, char *, int mt, int n0, int n_valid, int c_begin, uint32_t ttot,
                               int ew, int lane, int) {
     const int m = mt * GEMM_BM + ew * 32 + lane;
     const float mw = p.muw1[m];
@@ -119,7 +119,7 @@ struct EpiQuantRegs {
   __device__ static void list_row(const Params &p, int row) {
     if (atomicExch(&p.rowflag[row], 1u) == 0u) p.full_list[atomicAdd(&p.counters[1], 1u)] = (uint32_t)row;
   }
-  __device__ static __noinline__ void flag(const Params &pp, int row, int c) {
+  __device__ static void flag(const Params &pp, int row, int c) {
     if (pp.row_norm[row] > REFINE_NORM_FULL) {
       list_row(pp, row);
     } else {
@@ -128,15 +128,31 @@ struct EpiQuantRegs {
       else list_row(pp, row);
     }
   }
+  // per tile column: padded even row (or -1) and the guard-band width's row term
+  static constexpr int SMEM_BYTES = GEMM_MAX_BN * 8;
+  __device__ __forceinline__ static void stage(const Params &pp, char *buf, int n0, int n_valid, int tid,
+                                               int nthreads) {
+    int32_t *s_e = reinterpret_cast<int32_t *>(buf);
+    float *s_w = reinterpret_cast<float *>(buf + GEMM_MAX_BN * 4);
+    for (int j = tid; j < n_valid; j += nthreads) {
+      s_e[j] = __ldg(pp.q.row_edst + n0 + j);
+      s_w[j] = __ldg(pp.row_norm + n0 + j);
+    }
+  }
   template <int NC>
-  __device__ static void finish(const Params &pp, const float (&tot)[NC], int mt, int n0, int n_valid, int col0,
-                                int ew, int lane) {
+  __device__ __forceinline__ static void finish(const Params &pp, const char *buf, const float (&tot)[NC], int mt,
+                                                int n0, int n_valid, int col0, int ew, int lane) {
     const EpiQuant::Params &p = pp.q;
+    const int32_t *s_e = reinterpret_cast<const int32_t *>(buf);
+    const float *s_w = reinterpret_cast<const float *>(buf + GEMM_MAX_BN * 4);
     const int c = mt * GEMM_BM + ew * 32 + lane;
     const float mb = p.mub[c];
     const float dl = p.delta[c];
     const bool kp = p.keep[c] != 0;
     const float wk = REFINE_KAPPA / dl;
+    uint32_t fm[(NC + 31) / 32];  // columns whose code goes to the exact recomputation
+#pragma unroll
+    for (int w = 0; w < (NC + 31) / 32; ++w) fm[w] = 0u;
 #pragma unroll
     for (int j = 0; j < NC; ++j) {
       const int col = col0 + j;
@@ -146,13 +162,20 @@ struct EpiQuantRegs {
         const float ratio = __fdiv_rn(y, dl);
         const int q = kp ? __float2int_rn(ratio) : 0;
         p.q32[(int64_t)row * N_COEF + c] = q;
-        const int e = p.row_edst[row];
+        const int e = s_e[col];
         if (e >= 0) p.qe[(int64_t)e * N_COEF + c] = __float2bfloat16_rn((float)q);
         if (pp.dbg_ratio) pp.dbg_ratio[(int64_t)row * N_COEF + c] = ratio;
-        if (kp) {
-          const float w = wk * pp.row_norm[row] + REFINE_W0;
-          if (0.5f - fabsf(ratio - rintf(ratio)) < w || !(fabsf(ratio) < 1.0e6f)) flag(pp, row, c);
-        }
+        const float w = wk * s_w[col] + REFINE_W0;
+        if (kp && (0.5f - fabsf(ratio - rintf(ratio)) < w || !(fabsf(ratio) < 1.0e6f))) fm[j >> 5] |= 1u << (j & 31);
+      }
+    }
+#pragma unroll
+    for (int w = 0; w < (NC + 31) / 32; ++w) {
+      uint32_t m = fm[w];
+      while (m) {
+        const int b = __ffs(m) - 1;
+        m &= m - 1u;
+        flag(pp, n0 + col0 + w * 32 + b, c);
       }
     }
   }
@@ -175,19 +198,19 @@ struct EpiMeanOdd {
   };
   // per tile column: t_odd row offset (or -1) and the slot row (each group stages its own)
   static constexpr int SMEM_BYTES = 256 * 16;
-  __device__ static void tile(const Params &p, const EpiCtx &cx) {
+  __device__ __forceinline__ static void tile(const Params &p, const EpiCtx &cx) {
     int64_t *s_row = reinterpret_cast<int64_t *>(cx.scratch);
     int32_t *s_slot = reinterpret_cast<int32_t *>(cx.scratch + 256 * 8);
     const int n_valid = cx.n_valid;
     for (int j = cx.et; j < n_valid; j += 128) {
-      const int ti = p.e_tok[cx.n0 + j];
+      const int ti = __ldg(p.e_tok + cx.n0 + j);
       int64_t off = -1;
       if (ti >= 0) {
-        const int tok = min(max(p.tok_ids[ti], 0), p.vocab - 1);
+        const int tok = min(max(__ldg(p.tok_ids + ti), 0), p.vocab - 1);
         off = (int64_t)tok * N_COEF;
       }
       s_row[j] = off;
-      s_slot[j] = p.e_slot[cx.n0 + j];
+      s_slot[j] = __ldg(p.e_slot + cx.n0 + j);
     }
     named_bar_sync(cx.bar, 128);
     const int c = cx.mt * GEMM_BM + cx.ew * 32 + cx.lane;
@@ -244,7 +267,7 @@ struct EpiInverse {
   static constexpr int CW = 16;
   static constexpr int XCH_LD = CW + 1;
   static constexpr int SMEM_BYTES = 128 * XCH_LD * 4 + CW * 128 * 2;
-  __device__ static void tile(const Params &p, const EpiCtx &cx) {
+  __device__ __forceinline__ static void tile(const Params &p, const EpiCtx &cx) {
     float *xch = reinterpret_cast<float *>(cx.scratch);
     __nv_bfloat16 *ob = reinterpret_cast<__nv_bfloat16 *>(cx.scratch + 128 * XCH_LD * 4);
     const int mt = cx.mt, n0 = cx.n0, n_valid = cx.n_valid, et = cx.et;
@@ -268,7 +291,7 @@ struct EpiInverse {
 #pragma unroll
         for (int j = 0; j < CW; ++j) {
           const int row = min(n0 + c0 + j, n0 + n_valid - 1);
-          cs[j] = __ldg(p.rope + (int64_t)p.row_pos[row] * 128 + fi);
+          cs[j] = __ldg(p.rope + (int64_t)__ldg(p.row_pos + row) * 128 + fi);
           xch[ml * XCH_LD + j] = v[j];
         }
         named_bar_sync(cx.bar, 128);
@@ -288,7 +311,7 @@ struct EpiInverse {
         const int j = qid >> 4, sub = qid & 15, seg = sub >> 3, w = sub & 7;
         if (c0 + j < n_valid) {
           const int row = n0 + c0 + j;
-          const int64_t tok = p.row_tok[row];
+          const int64_t tok = __ldg(p.row_tok + row);
           const int64_t off = ((layer * p.n_tokens + tok) * 2 + head) * HEAD_DIM + seg * 128 + half * 64 + w * 8;
           *reinterpret_cast<uint4 *>(dst_base + off) = *reinterpret_cast<const uint4 *>(ob + j * 128 + seg * 64 + w * 8);
         }

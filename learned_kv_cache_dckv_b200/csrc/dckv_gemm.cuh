@@ -447,7 +447,9 @@ constexpr int gemm2_smem_bytes() {
 // eight epilogue warps of each CTA add each partial into running totals held in registers
 // (fp32 round-to-nearest adds, in chunk order) -- warp w >= 2 owns lane quarter w % 4 and
 // column half (w - 2) / 4, BN / 2 columns -- and after a tile's last chunk hand their totals
-// to Epi::finish.  Both P buffers stay free for the MMA while totals are finished.
+// to Epi::finish.  Both P buffers stay free for the MMA while totals are finished.  Per-column
+// metadata of a tile is staged into shared memory (Epi::stage, two buffers by tile parity)
+// before its chunks are drained, so that finish reads it without global-memory latency.
 constexpr int GEMM2C_THREADS = 320;
 
 template <class Epi, int STAGES, int MAX_SLABS, int CHUNK_STEPS, int BN>
@@ -467,6 +469,8 @@ __global__ void __launch_bounds__(GEMM2C_THREADS, 1)
   uint64_t *part_empty = part_full + 2;  // leader's: one arrival per epilogue warp of either CTA
   uint32_t *tmem_base_smem = reinterpret_cast<uint32_t *>(part_empty + 2);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_base_smem + 1);
+  constexpr int EPI_BUF = (Epi::SMEM_BYTES + 15) & ~15;
+  char *epi_buf = reinterpret_cast<char *>(base + STAGES * STAGE_BYTES + 1024);  // two buffers
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -609,10 +613,13 @@ __global__ void __launch_bounds__(GEMM2C_THREADS, 1)
     int pb = 0;
     uint32_t pph = 0;
     bool stop = false;
-    for (int t = pair; t < total_tiles && !stop; t += n_pairs) {
+    int tp = 0;
+    for (int t = pair; t < total_tiles && !stop; t += n_pairs, tp ^= 1) {
       const int mp = t % m_pairs;
       const int n0 = (t / m_pairs) * BN;
       const int n_valid = min(BN, prob.n_rows - n0);
+      char *buf = epi_buf + tp * EPI_BUF;
+      Epi::stage(ep, buf, n0, n_valid, threadIdx.x - 64, GEMM2C_THREADS - 64);
       float tot[NC];
 #pragma unroll
       for (int j = 0; j < NC; ++j) tot[j] = 0.f;
@@ -642,7 +649,8 @@ __global__ void __launch_bounds__(GEMM2C_THREADS, 1)
         }
       }
       if (stop) break;
-      Epi::template finish<NC>(ep, tot, 2 * mp + (int)rank, n0, n_valid, col0, ew, lane);
+      named_bar_sync(1, GEMM2C_THREADS - 64);  // the tile's staged metadata is visible
+      Epi::template finish<NC>(ep, buf, tot, 2 * mp + (int)rank, n0, n_valid, col0, ew, lane);
     }
   }
 
@@ -655,9 +663,9 @@ __global__ void __launch_bounds__(GEMM2C_THREADS, 1)
   }
 }
 
-template <int STAGES, int MAX_SLABS>
+template <class Epi, int STAGES, int MAX_SLABS>
 constexpr int gemm2_chunked_smem_bytes() {
-  return 1024 + STAGES * Gemm2Smem<MAX_SLABS>::STAGE_BYTES + 1024;
+  return 1024 + STAGES * Gemm2Smem<MAX_SLABS>::STAGE_BYTES + 1024 + 2 * ((Epi::SMEM_BYTES + 15) & ~15);
 }
 
 // ------------------------------------------------------------------------------------------

@@ -45,6 +45,9 @@ constexpr float REFINE_NORM_FULL = 32.0f;
 constexpr int TRANSFORM_BN = 224;
 constexpr int MEAN_ODD_BN = 224;
 constexpr int INVERSE_BN = 224;
+// K steps (of 64) per TMEM partial of the transform before it is added into the fp32
+// totals: bounds the growth of the tensor core's accumulation error over K = 6,144.
+constexpr int TRANSFORM_CHUNK_STEPS = 4;
 
 struct PromptInfo {
   int64_t tok_base;  // first row (token) of the prompt in the batch
@@ -124,7 +127,7 @@ struct dckv_codec {
   uint16_t *lut = nullptr;   // [64][1024] decoder lookup (symbol holding slot b * 64)
   uint32_t *tail = nullptr;  // [64] lengths of the frequency-1 runs at both ends
   uint16_t *dcdf = nullptr;  // [64][512] cdf, padded with two zero entries (decoder)
-  uint32_t *rcp = nullptr;   // [64][510] division multiplier of each frequency (encoder)
+  uint2 *cfm_tab = nullptr;  // [64][510] {cdf | (freq - 1) << 16, division multiplier} (encoder)
   int16_t *kidx = nullptr;   // [2048] kept index of a component, -1 if dropped
   double model_bits_per_row = 0.0;  // entropy of the kept components' tables
   float *dbg_ratio = nullptr;       // optional [rows][2048] export of the fp32 ratios y / Delta

@@ -221,9 +221,11 @@ __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-// Arrive on an mbarrier given by its shared::cluster address (own CTA or peer).
+// Arrive on an mbarrier given by its shared::cluster address (own CTA or peer).  The
+// barriers signalled this way only hand TMEM back to the MMA issuer (ordered by the
+// tcgen05 fences), so the default CTA-scope semantics suffice.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cl_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cl_addr) : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cl_addr) : "memory");
 }
 
 // TMA tile loads into this CTA's shared memory whose completion is counted on an mbarrier

@@ -63,13 +63,24 @@ __global__ void __launch_bounds__(256) k_centres_even(int64_t n_rows, const int3
 }
 
 // Encoder inputs in slot order: the symbol (ESC if |q| > 127 else q - centre + 254), its
-// table entry {cdf | (freq - 1) << 16, division multiplier of freq}, and the escape count
-// of each chunk.
-__global__ void __launch_bounds__(256) k_symbols(int64_t n_rows, const int32_t *row_slot, const int32_t *slot_chunk,
-                                                 const int32_t *q32, const int8_t *cen8, const int16_t *kept_list,
-                                                 const uint8_t *kept_scale, const uint16_t *cdf, const uint32_t *rcp,
-                                                 int k_eff, uint16_t *sym16, uint2 *cfm, uint32_t *nesc) {
+// table entry {cdf | (freq - 1) << 16, division multiplier of freq} (from the codec's
+// packed per-(scale, symbol) table), and the escape count of each chunk.  Four positions
+// per thread are in flight at a time.
+constexpr int SYM_THREADS = 256;
+constexpr int SYM_UNROLL = 4;
+
+__global__ void __launch_bounds__(SYM_THREADS) k_symbols(int64_t n_rows, const int32_t *row_slot,
+                                                         const int32_t *slot_chunk, const int32_t *q32,
+                                                         const int8_t *cen8, const int16_t *kept_list,
+                                                         const uint8_t *kept_scale, const uint2 *cfm_tab, int k_eff,
+                                                         uint16_t *sym16, uint2 *cfm, uint32_t *nesc) {
   __shared__ int esc_count;
+  __shared__ int16_t s_kl[N_COEF];
+  __shared__ uint8_t s_ks[N_COEF];
+  for (int k = threadIdx.x; k < k_eff; k += SYM_THREADS) {
+    s_kl[k] = kept_list[k];
+    s_ks[k] = kept_scale[k];
+  }
   for (int64_t row = blockIdx.x; row < n_rows; row += gridDim.x) {
     if (threadIdx.x == 0) esc_count = 0;
     __syncthreads();
@@ -77,16 +88,25 @@ __global__ void __launch_bounds__(256) k_symbols(int64_t n_rows, const int32_t *
     const int64_t base = (int64_t)slot * k_eff;
     const int32_t *q = q32 + row * N_COEF;
     int esc = 0;
-    for (int k = threadIdx.x; k < k_eff; k += blockDim.x) {
-      const int v = q[kept_list[k]];
-      const bool is_esc = v > ESC_LIMIT || v < -ESC_LIMIT;
-      const int sym = is_esc ? ESC_SYM : v - cen8[base + k] + R_MAX;
-      esc += is_esc;
-      const int ti = kept_scale[k] * N_SYM + sym;
-      const uint32_t c = cdf[ti];
-      const uint32_t f = cdf_at(cdf + (ti - sym), sym + 1) - c;
-      sym16[base + k] = (uint16_t)sym;
-      cfm[base + k] = make_uint2(c | ((f - 1u) << 16), rcp[ti]);
+    for (int k0 = threadIdx.x; k0 < k_eff; k0 += SYM_UNROLL * SYM_THREADS) {
+      int v[SYM_UNROLL], ce[SYM_UNROLL];
+#pragma unroll
+      for (int u = 0; u < SYM_UNROLL; ++u) {
+        const int k = k0 + u * SYM_THREADS;
+        v[u] = k < k_eff ? __ldg(q + s_kl[k]) : 0;
+        ce[u] = k < k_eff ? (int)__ldg(cen8 + base + k) : 0;
+      }
+#pragma unroll
+      for (int u = 0; u < SYM_UNROLL; ++u) {
+        const int k = k0 + u * SYM_THREADS;
+        if (k < k_eff) {
+          const bool is_esc = v[u] > ESC_LIMIT || v[u] < -ESC_LIMIT;
+          const int sym = is_esc ? ESC_SYM : v[u] - ce[u] + R_MAX;
+          esc += is_esc;
+          sym16[base + k] = (uint16_t)sym;
+          cfm[base + k] = __ldg(cfm_tab + s_ks[k] * N_SYM + sym);
+        }
+      }
     }
     if (esc) atomicAdd(&esc_count, esc);
     __syncthreads();
@@ -278,30 +298,44 @@ struct CompactArgs {
   uint64_t blob_cap, off_streams;
 };
 
-__global__ void __launch_bounds__(RANS_WARPS * 32) compact_kernel(CompactArgs a) {
-  const int lane = threadIdx.x & 31;
-  const int ci = blockIdx.x * RANS_WARPS + (threadIdx.x >> 5);
+constexpr int COMPACT_THREADS = 128;
+
+// One block per chunk.  Escape values are found in two passes over the chunk's symbols
+// (count per warp, then write at the warp's prefix), only in chunks that have escapes.
+__global__ void __launch_bounds__(COMPACT_THREADS) compact_kernel(CompactArgs a) {
+  __shared__ uint32_t s_cnt[COMPACT_THREADS / 32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  constexpr int NW = COMPACT_THREADS / 32;
+  const int ci = blockIdx.x;
   if (ci >= a.n_chunks) return;
   const uint64_t beg = a.off_streams + a.offs[ci];
   const uint64_t end = a.off_streams + a.offs[ci + 1];
   if (end > a.blob_cap) return;  // capacity error already reported by the scan
   uint8_t *sec = a.blob + beg;
   const uint32_t ne = a.nesc[ci], nw = a.nwords[ci];
-  reinterpret_cast<uint32_t *>(sec)[lane] = a.states[(int64_t)ci * 32 + lane];
-  if (lane == 0) reinterpret_cast<uint32_t *>(sec)[32] = ne;
+  if (threadIdx.x < 32) reinterpret_cast<uint32_t *>(sec)[lane] = a.states[(int64_t)ci * 32 + lane];
+  if (threadIdx.x == 0) reinterpret_cast<uint32_t *>(sec)[32] = ne;
   const ChunkDesc cd = a.chunks[ci];
-  const PromptInfo pi = a.prompts[cd.prompt];
   const int K = a.k_eff;
   const int64_t S = (int64_t)cd.nrows * K;
   // escaped codes in symbol order, 64 raw bits each (sections are 4-byte aligned)
   if (ne) {
+    const PromptInfo pi = a.prompts[cd.prompt];
     uint32_t *ev = reinterpret_cast<uint32_t *>(sec + CHUNK_FIXED_BYTES);
-    uint32_t ep = 0;
     const uint32_t lt_mask = (1u << lane) - 1u;
     const uint16_t *syms = a.sym16 + cd.sym_base;
-    for (int64_t i0 = 0; i0 < S && ep < ne; i0 += 32) {
+    const int64_t per = ((S + NW - 1) / NW + 31) & ~int64_t(31);  // warp w scans [w per, (w+1) per)
+    const int64_t i_beg = warp * per, i_end = min(S, i_beg + per);
+    uint32_t n = 0;
+    for (int64_t i = i_beg + lane; i < i_end; i += 32) n += syms[i] == ESC_SYM;
+    for (int o = 16; o; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
+    if (lane == 0) s_cnt[warp] = n;
+    __syncthreads();
+    uint32_t ep = 0;
+    for (int w = 0; w < warp; ++w) ep += s_cnt[w];
+    for (int64_t i0 = i_beg; i0 < i_end; i0 += 32) {
       const int64_t i = i0 + lane;
-      const bool esc = i < S && syms[i] == ESC_SYM;
+      const bool esc = i < i_end && syms[i] == ESC_SYM;
       const uint32_t m = __ballot_sync(0xffffffffu, esc);
       if (esc) {
         const int rl = (int)(i / K);
@@ -309,8 +343,10 @@ __global__ void __launch_bounds__(RANS_WARPS * 32) compact_kernel(CompactArgs a)
         const int64_t row = (int64_t)pi.row_base + 2 * (cd.j0 + rl) + cd.parity;
         const int64_t v = (int64_t)a.q32[row * N_COEF + a.kept_list[k]];
         const uint32_t slot = ep + __popc(m & lt_mask);
-        ev[2 * slot] = (uint32_t)(uint64_t)v;
-        ev[2 * slot + 1] = (uint32_t)((uint64_t)v >> 32);
+        if (slot < ne) {
+          ev[2 * slot] = (uint32_t)(uint64_t)v;
+          ev[2 * slot + 1] = (uint32_t)((uint64_t)v >> 32);
+        }
       }
       ep += __popc(m);
     }
@@ -318,9 +354,21 @@ __global__ void __launch_bounds__(RANS_WARPS * 32) compact_kernel(CompactArgs a)
   // words (decoder order) follow the escapes; then zero padding to 4 bytes
   uint16_t *wd = reinterpret_cast<uint16_t *>(sec + CHUNK_FIXED_BYTES + 8ull * ne);
   const uint16_t *ws = a.words + cd.sym_base + (S - nw);
-  for (uint32_t w = lane; w < nw; w += 32) wd[w] = ws[w];
+  for (uint32_t w0 = threadIdx.x; w0 < nw; w0 += 4 * COMPACT_THREADS) {
+    uint16_t v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const uint32_t w = w0 + u * COMPACT_THREADS;
+      v[u] = w < nw ? ws[w] : (uint16_t)0;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const uint32_t w = w0 + u * COMPACT_THREADS;
+      if (w < nw) wd[w] = v[u];
+    }
+  }
   const uint64_t used = CHUNK_FIXED_BYTES + 8ull * ne + 2ull * nw;
-  if (lane == 0 && (end - beg) > used) wd[nw] = 0;
+  if (threadIdx.x == 0 && (end - beg) > used) wd[nw] = 0;
 }
 
 // ------------------------------------------------------------------------------ decode
@@ -333,8 +381,8 @@ __global__ void __launch_bounds__(RANS_WARPS * 32) compact_kernel(CompactArgs a)
 //   tail[s] = length of the leading run of frequency-1 symbols (cdf[sym] = sym) in bits
 //     0-15 and length n of the trailing run (cdf[sym] = 65536 - 510 + sym, ESC last;
 //     slots 65536 - n .. 65535) in bits 16-31; slots in a run decode by arithmetic;
-//   rcp[s][sym] = division multiplier of the symbol's frequency (encoder).
-__global__ void k_build_lut(const uint16_t *cdf, uint16_t *dcdf, uint16_t *lut, uint32_t *tail, uint32_t *rcp) {
+//   cfm_tab[s][sym] = {cdf | (freq - 1) << 16, division multiplier of freq} (encoder).
+__global__ void k_build_lut(const uint16_t *cdf, uint16_t *dcdf, uint16_t *lut, uint32_t *tail, uint2 *cfm_tab) {
   const int s = blockIdx.x;
   const uint16_t *tab = cdf + s * N_SYM;
   auto holder = [&](uint32_t slot) {
@@ -353,7 +401,10 @@ __global__ void k_build_lut(const uint16_t *cdf, uint16_t *dcdf, uint16_t *lut, 
   }
   for (int k = threadIdx.x; k < DEC_CDF_STRIDE; k += blockDim.x) {
     dcdf[s * DEC_CDF_STRIDE + k] = k < N_SYM ? tab[k] : (uint16_t)0;
-    if (k < N_SYM) rcp[s * N_SYM + k] = div_multiplier(cdf_at(tab, k + 1) - tab[k]);
+    if (k < N_SYM) {
+      const uint32_t f = cdf_at(tab, k + 1) - tab[k];
+      cfm_tab[s * N_SYM + k] = make_uint2((uint32_t)tab[k] | ((f - 1u) << 16), div_multiplier(f));
+    }
   }
   if (threadIdx.x == 0) {
     int lead = 0;  // symbols 0 .. lead-1 have frequency 1
@@ -565,10 +616,14 @@ struct DecCodesArgs {
 };
 
 constexpr int DEC_CODES_THREADS = 256;
+constexpr int DEC_UNROLL = 4;
 
 __global__ void __launch_bounds__(DEC_CODES_THREADS) k_decode_codes(DecCodesArgs a) {
   __shared__ uint32_t s_esc[256];  // escapes per row of the chunk (at most 256 rows)
+  __shared__ int16_t s_kl[N_COEF];
   if (*a.valid != 1) return;
+  for (int k = threadIdx.x; k < a.k_eff; k += DEC_CODES_THREADS) s_kl[k] = a.kept_list[k];
+  __syncthreads();
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int nw = DEC_CODES_THREADS / 32;
@@ -605,31 +660,40 @@ __global__ void __launch_bounds__(DEC_CODES_THREADS) k_decode_codes(DecCodesArgs
       __half *q16 = a.q16 + row * N_COEF;
       __nv_bfloat16 *qe = cd.parity == 0 ? a.qe + (int64_t)(pi.ebase + j) * N_COEF : nullptr;
       bool bad = false;
-      for (int k0 = 0; k0 < K; k0 += 32) {
-        const int k = k0 + lane;
-        const bool valid = k < K;
-        const int sym = valid ? sy[k] : 0;
-        const bool is_esc = valid && sym == ESC_SYM;
-        const uint32_t me = __ballot_sync(0xffffffffu, is_esc);
-        int q = valid ? sym - R_MAX + ce[k] : 0;
-        if (is_esc) {
-          const uint32_t e = ep + __popc(me & lt_mask);
-          if (e < ne) {
-            const int64_t sv = (int64_t)((uint64_t)ev[2 * e] | ((uint64_t)ev[2 * e + 1] << 32));
-            q = (int)max(min(sv, (int64_t)INT32_MAX), (int64_t)INT32_MIN);
-            if (sv >= -ESC_LIMIT && sv <= ESC_LIMIT) bad = true;  // not an escape value
-          } else {
-            bad = true;
-          }
+      for (int k0 = 0; k0 < K; k0 += 32 * DEC_UNROLL) {
+        int sym[DEC_UNROLL], cen[DEC_UNROLL];
+#pragma unroll
+        for (int u = 0; u < DEC_UNROLL; ++u) {  // loads first: DEC_UNROLL positions in flight
+          const int k = k0 + u * 32 + lane;
+          sym[u] = k < K ? (int)sy[k] : 0;
+          cen[u] = k < K ? (int)ce[k] : 0;
         }
-        ep += __popc(me);
-        if (valid) {
-          const int comp = a.kept_list[k];
-          q16[comp] = __float2half_rn((float)q);
-          if (qe) qe[comp] = __float2bfloat16_rn((float)q);
-          if (q >= BIG_CODE || q <= -BIG_CODE) {
-            a.qbig[row * N_COEF + comp] = q;
-            if (atomicExch(&a.bigflag[row], 1u) == 0u) a.biglist[atomicAdd(a.bigcount, 1u)] = (int32_t)row;
+#pragma unroll
+        for (int u = 0; u < DEC_UNROLL; ++u) {
+          const int k = k0 + u * 32 + lane;
+          const bool valid = k < K;
+          const bool is_esc = valid && sym[u] == ESC_SYM;
+          const uint32_t me = __ballot_sync(0xffffffffu, is_esc);
+          int q = valid ? sym[u] - R_MAX + cen[u] : 0;
+          if (is_esc) {
+            const uint32_t e = ep + __popc(me & lt_mask);
+            if (e < ne) {
+              const int64_t sv = (int64_t)((uint64_t)ev[2 * e] | ((uint64_t)ev[2 * e + 1] << 32));
+              q = (int)max(min(sv, (int64_t)INT32_MAX), (int64_t)INT32_MIN);
+              if (sv >= -ESC_LIMIT && sv <= ESC_LIMIT) bad = true;  // not an escape value
+            } else {
+              bad = true;
+            }
+          }
+          ep += __popc(me);
+          if (valid) {
+            const int comp = s_kl[k];
+            q16[comp] = __float2half_rn((float)q);
+            if (qe) qe[comp] = __float2bfloat16_rn((float)q);
+            if (q >= BIG_CODE || q <= -BIG_CODE) {
+              a.qbig[row * N_COEF + comp] = q;
+              if (atomicExch(&a.bigflag[row], 1u) == 0u) a.biglist[atomicAdd(a.bigcount, 1u)] = (int32_t)row;
+            }
           }
         }
       }
