@@ -105,6 +105,18 @@ def dist_env():
     return ws, rank, local
 
 
+def max_over_ranks(values, dist=None, device="cpu"):
+    """Element-wise maximum of per-rank timings over all ranks (every rank gets it); the
+    slowest rank decides a replica step's time."""
+    if dist is None:
+        return [float(v) for v in values]
+    import torch
+
+    t = torch.tensor([float(v) for v in values], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
 def make_inputs(cfg_name, rank, device):
     import dckv_synth as S
 
@@ -293,10 +305,7 @@ def run_gpu(args):
     ms_step = statistics.mean(step_ms)
     ms_enc = statistics.mean(enc_ms)
     ms_dec = statistics.mean(dec_ms)
-    if dist:
-        t = torch.tensor([ms_step, ms_enc, ms_dec], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step, ms_enc, ms_dec = t.tolist()
+    ms_step, ms_enc, ms_dec = max_over_ranks([ms_step, ms_enc, ms_dec], dist, dev)
 
     # end to end through the public API with host buffers: H2D rows + ids, encode,
     # D2H blob; H2D blob, decode, D2H K and V -- all inside the timed region
@@ -328,12 +337,9 @@ def run_gpu(args):
     h2d = x.numel() * 2 + tok.numel() * 4 + size
     d2h = size + 2 * k_out.numel() * 2
     ms_e2e = statistics.mean(e2e_ms)
-    if dist:
-        t = torch.tensor([ms_e2e], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_e2e = t.item()
+    ms_e2e = max_over_ranks([ms_e2e], dist, dev)[0]
 
-    # roofline of the dominant kernel (largest mean stage time among the GEMMs)
+    # roofline of the dominant kernel (largest mean stage time), plus the largest GEMM
     peaks, peak_kind = load_peaks()
     means = {k: statistics.mean(v) for k, v in stage_ms.items()}
     n_even = sum((max(0, int(n) - 132) + 1) // 2 for n in np.diff(offs))
@@ -346,20 +352,49 @@ def run_gpu(args):
         "dec:gemm_mean_odd": 2.0 * n_odd * 4096 * 2048,
         "dec:gemm_inverse": 2.0 * n_rows * 2048 * 6144,
     }
+    pad = lambda n, t: -(-n // t) * t
     issued_flops = {  # what the tensor pipe executes (split operands, padded tiles)
-        "enc:gemm_hidden": 2.0 * 2 * (-(-n_rows // 128) * 128) * 6144 * 256,
-        "enc:gemm_transform": 2.0 * (-(-n_rows // 256) * 256) * (2 * 6144 * 2048 + 4 * 256 * 2048),
-        "enc:gemm_mean_odd": 2.0 * (-(-(n_even + len(offs) - 1) // 256) * 256) * 4096 * 2048,
-        "dec:gemm_mean_odd": 2.0 * (-(-(n_even + len(offs) - 1) // 256) * 256) * 4096 * 2048,
-        "dec:gemm_inverse": 2.0 * 2 * (-(-n_rows // 256) * 256) * 2048 * 6144,
+        "enc:gemm_hidden": 2.0 * 2 * pad(n_rows, 128) * 6144 * 256,
+        "enc:gemm_transform": 2.0 * pad(n_rows, 224) * (2 * 6144 * 2048 + 4 * 256 * 2048),
+        "enc:gemm_mean_odd": 2.0 * pad(n_even + len(offs) - 1, 224) * 4096 * 2048,
+        "dec:gemm_mean_odd": 2.0 * pad(n_even + len(offs) - 1, 224) * 4096 * 2048,
+        "dec:gemm_inverse": 2.0 * 2 * pad(n_rows, 224) * 2048 * 6144,
     }
-    dom = max(algo_flops, key=lambda k: means.get(k, 0.0))
-    peak = float(peaks.get("bf16_tflops", 1590.0))
-    achieved = algo_flops[dom] / (means[dom] * 1e-3) / 1e12
-    roofline = {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "peak_source": f"{peak_kind} dense bf16 (fp16 operands run at the same rate)",
-                "issued_frac": issued_flops[dom] / (means[dom] * 1e-3) / 1e12 / peak,
-                "traffic": None}
+    # DRAM bytes (read + write) per launch from the committed ncu captures of this workload
+    # (profiles/*_c2.md); null for other workloads
+    traffic = {"enc:gemm_transform": 191.2e6, "dec:gemm_inverse": 158.6e6, "enc:gemm_mean_odd": 41.1e6,
+               "dec:gemm_mean_odd": 41.1e6} if args.config == "c2" else {}
+    bf16_peak = float(peaks.get("bf16_tflops", 1590.0))
+    sm_mhz = float(peaks.get("sm_max_mhz", 1965.0))
+    alu_peak = 148 * 128 * sm_mhz * 1e6 / 1e12  # int32 lanes x clock, Tops/s
+
+    def tensor_roofline(k):
+        achieved = algo_flops[k] / (means[k] * 1e-3) / 1e12
+        return {"kernel": k, "bound": "tensor", "achieved": achieved, "peak": bf16_peak, "unit": "TFLOP/s",
+                "frac": achieved / bf16_peak,
+                "peak_source": f"{peak_kind} dense bf16, burst (fp16 operands run at the bf16 rate)",
+                "issued_frac": issued_flops[k] / (means[k] * 1e-3) / 1e12 / bf16_peak,
+                "traffic": traffic.get(k)}
+
+    def rans_roofline(k):
+        # 8 integer operations per decoded symbol: slot mask, bucket lookup, cdf lookup,
+        # multiply-add, subtract, renormalisation test, shift-or, word fetch
+        ops = 8.0 * n_rows * k_eff
+        achieved = ops / (means[k] * 1e-3) / 1e12
+        return {"kernel": k, "bound": "alu", "achieved": achieved, "peak": alu_peak, "unit": "Tops/s",
+                "frac": achieved / alu_peak, "peak_source": "148 SMs x 128 int32 lanes x max SM clock",
+                "note": "latency-bound: one warp per chunk runs its states' dependency chain",
+                "traffic": traffic.get(k)}
+
+    dom = max(means, key=means.get)
+    gemm_dom = max(algo_flops, key=lambda k: means.get(k, 0.0))
+    if dom in algo_flops:
+        roofline = tensor_roofline(dom)
+    elif dom == "dec:rans_loop":
+        roofline = rans_roofline(dom)
+    else:
+        roofline = tensor_roofline(gemm_dom)
+    roofline_gemm = tensor_roofline(gemm_dom)
 
     model_bpt = model_bytes_per_row(D, gc, x, tok, offs, blob)
 
@@ -386,6 +421,7 @@ def run_gpu(args):
         "compression_vs_bf16": 12288.0 * n_rows / max(payload, 1),
         "stage_ms": {k: round(v, 5) for k, v in sorted(means.items())},
         "roofline": roofline,
+        "roofline_gemm": roofline_gemm,
         "e2e": {"value": tokens * ws / (ms_e2e * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": launches,

@@ -103,9 +103,10 @@ typedef struct {
  * embed @ w_odd[0:2048] (fp32).  chunk_rows (1..256) is the number of same-parity rows
  * per rANS chunk; 0 selects 16; -1 selects the smallest count whose fixed per-chunk bytes
  * (states, escape count, offset) stay within 3.5% of the tables' own entropy per row.
- * Fewer rows per chunk give more independent streams (faster decode) and more bytes.  Allocates device memory (about
- * 2 * vocab * 8 KiB + 230 MiB).  Synchronises the device.  Returns DCKV_OK or an error;
- * *out is NULL on error. */
+ * Fewer rows per chunk give more independent streams (faster decode) and more bytes.
+ * Allocates device memory (about 2 * vocab * 8 KiB + 192 MiB: split GEMM operands, fp32
+ * weight copies for the exact recomputation of near-boundary codes, tables).
+ * Synchronises the device.  Returns DCKV_OK or an error; *out is NULL on error. */
 int dckv_codec_create(const dckv_params *params, int device, int chunk_rows, dckv_codec **out);
 void dckv_codec_destroy(dckv_codec *codec);
 

@@ -887,7 +887,7 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
   const uint64_t o_kl = take(2ull * N_COEF);
   const uint64_t o_ks = take(N_COEF);
   const uint64_t o_cdf = take(2ull * N_SCALES * N_SYM);
-  const uint64_t o_lut = take(2ull * N_SCALES * LUT_SIZE);
+  const uint64_t o_lut = take(2ull * N_SCALES * LUT_STRIDE);
   const uint64_t o_tail = take(4ull * N_SCALES);
   const uint64_t o_dcdf = take(2ull * N_SCALES * DEC_CDF_STRIDE);
   const uint64_t o_cfm = take(8ull * N_SCALES * N_SYM);

@@ -21,11 +21,16 @@ namespace dckv {
 
 constexpr int RANS_WARPS = 4;                            // chunks per block
 constexpr int PF = 16;                                   // steps of look-ahead for state-free data
-constexpr int DEC_CDF_STRIDE = 512;                     // decoder cdf rows: 510 entries, then 0, 0
-constexpr int CDF_SMEM_BYTES = N_SCALES * DEC_CDF_STRIDE * 2;  // 65,536
+// Decoder tables in shared memory.  Rows are padded by 4 bytes so that the same entry of
+// different scales falls in different banks: most lanes of a step decode the central
+// symbol, each under its own component's scale, and unpadded 1 KiB / 2 KiB rows would put
+// all of them in one bank.
+constexpr int DEC_CDF_STRIDE = 514;                      // 510 entries, then zeros
+constexpr int CDF_SMEM_BYTES = N_SCALES * DEC_CDF_STRIDE * 2;  // 65,792
 constexpr int LUT_BITS = 10;                             // decoder lookup on slot >> 6
 constexpr int LUT_SIZE = 1 << LUT_BITS;
-constexpr int LUT_SMEM_BYTES = N_SCALES * LUT_SIZE * 2;  // 131,072
+constexpr int LUT_STRIDE = LUT_SIZE + 2;
+constexpr int LUT_SMEM_BYTES = N_SCALES * LUT_STRIDE * 2;  // 131,328
 constexpr int TAIL_SMEM_BYTES = N_SCALES * 4;
 constexpr int RANS_DEC_SMEM = CDF_SMEM_BYTES + LUT_SMEM_BYTES + TAIL_SMEM_BYTES + N_COEF;
 constexpr uint32_t CF_INVALID = 0xFFFFFFFFu;  // no table entry has cdf 65535 and freq 65536
@@ -373,7 +378,7 @@ __global__ void __launch_bounds__(COMPACT_THREADS) compact_kernel(CompactArgs a)
 
 // ------------------------------------------------------------------------------ decode
 // Decoder tables, per scale s:
-//   dcdf[s][0..509] = cdf, dcdf[s][510] = dcdf[s][511] = 0 (65536 mod 2^16, so that
+//   dcdf[s][0..509] = cdf, dcdf[s][510..513] = 0 (65536 mod 2^16, so that
 //     freq = (dcdf[sym + 1] - dcdf[sym]) mod 2^16 for every symbol);
 //   lut[s][b] for the 64 slots b * 64 .. b * 64 + 63: bits 0-9 the symbol holding the
 //     first of them, LUT_SINGLE if one symbol holds all of them, LUT_MULTI if two or more
@@ -397,8 +402,9 @@ __global__ void k_build_lut(const uint16_t *cdf, uint16_t *dcdf, uint16_t *lut, 
     const uint32_t slot = (uint32_t)b << (16 - LUT_BITS);
     const int lo = holder(slot);
     const int hi = holder(slot + (1u << (16 - LUT_BITS)) - 1u);
-    lut[s * LUT_SIZE + b] = (uint16_t)(lo | (hi == lo ? LUT_SINGLE : 0) | (hi >= lo + 2 ? LUT_MULTI : 0));
+    lut[s * LUT_STRIDE + b] = (uint16_t)(lo | (hi == lo ? LUT_SINGLE : 0) | (hi >= lo + 2 ? LUT_MULTI : 0));
   }
+  if (threadIdx.x < LUT_STRIDE - LUT_SIZE) lut[s * LUT_STRIDE + LUT_SIZE + threadIdx.x] = 0;
   for (int k = threadIdx.x; k < DEC_CDF_STRIDE; k += blockDim.x) {
     dcdf[s * DEC_CDF_STRIDE + k] = k < N_SYM ? tab[k] : (uint16_t)0;
     if (k < N_SYM) {
@@ -422,7 +428,7 @@ __device__ __forceinline__ int find_symbol(uint32_t slot, int s, const uint16_t 
                                            const uint32_t *s_tail, uint32_t &c, uint32_t &f) {
   const uint16_t *tab = s_cdf + s * DEC_CDF_STRIDE;
   const uint32_t b = slot >> (16 - LUT_BITS);
-  const uint32_t e = s_lut[s * LUT_SIZE + b];
+  const uint32_t e = s_lut[s * LUT_STRIDE + b];
   int sym = (int)(e & LUT_SYM);
   if (!(e & LUT_MULTI)) {
     const uint32_t c0 = tab[sym], c1 = tab[sym + 1], c2 = tab[sym + 2];
@@ -444,7 +450,7 @@ __device__ __forceinline__ int find_symbol(uint32_t slot, int s, const uint16_t 
     f = 1;
     return (int)(slot - (PREC_TOTAL - (uint32_t)N_SYM));
   }
-  int hi = b + 1 < (uint32_t)LUT_SIZE ? (int)(s_lut[s * LUT_SIZE + b + 1] & LUT_SYM) : N_SYM - 1;  // in [sym, hi]
+  int hi = b + 1 < (uint32_t)LUT_SIZE ? (int)(s_lut[s * LUT_STRIDE + b + 1] & LUT_SYM) : N_SYM - 1;  // in [sym, hi]
   while (hi > sym) {
     const int mid = (sym + hi + 1) >> 1;
     if (tab[mid] <= slot) sym = mid; else hi = mid - 1;
