@@ -170,7 +170,7 @@ template <class Epi, int STAGES, int MAX_SLABS, int CHUNK_STEPS, int BN>
 static int run_gemm2_chunked(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &b0,
                              const CUtensorMap &b1, GemmProblem prob, const typename Epi::Params &ep, int num_sms,
                              bool bf16, cudaStream_t st) {
-  constexpr int smem = gemm2_chunked_smem_bytes<Epi, STAGES, MAX_SLABS>();
+  constexpr int smem = gemm2_chunked_smem_bytes<Epi, STAGES, MAX_SLABS, BN>();
   static_assert(smem <= 232448, "GEMM shared memory above the sm_100 limit");
   auto kern = gemm2_chunked_kernel<Epi, STAGES, MAX_SLABS, CHUNK_STEPS, BN>;
   CK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
@@ -185,24 +185,6 @@ static int run_gemm2_chunked(const CUtensorMap &a0, const CUtensorMap &a1, const
   return launch_pairs((const void *)kern, tiles, num_sms, GEMM2C_THREADS, smem, st, args);
 }
 
-template <class Epi, int STAGES, int MAX_SLABS, int CHUNK_STEPS>
-static int run_gemm_chunked(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &b0,
-                            const CUtensorMap &b1, const GemmProblem &prob, const typename Epi::Params &ep,
-                            int num_sms, cudaStream_t st) {
-  constexpr int smem = gemm_chunked_smem_bytes<Epi, STAGES, MAX_SLABS>();
-  static_assert(smem <= 232448, "GEMM shared memory above the sm_100 limit");
-  auto kern = gemm_chunked_kernel<Epi, STAGES, MAX_SLABS, CHUNK_STEPS>;
-  CK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-  const int tiles = prob.m_tiles * prob.n_tiles;
-  if (tiles <= 0) return DCKV_OK;
-  if (prob.bn != GEMMC_BN) return fail(DCKV_EINVAL, "chunked GEMM tile width mismatch");
-  for (int i = 0; i < prob.n_seg; ++i)
-    if (prob.seg[i].n_slab < 1 || prob.seg[i].n_slab > MAX_SLABS) return fail(DCKV_EINVAL, "bad slab count");
-  const int grid = std::min(tiles, num_sms);
-  { kern<<<grid, GEMMC_THREADS, smem, st>>>(a0, a1, b0, b1, prob, ep); ++g_launches; }
-  CK(cudaGetLastError());
-  return DCKV_OK;
-}
 
 static GemmProblem make_problem(int m_tiles, int64_t n_rows, int bn, bool bf16, int32_t *status) {
   GemmProblem p;
@@ -1150,18 +1132,17 @@ extern "C" int dckv_encode(const dckv_codec *c, const void *rows, const int32_t 
   CK(cudaGetLastError());
   stage_mark(c, st, "layout+convert");
   if (L.n_rows > 0) {
-    CUtensorMap mb_x128, mb_xt, mb_gt, mb_qe;
-    RET(map_b(&mb_x128, x16, false, ROW_DIM, L.n_rows, 128));
+    CUtensorMap mb_xh, mb_xt, mb_gt, mb_qe;
+    RET(map_b(&mb_xh, x16, false, ROW_DIM, L.n_rows, HIDDEN_BN / 2));
     RET(map_b(&mb_xt, x16, false, ROW_DIM, L.n_rows, TRANSFORM_BN / 2));
     RET(map_b(&mb_gt, g16, false, 2 * N_HIDDEN, L.n_rows, TRANSFORM_BN / 2));
     RET(map_b(&mb_qe, qe, true, N_COEF, L.ne_pad, MEAN_ODD_BN / 2));
     // correction hidden layer: h = x @ w1 - mu @ w1, GELU, fp16 hi/lo
     {
-      GemmProblem pr = make_problem(N_HIDDEN / GEMM_BM, L.n_rows, 128, false, status_dev);
+      GemmProblem pr = make_problem(N_HIDDEN / GEMM_BM, L.n_rows, HIDDEN_BN, false, status_dev);
       add_seg(pr, 0, 0, 2, 0, 0, 0, 0, ROW_DIM / GEMM_BK);
       EpiGelu::Params ep{c->muw1, (float)std::ldexp(1.0, -c->p_h), g16};
-      RET((run_gemm_chunked<EpiGeluTotals, 4, 2, 4>(c->map_ah2, c->map_ah2, mb_x128, mb_x128, pr, ep,
-                                                          c->num_sms, st)));
+      RET((run_gemm2<EpiGelu, 4, 2, 4>(c->map_ah2, c->map_ah2, mb_xh, mb_xh, pr, ep, c->num_sms, false, st)));
     }
     stage_mark(c, st, "gemm_hidden");
     // transform + quantiser: y = x @ B + g @ w2 - mu @ B

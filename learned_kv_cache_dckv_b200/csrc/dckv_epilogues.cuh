@@ -52,32 +52,22 @@ struct EpiGelu {
     float scale;
     __half *g;  // [rows][512]
   };
-};
-
-// Chunk-accumulated form of EpiGelu (the hidden units feed the exact refinement too):
-// reads this thread's totals (columns c_begin .. c_begin + 63) from TMEM.
-struct EpiGeluTotals {
-  using Params = EpiGelu::Params;
   static constexpr int SMEM_BYTES = 0;
-  __device__ __forceinline__ static void tile(const Params &p, char *, int mt, int n0, int n_valid, int c_begin, uint32_t ttot,
-                              int ew, int lane, int) {
-    const int m = mt * GEMM_BM + ew * 32 + lane;
+  __device__ __forceinline__ static void tile(const Params &p, const EpiCtx &cx) {
+    const int m = cx.mt * GEMM_BM + cx.ew * 32 + cx.lane;
     const float mw = p.muw1[m];
-#pragma unroll 1
-    for (int g = 0; g < 2; ++g) {
-      const int col0 = c_begin + g * 32;
-      if (col0 >= n_valid) break;
+    for (int c0 = cx.grp * 32; c0 < cx.n_valid; c0 += 32 * cx.n_grp) {
       uint32_t r[32];
-      tmem_ld_32x32b_x32(ttot + (uint32_t)(g * 32), r);
+      tmem_ld_32x32b_x32(cx.tacc + (uint32_t)c0, r);
       tmem_ld_wait();
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
-        if (col0 + j < n_valid) {
+        if (c0 + j < cx.n_valid) {
           const float h = u2f(r[j]) * p.scale - mw;
-          const float gl = 0.5f * h * (1.0f + erff(h * 0.70710678118654752f));
-          const __half hi = __float2half_rn(gl);
-          const __half lo = __float2half_rn(gl - __half2float(hi));
-          __half *row = p.g + (int64_t)(n0 + col0 + j) * (2 * N_HIDDEN);
+          const float g = 0.5f * h * (1.0f + erff(h * 0.70710678118654752f));
+          const __half hi = __float2half_rn(g);
+          const __half lo = __float2half_rn(g - __half2float(hi));
+          __half *row = p.g + (int64_t)(cx.n0 + c0 + j) * (2 * N_HIDDEN);
           row[m] = hi;
           row[N_HIDDEN + m] = lo;
         }

@@ -249,9 +249,10 @@ constexpr int gemm_smem_bytes() {
 // prob.m_tiles counts 128-row tiles and must be even; prob.bn <= 256, bn / 2 a multiple of 8.
 constexpr int GEMM_B_HALF_BYTES = (GEMM_MAX_BN / 2) * GEMM_BK * 2;  // 16 KiB
 
-template <int MAX_SLABS>
-struct Gemm2Smem {
-  static constexpr int STAGE_BYTES = MAX_SLABS * GEMM_SLAB_BYTES + GEMM_B_HALF_BYTES;
+template <int MAX_SLABS, int BN = GEMM_MAX_BN>
+struct Gemm2Smem {  // one stage: the A slabs, then this CTA's half of the B tile (a multiple of 1 KiB)
+  static_assert((BN / 2) % 8 == 0, "half tile must hold whole 8-row swizzle atoms");
+  static constexpr int STAGE_BYTES = MAX_SLABS * GEMM_SLAB_BYTES + (BN / 2) * GEMM_BK * 2;
 };
 
 template <class Epi, int STAGES, int MAX_SLABS, int EPI_WARPS>
@@ -460,7 +461,7 @@ __global__ void __launch_bounds__(GEMM2C_THREADS, 1)
   static_assert(BN % 32 == 0 && BN <= GEMM_MAX_BN, "BN / 2 must be a multiple of 16");
   constexpr int NC = BN / 2;  // columns per epilogue thread
   extern __shared__ __align__(1024) uint8_t dyn_smem[];
-  constexpr int STAGE_BYTES = Gemm2Smem<MAX_SLABS>::STAGE_BYTES;
+  constexpr int STAGE_BYTES = Gemm2Smem<MAX_SLABS, BN>::STAGE_BYTES;
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
   uint8_t *stages = base;
   uint64_t *full_bar = reinterpret_cast<uint64_t *>(base + STAGES * STAGE_BYTES);
@@ -663,218 +664,10 @@ __global__ void __launch_bounds__(GEMM2C_THREADS, 1)
   }
 }
 
-template <class Epi, int STAGES, int MAX_SLABS>
+template <class Epi, int STAGES, int MAX_SLABS, int BN>
 constexpr int gemm2_chunked_smem_bytes() {
-  return 1024 + STAGES * Gemm2Smem<MAX_SLABS>::STAGE_BYTES + 1024 + 2 * ((Epi::SMEM_BYTES + 15) & ~15);
+  return 1024 + STAGES * Gemm2Smem<MAX_SLABS, BN>::STAGE_BYTES + 1024 + 2 * ((Epi::SMEM_BYTES + 15) & ~15);
 }
 
-// ------------------------------------------------------------------------------------------
-// Chunk-accumulated variant (bn = 128).  The tensor core sums each MMA's products into the
-// fp32 accumulator with truncation, so over a long K the error grows with the number of
-// MMA steps times the accumulator's ulp.  Here every CHUNK_STEPS * 64 elements of K go into
-// a fresh TMEM partial P (two alternate, columns 0-127 and 128-255), and the epilogue warps
-// add each partial into a TMEM running total T (two alternate per tile, columns 256-383
-// and 384-511) with fp32 round-to-nearest adds.  After a tile's last chunk, Epi::tile reads
-// its totals from T.  Eight epilogue warps: warp w >= 2 owns TMEM lane quarter w % 4 and
-// column half (w - 2) / 4 (64 columns).
-constexpr int GEMMC_THREADS = 320;
-constexpr int GEMMC_BN = 128;
-
-template <class Epi, int STAGES, int MAX_SLABS, int CHUNK_STEPS>
-__global__ void __launch_bounds__(GEMMC_THREADS, 1)
-    gemm_chunked_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
-                        const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
-                        const GemmProblem prob, const typename Epi::Params ep) {
-  extern __shared__ __align__(1024) uint8_t dyn_smem[];
-  constexpr int STAGE_BYTES = GemmSmem<MAX_SLABS, GEMMC_BN>::STAGE_BYTES;
-  uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
-  uint8_t *stages = base;
-  uint64_t *full_bar = reinterpret_cast<uint64_t *>(base + STAGES * STAGE_BYTES);
-  uint64_t *empty_bar = full_bar + STAGES;
-  uint64_t *part_full = empty_bar + STAGES;
-  uint64_t *part_empty = part_full + 2;
-  uint32_t *tmem_base_smem = reinterpret_cast<uint32_t *>(part_empty + 2);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_base_smem + 1);
-  char *epi_scratch = reinterpret_cast<char *>(base + STAGES * STAGE_BYTES + 1024);
-
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const int total_tiles = prob.m_tiles * prob.n_tiles;
-  int ksteps = 0;
-  for (int si = 0; si < prob.n_seg; ++si) ksteps += prob.seg[si].k_steps;
-  const int n_chunks = (ksteps + CHUNK_STEPS - 1) / CHUNK_STEPS;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full_bar[s], 1);
-      mbar_init(&empty_bar[s], 1);
-    }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(&part_full[a], 1);
-      mbar_init(&part_empty[a], 256);
-    }
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == 0 && lane == 0) {
-    prefetch_tmap(&tmA0);
-    prefetch_tmap(&tmA1);
-    prefetch_tmap(&tmB0);
-    prefetch_tmap(&tmB1);
-  }
-  if (warp == 1) {
-    tmem_alloc(tmem_base_smem, 512);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem_base = *tmem_base_smem;
-
-  if (warp == 0) {
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
-        const int mt = t % prob.m_tiles;
-        const int n0 = (t / prob.m_tiles) * prob.bn;
-        for (int si = 0; si < prob.n_seg; ++si) {
-          const GemmSeg sg = prob.seg[si];
-          const void *ta = sg.a_map ? (const void *)&tmA1 : (const void *)&tmA0;
-          const void *tb = sg.b_map ? (const void *)&tmB1 : (const void *)&tmB0;
-          const uint32_t bytes = (uint32_t)(sg.n_slab * GEMM_SLAB_BYTES + prob.bn * GEMM_BK * 2);
-          for (int ks = 0; ks < sg.k_steps; ++ks) {
-            if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) goto producer_done;
-            uint8_t *sa = stages + stage * STAGE_BYTES;
-            uint8_t *sb = sa + MAX_SLABS * GEMM_SLAB_BYTES;
-            mbar_arrive_expect_tx(&full_bar[stage], bytes);
-            tma_load_3d(sa, ta, &full_bar[stage], sg.a_k0 + ks * GEMM_BK, mt * GEMM_BM, sg.a_slab0);
-            tma_load_2d(sb, tb, &full_bar[stage], sg.b_k0 + ks * GEMM_BK, n0 + sg.b_row_shift);
-            if (++stage == STAGES) {
-              stage = 0;
-              phase ^= 1u;
-            }
-          }
-        }
-      }
-    producer_done:;
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      int pb = 0;
-      uint32_t pph = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
-        int in_chunk = 0, done = 0;
-        uint32_t d_tmem = 0, accumulate = 0;
-        for (int si = 0; si < prob.n_seg && ok; ++si) {
-          const GemmSeg sg = prob.seg[si];
-          for (int ks = 0; ks < sg.k_steps; ++ks) {
-            if (in_chunk == 0) {
-              if (!mbar_wait(&part_empty[pb], pph ^ 1u, abort_flag)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
-              d_tmem = tmem_base + (uint32_t)(pb * GEMMC_BN);
-              accumulate = 0;
-            }
-            if (!mbar_wait(&full_bar[stage], phase, abort_flag)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t sa = smem_u32(stages + stage * STAGE_BYTES);
-            const uint32_t sb = sa + MAX_SLABS * GEMM_SLAB_BYTES;
-            for (int sl = 0; sl < sg.n_slab; ++sl) {
-#pragma unroll
-              for (int kk = 0; kk < GEMM_BK / 16; ++kk) {
-                umma_f16(d_tmem, sw128_desc(sa + sl * GEMM_SLAB_BYTES + kk * 32), sw128_desc(sb + kk * 32),
-                         prob.idesc, accumulate);
-                accumulate = 1;
-              }
-            }
-            umma_commit(&empty_bar[stage]);
-            if (++stage == STAGES) {
-              stage = 0;
-              phase ^= 1u;
-            }
-            ++done;
-            if (++in_chunk == CHUNK_STEPS || done == ksteps) {
-              umma_commit(&part_full[pb]);
-              in_chunk = 0;
-              if (++pb == 2) {
-                pb = 0;
-                pph ^= 1u;
-              }
-            }
-          }
-        }
-      }
-    }
-  } else {
-    const int et = threadIdx.x - 64;  // 0..255
-    const int ew = warp & 3;
-    const int half = (warp - 2) >> 2;
-    const uint32_t lane_base = (uint32_t)(ew * 32) << 16;
-    int pb = 0, tbuf = 0;
-    uint32_t pph = 0;
-    bool stop = false;
-    for (int t = blockIdx.x; t < total_tiles && !stop; t += gridDim.x) {
-      const int mt = t % prob.m_tiles;
-      const int n0 = (t / prob.m_tiles) * prob.bn;
-      const int n_valid = min(prob.bn, prob.n_rows - n0);
-      const uint32_t tot = tmem_base + lane_base + (uint32_t)(2 * GEMMC_BN + tbuf * GEMMC_BN + half * 64);
-      for (int ch = 0; ch < n_chunks; ++ch) {
-        if (!mbar_wait(&part_full[pb], pph, abort_flag)) {
-          stop = true;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t part = tmem_base + lane_base + (uint32_t)(pb * GEMMC_BN + half * 64);
-#pragma unroll 1
-        for (int g = 0; g < 2; ++g) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(part + g * 32, r);
-          if (ch > 0) {
-            uint32_t s[32];
-            tmem_ld_32x32b_x32(tot + g * 32, s);
-            tmem_ld_wait();
-#pragma unroll
-            for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) + __uint_as_float(s[j]));
-          } else {
-            tmem_ld_wait();
-          }
-          tmem_st_32x32b_x32(tot + g * 32, r);
-        }
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(&part_empty[pb]);
-        if (++pb == 2) {
-          pb = 0;
-          pph ^= 1u;
-        }
-      }
-      if (stop) break;
-      tc_fence_after();
-      Epi::tile(ep, epi_scratch, mt, n0, n_valid, half * 64, tot, ew, lane, et);
-      tbuf ^= 1;
-    }
-  }
-
-  __syncthreads();
-  if (*abort_flag && threadIdx.x == 0 && prob.status) atomicExch(prob.status, 5);
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem_base, 512);
-  }
-}
-
-template <class Epi, int STAGES, int MAX_SLABS>
-constexpr int gemm_chunked_smem_bytes() {
-  return 1024 + STAGES * GemmSmem<MAX_SLABS, GEMMC_BN>::STAGE_BYTES + 1024 + Epi::SMEM_BYTES;
-}
 
 }  // namespace dckv

@@ -45,6 +45,9 @@ constexpr float REFINE_NORM_FULL = 32.0f;
 constexpr int TRANSFORM_BN = 224;
 constexpr int MEAN_ODD_BN = 224;
 constexpr int INVERSE_BN = 224;
+// correction hidden layer: one 256-row pair tile in M, so narrow token tiles (62 pairs for
+// a 4K-token prompt) spread the GEMM over the GPU
+constexpr int HIDDEN_BN = 64;
 // K steps (of 64) per TMEM partial of the transform before it is added into the fp32
 // totals: bounds the growth of the tensor core's accumulation error over K = 6,144.
 constexpr int TRANSFORM_CHUNK_STEPS = 4;
