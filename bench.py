@@ -30,10 +30,13 @@ CONFIGS = {
     "c1": ([256], None, 0.0, "1 x 256-token prompt (124 coded rows), literal codec b = 0.6 Delta"),
     "c2": ([4096], 220.0, 0.0, "1 x 4096-token prompt, 6144-dim bf16 rows, step scale for ~220 B/token"),
     "c3": ([32768], 220.0, 0.0, "1 x 32768-token prompt, ~220 B/token"),
-    "c3b": ([32768], 110.0, 0.0, "1 x 32768-token prompt, ~110 B/token (many components dropped)"),
+    "c3b": ([32768], 110.0, 0.0, "1 x 32768-token prompt, ~110 B/token (many components dropped), 32 rows per chunk"),
     "c4": ([131072], 220.0, 0.0, "1 x 131072-token prompt, ~220 B/token"),
     "c5": ([4096] * 64, 220.0, 0.01, "64 x 4096-token prompts, 1% Student-t (nu=2) rows, ~220 B/token"),
 }
+
+# rows per rANS chunk (codec creation); 0 = the library default (16)
+CHUNK_ROWS = {"c3b": 32}
 
 GEMM_STAGES = {"gemm_hidden", "gemm_transform", "gemm_mean_odd", "gemm_inverse"}
 
@@ -233,7 +236,7 @@ def run_gpu(args):
     _, cod, x, tok, offs = make_inputs(args.config, rank, dev)
     n_tok = int(offs[-1])
     n_rows = sum(max(0, int(n) - 132) for n in np.diff(offs))
-    gc = D.Codec(D.upload_params(cod, dev), dev.index)
+    gc = D.Codec(D.upload_params(cod, dev), dev.index, CHUNK_ROWS.get(args.config, 0))
     stream = torch.cuda.current_stream()
     blob = torch.empty(D.dckv_blob_bound(gc.handle, offs), dtype=torch.uint8, device=dev)
     k_out = torch.empty((6, n_tok, 2, 256), dtype=torch.bfloat16, device=dev)

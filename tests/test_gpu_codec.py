@@ -331,6 +331,73 @@ def test_full_size_4k_prompt_sampled(src, codec_55):
     assert rel_frob(O.bf16_to_f64(vg), O.bf16_to_f64(want[:, :, 1])) <= ROW_TOL
 
 
+_FULL_CODECS = {}
+
+
+def _full_codec(src, target):
+    if target not in _FULL_CODECS:
+        _FULL_CODECS[target] = S.codec(src, step_scale=None, target_bytes=target)
+    return _FULL_CODECS[target]
+
+
+# the larger configurations: (prompt lengths, target bytes per coded row, Student-t fraction,
+# rows per rANS chunk).  At ~110 B per row a chunk's fixed 136 bytes need 32 rows to stay
+# within the 5% payload bound.
+FULL_CONFIGS = {
+    "32k_220B": ([32768], 220.0, 0.0, 16),
+    "32k_110B": ([32768], 110.0, 0.0, 32),
+    "131k_220B": ([131072], 220.0, 0.0, 16),
+    "64x4k_220B_student_t": ([4096] * 64, 220.0, 0.01, 16),
+}
+
+
+@pytest.mark.parametrize("name", sorted(FULL_CONFIGS))
+def test_full_size_configs_sampled(src, name):
+    """Full-size configurations: sampled rows' codes against the oracle, the whole blob
+    re-coded by the oracle coder from the GPU's codes and centres, the payload against the
+    model code length, exact code round trip through the GPU decoder, and sampled decoded
+    rows against the oracle's reconstruction."""
+    lens, target, st, chunk_rows = FULL_CONFIGS[name]
+    cod = _full_codec(src, target)
+    gc = gpu_codec(cod, chunk_rows)
+    seeds = [200 + 7 * i for i in range(len(lens))]
+    x, tok, offs = make_batch(src, cod, lens, seeds, student_t=st)
+    res = encode_gpu(gc, x, tok, offs)
+    assert res["status"] == D.DCKV_OK, D.STATUS_NAMES[res["status"]]
+    lay = O.prompt_layout(np.diff(offs))
+    n = sum(L["n"] for L in lay)
+    rng = np.random.default_rng(1)
+    rows = np.sort(rng.choice(n, 48, replace=False))  # coded-row indices over the batch
+    starts = np.array([L["row_base"] for L in lay])
+    pidx = np.searchsorted(starts, rows, side="right") - 1
+    tok_rows = np.array([lay[p]["tok_base"] + 4 + (r - lay[p]["row_base"]) for p, r in zip(pidx, rows)])
+    pos = np.array([4 + (r - lay[p]["row_base"]) for p, r in zip(pidx, rows)])
+    xb = bits(x)
+    keep = O.scale_index(cod.laplace_b, cod.delta)[1]
+    q_o, ratio = O.quantise(O.transform(xb[tok_rows], cod), cod.delta, keep)
+    check_codes(res["q32"][rows].astype(np.int64), dict(q=q_o, ratio=ratio))
+    codes = split_gpu_codes(gc, cod, res, tok, offs)
+    aux = {}
+    G = D.dckv_codec_info(gc.handle)["chunk_rows"]
+    ora_blob = O.assemble_blob(xb, offs, codes, cod.laplace_b, cod.delta, G, aux=aux)
+    assert len(ora_blob) == res["size"] and ora_blob == res["blob"]
+    kept = sum(L["N"] - L["n"] for L in lay)
+    payload = res["size"] - kept * 12288
+    assert payload <= 1.05 * aux["code_bits"] / 8, (payload, aux["code_bits"] / 8)
+    if st > 0:
+        assert aux["n_esc"] > 0  # heavy-tailed rows force escapes
+    k, v, status, q16 = decode_gpu(gc, res["blob_dev"], res["size"], tok, offs)
+    assert status == D.DCKV_OK
+    small = np.abs(res["q32"]) < 2048
+    assert np.array_equal(q16[small], res["q32"][small].astype(np.float32))
+    xh = O.reconstruct(res["q32"][rows].astype(np.int64), cod)
+    want = O.f64_to_bf16(O.output_rows(xh, pos)).reshape(-1, 6, 2, 2, 256)
+    kg = bits(k)[:, tok_rows].transpose(1, 0, 2, 3)
+    vg = bits(v)[:, tok_rows].transpose(1, 0, 2, 3)
+    assert rel_frob(O.bf16_to_f64(kg), O.bf16_to_f64(want[:, :, 0])) <= ROW_TOL
+    assert rel_frob(O.bf16_to_f64(vg), O.bf16_to_f64(want[:, :, 1])) <= ROW_TOL
+
+
 @pytest.mark.parametrize("which", ["literal", "fitted"])
 def test_guard_band_bounds_fp32_error(src, codec_literal, codec_55, which):
     """The fp32 transform ratio y / Delta (before exact recomputation) stays within the
