@@ -33,6 +33,8 @@ CONFIGS = {
     "c3b": ([32768], 110.0, 0.0, "1 x 32768-token prompt, ~110 B/token (many components dropped), 32 rows per chunk"),
     "c4": ([131072], 220.0, 0.0, "1 x 131072-token prompt, ~220 B/token"),
     "c5": ([4096] * 64, 220.0, 0.01, "64 x 4096-token prompts, 1% Student-t (nu=2) rows, ~220 B/token"),
+    "c2lin": ([4096], 220.0, 0.0, "1 x 4096-token prompt, linear codec (no correction, unconditional "
+                                  "zero-mean tables), step scale for ~220 B/token"),
 }
 
 # rows per rANS chunk (codec creation); 0 = the library default (16)
@@ -125,10 +127,11 @@ def make_inputs(cfg_name, rank, device):
 
     lens, target, st, _ = CONFIGS[cfg_name]
     src = S.source(0)
+    linear = cfg_name.endswith("lin")
     if target is None:
-        cod = S.codec(src, step_scale=1.0, literal_b=True)
+        cod = S.codec(src, step_scale=1.0, literal_b=True, linear=linear)
     else:
-        cod = S.codec(src, step_scale=None, target_bytes=target)
+        cod = S.codec(src, step_scale=None, target_bytes=target, linear=linear)
     seeds = [1000 * rank + i for i in range(len(lens))]
     x, tok, offs = S.batch(src, lens, seeds, student_t_frac=st, device=device)
     return src, cod, x, tok, offs

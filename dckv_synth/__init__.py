@@ -129,13 +129,13 @@ class Codec:
 
     mu: np.ndarray  # fp32 [6144]        codec mean
     basis: np.ndarray  # fp32 [6144, 2048]  shared linear basis (columns)
-    w1: np.ndarray  # fp32 [6144, 256]   correction, first layer
-    w2: np.ndarray  # fp32 [256, 2048]   correction, second layer
+    w1: np.ndarray | None  # fp32 [6144, 256]   correction, first layer (None: linear codec)
+    w2: np.ndarray | None  # fp32 [256, 2048]   correction, second layer
     delta: np.ndarray  # fp32 [2048]        quantiser steps (data units)
     laplace_b: np.ndarray  # fp32 [2048]    Laplace scales (data units)
-    embed: np.ndarray  # u16 bf16 bits [32768, 2048]
-    w_even: np.ndarray  # u16 bf16 bits [2048, 2048]   mu_even = e @ w_even
-    w_odd: np.ndarray  # u16 bf16 bits [6144, 2048]    mu_odd = [e, bf16(qL), bf16(qR)] @ w_odd
+    embed: np.ndarray | None  # u16 bf16 bits [32768, 2048] (None: unconditional tables)
+    w_even: np.ndarray | None  # u16 bf16 bits [2048, 2048]   mu_even = e @ w_even
+    w_odd: np.ndarray | None  # u16 bf16 bits [6144, 2048]    mu_odd = [e, bf16(qL), bf16(qR)] @ w_odd
     step_scale: float
     note: str = ""
 
@@ -200,6 +200,7 @@ def codec(
     neigh_gain: float = 1.0,
     zero_mlp: bool = False,
     seed: int | None = None,
+    linear: bool = False,
 ) -> Codec:
     """Draw a synthetic codec.
 
@@ -208,6 +209,8 @@ def codec(
     literal_b: b_c = 0.6 * Delta_c (the small configuration as written) instead of the fit.
     mean_gain / neigh_gain scale the mean-model weights (test variants with non-zero
     centres); zero_mlp sets the correction to zero (its initial state on the pages).
+    linear: the linear codec the pages compare against -- no correction (w1 = w2 = None)
+    and unconditional zero-mean tables (embed = w_even = w_odd = None).
     """
     seed = src.seed if seed is None else seed
     rng = np.random.default_rng([seed, 0x53])
@@ -248,10 +251,13 @@ def codec(
     w_odd_n = 0.02 * neigh_gain * rng.standard_normal((2 * N_COEF, N_COEF))
     w_odd_n *= np.concatenate([delta, delta]).astype(np.float64)[:, None]
     w_odd = f32_to_bf16_bits(np.concatenate([w_odd_e, w_odd_n], axis=0))
+    if linear:
+        w1 = w2 = embed = w_even = w_odd = None
     return Codec(
         mu=src.mu.copy(), basis=basis, w1=w1, w2=w2, delta=delta, laplace_b=b,
         embed=embed, w_even=w_even, w_odd=w_odd, step_scale=float(step_scale),
-        note=("literal b=0.6*Delta" if literal_b else "fitted b") + (", zero MLP" if zero_mlp else ""),
+        note=("literal b=0.6*Delta" if literal_b else "fitted b") + (", zero MLP" if zero_mlp else "")
+        + (", linear codec" if linear else ""),
     )
 
 

@@ -66,7 +66,11 @@ extern "C" {
 typedef struct dckv_codec dckv_codec; /* opaque */
 
 /* Codec weights, as trained (here: seeded synthetics).  All DEVICE pointers, read only,
- * caller-owned; they are read during dckv_codec_create and may be freed afterwards. */
+ * caller-owned; they are read during dckv_codec_create and may be freed afterwards.
+ * The linear codec the pages compare DCKV with ("Evidence": no correction, unconditional
+ * zero-mean Laplace tables) is w1 = w2 = NULL and embed = w_even = w_odd = NULL (vocab
+ * ignored); either pair may be absent on its own.  Without mean models every centre is 0
+ * and token_ids may be NULL in encode and decode. */
 typedef struct {
   const float *mu;          /* [6144]        codec mean subtracted before the transform   */
   const float *basis;       /* [6144][2048]  shared basis, row-major (basis[d*2048 + c])  */
@@ -78,7 +82,7 @@ typedef struct {
   const uint16_t *w_even;   /* bf16 [2048][2048] even mean model: mu = e @ w_even         */
   const uint16_t *w_odd;    /* bf16 [6144][2048] odd mean model: mu = [e, bf16(q_left),
                                bf16(q_right)] @ w_odd; the neighbour blocks carry Delta_c */
-  int32_t vocab;            /* rows of embed (1 .. 2^20)                                 */
+  int32_t vocab;            /* rows of embed (1 .. 2^20; ignored without mean models)    */
 } dckv_params;
 
 /* Per-blob byte accounting (host-side parse of a blob header and tables). */

@@ -121,6 +121,11 @@ def _offs(seq_offsets):
     return a, a.ctypes.data_as(ctypes.c_void_p), a.size - 1
 
 
+def _ptr(t):
+    """Device address of a tensor, or NULL for None (token ids of a codec without mean models)."""
+    return None if t is None else t.data_ptr()
+
+
 def _stream_ptr(stream):
     import torch
 
@@ -132,11 +137,13 @@ def _stream_ptr(stream):
 # ---------------------------------------------------------------------------------- C ABI
 def dckv_codec_create(params: dict, device: int = 0, chunk_rows: int = 0):
     """params: device tensors mu, basis, w1, w2, delta, laplace_b (fp32), embed, w_even,
-    w_odd (bf16 or int16 holding bf16 bits); returns an opaque handle."""
+    w_odd (bf16 or int16 holding bf16 bits); w1 / w2 None for a linear codec, embed /
+    w_even / w_odd None for unconditional tables.  Returns an opaque handle."""
     p = _Params()
     for k in ("mu", "basis", "w1", "w2", "delta", "laplace_b", "embed", "w_even", "w_odd"):
-        setattr(p, k, params[k].data_ptr())
-    p.vocab = int(params["embed"].shape[0])
+        v = params.get(k)
+        setattr(p, k, None if v is None else v.data_ptr())
+    p.vocab = 0 if params.get("embed") is None else int(params["embed"].shape[0])
     h = ctypes.c_void_p()
     _check(lib().dckv_codec_create(ctypes.byref(p), int(device), int(chunk_rows), ctypes.byref(h)),
            "dckv_codec_create")
@@ -165,7 +172,7 @@ def dckv_encode(handle, rows, token_ids, seq_offsets, blob, blob_size, status, w
     """rows bf16 [sum N, 6144], token_ids int32 [sum N], blob uint8 (device), blob_size
     uint64[1]/int64[1] (device), status int32[1] (device), workspace uint8 (device)."""
     a, ptr, b = _offs(seq_offsets)
-    _check(lib().dckv_encode(handle, rows.data_ptr(), token_ids.data_ptr(), ptr, b, blob.data_ptr(),
+    _check(lib().dckv_encode(handle, rows.data_ptr(), _ptr(token_ids), ptr, b, blob.data_ptr(),
                              blob.numel() * blob.element_size(), blob_size.data_ptr(), status.data_ptr(),
                              workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                              _stream_ptr(stream)), "dckv_encode")
@@ -173,7 +180,7 @@ def dckv_encode(handle, rows, token_ids, seq_offsets, blob, blob_size, status, w
 
 def dckv_decode(handle, blob, blob_bytes, token_ids, seq_offsets, k_out, v_out, status, workspace, stream=None):
     a, ptr, b = _offs(seq_offsets)
-    _check(lib().dckv_decode(handle, blob.data_ptr(), int(blob_bytes), token_ids.data_ptr(), ptr, b,
+    _check(lib().dckv_decode(handle, blob.data_ptr(), int(blob_bytes), _ptr(token_ids), ptr, b,
                              k_out.data_ptr(), v_out.data_ptr(), status.data_ptr(), workspace.data_ptr(),
                              workspace.numel() * workspace.element_size(), _stream_ptr(stream)), "dckv_decode")
 
@@ -181,7 +188,7 @@ def dckv_decode(handle, blob, blob_bytes, token_ids, seq_offsets, k_out, v_out, 
 def dckv_decode_static(handle, blob, blob_bytes, token_ids, seq_offsets, k_out, v_out, status, stream=None):
     """dckv_decode on the library's static per-device scratch (no workspace argument)."""
     a, ptr, b = _offs(seq_offsets)
-    _check(lib().dckv_decode_static(handle, blob.data_ptr(), int(blob_bytes), token_ids.data_ptr(), ptr, b,
+    _check(lib().dckv_decode_static(handle, blob.data_ptr(), int(blob_bytes), _ptr(token_ids), ptr, b,
                                     k_out.data_ptr(), v_out.data_ptr(), status.data_ptr(), _stream_ptr(stream)),
            "dckv_decode_static")
 
@@ -257,9 +264,14 @@ def upload_params(codec, device="cuda"):
 
     out = {}
     for k in ("mu", "basis", "w1", "w2", "delta", "laplace_b"):
-        out[k] = torch.from_numpy(np.ascontiguousarray(getattr(codec, k), np.float32)).to(device)
+        v = getattr(codec, k)
+        out[k] = None if v is None else torch.from_numpy(np.ascontiguousarray(v, np.float32)).to(device)
     for k in ("embed", "w_even", "w_odd"):
-        a = np.ascontiguousarray(getattr(codec, k), np.uint16).view(np.int16)
+        v = getattr(codec, k)
+        if v is None:
+            out[k] = None
+            continue
+        a = np.ascontiguousarray(v, np.uint16).view(np.int16)
         out[k] = torch.from_numpy(a).to(device).view(torch.bfloat16)
     return out
 

@@ -638,9 +638,11 @@ __global__ void __launch_bounds__(256) k_refine_codes(const uint32_t *el_list, c
     const float *bt = bt32 + (int64_t)c * ROW_DIM;
     double acc = 0.0;
     for (int i = lane; i < ROW_DIM; i += 32) acc += ((double)__bfloat162float(xr[i]) - (double)mu32[i]) * (double)bt[i];
-    const __half *g = g16 + row * (2 * N_HIDDEN);
-    for (int h = lane; h < N_HIDDEN; h += 32)
-      acc += ((double)__half2float(g[h]) + (double)__half2float(g[N_HIDDEN + h])) * (double)w2t32[c * N_HIDDEN + h];
+    if (w2t32) {  // the correction (absent in a linear codec)
+      const __half *g = g16 + row * (2 * N_HIDDEN);
+      for (int h = lane; h < N_HIDDEN; h += 32)
+        acc += ((double)__half2float(g[h]) + (double)__half2float(g[N_HIDDEN + h])) * (double)w2t32[c * N_HIDDEN + h];
+    }
     acc = warp_sum(acc);
     if (lane == 0) store_code(row, c, acc / (double)delta[c], q32, qe, row_edst);
   }
@@ -662,7 +664,7 @@ __global__ void __launch_bounds__(256) k_refine_rows(const uint32_t *full_list, 
     const __nv_bfloat16 *xr = rows + (int64_t)row_tok[row] * ROW_DIM;
     for (int i = threadIdx.x; i < ROW_DIM; i += blockDim.x) xc[i] = (double)__bfloat162float(xr[i]) - (double)mu32[i];
     __syncthreads();
-    for (int h = warp; h < N_HIDDEN; h += nw) {
+    for (int h = warp; w1t32 && h < N_HIDDEN; h += nw) {
       const float *w = w1t32 + (int64_t)h * ROW_DIM;
       double acc = 0.0;
       for (int i = lane; i < ROW_DIM; i += 32) acc += xc[i] * (double)w[i];
@@ -674,7 +676,8 @@ __global__ void __launch_bounds__(256) k_refine_rows(const uint32_t *full_list, 
       const float *bt = bt32 + (int64_t)c * ROW_DIM;
       double acc = 0.0;
       for (int i = lane; i < ROW_DIM; i += 32) acc += xc[i] * (double)bt[i];
-      for (int h = lane; h < N_HIDDEN; h += 32) acc += gs[h] * (double)w2t32[c * N_HIDDEN + h];
+      if (w2t32)
+        for (int h = lane; h < N_HIDDEN; h += 32) acc += gs[h] * (double)w2t32[c * N_HIDDEN + h];
       acc = warp_sum(acc);
       if (lane == 0) store_code(row, c, keep[c] ? acc / (double)delta[c] : 0.0, q32, qe, row_edst);
     }
@@ -818,10 +821,13 @@ static void stage_mark(const dckv_codec *cc, cudaStream_t st, const char *name) 
 extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_rows, dckv_codec **out) {
   if (!out) return fail(DCKV_EINVAL, "out is NULL");
   *out = nullptr;
-  if (!prm || !prm->mu || !prm->basis || !prm->w1 || !prm->w2 || !prm->delta || !prm->laplace_b || !prm->embed ||
-      !prm->w_even || !prm->w_odd)
+  if (!prm || !prm->mu || !prm->basis || !prm->delta || !prm->laplace_b)
     return fail(DCKV_EINVAL, "a parameter pointer is NULL");
-  if (prm->vocab < 1 || prm->vocab > (1 << 20)) return fail(DCKV_EINVAL, "vocab out of range");
+  if (!prm->w1 != !prm->w2) return fail(DCKV_EINVAL, "w1 and w2 must both be given or both be NULL");
+  if (!prm->embed != !prm->w_even || !prm->embed != !prm->w_odd)
+    return fail(DCKV_EINVAL, "embed, w_even and w_odd must all be given or all be NULL");
+  const bool has_mlp = prm->w1 != nullptr, has_means = prm->embed != nullptr;
+  if (has_means && (prm->vocab < 1 || prm->vocab > (1 << 20))) return fail(DCKV_EINVAL, "vocab out of range");
   if (chunk_rows < -1 || chunk_rows > 256) return fail(DCKV_EINVAL, "chunk_rows out of range");
   if (((uintptr_t)prm->embed | (uintptr_t)prm->w_even | (uintptr_t)prm->w_odd) & 15)
     return fail(DCKV_EINVAL, "bf16 parameters must be 16-byte aligned");
@@ -836,7 +842,9 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
   c->device = device;
   c->num_sms = prop.multiProcessorCount;
   c->chunk_rows = chunk_rows;
-  c->vocab = prm->vocab;
+  c->vocab = has_means ? prm->vocab : 0;
+  c->has_mlp = has_mlp;
+  c->has_means = has_means;
   c->p = *prm;
   for (int i = 0; i < 24; ++i) cudaEventCreate(&c->ev[i]);
 
@@ -846,7 +854,7 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
   };
 
   // one device block for every derived tensor
-  const uint64_t V = (uint64_t)prm->vocab;
+  const uint64_t V = has_means ? (uint64_t)prm->vocab : 0;
   uint64_t o = 0;
   auto take = [&](uint64_t bytes) {
     const uint64_t at = o;
@@ -922,8 +930,10 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
   cudaMemcpyAsync(c->delta, prm->delta, 4ull * N_COEF, cudaMemcpyDeviceToDevice, st);
   // scale exponents: largest |value| of each split operand brought to about 2^12
   { k_absmax<<<256, 256, 0, st>>>(prm->basis, (int64_t)ROW_DIM * N_COEF, N_COEF, nullptr, scr + 1); ++g_launches; }
-  { k_absmax<<<64, 256, 0, st>>>(prm->w2, (int64_t)N_HIDDEN * N_COEF, N_COEF, nullptr, scr + 2); ++g_launches; }
-  { k_absmax<<<256, 256, 0, st>>>(prm->w1, (int64_t)ROW_DIM * N_HIDDEN, N_HIDDEN, nullptr, scr + 3); ++g_launches; }
+  if (has_mlp) {
+    { k_absmax<<<64, 256, 0, st>>>(prm->w2, (int64_t)N_HIDDEN * N_COEF, N_COEF, nullptr, scr + 2); ++g_launches; }
+    { k_absmax<<<256, 256, 0, st>>>(prm->w1, (int64_t)ROW_DIM * N_HIDDEN, N_HIDDEN, nullptr, scr + 3); ++g_launches; }
+  }
   { k_absmax<<<256, 256, 0, st>>>(prm->basis, (int64_t)ROW_DIM * N_COEF, N_COEF, prm->delta, scr + 4); ++g_launches; }
   int32_t host_scr[8];
   uint8_t keep_h[N_COEF], scale_h[N_COEF];
@@ -996,24 +1006,30 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
     return cleanup(fail(DCKV_ECUDA, "setup upload failed"));
   // mean projections in fp64
   { k_vec_mat<<<(N_COEF + 255) / 256, 256, 0, st>>>(prm->mu, prm->basis, ROW_DIM, N_COEF, c->mub); ++g_launches; }
-  { k_vec_mat<<<1, 256, 0, st>>>(prm->mu, prm->w1, ROW_DIM, N_HIDDEN, c->muw1); ++g_launches; }
+  if (has_mlp) { k_vec_mat<<<1, 256, 0, st>>>(prm->mu, prm->w1, ROW_DIM, N_HIDDEN, c->muw1); ++g_launches; }
   { k_permute_mu<<<(ROW_DIM + 255) / 256, 256, 0, st>>>(prm->mu, c->mu_perm); ++g_launches; }
   // split operands (hi/lo fp16, power-of-two scaled)
   dim3 tb(32, 8);
   { k_split<<<dim3(ROW_DIM / 32, N_COEF / 32), tb, 0, st>>>(prm->basis, N_COEF, ROW_DIM, 0, nullptr, std::ldexp(1.0, c->p_y), c->a_y); ++g_launches; }
-  { k_split<<<dim3(N_HIDDEN / 32, N_COEF / 32), tb, 0, st>>>(prm->w2, N_COEF, N_HIDDEN, 0, nullptr, std::ldexp(1.0, c->p_y), c->a_w2); ++g_launches; }
-  { k_split<<<dim3(ROW_DIM / 32, N_HIDDEN / 32), tb, 0, st>>>(prm->w1, N_HIDDEN, ROW_DIM, 0, nullptr, std::ldexp(1.0, c->p_h), c->a_h); ++g_launches; }
+  if (has_mlp) {
+    { k_split<<<dim3(N_HIDDEN / 32, N_COEF / 32), tb, 0, st>>>(prm->w2, N_COEF, N_HIDDEN, 0, nullptr, std::ldexp(1.0, c->p_y), c->a_w2); ++g_launches; }
+    { k_split<<<dim3(ROW_DIM / 32, N_HIDDEN / 32), tb, 0, st>>>(prm->w1, N_HIDDEN, ROW_DIM, 0, nullptr, std::ldexp(1.0, c->p_h), c->a_h); ++g_launches; }
+  }
   { k_split<<<dim3(N_COEF / 32, ROW_DIM / 32), tb, 0, st>>>(prm->basis, ROW_DIM, N_COEF, 1, prm->delta, std::ldexp(1.0, c->p_inv), c->a_inv); ++g_launches; }
   // fp32 copies for the exact refinement
   { k_transpose32<<<dim3(ROW_DIM / 32, N_COEF / 32), tb, 0, st>>>(prm->basis, ROW_DIM, N_COEF, c->bt32); ++g_launches; }
-  { k_transpose32<<<dim3(ROW_DIM / 32, N_HIDDEN / 32), tb, 0, st>>>(prm->w1, ROW_DIM, N_HIDDEN, c->w1t32); ++g_launches; }
-  { k_transpose32<<<dim3(N_HIDDEN / 32, N_COEF / 32), tb, 0, st>>>(prm->w2, N_HIDDEN, N_COEF, c->w2t32); ++g_launches; }
+  if (has_mlp) {
+    { k_transpose32<<<dim3(ROW_DIM / 32, N_HIDDEN / 32), tb, 0, st>>>(prm->w1, ROW_DIM, N_HIDDEN, c->w1t32); ++g_launches; }
+    { k_transpose32<<<dim3(N_HIDDEN / 32, N_COEF / 32), tb, 0, st>>>(prm->w2, N_HIDDEN, N_COEF, c->w2t32); ++g_launches; }
+  }
   cudaMemcpyAsync(c->mu32, prm->mu, 4ull * ROW_DIM, cudaMemcpyDeviceToDevice, st);
   // mean-model weights, K-major
-  { k_transpose16<<<dim3(2 * N_COEF / 32, N_COEF / 32), tb, 0, st>>>(prm->w_odd, N_COEF, N_COEF, N_COEF, 2 * N_COEF,
-                                                                   (uint16_t *)c->a_on); ++g_launches; }
-  { k_transpose16<<<dim3(N_COEF / 32, N_COEF / 32), tb, 0, st>>>(prm->w_even, N_COEF, 0, N_COEF, N_COEF, tmp_e); ++g_launches; }
-  { k_transpose16<<<dim3(N_COEF / 32, N_COEF / 32), tb, 0, st>>>(prm->w_odd, N_COEF, 0, N_COEF, N_COEF, tmp_oe); ++g_launches; }
+  if (has_means) {
+    { k_transpose16<<<dim3(2 * N_COEF / 32, N_COEF / 32), tb, 0, st>>>(prm->w_odd, N_COEF, N_COEF, N_COEF, 2 * N_COEF,
+                                                                     (uint16_t *)c->a_on); ++g_launches; }
+    { k_transpose16<<<dim3(N_COEF / 32, N_COEF / 32), tb, 0, st>>>(prm->w_even, N_COEF, 0, N_COEF, N_COEF, tmp_e); ++g_launches; }
+    { k_transpose16<<<dim3(N_COEF / 32, N_COEF / 32), tb, 0, st>>>(prm->w_odd, N_COEF, 0, N_COEF, N_COEF, tmp_oe); ++g_launches; }
+  }
   if (cudaGetLastError() != cudaSuccess) return cleanup(fail(DCKV_ECUDA, "setup kernels failed to launch"));
   // tensor maps of the static operands
   int r = DCKV_OK;
@@ -1025,7 +1041,7 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
       (r = map_a(&c->map_aon1, c->a_on, true, 2 * N_COEF, N_COEF, 1, 1)))
     return cleanup(r);
   // per-vocabulary mean tables: t_even = embed @ w_even, t_odd = embed @ w_odd[0:2048]
-  {
+  if (has_means) {
     CUtensorMap ma_e, ma_o, mb_emb;
     if ((r = map_a(&ma_e, tmp_e, true, N_COEF, N_COEF, 1, 1)) || (r = map_a(&ma_o, tmp_oe, true, N_COEF, N_COEF, 1, 1)) ||
         (r = map_b(&mb_emb, prm->embed, true, N_COEF, V, 256)))
@@ -1084,7 +1100,7 @@ static int upload_tables(const Layout &L, uint8_t *ws, const WsPlan &w, cudaStre
 extern "C" int dckv_encode(const dckv_codec *c, const void *rows, const int32_t *token_ids, const int64_t *seq_offsets,
                            int batch, void *blob, size_t blob_cap, uint64_t *blob_size_dev, int32_t *status_dev,
                            void *workspace, size_t ws_bytes, void *stream) {
-  if (!c || !rows || !token_ids || !blob || !blob_size_dev || !status_dev || !workspace)
+  if (!c || !rows || !blob || !blob_size_dev || !status_dev || !workspace || (c->has_means && !token_ids))
     return fail(DCKV_EINVAL, "a pointer argument is NULL");
   if (((uintptr_t)rows & 15) || ((uintptr_t)blob & 15) || ((uintptr_t)workspace & 255))
     return fail(DCKV_EINVAL, "rows/blob must be 16-byte and workspace 256-byte aligned");
@@ -1138,7 +1154,7 @@ extern "C" int dckv_encode(const dckv_codec *c, const void *rows, const int32_t 
     RET(map_b(&mb_gt, g16, false, 2 * N_HIDDEN, L.n_rows, TRANSFORM_BN / 2));
     RET(map_b(&mb_qe, qe, true, N_COEF, L.ne_pad, MEAN_ODD_BN / 2));
     // correction hidden layer: h = x @ w1 - mu @ w1, GELU, fp16 hi/lo
-    {
+    if (c->has_mlp) {
       GemmProblem pr = make_problem(N_HIDDEN / GEMM_BM, L.n_rows, HIDDEN_BN, false, status_dev);
       add_seg(pr, 0, 0, 2, 0, 0, 0, 0, ROW_DIM / GEMM_BK);
       EpiGelu::Params ep{c->muw1, (float)std::ldexp(1.0, -c->p_h), g16};
@@ -1149,8 +1165,10 @@ extern "C" int dckv_encode(const dckv_codec *c, const void *rows, const int32_t 
     {
       GemmProblem pr = make_problem(N_COEF / GEMM_BM, L.n_rows, TRANSFORM_BN, false, status_dev);
       add_seg(pr, 0, 0, 2, 0, 0, 0, 0, ROW_DIM / GEMM_BK);
-      add_seg(pr, 1, 0, 2, 0, 1, 0, 0, N_HIDDEN / GEMM_BK);
-      add_seg(pr, 1, 0, 2, 0, 1, 0, N_HIDDEN, N_HIDDEN / GEMM_BK);
+      if (c->has_mlp) {  // + g @ w2 (hi/lo on both sides)
+        add_seg(pr, 1, 0, 2, 0, 1, 0, 0, N_HIDDEN / GEMM_BK);
+        add_seg(pr, 1, 0, 2, 0, 1, 0, N_HIDDEN, N_HIDDEN / GEMM_BK);
+      }
       EpiQuantRegs::Params ep{{c->mub, c->delta, c->keep, (float)std::ldexp(1.0, -c->p_y), q32, qe, row_edst},
                               row_norm, rowflag, el_list, full_list, counters, w.el_cap, c->dbg_ratio};
       RET((run_gemm2_chunked<EpiQuantRegs, 4, 2, TRANSFORM_CHUNK_STEPS, TRANSFORM_BN>(c->map_ay2, c->map_aw2_2, mb_xt, mb_gt, pr, ep,
@@ -1159,16 +1177,18 @@ extern "C" int dckv_encode(const dckv_codec *c, const void *rows, const int32_t 
     stage_mark(c, st, "gemm_transform");
     // codes whose fp32 ratio lies in the guard band around a half step: exact fp64 values
     { k_refine_codes<<<c->num_sms * 4, 256, 0, st>>>(el_list, counters, w.el_cap, (const __nv_bfloat16 *)rows, row_tok,
-                                                  c->mu32, c->bt32, c->w2t32, g16, c->delta, rowflag, q32, qe,
-                                                  row_edst); ++g_launches; }
+                                                  c->mu32, c->bt32, c->has_mlp ? c->w2t32 : nullptr, g16, c->delta,
+                                                  rowflag, q32, qe, row_edst); ++g_launches; }
     const int rsmem = (ROW_DIM + N_HIDDEN) * 8;
     CK(cudaFuncSetAttribute(k_refine_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, rsmem));
     { k_refine_rows<<<c->num_sms, 256, rsmem, st>>>(full_list, counters, (const __nv_bfloat16 *)rows, row_tok, c->mu32,
-                                                  c->bt32, c->w1t32, c->w2t32, c->delta, c->keep, q32, qe, row_edst); ++g_launches; }
+                                                  c->bt32, c->has_mlp ? c->w1t32 : nullptr,
+                                                  c->has_mlp ? c->w2t32 : nullptr, c->delta, c->keep, q32, qe,
+                                                  row_edst); ++g_launches; }
     CK(cudaGetLastError());
     stage_mark(c, st, "refine");
     // odd mean model: [e, bf16(q_left), bf16(q_right)] @ w_odd -> centres
-    {
+    if (c->has_means) {
       GemmProblem pr = make_problem(N_COEF / GEMM_BM, L.ne_pad, MEAN_ODD_BN, true, status_dev);
       add_seg(pr, 0, 0, 1, 0, 0, 0, 0, N_COEF / GEMM_BK);
       add_seg(pr, 0, 0, 1, N_COEF, 0, 1, 0, N_COEF / GEMM_BK);
@@ -1178,8 +1198,13 @@ extern "C" int dckv_encode(const dckv_codec *c, const void *rows, const int32_t 
     stage_mark(c, st, "gemm_mean_odd");
     // even centres from the vocabulary table, then every symbol, in slot order
     const unsigned rg = (unsigned)std::min<int64_t>(L.n_rows, 65535);
-    { k_centres_even<<<rg, 256, 0, st>>>(L.n_rows, row_slot, row_edst, row_tok, token_ids, c->t_even, c->vocab,
-                                       c->kept_list, c->k_eff, cen8, nullptr); ++g_launches; }
+    if (c->has_means) {
+      k_centres_even<<<rg, 256, 0, st>>>(L.n_rows, row_slot, row_edst, row_tok, token_ids, c->t_even, c->vocab,
+                                         c->kept_list, c->k_eff, cen8, nullptr);
+      ++g_launches;
+    } else if (L.n_symbols > 0) {
+      CK(cudaMemsetAsync(cen8, 0, (size_t)L.n_symbols, st));  // unconditional tables: every centre 0
+    }
     { k_symbols<<<rg, SYM_THREADS, 0, st>>>(L.n_rows, row_slot, slot_chunk, q32, cen8, c->kept_list, c->kept_scale,
                                           c->cfm_tab, c->k_eff, sym16, cfm, nesc_w); ++g_launches; }
     CK(cudaGetLastError());
@@ -1213,7 +1238,7 @@ extern "C" int dckv_encode(const dckv_codec *c, const void *rows, const int32_t 
 extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_bytes, const int32_t *token_ids,
                            const int64_t *seq_offsets, int batch, void *k_out, void *v_out, int32_t *status_dev,
                            void *workspace, size_t ws_bytes, void *stream) {
-  if (!c || !blob || !token_ids || !k_out || !v_out || !status_dev || !workspace)
+  if (!c || !blob || !k_out || !v_out || !status_dev || !workspace || (c->has_means && !token_ids))
     return fail(DCKV_EINVAL, "a pointer argument is NULL");
   if (((uintptr_t)blob & 15) || ((uintptr_t)k_out & 15) || ((uintptr_t)v_out & 15) || ((uintptr_t)workspace & 255))
     return fail(DCKV_EINVAL, "blob/k_out/v_out must be 16-byte and workspace 256-byte aligned");
@@ -1263,9 +1288,13 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
   CK(cudaGetLastError());
   stage_mark(c, st, "layout+check");
   const uint32_t *offs = (const uint32_t *)(bl + HEADER_BYTES + 4ull * L.batch);
-  if (L.n_rows > 0)
-    { k_centres_even<<<(unsigned)std::min<int64_t>(L.n_rows, 65535), 256, 0, st>>>(
-        L.n_rows, row_slot, row_edst, row_tok, token_ids, c->t_even, c->vocab, c->kept_list, c->k_eff, cen8, valid); ++g_launches; }
+  if (L.n_rows > 0 && c->has_means) {
+    k_centres_even<<<(unsigned)std::min<int64_t>(L.n_rows, 65535), 256, 0, st>>>(
+        L.n_rows, row_slot, row_edst, row_tok, token_ids, c->t_even, c->vocab, c->kept_list, c->k_eff, cen8, valid);
+    ++g_launches;
+  } else if (L.n_symbols > 0) {
+    CK(cudaMemsetAsync(cen8, 0, (size_t)L.n_symbols, st));  // unconditional tables: every centre 0
+  }
   CK(cudaFuncSetAttribute(rans_decode_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, RANS_DEC_SMEM));
   CK(cudaFuncSetAttribute(rans_decode_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, RANS_DEC_SMEM));
   RansDecArgs da{d_chunks, 0, L.n_chunks, c->k_eff, c->kept_scale, c->dcdf, c->lut, c->tail, bl, L.off_streams,
@@ -1285,7 +1314,7 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
     { k_decode_codes<<<(unsigned)L.n_chunks_e, DEC_CODES_THREADS, 0, st>>>(fa); ++g_launches; }
   CK(cudaGetLastError());
   stage_mark(c, st, "codes_even");
-  if (L.n_rows > 0) {
+  if (L.n_rows > 0 && c->has_means) {
     CUtensorMap mb_qe;
     RET(map_b(&mb_qe, qe, true, N_COEF, L.ne_pad, MEAN_ODD_BN / 2));
     GemmProblem pr = make_problem(N_COEF / GEMM_BM, L.ne_pad, MEAN_ODD_BN, true, status_dev);

@@ -107,6 +107,8 @@ struct dckv_codec {
   int chunk_rows = 32;
   int vocab = 0;
   int k_eff = 0;
+  bool has_mlp = true;    // correction layer present (false: linear codec)
+  bool has_means = true;  // mean models present (false: unconditional zero-mean tables)
   // caller-owned parameter pointers (read at create)
   dckv_params p{};
   // derived, library-owned device buffers

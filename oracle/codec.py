@@ -34,7 +34,8 @@ __all__ = [
     "N_SYMBOLS", "PREC_TOTAL", "LANES", "B0_STEPS", "N_SCALES", "ROPE_BASE", "MAGIC",
     "VERSION", "HEADER_BYTES", "DEFAULT_CHUNK_ROWS",
     "bf16_to_f64", "f64_to_bf16", "gelu", "transform", "scale_index", "quantise",
-    "laplace_tables", "prompt_layout", "chunk_list", "mean_even", "mean_odd", "centres",
+    "laplace_tables", "prompt_layout", "chunk_list", "mean_even", "mean_odd", "codec_means_even",
+    "codec_means_odd", "centres",
     "symbols", "rans_encode", "rans_decode", "encode", "decode", "parse_blob", "analyse",
     "assemble_blob",
     "byte_report", "model_code_length_bits", "rope", "reconstruct", "kept_positions",
@@ -116,9 +117,13 @@ def transform(x, codec) -> np.ndarray:
     """y = (x - mu) B + GELU((x - mu) W1) W2  [xform].
 
     B is the shared 6,144 x 2,048 basis, W1 (6,144 x 256) and W2 (256 x 2,048) the
-    one-hidden-layer correction; no biases (reading).  fp64 throughout."""
+    one-hidden-layer correction; no biases (reading).  fp64 throughout.  A codec without
+    W1 / W2 is the linear codec the pages compare DCKV with ("Evidence": payload 5% above
+    its models' code length, 96 MiB of weights): y = (x - mu) B."""
     xc = _as_f64_rows(x) - np.asarray(codec.mu, np.float64)[None, :]
     lin = xc @ np.asarray(codec.basis, np.float64)
+    if codec.w1 is None or codec.w2 is None:
+        return lin
     hid = gelu(xc @ np.asarray(codec.w1, np.float64))
     return lin + hid @ np.asarray(codec.w2, np.float64)
 
@@ -178,6 +183,21 @@ def laplace_tables():
 def mean_even(embed_rows_bits, w_even_bits) -> np.ndarray:
     """Even-position code means: mu = e(token) W_e, in code units  [cond]."""
     return bf16_to_f64(embed_rows_bits) @ bf16_to_f64(w_even_bits)
+
+
+def codec_means_even(codec, toks) -> np.ndarray:
+    """Even-position means of a codec; a codec without mean models (the linear codec's
+    unconditional zero-mean tables, "Evidence") gives zeros."""
+    if codec.embed is None:
+        return np.zeros((len(toks), N_COEF))
+    return mean_even(codec.embed[toks], codec.w_even)
+
+
+def codec_means_odd(codec, toks, q_left, q_right) -> np.ndarray:
+    """Odd-position means of a codec (zeros without mean models, as above)."""
+    if codec.embed is None:
+        return np.zeros((len(toks), N_COEF))
+    return mean_odd(codec.embed[toks], q_left, q_right, codec.w_odd)
 
 
 def mean_odd(embed_rows_bits, q_left, q_right, w_odd_bits) -> np.ndarray:
@@ -404,9 +424,9 @@ def analyse(x, tok, seq_offsets, codec):
         qe, qo = q[0::2], q[1::2]
         te = tok[t0 + HEAD_KEPT: t0 + HEAD_KEPT + n: 2]
         to = tok[t0 + HEAD_KEPT + 1: t0 + HEAD_KEPT + n: 2]
-        mu_e = mean_even(codec.embed[te], codec.w_even) if qe.shape[0] else np.zeros((0, N_COEF))
+        mu_e = codec_means_even(codec, te) if qe.shape[0] else np.zeros((0, N_COEF))
         q_right = np.concatenate([qe[1:], np.zeros((1, N_COEF), np.int64)], 0)[: qo.shape[0]]
-        mu_o = (mean_odd(codec.embed[to], qe[: qo.shape[0]], q_right, codec.w_odd)
+        mu_o = (codec_means_odd(codec, to, qe[: qo.shape[0]], q_right)
                 if qo.shape[0] else np.zeros((0, N_COEF)))
         out.append(dict(q=q, ratio=ratio, qe=qe, qo=qo, mu_e=mu_e, mu_o=mu_o, ce=centres(mu_e), co=centres(mu_o)))
     return out
@@ -576,11 +596,11 @@ def decode(blob, tok, seq_offsets, codec, aux: dict | None = None):
             js = np.arange(j0, j0 + nr)
             toks = tok[t0 + 2 * js + par]
             if par == 0:
-                mu = mean_even(codec.embed[toks], codec.w_even)
+                mu = codec_means_even(codec, toks)
             else:
                 qe = qe_all[b]
                 right = np.concatenate([qe[1:], np.zeros((1, N_COEF), np.int64)], 0)
-                mu = mean_odd(codec.embed[toks], qe[js], right[js], codec.w_odd)
+                mu = codec_means_odd(codec, toks, qe[js], right[js])
             cen = centres(mu)[:, kept_c].reshape(-1)
             states, escv, words = _chunk_payload(blob, hdr, c)
             scl = np.tile(s_idx[kept_c], nr).astype(np.uint8)

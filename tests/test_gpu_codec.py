@@ -125,11 +125,11 @@ def check_centres(gc_codes, np_codec, tok, offs):
             if toks.size == 0:
                 continue
             if par == 0:
-                mu = O.mean_even(np_codec.embed[toks], np_codec.w_even)
+                mu = O.codec_means_even(np_codec, toks)
             else:
                 qe = G["qe"]
                 right = np.concatenate([qe[1:], np.zeros((1, 2048), np.int64)])[: toks.size]
-                mu = O.mean_odd(np_codec.embed[toks], qe[: toks.size], right, np_codec.w_odd)
+                mu = O.codec_means_odd(np_codec, toks, qe[: toks.size], right)
             keep = O.scale_index(np_codec.laplace_b, np_codec.delta)[1]
             ora_c = O.centres(mu)[:, keep]
             gpu_c = (G["ce"] if par == 0 else G["co"])[:, keep]
@@ -237,6 +237,31 @@ def test_parity_fewer_than_32_kept_components(src, step_scale, chunk_rows, k_ran
     k = int(O.scale_index(cod.laplace_b, cod.delta)[1].sum())
     assert k_range[0] <= k <= k_range[1]
     full_check(src, cod, [132 + 200, 140, 132 + 37], seeds=[41, 42, 43], chunk_rows=chunk_rows)
+
+
+_LINEAR = {}
+
+
+@pytest.mark.parametrize("variant", ["literal", "fitted"])
+def test_parity_linear_codec(src, variant):
+    # the linear codec: no correction, unconditional zero-mean tables (all centres 0)
+    if variant not in _LINEAR:
+        _LINEAR[variant] = (S.codec(src, step_scale=1.0, literal_b=True, linear=True) if variant == "literal"
+                            else S.codec(src, step_scale=None, target_bytes=220.0, linear=True))
+    cod = _LINEAR[variant]
+    r = full_check(src, cod, [132 + 300, 140, 132 + 77], seeds=[71, 72, 73])
+    assert not r["res"]["cen"].any()
+    # without mean models the token ids are not needed: NULL gives the same blob and rows
+    gc = r["gc"]
+    blob2 = gc.encode(r["x"], None, r["offs"])
+    torch.cuda.synchronize()
+    assert int(gc.status.item()) == D.DCKV_OK
+    size = int(gc.blob_size.item())
+    assert blob2[:size].cpu().numpy().tobytes() == r["res"]["blob"]
+    k2, v2 = gc.decode(blob2, size, None, r["offs"])
+    torch.cuda.synchronize()
+    assert int(gc.status.item()) == D.DCKV_OK
+    assert torch.equal(k2, r["k"]) and torch.equal(v2, r["v"])
 
 
 def test_determinism(src, codec_55):

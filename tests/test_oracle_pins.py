@@ -314,6 +314,40 @@ def test_lattice_rows_round_trip_exactly(src):
     assert np.array_equal(got_k[kp], kept[kp, :, 0]) and np.array_equal(got_v[kp], kept[kp, :, 1])
 
 
+def test_linear_codec_projection_zero_centres_and_lattice_round_trip(src):
+    """The linear codec ("Evidence": no correction, unconditional zero-mean tables): for
+    rows x = mu + z B^T the transform returns z; every centre is 0, so a kept code's
+    symbol is q + 254 (ESC beyond +-127); rows on the quantiser lattice encode to their
+    codes exactly and decode to bf16(RoPE(x)).  The decoder never reads token ids."""
+    cod = S.codec(src, step_scale=None, target_bytes=220.0, linear=True)
+    assert cod.w1 is None and cod.embed is None
+    rng = np.random.default_rng(12)
+    z = rng.standard_normal((5, O.N_COEF))
+    y = O.transform(cod.mu.astype(np.float64)[None, :] + z @ cod.basis.astype(np.float64).T, cod)
+    assert np.max(np.abs(y - z)) < 1e-6
+    s_idx, keep = O.scale_index(cod.laplace_b, cod.delta)
+    N = 132 + 9
+    q = rng.integers(-4, 5, (N, 2048))
+    q[:, :6] = rng.integers(-300, 300, (N, 6))
+    q[:, ~keep] = 0
+    x = O.reconstruct(q, cod)
+    aux = {}
+    tok = rng.integers(0, 32768, N)
+    blob = O.encode(x, tok, [0, N], cod, chunk_rows=4, aux=aux)
+    P = aux["per_prompt"][0]
+    assert np.array_equal(P["q"], q[4:4 + 9])
+    assert not P["ce"].any() and not P["co"].any()
+    sym, esc = O.symbols(P["qe"], P["ce"], keep)
+    want_sym = np.where(np.abs(P["qe"][:, keep]) > 127, 509, P["qe"][:, keep] + 254)
+    assert np.array_equal(sym, want_sym) and np.array_equal(esc, np.abs(P["qe"][:, keep]) > 127)
+    other = rng.integers(0, 32768, N)  # different token ids: the same decode
+    k, v = O.decode(blob, other, [0, N], cod)
+    want = O.f64_to_bf16(O.output_rows(x, np.arange(N))).reshape(N, 6, 2, 2, 256)
+    coded = np.arange(4, 13)
+    assert np.array_equal(np.transpose(k, (1, 0, 2, 3))[coded], want[coded, :, 0])
+    assert np.array_equal(np.transpose(v, (1, 0, 2, 3))[coded], want[coded, :, 1])
+
+
 def test_batch_round_trip_payload_and_escapes(src, codec_centred):
     lens = [132 + 37, 50, 132, 132 + 64]
     x, tok, offs = S.batch(src, lens, seeds=[11, 12, 13, 14], student_t_frac=0.2)
