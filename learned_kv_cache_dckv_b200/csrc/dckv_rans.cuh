@@ -390,6 +390,17 @@ __global__ void __launch_bounds__(COMPACT_THREADS) compact_kernel(CompactArgs a)
 __global__ void k_build_lut(const uint16_t *cdf, uint16_t *dcdf, uint16_t *lut, uint32_t *tail, uint2 *cfm_tab) {
   const int s = blockIdx.x;
   const uint16_t *tab = cdf + s * N_SYM;
+  __shared__ uint32_t runs[2];
+  if (threadIdx.x == 0) {
+    int lead = 0;  // symbols 0 .. lead-1 have frequency 1
+    while (lead < N_SYM && cdf_at(tab, lead + 1) - tab[lead] == 1u) ++lead;
+    int trail = N_SYM;  // symbols trail .. 509 have frequency 1
+    while (trail > lead && cdf_at(tab, trail) - tab[trail - 1] == 1u) --trail;
+    tail[s] = (uint32_t)lead | ((uint32_t)(N_SYM - trail) << 16);
+    runs[0] = (uint32_t)lead;                     // slots below this decode by arithmetic
+    runs[1] = PREC_TOTAL - (uint32_t)(N_SYM - trail);  // slots from this one on likewise
+  }
+  __syncthreads();
   auto holder = [&](uint32_t slot) {
     int lo = 0, hi = N_SYM;
     while (hi - lo > 1) {
@@ -399,10 +410,18 @@ __global__ void k_build_lut(const uint16_t *cdf, uint16_t *dcdf, uint16_t *lut, 
     return lo;
   };
   for (int b = threadIdx.x; b < LUT_SIZE; b += blockDim.x) {
-    const uint32_t slot = (uint32_t)b << (16 - LUT_BITS);
-    const int lo = holder(slot);
-    const int hi = holder(slot + (1u << (16 - LUT_BITS)) - 1u);
-    lut[s * LUT_STRIDE + b] = (uint16_t)(lo | (hi == lo ? LUT_SINGLE : 0) | (hi >= lo + 2 ? LUT_MULTI : 0));
+    // classify the bucket by its slots outside the frequency-1 runs (those are resolved
+    // by arithmetic); a bucket wholly inside a run is marked as one symbol
+    const uint32_t first = max((uint32_t)b << (16 - LUT_BITS), runs[0]);
+    const uint32_t last = min(((uint32_t)(b + 1) << (16 - LUT_BITS)) - 1u, runs[1] - 1u);
+    uint16_t e;
+    if (first > last) {
+      e = (uint16_t)(holder((uint32_t)b << (16 - LUT_BITS)) | LUT_SINGLE);
+    } else {
+      const int lo = holder(first), hi = holder(last);
+      e = (uint16_t)(lo | (hi == lo ? LUT_SINGLE : 0) | (hi >= lo + 2 ? LUT_MULTI : 0));
+    }
+    lut[s * LUT_STRIDE + b] = e;
   }
   if (threadIdx.x < LUT_STRIDE - LUT_SIZE) lut[s * LUT_STRIDE + LUT_SIZE + threadIdx.x] = 0;
   for (int k = threadIdx.x; k < DEC_CDF_STRIDE; k += blockDim.x) {
@@ -412,44 +431,13 @@ __global__ void k_build_lut(const uint16_t *cdf, uint16_t *dcdf, uint16_t *lut, 
       cfm_tab[s * N_SYM + k] = make_uint2((uint32_t)tab[k] | ((f - 1u) << 16), div_multiplier(f));
     }
   }
-  if (threadIdx.x == 0) {
-    int lead = 0;  // symbols 0 .. lead-1 have frequency 1
-    while (lead < N_SYM && cdf_at(tab, lead + 1) - tab[lead] == 1u) ++lead;
-    int trail = N_SYM;  // symbols trail .. 509 have frequency 1
-    while (trail > lead && cdf_at(tab, trail) - tab[trail - 1] == 1u) --trail;
-    tail[s] = (uint32_t)lead | ((uint32_t)(N_SYM - trail) << 16);
-  }
 }
 
-// Symbol holding `slot` under scale s, with its cumulative frequency c and frequency f.
-// Buckets with at most one boundary resolve without branches; the rest (frequency-1 runs
-// at the tails, several boundaries) take the second path.
-__device__ __forceinline__ int find_symbol(uint32_t slot, int s, const uint16_t *s_cdf, const uint16_t *s_lut,
-                                           const uint32_t *s_tail, uint32_t &c, uint32_t &f) {
-  const uint16_t *tab = s_cdf + s * DEC_CDF_STRIDE;
-  const uint32_t b = slot >> (16 - LUT_BITS);
-  const uint32_t e = s_lut[s * LUT_STRIDE + b];
-  int sym = (int)(e & LUT_SYM);
-  if (!(e & LUT_MULTI)) {
-    const uint32_t c0 = tab[sym], c1 = tab[sym + 1], c2 = tab[sym + 2];
-    const bool up = !(e & LUT_SINGLE) && slot >= c1;
-    sym += up;
-    c = up ? c1 : c0;
-    f = ((up ? c2 : c1) - c) & 0xFFFFu;
-    return sym;
-  }
-  const uint32_t tl = s_tail[s];
-  const uint32_t n_lead = tl & 0xFFFFu, n_trail = tl >> 16;
-  if (slot < n_lead) {
-    c = slot;
-    f = 1;
-    return (int)slot;
-  }
-  if (slot + n_trail >= PREC_TOTAL) {
-    c = slot;
-    f = 1;
-    return (int)(slot - (PREC_TOTAL - (uint32_t)N_SYM));
-  }
+// Several symbol ranges start inside the slot's bucket (outside the tail runs): binary
+// search between the bucket's first symbol and the next bucket's.
+__device__ __noinline__ int search_symbol(uint32_t slot, int s, uint32_t b, const uint16_t *tab,
+                                          const uint16_t *s_lut, uint32_t &c, uint32_t &f) {
+  int sym = (int)(s_lut[s * LUT_STRIDE + b] & LUT_SYM);
   int hi = b + 1 < (uint32_t)LUT_SIZE ? (int)(s_lut[s * LUT_STRIDE + b + 1] & LUT_SYM) : N_SYM - 1;  // in [sym, hi]
   while (hi > sym) {
     const int mid = (sym + hi + 1) >> 1;
@@ -457,6 +445,33 @@ __device__ __forceinline__ int find_symbol(uint32_t slot, int s, const uint16_t 
   }
   c = tab[sym];
   f = ((uint32_t)tab[sym + 1] - c) & 0xFFFFu;
+  return sym;
+}
+
+// Symbol holding `slot` under scale s, with its cumulative frequency c and frequency f.
+// The bucket entry settles any bucket with at most one boundary outside the tail runs by
+// one comparison; slots inside the frequency-1 runs at both tails decode by arithmetic
+// (selects, no branch); only a bucket with several boundaries outside the runs (central
+// symbols of frequency below 64) takes the search.
+__device__ __forceinline__ int find_symbol(uint32_t slot, int s, const uint16_t *s_cdf, const uint16_t *s_lut,
+                                           const uint32_t *s_tail, uint32_t &c, uint32_t &f) {
+  const uint16_t *tab = s_cdf + s * DEC_CDF_STRIDE;
+  const uint32_t b = slot >> (16 - LUT_BITS);
+  const uint32_t e = s_lut[s * LUT_STRIDE + b];
+  const uint32_t tl = s_tail[s];
+  int sym = (int)(e & LUT_SYM);
+  const uint32_t c0 = tab[sym], c1 = tab[sym + 1], c2 = tab[sym + 2];
+  const bool up = !(e & LUT_SINGLE) && slot >= c1;
+  sym += up;
+  c = up ? c1 : c0;
+  f = ((up ? c2 : c1) - c) & 0xFFFFu;
+  const bool lo_run = slot < (tl & 0xFFFFu);
+  const bool hi_run = slot + (tl >> 16) >= PREC_TOTAL;
+  const bool run = lo_run || hi_run;
+  sym = run ? (lo_run ? (int)slot : (int)(slot - (PREC_TOTAL - (uint32_t)N_SYM))) : sym;
+  c = run ? slot : c;
+  f = run ? 1u : f;
+  if ((e & LUT_MULTI) && !run) sym = search_symbol(slot, s, b, tab, s_lut, c, f);
   return sym;
 }
 
@@ -475,6 +490,35 @@ struct RansDecArgs {
   const int32_t *valid;  // header check result (1 = ok)
   int32_t *status;
 };
+
+// The decoder's tables (cdf rows, bucket lookup, tail runs, component scales) into shared
+// memory with bulk copies issued by one thread, in pieces of at most 32 KiB; every thread
+// waits (bounded) for their completion.  Returns false on timeout.
+__device__ __forceinline__ bool bulk_load_tables(uint8_t *sm, const uint16_t *dcdf, const uint16_t *lut,
+                                                 const uint32_t *tail, const uint8_t *scale, uint64_t *bar,
+                                                 volatile int *abort_flag) {
+  const uint8_t *src[4] = {reinterpret_cast<const uint8_t *>(dcdf), reinterpret_cast<const uint8_t *>(lut),
+                           reinterpret_cast<const uint8_t *>(tail), scale};
+  constexpr uint32_t len[4] = {CDF_SMEM_BYTES, LUT_SMEM_BYTES, TAIL_SMEM_BYTES, N_COEF};
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init(bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(bar, len[0] + len[1] + len[2] + len[3]);
+    uint32_t off = 0;
+    for (int t = 0; t < 4; ++t) {
+      for (uint32_t o = 0; o < len[t]; o += 32768u) {
+        const uint32_t n = min(32768u, len[t] - o);
+        bulk_load(sm + off + o, src[t] + o, n, bar);
+      }
+      off += len[t];
+    }
+  }
+  return mbar_wait(bar, 0, abort_flag);
+}
 
 __device__ __forceinline__ void load_tables(uint8_t *sm, const uint16_t *dcdf, const uint16_t *lut,
                                             const uint32_t *tail) {
@@ -540,10 +584,14 @@ __global__ void __launch_bounds__(RANS_WARPS * 32) rans_decode_kernel(RansDecArg
   const uint16_t *s_lut = reinterpret_cast<const uint16_t *>(sm + CDF_SMEM_BYTES);
   const uint32_t *s_tail = reinterpret_cast<const uint32_t *>(sm + CDF_SMEM_BYTES + LUT_SMEM_BYTES);
   uint8_t *s_scale = sm + CDF_SMEM_BYTES + LUT_SMEM_BYTES + TAIL_SMEM_BYTES;
+  __shared__ uint64_t tab_bar;
+  __shared__ int tab_abort;
   if (*a.valid != 1) return;
-  load_tables(sm, a.dcdf, a.lut, a.tail);
-  copy_smem16(s_scale, a.kept_scale, N_COEF);
-  __syncthreads();
+  static_assert(CDF_SMEM_BYTES % 16 == 0 && LUT_SMEM_BYTES % 16 == 0 && TAIL_SMEM_BYTES % 16 == 0, "bulk sizes");
+  if (!bulk_load_tables(sm, a.dcdf, a.lut, a.tail, a.kept_scale, &tab_bar, &tab_abort)) {
+    if (threadIdx.x == 0) atomicExch(a.status, DCKV_ETIMEOUT);
+    return;
+  }
   const int lane = threadIdx.x & 31;
   const int wi = blockIdx.x * RANS_WARPS + (threadIdx.x >> 5);
   if (wi >= a.n_chunks) return;
