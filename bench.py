@@ -437,6 +437,11 @@ def run_gpu(args):
     roofline_gemm = tensor_roofline(gemm_dom)
 
     model_bpt = model_bytes_per_row(D, gc, x, tok, offs, blob)
+    # codes the last encode recomputed exactly (guard band around a half step) and rows
+    # recomputed whole
+    v = D.dckv_ws_offsets(gc.handle, offs, 0)
+    cnt = gc._ws[v["counters"]: v["counters"] + 8].view(torch.int32).cpu().tolist()
+    refined = {"codes": int(cnt[0]), "rows": int(cnt[1]), "of_codes": int(n_rows * k_eff)}
 
     tokens = n_tok
     value = tokens * ws / (ms_step * 1e-3)
@@ -457,6 +462,7 @@ def run_gpu(args):
         "encode_ms": ms_enc, "decode_ms": ms_dec,
         "bytes_per_token": payload / max(n_rows, 1),
         "model_bytes_per_token": model_bpt,
+        "exact_recomputation": refined,
         "bytes_vs_model": payload / max(n_rows, 1) / model_bpt if model_bpt else None,
         "compression_vs_bf16": 12288.0 * n_rows / max(payload, 1),
         "stage_ms": {k: round(v, 5) for k, v in sorted(means.items())},

@@ -487,7 +487,7 @@ __global__ void k_check_header(HeaderCheck h) {
 
 // Kept rows: bf16 from the blob, RoPE on keys (same rotation as the inverse epilogue), bf16.
 __global__ void __launch_bounds__(256) k_kept(const uint8_t *blob, uint64_t off_kept, const PromptInfo *prompts,
-                                              int batch, const double *theta, __nv_bfloat16 *k_out,
+                                              int batch, const float2 *rope, __nv_bfloat16 *k_out,
                                               __nv_bfloat16 *v_out, int64_t n_tokens, const int32_t *valid) {
   if (*valid != 1) return;
   const int64_t kr = blockIdx.x;  // kept row index in the blob
@@ -508,9 +508,8 @@ __global__ void __launch_bounds__(256) k_kept(const uint8_t *blob, uint64_t off_
     float a = __bfloat162float(row[hv * HEAD_DIM + i]);
     float b = __bfloat162float(row[hv * HEAD_DIM + 128 + i]);
     if (kv == 0) {
-      float cs, sn;
-      rope_cs(pos, i, theta, cs, sn);
-      const float a2 = a * cs - b * sn, b2 = b * cs + a * sn;
+      const float2 cs = __ldg(rope + (int64_t)pos * 128 + i);
+      const float a2 = a * cs.x - b * cs.y, b2 = b * cs.x + a * cs.y;
       a = a2;
       b = b2;
     }
@@ -521,7 +520,7 @@ __global__ void __launch_bounds__(256) k_kept(const uint8_t *blob, uint64_t off_
 }
 
 // RoPE table of a decode call: rope[pos][i] = (cos, sin) of pos * theta_i, the same values
-// rope_cs gives the kept-row and fix-up kernels.
+// rope_cs gives the fix-up kernel.
 __global__ void __launch_bounds__(128) k_rope_table(float2 *rope, int64_t n_pos, const double *theta,
                                                    const int32_t *valid) {
   if (*valid != 1) return;
@@ -617,34 +616,63 @@ __device__ __forceinline__ void store_code(int64_t row, int c, double ratio, int
   if (e >= 0) qe[(int64_t)e * N_COEF + c] = __float2bfloat16_rn((float)q);
 }
 
-// Exact recomputation of listed codes near a half-step boundary, one warp per code:
+// Exact recomputation of listed codes near a half-step boundary, one block per code:
 // y = (x - mu) . basis[:, c] + g . w2[:, c] in fp64 (x from the caller's bf16 rows, g the
-// correction's hidden units from the chunk-accumulated GEMM), q = round(y / Delta_c).
-__global__ void __launch_bounds__(256) k_refine_codes(const uint32_t *el_list, const uint32_t *counters,
-                                                      int64_t el_cap, const __nv_bfloat16 *rows,
-                                                      const int32_t *row_tok, const float *mu32, const float *bt32,
-                                                      const float *w2t32, const __half *g16, const float *delta,
-                                                      const uint32_t *rowflag, int32_t *q32, __nv_bfloat16 *qe,
-                                                      const int32_t *row_edst) {
-  const int lane = threadIdx.x & 31;
+// correction's hidden units), q = round(y / Delta_c).  Each of the 256 threads sums 24
+// products in eight independent partial sums (all their loads in flight together), then
+// the block adds the partial sums in a fixed order.
+constexpr int REFINE_THREADS = 256;
+
+__global__ void __launch_bounds__(REFINE_THREADS) k_refine_codes(
+    const uint32_t *el_list, const uint32_t *counters, int64_t el_cap, const __nv_bfloat16 *rows,
+    const int32_t *row_tok, const float *mu32, const float *bt32, const float *w2t32, const __half *g16,
+    const float *delta, const uint32_t *rowflag, int32_t *q32, __nv_bfloat16 *qe, const int32_t *row_edst) {
+  constexpr int PER = ROW_DIM / REFINE_THREADS;  // 24
+  constexpr int U = 8;
+  static_assert(PER % U == 0, "partial sums");
+  __shared__ double red[REFINE_THREADS / 32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t n = min((int64_t)counters[0], el_cap);
-  const int64_t wpb = blockDim.x >> 5;
-  for (int64_t idx = blockIdx.x * wpb + (threadIdx.x >> 5); idx < n; idx += gridDim.x * wpb) {
+  for (int64_t idx = blockIdx.x; idx < n; idx += gridDim.x) {
     const uint32_t code = el_list[idx];
     const int64_t row = code >> 11;
     const int c = (int)(code & 2047u);
-    if (rowflag[row]) continue;  // recomputed whole by k_refine_rows
+    if (rowflag[row]) continue;  // recomputed whole by k_refine_rows (block-uniform)
     const __nv_bfloat16 *xr = rows + (int64_t)row_tok[row] * ROW_DIM;
     const float *bt = bt32 + (int64_t)c * ROW_DIM;
+    double part[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) part[u] = 0.0;
+#pragma unroll
+    for (int r = 0; r < PER / U; ++r) {
+      float xv[U], mv[U], bv[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int i = (r * U + u) * REFINE_THREADS + threadIdx.x;
+        xv[u] = __bfloat162float(xr[i]);
+        mv[u] = __ldg(mu32 + i);
+        bv[u] = __ldg(bt + i);
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) part[u] += ((double)xv[u] - (double)mv[u]) * (double)bv[u];
+    }
     double acc = 0.0;
-    for (int i = lane; i < ROW_DIM; i += 32) acc += ((double)__bfloat162float(xr[i]) - (double)mu32[i]) * (double)bt[i];
-    if (w2t32) {  // the correction (absent in a linear codec)
+#pragma unroll
+    for (int u = 0; u < U; ++u) acc += part[u];
+    if (w2t32) {  // the correction (absent in a linear codec): one hidden unit per thread
       const __half *g = g16 + row * (2 * N_HIDDEN);
-      for (int h = lane; h < N_HIDDEN; h += 32)
-        acc += ((double)__half2float(g[h]) + (double)__half2float(g[N_HIDDEN + h])) * (double)w2t32[c * N_HIDDEN + h];
+      const int h = threadIdx.x;
+      acc += ((double)__half2float(g[h]) + (double)__half2float(g[N_HIDDEN + h])) * (double)w2t32[c * N_HIDDEN + h];
     }
     acc = warp_sum(acc);
-    if (lane == 0) store_code(row, c, acc / (double)delta[c], q32, qe, row_edst);
+    if (lane == 0) red[warp] = acc;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      double y = 0.0;
+      for (int w = 0; w < REFINE_THREADS / 32; ++w) y += red[w];
+      store_code(row, c, y / (double)delta[c], q32, qe, row_edst);
+    }
+    __syncthreads();
   }
 }
 
@@ -1089,10 +1117,56 @@ extern "C" size_t dckv_blob_bound(const dckv_codec *c, const int64_t *offs, int 
   return L.off_streams + (uint64_t)L.n_chunks * (CHUNK_FIXED_BYTES + 4) + 10ull * L.n_symbols;
 }
 
-static int upload_tables(const Layout &L, uint8_t *ws, const WsPlan &w, cudaStream_t st) {
-  CK(cudaMemcpyAsync(ws + w.prompts, L.prompts.data(), sizeof(PromptInfo) * L.batch, cudaMemcpyHostToDevice, st));
-  if (L.n_chunks)
-    CK(cudaMemcpyAsync(ws + w.chunks, L.chunks.data(), sizeof(ChunkDesc) * L.n_chunks, cudaMemcpyHostToDevice, st));
+// The call's prompt table reaches the device as a kernel parameter (up to
+// PROMPT_PARAM_MAX prompts; beyond that one host-to-device copy), and the chunk table is
+// built from it on the device: no pageable copy on the launch path of ordinary batches.
+constexpr int PROMPT_PARAM_MAX = 400;  // 400 x 56 B of kernel parameters
+struct PromptPack {
+  PromptInfo p[PROMPT_PARAM_MAX];
+};
+
+__global__ void k_build_tables(const __grid_constant__ PromptPack pk, const PromptInfo *src, int batch,
+                               int n_chunks_e, int n_chunks, int G, int K, PromptInfo *prompts, ChunkDesc *chunks) {
+  const PromptInfo *P = src ? src : pk.p;
+  const int tid = blockIdx.x * blockDim.x + threadIdx.x, nth = gridDim.x * blockDim.x;
+  if (!src)
+    for (int b = tid; b < batch; b += nth) prompts[b] = pk.p[b];
+  for (int ci = tid; ci < n_chunks; ci += nth) {
+    const int par = ci >= n_chunks_e;
+    int lo = 0, hi = batch;  // last prompt whose first chunk of this parity is <= ci
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if ((par ? P[mid].chunk_o0 : P[mid].chunk_e0) <= ci) lo = mid; else hi = mid;
+    }
+    const PromptInfo pi = P[lo];
+    const int j0 = (ci - (par ? pi.chunk_o0 : pi.chunk_e0)) * G;
+    const int nr = par ? pi.n_o : pi.n_e;
+    ChunkDesc d;
+    d.prompt = lo;
+    d.parity = par;
+    d.j0 = j0;
+    d.nrows = min(G, nr - j0);
+    d.sym_base = (int64_t)((par ? pi.slot_o0 : pi.slot_e0) + j0) * K;
+    chunks[ci] = d;
+  }
+}
+
+static int upload_tables(const dckv_codec *c, const Layout &L, uint8_t *ws, const WsPlan &w, cudaStream_t st) {
+  static thread_local PromptPack pk;
+  PromptInfo *dp = (PromptInfo *)(ws + w.prompts);
+  const PromptInfo *src = nullptr;
+  if (L.batch <= PROMPT_PARAM_MAX) {
+    memcpy(pk.p, L.prompts.data(), sizeof(PromptInfo) * L.batch);
+  } else {
+    CK(cudaMemcpyAsync(dp, L.prompts.data(), sizeof(PromptInfo) * L.batch, cudaMemcpyHostToDevice, st));
+    src = dp;
+  }
+  const int work = std::max(L.batch, L.n_chunks);
+  const unsigned blocks = (unsigned)std::max(1, std::min((work + 255) / 256, 1024));
+  k_build_tables<<<blocks, 256, 0, st>>>(pk, src, L.batch, L.n_chunks_e, L.n_chunks, c->chunk_rows, c->k_eff, dp,
+                                         (ChunkDesc *)(ws + w.chunks));
+  ++g_launches;
+  CK(cudaGetLastError());
   return DCKV_OK;
 }
 
@@ -1139,7 +1213,7 @@ extern "C" int dckv_encode(const dckv_codec *c, const void *rows, const int32_t 
   CK(cudaMemsetAsync(counters, 0, 256, st));
   if (L.n_rows) CK(cudaMemsetAsync(rowflag, 0, 4ull * L.n_rows, st));
   if (L.n_chunks) CK(cudaMemsetAsync(nesc_w, 0, 4ull * L.n_chunks, st));
-  RET(upload_tables(L, ws, w, st));
+  RET(upload_tables(c, L, ws, w, st));
   { k_layout<<<dim3(L.batch, LAYOUT_SPLIT), 256, 0, st>>>(d_prompts, row_tok, row_pos, row_edst, row_slot, e_tok, e_slot, slot_chunk,
                                     c->chunk_rows, qe); ++g_launches; }
   if (L.n_tokens > 0)
@@ -1176,7 +1250,7 @@ extern "C" int dckv_encode(const dckv_codec *c, const void *rows, const int32_t 
     }
     stage_mark(c, st, "gemm_transform");
     // codes whose fp32 ratio lies in the guard band around a half step: exact fp64 values
-    { k_refine_codes<<<c->num_sms * 4, 256, 0, st>>>(el_list, counters, w.el_cap, (const __nv_bfloat16 *)rows, row_tok,
+    { k_refine_codes<<<c->num_sms * 8, REFINE_THREADS, 0, st>>>(el_list, counters, w.el_cap, (const __nv_bfloat16 *)rows, row_tok,
                                                   c->mu32, c->bt32, c->has_mlp ? c->w2t32 : nullptr, g16, c->delta,
                                                   rowflag, q32, qe, row_edst); ++g_launches; }
     const int rsmem = (ROW_DIM + N_HIDDEN) * 8;
@@ -1198,15 +1272,11 @@ extern "C" int dckv_encode(const dckv_codec *c, const void *rows, const int32_t 
     stage_mark(c, st, "gemm_mean_odd");
     // even centres from the vocabulary table, then every symbol, in slot order
     const unsigned rg = (unsigned)std::min<int64_t>(L.n_rows, 65535);
-    if (c->has_means) {
-      k_centres_even<<<rg, 256, 0, st>>>(L.n_rows, row_slot, row_edst, row_tok, token_ids, c->t_even, c->vocab,
-                                         c->kept_list, c->k_eff, cen8, nullptr);
-      ++g_launches;
-    } else if (L.n_symbols > 0) {
+    if (!c->has_means && L.n_symbols > 0)
       CK(cudaMemsetAsync(cen8, 0, (size_t)L.n_symbols, st));  // unconditional tables: every centre 0
-    }
     { k_symbols<<<rg, SYM_THREADS, 0, st>>>(L.n_rows, row_slot, slot_chunk, q32, cen8, c->kept_list, c->kept_scale,
-                                          c->cfm_tab, c->k_eff, sym16, cfm, nesc_w); ++g_launches; }
+                                          c->cfm_tab, c->k_eff, c->has_means ? c->t_even : nullptr, token_ids,
+                                          row_tok, row_edst, c->vocab, sym16, cfm, nesc_w); ++g_launches; }
     CK(cudaGetLastError());
     stage_mark(c, st, "symbols");
   }
@@ -1272,7 +1342,7 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
   stage_mark(c, st, "start");
   CK(cudaMemsetAsync(status_dev, 0, 4, st));
   CK(cudaMemsetAsync(counters, 0, 256, st));
-  RET(upload_tables(L, ws, w, st));
+  RET(upload_tables(c, L, ws, w, st));
   CK(cudaMemsetAsync(qe, 0, 2ull * L.ne_pad * N_COEF, st));
   if (L.n_rows) {
     CK(cudaMemsetAsync(q16, 0, 2ull * L.n_rows * N_COEF, st));
@@ -1283,7 +1353,7 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
   HeaderCheck hc{bl, blob_bytes, d_prompts, L.batch, c->chunk_rows, c->k_eff, L.n_chunks_e, L.n_chunks_o,
                  L.n_kept, L.off_kept, L.off_streams, valid, status_dev};
   { k_check_header<<<1, 256, 0, st>>>(hc); ++g_launches; }
-  if (L.n_rows > 0)
+  if (L.max_len > 0)
     { k_rope_table<<<(unsigned)std::min<int64_t>(L.max_len, 4096), 128, 0, st>>>(rope, L.max_len, c->theta, valid); ++g_launches; }
   CK(cudaGetLastError());
   stage_mark(c, st, "layout+check");
@@ -1342,7 +1412,7 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
   }
   stage_mark(c, st, "gemm_inverse");
   if (L.n_kept > 0)
-    { k_kept<<<(unsigned)L.n_kept, 256, 0, st>>>(bl, L.off_kept, d_prompts, L.batch, c->theta, (__nv_bfloat16 *)k_out,
+    { k_kept<<<(unsigned)L.n_kept, 256, 0, st>>>(bl, L.off_kept, d_prompts, L.batch, rope, (__nv_bfloat16 *)k_out,
                                               (__nv_bfloat16 *)v_out, L.n_tokens, valid); ++g_launches; }
   if (L.n_rows > 0)
     { k_fixup<<<c->num_sms, 256, 0, st>>>(biglist, counters, q16, qbig, c->a_inv, (float)std::ldexp(1.0, -c->p_inv),

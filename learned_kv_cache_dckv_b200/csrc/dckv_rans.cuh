@@ -47,7 +47,7 @@ __device__ __forceinline__ void copy_smem16(void *dst, const void *src, int byte
 __device__ __forceinline__ uint32_t cdf_at(const uint16_t *tab, int k) { return k < N_SYM ? tab[k] : PREC_TOTAL; }
 
 // ------------------------------------------------------------------------------ symbols
-// Centres of even rows, clamp(round(T_even[token][c]), +-127), in slot order.
+// Centres of even rows for the decoder, clamp(round(T_even[token][c]), +-127), in slot order.
 __global__ void __launch_bounds__(256) k_centres_even(int64_t n_rows, const int32_t *row_slot,
                                                       const int32_t *row_edst, const int32_t *row_tok,
                                                       const int32_t *tok_ids, const float *t_even, int vocab,
@@ -74,10 +74,19 @@ __global__ void __launch_bounds__(256) k_centres_even(int64_t n_rows, const int3
 constexpr int SYM_THREADS = 256;
 constexpr int SYM_UNROLL = 4;
 
+// Even rows take their centres straight from the vocabulary table t_even (and store them
+// in cen8 too, where the odd rows' centres already are); with t_even NULL (no mean models)
+// every centre is 0.
+__device__ __forceinline__ int even_centre(const float *t_row, int comp) {
+  return (int)fminf(fmaxf(rintf(__ldg(t_row + comp)), -(float)ESC_LIMIT), (float)ESC_LIMIT);
+}
+
 __global__ void __launch_bounds__(SYM_THREADS) k_symbols(int64_t n_rows, const int32_t *row_slot,
                                                          const int32_t *slot_chunk, const int32_t *q32,
-                                                         const int8_t *cen8, const int16_t *kept_list,
+                                                         int8_t *cen8, const int16_t *kept_list,
                                                          const uint8_t *kept_scale, const uint2 *cfm_tab, int k_eff,
+                                                         const float *t_even, const int32_t *tok_ids,
+                                                         const int32_t *row_tok, const int32_t *row_edst, int vocab,
                                                          uint16_t *sym16, uint2 *cfm, uint32_t *nesc) {
   __shared__ int esc_count;
   __shared__ int16_t s_kl[N_COEF];
@@ -92,6 +101,9 @@ __global__ void __launch_bounds__(SYM_THREADS) k_symbols(int64_t n_rows, const i
     const int slot = row_slot[row];
     const int64_t base = (int64_t)slot * k_eff;
     const int32_t *q = q32 + row * N_COEF;
+    const bool even = row_edst[row] >= 0;
+    const float *t_row = nullptr;
+    if (even && t_even) t_row = t_even + (int64_t)min(max(tok_ids[row_tok[row]], 0), vocab - 1) * N_COEF;
     int esc = 0;
     for (int k0 = threadIdx.x; k0 < k_eff; k0 += SYM_UNROLL * SYM_THREADS) {
       int v[SYM_UNROLL], ce[SYM_UNROLL];
@@ -99,7 +111,7 @@ __global__ void __launch_bounds__(SYM_THREADS) k_symbols(int64_t n_rows, const i
       for (int u = 0; u < SYM_UNROLL; ++u) {
         const int k = k0 + u * SYM_THREADS;
         v[u] = k < k_eff ? __ldg(q + s_kl[k]) : 0;
-        ce[u] = k < k_eff ? (int)__ldg(cen8 + base + k) : 0;
+        ce[u] = k >= k_eff ? 0 : even ? (t_row ? even_centre(t_row, s_kl[k]) : 0) : (int)__ldg(cen8 + base + k);
       }
 #pragma unroll
       for (int u = 0; u < SYM_UNROLL; ++u) {
@@ -108,6 +120,7 @@ __global__ void __launch_bounds__(SYM_THREADS) k_symbols(int64_t n_rows, const i
           const bool is_esc = v[u] > ESC_LIMIT || v[u] < -ESC_LIMIT;
           const int sym = is_esc ? ESC_SYM : v[u] - ce[u] + R_MAX;
           esc += is_esc;
+          if (even) cen8[base + k] = (int8_t)ce[u];
           sym16[base + k] = (uint16_t)sym;
           cfm[base + k] = __ldg(cfm_tab + s_ks[k] * N_SYM + sym);
         }
@@ -654,7 +667,7 @@ struct DecCodesArgs {
   int chunk0, n_chunks;
   int k_eff;
   const int16_t *kept_list;
-  const int8_t *cen8;
+  const int8_t *cen8;       // centres (slot order)
   const uint16_t *syms;     // slot order
   const uint8_t *blob;
   uint64_t off_streams;
