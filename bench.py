@@ -35,12 +35,14 @@ CONFIGS = {
     "c5": ([4096] * 64, 220.0, 0.01, "64 x 4096-token prompts, 1% Student-t (nu=2) rows, ~220 B/token"),
     "c2lin": ([4096], 220.0, 0.0, "1 x 4096-token prompt, linear codec (no correction, unconditional "
                                   "zero-mean tables), step scale for ~220 B/token"),
+    "c2syn": ([4096], 220.0, 0.0, "1 x 4096-token prompt, ~220 B/token, decoder-side synthesis MLP "
+                                  "(2048 -> 256 GELU -> 6144) added to the linear inverse"),
 }
 
 # rows per rANS chunk (codec creation); 0 = the library default (16)
 CHUNK_ROWS = {"c3b": 32}
 
-GEMM_STAGES = {"gemm_hidden", "gemm_transform", "gemm_mean_odd", "gemm_inverse"}
+GEMM_STAGES = {"gemm_hidden", "gemm_transform", "gemm_mean_odd", "gemm_inverse", "gemm_synth_hidden"}
 
 
 def load_peaks():
@@ -128,10 +130,11 @@ def make_inputs(cfg_name, rank, device):
     lens, target, st, _ = CONFIGS[cfg_name]
     src = S.source(0)
     linear = cfg_name.endswith("lin")
+    synthesis = cfg_name.endswith("syn")
     if target is None:
         cod = S.codec(src, step_scale=1.0, literal_b=True, linear=linear)
     else:
-        cod = S.codec(src, step_scale=None, target_bytes=target, linear=linear)
+        cod = S.codec(src, step_scale=None, target_bytes=target, linear=linear, synthesis=synthesis)
     seeds = [1000 * rank + i for i in range(len(lens))]
     x, tok, offs = S.batch(src, lens, seeds, student_t_frac=st, device=device)
     return src, cod, x, tok, offs
@@ -400,9 +403,14 @@ def run_gpu(args):
         "dec:gemm_mean_odd": 2.0 * pad(n_even + len(offs) - 1, 224) * 4096 * 2048,
         "dec:gemm_inverse": 2.0 * 2 * pad(n_rows, 224) * 2048 * 6144,
     }
+    if args.config.endswith("syn"):  # decoder-side synthesis: hidden GEMM, and g V2 in the inverse
+        algo_flops["dec:gemm_synth_hidden"] = 2.0 * n_rows * 2048 * 256
+        issued_flops["dec:gemm_synth_hidden"] = 2.0 * 2 * pad(n_rows, 64) * 2048 * 256
+        algo_flops["dec:gemm_inverse"] += 2.0 * n_rows * 256 * 6144
+        issued_flops["dec:gemm_inverse"] += 2.0 * 4 * pad(n_rows, 224) * 256 * 6144
     # DRAM bytes (read + write) per launch from the committed ncu captures of this workload
     # (profiles/*_c2.md); null for other workloads
-    traffic = {"enc:gemm_transform": 191.2e6, "dec:gemm_inverse": 158.6e6, "enc:gemm_mean_odd": 41.1e6,
+    traffic = {"enc:gemm_transform": 191.4e6, "dec:gemm_inverse": 158.6e6, "enc:gemm_mean_odd": 41.1e6,
                "dec:gemm_mean_odd": 41.1e6} if args.config == "c2" else {}
     bf16_peak = float(peaks.get("bf16_tflops", 1590.0))
     sm_mhz = float(peaks.get("sm_max_mhz", 1965.0))

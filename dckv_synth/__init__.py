@@ -138,6 +138,8 @@ class Codec:
     w_odd: np.ndarray | None  # u16 bf16 bits [6144, 2048]    mu_odd = [e, bf16(qL), bf16(qR)] @ w_odd
     step_scale: float
     note: str = ""
+    v1: np.ndarray | None = None  # fp32 [2048, 256]  decoder-side synthesis, first layer
+    v2: np.ndarray | None = None  # fp32 [256, 6144]  decoder-side synthesis, second layer
 
 
 def coefficient_variance(src: Source) -> np.ndarray:
@@ -201,6 +203,8 @@ def codec(
     zero_mlp: bool = False,
     seed: int | None = None,
     linear: bool = False,
+    synthesis: bool = False,
+    synthesis_gain: float = 1.0,
 ) -> Codec:
     """Draw a synthetic codec.
 
@@ -211,6 +215,8 @@ def codec(
     centres); zero_mlp sets the correction to zero (its initial state on the pages).
     linear: the linear codec the pages compare against -- no correction (w1 = w2 = None)
     and unconditional zero-mean tables (embed = w_even = w_odd = None).
+    synthesis: add decoder-side synthesis weights V1 [2048, 256], V2 [256, 6144], both
+    std 0.01 * synthesis_gain (0.01 like the encoder's correction).
     """
     seed = src.seed if seed is None else seed
     rng = np.random.default_rng([seed, 0x53])
@@ -251,13 +257,19 @@ def codec(
     w_odd_n = 0.02 * neigh_gain * rng.standard_normal((2 * N_COEF, N_COEF))
     w_odd_n *= np.concatenate([delta, delta]).astype(np.float64)[:, None]
     w_odd = f32_to_bf16_bits(np.concatenate([w_odd_e, w_odd_n], axis=0))
+    v1 = v2 = None
+    if synthesis:
+        srng = np.random.default_rng([seed, 0x5E])
+        v1 = (0.01 * synthesis_gain * srng.standard_normal((N_COEF, N_HIDDEN))).astype(np.float32)
+        v2 = (0.01 * synthesis_gain * srng.standard_normal((N_HIDDEN, ROW_DIM))).astype(np.float32)
     if linear:
         w1 = w2 = embed = w_even = w_odd = None
     return Codec(
         mu=src.mu.copy(), basis=basis, w1=w1, w2=w2, delta=delta, laplace_b=b,
         embed=embed, w_even=w_even, w_odd=w_odd, step_scale=float(step_scale),
         note=("literal b=0.6*Delta" if literal_b else "fitted b") + (", zero MLP" if zero_mlp else "")
-        + (", linear codec" if linear else ""),
+        + (", linear codec" if linear else "") + (", synthesis MLP" if synthesis else ""),
+        v1=v1, v2=v2,
     )
 
 

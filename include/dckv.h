@@ -83,6 +83,11 @@ typedef struct {
   const uint16_t *w_odd;    /* bf16 [6144][2048] odd mean model: mu = [e, bf16(q_left),
                                bf16(q_right)] @ w_odd; the neighbour blocks carry Delta_c */
   int32_t vocab;            /* rows of embed (1 .. 2^20; ignored without mean models)    */
+  const float *v1;          /* [2048][256]   decoder-side synthesis, first layer, or NULL   */
+  const float *v2;          /* [256][6144]   decoder-side synthesis, second layer, or NULL:
+                               decode adds GELU((q * Delta) @ v1) @ v2 to mu + (q * Delta) B^T
+                               before RoPE (no counterpart on the pages beyond the weight
+                               count they report; zero-initialise to leave it out)        */
 } dckv_params;
 
 /* Per-blob byte accounting (host-side parse of a blob header and tables). */

@@ -38,7 +38,7 @@ class DckvError(RuntimeError):
 class _Params(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("mu", "basis", "w1", "w2", "delta", "laplace_b", "embed", "w_even", "w_odd")] + [
-                   ("vocab", ctypes.c_int32)]
+                   ("vocab", ctypes.c_int32), ("v1", ctypes.c_void_p), ("v2", ctypes.c_void_p)]
 
 
 class ByteReport(ctypes.Structure):
@@ -137,10 +137,11 @@ def _stream_ptr(stream):
 # ---------------------------------------------------------------------------------- C ABI
 def dckv_codec_create(params: dict, device: int = 0, chunk_rows: int = 0):
     """params: device tensors mu, basis, w1, w2, delta, laplace_b (fp32), embed, w_even,
-    w_odd (bf16 or int16 holding bf16 bits); w1 / w2 None for a linear codec, embed /
-    w_even / w_odd None for unconditional tables.  Returns an opaque handle."""
+    w_odd (bf16 or int16 holding bf16 bits), v1, v2 (fp32, optional); w1 / w2 None for a
+    linear codec, embed / w_even / w_odd None for unconditional tables, v1 / v2 None for a
+    linear synthesis.  Returns an opaque handle."""
     p = _Params()
-    for k in ("mu", "basis", "w1", "w2", "delta", "laplace_b", "embed", "w_even", "w_odd"):
+    for k in ("mu", "basis", "w1", "w2", "delta", "laplace_b", "embed", "w_even", "w_odd", "v1", "v2"):
         v = params.get(k)
         setattr(p, k, None if v is None else v.data_ptr())
     p.vocab = 0 if params.get("embed") is None else int(params["embed"].shape[0])
@@ -259,12 +260,13 @@ def dckv_debug_gemm(bf16: bool, A, slabs: int, B, M: int, N: int, K: int, D, bn:
 # ---------------------------------------------------------------------------------- helpers
 def upload_params(codec, device="cuda"):
     """Device tensors for dckv_codec_create from an object with numpy attributes mu, basis,
-    w1, w2, delta, laplace_b (float32) and embed, w_even, w_odd (bf16 bits as uint16)."""
+    w1, w2, delta, laplace_b (float32), embed, w_even, w_odd (bf16 bits as uint16) and,
+    optionally, v1, v2 (float32)."""
     import torch
 
     out = {}
-    for k in ("mu", "basis", "w1", "w2", "delta", "laplace_b"):
-        v = getattr(codec, k)
+    for k in ("mu", "basis", "w1", "w2", "delta", "laplace_b", "v1", "v2"):
+        v = getattr(codec, k, None)
         out[k] = None if v is None else torch.from_numpy(np.ascontiguousarray(v, np.float32)).to(device)
     for k in ("embed", "w_even", "w_odd"):
         v = getattr(codec, k)

@@ -297,7 +297,18 @@ __global__ void k_split(const float *src, int M, int K, int mode, const float *d
     for (int y = ty; y < 32; y += 8) {
       const int m = m0 + y, k = k0 + tx;
       if (m < M && k < K) {
-        const double v = (double)tile[tx][y] * scale;
+        const double v = (double)tile[tx][y] * (delta ? (double)delta[k] : 1.0) * scale;
+        const __half hi = __double2half(v);
+        const __half lo = __double2half(v - (double)__half2float(hi));
+        out[(int64_t)m * K + k] = hi;
+        out[(int64_t)M * K + (int64_t)m * K + k] = lo;
+      }
+    }
+  } else if (mode == 2) {  // src [K][dims]: out[p][k] = src[k][dim(p)] (inverse GEMM row order)
+    for (int y = ty; y < 32; y += 8) {
+      const int m = m0 + y, k = k0 + tx;
+      if (m < M && k < K) {
+        const double v = (double)src[(int64_t)k * M + inv_row_to_dim(m)] * scale;
         const __half hi = __double2half(v);
         const __half lo = __double2half(v - (double)__half2float(hi));
         out[(int64_t)m * K + k] = hi;
@@ -544,9 +555,11 @@ __global__ void __launch_bounds__(256) k_fixup(const int32_t *biglist, const uin
                                                const int32_t *qbig, const __half *a_inv, float inv_scale,
                                                const float *mu_perm, const double *theta, const int32_t *row_tok,
                                                const int32_t *row_pos, __nv_bfloat16 *k_out, __nv_bfloat16 *v_out,
-                                               int64_t n_tokens) {
+                                               int64_t n_tokens, const float *v1t32, const float *v2_32,
+                                               const float *delta) {
   __shared__ float qs[N_COEF];
   __shared__ float xs[ROW_DIM];
+  __shared__ float gs[N_HIDDEN];
   const uint32_t n = *bigcount;
   for (uint32_t li = blockIdx.x; li < n; li += gridDim.x) {
     const int64_t r = biglist[li];
@@ -563,6 +576,20 @@ __global__ void __launch_bounds__(256) k_fixup(const int32_t *biglist, const uin
       for (int c = 0; c < N_COEF; ++c)
         acc = fmaf(qs[c], __half2float(a_inv[p * N_COEF + c]) + __half2float(lo[p * N_COEF + c]), acc);
       xs[d] = acc * inv_scale + mu_perm[p];
+    }
+    if (v1t32) {  // decoder-side synthesis: + GELU((q Delta) V1) V2, fp32
+      for (int h = threadIdx.x; h < N_HIDDEN; h += blockDim.x) {
+        const float *w = v1t32 + (int64_t)h * N_COEF;
+        float acc = 0.f;
+        for (int c = 0; c < N_COEF; ++c) acc = fmaf(qs[c] * delta[c], w[c], acc);
+        gs[h] = 0.5f * acc * (1.0f + erff(acc * 0.70710678118654752f));
+      }
+      __syncthreads();
+      for (int d = threadIdx.x; d < ROW_DIM; d += blockDim.x) {
+        float acc = 0.f;
+        for (int h = 0; h < N_HIDDEN; ++h) acc = fmaf(gs[h], v2_32[(int64_t)h * ROW_DIM + d], acc);
+        xs[d] += acc;
+      }
     }
     __syncthreads();
     const int pos = row_pos[r];
@@ -828,6 +855,7 @@ static WsPlan plan_ws(const Layout &L, int which /*0 encode, 1 decode*/) {
     w.full_list = take(4ull * L.n_rows);
   } else {
     w.slots16 = take(2ull * L.n_symbols);
+    w.g16 = take(2ull * L.n_rows * 2 * N_HIDDEN);  // synthesis hidden units (hi/lo)
     w.rope = take(8ull * 128 * std::max<int64_t>(L.max_len, 1));
     w.q16 = take(2ull * L.n_rows * N_COEF);
     w.qbig = take(4ull * L.n_rows * N_COEF);
@@ -854,7 +882,8 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
   if (!prm->w1 != !prm->w2) return fail(DCKV_EINVAL, "w1 and w2 must both be given or both be NULL");
   if (!prm->embed != !prm->w_even || !prm->embed != !prm->w_odd)
     return fail(DCKV_EINVAL, "embed, w_even and w_odd must all be given or all be NULL");
-  const bool has_mlp = prm->w1 != nullptr, has_means = prm->embed != nullptr;
+  if (!prm->v1 != !prm->v2) return fail(DCKV_EINVAL, "v1 and v2 must both be given or both be NULL");
+  const bool has_mlp = prm->w1 != nullptr, has_means = prm->embed != nullptr, has_synth = prm->v1 != nullptr;
   if (has_means && (prm->vocab < 1 || prm->vocab > (1 << 20))) return fail(DCKV_EINVAL, "vocab out of range");
   if (chunk_rows < -1 || chunk_rows > 256) return fail(DCKV_EINVAL, "chunk_rows out of range");
   if (((uintptr_t)prm->embed | (uintptr_t)prm->w_even | (uintptr_t)prm->w_odd) & 15)
@@ -873,6 +902,7 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
   c->vocab = has_means ? prm->vocab : 0;
   c->has_mlp = has_mlp;
   c->has_means = has_means;
+  c->has_synth = has_synth;
   c->p = *prm;
   for (int i = 0; i < 24; ++i) cudaEventCreate(&c->ev[i]);
 
@@ -915,6 +945,11 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
   const uint64_t o_w1t32 = take(4ull * N_HIDDEN * ROW_DIM);
   const uint64_t o_w2t32 = take(4ull * N_COEF * N_HIDDEN);
   const uint64_t o_mu32 = take(4ull * ROW_DIM);
+  const uint64_t o_av1 = take(has_synth ? 2ull * 2 * N_HIDDEN * N_COEF : 0);
+  const uint64_t o_av2 = take(has_synth ? 2ull * 2 * ROW_DIM * N_HIDDEN : 0);
+  const uint64_t o_v1t32 = take(has_synth ? 4ull * N_HIDDEN * N_COEF : 0);
+  const uint64_t o_v2_32 = take(has_synth ? 4ull * N_HIDDEN * ROW_DIM : 0);
+  const uint64_t o_zero = take(4ull * N_HIDDEN);
   const uint64_t o_tmp = take(2ull * 2 * N_COEF * N_COEF);  // W_e^T and W_oE^T (setup only)
   const uint64_t o_scr = take(64);
   if (cudaMalloc(&c->blk, o) != cudaSuccess) return cleanup(fail(DCKV_ECUDA, "cudaMalloc(%llu) failed", (unsigned long long)o));
@@ -945,12 +980,18 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
   c->w1t32 = (float *)(B + o_w1t32);
   c->w2t32 = (float *)(B + o_w2t32);
   c->mu32 = (float *)(B + o_mu32);
+  c->a_v1 = (__half *)(B + o_av1);
+  c->a_v2 = (__half *)(B + o_av2);
+  c->v1t32 = (float *)(B + o_v1t32);
+  c->v2_32 = (float *)(B + o_v2_32);
+  c->zero256 = (float *)(B + o_zero);
   uint16_t *tmp_e = (uint16_t *)(B + o_tmp);
   uint16_t *tmp_oe = tmp_e + (size_t)N_COEF * N_COEF;
   int32_t *scr = (int32_t *)(B + o_scr);
   cudaStream_t st = 0;
 
-  if (cudaMemset(scr, 0, 64) != cudaSuccess) return cleanup(fail(DCKV_ECUDA, "memset"));
+  if (cudaMemset(scr, 0, 64) != cudaSuccess || cudaMemset(c->zero256, 0, 4ull * N_HIDDEN) != cudaSuccess)
+    return cleanup(fail(DCKV_ECUDA, "memset"));
   // drop mask, scale index, tables
   { k_scale_keep<<<(N_COEF + 255) / 256, 256, 0, st>>>(prm->laplace_b, prm->delta, c->scale, c->keep, scr); ++g_launches; }
   { k_tables<<<N_SCALES, 512, 0, st>>>(c->cdf); ++g_launches; }
@@ -963,9 +1004,14 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
     { k_absmax<<<256, 256, 0, st>>>(prm->w1, (int64_t)ROW_DIM * N_HIDDEN, N_HIDDEN, nullptr, scr + 3); ++g_launches; }
   }
   { k_absmax<<<256, 256, 0, st>>>(prm->basis, (int64_t)ROW_DIM * N_COEF, N_COEF, prm->delta, scr + 4); ++g_launches; }
-  int32_t host_scr[8];
+  if (has_synth) {  // synthesis operands: |V1| and |Delta| bound Delta * V1; |V2| joins the inverse's scale
+    { k_absmax<<<128, 256, 0, st>>>(prm->v1, (int64_t)N_COEF * N_HIDDEN, N_HIDDEN, nullptr, scr + 6); ++g_launches; }
+    { k_absmax<<<8, 256, 0, st>>>(prm->delta, (int64_t)N_COEF, N_COEF, nullptr, scr + 7); ++g_launches; }
+    { k_absmax<<<256, 256, 0, st>>>(prm->v2, (int64_t)N_HIDDEN * ROW_DIM, ROW_DIM, nullptr, scr + 8); ++g_launches; }
+  }
+  int32_t host_scr[16];
   uint8_t keep_h[N_COEF], scale_h[N_COEF];
-  if (cudaMemcpy(host_scr, scr, 32, cudaMemcpyDeviceToHost) != cudaSuccess ||
+  if (cudaMemcpy(host_scr, scr, 64, cudaMemcpyDeviceToHost) != cudaSuccess ||
       cudaMemcpy(keep_h, c->keep, N_COEF, cudaMemcpyDeviceToHost) != cudaSuccess ||
       cudaMemcpy(scale_h, c->scale, N_COEF, cudaMemcpyDeviceToHost) != cudaSuccess)
     return cleanup(fail(DCKV_ECUDA, "setup readback failed: %s", cudaGetErrorString(cudaGetLastError())));
@@ -985,7 +1031,21 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
   memcpy(&mboth, &mmax, 4);
   c->p_y = exp_for(mboth);
   c->p_h = exp_for(host_scr[3]);
-  c->p_inv = exp_for(host_scr[4]);
+  {
+    float mi, mv2;
+    memcpy(&mi, &host_scr[4], 4);
+    memcpy(&mv2, &host_scr[8], 4);
+    const float m = std::max(mi, has_synth ? mv2 : 0.f);  // the inverse GEMM's A: Delta B and V2
+    int32_t bits;
+    memcpy(&bits, &m, 4);
+    c->p_inv = exp_for(bits);
+    float mv1, md;
+    memcpy(&mv1, &host_scr[6], 4);
+    memcpy(&md, &host_scr[7], 4);
+    const float mvd = mv1 * md;
+    memcpy(&bits, &mvd, 4);
+    c->p_v1 = has_synth ? exp_for(bits) : 0;
+  }
   // kept components
   std::vector<int16_t> kl;
   std::vector<uint8_t> ks;
@@ -1051,6 +1111,13 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
     { k_transpose32<<<dim3(N_HIDDEN / 32, N_COEF / 32), tb, 0, st>>>(prm->w2, N_HIDDEN, N_COEF, c->w2t32); ++g_launches; }
   }
   cudaMemcpyAsync(c->mu32, prm->mu, 4ull * ROW_DIM, cudaMemcpyDeviceToDevice, st);
+  if (has_synth) {
+    // a_v1[slab][h][c] = split(Delta_c V1[c][h] 2^p_v1); a_v2[slab][p][h] = split(V2[h][dim(p)] 2^p_inv)
+    { k_split<<<dim3(N_COEF / 32, N_HIDDEN / 32), tb, 0, st>>>(prm->v1, N_HIDDEN, N_COEF, 0, prm->delta, std::ldexp(1.0, c->p_v1), c->a_v1); ++g_launches; }
+    { k_split<<<dim3(N_HIDDEN / 32, ROW_DIM / 32), tb, 0, st>>>(prm->v2, ROW_DIM, N_HIDDEN, 2, nullptr, std::ldexp(1.0, c->p_inv), c->a_v2); ++g_launches; }
+    { k_transpose32<<<dim3(N_COEF / 32, N_HIDDEN / 32), tb, 0, st>>>(prm->v1, N_COEF, N_HIDDEN, c->v1t32); ++g_launches; }
+    cudaMemcpyAsync(c->v2_32, prm->v2, 4ull * N_HIDDEN * ROW_DIM, cudaMemcpyDeviceToDevice, st);
+  }
   // mean-model weights, K-major
   if (has_means) {
     { k_transpose16<<<dim3(2 * N_COEF / 32, N_COEF / 32), tb, 0, st>>>(prm->w_odd, N_COEF, N_COEF, N_COEF, 2 * N_COEF,
@@ -1066,7 +1133,9 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
       (r = map_a(&c->map_aw2_1, c->a_w2, false, N_HIDDEN, N_COEF, 2, 1)) ||
       (r = map_a(&c->map_ah2, c->a_h, false, ROW_DIM, N_HIDDEN, 2, 2)) ||
       (r = map_a(&c->map_ainv2, c->a_inv, false, N_COEF, ROW_DIM, 2, 2)) ||
-      (r = map_a(&c->map_aon1, c->a_on, true, 2 * N_COEF, N_COEF, 1, 1)))
+      (r = map_a(&c->map_aon1, c->a_on, true, 2 * N_COEF, N_COEF, 1, 1)) ||
+      (has_synth && (r = map_a(&c->map_av1, c->a_v1, false, N_COEF, N_HIDDEN, 2, 2))) ||
+      (has_synth && (r = map_a(&c->map_av2, c->a_v2, false, N_HIDDEN, ROW_DIM, 2, 2))))
     return cleanup(r);
   // per-vocabulary mean tables: t_even = embed @ w_even, t_odd = embed @ w_odd[0:2048]
   if (has_means) {
@@ -1401,14 +1470,32 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
     CK(cudaGetLastError());
   }
   stage_mark(c, st, "codes_odd");
+  __half *g16d = (__half *)(ws + w.g16);
+  if (L.n_rows > 0 && c->has_synth) {  // decoder-side synthesis, hidden layer: GELU((q Delta) V1)
+    CUtensorMap mb_qh;
+    RET(map_b(&mb_qh, q16, false, N_COEF, L.n_rows, HIDDEN_BN / 2));
+    GemmProblem pr = make_problem(N_HIDDEN / GEMM_BM, L.n_rows, HIDDEN_BN, false, status_dev);
+    add_seg(pr, 0, 0, 2, 0, 0, 0, 0, N_COEF / GEMM_BK);
+    EpiGelu::Params ep{c->zero256, (float)std::ldexp(1.0, -c->p_v1), g16d};
+    RET((run_gemm2<EpiGelu, 4, 2, 4>(c->map_av1, c->map_av1, mb_qh, mb_qh, pr, ep, c->num_sms, false, st)));
+    stage_mark(c, st, "gemm_synth_hidden");
+  }
   if (L.n_rows > 0) {
-    CUtensorMap mb_q;
+    CUtensorMap mb_q, mb_g;
     RET(map_b(&mb_q, q16, false, N_COEF, L.n_rows, INVERSE_BN / 2));
     GemmProblem pr = make_problem(ROW_DIM / GEMM_BM, L.n_rows, INVERSE_BN, false, status_dev);
     add_seg(pr, 0, 0, 2, 0, 0, 0, 0, N_COEF / GEMM_BK);
+    if (c->has_synth) {  // + g V2 (hi/lo on both sides)
+      RET(map_b(&mb_g, g16d, false, 2 * N_HIDDEN, L.n_rows, INVERSE_BN / 2));
+      add_seg(pr, 1, 0, 2, 0, 1, 0, 0, N_HIDDEN / GEMM_BK);
+      add_seg(pr, 1, 0, 2, 0, 1, 0, N_HIDDEN, N_HIDDEN / GEMM_BK);
+    } else {
+      mb_g = mb_q;
+    }
     EpiInverse::Params ep{c->mu_perm, (float)std::ldexp(1.0, -c->p_inv), rope, row_tok, row_pos,
                           (__nv_bfloat16 *)k_out, (__nv_bfloat16 *)v_out, L.n_tokens};
-    RET((run_gemm2<EpiInverse, 4, 2, 8>(c->map_ainv2, c->map_ainv2, mb_q, mb_q, pr, ep, c->num_sms, false, st)));
+    RET((run_gemm2<EpiInverse, 4, 2, 8>(c->map_ainv2, c->has_synth ? c->map_av2 : c->map_ainv2, mb_q, mb_g, pr, ep,
+                                        c->num_sms, false, st)));
   }
   stage_mark(c, st, "gemm_inverse");
   if (L.n_kept > 0)
@@ -1417,7 +1504,8 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
   if (L.n_rows > 0)
     { k_fixup<<<c->num_sms, 256, 0, st>>>(biglist, counters, q16, qbig, c->a_inv, (float)std::ldexp(1.0, -c->p_inv),
                                        c->mu_perm, c->theta, row_tok, row_pos, (__nv_bfloat16 *)k_out,
-                                       (__nv_bfloat16 *)v_out, L.n_tokens); ++g_launches; }
+                                       (__nv_bfloat16 *)v_out, L.n_tokens, c->has_synth ? c->v1t32 : nullptr,
+                                       c->v2_32, c->delta); ++g_launches; }
   CK(cudaGetLastError());
   stage_mark(c, st, "kept+fixup");
   return DCKV_OK;

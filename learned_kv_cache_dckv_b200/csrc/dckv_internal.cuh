@@ -109,6 +109,7 @@ struct dckv_codec {
   int k_eff = 0;
   bool has_mlp = true;    // correction layer present (false: linear codec)
   bool has_means = true;  // mean models present (false: unconditional zero-mean tables)
+  bool has_synth = false; // decoder-side synthesis correction present
   // caller-owned parameter pointers (read at create)
   dckv_params p{};
   // derived, library-owned device buffers
@@ -142,8 +143,14 @@ struct dckv_codec {
   float *w1t32 = nullptr;    // [256][6144]  w1^T
   float *w2t32 = nullptr;    // [2048][256]  w2^T
   float *mu32 = nullptr;     // [6144]
-  int p_y = 0, p_h = 0, p_inv = 0;  // power-of-two operand scales
-  CUtensorMap map_ay2, map_aw2_2, map_aw2_1, map_ah2, map_ainv2, map_aon1;
+  // decoder-side synthesis (optional): split operands and fp32 copies for the exact fix-up
+  __half *a_v1 = nullptr;    // [2][256][2048]  (Delta_c V1[c][h]) * 2^p_v1, split
+  __half *a_v2 = nullptr;    // [2][6144][256]  V2[h][d] * 2^p_inv, split, dims permuted like a_inv
+  float *v1t32 = nullptr;    // [256][2048]  V1^T
+  float *v2_32 = nullptr;    // [256][6144]  V2
+  float *zero256 = nullptr;  // [256] zeros (the synthesis hidden layer has no offset)
+  int p_y = 0, p_h = 0, p_inv = 0, p_v1 = 0;  // power-of-two operand scales
+  CUtensorMap map_ay2, map_aw2_2, map_aw2_1, map_ah2, map_ainv2, map_aon1, map_av1, map_av2;
   // stage timing (optional)
   int timing = 0;
   cudaEvent_t ev[24];

@@ -371,9 +371,19 @@ def rope(head_vecs, positions):
 
 def reconstruct(q, codec) -> np.ndarray:
     """x_hat = mu + sum_c q_c Delta_c B[:, c] (linear synthesis; the decoder has no x to
-    evaluate the correction MLP on)  [rows], [xform]."""
+    evaluate the encoder's correction on)  [rows], [xform].
+
+    With synthesis weights V1 [2048, 256] and V2 [256, 6144] (the decoder-side learned
+    synthesis the weight count on the pages leaves room for, "How to use it": 176 MiB
+    against 96 MiB for the linear codec) the same kind of one-hidden-layer GELU correction
+    is added on the decoded coefficients: + GELU((q Delta) V1) V2, no biases."""
     qd = np.asarray(q, np.float64) * np.asarray(codec.delta, np.float64)[None, :]
-    return np.asarray(codec.mu, np.float64)[None, :] + qd @ np.asarray(codec.basis, np.float64).T
+    x = np.asarray(codec.mu, np.float64)[None, :] + qd @ np.asarray(codec.basis, np.float64).T
+    v1 = getattr(codec, "v1", None)
+    v2 = getattr(codec, "v2", None)
+    if v1 is not None and v2 is not None:
+        x = x + gelu(qd @ np.asarray(v1, np.float64)) @ np.asarray(v2, np.float64)
+    return x
 
 
 def output_rows(rows_f64, positions):

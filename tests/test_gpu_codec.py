@@ -12,6 +12,8 @@ Parity rules (one GPU, seeded synthetic inputs):
              codes exactly;
   determinism  repeated calls give identical blobs and rows.
 """
+import copy
+
 import numpy as np
 import pytest
 import torch
@@ -262,6 +264,30 @@ def test_parity_linear_codec(src, variant):
     torch.cuda.synchronize()
     assert int(gc.status.item()) == D.DCKV_OK
     assert torch.equal(k2, r["k"]) and torch.equal(v2, r["v"])
+
+
+_SYNTH = {}
+
+
+@pytest.mark.parametrize("big", [False, True])
+def test_parity_decoder_side_synthesis(src, big):
+    # decode adds GELU((q Delta) V1) V2 to the linear synthesis; rows pushed far out reach
+    # codes beyond 2048, which the fix-up recomputes with the synthesis term included
+    if "c" not in _SYNTH:
+        _SYNTH["c"] = S.codec(src, step_scale=None, target_bytes=220.0, embed_std=1.0, mean_gain=1.0,
+                              neigh_gain=40.0, synthesis=True, synthesis_gain=10.0)
+    cod = _SYNTH["c"]
+    if big:
+        r = full_check(src, cod, [132 + 90, 140, 132 + 41], seeds=[81, 82, 83], chunk_rows=8,
+                       boost=(4, 30, 60, 90 + 8), boost_gain=400.0, expect_big=True)
+    else:
+        r = full_check(src, cod, [132 + 300, 132 + 77], seeds=[84, 85])
+    # the synthesis term is not negligible: the oracle's linear decode of the same blob
+    # lies well outside the row tolerance
+    lin = copy.copy(cod)
+    lin.v1 = lin.v2 = None
+    k_l, v_l = O.decode(r["res"]["blob"], r["tok"].cpu().numpy(), r["offs"], lin)
+    assert rel_frob(O.bf16_to_f64(bits(r["k"])), O.bf16_to_f64(k_l)) > 20 * ROW_TOL
 
 
 def test_determinism(src, codec_55):

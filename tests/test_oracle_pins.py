@@ -92,6 +92,28 @@ def test_transform_correction_single_unit(src):
     assert np.max(np.abs(expect)) > 0.1
 
 
+def test_synthesis_correction_single_unit(src):
+    """Decoder-side synthesis with one hidden unit fed by one coefficient: x_hat minus the
+    linear reconstruction is GELU(a q_c Delta_c) * V2[h] (torch's GELU, fp64); without
+    synthesis weights the reconstruction is the linear one."""
+    cod = S.codec(src, step_scale=1.0, synthesis=True)
+    c, h, a = 321, 45, 2.5
+    cod.v1 = np.zeros_like(cod.v1)
+    cod.v1[c, h] = a
+    rng = np.random.default_rng(4)
+    cod.v2 = np.zeros_like(cod.v2)
+    cod.v2[h] = rng.standard_normal(O.ROW_DIM).astype(np.float32)
+    q = rng.integers(-40, 41, (6, O.N_COEF))
+    x = O.reconstruct(q, cod)
+    lin = cod.mu.astype(np.float64)[None, :] + (q * cod.delta.astype(np.float64)) @ cod.basis.astype(np.float64).T
+    u = a * q[:, c] * float(cod.delta[c])
+    expect = torch.nn.functional.gelu(torch.from_numpy(u)).numpy()[:, None] * cod.v2[h].astype(np.float64)[None, :]
+    assert np.max(np.abs((x - lin) - expect)) < 1e-12
+    assert np.max(np.abs(expect)) > 0.01
+    cod.v1 = cod.v2 = None
+    assert np.array_equal(O.reconstruct(q, cod), lin)
+
+
 # ----------------------------------------------------------------------------- quantiser
 def test_quantise_hand_cases():
     delta = np.array([2.0, 0.5, 1.0, 1.0], np.float32)
