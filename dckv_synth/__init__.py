@@ -333,6 +333,65 @@ def batch(src: Source, lengths, seeds, student_t_frac: float = 0.0, device="cpu"
     return torch.cat(xs, 0), torch.cat(ts, 0), offs
 
 
+def structured_prompt(src: Source, embed_bits, n_tokens: int, seed: int, token_gain: float = 0.5,
+                      ar: float = 0.7, device="cpu"):
+    """A prompt whose rows depend on their own token and on their neighbours: the input
+    on which fitting the conditional models has something to find ("Evidence": the mean
+    models predict codes from the token embedding and from both decoded neighbours).
+
+    Latent z_t = sqrt(1 - g^2) u_t + g v(tok_t): u is an AR(1) process along the prompt's
+    positions (u_t = a u_{t-1} + sqrt(1 - a^2) eps_t, unit variance), v(tok) = e(tok) P
+    normalised to unit variance, e the embedding table the codec uses (bf16 bits) and P
+    a seeded Gaussian [2048, 6144] matrix of the source.  Rows are then drawn as for plain
+    prompts: x_t = bf16(mu + (z_t diag(sigma) Q^T) * s).  Returns x bf16 [N, 6144] and
+    token ids int32 [N] (torch, on `device`).
+    """
+    import torch
+
+    dev = torch.device(device)
+    g = torch.Generator(device=dev)
+    g.manual_seed(int(seed) * 7919 + 23)
+    gp = torch.Generator(device=dev)
+    gp.manual_seed(int(src.seed) * 31 + 5)
+    tok = torch.randint(0, VOCAB, (n_tokens,), generator=g, device=dev, dtype=torch.int64)
+    emb = torch.from_numpy(np.ascontiguousarray(embed_bits, np.uint16).view(np.int16)).to(dev)
+    emb = emb.view(torch.bfloat16)
+    rms = float(emb.float().pow(2).mean().sqrt())
+    P = torch.randn((EMBED_DIM, ROW_DIM), generator=gp, device=dev, dtype=torch.float32)
+    qt = torch.from_numpy(src.q).to(dev).t().contiguous()
+    sig = torch.from_numpy(src.sigma.astype(np.float32)).to(dev)
+    s = torch.from_numpy(src.chan_scale).to(dev)
+    mu = torch.from_numpy(src.mu).to(dev)
+    prev = torch.backends.cuda.matmul.allow_tf32
+    torch.backends.cuda.matmul.allow_tf32 = False
+    try:
+        eps = torch.randn((n_tokens, ROW_DIM), generator=g, device=dev, dtype=torch.float32)
+        c = math.sqrt(1.0 - ar * ar)
+        for t in range(1, n_tokens):
+            eps[t] = ar * eps[t - 1] + c * eps[t]
+        v = (emb[tok].float() @ P) / (rms * math.sqrt(EMBED_DIM))
+        z = math.sqrt(1.0 - token_gain * token_gain) * eps + token_gain * v
+        x = (mu[None, :] + ((z * sig[None, :]) @ qt) * s[None, :]).to(torch.bfloat16)
+    finally:
+        torch.backends.cuda.matmul.allow_tf32 = prev
+    return x, tok.to(torch.int32)
+
+
+def structured_batch(src: Source, embed_bits, lengths, seeds, token_gain: float = 0.5, ar: float = 0.7,
+                     device="cpu"):
+    """Concatenated structured prompts: x [sum N, 6144], tok [sum N], seq_offsets (numpy)."""
+    import torch
+
+    xs, ts = [], []
+    for n, sd in zip(lengths, seeds):
+        x, t = structured_prompt(src, embed_bits, int(n), int(sd), token_gain, ar, device)
+        xs.append(x)
+        ts.append(t)
+    offs = np.zeros(len(lengths) + 1, np.int64)
+    offs[1:] = np.cumsum(np.asarray(lengths, np.int64))
+    return torch.cat(xs, 0), torch.cat(ts, 0), offs
+
+
 # Step scales for the configurations, found with codec(target_bytes=...) on seed 0.
 # They are recomputed on demand; the constants only save the bisection.
 def step_scale_for(src: Source, target_bytes: float) -> float:

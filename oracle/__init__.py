@@ -12,4 +12,8 @@ works") that it follows.  Where the pages leave a step open, the reading taken i
 stated in the function's docstring.
 """
 from .codec import *  # noqa: F401,F403
-from .codec import __all__  # noqa: F401
+from .fit import *  # noqa: F401,F403
+from .codec import __all__ as _all_codec
+from .fit import __all__ as _all_fit
+
+__all__ = list(_all_codec) + list(_all_fit)
