@@ -62,6 +62,7 @@ extern "C" {
 #define DCKV_ECORRUPT 4    /* blob header/tables/streams inconsistent (decode)        */
 #define DCKV_ETIMEOUT 5    /* a bounded device wait gave up                           */
 #define DCKV_ERANGE 6      /* encode: an input element beyond +-65504 was clamped     */
+#define DCKV_ESINGULAR 7   /* fit: a non-positive pivot in the Cholesky factorisation */
 
 typedef struct dckv_codec dckv_codec; /* opaque */
 

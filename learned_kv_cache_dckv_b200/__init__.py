@@ -23,8 +23,17 @@ N_HIDDEN = 256
 HEAD_KEPT = 4
 TAIL_KEPT = 128
 
-DCKV_OK, DCKV_EINVAL, DCKV_ECAPACITY, DCKV_ECUDA, DCKV_ECORRUPT, DCKV_ETIMEOUT, DCKV_ERANGE = range(7)
-STATUS_NAMES = {0: "OK", 1: "EINVAL", 2: "ECAPACITY", 3: "ECUDA", 4: "ECORRUPT", 5: "ETIMEOUT", 6: "ERANGE"}
+DCKV_OK, DCKV_EINVAL, DCKV_ECAPACITY, DCKV_ECUDA, DCKV_ECORRUPT, DCKV_ETIMEOUT, DCKV_ERANGE, DCKV_ESINGULAR = range(8)
+STATUS_NAMES = {0: "OK", 1: "EINVAL", 2: "ECAPACITY", 3: "ECUDA", 4: "ECORRUPT", 5: "ETIMEOUT", 6: "ERANGE",
+                7: "ESINGULAR"}
+
+# fp64 layout of the closed-form fit's sums (include/dckv_fit.h)
+FIT_OFF_GE = 0
+FIT_OFF_CE = 2048 * 2048
+FIT_OFF_GO = 2 * 2048 * 2048
+FIT_OFF_CO = FIT_OFF_GO + 6144 * 6144
+FIT_OFF_N = FIT_OFF_CO + 6144 * 2048
+FIT_STATS_DOUBLES = FIT_OFF_N + 8
 
 _lib = None
 
@@ -87,6 +96,13 @@ def lib():
         "dckv_debug_ratio": (I, [P, P]),
         "dckv_codec_info": (I, [P, P, P]),
         "dckv_launch_count": (ctypes.c_longlong, []),
+        "dckv_fit_workspace_bytes": (Z, [P, P, I]),
+        "dckv_fit_accumulate": (I, [P, P, ctypes.c_int32, P, P, P, I, P, P, P, Z, P]),
+        "dckv_fit_solve_workspace_bytes": (Z, []),
+        "dckv_fit_solve": (I, [P, ctypes.c_double, P, P, P, P, Z, P]),
+        "dckv_fit_to_bf16": (I, [P, ctypes.c_int64, P, P]),
+        "dckv_fit_scales_accumulate": (I, [P, P, P, P, I, P, P, P, Z, P]),
+        "dckv_fit_scales_finish": (I, [P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -258,6 +274,54 @@ def dckv_debug_gemm(bf16: bool, A, slabs: int, B, M: int, N: int, K: int, D, bn:
 
 
 # ---------------------------------------------------------------------------------- helpers
+# ------------------------------------------------------------- closed-form fit (dckv_fit.h)
+def dckv_fit_workspace_bytes(handle, seq_offsets) -> int:
+    a, ptr, b = _offs(seq_offsets)
+    return int(lib().dckv_fit_workspace_bytes(handle, ptr, b))
+
+
+def dckv_fit_accumulate(handle, embed, rows, token_ids, seq_offsets, stats, status, workspace, stream=None):
+    """embed bf16 [vocab, 2048] (device), rows bf16 [sum N, 6144], token_ids int32, stats fp64
+    [FIT_STATS_DOUBLES] (accumulated into), status int32[1], workspace uint8 (device)."""
+    a, ptr, b = _offs(seq_offsets)
+    _check(lib().dckv_fit_accumulate(handle, embed.data_ptr(), int(embed.shape[0]), rows.data_ptr(),
+                                     token_ids.data_ptr(), ptr, b, stats.data_ptr(), status.data_ptr(),
+                                     workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                     _stream_ptr(stream)), "dckv_fit_accumulate")
+
+
+def dckv_fit_solve_workspace_bytes() -> int:
+    return int(lib().dckv_fit_solve_workspace_bytes())
+
+
+def dckv_fit_solve(stats, ridge, w_even, w_odd, status, workspace, stream=None):
+    """w_even fp64 [2048, 2048] and w_odd fp64 [6144, 2048] (device) receive the weights."""
+    _check(lib().dckv_fit_solve(stats.data_ptr(), float(ridge), w_even.data_ptr(), w_odd.data_ptr(),
+                                status.data_ptr(), workspace.data_ptr(),
+                                workspace.numel() * workspace.element_size(), _stream_ptr(stream)),
+           "dckv_fit_solve")
+
+
+def dckv_fit_to_bf16(w, out, stream=None):
+    """bf16 bits (out: int16/uint16-sized device tensor) of fp64 w, one RNE step."""
+    _check(lib().dckv_fit_to_bf16(w.data_ptr(), int(w.numel()), out.data_ptr(), _stream_ptr(stream)),
+           "dckv_fit_to_bf16")
+
+
+def dckv_fit_scales_accumulate(handle, rows, token_ids, seq_offsets, abs_sum, status, workspace, stream=None):
+    """abs_sum int64 [2049] (device), accumulated into."""
+    a, ptr, b = _offs(seq_offsets)
+    _check(lib().dckv_fit_scales_accumulate(handle, rows.data_ptr(), _ptr(token_ids), ptr, b, abs_sum.data_ptr(),
+                                            status.data_ptr(), workspace.data_ptr(),
+                                            workspace.numel() * workspace.element_size(), _stream_ptr(stream)),
+           "dckv_fit_scales_accumulate")
+
+
+def dckv_fit_scales_finish(handle, abs_sum, laplace_b, stream=None):
+    _check(lib().dckv_fit_scales_finish(handle, abs_sum.data_ptr(), laplace_b.data_ptr(), _stream_ptr(stream)),
+           "dckv_fit_scales_finish")
+
+
 def upload_params(codec, device="cuda"):
     """Device tensors for dckv_codec_create from an object with numpy attributes mu, basis,
     w1, w2, delta, laplace_b (float32), embed, w_even, w_odd (bf16 bits as uint16) and,

@@ -26,6 +26,7 @@
 #include <string>
 #include <vector>
 
+#include "../../include/dckv_fit.h"
 #include "../../include/dckv_inspect.h"
 #include "dckv_epilogues.cuh"
 #include "dckv_gemm.cuh"
@@ -930,6 +931,7 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
   const uint64_t o_muw1 = take(4ull * N_HIDDEN);
   const uint64_t o_mup = take(4ull * ROW_DIM);
   const uint64_t o_delta = take(4ull * N_COEF);
+  const uint64_t o_lapb = take(4ull * N_COEF);
   const uint64_t o_keep = take(N_COEF);
   const uint64_t o_scale = take(N_COEF);
   const uint64_t o_kl = take(2ull * N_COEF);
@@ -965,6 +967,7 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
   c->muw1 = (float *)(B + o_muw1);
   c->mu_perm = (float *)(B + o_mup);
   c->delta = (float *)(B + o_delta);
+  c->lapb = (float *)(B + o_lapb);
   c->keep = B + o_keep;
   c->scale = B + o_scale;
   c->kept_list = (int16_t *)(B + o_kl);
@@ -997,6 +1000,7 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
   { k_tables<<<N_SCALES, 512, 0, st>>>(c->cdf); ++g_launches; }
   { k_build_lut<<<N_SCALES, 256, 0, st>>>(c->cdf, c->dcdf, c->lut, c->tail, c->cfm_tab); ++g_launches; }
   cudaMemcpyAsync(c->delta, prm->delta, 4ull * N_COEF, cudaMemcpyDeviceToDevice, st);
+  cudaMemcpyAsync(c->lapb, prm->laplace_b, 4ull * N_COEF, cudaMemcpyDeviceToDevice, st);
   // scale exponents: largest |value| of each split operand brought to about 2^12
   { k_absmax<<<256, 256, 0, st>>>(prm->basis, (int64_t)ROW_DIM * N_COEF, N_COEF, nullptr, scr + 1); ++g_launches; }
   if (has_mlp) {
@@ -1240,11 +1244,16 @@ static int upload_tables(const dckv_codec *c, const Layout &L, uint8_t *ws, cons
 }
 
 // ============================================================================ encode
-extern "C" int dckv_encode(const dckv_codec *c, const void *rows, const int32_t *token_ids, const int64_t *seq_offsets,
-                           int batch, void *blob, size_t blob_cap, uint64_t *blob_size_dev, int32_t *status_dev,
-                           void *workspace, size_t ws_bytes, void *stream) {
-  if (!c || !rows || !blob || !blob_size_dev || !status_dev || !workspace || (c->has_means && !token_ids))
+// The encoder.  stop = 0: the whole path; 1: stop once every code is final (after the
+// exact recomputation; the closed-form fit reads the codes); 2: stop after the symbol
+// kernel (centres final too).  With stop != 0 the blob may be NULL (kept rows are skipped).
+static int encode_impl(const dckv_codec *c, const void *rows, const int32_t *token_ids, const int64_t *seq_offsets,
+                       int batch, void *blob, size_t blob_cap, uint64_t *blob_size_dev, int32_t *status_dev,
+                       void *workspace, size_t ws_bytes, void *stream, int stop) {
+  if (!c || !rows || (!stop && (!blob || !blob_size_dev)) || !status_dev || !workspace ||
+      (c->has_means && !token_ids))
     return fail(DCKV_EINVAL, "a pointer argument is NULL");
+  if (!blob) blob_cap = 0;
   if (((uintptr_t)rows & 15) || ((uintptr_t)blob & 15) || ((uintptr_t)workspace & 255))
     return fail(DCKV_EINVAL, "rows/blob must be 16-byte and workspace 256-byte aligned");
   Layout L;
@@ -1330,6 +1339,7 @@ extern "C" int dckv_encode(const dckv_codec *c, const void *rows, const int32_t 
                                                   row_edst); ++g_launches; }
     CK(cudaGetLastError());
     stage_mark(c, st, "refine");
+    if (stop == 1) return DCKV_OK;
     // odd mean model: [e, bf16(q_left), bf16(q_right)] @ w_odd -> centres
     if (c->has_means) {
       GemmProblem pr = make_problem(N_COEF / GEMM_BM, L.ne_pad, MEAN_ODD_BN, true, status_dev);
@@ -1349,6 +1359,7 @@ extern "C" int dckv_encode(const dckv_codec *c, const void *rows, const int32_t 
     CK(cudaGetLastError());
     stage_mark(c, st, "symbols");
   }
+  if (stop) return DCKV_OK;
   uint32_t *states = (uint32_t *)(ws + w.states), *nwords = (uint32_t *)(ws + w.nwords);
   uint32_t *nesc = (uint32_t *)(ws + w.nesc), *offs = (uint32_t *)(ws + w.offs);
   if (L.n_chunks > 0) {
@@ -1371,6 +1382,13 @@ extern "C" int dckv_encode(const dckv_codec *c, const void *rows, const int32_t 
   }
   stage_mark(c, st, "scan+compact");
   return DCKV_OK;
+}
+
+extern "C" int dckv_encode(const dckv_codec *c, const void *rows, const int32_t *token_ids, const int64_t *seq_offsets,
+                           int batch, void *blob, size_t blob_cap, uint64_t *blob_size_dev, int32_t *status_dev,
+                           void *workspace, size_t ws_bytes, void *stream) {
+  return encode_impl(c, rows, token_ids, seq_offsets, batch, blob, blob_cap, blob_size_dev, status_dev, workspace,
+                     ws_bytes, stream, 0);
 }
 
 // ============================================================================ decode
@@ -1705,3 +1723,6 @@ extern "C" int dckv_decode_static(const dckv_codec *c, const void *blob, size_t 
   return dckv_decode(c, blob, blob_bytes, token_ids, seq_offsets, batch, k_out, v_out, status_dev, scratch,
                      (size_t)DCKV_STATIC_SCRATCH_BYTES, stream);
 }
+
+// closed-form fit of the conditional models (calibration; not on the encode/decode path)
+#include "dckv_fit.cuh"

@@ -43,6 +43,30 @@ struct EpiStoreF32 {
   }
 };
 
+// ------------------------------------------------------------------ fp64 accumulation
+// out[n][m] += D[m][n] in fp64 (the closed-form fit's normal-equation sums: the GEMM runs
+// over a slice of calibration rows, fp32 in TMEM, and every slice is added in fp64).
+// Lanes hold consecutive m, so the transposed store is coalesced; for a symmetric product
+// (G = X^T X) the transpose is the same matrix.
+struct EpiAccF64 {
+  struct Params {
+    double *out;
+    int64_t ld;
+  };
+  static constexpr int SMEM_BYTES = 0;
+  __device__ __forceinline__ static void tile(const Params &p, const EpiCtx &cx) {
+    const int m = cx.mt * GEMM_BM + cx.ew * 32 + cx.lane;
+    for (int c0 = cx.grp * 32; c0 < cx.n_valid; c0 += 32 * cx.n_grp) {
+      uint32_t r[32];
+      tmem_ld_32x32b_x32(cx.tacc + (uint32_t)c0, r);
+      tmem_ld_wait();
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (c0 + j < cx.n_valid) p.out[(int64_t)(cx.n0 + c0 + j) * p.ld + m] += (double)u2f(r[j]);
+    }
+  }
+};
+
 // ------------------------------------------------------------------ correction layer 1
 // h = D * 2^-p_h - (mu @ w1)[m];  g = GELU(h) (erf form);  G[row][m] = fp16(g),
 // G[row][256 + m] = fp16(g - fp16(g))  (the hi/lo pair feeds the second layer's GEMM)

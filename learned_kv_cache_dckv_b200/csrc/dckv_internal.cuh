@@ -125,6 +125,7 @@ struct dckv_codec {
   float *muw1 = nullptr;     // [256]   mu @ w1
   float *mu_perm = nullptr;  // [6144]  mu in the inverse GEMM's row order
   float *delta = nullptr;    // [2048]
+  float *lapb = nullptr;     // [2048]  Laplace scales as given (the fit keeps dropped ones)
   uint8_t *keep = nullptr;   // [2048]
   uint8_t *scale = nullptr;  // [2048]
   int16_t *kept_list = nullptr;   // [2048] kept component indices (first k_eff valid)
