@@ -655,12 +655,13 @@ __global__ void __launch_bounds__(RANS_WARPS * 32) rans_decode_kernel(RansDecArg
   if (__any_sync(0xffffffffu, bad) && lane == 0) atomicExch(a.status, DCKV_ECORRUPT);
 }
 
-// Finishing a decoded pass, one block per chunk, one warp per row: code = centre +
-// symbol - 254, or the chunk's next escape value for ESC; codes go to q16 (fp16, exact
-// below 2048), even rows also to qe (bf16, the odd mean model's input), codes of 2048 or
-// more to qbig with the row listed for the exact fix-up.  Escape values are stored in
-// symbol order, so each row first counts its escapes and takes its base from the rows
-// before it.
+// Finishing a decoded pass, one block per chunk: code = centre + symbol - 254, or the
+// chunk's next escape value for ESC; codes go to q16 (fp16, exact below 2048), even rows
+// also to qe (bf16, the odd mean model's input), codes of 2048 or more to qbig with the
+// row listed for the exact fix-up.  The chunk's symbols are cut into tiles of 128 in
+// symbol order; a first pass counts each tile's escapes, a scan gives each tile the rank
+// of its first escape (escape values are stored in symbol order), and a second pass
+// writes the codes.  Both passes keep several tiles' loads in flight per warp.
 struct DecCodesArgs {
   const ChunkDesc *chunks;
   const PromptInfo *prompts;
@@ -682,91 +683,124 @@ struct DecCodesArgs {
   int32_t *status;
 };
 
-constexpr int DEC_CODES_THREADS = 256;
-constexpr int DEC_UNROLL = 4;
+constexpr int DEC_CODES_THREADS = 512;
+constexpr int DEC_TILE = 128;                         // symbols per tile (4 per lane)
+constexpr int DEC_MAX_TILES = 256 * N_COEF / DEC_TILE;  // 256 rows per chunk at most
+constexpr int DEC_TILE_BATCH = 4;                     // tiles per warp in flight
 
 __global__ void __launch_bounds__(DEC_CODES_THREADS) k_decode_codes(DecCodesArgs a) {
-  __shared__ uint32_t s_esc[256];  // escapes per row of the chunk (at most 256 rows)
+  __shared__ uint32_t s_cnt[DEC_MAX_TILES];  // escapes per tile, then the rank of its first
   __shared__ int16_t s_kl[N_COEF];
+  __shared__ uint32_t s_total;
   if (*a.valid != 1) return;
   for (int k = threadIdx.x; k < a.k_eff; k += DEC_CODES_THREADS) s_kl[k] = a.kept_list[k];
-  __syncthreads();
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
-  const int nw = DEC_CODES_THREADS / 32;
+  constexpr int NW = DEC_CODES_THREADS / 32;
   const uint32_t lt_mask = (1u << lane) - 1u;
   const int K = a.k_eff;
   for (int cb = blockIdx.x; cb < a.n_chunks; cb += gridDim.x) {
     const int ci = a.chunk0 + cb;
     const ChunkDesc cd = a.chunks[ci];
     const PromptInfo pi = a.prompts[cd.prompt];
-    const int64_t slot_row0 = cd.sym_base / (K > 0 ? K : 1);
+    const uint32_t S = (uint32_t)cd.nrows * (uint32_t)K;
+    const int n_tiles = (int)((S + DEC_TILE - 1) / DEC_TILE);
+    const uint16_t *sy = a.syms + cd.sym_base;
+    const int8_t *ce = a.cen8 + cd.sym_base;
     const uint8_t *sec = a.blob + a.off_streams + a.offs[ci];
     const uint32_t ne = reinterpret_cast<const uint32_t *>(sec)[32];
     const uint32_t *ev = reinterpret_cast<const uint32_t *>(sec + CHUNK_FIXED_BYTES);
-    for (int rl = warp; rl < cd.nrows; rl += nw) {
-      const uint16_t *sy = a.syms + (slot_row0 + rl) * K;
-      uint32_t n = 0;
-      for (int k = lane; k < K; k += 32) n += sy[k] == ESC_SYM;
-      for (int o = 16; o; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
-      if (lane == 0) s_esc[rl] = n;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      uint32_t tot = 0;
-      for (int r = 0; r < cd.nrows; ++r) tot += s_esc[r];
-      if (tot != ne) atomicExch(a.status, DCKV_ECORRUPT);  // every escape value used exactly once
-    }
-    for (int rl = warp; rl < cd.nrows; rl += nw) {
-      uint32_t ep = 0;
-      for (int r = 0; r < rl; ++r) ep += s_esc[r];
-      const uint16_t *sy = a.syms + (slot_row0 + rl) * K;
-      const int8_t *ce = a.cen8 + (slot_row0 + rl) * K;
-      const int j = cd.j0 + rl;
-      const int64_t row = (int64_t)pi.row_base + 2 * j + cd.parity;
-      __half *q16 = a.q16 + row * N_COEF;
-      __nv_bfloat16 *qe = cd.parity == 0 ? a.qe + (int64_t)(pi.ebase + j) * N_COEF : nullptr;
-      bool bad = false;
-      for (int k0 = 0; k0 < K; k0 += 32 * DEC_UNROLL) {
-        int sym[DEC_UNROLL], cen[DEC_UNROLL];
+    __syncthreads();  // s_kl loaded; the previous chunk's ranks are no longer read
+    // pass 1: escapes per tile
+    for (int t0 = warp * DEC_TILE_BATCH; t0 < n_tiles; t0 += NW * DEC_TILE_BATCH) {
+      uint16_t v[DEC_TILE_BATCH][4];
 #pragma unroll
-        for (int u = 0; u < DEC_UNROLL; ++u) {  // loads first: DEC_UNROLL positions in flight
-          const int k = k0 + u * 32 + lane;
-          sym[u] = k < K ? (int)sy[k] : 0;
-          cen[u] = k < K ? (int)ce[k] : 0;
+      for (int b = 0; b < DEC_TILE_BATCH; ++b)
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const uint32_t i = (uint32_t)(t0 + b) * DEC_TILE + u * 32 + lane;
+          v[b][u] = i < S ? sy[i] : (uint16_t)0;
         }
 #pragma unroll
-        for (int u = 0; u < DEC_UNROLL; ++u) {
-          const int k = k0 + u * 32 + lane;
-          const bool valid = k < K;
-          const bool is_esc = valid && sym[u] == ESC_SYM;
+      for (int b = 0; b < DEC_TILE_BATCH; ++b) {
+        uint32_t n = 0;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) n += __popc(__ballot_sync(0xffffffffu, v[b][u] == ESC_SYM));
+        if (lane == 0 && t0 + b < n_tiles) s_cnt[t0 + b] = n;
+      }
+    }
+    __syncthreads();
+    if (warp == 0) {  // exclusive scan of the tile counts, 32 contiguous runs
+      const int per = (n_tiles + 31) / 32;
+      const int lo = min(n_tiles, lane * per), hi = min(n_tiles, lo + per);
+      uint32_t sum = 0;
+      for (int t = lo; t < hi; ++t) sum += s_cnt[t];
+      uint32_t inc = sum;
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += y;
+      }
+      uint32_t run = inc - sum;
+      for (int t = lo; t < hi; ++t) {
+        const uint32_t c = s_cnt[t];
+        s_cnt[t] = run;
+        run += c;
+      }
+      if (lane == 31) s_total = inc;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && s_total != ne) atomicExch(a.status, DCKV_ECORRUPT);  // every escape value used once
+    // pass 2: codes
+    bool bad = false;
+    const int64_t row0 = (int64_t)pi.row_base + 2 * cd.j0 + cd.parity;
+    for (int t0 = warp * DEC_TILE_BATCH; t0 < n_tiles; t0 += NW * DEC_TILE_BATCH) {
+      uint16_t v[DEC_TILE_BATCH][4];
+      int8_t cv[DEC_TILE_BATCH][4];
+#pragma unroll
+      for (int b = 0; b < DEC_TILE_BATCH; ++b)
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const uint32_t i = (uint32_t)(t0 + b) * DEC_TILE + u * 32 + lane;
+          v[b][u] = i < S ? sy[i] : (uint16_t)0;
+          cv[b][u] = i < S ? ce[i] : (int8_t)0;
+        }
+#pragma unroll
+      for (int b = 0; b < DEC_TILE_BATCH; ++b) {
+        if (t0 + b >= n_tiles) break;  // warp-uniform
+        uint32_t ep = s_cnt[t0 + b];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const uint32_t i = (uint32_t)(t0 + b) * DEC_TILE + u * 32 + lane;
+          const bool valid = i < S;
+          const bool is_esc = valid && v[b][u] == ESC_SYM;
           const uint32_t me = __ballot_sync(0xffffffffu, is_esc);
-          int q = valid ? sym[u] - R_MAX + cen[u] : 0;
-          if (is_esc) {
-            const uint32_t e = ep + __popc(me & lt_mask);
-            if (e < ne) {
-              const int64_t sv = (int64_t)((uint64_t)ev[2 * e] | ((uint64_t)ev[2 * e + 1] << 32));
-              q = (int)max(min(sv, (int64_t)INT32_MAX), (int64_t)INT32_MIN);
-              if (sv >= -ESC_LIMIT && sv <= ESC_LIMIT) bad = true;  // not an escape value
-            } else {
-              bad = true;
-            }
-          }
-          ep += __popc(me);
           if (valid) {
-            const int comp = s_kl[k];
-            q16[comp] = __float2half_rn((float)q);
-            if (qe) qe[comp] = __float2bfloat16_rn((float)q);
+            int q = (int)v[b][u] - R_MAX + (int)cv[b][u];
+            if (is_esc) {
+              const uint32_t e = ep + __popc(me & lt_mask);
+              if (e < ne) {
+                const int64_t sval = (int64_t)((uint64_t)ev[2 * e] | ((uint64_t)ev[2 * e + 1] << 32));
+                q = (int)max(min(sval, (int64_t)INT32_MAX), (int64_t)INT32_MIN);
+                if (sval >= -ESC_LIMIT && sval <= ESC_LIMIT) bad = true;  // not an escape value
+              } else {
+                bad = true;
+              }
+            }
+            const uint32_t r = i / (uint32_t)K;
+            const int comp = s_kl[i - r * (uint32_t)K];
+            const int64_t row = row0 + 2 * (int64_t)r;
+            a.q16[row * N_COEF + comp] = __float2half_rn((float)q);
+            if (cd.parity == 0) a.qe[(int64_t)(pi.ebase + cd.j0 + r) * N_COEF + comp] = __float2bfloat16_rn((float)q);
             if (q >= BIG_CODE || q <= -BIG_CODE) {
               a.qbig[row * N_COEF + comp] = q;
               if (atomicExch(&a.bigflag[row], 1u) == 0u) a.biglist[atomicAdd(a.bigcount, 1u)] = (int32_t)row;
             }
           }
+          ep += __popc(me);
         }
       }
-      if (__any_sync(0xffffffffu, bad) && lane == 0) atomicExch(a.status, DCKV_ECORRUPT);
     }
-    __syncthreads();
+    if (__any_sync(0xffffffffu, bad) && lane == 0) atomicExch(a.status, DCKV_ECORRUPT);
   }
 }
 
