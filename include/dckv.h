@@ -115,7 +115,8 @@ typedef struct {
  * (states, escape count, offset) stay within 3.5% of the tables' own entropy per row.
  * Fewer rows per chunk give more independent streams (faster decode) and more bytes.
  * Allocates device memory (about 2 * vocab * 8 KiB + 192 MiB: split GEMM operands, fp32
- * weight copies for the exact recomputation of near-boundary codes, tables).
+ * weight copies for the exact recomputation of near-boundary codes, tables; 16 MiB more
+ * with decoder-side synthesis weights).
  * Synchronises the device.  Returns DCKV_OK or an error; *out is NULL on error. */
 int dckv_codec_create(const dckv_params *params, int device, int chunk_rows, dckv_codec **out);
 void dckv_codec_destroy(dckv_codec *codec);
