@@ -149,14 +149,14 @@ static int launch_pairs(const void *kern, int tiles, int num_sms, int threads, i
   return DCKV_OK;
 }
 
-template <class Epi, int STAGES, int MAX_SLABS, int EPI_WARPS>
+template <class Epi, int STAGES, int MAX_SLABS, int EPI_WARPS, int BN_MAX = GEMM_MAX_BN>
 static int run_gemm2(const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &b0, const CUtensorMap &b1,
                      GemmProblem prob, const typename Epi::Params &ep, int num_sms, bool bf16, cudaStream_t st) {
-  constexpr int smem = gemm2_smem_bytes<Epi, STAGES, MAX_SLABS, EPI_WARPS>();
+  constexpr int smem = gemm2_smem_bytes<Epi, STAGES, MAX_SLABS, EPI_WARPS, BN_MAX>();
   static_assert(smem <= 232448, "GEMM shared memory above the sm_100 limit");
-  auto kern = gemm2_kernel<Epi, STAGES, MAX_SLABS, EPI_WARPS>;
+  auto kern = gemm2_kernel<Epi, STAGES, MAX_SLABS, EPI_WARPS, BN_MAX>;
   CK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-  if (prob.m_tiles % 2 || prob.bn % 16 || prob.bn > GEMM_MAX_BN) return fail(DCKV_EINVAL, "bad CTA-pair GEMM shape");
+  if (prob.m_tiles % 2 || prob.bn % 16 || prob.bn > BN_MAX) return fail(DCKV_EINVAL, "bad CTA-pair GEMM shape");
   const int tiles = (prob.m_tiles / 2) * prob.n_tiles;
   if (tiles <= 0) return DCKV_OK;
   for (int i = 0; i < prob.n_seg; ++i)
@@ -1310,7 +1310,7 @@ static int encode_impl(const dckv_codec *c, const void *rows, const int32_t *tok
       GemmProblem pr = make_problem(N_HIDDEN / GEMM_BM, L.n_rows, HIDDEN_BN, false, status_dev);
       add_seg(pr, 0, 0, 2, 0, 0, 0, 0, ROW_DIM / GEMM_BK);
       EpiGelu::Params ep{c->muw1, (float)std::ldexp(1.0, -c->p_h), g16};
-      RET((run_gemm2<EpiGelu, 4, 2, 4>(c->map_ah2, c->map_ah2, mb_xh, mb_xh, pr, ep, c->num_sms, false, st)));
+      RET((run_gemm2<EpiGelu, 4, 2, 4, HIDDEN_BN>(c->map_ah2, c->map_ah2, mb_xh, mb_xh, pr, ep, c->num_sms, false, st)));
     }
     stage_mark(c, st, "gemm_hidden");
     // transform + quantiser: y = x @ B + g @ w2 - mu @ B
@@ -1346,7 +1346,7 @@ static int encode_impl(const dckv_codec *c, const void *rows, const int32_t *tok
       add_seg(pr, 0, 0, 1, 0, 0, 0, 0, N_COEF / GEMM_BK);
       add_seg(pr, 0, 0, 1, N_COEF, 0, 1, 0, N_COEF / GEMM_BK);
       EpiMeanOdd::Params ep{c->t_odd, token_ids, e_tok, e_slot, c->kidx, cen8, c->k_eff, c->vocab};
-      RET((run_gemm2<EpiMeanOdd, 6, 1, 8>(c->map_aon1, c->map_aon1, mb_qe, mb_qe, pr, ep, c->num_sms, true, st)));
+      RET((run_gemm2<EpiMeanOdd, 6, 1, 8, MEAN_ODD_BN>(c->map_aon1, c->map_aon1, mb_qe, mb_qe, pr, ep, c->num_sms, true, st)));
     }
     stage_mark(c, st, "gemm_mean_odd");
     // even centres from the vocabulary table, then every symbol, in slot order
@@ -1478,7 +1478,7 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
     add_seg(pr, 0, 0, 1, 0, 0, 0, 0, N_COEF / GEMM_BK);
     add_seg(pr, 0, 0, 1, N_COEF, 0, 1, 0, N_COEF / GEMM_BK);
     EpiMeanOdd::Params ep{c->t_odd, token_ids, e_tok, e_slot, c->kidx, cen8, c->k_eff, c->vocab};
-    RET((run_gemm2<EpiMeanOdd, 6, 1, 8>(c->map_aon1, c->map_aon1, mb_qe, mb_qe, pr, ep, c->num_sms, true, st)));
+    RET((run_gemm2<EpiMeanOdd, 6, 1, 8, MEAN_ODD_BN>(c->map_aon1, c->map_aon1, mb_qe, mb_qe, pr, ep, c->num_sms, true, st)));
   }
   stage_mark(c, st, "gemm_mean_odd");
   if (L.n_chunks_o > 0) {
@@ -1495,7 +1495,7 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
     GemmProblem pr = make_problem(N_HIDDEN / GEMM_BM, L.n_rows, HIDDEN_BN, false, status_dev);
     add_seg(pr, 0, 0, 2, 0, 0, 0, 0, N_COEF / GEMM_BK);
     EpiGelu::Params ep{c->zero256, (float)std::ldexp(1.0, -c->p_v1), g16d};
-    RET((run_gemm2<EpiGelu, 4, 2, 4>(c->map_av1, c->map_av1, mb_qh, mb_qh, pr, ep, c->num_sms, false, st)));
+    RET((run_gemm2<EpiGelu, 4, 2, 4, HIDDEN_BN>(c->map_av1, c->map_av1, mb_qh, mb_qh, pr, ep, c->num_sms, false, st)));
     stage_mark(c, st, "gemm_synth_hidden");
   }
   if (L.n_rows > 0) {

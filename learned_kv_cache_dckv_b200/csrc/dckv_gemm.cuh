@@ -255,13 +255,13 @@ struct Gemm2Smem {  // one stage: the A slabs, then this CTA's half of the B til
   static constexpr int STAGE_BYTES = MAX_SLABS * GEMM_SLAB_BYTES + (BN / 2) * GEMM_BK * 2;
 };
 
-template <class Epi, int STAGES, int MAX_SLABS, int EPI_WARPS>
+template <class Epi, int STAGES, int MAX_SLABS, int EPI_WARPS, int BN_MAX = GEMM_MAX_BN>
 __global__ void __launch_bounds__(64 + 32 * EPI_WARPS, 1)
     gemm2_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                  const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
                  const GemmProblem prob, const typename Epi::Params ep) {
   extern __shared__ __align__(1024) uint8_t dyn_smem[];
-  constexpr int STAGE_BYTES = Gemm2Smem<MAX_SLABS>::STAGE_BYTES;
+  constexpr int STAGE_BYTES = Gemm2Smem<MAX_SLABS, BN_MAX>::STAGE_BYTES;  // stages sized for tiles up to BN_MAX
   constexpr int N_GRP = EPI_WARPS / 4;
   constexpr int EPI_SCRATCH = (Epi::SMEM_BYTES + 15) & ~15;
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
@@ -437,9 +437,10 @@ __global__ void __launch_bounds__(64 + 32 * EPI_WARPS, 1)
   }
 }
 
-template <class Epi, int STAGES, int MAX_SLABS, int EPI_WARPS>
+template <class Epi, int STAGES, int MAX_SLABS, int EPI_WARPS, int BN_MAX = GEMM_MAX_BN>
 constexpr int gemm2_smem_bytes() {
-  return 1024 + STAGES * Gemm2Smem<MAX_SLABS>::STAGE_BYTES + 1024 + (EPI_WARPS / 4) * ((Epi::SMEM_BYTES + 15) & ~15);
+  return 1024 + STAGES * Gemm2Smem<MAX_SLABS, BN_MAX>::STAGE_BYTES + 1024 +
+         (EPI_WARPS / 4) * ((Epi::SMEM_BYTES + 15) & ~15);
 }
 
 // ------------------------------------------------------------------------------------------
