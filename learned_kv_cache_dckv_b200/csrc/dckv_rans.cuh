@@ -768,9 +768,13 @@ __global__ void __launch_bounds__(DEC_CODES_THREADS) k_decode_codes(DecCodesArgs
       for (int b = 0; b < DEC_TILE_BATCH; ++b) {
         if (t0 + b >= n_tiles) break;  // warp-uniform
         uint32_t ep = s_cnt[t0 + b];
+        // row and kept component of this lane's first symbol in the tile; later ones by steps of 32
+        const uint32_t i0 = (uint32_t)(t0 + b) * DEC_TILE + lane;
+        uint32_t r = i0 / (uint32_t)K;
+        int kc = (int)(i0 - r * (uint32_t)K);
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const uint32_t i = (uint32_t)(t0 + b) * DEC_TILE + u * 32 + lane;
+          const uint32_t i = i0 + u * 32;
           const bool valid = i < S;
           const bool is_esc = valid && v[b][u] == ESC_SYM;
           const uint32_t me = __ballot_sync(0xffffffffu, is_esc);
@@ -786,8 +790,7 @@ __global__ void __launch_bounds__(DEC_CODES_THREADS) k_decode_codes(DecCodesArgs
                 bad = true;
               }
             }
-            const uint32_t r = i / (uint32_t)K;
-            const int comp = s_kl[i - r * (uint32_t)K];
+            const int comp = s_kl[kc];
             const int64_t row = row0 + 2 * (int64_t)r;
             a.q16[row * N_COEF + comp] = __float2half_rn((float)q);
             if (cd.parity == 0) a.qe[(int64_t)(pi.ebase + cd.j0 + r) * N_COEF + comp] = __float2bfloat16_rn((float)q);
@@ -797,6 +800,11 @@ __global__ void __launch_bounds__(DEC_CODES_THREADS) k_decode_codes(DecCodesArgs
             }
           }
           ep += __popc(me);
+          kc += 32;
+          while (kc >= K) {
+            kc -= K;
+            ++r;
+          }
         }
       }
     }
