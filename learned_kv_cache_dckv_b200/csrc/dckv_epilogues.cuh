@@ -59,10 +59,18 @@ struct EpiAccF64 {
     for (int c0 = cx.grp * 32; c0 < cx.n_valid; c0 += 32 * cx.n_grp) {
       uint32_t r[32];
       tmem_ld_32x32b_x32(cx.tacc + (uint32_t)c0, r);
+      double *o = p.out + (int64_t)(cx.n0 + c0) * p.ld + m;
+      const int nv = min(32, cx.n_valid - c0);
       tmem_ld_wait();
 #pragma unroll
-      for (int j = 0; j < 32; ++j)
-        if (c0 + j < cx.n_valid) p.out[(int64_t)(cx.n0 + c0 + j) * p.ld + m] += (double)u2f(r[j]);
+      for (int h = 0; h < 32; h += 16) {
+        double v[16];  // 16 loads before their stores: the compiler cannot tell that they do not alias
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[j] = h + j < nv ? o[(int64_t)(h + j) * p.ld] : 0.0;
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          if (h + j < nv) o[(int64_t)(h + j) * p.ld] = v[j] + (double)u2f(r[h + j]);
+      }
     }
   }
 };
