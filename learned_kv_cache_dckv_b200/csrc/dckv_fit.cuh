@@ -167,7 +167,19 @@ __global__ void __launch_bounds__(256) k_fit_prep(const double *G, int n, double
 __global__ void __launch_bounds__(256) k_chol_diag(double *A, int n, int k, int32_t *status) {
   __shared__ double s[FB][FB + 1];
   const int k0 = k * FB;
-  for (int e = threadIdx.x; e < FB * FB; e += blockDim.x) s[e / FB][e % FB] = A[(int64_t)(k0 + e / FB) * n + k0 + e % FB];
+  {  // loads into registers first: a shared-memory store between two global loads serialises them
+    double v[FB * FB / 256];
+#pragma unroll
+    for (int u = 0; u < FB * FB / 256; ++u) {
+      const int e = threadIdx.x + 256 * u;
+      v[u] = A[(int64_t)(k0 + e / FB) * n + k0 + e % FB];
+    }
+#pragma unroll
+    for (int u = 0; u < FB * FB / 256; ++u) {
+      const int e = threadIdx.x + 256 * u;
+      s[e / FB][e % FB] = v[u];
+    }
+  }
   __syncthreads();
   for (int j = 0; j < FB; ++j) {
     if (threadIdx.x == 0) {
@@ -202,9 +214,19 @@ __global__ void __launch_bounds__(FB) k_chol_panel(double *A, int n, int k) {
   const int k0 = k * FB;
   const int64_t r0 = k0 + FB + (int64_t)blockIdx.x * FB;
   const int t = threadIdx.x;
-  for (int i = 0; i < FB; ++i) {
-    Lk[i][t] = A[(int64_t)(k0 + i) * n + k0 + t];
-    P[i][t] = A[(r0 + i) * n + k0 + t];
+#pragma unroll
+  for (int i0 = 0; i0 < FB; i0 += 16) {  // 32 loads in flight, then their shared-memory stores
+    double lv[16], pv[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      lv[u] = A[(int64_t)(k0 + i0 + u) * n + k0 + t];
+      pv[u] = A[(r0 + i0 + u) * n + k0 + t];
+    }
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      Lk[i0 + u][t] = lv[u];
+      P[i0 + u][t] = pv[u];
+    }
   }
   __syncthreads();
   for (int j = 0; j < FB; ++j) {
@@ -229,12 +251,26 @@ __global__ void __launch_bounds__(256) k_dgemm64(int M, int N, const double *P, 
   if (LOWER && bj > bi) return;
   const int i0 = bi * FB, j0 = bj * FB;
   const int t = threadIdx.x;
-  for (int e = t; e < FB * FB; e += 256) {
-    const int a = e / FB, b = e % FB;  // b runs along memory
-    if (TP) Ps[b][a] = (i0 + b < M) ? P[(int64_t)a * ldp + i0 + b] : 0.0;
-    else Ps[a][b] = (i0 + a < M) ? P[(int64_t)(i0 + a) * ldp + b] : 0.0;
-    if (TQ) Qs[b][a] = (j0 + a < N) ? Q[(int64_t)(j0 + a) * ldq + b] : 0.0;
-    else Qs[a][b] = (j0 + b < N) ? Q[(int64_t)a * ldq + j0 + b] : 0.0;
+  {  // 32 loads in flight, then their shared-memory stores
+    double pv[FB * FB / 256], qv[FB * FB / 256];
+#pragma unroll
+    for (int u = 0; u < FB * FB / 256; ++u) {
+      const int e = t + 256 * u;
+      const int a = e / FB, b = e % FB;  // b runs along memory
+      if (TP) pv[u] = (i0 + b < M) ? P[(int64_t)a * ldp + i0 + b] : 0.0;
+      else pv[u] = (i0 + a < M) ? P[(int64_t)(i0 + a) * ldp + b] : 0.0;
+      if (TQ) qv[u] = (j0 + a < N) ? Q[(int64_t)(j0 + a) * ldq + b] : 0.0;
+      else qv[u] = (j0 + b < N) ? Q[(int64_t)a * ldq + j0 + b] : 0.0;
+    }
+#pragma unroll
+    for (int u = 0; u < FB * FB / 256; ++u) {
+      const int e = t + 256 * u;
+      const int a = e / FB, b = e % FB;
+      if (TP) Ps[b][a] = pv[u];
+      else Ps[a][b] = pv[u];
+      if (TQ) Qs[b][a] = qv[u];
+      else Qs[a][b] = qv[u];
+    }
   }
   __syncthreads();
   const int tx = t & 15, ty = t >> 4;
@@ -255,12 +291,21 @@ __global__ void __launch_bounds__(256) k_dgemm64(int M, int N, const double *P, 
 #pragma unroll
       for (int c = 0; c < 4; ++c) acc[r][c] = fma(av[r], bv[c], acc[r][c]);
   }
+  // all sixteen loads before the stores (O may alias P or Q as far as the compiler knows)
+  double cur[4][4];
 #pragma unroll
   for (int r = 0; r < 4; ++r)
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       const int i = i0 + ty + 16 * r, j = j0 + tx + 16 * c;
-      if (i < M && j < N) O[(int64_t)i * ldo + j] -= acc[r][c];
+      cur[r][c] = (i < M && j < N) ? O[(int64_t)i * ldo + j] : 0.0;
+    }
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int i = i0 + ty + 16 * r, j = j0 + tx + 16 * c;
+      if (i < M && j < N) O[(int64_t)i * ldo + j] = cur[r][c] - acc[r][c];
     }
 }
 
@@ -272,9 +317,29 @@ __global__ void __launch_bounds__(128) k_trsm_rhs(const double *A, int n, int k,
   double(*Lk)[FB + 1] = reinterpret_cast<double(*)[FB + 1]>(dsm);
   double(*Ys)[129] = reinterpret_cast<double(*)[129]>(dsm + FB * (FB + 1));
   const int k0 = k * FB, c0 = blockIdx.x * 128, t = threadIdx.x;
-  for (int e = t; e < FB * FB; e += 128) Lk[e / FB][e % FB] = A[(int64_t)(k0 + e / FB) * n + k0 + e % FB];
   const bool ok = c0 + t < r;
-  for (int i = 0; i < FB; ++i) Ys[i][t] = ok ? Y[(int64_t)(k0 + i) * r + c0 + t] : 0.0;
+#pragma unroll
+  for (int g = 0; g < FB * FB / 128; g += 16) {  // 16 loads in flight, then their stores
+    double v[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const int e = t + 128 * (g + u);
+      v[u] = A[(int64_t)(k0 + e / FB) * n + k0 + e % FB];
+    }
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const int e = t + 128 * (g + u);
+      Lk[e / FB][e % FB] = v[u];
+    }
+  }
+#pragma unroll
+  for (int i0 = 0; i0 < FB; i0 += 16) {
+    double v[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) v[u] = ok ? Y[(int64_t)(k0 + i0 + u) * r + c0 + t] : 0.0;
+#pragma unroll
+    for (int u = 0; u < 16; ++u) Ys[i0 + u][t] = v[u];
+  }
   __syncthreads();
   if (FWD) {
     for (int i = 0; i < FB; ++i) {
