@@ -157,7 +157,12 @@ static int run_gemm2(const CUtensorMap &a0, const CUtensorMap &a1, const CUtenso
   auto kern = gemm2_kernel<Epi, STAGES, MAX_SLABS, EPI_WARPS, BN_MAX>;
   CK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   if (prob.m_tiles % 2 || prob.bn % 16 || prob.bn > BN_MAX) return fail(DCKV_EINVAL, "bad CTA-pair GEMM shape");
-  const int tiles = (prob.m_tiles / 2) * prob.n_tiles;
+  int tiles = (prob.m_tiles / 2) * prob.n_tiles;
+  if (prob.k_split > 1) {  // one segment, every part non-empty
+    const int per = prob.n_seg == 1 ? (prob.seg[0].k_steps + prob.k_split - 1) / prob.k_split : 0;
+    if (prob.n_seg != 1 || per * (prob.k_split - 1) >= prob.seg[0].k_steps) return fail(DCKV_EINVAL, "bad split-K");
+    tiles *= prob.k_split;
+  }
   if (tiles <= 0) return DCKV_OK;
   for (int i = 0; i < prob.n_seg; ++i)
     if (prob.seg[i].n_slab < 1 || prob.seg[i].n_slab > MAX_SLABS) return fail(DCKV_EINVAL, "bad slab count");
@@ -210,6 +215,24 @@ static void add_seg(GemmProblem &p, int a_map, int a_slab0, int n_slab, int a_k0
   s.b_row_shift = b_row_shift;
   s.b_k0 = b_k0;
   s.k_steps = k_steps;
+}
+
+// Hidden layer from split-K parts: h = (sum of the parts, in part order) * 2^-p - offset[m],
+// g = GELU(h) (erf form), G[row][m] = fp16(g), G[row][256 + m] = fp16(g - fp16(g)).
+__global__ void __launch_bounds__(256) k_gelu_parts(const float *part, int n_part, int64_t n_rows, const float *offset,
+                                                    float scale, __half *g) {
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= n_rows * N_HIDDEN) return;
+  const int m = (int)(e % N_HIDDEN);
+  float acc = part[e];
+  for (int k = 1; k < n_part; ++k) acc += part[(int64_t)k * n_rows * N_HIDDEN + e];
+  const float h = acc * scale - offset[m];
+  const float v = 0.5f * h * (1.0f + erff(h * 0.70710678118654752f));
+  const __half hi = __float2half_rn(v);
+  const __half lo = __float2half_rn(v - __half2float(hi));
+  __half *row = g + (e / N_HIDDEN) * (2 * N_HIDDEN);
+  row[m] = hi;
+  row[N_HIDDEN + m] = lo;
 }
 
 // ============================================================================ setup kernels
@@ -841,6 +864,7 @@ static WsPlan plan_ws(const Layout &L, int which /*0 encode, 1 decode*/) {
   if (which == 0) {
     w.x16 = take(2ull * L.n_rows * ROW_DIM);
     w.g16 = take(2ull * L.n_rows * 2 * N_HIDDEN);
+    w.hpart = take(4ull * HIDDEN_SPLIT * L.n_rows * N_HIDDEN);
     w.q32 = take(4ull * L.n_rows * N_COEF);
     w.sym16 = take(2ull * L.n_symbols);
     w.cf32 = take(8ull * L.n_symbols);
@@ -1301,16 +1325,20 @@ static int encode_impl(const dckv_codec *c, const void *rows, const int32_t *tok
   stage_mark(c, st, "layout+convert");
   if (L.n_rows > 0) {
     CUtensorMap mb_xh, mb_xt, mb_gt, mb_qe;
-    RET(map_b(&mb_xh, x16, false, ROW_DIM, L.n_rows, HIDDEN_BN / 2));
+    RET(map_b(&mb_xh, x16, false, ROW_DIM, L.n_rows, HIDDEN_SPLIT_BN / 2));
     RET(map_b(&mb_xt, x16, false, ROW_DIM, L.n_rows, TRANSFORM_BN / 2));
     RET(map_b(&mb_gt, g16, false, 2 * N_HIDDEN, L.n_rows, TRANSFORM_BN / 2));
     RET(map_b(&mb_qe, qe, true, N_COEF, L.ne_pad, MEAN_ODD_BN / 2));
     // correction hidden layer: h = x @ w1 - mu @ w1, GELU, fp16 hi/lo
     if (c->has_mlp) {
-      GemmProblem pr = make_problem(N_HIDDEN / GEMM_BM, L.n_rows, HIDDEN_BN, false, status_dev);
+      GemmProblem pr = make_problem(N_HIDDEN / GEMM_BM, L.n_rows, HIDDEN_SPLIT_BN, false, status_dev);
       add_seg(pr, 0, 0, 2, 0, 0, 0, 0, ROW_DIM / GEMM_BK);
-      EpiGelu::Params ep{c->muw1, (float)std::ldexp(1.0, -c->p_h), g16};
-      RET((run_gemm2<EpiGelu, 4, 2, 4, HIDDEN_BN>(c->map_ah2, c->map_ah2, mb_xh, mb_xh, pr, ep, c->num_sms, false, st)));
+      pr.k_split = HIDDEN_SPLIT;
+      float *hpart = (float *)(ws + w.hpart);
+      EpiPartF32::Params ep{hpart, N_HIDDEN, (int64_t)L.n_rows * N_HIDDEN};
+      RET((run_gemm2<EpiPartF32, 4, 2, 8>(c->map_ah2, c->map_ah2, mb_xh, mb_xh, pr, ep, c->num_sms, false, st)));
+      { k_gelu_parts<<<(unsigned)((L.n_rows * N_HIDDEN + 255) / 256), 256, 0, st>>>(
+            hpart, HIDDEN_SPLIT, L.n_rows, c->muw1, (float)std::ldexp(1.0, -c->p_h), g16); ++g_launches; }
     }
     stage_mark(c, st, "gemm_hidden");
     // transform + quantiser: y = x @ B + g @ w2 - mu @ B

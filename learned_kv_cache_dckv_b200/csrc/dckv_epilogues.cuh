@@ -75,6 +75,30 @@ struct EpiAccF64 {
   }
 };
 
+// ------------------------------------------------------------------ split-K part
+// part[ks][n][m] = D[m][n] (fp32): one K part of a split-K product, summed afterwards in a
+// fixed order by the consumer.  Lanes hold consecutive m, so the store is coalesced.
+struct EpiPartF32 {
+  struct Params {
+    float *part;
+    int64_t ld;         // M
+    int64_t ks_stride;  // rows * M
+  };
+  static constexpr int SMEM_BYTES = 0;
+  __device__ __forceinline__ static void tile(const Params &p, const EpiCtx &cx) {
+    const int m = cx.mt * GEMM_BM + cx.ew * 32 + cx.lane;
+    float *o = p.part + cx.ks * p.ks_stride + (int64_t)cx.n0 * p.ld + m;
+    for (int c0 = cx.grp * 32; c0 < cx.n_valid; c0 += 32 * cx.n_grp) {
+      uint32_t r[32];
+      tmem_ld_32x32b_x32(cx.tacc + (uint32_t)c0, r);
+      tmem_ld_wait();
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (c0 + j < cx.n_valid) o[(int64_t)(c0 + j) * p.ld] = u2f(r[j]);
+    }
+  }
+};
+
 // ------------------------------------------------------------------ correction layer 1
 // h = D * 2^-p_h - (mu @ w1)[m];  g = GELU(h) (erf form);  G[row][m] = fp16(g),
 // G[row][256 + m] = fp16(g - fp16(g))  (the hi/lo pair feeds the second layer's GEMM)

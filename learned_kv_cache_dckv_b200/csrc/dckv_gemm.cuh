@@ -47,6 +47,8 @@ struct GemmProblem {
   GemmSeg seg[GEMM_MAX_SEG];
   uint32_t idesc;
   int *status;  // device int32; DCKV_ETIMEOUT (5) is written on a timed-out wait
+  int k_split;  // CTA-pair kernel, one segment: K cut into k_split parts, each its own tile
+                // (the epilogue writes part ks of the sum; 0 or 1: no split)
 };
 
 // What an epilogue sees of one output tile.  The epilogue threads form groups of 128 (four
@@ -63,6 +65,7 @@ struct EpiCtx {
   int grp, n_grp;
   int bar;
   char *scratch;
+  int ks = 0;        // split-K part of this tile (CTA-pair kernel with prob.k_split > 1)
 };
 
 template <int MAX_SLABS, int BN_MAX = GEMM_MAX_BN>
@@ -280,7 +283,9 @@ __global__ void __launch_bounds__(64 + 32 * EPI_WARPS, 1)
   const int pair = blockIdx.x >> 1;
   const int n_pairs = gridDim.x >> 1;
   const int m_pairs = prob.m_tiles >> 1;
-  const int total_tiles = m_pairs * prob.n_tiles;
+  const int n_split = prob.k_split > 1 ? prob.k_split : 1;
+  const int mn_tiles = m_pairs * prob.n_tiles;
+  const int total_tiles = mn_tiles * n_split;
   const int half_bn = prob.bn >> 1;
 
   if (threadIdx.x == 0) {
@@ -318,14 +323,17 @@ __global__ void __launch_bounds__(64 + 32 * EPI_WARPS, 1)
       uint32_t phase = 0;
       bool ok = true;
       for (int t = pair; t < total_tiles && ok; t += n_pairs) {
-        const int mp = t % m_pairs;
-        const int n0 = (t / m_pairs) * prob.bn;
+        const int mp = (t % mn_tiles) % m_pairs;
+        const int n0 = ((t % mn_tiles) / m_pairs) * prob.bn;
+        const int part = t / mn_tiles;
         for (int si = 0; si < prob.n_seg && ok; ++si) {
           const GemmSeg sg = prob.seg[si];
           const void *ta = sg.a_map ? (const void *)&tmA1 : (const void *)&tmA0;
           const void *tb = sg.b_map ? (const void *)&tmB1 : (const void *)&tmB0;
           const uint32_t bytes = (uint32_t)(sg.n_slab * GEMM_SLAB_BYTES + half_bn * GEMM_BK * 2);
-          for (int ks = 0; ks < sg.k_steps; ++ks) {
+          const int per = (sg.k_steps + n_split - 1) / n_split;
+          const int k_beg = part * per, k_end = min(sg.k_steps, k_beg + per);
+          for (int ks = k_beg; ks < k_end; ++ks) {
             if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) {
               ok = false;
               break;
@@ -366,9 +374,12 @@ __global__ void __launch_bounds__(64 + 32 * EPI_WARPS, 1)
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * GEMM_MAX_BN);
         uint32_t accumulate = 0;
         bool ok = true;
+        const int part = t / mn_tiles;
         for (int si = 0; si < prob.n_seg && ok; ++si) {
           const GemmSeg sg = prob.seg[si];
-          for (int ks = 0; ks < sg.k_steps; ++ks) {
+          const int per = (sg.k_steps + n_split - 1) / n_split;
+          const int k_beg = part * per, k_end = min(sg.k_steps, k_beg + per);
+          for (int ks = k_beg; ks < k_end; ++ks) {
             if (!mbar_wait(&full_bar[stage], phase, abort_flag)) {
               ok = false;
               break;
@@ -411,12 +422,12 @@ __global__ void __launch_bounds__(64 + 32 * EPI_WARPS, 1)
       named_bar_sync(1 + grp, 128);
       if (*abort_flag) break;
       tc_fence_after();
-      const int mp = t % m_pairs;
-      const int n0 = (t / m_pairs) * prob.bn;
+      const int mp = (t % mn_tiles) % m_pairs;
+      const int n0 = ((t % mn_tiles) / m_pairs) * prob.bn;
       const int n_valid = min(prob.bn, prob.n_rows - n0);
       const uint32_t tacc = tmem_base + ((uint32_t)(ew * 32) << 16) + (uint32_t)(acc * GEMM_MAX_BN);
       const EpiCtx cx{2 * mp + (int)rank, n0, n_valid, prob.bn, tacc, ew, lane, et, grp, N_GRP, 1 + grp,
-                      epi_scratch + grp * EPI_SCRATCH};
+                      epi_scratch + grp * EPI_SCRATCH, t / mn_tiles};
       Epi::tile(ep, cx);
       tc_fence_before();
       __syncwarp();

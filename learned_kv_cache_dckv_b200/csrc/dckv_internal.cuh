@@ -45,9 +45,13 @@ constexpr float REFINE_NORM_FULL = 32.0f;
 constexpr int TRANSFORM_BN = 224;
 constexpr int MEAN_ODD_BN = 224;
 constexpr int INVERSE_BN = 224;
-// correction hidden layer: one 256-row pair tile in M, so narrow token tiles (62 pairs for
-// a 4K-token prompt) spread the GEMM over the GPU
+// Hidden layers (256 rows of M, one pair tile): the decoder's synthesis layer runs narrow
+// 64-token tiles (62 pairs for a 4K-token prompt); the encoder's correction layer, K = 6,144,
+// runs 256-token tiles with K cut into HIDDEN_SPLIT parts (64 pairs), each tile then reading
+// its A slice once per 256 tokens instead of once per 64, and sums the parts afterwards.
 constexpr int HIDDEN_BN = 64;
+constexpr int HIDDEN_SPLIT_BN = 256;
+constexpr int HIDDEN_SPLIT = 4;
 // K steps (of 64) per TMEM partial of the transform before it is added into the fp32
 // totals: bounds the growth of the tensor core's accumulation error over K = 6,144.
 constexpr int TRANSFORM_CHUNK_STEPS = 4;
@@ -90,6 +94,7 @@ struct WsPlan {
   size_t prompts, chunks, row_tok, row_pos, row_edst, e_tok, row_slot, e_slot, slot_chunk;  // tables
   size_t qe, cen8;                                                               // both
   size_t x16, g16, q32, sym16, cf32, words, states, nwords, nesc, offs;           // encode
+  size_t hpart;    // encode: split-K parts of the correction hidden layer, fp32
   size_t slots16;  // decode: decoded symbols (slot order)
   size_t rope;     // decode: float2 [max_len][128] RoPE (cos, sin)
   size_t row_norm, rowflag, el_list, full_list;                         // encode refinement
