@@ -60,9 +60,17 @@ __global__ void __launch_bounds__(256) k_centres_even(int64_t n_rows, const int3
     tok = min(max(tok, 0), vocab - 1);
     const float *te = t_even + (int64_t)tok * N_COEF;
     int8_t *dst = cen8 + (int64_t)row_slot[row] * k_eff;
-    for (int k = threadIdx.x; k < k_eff; k += blockDim.x) {
-      const float mu = te[kept_list[k]];
-      dst[k] = (int8_t)fminf(fmaxf(rintf(mu), -(float)ESC_LIMIT), (float)ESC_LIMIT);
+    constexpr int PER = N_COEF / 256;  // blockDim.x == 256: every load before the stores
+    float mu[PER];
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+      const int k = threadIdx.x + 256 * u;
+      mu[u] = k < k_eff ? __ldg(te + __ldg(kept_list + k)) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+      const int k = threadIdx.x + 256 * u;
+      if (k < k_eff) dst[k] = (int8_t)fminf(fmaxf(rintf(mu[u]), -(float)ESC_LIMIT), (float)ESC_LIMIT);
     }
   }
 }
