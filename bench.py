@@ -411,7 +411,7 @@ def run_gpu(args):
     # DRAM bytes (read + write) per launch from the committed ncu captures of this workload
     # (profiles/*_c2.md); null for other workloads
     traffic = {"enc:gemm_transform": 191.4e6, "dec:gemm_inverse": 158.6e6, "enc:gemm_mean_odd": 41.2e6,
-               "dec:gemm_mean_odd": 41.2e6, "enc:gemm_hidden": 56.5e6, "dec:rans_loop": 1.22e6} if args.config == "c2" else {}
+               "enc:gemm_hidden": 56.5e6, "dec:rans_loop": 1.22e6} if args.config == "c2" else {}
     bf16_peak = float(peaks.get("bf16_tflops", 1590.0))
     sm_mhz = float(peaks.get("sm_max_mhz", 1965.0))
     alu_peak = 148 * 128 * sm_mhz * 1e6 / 1e12  # int32 lanes x clock, Tops/s

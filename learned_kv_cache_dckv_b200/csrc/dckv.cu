@@ -380,8 +380,8 @@ __global__ void k_permute_mu(const float *mu, float *mu_perm) {
 constexpr int LAYOUT_SPLIT = 8;
 
 __global__ void k_layout(const PromptInfo *prompts, int32_t *row_tok, int32_t *row_pos, int32_t *row_edst,
-                         int32_t *row_slot, int32_t *e_tok, int32_t *e_slot, int32_t *slot_chunk, int chunk_rows,
-                         __nv_bfloat16 *qe_zero_pad) {
+                         int32_t *row_slot, int32_t *e_tok, int32_t *e_slot, int32_t *e_row, int32_t *slot_chunk,
+                         int chunk_rows, __nv_bfloat16 *qe_zero_pad) {
   const PromptInfo pi = prompts[blockIdx.x];
   const int t0 = blockIdx.y * blockDim.x + threadIdx.x, ts = gridDim.y * blockDim.x;
   for (int j = t0; j < pi.n_e; j += ts) slot_chunk[pi.slot_e0 + j] = pi.chunk_e0 + j / chunk_rows;
@@ -397,6 +397,7 @@ __global__ void k_layout(const PromptInfo *prompts, int32_t *row_tok, int32_t *r
     const bool odd = e < pi.n_o;
     e_tok[pi.ebase + e] = odd ? (int32_t)(pi.tok_base + HEAD_KEPT + 2 * e + 1) : -1;
     e_slot[pi.ebase + e] = odd ? pi.slot_o0 + e : 0;
+    e_row[pi.ebase + e] = odd ? pi.row_base + 2 * e + 1 : -1;
   }
   if (qe_zero_pad)  // the row after a prompt's last even row is its odd rows' zero right neighbour
     for (int k = t0; k < N_COEF; k += ts)
@@ -857,6 +858,8 @@ static WsPlan plan_ws(const Layout &L, int which /*0 encode, 1 decode*/) {
   w.e_tok = take(4ull * L.ne_pad);
   w.row_slot = take(4ull * L.n_rows);
   w.e_slot = take(4ull * L.ne_pad);
+  w.e_row = take(4ull * L.ne_pad);
+  w.escflag = take(4ull * std::max(L.n_chunks, 1));
   w.slot_chunk = take(4ull * L.n_rows);
   w.qe = take(2ull * L.ne_pad * N_COEF);
   w.cen8 = take(1ull * L.n_symbols);
@@ -1294,6 +1297,7 @@ static int encode_impl(const dckv_codec *c, const void *rows, const int32_t *tok
   ChunkDesc *d_chunks = (ChunkDesc *)(ws + w.chunks);
   int32_t *row_tok = (int32_t *)(ws + w.row_tok), *row_pos = (int32_t *)(ws + w.row_pos);
   int32_t *row_edst = (int32_t *)(ws + w.row_edst), *e_tok = (int32_t *)(ws + w.e_tok);
+  int32_t *e_row = (int32_t *)(ws + w.e_row);
   __half *x16 = (__half *)(ws + w.x16);
   __half *g16 = (__half *)(ws + w.g16);
   int32_t *q32 = (int32_t *)(ws + w.q32);
@@ -1316,7 +1320,7 @@ static int encode_impl(const dckv_codec *c, const void *rows, const int32_t *tok
   if (L.n_rows) CK(cudaMemsetAsync(rowflag, 0, 4ull * L.n_rows, st));
   if (L.n_chunks) CK(cudaMemsetAsync(nesc_w, 0, 4ull * L.n_chunks, st));
   RET(upload_tables(c, L, ws, w, st));
-  { k_layout<<<dim3(L.batch, LAYOUT_SPLIT), 256, 0, st>>>(d_prompts, row_tok, row_pos, row_edst, row_slot, e_tok, e_slot, slot_chunk,
+  { k_layout<<<dim3(L.batch, LAYOUT_SPLIT), 256, 0, st>>>(d_prompts, row_tok, row_pos, row_edst, row_slot, e_tok, e_slot, e_row, slot_chunk,
                                     c->chunk_rows, qe); ++g_launches; }
   if (L.n_tokens > 0)
     { k_convert<<<(unsigned)L.n_tokens, 192, 0, st>>>((const __nv_bfloat16 *)rows, d_prompts, L.batch, x16, bl, blob_cap,
@@ -1373,8 +1377,8 @@ static int encode_impl(const dckv_codec *c, const void *rows, const int32_t *tok
       GemmProblem pr = make_problem(N_COEF / GEMM_BM, L.ne_pad, MEAN_ODD_BN, true, status_dev);
       add_seg(pr, 0, 0, 1, 0, 0, 0, 0, N_COEF / GEMM_BK);
       add_seg(pr, 0, 0, 1, N_COEF, 0, 1, 0, N_COEF / GEMM_BK);
-      EpiMeanOdd::Params ep{c->t_odd, token_ids, e_tok, e_slot, c->kidx, cen8, c->k_eff, c->vocab};
-      RET((run_gemm2<EpiMeanOdd, 6, 1, 8, MEAN_ODD_BN>(c->map_aon1, c->map_aon1, mb_qe, mb_qe, pr, ep, c->num_sms, true, st)));
+      EpiMeanOdd<false>::Params ep{c->t_odd, token_ids, e_tok, e_slot, c->kidx, cen8, c->k_eff, c->vocab};
+      RET((run_gemm2<EpiMeanOdd<false>, 6, 1, 8, MEAN_ODD_BN>(c->map_aon1, c->map_aon1, mb_qe, mb_qe, pr, ep, c->num_sms, true, st)));
     }
     stage_mark(c, st, "gemm_mean_odd");
     // even centres from the vocabulary table, then every symbol, in slot order
@@ -1441,6 +1445,7 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
   ChunkDesc *d_chunks = (ChunkDesc *)(ws + w.chunks);
   int32_t *row_tok = (int32_t *)(ws + w.row_tok), *row_pos = (int32_t *)(ws + w.row_pos);
   int32_t *row_edst = (int32_t *)(ws + w.row_edst), *e_tok = (int32_t *)(ws + w.e_tok);
+  int32_t *e_row = (int32_t *)(ws + w.e_row);
   __nv_bfloat16 *qe = (__nv_bfloat16 *)(ws + w.qe);
   int32_t *row_slot = (int32_t *)(ws + w.row_slot), *e_slot = (int32_t *)(ws + w.e_slot);
   int8_t *cen8 = (int8_t *)(ws + w.cen8);
@@ -1463,7 +1468,8 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
     CK(cudaMemsetAsync(q16, 0, 2ull * L.n_rows * N_COEF, st));
     CK(cudaMemsetAsync(bigflag, 0, 4ull * L.n_rows, st));
   }
-  { k_layout<<<dim3(L.batch, LAYOUT_SPLIT), 256, 0, st>>>(d_prompts, row_tok, row_pos, row_edst, row_slot, e_tok, e_slot, slot_chunk,
+  if (L.n_chunks) CK(cudaMemsetAsync(ws + w.escflag, 0, 4ull * L.n_chunks, st));
+  { k_layout<<<dim3(L.batch, LAYOUT_SPLIT), 256, 0, st>>>(d_prompts, row_tok, row_pos, row_edst, row_slot, e_tok, e_slot, e_row, slot_chunk,
                                     c->chunk_rows, nullptr); ++g_launches; }
   HeaderCheck hc{bl, blob_bytes, d_prompts, L.batch, c->chunk_rows, c->k_eff, L.n_chunks_e, L.n_chunks_o,
                  L.n_kept, L.off_kept, L.off_streams, valid, status_dev};
@@ -1484,8 +1490,10 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
   CK(cudaFuncSetAttribute(rans_decode_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, RANS_DEC_SMEM));
   RansDecArgs da{d_chunks, 0, L.n_chunks, c->k_eff, c->kept_scale, c->dcdf, c->lut, c->tail, bl, L.off_streams,
                  offs, syms16, valid, status_dev};
-  DecCodesArgs fa{d_chunks, d_prompts, 0, L.n_chunks_e, c->k_eff, c->kept_list, cen8, syms16, bl, L.off_streams,
-                  offs, q16, qe, qbig, bigflag, biglist, counters, valid, status_dev};
+  uint32_t *escflag = (uint32_t *)(ws + w.escflag);
+  DecCodesArgs fa{d_chunks, d_prompts, 0, L.n_chunks_e, c->k_eff, c->kept_list, syms16, bl, L.off_streams,
+                  offs, q16, qe, qbig, bigflag, biglist, counters, escflag, valid, status_dev};
+  const unsigned rg = (unsigned)std::max<int64_t>(1, std::min<int64_t>(L.n_rows, 65535));
   if (L.n_chunks > 0) {
     const unsigned g = (L.n_chunks + RANS_WARPS - 1) / RANS_WARPS;
     if (c->k_eff >= 32)
@@ -1495,8 +1503,11 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
   }
   CK(cudaGetLastError());
   stage_mark(c, st, "rans_loop");
-  if (L.n_chunks_e > 0)
-    { k_decode_codes<<<(unsigned)L.n_chunks_e, DEC_CODES_THREADS, 0, st>>>(fa); ++g_launches; }
+  if (L.n_chunks_e > 0) {
+    { k_codes_elem<<<rg, 256, 0, st>>>(0, L.n_rows, row_edst, row_slot, slot_chunk, syms16, cen8, c->kept_list,
+                                       c->k_eff, q16, qe, escflag, valid); ++g_launches; }
+    { k_escape_patch<<<(unsigned)L.n_chunks_e, PATCH_THREADS, 0, st>>>(fa); ++g_launches; }
+  }
   CK(cudaGetLastError());
   stage_mark(c, st, "codes_even");
   if (L.n_rows > 0 && c->has_means) {
@@ -1505,14 +1516,19 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
     GemmProblem pr = make_problem(N_COEF / GEMM_BM, L.ne_pad, MEAN_ODD_BN, true, status_dev);
     add_seg(pr, 0, 0, 1, 0, 0, 0, 0, N_COEF / GEMM_BK);
     add_seg(pr, 0, 0, 1, N_COEF, 0, 1, 0, N_COEF / GEMM_BK);
-    EpiMeanOdd::Params ep{c->t_odd, token_ids, e_tok, e_slot, c->kidx, cen8, c->k_eff, c->vocab};
-    RET((run_gemm2<EpiMeanOdd, 6, 1, 8, MEAN_ODD_BN>(c->map_aon1, c->map_aon1, mb_qe, mb_qe, pr, ep, c->num_sms, true, st)));
+    // odd centres, and with them the odd codes (ESC symbols are left to the patch)
+    EpiMeanOdd<true>::Params ep{c->t_odd, token_ids, e_tok, e_slot, c->kidx, cen8, c->k_eff, c->vocab,
+                                syms16, q16, e_row, slot_chunk, escflag};
+    RET((run_gemm2<EpiMeanOdd<true>, 6, 1, 8, MEAN_ODD_BN>(c->map_aon1, c->map_aon1, mb_qe, mb_qe, pr, ep, c->num_sms, true, st)));
   }
   stage_mark(c, st, "gemm_mean_odd");
   if (L.n_chunks_o > 0) {
+    if (!c->has_means)  // unconditional tables: every odd centre is 0
+      { k_codes_elem<<<rg, 256, 0, st>>>(1, L.n_rows, row_edst, row_slot, slot_chunk, syms16, cen8, c->kept_list,
+                                         c->k_eff, q16, qe, escflag, valid); ++g_launches; }
     fa.chunk0 = L.n_chunks_e;
     fa.n_chunks = L.n_chunks_o;
-    { k_decode_codes<<<(unsigned)L.n_chunks_o, DEC_CODES_THREADS, 0, st>>>(fa); ++g_launches; }
+    { k_escape_patch<<<(unsigned)L.n_chunks_o, PATCH_THREADS, 0, st>>>(fa); ++g_launches; }
     CK(cudaGetLastError());
   }
   stage_mark(c, st, "codes_odd");

@@ -231,6 +231,7 @@ struct EpiQuantRegs {
 // mu = D + (embed @ w_odd[0:2048])[token][c]  (code units);  centre = clamp(round(mu), +-127)
 // Tile columns are padded even rows e; column e is the odd row whose left neighbour is
 // even row e (e_tok[e] = its token's row in the batch, or -1 where there is no odd row).
+template <bool DEC>  // false: the encoder's centres; true: the decoder's odd codes
 struct EpiMeanOdd {
   struct Params {
     const float *t_odd;      // [vocab][2048]
@@ -238,16 +239,25 @@ struct EpiMeanOdd {
     const int32_t *e_tok;    // [ne_pad] token row of the odd row, -1 if none
     const int32_t *e_slot;   // [ne_pad] slot row of that odd row
     const int16_t *kidx;     // [2048] kept index, -1 if dropped
-    int8_t *cen8;            // [slots][k_eff]
+    int8_t *cen8;            // [slots][k_eff]  (encoder: the odd centres)
     int k_eff;
     int vocab;
+    // decoder: the odd codes themselves, code = centre + symbol - 254 (q16 != NULL); an
+    // ESC symbol leaves its code to the escape patch and flags its chunk
+    const uint16_t *syms;    // [slots][k_eff] decoded symbols
+    __half *q16;             // [rows][2048]
+    const int32_t *e_row;    // [ne_pad] natural coded row of that odd row
+    const int32_t *slot_chunk;
+    uint32_t *escflag;       // [chunks]
   };
-  // per tile column: t_odd row offset (or -1) and the slot row (each group stages its own)
+  // per tile column: t_odd row offset (or -1), slot row and natural row (each group its own)
   static constexpr int SMEM_BYTES = 256 * 16;
   __device__ __forceinline__ static void tile(const Params &p, const EpiCtx &cx) {
     int64_t *s_row = reinterpret_cast<int64_t *>(cx.scratch);
     int32_t *s_slot = reinterpret_cast<int32_t *>(cx.scratch + 256 * 8);
+    int32_t *s_nat = reinterpret_cast<int32_t *>(cx.scratch + 256 * 12);
     const int n_valid = cx.n_valid;
+    constexpr bool dec = DEC;
     for (int j = cx.et; j < n_valid; j += 128) {
       const int ti = __ldg(p.e_tok + cx.n0 + j);
       int64_t off = -1;
@@ -257,6 +267,7 @@ struct EpiMeanOdd {
       }
       s_row[j] = off;
       s_slot[j] = __ldg(p.e_slot + cx.n0 + j);
+      if (dec) s_nat[j] = __ldg(p.e_row + cx.n0 + j);
     }
     named_bar_sync(cx.bar, 128);
     const int c = cx.mt * GEMM_BM + cx.ew * 32 + cx.lane;
@@ -265,10 +276,12 @@ struct EpiMeanOdd {
       uint32_t r[32];
       tmem_ld_32x32b_x32(cx.tacc + (uint32_t)c0, r);
       float tv[32];
+      uint16_t sv[DEC ? 32 : 1];
 #pragma unroll
       for (int j = 0; j < 32; ++j) {  // independent loads, issued together
         const int64_t off = (kc >= 0 && c0 + j < n_valid) ? s_row[c0 + j] : -1;
         tv[j] = off >= 0 ? __ldg(p.t_odd + off + c) : 0.f;
+        if constexpr (DEC) sv[j] = off >= 0 ? __ldg(p.syms + (int64_t)s_slot[c0 + j] * p.k_eff + kc) : (uint16_t)0;
       }
       tmem_ld_wait();
       if (kc < 0) continue;
@@ -277,7 +290,13 @@ struct EpiMeanOdd {
         if (c0 + j < n_valid && s_row[c0 + j] >= 0) {
           const float mu = u2f(r[j]) + tv[j];
           const float cen = fminf(fmaxf(rintf(mu), -(float)ESC_LIMIT), (float)ESC_LIMIT);
-          p.cen8[(int64_t)s_slot[c0 + j] * p.k_eff + kc] = (int8_t)cen;
+          if constexpr (!DEC) {
+            p.cen8[(int64_t)s_slot[c0 + j] * p.k_eff + kc] = (int8_t)cen;
+          } else if (sv[j] == ESC_SYM) {
+            p.escflag[__ldg(p.slot_chunk + s_slot[c0 + j])] = 1u;
+          } else {
+            p.q16[(int64_t)s_nat[c0 + j] * N_COEF + c] = __float2half_rn((float)((int)sv[j] - R_MAX + (int)cen));
+          }
         }
       }
     }

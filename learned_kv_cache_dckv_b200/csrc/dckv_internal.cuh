@@ -92,6 +92,8 @@ struct Layout {
 // Workspace carving (byte offsets from the workspace base, each 256-aligned).
 struct WsPlan {
   size_t prompts, chunks, row_tok, row_pos, row_edst, e_tok, row_slot, e_slot, slot_chunk;  // tables
+  size_t e_row;    // natural coded row of the odd row after each padded even row (-1: none)
+  size_t escflag;  // decode: per chunk, 1 if an ESC symbol was seen while writing codes
   size_t qe, cen8;                                                               // both
   size_t x16, g16, q32, sym16, cf32, words, states, nwords, nesc, offs;           // encode
   size_t hpart;    // encode: split-K parts of the correction hidden layer, fp32

@@ -663,20 +663,58 @@ __global__ void __launch_bounds__(RANS_WARPS * 32) rans_decode_kernel(RansDecArg
   if (__any_sync(0xffffffffu, bad) && lane == 0) atomicExch(a.status, DCKV_ECORRUPT);
 }
 
-// Finishing a decoded pass, one block per chunk: code = centre + symbol - 254, or the
-// chunk's next escape value for ESC; codes go to q16 (fp16, exact below 2048), even rows
-// also to qe (bf16, the odd mean model's input), codes of 2048 or more to qbig with the
-// row listed for the exact fix-up.  The chunk's symbols are cut into tiles of 128 in
-// symbol order; a first pass counts each tile's escapes, a scan gives each tile the rank
-// of its first escape (escape values are stored in symbol order), and a second pass
-// writes the codes.  Both passes keep several tiles' loads in flight per warp.
+// Finishing a decoded pass in two steps.  k_codes_elem writes code = centre + symbol - 254
+// for every symbol of the pass's rows, fully parallel (fp16 to q16; even rows also bf16 to
+// qe, the odd mean model's input); an ESC symbol only flags its chunk.  (The odd pass of a
+// codec with mean models gets the same from the odd mean GEMM's epilogue.)  k_escape_patch
+// then visits the chunks that store escape values or hold a flagged ESC, ranks the ESC
+// symbols in symbol order (escape values are stored in that order), writes those codes,
+// lists codes of 2048 or more for the exact fix-up (only escapes reach them: any other code
+// lies within 127 + 254), and checks that every escape value is used exactly once.
+__global__ void __launch_bounds__(256) k_codes_elem(int parity, int64_t n_rows, const int32_t *row_edst,
+                                                    const int32_t *row_slot, const int32_t *slot_chunk,
+                                                    const uint16_t *syms, const int8_t *cen8,
+                                                    const int16_t *kept_list, int k_eff, __half *q16,
+                                                    __nv_bfloat16 *qe, uint32_t *escflag, const int32_t *valid) {
+  if (*valid != 1) return;
+  constexpr int PER = N_COEF / 256;  // blockDim.x == 256
+  for (int64_t r = blockIdx.x; r < n_rows; r += gridDim.x) {
+    const int e = row_edst[r];
+    if ((e >= 0) != (parity == 0)) continue;  // block-uniform
+    const int64_t slot = row_slot[r];
+    const uint16_t *sy = syms + slot * k_eff;
+    const int8_t *ce = cen8 + slot * k_eff;
+    int sv[PER], cv[PER], kl[PER];
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {  // every load before the stores
+      const int k = threadIdx.x + 256 * u;
+      sv[u] = k < k_eff ? (int)__ldg(sy + k) : 0;
+      cv[u] = k < k_eff ? (int)__ldg(ce + k) : 0;
+      kl[u] = k < k_eff ? (int)__ldg(kept_list + k) : 0;
+    }
+    bool esc = false;
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+      const int k = threadIdx.x + 256 * u;
+      if (k >= k_eff) continue;
+      if (sv[u] == ESC_SYM) {
+        esc = true;
+        continue;
+      }
+      const int q = sv[u] - R_MAX + cv[u];
+      q16[r * N_COEF + kl[u]] = __float2half_rn((float)q);
+      if (e >= 0) qe[(int64_t)e * N_COEF + kl[u]] = __float2bfloat16_rn((float)q);
+    }
+    if (__syncthreads_or(esc) && threadIdx.x == 0) escflag[slot_chunk[slot]] = 1u;
+  }
+}
+
 struct DecCodesArgs {
   const ChunkDesc *chunks;
   const PromptInfo *prompts;
   int chunk0, n_chunks;
   int k_eff;
   const int16_t *kept_list;
-  const int8_t *cen8;       // centres (slot order)
   const uint16_t *syms;     // slot order
   const uint8_t *blob;
   uint64_t off_streams;
@@ -687,137 +725,70 @@ struct DecCodesArgs {
   uint32_t *bigflag;
   int32_t *biglist;
   uint32_t *bigcount;
+  const uint32_t *escflag;
   const int32_t *valid;
   int32_t *status;
 };
 
-constexpr int DEC_CODES_THREADS = 512;
-constexpr int DEC_TILE = 128;                         // symbols per tile (4 per lane)
-constexpr int DEC_MAX_TILES = 256 * N_COEF / DEC_TILE;  // 256 rows per chunk at most
-constexpr int DEC_TILE_BATCH = 4;                     // tiles per warp in flight
+constexpr int PATCH_THREADS = 256;
 
-__global__ void __launch_bounds__(DEC_CODES_THREADS) k_decode_codes(DecCodesArgs a) {
-  __shared__ uint32_t s_cnt[DEC_MAX_TILES];  // escapes per tile, then the rank of its first
-  __shared__ int16_t s_kl[N_COEF];
-  __shared__ uint32_t s_total;
+__global__ void __launch_bounds__(PATCH_THREADS) k_escape_patch(DecCodesArgs a) {
+  __shared__ uint32_t s_cnt[PATCH_THREADS / 32];
   if (*a.valid != 1) return;
-  for (int k = threadIdx.x; k < a.k_eff; k += DEC_CODES_THREADS) s_kl[k] = a.kept_list[k];
-  const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
-  constexpr int NW = DEC_CODES_THREADS / 32;
+  const int ci = a.chunk0 + blockIdx.x;
+  if ((int)blockIdx.x >= a.n_chunks) return;
+  const uint8_t *sec = a.blob + a.off_streams + a.offs[ci];
+  const uint32_t ne = reinterpret_cast<const uint32_t *>(sec)[32];
+  if (ne == 0 && a.escflag[ci] == 0) return;  // block-uniform: no escapes here
+  const uint32_t *ev = reinterpret_cast<const uint32_t *>(sec + CHUNK_FIXED_BYTES);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  constexpr int NW = PATCH_THREADS / 32;
   const uint32_t lt_mask = (1u << lane) - 1u;
+  const ChunkDesc cd = a.chunks[ci];
+  const PromptInfo pi = a.prompts[cd.prompt];
   const int K = a.k_eff;
-  for (int cb = blockIdx.x; cb < a.n_chunks; cb += gridDim.x) {
-    const int ci = a.chunk0 + cb;
-    const ChunkDesc cd = a.chunks[ci];
-    const PromptInfo pi = a.prompts[cd.prompt];
-    const uint32_t S = (uint32_t)cd.nrows * (uint32_t)K;
-    const int n_tiles = (int)((S + DEC_TILE - 1) / DEC_TILE);
-    const uint16_t *sy = a.syms + cd.sym_base;
-    const int8_t *ce = a.cen8 + cd.sym_base;
-    const uint8_t *sec = a.blob + a.off_streams + a.offs[ci];
-    const uint32_t ne = reinterpret_cast<const uint32_t *>(sec)[32];
-    const uint32_t *ev = reinterpret_cast<const uint32_t *>(sec + CHUNK_FIXED_BYTES);
-    __syncthreads();  // s_kl loaded; the previous chunk's ranks are no longer read
-    // pass 1: escapes per tile
-    for (int t0 = warp * DEC_TILE_BATCH; t0 < n_tiles; t0 += NW * DEC_TILE_BATCH) {
-      uint16_t v[DEC_TILE_BATCH][4];
-#pragma unroll
-      for (int b = 0; b < DEC_TILE_BATCH; ++b)
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const uint32_t i = (uint32_t)(t0 + b) * DEC_TILE + u * 32 + lane;
-          v[b][u] = i < S ? sy[i] : (uint16_t)0;
-        }
-#pragma unroll
-      for (int b = 0; b < DEC_TILE_BATCH; ++b) {
-        uint32_t n = 0;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) n += __popc(__ballot_sync(0xffffffffu, v[b][u] == ESC_SYM));
-        if (lane == 0 && t0 + b < n_tiles) s_cnt[t0 + b] = n;
-      }
-    }
-    __syncthreads();
-    if (warp == 0) {  // exclusive scan of the tile counts, 32 contiguous runs
-      const int per = (n_tiles + 31) / 32;
-      const int lo = min(n_tiles, lane * per), hi = min(n_tiles, lo + per);
-      uint32_t sum = 0;
-      for (int t = lo; t < hi; ++t) sum += s_cnt[t];
-      uint32_t inc = sum;
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
-        if (lane >= o) inc += y;
-      }
-      uint32_t run = inc - sum;
-      for (int t = lo; t < hi; ++t) {
-        const uint32_t c = s_cnt[t];
-        s_cnt[t] = run;
-        run += c;
-      }
-      if (lane == 31) s_total = inc;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0 && s_total != ne) atomicExch(a.status, DCKV_ECORRUPT);  // every escape value used once
-    // pass 2: codes
-    bool bad = false;
-    const int64_t row0 = (int64_t)pi.row_base + 2 * cd.j0 + cd.parity;
-    for (int t0 = warp * DEC_TILE_BATCH; t0 < n_tiles; t0 += NW * DEC_TILE_BATCH) {
-      uint16_t v[DEC_TILE_BATCH][4];
-      int8_t cv[DEC_TILE_BATCH][4];
-#pragma unroll
-      for (int b = 0; b < DEC_TILE_BATCH; ++b)
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const uint32_t i = (uint32_t)(t0 + b) * DEC_TILE + u * 32 + lane;
-          v[b][u] = i < S ? sy[i] : (uint16_t)0;
-          cv[b][u] = i < S ? ce[i] : (int8_t)0;
-        }
-#pragma unroll
-      for (int b = 0; b < DEC_TILE_BATCH; ++b) {
-        if (t0 + b >= n_tiles) break;  // warp-uniform
-        uint32_t ep = s_cnt[t0 + b];
-        // row and kept component of this lane's first symbol in the tile; later ones by steps of 32
-        const uint32_t i0 = (uint32_t)(t0 + b) * DEC_TILE + lane;
-        uint32_t r = i0 / (uint32_t)K;
-        int kc = (int)(i0 - r * (uint32_t)K);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const uint32_t i = i0 + u * 32;
-          const bool valid = i < S;
-          const bool is_esc = valid && v[b][u] == ESC_SYM;
-          const uint32_t me = __ballot_sync(0xffffffffu, is_esc);
-          if (valid) {
-            int q = (int)v[b][u] - R_MAX + (int)cv[b][u];
-            if (is_esc) {
-              const uint32_t e = ep + __popc(me & lt_mask);
-              if (e < ne) {
-                const int64_t sval = (int64_t)((uint64_t)ev[2 * e] | ((uint64_t)ev[2 * e + 1] << 32));
-                q = (int)max(min(sval, (int64_t)INT32_MAX), (int64_t)INT32_MIN);
-                if (sval >= -ESC_LIMIT && sval <= ESC_LIMIT) bad = true;  // not an escape value
-              } else {
-                bad = true;
-              }
-            }
-            const int comp = s_kl[kc];
-            const int64_t row = row0 + 2 * (int64_t)r;
-            a.q16[row * N_COEF + comp] = __float2half_rn((float)q);
-            if (cd.parity == 0) a.qe[(int64_t)(pi.ebase + cd.j0 + r) * N_COEF + comp] = __float2bfloat16_rn((float)q);
-            if (q >= BIG_CODE || q <= -BIG_CODE) {
-              a.qbig[row * N_COEF + comp] = q;
-              if (atomicExch(&a.bigflag[row], 1u) == 0u) a.biglist[atomicAdd(a.bigcount, 1u)] = (int32_t)row;
-            }
-          }
-          ep += __popc(me);
-          kc += 32;
-          while (kc >= K) {
-            kc -= K;
-            ++r;
-          }
-        }
-      }
-    }
-    if (__any_sync(0xffffffffu, bad) && lane == 0) atomicExch(a.status, DCKV_ECORRUPT);
+  const int64_t S = (int64_t)cd.nrows * K;
+  const uint16_t *sy = a.syms + cd.sym_base;
+  const int64_t per = ((S + NW - 1) / NW + 31) & ~int64_t(31);  // warp w scans [w per, (w+1) per)
+  const int64_t i_beg = warp * per, i_end = min(S, i_beg + per);
+  uint32_t n = 0;
+  for (int64_t i = i_beg + lane; i < i_end; i += 32) n += sy[i] == ESC_SYM;
+  for (int o = 16; o; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
+  if (lane == 0) s_cnt[warp] = n;
+  __syncthreads();
+  uint32_t ep = 0, total = 0;
+  for (int w = 0; w < NW; ++w) {
+    if (w < warp) ep += s_cnt[w];
+    total += s_cnt[w];
   }
+  bool bad = threadIdx.x == 0 && total != ne;  // every escape value used exactly once
+  for (int64_t i0 = i_beg; i0 < i_end; i0 += 32) {
+    const int64_t i = i0 + lane;
+    const bool esc = i < i_end && sy[i] == ESC_SYM;
+    const uint32_t m = __ballot_sync(0xffffffffu, esc);
+    if (esc) {
+      const uint32_t e = ep + __popc(m & lt_mask);
+      int q = 0;
+      if (e < ne) {
+        const int64_t sval = (int64_t)((uint64_t)ev[2 * e] | ((uint64_t)ev[2 * e + 1] << 32));
+        q = (int)max(min(sval, (int64_t)INT32_MAX), (int64_t)INT32_MIN);
+        if (sval >= -ESC_LIMIT && sval <= ESC_LIMIT) bad = true;  // not an escape value
+      } else {
+        bad = true;
+      }
+      const int rl = (int)(i / K);
+      const int comp = a.kept_list[i - (int64_t)rl * K];
+      const int64_t row = (int64_t)pi.row_base + 2 * (cd.j0 + rl) + cd.parity;
+      a.q16[row * N_COEF + comp] = __float2half_rn((float)q);
+      if (cd.parity == 0) a.qe[(int64_t)(pi.ebase + cd.j0 + rl) * N_COEF + comp] = __float2bfloat16_rn((float)q);
+      if (q >= BIG_CODE || q <= -BIG_CODE) {
+        a.qbig[row * N_COEF + comp] = q;
+        if (atomicExch(&a.bigflag[row], 1u) == 0u) a.biglist[atomicAdd(a.bigcount, 1u)] = (int32_t)row;
+      }
+    }
+    ep += __popc(m);
+  }
+  if (__any_sync(0xffffffffu, bad) && lane == 0) atomicExch(a.status, DCKV_ECORRUPT);
 }
 
 }  // namespace dckv
