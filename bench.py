@@ -498,6 +498,20 @@ def run_gpu(args):
     return 0
 
 
+def fit_shard(items, rank, world):
+    """The calibration items (prompt batches or prompts) this rank accumulates."""
+    return list(items)[rank::world]
+
+
+def fit_allreduce(t, dist=None):
+    """Sum a rank's normal-equation or scale sums over all ranks, in place (the sums are
+    linear in the calibration rows, so each rank adds its shard and one all-reduce joins
+    them).  Without a process group the local sums are the total."""
+    if dist is not None and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return t
+
+
 def run_fit(args):
     """Closed-form fit of the conditional models ("Evidence"): 16 calibration prompts of
     4,096 tokens whose rows depend on their token and their neighbours; sums, solve, scale
@@ -507,18 +521,30 @@ def run_fit(args):
     import dckv_synth as S
     import learned_kv_cache_dckv_b200 as D
 
-    torch.cuda.set_device(0)
-    dev = torch.device("cuda", 0)
+    world, rank, local = dist_env()
+    dist = None
+    if world > 1:  # calibration shards over the ranks; one all-reduce joins their sums
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
     src = S.source(0)
     cod = S.codec(src, step_scale=None, target_bytes=220.0)
-    gc = D.Codec(D.upload_params(cod, dev), 0, 0)
+    gc = D.Codec(D.upload_params(cod, dev), dev.index, 0)
     emb = torch.from_numpy(np.ascontiguousarray(cod.embed).view(np.int16)).to(dev)
     n_batch, per, tg, ar, ridge = 4, 4, 0.8, 0.95, 0.1
     batches = [S.structured_batch(src, cod.embed, [4096] * per, [500 + per * i + j for j in range(per)], tg, ar, dev)
-               for i in range(n_batch)]
+               for i in fit_shard(range(n_batch), rank, world)]
     # the scale pass runs on calibration prompts the mean fit did not see
-    scale_batch = S.structured_batch(src, cod.embed, [4096] * per, [700 + j for j in range(per)], tg, ar, dev)
-    offs = batches[0][2]
+    scale_seeds = fit_shard([700 + j for j in range(per)], rank, world)
+    scale_batch = (S.structured_batch(src, cod.embed, [4096] * len(scale_seeds), scale_seeds, tg, ar, dev)
+                   if scale_seeds else None)
+    offs = np.array([0] + [4096 * (j + 1) for j in range(per)], np.int64)
     n_tok = (n_batch + 1) * per * 4096
     ws = torch.empty(D.dckv_fit_workspace_bytes(gc.handle, offs), dtype=torch.uint8, device=dev)
     stats = torch.zeros(D.FIT_STATS_DOUBLES, dtype=torch.float64, device=dev)
@@ -536,6 +562,7 @@ def run_fit(args):
         stats.zero_()
         for x, tok, o in batches:
             D.dckv_fit_accumulate(gc.handle, emb, x, tok, o, stats, st, ws)
+        fit_allreduce(stats, dist)
 
     def solve():
         D.dckv_fit_solve(stats, ridge, w_e, w_o, st, sws)
@@ -544,8 +571,10 @@ def run_fit(args):
 
     def scale_pass(gm):
         acc.zero_()
-        x, tok, o = scale_batch
-        D.dckv_fit_scales_accumulate(gm.handle, x, tok, o, acc, st, ws)
+        if scale_batch is not None:
+            x, tok, o = scale_batch
+            D.dckv_fit_scales_accumulate(gm.handle, x, tok, o, acc, st, ws)
+        fit_allreduce(acc, dist)
         D.dckv_fit_scales_finish(gm.handle, acc, b_fit)
 
     def codec_with(b=None):
@@ -553,7 +582,7 @@ def run_fit(args):
         p["w_even"], p["w_odd"] = we_b.view(torch.bfloat16), wo_b.view(torch.bfloat16)
         if b is not None:
             p["laplace_b"] = b.clone()
-        return D.Codec(p, 0, 0)
+        return D.Codec(p, dev.index, 0)
 
     # warm-up pass (all kernels once)
     sums()
@@ -564,9 +593,12 @@ def run_fit(args):
     if int(st.item()) != D.DCKV_OK:
         raise RuntimeError(f"fit status {D.STATUS_NAMES[int(st.item())]}")
     vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
-    sampler = ClockSampler(vis.split(",")[0] if vis and vis.split(",")[0].strip().isdigit() else "0")
+    phys = vis.split(",")[dev.index] if vis and vis.split(",")[dev.index].strip().isdigit() else str(dev.index)
+    sampler = ClockSampler(phys)
     sampler.start()
     time.sleep(0.5)
+    if dist:
+        dist.barrier()
     t_sum, t_solve, t_scale, t_codec = [], [], [], []
     launches0 = D.dckv_launch_count()
     for _ in range(max(1, args.steps)):
@@ -594,6 +626,13 @@ def run_fit(args):
     clocks = sampler.stop()
     if int(st.item()) != D.DCKV_OK:
         raise RuntimeError(f"fit status {D.STATUS_NAMES[int(st.item())]}")
+    t_sum, t_solve, t_scale = (max_over_ranks([statistics.mean(v)], dist, dev)[0] for v in (t_sum, t_solve, t_scale))
+    if rank != 0:  # rank 0 alone measures stages and held-out bytes and prints
+        for g in (gc, gm):
+            g.close()
+        dist.barrier()
+        dist.destroy_process_group()
+        return 0
     # stage times of one calibration call
     D.dckv_set_timing(gc.handle, True)
     stage = {}
@@ -630,19 +669,18 @@ def run_fit(args):
     peak = float(peaks.get("bf16_tflops", 1590.0))
     achieved = flops / (stage["fit_gram"] * 1e-3) / 1e12
     solve_flops = sum(n ** 3 / 3.0 * 2 + 2 * 2.0 * n * n * 2048 for n in (2048, 6144))
-    ms = statistics.mean(t_sum) + statistics.mean(t_solve) + statistics.mean(t_scale)
+    ms = t_sum + t_solve + t_scale
     line = {
         "metric": "calibration tokens/s, closed-form fit of the conditional models (sums + solve + scales)",
-        "value": n_tok / (ms * 1e-3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": 1,
-        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16+f64",
+        "value": n_tok / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": 1,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16+f64",
         "data": "synthetic",
         "config": {"workload": "16 + 4 x 4096-token calibration prompts (means fitted on 16, scales on 4; rows "
                                "depend on their token, g = 0.8, and on their neighbours, AR a = 0.95), ~220 B/token "
                                "codec, ridge 0.1",
                    "calibration_tokens": n_tok, "l2": "inputs far above L2 (805 MB of rows)"},
-        "sums_ms": statistics.mean(t_sum), "solve_ms": statistics.mean(t_solve),
-        "scales_ms": statistics.mean(t_scale), "codec_create_ms": statistics.mean(t_codec),
-        "solve_fp64_tflops": solve_flops / (statistics.mean(t_solve) * 1e-3) / 1e12,
+        "sums_ms": t_sum, "solve_ms": t_solve, "scales_ms": t_scale, "codec_create_ms": statistics.mean(t_codec),
+        "solve_fp64_tflops": solve_flops / (t_solve * 1e-3) / 1e12,
         "stage_ms_per_call": {k: round(v, 4) for k, v in stage.items()},
         "held_out_bytes_per_token": {"trained": pay[0], "scales_only_refit": pay[1], "refit": pay[2],
                                      "refit_vs_trained": pay[2] / pay[0], "refit_vs_scales_only": pay[2] / pay[1]},
@@ -666,6 +704,9 @@ def run_fit(args):
     print(json.dumps(line), flush=True)
     for g in (gc, gm, gr, gs):
         g.close()
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
     return 0
 
 
