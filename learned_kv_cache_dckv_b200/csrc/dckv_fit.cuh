@@ -461,6 +461,8 @@ extern "C" int dckv_fit_accumulate(const dckv_codec *c, const uint16_t *embed, i
                                    int32_t *status_dev, void *workspace, size_t ws_bytes, void *stream) {
   if (!c || !embed || !token_ids || !stats) return fail(DCKV_EINVAL, "a pointer argument is NULL");
   if (vocab < 1) return fail(DCKV_EINVAL, "vocab must be positive");
+  if (((uintptr_t)stats & 7) || ((uintptr_t)embed & 1) || ((uintptr_t)token_ids & 3))
+    return fail(DCKV_EINVAL, "stats must be 8-byte, embed 2-byte and token ids 4-byte aligned");
   Layout L;
   RET(build_layout(c, seq_offsets, batch, L));
   const FitPlan f = plan_fit(L);
@@ -505,6 +507,8 @@ extern "C" int dckv_fit_accumulate(const dckv_codec *c, const uint16_t *embed, i
 extern "C" int dckv_fit_solve(const double *stats, double ridge, double *w_even, double *w_odd, int32_t *status_dev,
                               void *workspace, size_t ws_bytes, void *stream) {
   if (!stats || !w_even || !w_odd || !status_dev || !workspace) return fail(DCKV_EINVAL, "a pointer argument is NULL");
+  if (((uintptr_t)stats | (uintptr_t)w_even | (uintptr_t)w_odd | (uintptr_t)workspace) & 7)
+    return fail(DCKV_EINVAL, "fp64 buffers must be 8-byte aligned");
   if (!(ridge > 0.0) || !std::isfinite(ridge)) return fail(DCKV_EINVAL, "ridge must be positive and finite");
   if (ws_bytes < dckv_fit_solve_workspace_bytes()) return fail(DCKV_ECAPACITY, "solve workspace too small");
   cudaStream_t st = (cudaStream_t)stream;
@@ -523,7 +527,7 @@ extern "C" int dckv_fit_solve(const double *stats, double ridge, double *w_even,
 }
 
 extern "C" int dckv_fit_to_bf16(const double *w, int64_t count, uint16_t *out, void *stream) {
-  if (!w || !out || count < 0) return fail(DCKV_EINVAL, "bad arguments");
+  if (!w || !out || count < 0 || ((uintptr_t)w & 7) || ((uintptr_t)out & 1)) return fail(DCKV_EINVAL, "bad arguments");
   if (count == 0) return DCKV_OK;
   cudaStream_t st = (cudaStream_t)stream;
   { k_fit_bf16<<<(unsigned)std::min<int64_t>((count + 255) / 256, 4096), 256, 0, st>>>(w, count, out); ++g_launches; }
@@ -535,6 +539,7 @@ extern "C" int dckv_fit_scales_accumulate(const dckv_codec *c, const void *rows,
                                           const int64_t *seq_offsets, int batch, int64_t *abs_sum,
                                           int32_t *status_dev, void *workspace, size_t ws_bytes, void *stream) {
   if (!c || !abs_sum) return fail(DCKV_EINVAL, "a pointer argument is NULL");
+  if ((uintptr_t)abs_sum & 7) return fail(DCKV_EINVAL, "abs_sum must be 8-byte aligned");
   Layout L;
   RET(build_layout(c, seq_offsets, batch, L));
   const WsPlan w = plan_ws(L, 0);
@@ -552,6 +557,7 @@ extern "C" int dckv_fit_scales_accumulate(const dckv_codec *c, const void *rows,
 
 extern "C" int dckv_fit_scales_finish(const dckv_codec *c, const int64_t *abs_sum, float *laplace_b, void *stream) {
   if (!c || !abs_sum || !laplace_b) return fail(DCKV_EINVAL, "a pointer argument is NULL");
+  if (((uintptr_t)abs_sum & 7) || ((uintptr_t)laplace_b & 3)) return fail(DCKV_EINVAL, "misaligned buffer");
   cudaStream_t st = (cudaStream_t)stream;
   { k_fit_scales_finish<<<(N_COEF + 255) / 256, 256, 0, st>>>(abs_sum, c->lapb, c->delta, c->keep, laplace_b); ++g_launches; }
   CK(cudaGetLastError());

@@ -70,3 +70,32 @@ def test_host_argument_errors_need_no_gpu(lib):
     assert r == D.DCKV_EINVAL
     assert L.dckv_workspace_bytes(None, offs.ctypes.data_as(ctypes.c_void_p), 1) == 0
     assert "NULL" in D.last_error() or D.last_error() == ""
+
+
+def test_fit_host_argument_errors_need_no_gpu(lib):
+    L = D.lib()
+    offs = np.array([0, 300], np.int64)
+    po = offs.ctypes.data_as(ctypes.c_void_p)
+    fake = ctypes.c_void_p(0x1000)  # never dereferenced: every call below fails its host checks first
+    assert L.dckv_fit_workspace_bytes(None, po, 1) == 0
+    assert L.dckv_fit_accumulate(None, fake, 8, fake, fake, po, 1, fake, fake, fake, 1 << 30, None) == D.DCKV_EINVAL
+    assert L.dckv_fit_solve_workspace_bytes() == 8 * 6144 * 6144
+    assert L.dckv_fit_solve(None, 1e-3, fake, fake, fake, fake, 1 << 30, None) == D.DCKV_EINVAL
+    assert L.dckv_fit_solve(fake, 0.0, fake, fake, fake, fake, 1 << 30, None) == D.DCKV_EINVAL
+    assert "ridge" in D.last_error()
+    assert L.dckv_fit_solve(fake, float("nan"), fake, fake, fake, fake, 1 << 30, None) == D.DCKV_EINVAL
+    assert L.dckv_fit_solve(fake, 1e-3, fake, fake, fake, fake, 1024, None) == D.DCKV_ECAPACITY
+    assert L.dckv_fit_to_bf16(None, 4, fake, None) == D.DCKV_EINVAL
+    assert L.dckv_fit_to_bf16(fake, -1, fake, None) == D.DCKV_EINVAL
+    assert L.dckv_fit_to_bf16(fake, 0, fake, None) == D.DCKV_OK  # nothing to convert, no device work
+    assert L.dckv_fit_scales_accumulate(None, fake, fake, po, 1, fake, fake, fake, 1 << 30, None) == D.DCKV_EINVAL
+    assert L.dckv_fit_scales_finish(None, fake, fake, None) == D.DCKV_EINVAL
+
+
+def test_fit_rejects_misaligned_fp64_buffers(lib):
+    L = D.lib()
+    odd = ctypes.c_void_p(0x1004)  # 4-byte but not 8-byte aligned
+    ok = ctypes.c_void_p(0x1000)
+    assert L.dckv_fit_solve(odd, 1e-3, ok, ok, ok, ok, 1 << 30, None) == D.DCKV_EINVAL
+    assert "aligned" in D.last_error()
+    assert L.dckv_fit_to_bf16(odd, 4, ok, None) == D.DCKV_EINVAL
