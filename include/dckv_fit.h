@@ -35,6 +35,8 @@
  * are asynchronous on `stream` (a cudaStream_t, NULL = legacy default stream) and
  * return DCKV_OK or a host-detected error (dckv.h); device-detected errors go to the
  * int32 status word.  Token ids are clamped to [0, vocab - 1] like the codec does.
+ * Alignment: fp64 and int64 buffers 8 bytes, fp32 and int32 4, bf16 2, workspaces 256
+ * (DCKV_EINVAL otherwise).
  */
 #ifndef DCKV_FIT_H
 #define DCKV_FIT_H
