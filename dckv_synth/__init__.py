@@ -28,11 +28,15 @@ Synthetic recipe (the pages publish no weights and no data):
             mixing included, correction MLP and Student-t rows ignored): the Laplace
             maximum-likelihood scale of the quantised coefficient, evaluated on the
             source distribution instead of a calibration sample.
-  rate k    chosen by bisection so that a Gaussian-source estimate of the coded
-            payload hits a target in bytes per coded row (about 220 or 110).
+  rate k    for the benchmark's configurations, read from step_scales.json (written by
+            oracle/calibrate_step_scales.py: bisection on the payload the CPU oracle
+            writes for a seeded calibration sample, per target rate, rows per rANS chunk,
+            Student-t share and codec kind; calibrated_codec); otherwise chosen by
+            bisection on a Gaussian-source estimate of the payload (codec(target_bytes=)).
 """
 from __future__ import annotations
 
+import json
 import math
 import os
 from dataclasses import dataclass, field
@@ -392,8 +396,31 @@ def structured_batch(src: Source, embed_bits, lengths, seeds, token_gain: float 
     return torch.cat(xs, 0), torch.cat(ts, 0), offs
 
 
-# Step scales for the configurations, found with codec(target_bytes=...) on seed 0.
-# They are recomputed on demand; the constants only save the bisection.
-def step_scale_for(src: Source, target_bytes: float) -> float:
-    c = codec(src, step_scale=None, target_bytes=target_bytes)
-    return c.step_scale
+_STEP_SCALES = os.path.join(os.path.dirname(os.path.abspath(__file__)), "step_scales.json")
+
+
+def calibrated_step_scale(target_bytes: float, chunk_rows: int, student_t_frac: float = 0.0,
+                          linear: bool = False) -> float:
+    """Step scale k of a configuration from step_scales.json (source seed 0): the value at
+    which the payload the CPU oracle writes for a seeded calibration sample is target_bytes
+    per coded row, at the given rows per rANS chunk, Student-t share and codec kind."""
+    with open(_STEP_SCALES) as f:
+        table = json.load(f)
+    for e in table["entries"]:
+        if (e["target_bytes"] == float(target_bytes) and e["chunk_rows"] == int(chunk_rows)
+                and abs(e["student_t_frac"] - float(student_t_frac)) < 1e-12 and e["linear"] == bool(linear)):
+            return float(e["step_scale"])
+    raise KeyError(f"no calibrated step scale for {target_bytes} B/row, {chunk_rows} rows per chunk, "
+                   f"Student-t {student_t_frac}, linear {linear}")
+
+
+def calibrated_codec(src: Source, target_bytes: float, chunk_rows: int = 16, student_t_frac: float = 0.0,
+                     linear: bool = False, synthesis: bool = False) -> Codec:
+    """The codec of a benchmark configuration: fitted Laplace scales at the calibrated step
+    scale (decoder-side synthesis weights do not change the payload)."""
+    if src.seed != 0:
+        raise ValueError("step scales are calibrated for source seed 0")
+    k = calibrated_step_scale(target_bytes, chunk_rows, student_t_frac, linear)
+    c = codec(src, step_scale=k, linear=linear, synthesis=synthesis)
+    c.note += f", step scale calibrated for {target_bytes:g} B/row"
+    return c

@@ -38,3 +38,32 @@ def test_plain_prompt_rows_are_independent():
     zt = z[:, :64]
     lag1 = float((zt[1:] * zt[:-1]).sum() / (zt * zt).sum())
     assert abs(lag1) < 0.05, lag1
+
+
+def test_calibrated_step_scales_reproduce_their_payload():
+    """The stored step scales are what the calibration script's bisection found: every entry
+    met its target within 1%, and re-running the oracle's encoder at the stored step scale on
+    the calibration sample gives the recorded payload again (checked for the ~220 B/row,
+    16-rows-per-chunk entry of the plain codec)."""
+    import json
+    import os
+
+    from oracle import calibrate_step_scales as C
+
+    with open(os.path.join(os.path.dirname(S.__file__), "step_scales.json")) as f:
+        table = json.load(f)
+    keys = {(e["target_bytes"], e["chunk_rows"], e["student_t_frac"], e["linear"]) for e in table["entries"]}
+    assert keys == set(C.ENTRIES)
+    for e in table["entries"]:
+        assert abs(e["payload_per_row"] / e["target_bytes"] - 1.0) < 0.01, e
+        assert S.calibrated_step_scale(e["target_bytes"], e["chunk_rows"], e["student_t_frac"],
+                                       e["linear"]) == e["step_scale"]
+    src = S.source(0)
+    e = next(e for e in table["entries"] if e["target_bytes"] == 220.0 and e["student_t_frac"] == 0.0
+             and not e["linear"])
+    x, tok, offs = S.batch(src, [C.SAMPLE_LEN] * len(C.SAMPLE_SEEDS), list(C.SAMPLE_SEEDS))
+    xb = x.view(torch.int16).numpy().view(np.uint16)
+    got = C.payload_per_row(src, xb, tok.numpy(), offs, e["step_scale"], e["chunk_rows"], False)
+    assert abs(got - e["payload_per_row"]) < 0.01, (got, e["payload_per_row"])
+    cod = S.calibrated_codec(src, 220.0, 16)
+    assert cod.step_scale == e["step_scale"]
