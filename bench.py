@@ -1,13 +1,16 @@
-"""DCKV codec benchmark on B200: encode + decode throughput of a 4,096-token prompt.
+"""DCKV codec benchmark on B200: encode + decode throughput of the codec hot path.
 
-python bench.py [--gpus N] [--steps K] [--warmup W] [--impl dckv|reference] [--config c2|c1|c3|c3b|c4|c5]
+python bench.py [--gpus N] [--steps K] [--warmup W] [--impl dckv|reference]
+                [--config c5|c1|c2|c3|c3b|c4|c5p|c2lin|c2syn] [--profile] [--fit]
 
 A step is one pass of the whole codec hot path over one batch: encode (transform GEMMs,
 quantiser, mean models, rANS, compaction) then decode (two rANS passes, odd mean model,
 inverse GEMM with RoPE and scatter).  value = prompt tokens per second through that
-round trip, inputs resident in HBM.  Per-stage device times come from CUDA events the
-library records on its launch stream.  Under torchrun each rank codes its own prompt
-(replicas, weak scaling; no data-path collective) and the slowest rank's time is used.
+round trip, inputs resident in HBM.  The default workload is the largest configuration
+that fits one GPU: 64 prompts of 4,096 tokens with 1% Student-t rows at about 220 B per
+coded row.  Per-stage device times come from CUDA events the library records on its
+launch stream.  Under torchrun each rank codes its own batch (replicas, weak scaling; no
+data-path collective) and the slowest rank's time is used.
 """
 from __future__ import annotations
 
@@ -26,21 +29,31 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 CONFIGS = {
-    # name: (prompt lengths, target bytes/token (None = literal small codec), student-t fraction, description)
-    "c1": ([256], None, 0.0, "1 x 256-token prompt (124 coded rows), literal codec b = 0.6 Delta"),
-    "c2": ([4096], 220.0, 0.0, "1 x 4096-token prompt, 6144-dim bf16 rows, step scale for ~220 B/token"),
-    "c3": ([32768], 220.0, 0.0, "1 x 32768-token prompt, ~220 B/token"),
-    "c3b": ([32768], 110.0, 0.0, "1 x 32768-token prompt, ~110 B/token (many components dropped), 32 rows per chunk"),
-    "c4": ([131072], 220.0, 0.0, "1 x 131072-token prompt, ~220 B/token"),
-    "c5": ([4096] * 64, 220.0, 0.01, "64 x 4096-token prompts, 1% Student-t (nu=2) rows, ~220 B/token"),
-    "c2lin": ([4096], 220.0, 0.0, "1 x 4096-token prompt, linear codec (no correction, unconditional "
-                                  "zero-mean tables), step scale for ~220 B/token"),
-    "c2syn": ([4096], 220.0, 0.0, "1 x 4096-token prompt, ~220 B/token, decoder-side synthesis MLP "
-                                  "(2048 -> 256 GELU -> 6144) added to the linear inverse"),
+    # name: (prompt lengths, target bytes per coded row (None = literal small codec), Student-t
+    # fraction, rows per rANS chunk, description).  Step scales for a target come from the
+    # oracle-calibrated table (dckv_synth.calibrated_codec).
+    "c1": ([256], None, 0.0, 16, "1 x 256-token prompt (124 coded rows), literal codec b = 0.6 Delta"),
+    "c2": ([4096], 220.0, 0.0, 16, "1 x 4096-token prompt, 6144-dim bf16 rows, ~220 B/token"),
+    "c3": ([32768], 220.0, 0.0, 16, "1 x 32768-token prompt, ~220 B/token"),
+    "c3b": ([32768], 110.0, 0.0, 32, "1 x 32768-token prompt, ~110 B/token (many components dropped), "
+                                     "32 rows per chunk"),
+    "c4": ([131072], 220.0, 0.0, 16, "1 x 131072-token prompt, ~220 B/token"),
+    "c5": ([4096] * 64, 220.0, 0.01, 16, "64 x 4096-token prompts, 6144-dim bf16 rows, 1% Student-t (nu=2) "
+                                         "rows, ~220 B/token"),
+    "c5p": ([4096] * 8, 220.0, 0.01, 16, "8 x 4096-token prompts, 1% Student-t (nu=2) rows, ~220 B/token "
+                                         "(an eighth of the 64-prompt batch, rows above L2: the profiling case)"),
+    "c2lin": ([4096], 220.0, 0.0, 16, "1 x 4096-token prompt, linear codec (no correction, unconditional "
+                                      "zero-mean tables), ~220 B/token"),
+    "c2syn": ([4096], 220.0, 0.0, 16, "1 x 4096-token prompt, ~220 B/token, decoder-side synthesis MLP "
+                                      "(2048 -> 256 GELU -> 6144) added to the linear inverse"),
 }
+# the workload the benchmark reports by default: the largest configuration that fits one GPU
+DEFAULT_CONFIG = "c5"
 
-# rows per rANS chunk (codec creation); 0 = the library default (16)
-CHUNK_ROWS = {"c3b": 32}
+# DRAM read + write bytes per coded row of the dominant kernels, from the ncu captures of
+# the 4,096-token prompt (3,964 coded rows) in profiles/; a kernel changed after its capture
+# has no entry
+TRAFFIC_PER_CODED_ROW = {}
 
 GEMM_STAGES = {"gemm_hidden", "gemm_transform", "gemm_mean_odd", "gemm_inverse", "gemm_synth_hidden"}
 
@@ -124,25 +137,28 @@ def max_over_ranks(values, dist=None, device="cpu"):
     return t.tolist()
 
 
-def make_inputs(cfg_name, rank, device):
+def make_inputs(cfg_name, rank, device, first_prompt_only=False):
     import dckv_synth as S
 
-    lens, target, st, _ = CONFIGS[cfg_name]
+    lens, target, st, chunk_rows, _ = CONFIGS[cfg_name]
     src = S.source(0)
     linear = cfg_name.endswith("lin")
     synthesis = cfg_name.endswith("syn")
     if target is None:
         cod = S.codec(src, step_scale=1.0, literal_b=True, linear=linear)
     else:
-        cod = S.codec(src, step_scale=None, target_bytes=target, linear=linear, synthesis=synthesis)
+        cod = S.calibrated_codec(src, target, chunk_rows, st, linear=linear, synthesis=synthesis)
     seeds = [1000 * rank + i for i in range(len(lens))]
+    if first_prompt_only:  # the oracle's timed sample lies inside the first prompt
+        lens, seeds = lens[:1], seeds[:1]
     x, tok, offs = S.batch(src, lens, seeds, student_t_frac=st, device=device)
     return src, cod, x, tok, offs
 
 
-def oracle_sample(cod, x_cpu_bits, tok_cpu, n_rows):
-    """Oracle encode + decode of the first n_rows coded rows of the prompt (plus its kept
-    rows), timed on the host cores.  Returns (seconds, tokens processed)."""
+def oracle_sample(cod, x_cpu_bits, tok_cpu, n_rows, chunk_rows=16, aux=None):
+    """Oracle encode + decode of the first n_rows coded rows of the first prompt (plus its
+    kept rows), timed on the host cores.  Returns (seconds, tokens processed); `aux`, if
+    given, receives the oracle's per-prompt intermediates (codes, ratios, means, centres)."""
     import oracle as O
 
     N = min(x_cpu_bits.shape[0], n_rows + 132)
@@ -150,24 +166,54 @@ def oracle_sample(cod, x_cpu_bits, tok_cpu, n_rows):
     ts = tok_cpu[:N]
     offs = np.array([0, N], np.int64)
     t0 = time.perf_counter()
-    blob = O.encode(xs, ts, offs, cod)
+    blob = O.encode(xs, ts, offs, cod, chunk_rows=chunk_rows, aux=aux)
     O.decode(blob, ts, offs, cod)
     return time.perf_counter() - t0, N
 
 
-def model_bytes_per_row(D, gc, x, tok, offs, blob):
-    """Model code length of the encoder's own symbols, bytes per coded row: sum over coded
-    symbols of -log2(freq / 2^16) under each component's table, plus 64 bits per escape
-    (the figure the payload is compared with).  Reads the symbols the last encode left in
-    the workspace and the codec's exported tables."""
+def sample_parity(aux, q_gpu, cen_gpu, keep):
+    """The GPU encoder's codes and centres of the sample's coded rows against the oracle's:
+    half-step flips (|dq| = 1 where the oracle's y / Delta lies within 1e-3 of a half
+    step), codes differing otherwise, and centre mismatches (all but the sample's last odd
+    row, whose right neighbour lies outside the sample)."""
+    P = aux["per_prompt"][0]
+    n = P["q"].shape[0]
+    d = q_gpu[:n].astype(np.int64) - P["q"]
+    bad = d != 0
+    r = P["ratio"][bad]
+    near = np.abs(r - np.floor(r) - 0.5) < 1e-3
+    flips = int(np.sum(bad))
+    outside = int(np.sum(~((np.abs(d[bad]) == 1) & near)))
+    cen_o = np.zeros((n, 2048), np.int64)
+    cen_o[0::2] = P["ce"]
+    cen_o[1::2] = P["co"]
+    mu_o = np.zeros((n, 2048))
+    mu_o[0::2] = P["mu_e"]
+    mu_o[1::2] = P["mu_o"]
+    m = n - 1 if n % 2 == 0 else n
+    cb = cen_o[:m][:, keep] != cen_gpu[:m].astype(np.int64)
+    mu = mu_o[:m][:, keep][cb]
+    c_out = int(np.sum(np.abs(mu - np.floor(mu) - 0.5) >= 1e-4))
+    return {"rows": int(n), "codes": int(n * 2048), "half_step_flips": flips, "flips_outside_rule": outside,
+            "centres": int(m * int(keep.sum())), "centre_mismatches": int(cb.sum()),
+            "centre_mismatches_outside_rule": c_out}
+
+
+def encoder_readout(D, gc, x, tok, offs, blob, n_sample):
+    """Statistics of the encoder's own symbols after one more encode: model code length per
+    coded row (sum over coded symbols of -log2(freq / 2^16) under each component's table,
+    plus 64 bits per escape -- the figure the payload is compared with), escape count, and
+    the codes and centres of the first n_sample coded rows.  Reads the workspace and the
+    codec's exported tables."""
     import torch
 
     gc.encode(x, tok, offs, blob=blob)
     torch.cuda.synchronize()
     v = D.dckv_ws_offsets(gc.handle, offs, 0)
     n, K = v["n_rows"], gc.k_eff
+    out = {"model_bytes_per_row": 0.0, "n_esc": 0, "n_symbols": int(n * K)}
     if n == 0 or K == 0:
-        return 0.0
+        return out
     sym = gc._ws[v["sym16"]: v["sym16"] + 2 * n * K].view(torch.int16).cpu().numpy().view(np.uint16)
     sym = sym.reshape(n, K).astype(np.int64)
     cdf, scale, keep, _ = D.dckv_codec_export(gc.handle)
@@ -175,8 +221,15 @@ def model_bytes_per_row(D, gc, x, tok, offs, blob):
     freq = np.diff(cdf, axis=1)  # [64][510]
     s_k = scale[keep.astype(bool)].astype(np.int64)
     f = freq[s_k[None, :], sym]
-    bits = float(np.sum(16.0 - np.log2(f))) + 64.0 * float(np.sum(sym == 509))
-    return bits / 8.0 / n
+    n_esc = int(np.sum(sym == 509))
+    bits = float(np.sum(16.0 - np.log2(f))) + 64.0 * n_esc
+    m = min(n, n_sample)
+    q32 = gc.workspace_codes(offs, 0, rows=np.arange(m))
+    cen8 = gc._ws[v["cen8"]: v["cen8"] + n * K].view(torch.int8).reshape(n, K)
+    row_slot = gc._ws[v["row_slot"]: v["row_slot"] + 4 * m].view(torch.int32).long()
+    cen = cen8[row_slot].cpu().numpy()
+    out.update(model_bytes_per_row=bits / 8.0 / n, n_esc=n_esc, q32=q32, cen=cen, keep=keep.astype(bool))
+    return out
 
 
 def host_cores():
@@ -193,21 +246,22 @@ def run_reference(args):
         return 0
     import torch
 
-    _, cod, x, tok, offs = make_inputs(args.config, 0, "cpu")
+    _, cod, x, tok, offs = make_inputs(args.config, 0, "cpu", first_prompt_only=True)
     xb = x.view(torch.int16).numpy().view(np.uint16)
     tk = tok.numpy()
     rows = args.reference_rows
+    G = CONFIGS[args.config][3]
     for _ in range(args.warmup if args.warmup < 1 else 1):
-        oracle_sample(cod, xb, tk, min(rows, 32))
+        oracle_sample(cod, xb, tk, min(rows, 32), G)
     times = []
     toks = 0
     for _ in range(args.steps):
-        dt, n = oracle_sample(cod, xb, tk, rows)
+        dt, n = oracle_sample(cod, xb, tk, rows, G)
         times.append(dt)
         toks = n
     mean = statistics.mean(times)
     value = toks / mean
-    lens, _, _, desc = CONFIGS[args.config]
+    lens, _, _, _, desc = CONFIGS[args.config]
     line = {
         "metric": "decode & encode tokens/s (6144-dim rows) at 1 B200; bytes/token; % roofline",
         "impl": "reference", "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
@@ -242,7 +296,7 @@ def run_gpu(args):
     _, cod, x, tok, offs = make_inputs(args.config, rank, dev)
     n_tok = int(offs[-1])
     n_rows = sum(max(0, int(n) - 132) for n in np.diff(offs))
-    gc = D.Codec(D.upload_params(cod, dev), dev.index, CHUNK_ROWS.get(args.config, 0))
+    gc = D.Codec(D.upload_params(cod, dev), dev.index, CONFIGS[args.config][3])
     stream = torch.cuda.current_stream()
     blob = torch.empty(D.dckv_blob_bound(gc.handle, offs), dtype=torch.uint8, device=dev)
     k_out = torch.empty((6, n_tok, 2, 256), dtype=torch.bfloat16, device=dev)
@@ -294,6 +348,12 @@ def run_gpu(args):
     st = int(gc.status.item())
     if st != D.DCKV_OK:
         raise RuntimeError(f"codec status {D.STATUS_NAMES[st]}")
+
+    if args.profile:  # the steps alone (a small footprint for profiler captures): no further passes
+        if rank == 0:
+            print(json.dumps({"profile_run": args.config, "ms_per_step": statistics.mean(step_ms)}), flush=True)
+        gc.close()
+        return 0
 
     # per-stage device times: a separate pass with the library's stage events enabled
     stage_ms = {}
@@ -397,7 +457,7 @@ def run_gpu(args):
     }
     pad = lambda n, t: -(-n // t) * t
     issued_flops = {  # what the tensor pipe executes (split operands, padded tiles)
-        "enc:gemm_hidden": 2.0 * 2 * pad(n_rows, 128) * 6144 * 256,
+        "enc:gemm_hidden": 2.0 * 2 * pad(n_rows, 256) * 6144 * 256,
         "enc:gemm_transform": 2.0 * pad(n_rows, 224) * (2 * 6144 * 2048 + 4 * 256 * 2048),
         "enc:gemm_mean_odd": 2.0 * pad(n_even + len(offs) - 1, 224) * 4096 * 2048,
         "dec:gemm_mean_odd": 2.0 * pad(n_even + len(offs) - 1, 224) * 4096 * 2048,
@@ -408,10 +468,11 @@ def run_gpu(args):
         issued_flops["dec:gemm_synth_hidden"] = 2.0 * 2 * pad(n_rows, 64) * 2048 * 256
         algo_flops["dec:gemm_inverse"] += 2.0 * n_rows * 256 * 6144
         issued_flops["dec:gemm_inverse"] += 2.0 * 4 * pad(n_rows, 224) * 256 * 6144
-    # DRAM bytes (read + write) per launch from the committed ncu captures of this workload
-    # (profiles/*_c2.md); null for other workloads
-    traffic = {"enc:gemm_transform": 191.4e6, "dec:gemm_inverse": 158.6e6, "enc:gemm_mean_odd": 41.2e6,
-               "enc:gemm_hidden": 56.5e6, "dec:rans_loop": 1.22e6} if args.config == "c2" else {}
+    # DRAM bytes (read + write) per launch: the committed ncu captures (profiles/) of the
+    # 4,096-token prompt, per coded row of that capture, times this workload's coded rows
+    # (every such kernel's traffic grows with the rows it codes); kernels changed since
+    # their capture are absent (null)
+    traffic = {k: v * n_rows for k, v in TRAFFIC_PER_CODED_ROW.items()}
     bf16_peak = float(peaks.get("bf16_tflops", 1590.0))
     sm_mhz = float(peaks.get("sm_max_mhz", 1965.0))
     alu_peak = 148 * 128 * sm_mhz * 1e6 / 1e12  # int32 lanes x clock, Tops/s
@@ -444,7 +505,8 @@ def run_gpu(args):
         roofline = tensor_roofline(gemm_dom)
     roofline_gemm = tensor_roofline(gemm_dom)
 
-    model_bpt = model_bytes_per_row(D, gc, x, tok, offs, blob)
+    rd = encoder_readout(D, gc, x, tok, offs, blob, args.reference_rows)
+    model_bpt = rd["model_bytes_per_row"]
     # codes the last encode recomputed exactly (guard band around a half step) and rows
     # recomputed whole
     v = D.dckv_ws_offsets(gc.handle, offs, 0)
@@ -453,8 +515,19 @@ def run_gpu(args):
 
     tokens = n_tok
     value = tokens * ws / (ms_step * 1e-3)
-    lens, target, stf, desc = CONFIGS[args.config]
+    lens, target, stf, G, desc = CONFIGS[args.config]
     payload = size - sum(min(int(n), 132) for n in np.diff(offs)) * 12288
+    # the whole step against the tensor roofline: every GEMM's algorithmic (and issued)
+    # FLOPs of one encode + decode, over the step time, against the burst bf16 peak
+    step_algo = sum(algo_flops.values())
+    step_issued = sum(issued_flops.values())
+    step_roofline = {"bound": "tensor", "algo_tflop_per_step": step_algo / 1e12,
+                     "issued_tflop_per_step": step_issued / 1e12,
+                     "achieved": step_algo / (ms_step * 1e-3) / 1e12, "peak": bf16_peak, "unit": "TFLOP/s",
+                     "frac": step_algo / (ms_step * 1e-3) / 1e12 / bf16_peak,
+                     "issued_frac": step_issued / (ms_step * 1e-3) / 1e12 / bf16_peak,
+                     "hbm_gb_per_step_algorithmic": (n_tok * 12288 * 2 + n_rows * 4096 * 2 + 2 * payload) / 1e9,
+                     "peak_source": f"{peak_kind} dense bf16, burst"}
     line = {
         "metric": "decode & encode tokens/s (6144-dim rows) at 1 B200; bytes/token; % roofline",
         "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
@@ -471,11 +544,16 @@ def run_gpu(args):
         "bytes_per_token": payload / max(n_rows, 1),
         "model_bytes_per_token": model_bpt,
         "exact_recomputation": refined,
+        "escapes": {"count": rd["n_esc"], "rate": rd["n_esc"] / max(1, rd["n_symbols"]),
+                    "of_symbols": rd["n_symbols"]},
+        "components": {"kept": k_eff, "dropped": 2048 - k_eff},
+        "rows_per_chunk": G,
         "bytes_vs_model": payload / max(n_rows, 1) / model_bpt if model_bpt else None,
         "compression_vs_bf16": 12288.0 * n_rows / max(payload, 1),
         "stage_ms": {k: round(v, 5) for k, v in sorted(means.items())},
         "roofline": roofline,
         "roofline_gemm": roofline_gemm,
+        "step_roofline": step_roofline,
         "e2e": {"value": tokens * ws / (ms_e2e * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e, "steps": n_e2e,
                 "pipeline": "two buffer slots, three streams: upload of rows and ids of step i+1 and download "
@@ -486,9 +564,12 @@ def run_gpu(args):
     }
     if rank == 0 and not args.no_cpu_baseline:
         xb = x.cpu().view(torch.int16).numpy().view(np.uint16)
-        dt, ntok = oracle_sample(cod, xb, tok.cpu().numpy(), args.reference_rows)
+        aux = {}
+        dt, ntok = oracle_sample(cod, xb, tok.cpu().numpy(), args.reference_rows, G, aux=aux)
         line["cpu_baseline"] = {"value": ntok / dt, "unit": "tokens/s", "cores": host_cores(), "kind": "oracle",
                                 "sample": f"oracle encode+decode of the first {ntok} tokens ({ntok - 132} coded rows)"}
+        if "q32" in rd:
+            line["oracle_parity_on_sample"] = sample_parity(aux, rd["q32"], rd["cen"], rd["keep"])
     if rank == 0:
         print(json.dumps(line), flush=True)
     gc.close()
@@ -716,9 +797,11 @@ def main():
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="dckv", choices=["dckv", "reference"])
-    ap.add_argument("--config", default="c2", choices=sorted(CONFIGS))
+    ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(CONFIGS))
     ap.add_argument("--reference-rows", type=int, default=1024)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", action="store_true",
+                    help="run the warm-up and timed steps only and print their mean time (for profiler captures)")
     ap.add_argument("--fit", action="store_true",
                     help="time the closed-form fit of the conditional models instead of the codec")
     args = ap.parse_args()

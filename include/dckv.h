@@ -29,8 +29,12 @@
  * give bit-identical blobs and rows, and a decoder computes exactly the predictions
  * its encoder used (the pages' stated requirement for table selection, "Limits").
  *
- * All functions are thread-compatible: one codec may be used from several host
- * threads on different streams, each with its own workspace.
+ * Threads and devices.  dckv_encode and dckv_decode only read the codec, so one codec
+ * may be used from several host threads at once, on different streams, each call with
+ * its own workspace and outputs.  Creating, destroying and reconfiguring a codec
+ * (dckv_set_timing, dckv_debug_ratio) must not overlap other calls on it.  Every entry
+ * point makes the codec's device current while it runs and gives the caller's current
+ * device back before it returns.
  */
 #ifndef DCKV_H_
 #define DCKV_H_

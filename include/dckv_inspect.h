@@ -17,16 +17,19 @@ extern "C" {
 #endif
 
 /* Byte offsets (from the workspace base) of the intermediates of one call shape.
- * which = 0: encode layout, 1: decode layout.  After dckv_encode on a stream:
- *   q32  int32 [n_rows][2048] codes q = round(y / Delta) (0 for dropped components),
- *        rows in prompt order, coded rows only (positions 4 .. N-129 of each prompt);
- *   qe   bf16 [ne_pad][2048] even-row codes, one extra zero row after each prompt;
+ * which = 0: encode layout, 1: decode layout.  Code arrays hold the kept components only,
+ * in ascending component order (column m is the m-th kept component), code_width columns
+ * wide (K_eff rounded up to 64; the columns past K_eff are 0); dropped components have
+ * code 0.  After dckv_encode on a stream:
+ *   q32  int32 [n_rows][code_width] codes q = round(y / Delta), rows in prompt order,
+ *        coded rows only (positions 4 .. N-129 of each prompt);
+ *   qe   bf16 [ne_pad][code_width] even-row codes, one extra zero row after each prompt;
  *   cen8 int8 [n_rows][K_eff] centres in slot order: slot row row_slot[r] of coded row r
  *        (chunk order: every even row of every prompt, then every odd row), kept
  *        components in ascending order;
  *   sym16 uint16 [n_rows][K_eff] symbols in the same order;
  *   row_slot int32 [n_rows].
- * After dckv_decode: q16 fp16 [n_rows][2048] decoded codes (exact below 2048), qe, cen8.
+ * After dckv_decode: q16 fp16 [n_rows][code_width] decoded codes (exact below 2048), qe, cen8.
  * Encode recomputes in fp64 every code whose fp32 ratio y / Delta lies in a guard band
  * around a half-step boundary (whole rows when the row's norm is large). */
 typedef struct {
@@ -36,6 +39,7 @@ typedef struct {
   int64_t n_rows, ne_pad;
   int32_t n_chunks;
   uint64_t total;
+  int32_t code_width;
 } dckv_ws_view;
 
 int dckv_ws_offsets(const dckv_codec *codec, const int64_t *seq_offsets, int batch, int which, dckv_ws_view *out);
@@ -60,9 +64,10 @@ int dckv_codec_info(const dckv_codec *codec, int32_t *chunk_rows, double *model_
  * Pass NULL to stop.  The buffer must cover the largest call's coded rows. */
 int dckv_debug_ratio(dckv_codec *codec, void *ratio_dev);
 
-/* Per-stage device times of the last encode / decode issued with timing enabled.
- * Events are recorded on the call's stream; read after synchronising it.  Returns the
- * number of stages written to ms / names (at most max). */
+/* Per-stage device times of the last encode / decode that the calling host thread issued
+ * on this codec with timing enabled (each thread keeps its own events, so threads do not
+ * share them).  Events are recorded on the call's stream; read after synchronising it.
+ * Returns the number of stages written to ms / names (at most max). */
 int dckv_set_timing(dckv_codec *codec, int enable);
 int dckv_get_timing(const dckv_codec *codec, float *ms, const char **names, int max);
 

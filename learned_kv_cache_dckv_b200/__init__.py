@@ -64,7 +64,7 @@ class ByteReport(ctypes.Structure):
 class WsView(ctypes.Structure):
     _fields_ = [(n, ctypes.c_uint64) for n in ("q32", "qe", "cen8", "row_slot", "sym16", "q16", "x16", "g16", "counters")] + [
         ("n_rows", ctypes.c_int64), ("ne_pad", ctypes.c_int64), ("n_chunks", ctypes.c_int32),
-        ("total", ctypes.c_uint64)]
+        ("total", ctypes.c_uint64), ("code_width", ctypes.c_int32)]
 
 
 def lib():
@@ -385,6 +385,26 @@ class Codec:
         ws = self.workspace(seq_offsets)
         dckv_decode(self.handle, blob, blob_bytes, token_ids, seq_offsets, k_out, v_out, self.status, ws, stream)
         return k_out, v_out
+
+    def workspace_codes(self, seq_offsets, which: int = 0, rows=None):
+        """Codes the last encode (which=0: q32, int32) or decode (which=1: q16, fp16 as float32)
+        left in the workspace, as numpy [rows][2048] by component (the library keeps kept
+        components only, compact; dropped components are 0).  rows: coded-row indices (all
+        if None)."""
+        torch = self.torch
+        v = dckv_ws_offsets(self.handle, seq_offsets, which)
+        n, kw, k = v["n_rows"], v["code_width"], self.k_eff
+        if which == 0:
+            c = self._ws[v["q32"]: v["q32"] + 4 * n * kw].view(torch.int32).reshape(n, kw)
+        else:
+            c = self._ws[v["q16"]: v["q16"] + 2 * n * kw].view(torch.float16).reshape(n, kw).float()
+        if rows is not None:
+            c = c[torch.as_tensor(np.asarray(rows, np.int64), device=c.device)]
+        c = c[:, :k].cpu().numpy()
+        keep = dckv_codec_export(self.handle)[2].astype(bool)
+        out = np.zeros((c.shape[0], 2048), c.dtype)
+        out[:, keep] = c
+        return out
 
     def close(self):
         if self.handle is not None:

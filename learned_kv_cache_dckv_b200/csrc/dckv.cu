@@ -63,6 +63,24 @@ static int fail(int code, const char *fmt, ...) {
 
 extern "C" const char *dckv_last_error(void) { return g_err; }
 
+// Makes a codec's device current for the duration of an entry point and gives the
+// caller's current device back on return.
+struct DeviceScope {
+  int prev = -1;
+  cudaError_t err = cudaSuccess;
+  explicit DeviceScope(int dev) {
+    if (cudaGetDevice(&prev) != cudaSuccess) prev = -1;
+    if (prev != dev) err = cudaSetDevice(dev);
+    if (prev == dev) prev = -1;  // nothing to restore
+  }
+  ~DeviceScope() {
+    if (prev >= 0) cudaSetDevice(prev);
+  }
+};
+#define DEVICE_SCOPE(dev)  \
+  DeviceScope dev_scope_(dev); \
+  CK(dev_scope_.err)
+
 // ============================================================================ tensor maps
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
@@ -285,12 +303,13 @@ __global__ void k_tables(uint16_t *cdf_out) {
 }
 
 // out[c] = sum_r v[r] * mat[r][c] in fp64, one thread per column, sequential in r.
-__global__ void k_vec_mat(const float *v, const float *mat, int rows, int cols, float *out) {
+__global__ void k_vec_mat(const float *v, const float *mat, int rows, int cols, float *out, double *out64) {
   const int c = blockIdx.x * blockDim.x + threadIdx.x;
   if (c >= cols) return;
   double acc = 0.0;
   for (int r = 0; r < rows; ++r) acc += (double)v[r] * (double)mat[(int64_t)r * cols + c];
   out[c] = (float)acc;
+  out64[c] = acc;
 }
 
 // max |mat| (optionally times delta[column]) via integer atomicMax on non-negative floats.
@@ -354,6 +373,97 @@ __global__ void k_split(const float *src, int M, int K, int mode, const float *d
 }
 
 // out[o][k] = src[(k + k_off) * ld + o], o < O, k < K  (bf16 bits)
+// Split operands restricted to the kept components (the GEMMs compute and read kept
+// components only; compact index m is component kept[m], entries past k_eff are zero).
+// Rows: out[s][m][k] = split(src[k][kept[m]] * scale), m < M, src [K][2048] row-major
+// (basis, w2), through a shared-memory tile so that both sides are coalesced.
+__global__ void k_split_kept_rows(const float *src, int K, const int16_t *kept, int k_eff, int M, double scale,
+                                  __half *out) {
+  __shared__ float tile[32][33];
+  const int k0 = blockIdx.x * 32, m0 = blockIdx.y * 32;
+  const int tx = threadIdx.x, ty = threadIdx.y;  // 32 x 8
+  for (int y = ty; y < 32; y += 8) {
+    const int k = k0 + y, m = m0 + tx;
+    tile[y][tx] = (k < K && m < k_eff) ? src[(int64_t)k * N_COEF + kept[m]] : 0.f;
+  }
+  __syncthreads();
+  for (int y = ty; y < 32; y += 8) {
+    const int m = m0 + y, k = k0 + tx;
+    if (m < M && k < K) {
+      const double v = (double)tile[tx][y] * scale;
+      const __half hi = __double2half(v);
+      out[(int64_t)m * K + k] = hi;
+      out[(int64_t)M * K + (int64_t)m * K + k] = __double2half(v - (double)__half2float(hi));
+    }
+  }
+}
+
+// Columns: out[s][r][j] = split(src[row(r)][kept[j]] * delta[kept[j]] * scale) for j < kw,
+// src [R][2048] row-major; row(r) = the inverse GEMM's row order (inv = 1) or r itself.
+// (a_inv: src = basis, R = 6,144.)
+__global__ void k_split_kept_cols(const float *src, int R, bool inv, const int16_t *kept, int k_eff, int kw,
+                                  const float *delta, double scale, __half *out) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (int64_t)R * kw) return;
+  const int r = (int)(i / kw), j = (int)(i % kw);
+  double v = 0.0;
+  if (j < k_eff) {
+    const int c = kept[j];
+    v = (double)src[(int64_t)(inv ? inv_row_to_dim(r) : r) * N_COEF + c] * (double)delta[c] * scale;
+  }
+  const __half hi = __double2half(v);
+  out[i] = hi;
+  out[(int64_t)R * kw + i] = __double2half(v - (double)__half2float(hi));
+}
+
+// a_v1[s][h][j] = split(v1[kept[j]][h] * delta[kept[j]] * scale), v1 [2048][256].
+__global__ void k_split_v1_kept(const float *v1, const int16_t *kept, int k_eff, int kw, const float *delta,
+                                double scale, __half *out) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (int64_t)N_HIDDEN * kw) return;
+  const int h = (int)(i / kw), j = (int)(i % kw);
+  double v = 0.0;
+  if (j < k_eff) {
+    const int c = kept[j];
+    v = (double)v1[(int64_t)c * N_HIDDEN + h] * (double)delta[c] * scale;
+  }
+  const __half hi = __double2half(v);
+  out[i] = hi;
+  out[(int64_t)N_HIDDEN * kw + i] = __double2half(v - (double)__half2float(hi));
+}
+
+// The odd mean model's neighbour blocks, K-major over kept inputs and kept outputs:
+// a_on[m][j] = w_odd[2048 + b * 2048 + kept[j - b kw]][kept[m]] for block b = j / kw (left,
+// right neighbour), zero past k_eff on either side; bf16 bits, tiled through shared memory.
+__global__ void k_gather_on(const uint16_t *w_odd, const int16_t *kept, int k_eff, int kw, int mp, uint16_t *out) {
+  __shared__ uint16_t tile[32][33];
+  const int j0 = blockIdx.x * 32, m0 = blockIdx.y * 32;
+  const int tx = threadIdx.x, ty = threadIdx.y;
+  for (int y = ty; y < 32; y += 8) {
+    const int j = j0 + y, m = m0 + tx;
+    uint16_t v = 0;
+    if (j < 2 * kw && m < k_eff) {
+      const int b = j / kw, jj = j % kw;
+      if (jj < k_eff) v = w_odd[(int64_t)(N_COEF + b * N_COEF + kept[jj]) * N_COEF + kept[m]];
+    }
+    tile[y][tx] = v;
+  }
+  __syncthreads();
+  for (int y = ty; y < 32; y += 8) {
+    const int m = m0 + y, j = j0 + tx;
+    if (m < mp && j < 2 * kw) out[(int64_t)m * (2 * kw) + j] = tile[tx][y];
+  }
+}
+
+// Per-component constants of the kept components in compact order (pads: Delta 1, mean 0).
+__global__ void k_compact_meta(const float *delta, const float *mub, const int16_t *kept, int k_eff, int mp,
+                               float *delta_k, float *mub_k) {
+  const int m = blockIdx.x * blockDim.x + threadIdx.x;
+  if (m >= mp) return;
+  delta_k[m] = m < k_eff ? delta[kept[m]] : 1.f;
+  mub_k[m] = m < k_eff ? mub[kept[m]] : 0.f;
+}
+
 __global__ void k_transpose16(const uint16_t *src, int ld, int k_off, int O, int K, uint16_t *out) {
   __shared__ uint16_t tile[32][33];
   const int k0 = blockIdx.x * 32, o0 = blockIdx.y * 32;
@@ -381,7 +491,7 @@ constexpr int LAYOUT_SPLIT = 8;
 
 __global__ void k_layout(const PromptInfo *prompts, int32_t *row_tok, int32_t *row_pos, int32_t *row_edst,
                          int32_t *row_slot, int32_t *e_tok, int32_t *e_slot, int32_t *e_row, int32_t *slot_chunk,
-                         int chunk_rows, __nv_bfloat16 *qe_zero_pad) {
+                         int chunk_rows, __nv_bfloat16 *qe_zero_pad, int kw) {
   const PromptInfo pi = prompts[blockIdx.x];
   const int t0 = blockIdx.y * blockDim.x + threadIdx.x, ts = gridDim.y * blockDim.x;
   for (int j = t0; j < pi.n_e; j += ts) slot_chunk[pi.slot_e0 + j] = pi.chunk_e0 + j / chunk_rows;
@@ -400,8 +510,8 @@ __global__ void k_layout(const PromptInfo *prompts, int32_t *row_tok, int32_t *r
     e_row[pi.ebase + e] = odd ? pi.row_base + 2 * e + 1 : -1;
   }
   if (qe_zero_pad)  // the row after a prompt's last even row is its odd rows' zero right neighbour
-    for (int k = t0; k < N_COEF; k += ts)
-      qe_zero_pad[(int64_t)(pi.ebase + pi.n_e) * N_COEF + k] = __float2bfloat16_rn(0.f);
+    for (int k = t0; k < kw; k += ts)
+      qe_zero_pad[(int64_t)(pi.ebase + pi.n_e) * kw + k] = __float2bfloat16_rn(0.f);
 }
 
 __device__ __forceinline__ int find_prompt(const PromptInfo *p, int batch, int64_t tok) {
@@ -581,32 +691,35 @@ __global__ void __launch_bounds__(256) k_fixup(const int32_t *biglist, const uin
                                                const float *mu_perm, const double *theta, const int32_t *row_tok,
                                                const int32_t *row_pos, __nv_bfloat16 *k_out, __nv_bfloat16 *v_out,
                                                int64_t n_tokens, const float *v1t32, const float *v2_32,
-                                               const float *delta) {
+                                               const float *delta, const int16_t *kept_list, int k_eff, int kw) {
   __shared__ float qs[N_COEF];
   __shared__ float xs[ROW_DIM];
   __shared__ float gs[N_HIDDEN];
   const uint32_t n = *bigcount;
   for (uint32_t li = blockIdx.x; li < n; li += gridDim.x) {
     const int64_t r = biglist[li];
-    for (int c = threadIdx.x; c < N_COEF; c += blockDim.x) {
-      float v = __half2float(q16[r * N_COEF + c]);
-      if (fabsf(v) >= (float)BIG_CODE) v = (float)qbig[r * N_COEF + c];
-      qs[c] = v;
+    for (int m = threadIdx.x; m < kw; m += blockDim.x) {  // codes of the kept components, compact order
+      float v = __half2float(q16[r * kw + m]);
+      if (fabsf(v) >= (float)BIG_CODE) v = (float)qbig[r * kw + m];
+      qs[m] = v;
     }
     __syncthreads();
-    const __half *lo = a_inv + (int64_t)ROW_DIM * N_COEF;
+    const __half *lo = a_inv + (int64_t)ROW_DIM * kw;
     for (int d = threadIdx.x; d < ROW_DIM; d += blockDim.x) {
       const int64_t p = dim_to_inv_row(d);
       float acc = 0.f;
-      for (int c = 0; c < N_COEF; ++c)
-        acc = fmaf(qs[c], __half2float(a_inv[p * N_COEF + c]) + __half2float(lo[p * N_COEF + c]), acc);
+      for (int m = 0; m < k_eff; ++m)
+        acc = fmaf(qs[m], __half2float(a_inv[p * kw + m]) + __half2float(lo[p * kw + m]), acc);
       xs[d] = acc * inv_scale + mu_perm[p];
     }
     if (v1t32) {  // decoder-side synthesis: + GELU((q Delta) V1) V2, fp32
       for (int h = threadIdx.x; h < N_HIDDEN; h += blockDim.x) {
         const float *w = v1t32 + (int64_t)h * N_COEF;
         float acc = 0.f;
-        for (int c = 0; c < N_COEF; ++c) acc = fmaf(qs[c] * delta[c], w[c], acc);
+        for (int m = 0; m < k_eff; ++m) {
+          const int c = kept_list[m];
+          acc = fmaf(qs[m] * delta[c], w[c], acc);
+        }
         gs[h] = 0.5f * acc * (1.0f + erff(acc * 0.70710678118654752f));
       }
       __syncthreads();
@@ -659,107 +772,224 @@ __device__ __forceinline__ double warp_sum(double v) {
   return v;
 }
 
-__device__ __forceinline__ void store_code(int64_t row, int c, double ratio, int32_t *q32, __nv_bfloat16 *qe,
-                                           const int32_t *row_edst) {
+// code of compact component m of a row (code arrays kw wide)
+__device__ __forceinline__ void store_code(int64_t row, int m, double ratio, int32_t *q32, __nv_bfloat16 *qe,
+                                           const int32_t *row_edst, int kw) {
   const double qd = fmin(fmax(rint(ratio), -2147483648.0), 2147483647.0);
   const int q = (int)qd;
-  q32[row * N_COEF + c] = q;
+  q32[row * kw + m] = q;
   const int e = row_edst[row];
-  if (e >= 0) qe[(int64_t)e * N_COEF + c] = __float2bfloat16_rn((float)q);
+  if (e >= 0) qe[(int64_t)e * kw + m] = __float2bfloat16_rn((float)q);
 }
 
-// Exact recomputation of listed codes near a half-step boundary, one block per code:
-// y = (x - mu) . basis[:, c] + g . w2[:, c] in fp64 (x from the caller's bf16 rows, g the
-// correction's hidden units), q = round(y / Delta_c).  Each of the 256 threads sums 24
-// products in eight independent partial sums (all their loads in flight together), then
-// the block adds the partial sums in a fixed order.
+// bf16 bits to fp64, exactly: the sign, exponent and mantissa fields move into place
+// (normal numbers; zero, subnormal and non-finite values take the conversion instruction)
+__device__ __forceinline__ double bf16_bits_to_f64(uint32_t w) {
+  const uint32_t t = w & 0x7FFFu;
+  const uint32_t e = t >> 7;
+  if (e == 0u || e == 0xFFu) return (double)__uint_as_float(w << 16);
+  return __hiloint2double((int)(((w & 0x8000u) << 16) | ((t + 0x1C000u) << 13)), 0);
+}
+
+// x . b over a 6,144-dim row in fp64 by one warp: lane l takes the 8-element groups
+// v = l, l + 32, ... of the bf16 row (16-byte loads, twelve in flight per lane), eight
+// independent partial sums added in a fixed order (the caller reduces across lanes).
+// b sits in shared memory as fp64, element 8 v + j at b[j * 768 + v], so that the lanes of
+// a warp read consecutive words (no bank conflicts).  Products of a bf16 and an fp32 value
+// are exact in fp64.
+constexpr int DOT_GROUPS = ROW_DIM / 8;  // 768
+
+__device__ __forceinline__ double row_dot_smem(const uint4 *xr, const double *b, int lane) {
+  constexpr int R = ROW_DIM / 8 / 32;  // 24 groups per lane
+  constexpr int H = R / 2;
+  double part[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) part[u] = 0.0;
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    uint4 xv[H];
+#pragma unroll
+    for (int r = 0; r < H; ++r) xv[r] = __ldg(xr + (half * H + r) * 32 + lane);
+#pragma unroll
+    for (int r = 0; r < H; ++r) {
+      const double *bb = b + (half * H + r) * 32 + lane;
+      part[0] = fma(bf16_bits_to_f64(xv[r].x & 0xFFFFu), bb[0 * DOT_GROUPS], part[0]);
+      part[1] = fma(bf16_bits_to_f64(xv[r].x >> 16), bb[1 * DOT_GROUPS], part[1]);
+      part[2] = fma(bf16_bits_to_f64(xv[r].y & 0xFFFFu), bb[2 * DOT_GROUPS], part[2]);
+      part[3] = fma(bf16_bits_to_f64(xv[r].y >> 16), bb[3 * DOT_GROUPS], part[3]);
+      part[4] = fma(bf16_bits_to_f64(xv[r].z & 0xFFFFu), bb[4 * DOT_GROUPS], part[4]);
+      part[5] = fma(bf16_bits_to_f64(xv[r].z >> 16), bb[5 * DOT_GROUPS], part[5]);
+      part[6] = fma(bf16_bits_to_f64(xv[r].w & 0xFFFFu), bb[6 * DOT_GROUPS], part[6]);
+      part[7] = fma(bf16_bits_to_f64(xv[r].w >> 16), bb[7 * DOT_GROUPS], part[7]);
+    }
+  }
+  return ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
+}
+
+// x . w over a 6,144-dim row in fp64 by one warp, x (fp64) in shared memory and w fp32 in
+// global memory, lanes strided.
+__device__ __forceinline__ double smem_dot_lane(const double *xs, const float *w, int lane) {
+  double part[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll 4
+  for (int i = lane; i < ROW_DIM; i += 128) {
+    part[0] = fma(xs[i], (double)__ldg(w + i), part[0]);
+    part[1] = fma(xs[i + 32], (double)__ldg(w + i + 32), part[1]);
+    part[2] = fma(xs[i + 64], (double)__ldg(w + i + 64), part[2]);
+    part[3] = fma(xs[i + 96], (double)__ldg(w + i + 96), part[3]);
+  }
+  return (part[0] + part[1]) + (part[2] + part[3]);
+}
+
+// Exact recomputation of codes near a half-step boundary.  The transform's epilogue bins
+// them by component.  A work item is up to eight rows of one component's bin: the block
+// puts basis[:, c] into shared memory as fp64 and each warp takes one row:
+// y = x . basis[:, c] - (mu basis)[c] + g . w2[:, c] in fp64 (x the caller's bf16 row, the
+// mean term fp64-accumulated at codec creation, g the correction's hidden units as their
+// fp16 hi/lo pair), q = round(y / Delta_c).  Items are numbered by a prefix sum over the
+// bins (each block computes it for itself) and spread over the grid, so a crowded bin is
+// shared by many blocks.  Lane partial sums are added by a butterfly in a fixed order, so
+// the result is deterministic.
 constexpr int REFINE_THREADS = 256;
+constexpr int REFINE_ITEM_ROWS = REFINE_THREADS / 32;
+constexpr int REFINE_SMEM = ROW_DIM * 8 + (N_COEF + 1) * 4;
 
 __global__ void __launch_bounds__(REFINE_THREADS) k_refine_codes(
-    const uint32_t *el_list, const uint32_t *counters, int64_t el_cap, const __nv_bfloat16 *rows,
-    const int32_t *row_tok, const float *mu32, const float *bt32, const float *w2t32, const __half *g16,
-    const float *delta, const uint32_t *rowflag, int32_t *q32, __nv_bfloat16 *qe, const int32_t *row_edst) {
-  constexpr int PER = ROW_DIM / REFINE_THREADS;  // 24
-  constexpr int U = 8;
-  static_assert(PER % U == 0, "partial sums");
-  __shared__ double red[REFINE_THREADS / 32];
+    const uint32_t *el_bins, const uint32_t *bin_count, uint32_t bin_cap, const __nv_bfloat16 *rows,
+    const int32_t *row_tok, const double *mub64, const float *bt32, const float *w2t32, const __half *g16,
+    const float *delta, const uint32_t *rowflag, const int16_t *kept_list, int kw, int32_t *q32, __nv_bfloat16 *qe,
+    const int32_t *row_edst) {
+  extern __shared__ __align__(16) double bs[];
+  uint32_t *item0 = reinterpret_cast<uint32_t *>(bs + ROW_DIM);  // [2049] first item of each bin
+  __shared__ uint32_t warp_tot[REFINE_THREADS / 32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int64_t n = min((int64_t)counters[0], el_cap);
-  for (int64_t idx = blockIdx.x; idx < n; idx += gridDim.x) {
-    const uint32_t code = el_list[idx];
-    const int64_t row = code >> 11;
-    const int c = (int)(code & 2047u);
-    if (rowflag[row]) continue;  // recomputed whole by k_refine_rows (block-uniform)
-    const __nv_bfloat16 *xr = rows + (int64_t)row_tok[row] * ROW_DIM;
-    const float *bt = bt32 + (int64_t)c * ROW_DIM;
-    double part[U];
+  // items per bin, exclusive prefix sum: thread t owns bins 8t .. 8t + 7
+  {
+    constexpr int PER = N_COEF / REFINE_THREADS;
+    uint32_t cnt[PER], run = 0;
 #pragma unroll
-    for (int u = 0; u < U; ++u) part[u] = 0.0;
-#pragma unroll
-    for (int r = 0; r < PER / U; ++r) {
-      float xv[U], mv[U], bv[U];
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int i = (r * U + u) * REFINE_THREADS + threadIdx.x;
-        xv[u] = __bfloat162float(xr[i]);
-        mv[u] = __ldg(mu32 + i);
-        bv[u] = __ldg(bt + i);
-      }
-#pragma unroll
-      for (int u = 0; u < U; ++u) part[u] += ((double)xv[u] - (double)mv[u]) * (double)bv[u];
+    for (int u = 0; u < PER; ++u) {
+      const uint32_t n = min(bin_count[threadIdx.x * PER + u], bin_cap);
+      cnt[u] = (n + REFINE_ITEM_ROWS - 1) / REFINE_ITEM_ROWS;
+      run += cnt[u];
     }
-    double acc = 0.0;
+    uint32_t incl = run;
 #pragma unroll
-    for (int u = 0; u < U; ++u) acc += part[u];
-    if (w2t32) {  // the correction (absent in a linear codec): one hidden unit per thread
-      const __half *g = g16 + row * (2 * N_HIDDEN);
-      const int h = threadIdx.x;
-      acc += ((double)__half2float(g[h]) + (double)__half2float(g[N_HIDDEN + h])) * (double)w2t32[c * N_HIDDEN + h];
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
     }
-    acc = warp_sum(acc);
-    if (lane == 0) red[warp] = acc;
+    if (lane == 31) warp_tot[warp] = incl;
     __syncthreads();
-    if (threadIdx.x == 0) {
-      double y = 0.0;
-      for (int w = 0; w < REFINE_THREADS / 32; ++w) y += red[w];
-      store_code(row, c, y / (double)delta[c], q32, qe, row_edst);
+    uint32_t base = incl - run;
+    for (int w = 0; w < warp; ++w) base += warp_tot[w];
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+      item0[threadIdx.x * PER + u] = base;
+      base += cnt[u];
+    }
+    if (threadIdx.x == REFINE_THREADS - 1) item0[N_COEF] = base;
+    __syncthreads();
+  }
+  const uint32_t n_items = item0[N_COEF];
+  for (uint32_t item = blockIdx.x; item < n_items; item += gridDim.x) {
+    int lo = 0, hi = N_COEF;  // the bin holding this item: item0[lo] <= item < item0[lo + 1]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (item0[mid] <= item) lo = mid; else hi = mid;
+    }
+    const int m = lo;               // compact component index of the bin
+    const int c = kept_list[m];     // the component
+    const uint32_t n = min(bin_count[m], bin_cap);
+    const float4 *bt = reinterpret_cast<const float4 *>(bt32 + (int64_t)c * ROW_DIM);
+    for (int i = threadIdx.x; i < ROW_DIM / 4; i += blockDim.x) {  // elements 4 i .. 4 i + 3
+      const float4 v = __ldg(bt + i);
+      double *d = bs + (i & 1) * 4 * DOT_GROUPS + (i >> 1);  // group i / 2, j = 4 (i % 2) + t
+      d[0] = v.x;
+      d[DOT_GROUPS] = v.y;
+      d[2 * DOT_GROUPS] = v.z;
+      d[3 * DOT_GROUPS] = v.w;
+    }
+    __syncthreads();
+    const uint32_t k = (item - item0[m]) * REFINE_ITEM_ROWS + warp;
+    if (k < n) {
+      const int64_t row = el_bins[(int64_t)m * bin_cap + k];
+      if (!rowflag[row]) {  // rows listed for whole-row recomputation are left to k_refine_rows
+        double acc = row_dot_smem(reinterpret_cast<const uint4 *>(rows + (int64_t)row_tok[row] * ROW_DIM), bs, lane);
+        if (w2t32) {  // the correction (absent in a linear codec): eight hidden units per lane
+          const __half *g = g16 + row * (2 * N_HIDDEN);
+          const float *w = w2t32 + (int64_t)c * N_HIDDEN;
+          double h = 0.0;
+#pragma unroll
+          for (int u = 0; u < N_HIDDEN / 32; ++u) {
+            const int j = u * 32 + lane;
+            h += ((double)__half2float(g[j]) + (double)__half2float(g[N_HIDDEN + j])) * (double)w[j];
+          }
+          acc += h;
+        }
+        acc = warp_sum(acc) - mub64[c];
+        if (lane == 0) store_code(row, m, acc / (double)delta[c], q32, qe, row_edst, kw);
+      }
     }
     __syncthreads();
   }
 }
 
-// Whole-row exact recomputation (rows with a large norm), one block per listed row:
-// h = (x - mu) w1, g = GELU(h) (erf), y = (x - mu) basis + g w2, all in fp64.
+// Whole-row exact recomputation (rows with a large norm), in two launches whose work items
+// spread over the grid.  Each block first puts the listed row x (fp64) into shared memory.
+// k_refine_hidden: an item is (row, 8 hidden units), one unit per warp:
+// h = x . w1[:, u] - (mu w1)[u], g = GELU(h) (erf), fp64, into g64[list index][256].
+// k_refine_rows: an item is (row, 8 kept components), one component per warp:
+// y = x . basis[:, c] - (mu basis)[c] + g . w2[:, c], then the code (dropped components stay 0).
+constexpr int REFINE_GROUP = 8;
+
+__device__ __forceinline__ void load_row_f64(double *xs, const __nv_bfloat16 *xr) {
+  const uint16_t *xb = reinterpret_cast<const uint16_t *>(xr);
+  for (int i = threadIdx.x; i < ROW_DIM; i += blockDim.x) xs[i] = bf16_bits_to_f64(xb[i]);
+}
+
+__global__ void __launch_bounds__(256) k_refine_hidden(const uint32_t *full_list, const uint32_t *counters,
+                                                       const __nv_bfloat16 *rows, const int32_t *row_tok,
+                                                       const double *muw1_64, const float *w1t32, double *g64) {
+  extern __shared__ __align__(16) double xs[];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  constexpr uint32_t PER_ROW = N_HIDDEN / REFINE_GROUP;
+  const uint32_t n_items = counters[1] * PER_ROW;
+  for (uint32_t item = blockIdx.x; item < n_items; item += gridDim.x) {
+    const uint32_t li = item / PER_ROW;
+    const int h = (int)(item % PER_ROW) * REFINE_GROUP + warp;
+    load_row_f64(xs, rows + (int64_t)row_tok[full_list[li]] * ROW_DIM);
+    __syncthreads();
+    const double a = warp_sum(smem_dot_lane(xs, w1t32 + (int64_t)h * ROW_DIM, lane)) - muw1_64[h];
+    if (lane == 0) g64[(int64_t)li * N_HIDDEN + h] = 0.5 * a * (1.0 + erf(a * 0.70710678118654752440));
+    __syncthreads();
+  }
+}
+
 __global__ void __launch_bounds__(256) k_refine_rows(const uint32_t *full_list, const uint32_t *counters,
                                                      const __nv_bfloat16 *rows, const int32_t *row_tok,
-                                                     const float *mu32, const float *bt32, const float *w1t32,
-                                                     const float *w2t32, const float *delta, const uint8_t *keep,
-                                                     int32_t *q32, __nv_bfloat16 *qe, const int32_t *row_edst) {
-  extern __shared__ __align__(16) double xc[];  // [6144] then g[256]
-  double *gs = xc + ROW_DIM;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  const uint32_t n = counters[1];
-  for (uint32_t li = blockIdx.x; li < n; li += gridDim.x) {
+                                                     const double *mub64, const float *bt32, const float *w2t32,
+                                                     const double *g64, const float *delta, const int16_t *kept_list,
+                                                     int k_eff, int kw, int32_t *q32, __nv_bfloat16 *qe,
+                                                     const int32_t *row_edst) {
+  extern __shared__ __align__(16) double xs[];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint32_t per_row = (uint32_t)(k_eff + REFINE_GROUP - 1) / REFINE_GROUP;
+  const uint32_t n_items = counters[1] * per_row;
+  for (uint32_t item = blockIdx.x; item < n_items; item += gridDim.x) {
+    const uint32_t li = item / per_row;
     const int64_t row = full_list[li];
-    const __nv_bfloat16 *xr = rows + (int64_t)row_tok[row] * ROW_DIM;
-    for (int i = threadIdx.x; i < ROW_DIM; i += blockDim.x) xc[i] = (double)__bfloat162float(xr[i]) - (double)mu32[i];
+    const int m = (int)(item % per_row) * REFINE_GROUP + warp;
+    load_row_f64(xs, rows + (int64_t)row_tok[row] * ROW_DIM);
     __syncthreads();
-    for (int h = warp; w1t32 && h < N_HIDDEN; h += nw) {
-      const float *w = w1t32 + (int64_t)h * ROW_DIM;
-      double acc = 0.0;
-      for (int i = lane; i < ROW_DIM; i += 32) acc += xc[i] * (double)w[i];
-      acc = warp_sum(acc);
-      if (lane == 0) gs[h] = 0.5 * acc * (1.0 + erf(acc * 0.70710678118654752440));
-    }
-    __syncthreads();
-    for (int c = warp; c < N_COEF; c += nw) {
-      const float *bt = bt32 + (int64_t)c * ROW_DIM;
-      double acc = 0.0;
-      for (int i = lane; i < ROW_DIM; i += 32) acc += xc[i] * (double)bt[i];
-      if (w2t32)
-        for (int h = lane; h < N_HIDDEN; h += 32) acc += gs[h] * (double)w2t32[c * N_HIDDEN + h];
-      acc = warp_sum(acc);
-      if (lane == 0) store_code(row, c, keep[c] ? acc / (double)delta[c] : 0.0, q32, qe, row_edst);
+    if (m < k_eff) {  // warp-uniform
+      const int c = kept_list[m];
+      double acc = smem_dot_lane(xs, bt32 + (int64_t)c * ROW_DIM, lane);
+      if (w2t32) {
+        const double *g = g64 + (int64_t)li * N_HIDDEN;
+        for (int h = lane; h < N_HIDDEN; h += 32) acc = fma(g[h], (double)w2t32[c * N_HIDDEN + h], acc);
+      }
+      acc = warp_sum(acc) - mub64[c];
+      if (lane == 0) store_code(row, m, acc / (double)delta[c], q32, qe, row_edst, kw);
     }
     __syncthreads();
   }
@@ -836,6 +1066,7 @@ static int build_layout(const dckv_codec *c, const int64_t *offs, int batch, Lay
       }
     }
   L.n_symbols = rows * (int64_t)c->k_eff;
+  L.kw = c->kw;
   L.off_kept = align_up(HEADER_BYTES + 4ull * (batch + L.n_chunks + 1), 16);
   L.off_streams = L.off_kept + (uint64_t)kept * ROW_DIM * 2;
   return DCKV_OK;
@@ -861,14 +1092,14 @@ static WsPlan plan_ws(const Layout &L, int which /*0 encode, 1 decode*/) {
   w.e_row = take(4ull * L.ne_pad);
   w.escflag = take(4ull * std::max(L.n_chunks, 1));
   w.slot_chunk = take(4ull * L.n_rows);
-  w.qe = take(2ull * L.ne_pad * N_COEF);
+  w.qe = take(2ull * L.ne_pad * L.kw);
   w.cen8 = take(1ull * L.n_symbols);
   w.counters = take(256);
   if (which == 0) {
     w.x16 = take(2ull * L.n_rows * ROW_DIM);
     w.g16 = take(2ull * L.n_rows * 2 * N_HIDDEN);
     w.hpart = take(4ull * HIDDEN_SPLIT * L.n_rows * N_HIDDEN);
-    w.q32 = take(4ull * L.n_rows * N_COEF);
+    w.q32 = take(4ull * L.n_rows * L.kw);
     w.sym16 = take(2ull * L.n_symbols);
     w.cf32 = take(8ull * L.n_symbols);
     w.words = take(2ull * L.n_symbols);
@@ -878,15 +1109,19 @@ static WsPlan plan_ws(const Layout &L, int which /*0 encode, 1 decode*/) {
     w.offs = take(4ull * (L.n_chunks + 1));
     w.row_norm = take(4ull * L.n_rows);
     w.rowflag = take(4ull * L.n_rows);
-    w.el_cap = 64 * L.n_rows + 4096;
-    w.el_list = take(4ull * w.el_cap);
+    // codes to recompute exactly, binned by component; a code that finds its bin full
+    // sends its whole row to the whole-row recomputation instead
+    w.bin_cap = (uint32_t)std::min<int64_t>(L.n_rows / 32 + 64, (int64_t)1 << 30);
+    w.el_bins = take(4ull * N_COEF * w.bin_cap);
+    w.bin_count = take(4ull * N_COEF);
     w.full_list = take(4ull * L.n_rows);
+    w.g64 = take(8ull * N_HIDDEN * L.n_rows);  // hidden units of rows recomputed whole, by list index
   } else {
     w.slots16 = take(2ull * L.n_symbols);
     w.g16 = take(2ull * L.n_rows * 2 * N_HIDDEN);  // synthesis hidden units (hi/lo)
     w.rope = take(8ull * 128 * std::max<int64_t>(L.max_len, 1));
-    w.q16 = take(2ull * L.n_rows * N_COEF);
-    w.qbig = take(4ull * L.n_rows * N_COEF);
+    w.q16 = take(2ull * L.n_rows * L.kw);
+    w.qbig = take(4ull * L.n_rows * L.kw);
     w.bigflag = take(4ull * L.n_rows);
     w.biglist = take(4ull * L.n_rows);
   }
@@ -894,11 +1129,36 @@ static WsPlan plan_ws(const Layout &L, int which /*0 encode, 1 decode*/) {
   return w;
 }
 
-static void stage_mark(const dckv_codec *cc, cudaStream_t st, const char *name) {
-  dckv_codec *c = const_cast<dckv_codec *>(cc);
-  if (!c->timing || c->n_ev >= 24) return;
-  c->ev_names[c->n_ev] = name;
-  cudaEventRecord(c->ev[c->n_ev++], st);
+// Stage timing (diagnostics): each host thread keeps the events of its own last call on a
+// codec with timing enabled, so concurrent calls from several threads never share them.
+struct StageLog {
+  const dckv_codec *codec = nullptr;
+  int device = -1;
+  int n = 0;
+  const char *names[32];
+  cudaEvent_t ev[32] = {};
+};
+static thread_local StageLog t_stages;
+
+static void stage_begin(const dckv_codec *c) {
+  if (!c->timing) return;
+  StageLog &g = t_stages;
+  if (g.device != c->device) {  // events belong to a device: (re)create them on this one
+    for (auto &e : g.ev)
+      if (e) cudaEventDestroy(e), e = nullptr;
+    for (auto &e : g.ev)
+      if (cudaEventCreate(&e) != cudaSuccess) e = nullptr;
+    g.device = c->device;
+  }
+  g.codec = c;
+  g.n = 0;
+}
+
+static void stage_mark(const dckv_codec *c, cudaStream_t st, const char *name) {
+  StageLog &g = t_stages;
+  if (!c->timing || g.codec != c || g.n >= 32 || !g.ev[g.n]) return;
+  g.names[g.n] = name;
+  cudaEventRecord(g.ev[g.n++], st);
 }
 
 // ============================================================================ codec create
@@ -917,7 +1177,7 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
   if (((uintptr_t)prm->embed | (uintptr_t)prm->w_even | (uintptr_t)prm->w_odd) & 15)
     return fail(DCKV_EINVAL, "bf16 parameters must be 16-byte aligned");
   static_assert(RANS_DEC_SMEM <= 232448, "decoder tables exceed shared memory");
-  CK(cudaSetDevice(device));
+  DEVICE_SCOPE(device);
   cudaDeviceProp prop;
   CK(cudaGetDeviceProperties(&prop, device));
   if (prop.major != 10) return fail(DCKV_EINVAL, "needs an sm_100 device (found sm_%d%d)", prop.major, prop.minor);
@@ -932,7 +1192,6 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
   c->has_means = has_means;
   c->has_synth = has_synth;
   c->p = *prm;
-  for (int i = 0; i < 24; ++i) cudaEventCreate(&c->ev[i]);
 
   auto cleanup = [&](int code) {
     dckv_codec_destroy(c);
@@ -955,6 +1214,8 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
   const uint64_t o_te = take(4ull * V * N_COEF);
   const uint64_t o_to = take(4ull * V * N_COEF);
   const uint64_t o_mub = take(4ull * N_COEF);
+  const uint64_t o_mubk = take(4ull * N_COEF);
+  const uint64_t o_deltak = take(4ull * N_COEF);
   const uint64_t o_muw1 = take(4ull * N_HIDDEN);
   const uint64_t o_mup = take(4ull * ROW_DIM);
   const uint64_t o_delta = take(4ull * N_COEF);
@@ -973,7 +1234,8 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
   const uint64_t o_bt32 = take(4ull * N_COEF * ROW_DIM);
   const uint64_t o_w1t32 = take(4ull * N_HIDDEN * ROW_DIM);
   const uint64_t o_w2t32 = take(4ull * N_COEF * N_HIDDEN);
-  const uint64_t o_mu32 = take(4ull * ROW_DIM);
+  const uint64_t o_mub64 = take(8ull * N_COEF);
+  const uint64_t o_muw164 = take(8ull * N_HIDDEN);
   const uint64_t o_av1 = take(has_synth ? 2ull * 2 * N_HIDDEN * N_COEF : 0);
   const uint64_t o_av2 = take(has_synth ? 2ull * 2 * ROW_DIM * N_HIDDEN : 0);
   const uint64_t o_v1t32 = take(has_synth ? 4ull * N_HIDDEN * N_COEF : 0);
@@ -991,6 +1253,8 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
   c->t_even = (float *)(B + o_te);
   c->t_odd = (float *)(B + o_to);
   c->mub = (float *)(B + o_mub);
+  c->mub_k = (float *)(B + o_mubk);
+  c->delta_k = (float *)(B + o_deltak);
   c->muw1 = (float *)(B + o_muw1);
   c->mu_perm = (float *)(B + o_mup);
   c->delta = (float *)(B + o_delta);
@@ -1009,7 +1273,8 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
   c->bt32 = (float *)(B + o_bt32);
   c->w1t32 = (float *)(B + o_w1t32);
   c->w2t32 = (float *)(B + o_w2t32);
-  c->mu32 = (float *)(B + o_mu32);
+  c->mub64 = (double *)(B + o_mub64);
+  c->muw1_64 = (double *)(B + o_muw164);
   c->a_v1 = (__half *)(B + o_av1);
   c->a_v2 = (__half *)(B + o_av2);
   c->v1t32 = (float *)(B + o_v1t32);
@@ -1086,6 +1351,8 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
       ks.push_back(scale_h[i]);
     }
   c->k_eff = (int)kl.size();
+  c->kw = std::max(64, (c->k_eff + 63) / 64 * 64);
+  c->mp = std::max(256, (c->k_eff + 255) / 256 * 256);
   std::vector<int16_t> kx(N_COEF, -1);
   for (int i = 0; i < c->k_eff; ++i) kx[kl[i]] = (int16_t)i;
   kl.resize(N_COEF, 0);
@@ -1124,48 +1391,54 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
       cudaMemcpy(c->theta, theta_h, sizeof(theta_h), cudaMemcpyHostToDevice) != cudaSuccess)
     return cleanup(fail(DCKV_ECUDA, "setup upload failed"));
   // mean projections in fp64
-  { k_vec_mat<<<(N_COEF + 255) / 256, 256, 0, st>>>(prm->mu, prm->basis, ROW_DIM, N_COEF, c->mub); ++g_launches; }
-  if (has_mlp) { k_vec_mat<<<1, 256, 0, st>>>(prm->mu, prm->w1, ROW_DIM, N_HIDDEN, c->muw1); ++g_launches; }
+  { k_vec_mat<<<(N_COEF + 255) / 256, 256, 0, st>>>(prm->mu, prm->basis, ROW_DIM, N_COEF, c->mub, c->mub64); ++g_launches; }
+  if (has_mlp) { k_vec_mat<<<1, 256, 0, st>>>(prm->mu, prm->w1, ROW_DIM, N_HIDDEN, c->muw1, c->muw1_64); ++g_launches; }
   { k_permute_mu<<<(ROW_DIM + 255) / 256, 256, 0, st>>>(prm->mu, c->mu_perm); ++g_launches; }
-  // split operands (hi/lo fp16, power-of-two scaled)
+  { k_compact_meta<<<(c->mp + 255) / 256, 256, 0, st>>>(prm->delta, c->mub, c->kept_list, c->k_eff, c->mp,
+                                                       c->delta_k, c->mub_k); ++g_launches; }
+  // split operands (hi/lo fp16, power-of-two scaled), kept components only where the
+  // component is an index of the GEMM
   dim3 tb(32, 8);
-  { k_split<<<dim3(ROW_DIM / 32, N_COEF / 32), tb, 0, st>>>(prm->basis, N_COEF, ROW_DIM, 0, nullptr, std::ldexp(1.0, c->p_y), c->a_y); ++g_launches; }
+  { k_split_kept_rows<<<dim3(ROW_DIM / 32, c->mp / 32), tb, 0, st>>>(prm->basis, ROW_DIM, c->kept_list, c->k_eff,
+                                                                      c->mp, std::ldexp(1.0, c->p_y), c->a_y); ++g_launches; }
   if (has_mlp) {
-    { k_split<<<dim3(N_HIDDEN / 32, N_COEF / 32), tb, 0, st>>>(prm->w2, N_COEF, N_HIDDEN, 0, nullptr, std::ldexp(1.0, c->p_y), c->a_w2); ++g_launches; }
+    { k_split_kept_rows<<<dim3(N_HIDDEN / 32, c->mp / 32), tb, 0, st>>>(prm->w2, N_HIDDEN, c->kept_list, c->k_eff,
+                                                                         c->mp, std::ldexp(1.0, c->p_y), c->a_w2); ++g_launches; }
     { k_split<<<dim3(ROW_DIM / 32, N_HIDDEN / 32), tb, 0, st>>>(prm->w1, N_HIDDEN, ROW_DIM, 0, nullptr, std::ldexp(1.0, c->p_h), c->a_h); ++g_launches; }
   }
-  { k_split<<<dim3(N_COEF / 32, ROW_DIM / 32), tb, 0, st>>>(prm->basis, ROW_DIM, N_COEF, 1, prm->delta, std::ldexp(1.0, c->p_inv), c->a_inv); ++g_launches; }
+  { k_split_kept_cols<<<(unsigned)((ROW_DIM * (int64_t)c->kw + 255) / 256), 256, 0, st>>>(
+        prm->basis, ROW_DIM, true, c->kept_list, c->k_eff, c->kw, prm->delta, std::ldexp(1.0, c->p_inv), c->a_inv); ++g_launches; }
   // fp32 copies for the exact refinement
   { k_transpose32<<<dim3(ROW_DIM / 32, N_COEF / 32), tb, 0, st>>>(prm->basis, ROW_DIM, N_COEF, c->bt32); ++g_launches; }
   if (has_mlp) {
     { k_transpose32<<<dim3(ROW_DIM / 32, N_HIDDEN / 32), tb, 0, st>>>(prm->w1, ROW_DIM, N_HIDDEN, c->w1t32); ++g_launches; }
     { k_transpose32<<<dim3(N_HIDDEN / 32, N_COEF / 32), tb, 0, st>>>(prm->w2, N_HIDDEN, N_COEF, c->w2t32); ++g_launches; }
   }
-  cudaMemcpyAsync(c->mu32, prm->mu, 4ull * ROW_DIM, cudaMemcpyDeviceToDevice, st);
   if (has_synth) {
     // a_v1[slab][h][c] = split(Delta_c V1[c][h] 2^p_v1); a_v2[slab][p][h] = split(V2[h][dim(p)] 2^p_inv)
-    { k_split<<<dim3(N_COEF / 32, N_HIDDEN / 32), tb, 0, st>>>(prm->v1, N_HIDDEN, N_COEF, 0, prm->delta, std::ldexp(1.0, c->p_v1), c->a_v1); ++g_launches; }
+    { k_split_v1_kept<<<(unsigned)((N_HIDDEN * (int64_t)c->kw + 255) / 256), 256, 0, st>>>(
+          prm->v1, c->kept_list, c->k_eff, c->kw, prm->delta, std::ldexp(1.0, c->p_v1), c->a_v1); ++g_launches; }
     { k_split<<<dim3(N_HIDDEN / 32, ROW_DIM / 32), tb, 0, st>>>(prm->v2, ROW_DIM, N_HIDDEN, 2, nullptr, std::ldexp(1.0, c->p_inv), c->a_v2); ++g_launches; }
     { k_transpose32<<<dim3(N_COEF / 32, N_HIDDEN / 32), tb, 0, st>>>(prm->v1, N_COEF, N_HIDDEN, c->v1t32); ++g_launches; }
     cudaMemcpyAsync(c->v2_32, prm->v2, 4ull * N_HIDDEN * ROW_DIM, cudaMemcpyDeviceToDevice, st);
   }
   // mean-model weights, K-major
   if (has_means) {
-    { k_transpose16<<<dim3(2 * N_COEF / 32, N_COEF / 32), tb, 0, st>>>(prm->w_odd, N_COEF, N_COEF, N_COEF, 2 * N_COEF,
-                                                                     (uint16_t *)c->a_on); ++g_launches; }
+    { k_gather_on<<<dim3(2 * c->kw / 32, c->mp / 32), tb, 0, st>>>(prm->w_odd, c->kept_list, c->k_eff, c->kw, c->mp,
+                                                                  (uint16_t *)c->a_on); ++g_launches; }
     { k_transpose16<<<dim3(N_COEF / 32, N_COEF / 32), tb, 0, st>>>(prm->w_even, N_COEF, 0, N_COEF, N_COEF, tmp_e); ++g_launches; }
     { k_transpose16<<<dim3(N_COEF / 32, N_COEF / 32), tb, 0, st>>>(prm->w_odd, N_COEF, 0, N_COEF, N_COEF, tmp_oe); ++g_launches; }
   }
   if (cudaGetLastError() != cudaSuccess) return cleanup(fail(DCKV_ECUDA, "setup kernels failed to launch"));
   // tensor maps of the static operands
   int r = DCKV_OK;
-  if ((r = map_a(&c->map_ay2, c->a_y, false, ROW_DIM, N_COEF, 2, 2)) ||
-      (r = map_a(&c->map_aw2_2, c->a_w2, false, N_HIDDEN, N_COEF, 2, 2)) ||
-      (r = map_a(&c->map_aw2_1, c->a_w2, false, N_HIDDEN, N_COEF, 2, 1)) ||
+  if ((r = map_a(&c->map_ay2, c->a_y, false, ROW_DIM, c->mp, 2, 2)) ||
+      (r = map_a(&c->map_aw2_2, c->a_w2, false, N_HIDDEN, c->mp, 2, 2)) ||
+      (r = map_a(&c->map_aw2_1, c->a_w2, false, N_HIDDEN, c->mp, 2, 1)) ||
       (r = map_a(&c->map_ah2, c->a_h, false, ROW_DIM, N_HIDDEN, 2, 2)) ||
-      (r = map_a(&c->map_ainv2, c->a_inv, false, N_COEF, ROW_DIM, 2, 2)) ||
-      (r = map_a(&c->map_aon1, c->a_on, true, 2 * N_COEF, N_COEF, 1, 1)) ||
-      (has_synth && (r = map_a(&c->map_av1, c->a_v1, false, N_COEF, N_HIDDEN, 2, 2))) ||
+      (r = map_a(&c->map_ainv2, c->a_inv, false, c->kw, ROW_DIM, 2, 2)) ||
+      (r = map_a(&c->map_aon1, c->a_on, true, 2 * c->kw, c->mp, 1, 1)) ||
+      (has_synth && (r = map_a(&c->map_av1, c->a_v1, false, c->kw, N_HIDDEN, 2, 2))) ||
       (has_synth && (r = map_a(&c->map_av2, c->a_v2, false, N_HIDDEN, ROW_DIM, 2, 2))))
     return cleanup(r);
   // per-vocabulary mean tables: t_even = embed @ w_even, t_odd = embed @ w_odd[0:2048]
@@ -1193,10 +1466,9 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
 
 extern "C" void dckv_codec_destroy(dckv_codec *c) {
   if (!c) return;
-  cudaSetDevice(c->device);
+  DeviceScope dev_scope(c->device);
   if (c->blk) cudaFree(c->blk);
-  for (int i = 0; i < 24; ++i)
-    if (c->ev[i]) cudaEventDestroy(c->ev[i]);
+  if (t_stages.codec == c) t_stages.codec = nullptr;
   delete c;
 }
 
@@ -1288,9 +1560,8 @@ static int encode_impl(const dckv_codec *c, const void *rows, const int32_t *tok
   const WsPlan w = plan_ws(L, 0);
   if (ws_bytes < w.total) return fail(DCKV_ECAPACITY, "workspace too small (%zu < %zu)", ws_bytes, w.total);
   cudaStream_t st = (cudaStream_t)stream;
-  CK(cudaSetDevice(c->device));
-  dckv_codec *cm = const_cast<dckv_codec *>(c);
-  cm->n_ev = 0;
+  DEVICE_SCOPE(c->device);
+  stage_begin(c);
   uint8_t *ws = (uint8_t *)workspace;
   uint8_t *bl = (uint8_t *)blob;
   PromptInfo *d_prompts = (PromptInfo *)(ws + w.prompts);
@@ -1311,17 +1582,19 @@ static int encode_impl(const dckv_codec *c, const void *rows, const int32_t *tok
 
   float *row_norm = (float *)(ws + w.row_norm);
   uint32_t *rowflag = (uint32_t *)(ws + w.rowflag);
-  uint32_t *el_list = (uint32_t *)(ws + w.el_list), *full_list = (uint32_t *)(ws + w.full_list);
+  uint32_t *el_bins = (uint32_t *)(ws + w.el_bins), *full_list = (uint32_t *)(ws + w.full_list);
+  uint32_t *bin_count = (uint32_t *)(ws + w.bin_count);
   uint32_t *counters = (uint32_t *)(ws + w.counters);  // [0] codes to refine, [1] rows to refine
 
   stage_mark(c, st, "start");
   CK(cudaMemsetAsync(status_dev, 0, 4, st));
   CK(cudaMemsetAsync(counters, 0, 256, st));
   if (L.n_rows) CK(cudaMemsetAsync(rowflag, 0, 4ull * L.n_rows, st));
+  CK(cudaMemsetAsync(bin_count, 0, 4ull * N_COEF, st));
   if (L.n_chunks) CK(cudaMemsetAsync(nesc_w, 0, 4ull * L.n_chunks, st));
   RET(upload_tables(c, L, ws, w, st));
   { k_layout<<<dim3(L.batch, LAYOUT_SPLIT), 256, 0, st>>>(d_prompts, row_tok, row_pos, row_edst, row_slot, e_tok, e_slot, e_row, slot_chunk,
-                                    c->chunk_rows, qe); ++g_launches; }
+                                    c->chunk_rows, qe, c->kw); ++g_launches; }
   if (L.n_tokens > 0)
     { k_convert<<<(unsigned)L.n_tokens, 192, 0, st>>>((const __nv_bfloat16 *)rows, d_prompts, L.batch, x16, bl, blob_cap,
                                                     L.off_kept, row_norm, status_dev); ++g_launches; }
@@ -1332,7 +1605,7 @@ static int encode_impl(const dckv_codec *c, const void *rows, const int32_t *tok
     RET(map_b(&mb_xh, x16, false, ROW_DIM, L.n_rows, HIDDEN_SPLIT_BN / 2));
     RET(map_b(&mb_xt, x16, false, ROW_DIM, L.n_rows, TRANSFORM_BN / 2));
     RET(map_b(&mb_gt, g16, false, 2 * N_HIDDEN, L.n_rows, TRANSFORM_BN / 2));
-    RET(map_b(&mb_qe, qe, true, N_COEF, L.ne_pad, MEAN_ODD_BN / 2));
+    RET(map_b(&mb_qe, qe, true, c->kw, L.ne_pad, MEAN_ODD_BN / 2));
     // correction hidden layer: h = x @ w1 - mu @ w1, GELU, fp16 hi/lo
     if (c->has_mlp) {
       GemmProblem pr = make_problem(N_HIDDEN / GEMM_BM, L.n_rows, HIDDEN_SPLIT_BN, false, status_dev);
@@ -1347,37 +1620,47 @@ static int encode_impl(const dckv_codec *c, const void *rows, const int32_t *tok
     stage_mark(c, st, "gemm_hidden");
     // transform + quantiser: y = x @ B + g @ w2 - mu @ B
     {
-      GemmProblem pr = make_problem(N_COEF / GEMM_BM, L.n_rows, TRANSFORM_BN, false, status_dev);
+      GemmProblem pr = make_problem(c->mp / GEMM_BM, L.n_rows, TRANSFORM_BN, false, status_dev);
       add_seg(pr, 0, 0, 2, 0, 0, 0, 0, ROW_DIM / GEMM_BK);
       if (c->has_mlp) {  // + g @ w2 (hi/lo on both sides)
         add_seg(pr, 1, 0, 2, 0, 1, 0, 0, N_HIDDEN / GEMM_BK);
         add_seg(pr, 1, 0, 2, 0, 1, 0, N_HIDDEN, N_HIDDEN / GEMM_BK);
       }
-      EpiQuantRegs::Params ep{{c->mub, c->delta, c->keep, (float)std::ldexp(1.0, -c->p_y), q32, qe, row_edst},
-                              row_norm, rowflag, el_list, full_list, counters, w.el_cap, c->dbg_ratio};
+      EpiQuantRegs::Params ep{{c->mub_k, c->delta_k, c->k_eff, c->kw, (float)std::ldexp(1.0, -c->p_y), q32, qe,
+                               row_edst},
+                              row_norm, rowflag, el_bins, bin_count, full_list, counters, w.bin_cap,
+                              c->dbg_ratio, c->kept_list};
       RET((run_gemm2_chunked<EpiQuantRegs, 4, 2, TRANSFORM_CHUNK_STEPS, TRANSFORM_BN>(c->map_ay2, c->map_aw2_2, mb_xt, mb_gt, pr, ep,
                                                                    c->num_sms, false, st)));
     }
     stage_mark(c, st, "gemm_transform");
     // codes whose fp32 ratio lies in the guard band around a half step: exact fp64 values
-    { k_refine_codes<<<c->num_sms * 8, REFINE_THREADS, 0, st>>>(el_list, counters, w.el_cap, (const __nv_bfloat16 *)rows, row_tok,
-                                                  c->mu32, c->bt32, c->has_mlp ? c->w2t32 : nullptr, g16, c->delta,
-                                                  rowflag, q32, qe, row_edst); ++g_launches; }
-    const int rsmem = (ROW_DIM + N_HIDDEN) * 8;
-    CK(cudaFuncSetAttribute(k_refine_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, rsmem));
-    { k_refine_rows<<<c->num_sms, 256, rsmem, st>>>(full_list, counters, (const __nv_bfloat16 *)rows, row_tok, c->mu32,
-                                                  c->bt32, c->has_mlp ? c->w1t32 : nullptr,
-                                                  c->has_mlp ? c->w2t32 : nullptr, c->delta, c->keep, q32, qe,
-                                                  row_edst); ++g_launches; }
+    CK(cudaFuncSetAttribute(k_refine_codes, cudaFuncAttributeMaxDynamicSharedMemorySize, REFINE_SMEM));
+    CK(cudaFuncSetAttribute(k_refine_hidden, cudaFuncAttributeMaxDynamicSharedMemorySize, REFINE_SMEM));
+    CK(cudaFuncSetAttribute(k_refine_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, REFINE_SMEM));
+    { k_refine_codes<<<c->num_sms * 3, REFINE_THREADS, REFINE_SMEM, st>>>(
+          el_bins, bin_count, w.bin_cap, (const __nv_bfloat16 *)rows, row_tok, c->mub64, c->bt32,
+          c->has_mlp ? c->w2t32 : nullptr, g16, c->delta, rowflag, c->kept_list, c->kw, q32, qe, row_edst);
+      ++g_launches; }
+    stage_mark(c, st, "refine_codes");
+    double *g64 = (double *)(ws + w.g64);
+    if (c->has_mlp)
+      { k_refine_hidden<<<c->num_sms * 4, 256, REFINE_SMEM, st>>>(full_list, counters, (const __nv_bfloat16 *)rows,
+                                                                  row_tok, c->muw1_64, c->w1t32, g64); ++g_launches; }
+    { k_refine_rows<<<c->num_sms * 4, 256, REFINE_SMEM, st>>>(full_list, counters, (const __nv_bfloat16 *)rows,
+                                                            row_tok, c->mub64, c->bt32,
+                                                            c->has_mlp ? c->w2t32 : nullptr, g64, c->delta,
+                                                            c->kept_list, c->k_eff, c->kw, q32, qe, row_edst);
+      ++g_launches; }
     CK(cudaGetLastError());
-    stage_mark(c, st, "refine");
+    stage_mark(c, st, "refine_rows");
     if (stop == 1) return DCKV_OK;
     // odd mean model: [e, bf16(q_left), bf16(q_right)] @ w_odd -> centres
     if (c->has_means) {
-      GemmProblem pr = make_problem(N_COEF / GEMM_BM, L.ne_pad, MEAN_ODD_BN, true, status_dev);
-      add_seg(pr, 0, 0, 1, 0, 0, 0, 0, N_COEF / GEMM_BK);
-      add_seg(pr, 0, 0, 1, N_COEF, 0, 1, 0, N_COEF / GEMM_BK);
-      EpiMeanOdd<false>::Params ep{c->t_odd, token_ids, e_tok, e_slot, c->kidx, cen8, c->k_eff, c->vocab};
+      GemmProblem pr = make_problem(c->mp / GEMM_BM, L.ne_pad, MEAN_ODD_BN, true, status_dev);
+      add_seg(pr, 0, 0, 1, 0, 0, 0, 0, c->kw / GEMM_BK);
+      add_seg(pr, 0, 0, 1, c->kw, 0, 1, 0, c->kw / GEMM_BK);
+      EpiMeanOdd<false>::Params ep{c->t_odd, token_ids, e_tok, e_slot, c->kept_list, cen8, c->k_eff, c->kw, c->vocab};
       RET((run_gemm2<EpiMeanOdd<false>, 6, 1, 8, MEAN_ODD_BN>(c->map_aon1, c->map_aon1, mb_qe, mb_qe, pr, ep, c->num_sms, true, st)));
     }
     stage_mark(c, st, "gemm_mean_odd");
@@ -1386,7 +1669,7 @@ static int encode_impl(const dckv_codec *c, const void *rows, const int32_t *tok
     if (!c->has_means && L.n_symbols > 0)
       CK(cudaMemsetAsync(cen8, 0, (size_t)L.n_symbols, st));  // unconditional tables: every centre 0
     { k_symbols<<<rg, SYM_THREADS, 0, st>>>(L.n_rows, row_slot, slot_chunk, q32, cen8, c->kept_list, c->kept_scale,
-                                          c->cfm_tab, c->k_eff, c->has_means ? c->t_even : nullptr, token_ids,
+                                          c->cfm_tab, c->k_eff, c->kw, c->has_means ? c->t_even : nullptr, token_ids,
                                           row_tok, row_edst, c->vocab, sym16, cfm, nesc_w); ++g_launches; }
     CK(cudaGetLastError());
     stage_mark(c, st, "symbols");
@@ -1407,7 +1690,7 @@ static int encode_impl(const dckv_codec *c, const void *rows, const int32_t *tok
     CK(cudaGetLastError());
   }
   if (L.n_chunks > 0) {
-    CompactArgs a{d_chunks, d_prompts, L.n_chunks, c->k_eff, c->kept_list, q32, sym16,
+    CompactArgs a{d_chunks, d_prompts, L.n_chunks, c->k_eff, c->kw, q32, sym16,
                   (const uint16_t *)(ws + w.words), states, nwords, nesc, offs, bl, blob_cap, L.off_streams};
     { compact_kernel<<<L.n_chunks, COMPACT_THREADS, 0, st>>>(a); ++g_launches; }
     CK(cudaGetLastError());
@@ -1436,9 +1719,8 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
   const WsPlan w = plan_ws(L, 1);
   if (ws_bytes < w.total) return fail(DCKV_ECAPACITY, "workspace too small (%zu < %zu)", ws_bytes, w.total);
   cudaStream_t st = (cudaStream_t)stream;
-  CK(cudaSetDevice(c->device));
-  dckv_codec *cm = const_cast<dckv_codec *>(c);
-  cm->n_ev = 0;
+  DEVICE_SCOPE(c->device);
+  stage_begin(c);
   uint8_t *ws = (uint8_t *)workspace;
   const uint8_t *bl = (const uint8_t *)blob;
   PromptInfo *d_prompts = (PromptInfo *)(ws + w.prompts);
@@ -1463,14 +1745,14 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
   CK(cudaMemsetAsync(status_dev, 0, 4, st));
   CK(cudaMemsetAsync(counters, 0, 256, st));
   RET(upload_tables(c, L, ws, w, st));
-  CK(cudaMemsetAsync(qe, 0, 2ull * L.ne_pad * N_COEF, st));
+  CK(cudaMemsetAsync(qe, 0, 2ull * L.ne_pad * c->kw, st));
   if (L.n_rows) {
-    CK(cudaMemsetAsync(q16, 0, 2ull * L.n_rows * N_COEF, st));
+    CK(cudaMemsetAsync(q16, 0, 2ull * L.n_rows * c->kw, st));
     CK(cudaMemsetAsync(bigflag, 0, 4ull * L.n_rows, st));
   }
   if (L.n_chunks) CK(cudaMemsetAsync(ws + w.escflag, 0, 4ull * L.n_chunks, st));
   { k_layout<<<dim3(L.batch, LAYOUT_SPLIT), 256, 0, st>>>(d_prompts, row_tok, row_pos, row_edst, row_slot, e_tok, e_slot, e_row, slot_chunk,
-                                    c->chunk_rows, nullptr); ++g_launches; }
+                                    c->chunk_rows, nullptr, c->kw); ++g_launches; }
   HeaderCheck hc{bl, blob_bytes, d_prompts, L.batch, c->chunk_rows, c->k_eff, L.n_chunks_e, L.n_chunks_o,
                  L.n_kept, L.off_kept, L.off_streams, valid, status_dev};
   { k_check_header<<<1, 256, 0, st>>>(hc); ++g_launches; }
@@ -1491,20 +1773,21 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
   RansDecArgs da{d_chunks, 0, L.n_chunks, c->k_eff, c->kept_scale, c->dcdf, c->lut, c->tail, bl, L.off_streams,
                  offs, syms16, valid, status_dev};
   uint32_t *escflag = (uint32_t *)(ws + w.escflag);
-  DecCodesArgs fa{d_chunks, d_prompts, 0, L.n_chunks_e, c->k_eff, c->kept_list, syms16, bl, L.off_streams,
+  DecCodesArgs fa{d_chunks, d_prompts, 0, L.n_chunks_e, c->k_eff, c->kw, syms16, bl, L.off_streams,
                   offs, q16, qe, qbig, bigflag, biglist, counters, escflag, valid, status_dev};
   const unsigned rg = (unsigned)std::max<int64_t>(1, std::min<int64_t>(L.n_rows, 65535));
   if (L.n_chunks > 0) {
-    const unsigned g = (L.n_chunks + RANS_WARPS - 1) / RANS_WARPS;
+    // one block per SM at most (each holds the tables), chunks spread over the blocks
+    const unsigned g = (unsigned)std::max(1, std::min(c->num_sms, L.n_chunks));
     if (c->k_eff >= 32)
-      { rans_decode_kernel<true><<<g, RANS_WARPS * 32, RANS_DEC_SMEM, st>>>(da); ++g_launches; }
+      { rans_decode_kernel<true><<<g, DEC_WARPS * 32, RANS_DEC_SMEM, st>>>(da); ++g_launches; }
     else
-      { rans_decode_kernel<false><<<g, RANS_WARPS * 32, RANS_DEC_SMEM, st>>>(da); ++g_launches; }
+      { rans_decode_kernel<false><<<g, DEC_WARPS * 32, RANS_DEC_SMEM, st>>>(da); ++g_launches; }
   }
   CK(cudaGetLastError());
   stage_mark(c, st, "rans_loop");
   if (L.n_chunks_e > 0) {
-    { k_codes_elem<<<rg, 256, 0, st>>>(0, L.n_rows, row_edst, row_slot, slot_chunk, syms16, cen8, c->kept_list,
+    { k_codes_elem<<<rg, 256, 0, st>>>(0, L.n_rows, row_edst, row_slot, slot_chunk, syms16, cen8, c->kw,
                                        c->k_eff, q16, qe, escflag, valid); ++g_launches; }
     { k_escape_patch<<<(unsigned)L.n_chunks_e, PATCH_THREADS, 0, st>>>(fa); ++g_launches; }
   }
@@ -1512,19 +1795,19 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
   stage_mark(c, st, "codes_even");
   if (L.n_rows > 0 && c->has_means) {
     CUtensorMap mb_qe;
-    RET(map_b(&mb_qe, qe, true, N_COEF, L.ne_pad, MEAN_ODD_BN / 2));
-    GemmProblem pr = make_problem(N_COEF / GEMM_BM, L.ne_pad, MEAN_ODD_BN, true, status_dev);
-    add_seg(pr, 0, 0, 1, 0, 0, 0, 0, N_COEF / GEMM_BK);
-    add_seg(pr, 0, 0, 1, N_COEF, 0, 1, 0, N_COEF / GEMM_BK);
+    RET(map_b(&mb_qe, qe, true, c->kw, L.ne_pad, MEAN_ODD_BN / 2));
+    GemmProblem pr = make_problem(c->mp / GEMM_BM, L.ne_pad, MEAN_ODD_BN, true, status_dev);
+    add_seg(pr, 0, 0, 1, 0, 0, 0, 0, c->kw / GEMM_BK);
+    add_seg(pr, 0, 0, 1, c->kw, 0, 1, 0, c->kw / GEMM_BK);
     // odd centres, and with them the odd codes (ESC symbols are left to the patch)
-    EpiMeanOdd<true>::Params ep{c->t_odd, token_ids, e_tok, e_slot, c->kidx, cen8, c->k_eff, c->vocab,
+    EpiMeanOdd<true>::Params ep{c->t_odd, token_ids, e_tok, e_slot, c->kept_list, cen8, c->k_eff, c->kw, c->vocab,
                                 syms16, q16, e_row, slot_chunk, escflag};
     RET((run_gemm2<EpiMeanOdd<true>, 6, 1, 8, MEAN_ODD_BN>(c->map_aon1, c->map_aon1, mb_qe, mb_qe, pr, ep, c->num_sms, true, st)));
   }
   stage_mark(c, st, "gemm_mean_odd");
   if (L.n_chunks_o > 0) {
     if (!c->has_means)  // unconditional tables: every odd centre is 0
-      { k_codes_elem<<<rg, 256, 0, st>>>(1, L.n_rows, row_edst, row_slot, slot_chunk, syms16, cen8, c->kept_list,
+      { k_codes_elem<<<rg, 256, 0, st>>>(1, L.n_rows, row_edst, row_slot, slot_chunk, syms16, cen8, c->kw,
                                          c->k_eff, q16, qe, escflag, valid); ++g_launches; }
     fa.chunk0 = L.n_chunks_e;
     fa.n_chunks = L.n_chunks_o;
@@ -1535,18 +1818,18 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
   __half *g16d = (__half *)(ws + w.g16);
   if (L.n_rows > 0 && c->has_synth) {  // decoder-side synthesis, hidden layer: GELU((q Delta) V1)
     CUtensorMap mb_qh;
-    RET(map_b(&mb_qh, q16, false, N_COEF, L.n_rows, HIDDEN_BN / 2));
+    RET(map_b(&mb_qh, q16, false, c->kw, L.n_rows, HIDDEN_BN / 2));
     GemmProblem pr = make_problem(N_HIDDEN / GEMM_BM, L.n_rows, HIDDEN_BN, false, status_dev);
-    add_seg(pr, 0, 0, 2, 0, 0, 0, 0, N_COEF / GEMM_BK);
+    add_seg(pr, 0, 0, 2, 0, 0, 0, 0, c->kw / GEMM_BK);
     EpiGelu::Params ep{c->zero256, (float)std::ldexp(1.0, -c->p_v1), g16d};
     RET((run_gemm2<EpiGelu, 4, 2, 4, HIDDEN_BN>(c->map_av1, c->map_av1, mb_qh, mb_qh, pr, ep, c->num_sms, false, st)));
     stage_mark(c, st, "gemm_synth_hidden");
   }
   if (L.n_rows > 0) {
     CUtensorMap mb_q, mb_g;
-    RET(map_b(&mb_q, q16, false, N_COEF, L.n_rows, INVERSE_BN / 2));
+    RET(map_b(&mb_q, q16, false, c->kw, L.n_rows, INVERSE_BN / 2));
     GemmProblem pr = make_problem(ROW_DIM / GEMM_BM, L.n_rows, INVERSE_BN, false, status_dev);
-    add_seg(pr, 0, 0, 2, 0, 0, 0, 0, N_COEF / GEMM_BK);
+    add_seg(pr, 0, 0, 2, 0, 0, 0, 0, c->kw / GEMM_BK);
     if (c->has_synth) {  // + g V2 (hi/lo on both sides)
       RET(map_b(&mb_g, g16d, false, 2 * N_HIDDEN, L.n_rows, INVERSE_BN / 2));
       add_seg(pr, 1, 0, 2, 0, 1, 0, 0, N_HIDDEN / GEMM_BK);
@@ -1567,7 +1850,7 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
     { k_fixup<<<c->num_sms, 256, 0, st>>>(biglist, counters, q16, qbig, c->a_inv, (float)std::ldexp(1.0, -c->p_inv),
                                        c->mu_perm, c->theta, row_tok, row_pos, (__nv_bfloat16 *)k_out,
                                        (__nv_bfloat16 *)v_out, L.n_tokens, c->has_synth ? c->v1t32 : nullptr,
-                                       c->v2_32, c->delta); ++g_launches; }
+                                       c->v2_32, c->delta, c->kept_list, c->k_eff, c->kw); ++g_launches; }
   CK(cudaGetLastError());
   stage_mark(c, st, "kept+fixup");
   return DCKV_OK;
@@ -1631,18 +1914,19 @@ extern "C" int dckv_bytes(const void *blob_host, size_t len, dckv_byte_report *o
 extern "C" int dckv_set_timing(dckv_codec *c, int enable) {
   if (!c) return DCKV_EINVAL;
   c->timing = enable ? 1 : 0;
-  c->n_ev = 0;
+  if (t_stages.codec == c) t_stages.n = 0;
   return DCKV_OK;
 }
-
 extern "C" int dckv_get_timing(const dckv_codec *c, float *ms, const char **names, int max) {
   if (!c || !ms) return -1;
+  const StageLog &g = t_stages;
+  if (g.codec != c) return 0;
   int n = 0;
-  for (int i = 1; i < c->n_ev && n < max; ++i, ++n) {
+  for (int i = 1; i < g.n && n < max; ++i, ++n) {
     float t = 0.f;
-    cudaEventElapsedTime(&t, c->ev[i - 1], c->ev[i]);
+    cudaEventElapsedTime(&t, g.ev[i - 1], g.ev[i]);
     ms[n] = t;
-    if (names) names[n] = c->ev_names[i];
+    if (names) names[n] = g.names[i];
   }
   return n;
 }
@@ -1650,7 +1934,7 @@ extern "C" int dckv_get_timing(const dckv_codec *c, float *ms, const char **name
 extern "C" int dckv_codec_export(const dckv_codec *c, uint16_t *cdf_host, uint8_t *scale_host, uint8_t *keep_host,
                                  int32_t *exps_host) {
   if (!c) return fail(DCKV_EINVAL, "NULL codec");
-  CK(cudaSetDevice(c->device));
+  DEVICE_SCOPE(c->device);
   if (cdf_host) CK(cudaMemcpy(cdf_host, c->cdf, 2ull * N_SCALES * N_SYM, cudaMemcpyDeviceToHost));
   if (scale_host) CK(cudaMemcpy(scale_host, c->scale, N_COEF, cudaMemcpyDeviceToHost));
   if (keep_host) CK(cudaMemcpy(keep_host, c->keep, N_COEF, cudaMemcpyDeviceToHost));
@@ -1702,6 +1986,7 @@ extern "C" int dckv_ws_offsets(const dckv_codec *c, const int64_t *offs, int bat
   out->ne_pad = L.ne_pad;
   out->n_chunks = L.n_chunks;
   out->total = w.total;
+  out->code_width = c->kw;
   return DCKV_OK;
 }
 
@@ -1751,7 +2036,7 @@ extern "C" int dckv_decode_static(const dckv_codec *c, const void *blob, size_t 
     return fail(DCKV_ECAPACITY, "batch needs %zu bytes of decode scratch; the static scratch holds %zu", need,
                 (size_t)DCKV_STATIC_SCRATCH_BYTES);
   if (c->device < 0 || c->device >= MAX_DEVICES) return fail(DCKV_EINVAL, "device %d out of range", c->device);
-  CK(cudaSetDevice(c->device));
+  DEVICE_SCOPE(c->device);
   void *scratch = nullptr;
   {
     std::lock_guard<std::mutex> lock(g_static_mu);

@@ -138,12 +138,13 @@ struct EpiGelu {
 // model's input).
 struct EpiQuant {
   struct Params {
-    const float *mub;
-    const float *delta;
-    const uint8_t *keep;
+    const float *mub;         // [mp] (mu @ basis) of the kept components, compact order
+    const float *delta;       // [mp] Delta of the kept components
+    int k_eff;                // features m < k_eff are kept components; the rest give 0
+    int kw;                   // width of the code arrays (a multiple of 64, >= k_eff)
     float scale;
-    int32_t *q32;             // [rows][2048]
-    __nv_bfloat16 *qe;        // [ne_pad][2048]
+    int32_t *q32;             // [rows][kw]
+    __nv_bfloat16 *qe;        // [ne_pad][kw]
     const int32_t *row_edst;  // [rows]: padded even row or -1
   };
 };
@@ -156,11 +157,13 @@ struct EpiQuantRegs {
     EpiQuant::Params q;
     const float *row_norm;   // [rows] |x|_2 of the coded row
     uint32_t *rowflag;       // [rows] 1 once the row is listed for full refinement
-    uint32_t *el_list;       // codes to refine: row * 2048 + c
+    uint32_t *el_bins;       // codes to refine, binned by component: el_bins[c * bin_cap + i] = row
+    uint32_t *bin_count;     // [2048] codes listed per component
     uint32_t *full_list;     // rows to refine whole
     uint32_t *counters;      // [0] listed codes, [1] listed rows
-    int64_t el_cap;
-    float *dbg_ratio;        // optional export of the fp32 ratios (self-test)
+    uint32_t bin_cap;
+    float *dbg_ratio;        // optional export of the fp32 ratios (self-test), [rows][2048] by component
+    const int16_t *kept_list;  // compact index -> component (for dbg_ratio)
   };
   __device__ static void list_row(const Params &p, int row) {
     if (atomicExch(&p.rowflag[row], 1u) == 0u) p.full_list[atomicAdd(&p.counters[1], 1u)] = (uint32_t)row;
@@ -169,9 +172,13 @@ struct EpiQuantRegs {
     if (pp.row_norm[row] > REFINE_NORM_FULL) {
       list_row(pp, row);
     } else {
-      const uint32_t idx = atomicAdd(&pp.counters[0], 1u);
-      if ((int64_t)idx < pp.el_cap) pp.el_list[idx] = (uint32_t)row * N_COEF + (uint32_t)c;
-      else list_row(pp, row);
+      const uint32_t idx = atomicAdd(&pp.bin_count[c], 1u);
+      if (idx < pp.bin_cap) {
+        pp.el_bins[(int64_t)c * pp.bin_cap + idx] = (uint32_t)row;
+        atomicAdd(&pp.counters[0], 1u);
+      } else {
+        list_row(pp, row);  // a full bin: the whole row is recomputed instead
+      }
     }
   }
   // per tile column: padded even row (or -1) and the guard-band width's row term
@@ -191,10 +198,11 @@ struct EpiQuantRegs {
     const EpiQuant::Params &p = pp.q;
     const int32_t *s_e = reinterpret_cast<const int32_t *>(buf);
     const float *s_w = reinterpret_cast<const float *>(buf + GEMM_MAX_BN * 4);
-    const int c = mt * GEMM_BM + ew * 32 + lane;
+    const int c = mt * GEMM_BM + ew * 32 + lane;  // compact component index
+    if (c >= p.kw) return;  // rows of the tile past the code arrays' width (all zero operands)
     const float mb = p.mub[c];
     const float dl = p.delta[c];
-    const bool kp = p.keep[c] != 0;
+    const bool kp = c < p.k_eff;
     const float wk = REFINE_KAPPA / dl;
     uint32_t fm[(NC + 31) / 32];  // columns whose code goes to the exact recomputation
 #pragma unroll
@@ -207,10 +215,10 @@ struct EpiQuantRegs {
         const float y = tot[j] * p.scale - mb;
         const float ratio = __fdiv_rn(y, dl);
         const int q = kp ? __float2int_rn(ratio) : 0;
-        p.q32[(int64_t)row * N_COEF + c] = q;
+        p.q32[(int64_t)row * p.kw + c] = q;
         const int e = s_e[col];
-        if (e >= 0) p.qe[(int64_t)e * N_COEF + c] = __float2bfloat16_rn((float)q);
-        if (pp.dbg_ratio) pp.dbg_ratio[(int64_t)row * N_COEF + c] = ratio;
+        if (e >= 0) p.qe[(int64_t)e * p.kw + c] = __float2bfloat16_rn((float)q);
+        if (pp.dbg_ratio && kp) pp.dbg_ratio[(int64_t)row * N_COEF + pp.kept_list[c]] = ratio;
         const float w = wk * s_w[col] + REFINE_W0;
         if (kp && (0.5f - fabsf(ratio - rintf(ratio)) < w || !(fabsf(ratio) < 1.0e6f))) fm[j >> 5] |= 1u << (j & 31);
       }
@@ -238,14 +246,15 @@ struct EpiMeanOdd {
     const int32_t *tok_ids;  // [tokens]
     const int32_t *e_tok;    // [ne_pad] token row of the odd row, -1 if none
     const int32_t *e_slot;   // [ne_pad] slot row of that odd row
-    const int16_t *kidx;     // [2048] kept index, -1 if dropped
+    const int16_t *kept_list;  // compact index -> component (the GEMM's features are kept components)
     int8_t *cen8;            // [slots][k_eff]  (encoder: the odd centres)
     int k_eff;
+    int kw;                  // width of q16
     int vocab;
     // decoder: the odd codes themselves, code = centre + symbol - 254 (q16 != NULL); an
     // ESC symbol leaves its code to the escape patch and flags its chunk
     const uint16_t *syms;    // [slots][k_eff] decoded symbols
-    __half *q16;             // [rows][2048]
+    __half *q16;             // [rows][kw]
     const int32_t *e_row;    // [ne_pad] natural coded row of that odd row
     const int32_t *slot_chunk;
     uint32_t *escflag;       // [chunks]
@@ -270,8 +279,9 @@ struct EpiMeanOdd {
       if (dec) s_nat[j] = __ldg(p.e_row + cx.n0 + j);
     }
     named_bar_sync(cx.bar, 128);
-    const int c = cx.mt * GEMM_BM + cx.ew * 32 + cx.lane;
-    const int kc = p.kidx[c];
+    const int kc0 = cx.mt * GEMM_BM + cx.ew * 32 + cx.lane;  // compact index of this thread's feature
+    const int kc = kc0 < p.k_eff ? kc0 : -1;
+    const int c = kc >= 0 ? p.kept_list[kc] : 0;  // its component (t_odd column)
     for (int c0 = cx.grp * 32; c0 < n_valid; c0 += 32 * cx.n_grp) {
       uint32_t r[32];
       tmem_ld_32x32b_x32(cx.tacc + (uint32_t)c0, r);
@@ -295,7 +305,7 @@ struct EpiMeanOdd {
           } else if (sv[j] == ESC_SYM) {
             p.escflag[__ldg(p.slot_chunk + s_slot[c0 + j])] = 1u;
           } else {
-            p.q16[(int64_t)s_nat[c0 + j] * N_COEF + c] = __float2half_rn((float)((int)sv[j] - R_MAX + (int)cen));
+            p.q16[(int64_t)s_nat[c0 + j] * p.kw + kc] = __float2half_rn((float)((int)sv[j] - R_MAX + (int)cen));
           }
         }
       }

@@ -59,12 +59,20 @@ struct FitRegArgs {
   const int32_t *token_ids;
   const uint16_t *embed;     // bf16 [vocab][2048]
   int vocab;
-  const int32_t *q32;        // [n_rows][2048] final codes
+  const int32_t *q32;        // [n_rows][kw] final codes of the kept components (compact order)
+  const int16_t *kidx;       // [2048] compact index of a component, -1 if dropped (code 0)
+  int kw;
   int64_t slot0, n, kpad;    // first slot row of the parity, its rows, padded columns
   int n_x;                   // regressors: 2048 (even) or 6144 (odd)
   uint16_t *x_t;             // [n_x][kpad]        bf16 regressors, transposed
   uint16_t *y_t;             // [2][2048][kpad]    bf16 hi / lo of the clipped codes
 };
+
+// code of component c of coded row r (0 for a dropped component)
+__device__ __forceinline__ int32_t code_of(const FitRegArgs &a, int64_t r, int c) {
+  const int m = __ldg(a.kidx + c);
+  return m >= 0 ? __ldg(a.q32 + r * a.kw + m) : 0;
+}
 
 __device__ __forceinline__ uint16_t bf16_bits_of_code(int32_t q) {
   return __bfloat16_as_ushort(__double2bfloat16((double)q));  // one RNE step, as the mean model reads q
@@ -89,7 +97,7 @@ __global__ void __launch_bounds__(256) k_fit_regress(FitRegArgs a) {
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const int c = f0 - a.n_x + tx + 32 * h;
-          const int32_t q = min(max(__ldg(a.q32 + r * N_COEF + c), -CODE_CLIP), CODE_CLIP);
+          const int32_t q = min(max(code_of(a, r, c), -CODE_CLIP), CODE_CLIP);
           const __nv_bfloat16 bh = __float2bfloat16_rn((float)q);  // exact below 2^8, else the hi part
           vh[h] = __bfloat16_as_ushort(bh);
           vl[h] = __bfloat16_as_ushort(__float2bfloat16_rn((float)q - __bfloat162float(bh)));  // exact
@@ -107,9 +115,9 @@ __global__ void __launch_bounds__(256) k_fit_regress(FitRegArgs a) {
           if (f < N_COEF)
             vh[h] = __ldg(a.embed + (int64_t)tok * N_COEF + f);
           else if (f < 2 * N_COEF)
-            vh[h] = bf16_bits_of_code(__ldg(a.q32 + (r - 1) * N_COEF + (f - N_COEF)));
+            vh[h] = bf16_bits_of_code(code_of(a, r - 1, f - N_COEF));
           else
-            vh[h] = right_ok ? bf16_bits_of_code(__ldg(a.q32 + (r + 1) * N_COEF + (f - 2 * N_COEF))) : 0;
+            vh[h] = right_ok ? bf16_bits_of_code(code_of(a, r + 1, f - 2 * N_COEF)) : 0;
         }
       }
     }
@@ -405,7 +413,7 @@ __global__ void k_fit_bf16(const double *w, int64_t count, uint16_t *out) {
 // Scale sums: thread k of a block keeps the sum of |q - centre| of kept components
 // k, k + 256, ... over the block's rows; integer sums, so the result is exact.
 __global__ void __launch_bounds__(256) k_fit_absres(int64_t n_rows, const int32_t *row_slot, const int32_t *q32,
-                                                    const int8_t *cen8, const int16_t *kept_list, int k_eff,
+                                                    const int8_t *cen8, const int16_t *kept_list, int k_eff, int kw,
                                                     unsigned long long *abs_sum) {
   constexpr int PER = N_COEF / 256;
   long long acc[PER];
@@ -417,7 +425,7 @@ __global__ void __launch_bounds__(256) k_fit_absres(int64_t n_rows, const int32_
     for (int u = 0; u < PER; ++u) {
       const int k = threadIdx.x + 256 * u;
       if (k < k_eff) {
-        const long long d = (long long)__ldg(q32 + r * N_COEF + kept_list[k]) - (long long)cen8[base + k];
+        const long long d = (long long)__ldg(q32 + r * kw + k) - (long long)cen8[base + k];
         acc[u] += d < 0 ? -d : d;
       }
     }
@@ -478,7 +486,7 @@ extern "C" int dckv_fit_accumulate(const dckv_codec *c, const uint16_t *embed, i
     for (int par = 0; par < 2; ++par) {
       a[par] = FitRegArgs{(const PromptInfo *)(ws + f.enc.prompts), L.batch, inv,
                           (const int32_t *)(ws + f.enc.row_tok), token_ids, embed, vocab,
-                          (const int32_t *)(ws + f.enc.q32), par ? f.n_e : 0, par ? f.n_o : f.n_e,
+                          (const int32_t *)(ws + f.enc.q32), c->kidx, c->kw, par ? f.n_e : 0, par ? f.n_o : f.n_e,
                           par ? f.ko : f.ke, par ? 3 * N_COEF : N_COEF,
                           (uint16_t *)(ws + (par ? f.xot : f.et)), (uint16_t *)(ws + (par ? f.yot : f.yet))};
       if (a[par].n == 0) continue;
@@ -549,7 +557,7 @@ extern "C" int dckv_fit_scales_accumulate(const dckv_codec *c, const void *rows,
   uint8_t *ws = (uint8_t *)workspace;
   const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(L.n_rows, (int64_t)c->num_sms * 4));
   { k_fit_absres<<<grid, 256, 0, st>>>(L.n_rows, (const int32_t *)(ws + w.row_slot), (const int32_t *)(ws + w.q32),
-                                     (const int8_t *)(ws + w.cen8), c->kept_list, c->k_eff,
+                                     (const int8_t *)(ws + w.cen8), c->kept_list, c->k_eff, c->kw,
                                      (unsigned long long *)abs_sum); ++g_launches; }
   CK(cudaGetLastError());
   return DCKV_OK;

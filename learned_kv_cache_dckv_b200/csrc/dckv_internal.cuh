@@ -84,6 +84,7 @@ struct Layout {
   int64_t max_len = 0;    // longest prompt (RoPE table positions)
   int n_chunks = 0, n_chunks_e = 0, n_chunks_o = 0;
   int64_t n_symbols = 0;  // n_rows * K_eff
+  int kw = 64;            // width of the code arrays (the codec's kw)
   std::vector<PromptInfo> prompts;
   std::vector<ChunkDesc> chunks;
   uint64_t off_kept = 0, off_streams = 0;  // blob offsets
@@ -99,8 +100,8 @@ struct WsPlan {
   size_t hpart;    // encode: split-K parts of the correction hidden layer, fp32
   size_t slots16;  // decode: decoded symbols (slot order)
   size_t rope;     // decode: float2 [max_len][128] RoPE (cos, sin)
-  size_t row_norm, rowflag, el_list, full_list;                         // encode refinement
-  int64_t el_cap;
+  size_t row_norm, rowflag, el_bins, bin_count, full_list, g64;        // encode refinement
+  uint32_t bin_cap;
   size_t q16, qbig, bigflag, biglist, counters, valid;                  // decode
   size_t total;
 };
@@ -114,6 +115,11 @@ struct dckv_codec {
   int chunk_rows = 32;
   int vocab = 0;
   int k_eff = 0;
+  // Only kept components are computed: the GEMMs run on compacted operands.  kw = K_eff
+  // rounded up to 64 (the width of every code array and the K extent of the GEMMs that read
+  // codes), mp = K_eff rounded up to 256 (the M extent of the CTA-pair GEMMs that produce one
+  // value per kept component).  Compact index m is component kept_list[m].
+  int kw = 64, mp = 256;
   bool has_mlp = true;    // correction layer present (false: linear codec)
   bool has_means = true;  // mean models present (false: unconditional zero-mean tables)
   bool has_synth = false; // decoder-side synthesis correction present
@@ -121,14 +127,16 @@ struct dckv_codec {
   dckv_params p{};
   // derived, library-owned device buffers
   void *blk = nullptr;  // one allocation holding everything below
-  __half *a_y = nullptr;     // [2][2048][6144]  basis^T * 2^p_y, split hi/lo
-  __half *a_w2 = nullptr;    // [2][2048][256]   w2^T * 2^p_y, split
-  __half *a_h = nullptr;     // [2][256][6144]   w1^T * 2^p_h, split
-  __half *a_inv = nullptr;   // [2][6144][2048]  (Delta_c basis[d][c]) * 2^p_inv, dims permuted
-  __nv_bfloat16 *a_on = nullptr;  // [2048][4096]  odd mean model, neighbour blocks, transposed
+  __half *a_y = nullptr;     // [2][mp][6144]  basis^T * 2^p_y, split hi/lo, kept components (zero rows after)
+  __half *a_w2 = nullptr;    // [2][mp][256]   w2^T * 2^p_y, split, kept components
+  __half *a_h = nullptr;     // [2][256][6144] w1^T * 2^p_h, split
+  __half *a_inv = nullptr;   // [2][6144][kw]  (Delta_c basis[d][c]) * 2^p_inv, dims permuted, kept c
+  __nv_bfloat16 *a_on = nullptr;  // [mp][2 kw]  odd mean model, neighbour blocks, kept in and out
   float *t_even = nullptr;   // [vocab][2048]  embed @ w_even
   float *t_odd = nullptr;    // [vocab][2048]  embed @ w_odd[0:2048]
   float *mub = nullptr;      // [2048]  mu @ basis
+  float *mub_k = nullptr;    // [mp]    mu @ basis of kept components (0 after)
+  float *delta_k = nullptr;  // [mp]    Delta of kept components (1 after)
   float *muw1 = nullptr;     // [256]   mu @ w1
   float *mu_perm = nullptr;  // [6144]  mu in the inverse GEMM's row order
   float *delta = nullptr;    // [2048]
@@ -150,18 +158,16 @@ struct dckv_codec {
   float *bt32 = nullptr;     // [2048][6144] basis^T
   float *w1t32 = nullptr;    // [256][6144]  w1^T
   float *w2t32 = nullptr;    // [2048][256]  w2^T
-  float *mu32 = nullptr;     // [6144]
+  double *mub64 = nullptr;   // [2048]  mu @ basis, fp64
+  double *muw1_64 = nullptr; // [256]   mu @ w1, fp64
   // decoder-side synthesis (optional): split operands and fp32 copies for the exact fix-up
-  __half *a_v1 = nullptr;    // [2][256][2048]  (Delta_c V1[c][h]) * 2^p_v1, split
+  __half *a_v1 = nullptr;    // [2][256][kw]  (Delta_c V1[c][h]) * 2^p_v1, split, kept c
   __half *a_v2 = nullptr;    // [2][6144][256]  V2[h][d] * 2^p_inv, split, dims permuted like a_inv
   float *v1t32 = nullptr;    // [256][2048]  V1^T
   float *v2_32 = nullptr;    // [256][6144]  V2
   float *zero256 = nullptr;  // [256] zeros (the synthesis hidden layer has no offset)
   int p_y = 0, p_h = 0, p_inv = 0, p_v1 = 0;  // power-of-two operand scales
   CUtensorMap map_ay2, map_aw2_2, map_aw2_1, map_ah2, map_ainv2, map_aon1, map_av1, map_av2;
-  // stage timing (optional)
+  // stage timing (optional; the events live in a per-thread log of the calling thread)
   int timing = 0;
-  cudaEvent_t ev[24];
-  int n_ev = 0;
-  const char *ev_names[24];
 };

@@ -77,6 +77,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
   }
 }
 
+// Bounded wait that ignores the abort flag, for a CTA about to leave after a timeout: it
+// waits (at most another DCKV_WAIT_NS) for the copies it issued itself to land, so that it
+// does not exit while they may still be writing its shared memory.
+__device__ __forceinline__ bool mbar_drain(uint64_t *bar, uint32_t parity) {
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity))
+    if (global_timer_ns() - t0 > DCKV_WAIT_NS) return false;
+  return true;
+}
+
 // ---------------------------------------------------------------- TMA (no multicast)
 __device__ __forceinline__ void tma_load_2d(void *dst, const void *tmap, uint64_t *bar, int c0, int c1) {
   asm volatile(

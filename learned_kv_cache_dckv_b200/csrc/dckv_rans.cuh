@@ -19,7 +19,11 @@
 
 namespace dckv {
 
-constexpr int RANS_WARPS = 4;                            // chunks per block
+constexpr int RANS_WARPS = 4;                            // chunks per block (encoder)
+// Decoder: one block per SM (its tables fill the SM's shared memory), DEC_WARPS warps each
+// decoding one chunk at a time; a lane's step is a latency-bound dependency chain, so many
+// warps per SM keep the schedulers busy.
+constexpr int DEC_WARPS = 32;
 constexpr int PF = 16;                                   // steps of look-ahead for state-free data
 // Decoder tables in shared memory.  Rows are padded by 4 bytes so that the same entry of
 // different scales falls in different banks: most lanes of a step decode the central
@@ -92,7 +96,7 @@ __device__ __forceinline__ int even_centre(const float *t_row, int comp) {
 __global__ void __launch_bounds__(SYM_THREADS) k_symbols(int64_t n_rows, const int32_t *row_slot,
                                                          const int32_t *slot_chunk, const int32_t *q32,
                                                          int8_t *cen8, const int16_t *kept_list,
-                                                         const uint8_t *kept_scale, const uint2 *cfm_tab, int k_eff,
+                                                         const uint8_t *kept_scale, const uint2 *cfm_tab, int k_eff, int kw,
                                                          const float *t_even, const int32_t *tok_ids,
                                                          const int32_t *row_tok, const int32_t *row_edst, int vocab,
                                                          uint16_t *sym16, uint2 *cfm, uint32_t *nesc) {
@@ -108,7 +112,7 @@ __global__ void __launch_bounds__(SYM_THREADS) k_symbols(int64_t n_rows, const i
     __syncthreads();
     const int slot = row_slot[row];
     const int64_t base = (int64_t)slot * k_eff;
-    const int32_t *q = q32 + row * N_COEF;
+    const int32_t *q = q32 + row * kw;  // compact: kept component k at column k
     const bool even = row_edst[row] >= 0;
     const float *t_row = nullptr;
     if (even && t_even) t_row = t_even + (int64_t)min(max(tok_ids[row_tok[row]], 0), vocab - 1) * N_COEF;
@@ -118,7 +122,7 @@ __global__ void __launch_bounds__(SYM_THREADS) k_symbols(int64_t n_rows, const i
 #pragma unroll
       for (int u = 0; u < SYM_UNROLL; ++u) {
         const int k = k0 + u * SYM_THREADS;
-        v[u] = k < k_eff ? __ldg(q + s_kl[k]) : 0;
+        v[u] = k < k_eff ? __ldg(q + k) : 0;
         ce[u] = k >= k_eff ? 0 : even ? (t_row ? even_centre(t_row, s_kl[k]) : 0) : (int)__ldg(cen8 + base + k);
       }
 #pragma unroll
@@ -315,7 +319,7 @@ struct CompactArgs {
   const PromptInfo *prompts;
   int n_chunks;
   int k_eff;
-  const int16_t *kept_list;
+  int kw;                 // width of q32 (kept components, compact order)
   const int32_t *q32;
   const uint16_t *sym16;
   const uint16_t *words;
@@ -367,7 +371,7 @@ __global__ void __launch_bounds__(COMPACT_THREADS) compact_kernel(CompactArgs a)
         const int rl = (int)(i / K);
         const int k = (int)(i - (int64_t)rl * K);
         const int64_t row = (int64_t)pi.row_base + 2 * (cd.j0 + rl) + cd.parity;
-        const int64_t v = (int64_t)a.q32[row * N_COEF + a.kept_list[k]];
+        const int64_t v = (int64_t)a.q32[row * a.kw + k];
         const uint32_t slot = ep + __popc(m & lt_mask);
         if (slot < ne) {
           ev[2 * slot] = (uint32_t)(uint64_t)v;
@@ -595,28 +599,10 @@ __device__ __forceinline__ void dec_step(DecLane &d, uint32_t i, uint32_t S, int
   }
 }
 
-// The rANS arithmetic needs only the table (scale) of each component, never the code
-// means, so every chunk of both parities decodes in one launch; centres are applied
-// afterwards by the finishing kernel, pass by pass.
+// One warp decodes chunk ci: states, escape count and word stream from its section.
 template <bool BIG_K>
-__global__ void __launch_bounds__(RANS_WARPS * 32) rans_decode_kernel(RansDecArgs a) {
-  extern __shared__ __align__(16) uint8_t sm[];
-  const uint16_t *s_cdf = reinterpret_cast<const uint16_t *>(sm);
-  const uint16_t *s_lut = reinterpret_cast<const uint16_t *>(sm + CDF_SMEM_BYTES);
-  const uint32_t *s_tail = reinterpret_cast<const uint32_t *>(sm + CDF_SMEM_BYTES + LUT_SMEM_BYTES);
-  uint8_t *s_scale = sm + CDF_SMEM_BYTES + LUT_SMEM_BYTES + TAIL_SMEM_BYTES;
-  __shared__ uint64_t tab_bar;
-  __shared__ int tab_abort;
-  if (*a.valid != 1) return;
-  static_assert(CDF_SMEM_BYTES % 16 == 0 && LUT_SMEM_BYTES % 16 == 0 && TAIL_SMEM_BYTES % 16 == 0, "bulk sizes");
-  if (!bulk_load_tables(sm, a.dcdf, a.lut, a.tail, a.kept_scale, &tab_bar, &tab_abort)) {
-    if (threadIdx.x == 0) atomicExch(a.status, DCKV_ETIMEOUT);
-    return;
-  }
-  const int lane = threadIdx.x & 31;
-  const int wi = blockIdx.x * RANS_WARPS + (threadIdx.x >> 5);
-  if (wi >= a.n_chunks) return;
-  const int ci = a.chunk0 + wi;
+__device__ __forceinline__ void decode_chunk(const RansDecArgs &a, int ci, int lane, const uint8_t *s_scale,
+                                             const uint16_t *s_cdf, const uint16_t *s_lut, const uint32_t *s_tail) {
   const ChunkDesc cd = a.chunks[ci];
   const int K = a.k_eff;
   const uint32_t S = (uint32_t)cd.nrows * (uint32_t)K;  // < 2^20
@@ -663,6 +649,33 @@ __global__ void __launch_bounds__(RANS_WARPS * 32) rans_decode_kernel(RansDecArg
   if (__any_sync(0xffffffffu, bad) && lane == 0) atomicExch(a.status, DCKV_ECORRUPT);
 }
 
+// The rANS arithmetic needs only the table (scale) of each component, never the code
+// means, so every chunk of both parities decodes in one launch; centres are applied
+// afterwards by the finishing kernel, pass by pass.
+template <bool BIG_K>
+__global__ void __launch_bounds__(DEC_WARPS * 32, 1) rans_decode_kernel(RansDecArgs a) {
+  extern __shared__ __align__(16) uint8_t sm[];
+  const uint16_t *s_cdf = reinterpret_cast<const uint16_t *>(sm);
+  const uint16_t *s_lut = reinterpret_cast<const uint16_t *>(sm + CDF_SMEM_BYTES);
+  const uint32_t *s_tail = reinterpret_cast<const uint32_t *>(sm + CDF_SMEM_BYTES + LUT_SMEM_BYTES);
+  uint8_t *s_scale = sm + CDF_SMEM_BYTES + LUT_SMEM_BYTES + TAIL_SMEM_BYTES;
+  __shared__ uint64_t tab_bar;
+  __shared__ int tab_abort;
+  if (*a.valid != 1) return;
+  static_assert(CDF_SMEM_BYTES % 16 == 0 && LUT_SMEM_BYTES % 16 == 0 && TAIL_SMEM_BYTES % 16 == 0, "bulk sizes");
+  if (!bulk_load_tables(sm, a.dcdf, a.lut, a.tail, a.kept_scale, &tab_bar, &tab_abort)) {
+    if (threadIdx.x == 0) {
+      atomicExch(a.status, DCKV_ETIMEOUT);
+      mbar_drain(&tab_bar, 0);  // the CTA's shared memory stays allocated until its copies land
+    }
+    return;
+  }
+  const int lane = threadIdx.x & 31;
+  // chunk wi goes to block wi % gridDim.x: consecutive chunks land on different SMs
+  for (int wi = (threadIdx.x >> 5) * gridDim.x + blockIdx.x; wi < a.n_chunks; wi += gridDim.x * DEC_WARPS)
+    decode_chunk<BIG_K>(a, a.chunk0 + wi, lane, s_scale, s_cdf, s_lut, s_tail);
+}
+
 // Finishing a decoded pass in two steps.  k_codes_elem writes code = centre + symbol - 254
 // for every symbol of the pass's rows, fully parallel (fp16 to q16; even rows also bf16 to
 // qe, the odd mean model's input); an ESC symbol only flags its chunk.  (The odd pass of a
@@ -674,7 +687,7 @@ __global__ void __launch_bounds__(RANS_WARPS * 32) rans_decode_kernel(RansDecArg
 __global__ void __launch_bounds__(256) k_codes_elem(int parity, int64_t n_rows, const int32_t *row_edst,
                                                     const int32_t *row_slot, const int32_t *slot_chunk,
                                                     const uint16_t *syms, const int8_t *cen8,
-                                                    const int16_t *kept_list, int k_eff, __half *q16,
+                                                    int kw, int k_eff, __half *q16,
                                                     __nv_bfloat16 *qe, uint32_t *escflag, const int32_t *valid) {
   if (*valid != 1) return;
   constexpr int PER = N_COEF / 256;  // blockDim.x == 256
@@ -684,13 +697,12 @@ __global__ void __launch_bounds__(256) k_codes_elem(int parity, int64_t n_rows, 
     const int64_t slot = row_slot[r];
     const uint16_t *sy = syms + slot * k_eff;
     const int8_t *ce = cen8 + slot * k_eff;
-    int sv[PER], cv[PER], kl[PER];
+    int sv[PER], cv[PER];
 #pragma unroll
     for (int u = 0; u < PER; ++u) {  // every load before the stores
       const int k = threadIdx.x + 256 * u;
       sv[u] = k < k_eff ? (int)__ldg(sy + k) : 0;
       cv[u] = k < k_eff ? (int)__ldg(ce + k) : 0;
-      kl[u] = k < k_eff ? (int)__ldg(kept_list + k) : 0;
     }
     bool esc = false;
 #pragma unroll
@@ -702,8 +714,8 @@ __global__ void __launch_bounds__(256) k_codes_elem(int parity, int64_t n_rows, 
         continue;
       }
       const int q = sv[u] - R_MAX + cv[u];
-      q16[r * N_COEF + kl[u]] = __float2half_rn((float)q);
-      if (e >= 0) qe[(int64_t)e * N_COEF + kl[u]] = __float2bfloat16_rn((float)q);
+      q16[r * kw + k] = __float2half_rn((float)q);
+      if (e >= 0) qe[(int64_t)e * kw + k] = __float2bfloat16_rn((float)q);
     }
     if (__syncthreads_or(esc) && threadIdx.x == 0) escflag[slot_chunk[slot]] = 1u;
   }
@@ -714,7 +726,7 @@ struct DecCodesArgs {
   const PromptInfo *prompts;
   int chunk0, n_chunks;
   int k_eff;
-  const int16_t *kept_list;
+  int kw;                   // width of q16, qe, qbig (kept components, compact order)
   const uint16_t *syms;     // slot order
   const uint8_t *blob;
   uint64_t off_streams;
@@ -777,12 +789,12 @@ __global__ void __launch_bounds__(PATCH_THREADS) k_escape_patch(DecCodesArgs a) 
         bad = true;
       }
       const int rl = (int)(i / K);
-      const int comp = a.kept_list[i - (int64_t)rl * K];
+      const int k = (int)(i - (int64_t)rl * K);
       const int64_t row = (int64_t)pi.row_base + 2 * (cd.j0 + rl) + cd.parity;
-      a.q16[row * N_COEF + comp] = __float2half_rn((float)q);
-      if (cd.parity == 0) a.qe[(int64_t)(pi.ebase + cd.j0 + rl) * N_COEF + comp] = __float2bfloat16_rn((float)q);
+      a.q16[row * a.kw + k] = __float2half_rn((float)q);
+      if (cd.parity == 0) a.qe[(int64_t)(pi.ebase + cd.j0 + rl) * a.kw + k] = __float2bfloat16_rn((float)q);
       if (q >= BIG_CODE || q <= -BIG_CODE) {
-        a.qbig[row * N_COEF + comp] = q;
+        a.qbig[row * a.kw + k] = q;
         if (atomicExch(&a.bigflag[row], 1u) == 0u) a.biglist[atomicAdd(a.bigcount, 1u)] = (int32_t)row;
       }
     }

@@ -28,9 +28,10 @@ def codec_literal(src):
 
 @pytest.fixture(scope="session")
 def codec_55(src):
+    """The ~220 B/token codec of the single 4,096-token configuration (calibrated step scale)."""
     import dckv_synth
 
-    return dckv_synth.codec(src, step_scale=None, target_bytes=220.0)
+    return dckv_synth.calibrated_codec(src, 220.0, 16)
 
 
 @pytest.fixture(scope="session")

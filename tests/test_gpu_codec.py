@@ -66,7 +66,7 @@ def encode_gpu(gc, x, tok, offs):
     v = D.dckv_ws_offsets(gc.handle, offs, 0)
     ws = gc._ws
     n, ne = v["n_rows"], v["ne_pad"]
-    q32 = ws[v["q32"]: v["q32"] + 4 * n * 2048].view(torch.int32).reshape(n, 2048).cpu().numpy()
+    q32 = gc.workspace_codes(offs, 0)
     K = gc.k_eff
     cen8 = ws[v["cen8"]: v["cen8"] + n * K].view(torch.int8).reshape(n, K).cpu().numpy()
     row_slot = ws[v["row_slot"]: v["row_slot"] + 4 * n].view(torch.int32).cpu().numpy()
@@ -80,7 +80,7 @@ def decode_gpu(gc, blob_dev, size, tok, offs):
     torch.cuda.synchronize()
     w = D.dckv_ws_offsets(gc.handle, offs, 1)
     n = w["n_rows"]
-    q16 = gc._ws[w["q16"]: w["q16"] + 2 * n * 2048].view(torch.float16).reshape(n, 2048).float().cpu().numpy()
+    q16 = gc.workspace_codes(offs, 1)
     return k, v, int(gc.status.item()), q16
 
 
@@ -152,6 +152,72 @@ def rel_frob(a, b):
     return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30))
 
 
+def token_rows(k_bits, v_bits, tok_idx):
+    """Rows of the [6][T][2][256] K and V outputs at the given token indices, as fp64
+    [rows][2 * 6,144] (K then V)."""
+    kk = O.bf16_to_f64(k_bits[:, tok_idx]).transpose(1, 0, 2, 3).reshape(len(tok_idx), -1)
+    vv = O.bf16_to_f64(v_bits[:, tok_idx]).transpose(1, 0, 2, 3).reshape(len(tok_idx), -1)
+    return np.concatenate([kk, vv], axis=1)
+
+
+def row_errors(got, want):
+    """(relative Frobenius error over all the given rows, largest relative error of one
+    row) for fp64 rows [rows][d]."""
+    if got.shape[0] == 0:
+        return 0.0, 0.0
+    d = np.linalg.norm(got - want, axis=1)
+    w = np.linalg.norm(want, axis=1)
+    frob = float(np.sqrt(np.sum(d * d)) / max(np.sqrt(np.sum(w * w)), 1e-30))
+    return frob, float(np.max(d / np.maximum(w, 1e-30)))
+
+
+def coded_token_index(lay):
+    """Token indices of every coded row of a batch (prompt order, row order)."""
+    parts = [np.arange(L["tok_base"] + 4, L["tok_base"] + 4 + L["n"]) for L in lay]
+    return np.concatenate(parts) if parts else np.zeros(0, np.int64)
+
+
+def check_rows(k, v, k_o, v_o, lay, q_gpu, cod, dec_aux, centre_mismatches):
+    """Decoded rows against the oracle.
+    (1) The spec measure: relative Frobenius error against the oracle's decode of the
+        same blob, within 1e-3, taken over the coded rows alone (kept rows are stored
+        verbatim and would dilute it).
+    (2) The oracle's decoder computes its own centres; where one differs by one from the
+        centre the GPU encoder coded with (the 1e-4 rule of check_centres), the oracle
+        decodes that code one off.  So its codes must equal the GPU's except for at most
+        that many +-1 differences.
+    (3) Every coded row on its own: the oracle's reconstruction of the GPU's codes (RoPE,
+        bf16) against the GPU's row, relative error within 1e-3 for the worst row.
+    (4) Kept rows on their own, row by row, against the oracle's decode.
+    Returns (Frobenius error, worst row error)."""
+    kg, vg = bits(k), bits(v)
+    idx = coded_token_index(lay)
+    got = token_rows(kg, vg, idx)
+    frob, _ = row_errors(got, token_rows(k_o, v_o, idx))
+    assert frob <= ROW_TOL, frob
+    n_diff = 0
+    for L, qe, qo in zip(lay, dec_aux["qe"], dec_aux["qo"]):
+        q = np.zeros((L["n"], 2048), np.int64)
+        q[0::2], q[1::2] = qe, qo
+        d = q - q_gpu[L["row_base"]: L["row_base"] + L["n"]]
+        assert np.all(np.abs(d) <= 1), "oracle decode differs from the GPU's codes by more than one step"
+        n_diff += int(np.count_nonzero(d))
+    assert n_diff <= centre_mismatches, (n_diff, centre_mismatches)
+    if idx.size:
+        pos = np.concatenate([np.arange(4, 4 + L["n"]) for L in lay])
+        want = O.f64_to_bf16(O.output_rows(O.reconstruct(q_gpu.astype(np.int64), cod), pos)).reshape(-1, 6, 2, 2, 256)
+        want = np.concatenate([O.bf16_to_f64(want[:, :, 0]).reshape(idx.size, -1),
+                               O.bf16_to_f64(want[:, :, 1]).reshape(idx.size, -1)], axis=1)
+        _, worst = row_errors(got, want)
+        assert worst <= ROW_TOL, worst
+    else:
+        worst = 0.0
+    kept = np.setdiff1d(np.arange(kg.shape[1]), idx)
+    kf, kw = row_errors(token_rows(kg, vg, kept), token_rows(k_o, v_o, kept))
+    assert kf <= ROW_TOL and kw <= ROW_TOL, (kf, kw)
+    return frob, worst
+
+
 def full_check(src, np_codec, lens, seeds, chunk_rows=0, boost=(), boost_gain=60.0, student_t=0.0,
                expect_escapes=False, expect_big=False):
     gc = gpu_codec(np_codec, chunk_rows)
@@ -185,12 +251,11 @@ def full_check(src, np_codec, lens, seeds, chunk_rows=0, boost=(), boost_gain=60
     assert np.array_equal(q16[small], res["q32"][small].astype(np.float32))
     if expect_big:
         assert (~small).any()
-    k_o, v_o = O.decode(res["blob"], tok.cpu().numpy(), offs, np_codec)
-    kg, vg = bits(k), bits(v)
-    for g, o in ((kg, k_o), (vg, v_o)):
-        e = rel_frob(O.bf16_to_f64(g), O.bf16_to_f64(o))
-        assert e <= ROW_TOL, e
-    return dict(gc=gc, x=x, tok=tok, offs=offs, res=res, flips=flips, centre_mismatch=mism, k=k, v=v, aux=aux)
+    dec_aux = {}
+    k_o, v_o = O.decode(res["blob"], tok.cpu().numpy(), offs, np_codec, aux=dec_aux)
+    row_frob, row_worst = check_rows(k, v, k_o, v_o, O.prompt_layout(np.diff(offs)), res["q32"], np_codec,
+                                     dec_aux, mism)
+    return dict(row_frob=row_frob, row_worst=row_worst, gc=gc, x=x, tok=tok, offs=offs, res=res, flips=flips, centre_mismatch=mism, k=k, v=v, aux=aux)
 
 
 # ------------------------------------------------------------------------------------ tests
@@ -345,55 +410,138 @@ def test_capacity_error(src, codec_55):
                       torch.empty(1024, dtype=torch.uint8, device="cuda"))
 
 
-def test_full_size_4k_prompt_sampled(src, codec_55):
-    """4,096-token prompt at about 220 B/token, in the configuration the benchmark times:
-    sampled rows against the oracle, every chunk's section re-coded by the oracle coder,
-    and the payload against the model code length."""
-    gc = gpu_codec(codec_55)
-    x, tok, offs = make_batch(src, codec_55, [4096], [100])
-    res = encode_gpu(gc, x, tok, offs)
-    assert res["status"] == D.DCKV_OK
-    n = 4096 - 132
-    rng = np.random.default_rng(0)
-    rows = np.sort(rng.choice(n, 48, replace=False))
+def sample_rows(lay, rng, n_random, chunk_rows):
+    """Coded rows (batch-wide indices) for the full-size checks: n_random drawn at random,
+    plus in every prompt its first three and last three coded rows (both parities at both
+    ends, the last odd row's missing right neighbour included), the rows on both sides of
+    the first chunk boundary of each parity, and the rows around every multiple of 2^16
+    of the prompt's own and of the batch-wide coded-row index."""
+    n = sum(L["n"] for L in lay)
+    picks = set(int(r) for r in rng.choice(n, min(n_random, n), replace=False)) if n else set()
+    for L in lay:
+        m, b = L["n"], L["row_base"]
+        rel = {0, 1, 2, m - 3, m - 2, m - 1}
+        g = 2 * chunk_rows  # first row of the second chunk of each parity: 2G (even), 2G + 1 (odd)
+        rel |= {g - 2, g - 1, g, g + 1}
+        for mark in range(1 << 16, m + 2, 1 << 16):
+            rel |= {mark - 2, mark - 1, mark, mark + 1}
+        picks |= {b + j for j in rel if 0 <= j < m}
+    for mark in range(1 << 16, n + 2, 1 << 16):
+        picks |= {r for r in (mark - 2, mark - 1, mark, mark + 1) if 0 <= r < n}
+    return np.array(sorted(picks), np.int64)
+
+
+def check_sampled(gc, cod, res, x, tok, offs, rows, k, v):
+    """Full-size parity on selected coded rows (batch-wide indices):
+    codes     the oracle's transform and quantiser on the rows' inputs (flip rule);
+    centres   the oracle's mean models on the rows' tokens and, for odd rows, the GPU's
+              own codes of both even neighbours (zero past a prompt's last even row),
+              against the GPU encoder's centres (1e-4 rule); encoder and decoder share
+              the tables, so this is what catches a centre both would get wrong;
+    rows      the oracle's reconstruction of the GPU's codes, RoPE'd at each row's
+              position, against the decoded K and V: relative Frobenius over the rows and
+              the largest single-row error, both within 1e-3.
+    Returns (flips, centre mismatches, row Frobenius error, worst row error)."""
+    lay = O.prompt_layout(np.diff(offs))
+    starts = np.array([L["row_base"] for L in lay])
+    pidx = np.searchsorted(starts, rows, side="right") - 1
+    rel = rows - starts[pidx]
+    tbase = np.array([L["tok_base"] for L in lay])[pidx]
+    tok_rows = tbase + 4 + rel
     xb = bits(x)
-    y = O.transform(xb[4 + rows], codec_55)
-    q_o, ratio = O.quantise(y, codec_55.delta, O.scale_index(codec_55.laplace_b, codec_55.delta)[1])
-    check_codes(res["q32"][rows].astype(np.int64), dict(q=q_o, ratio=ratio))
-    codes = split_gpu_codes(gc, codec_55, res, tok, offs)
-    # the whole blob from the GPU's codes and centres through the oracle coder
-    aux = {}
+    keep = O.scale_index(cod.laplace_b, cod.delta)[1]
+    q_o, ratio = O.quantise(O.transform(xb[tok_rows], cod), cod.delta, keep)
+    q_gpu = res["q32"][rows].astype(np.int64)
+    flips = check_codes(q_gpu, dict(q=q_o, ratio=ratio))
+    # centres
+    tok_np = tok.cpu().numpy().astype(np.int64)
+    n_rel = np.array([L["n"] for L in lay])[pidx]
+    mism = 0
+    for par in (0, 1):
+        sel = np.nonzero((rel & 1) == par)[0]
+        if sel.size == 0:
+            continue
+        toks = tok_np[tok_rows[sel]]
+        if par == 0:
+            mu = O.codec_means_even(cod, toks)
+        else:
+            left = res["q32"][rows[sel] - 1].astype(np.int64)
+            has_right = rel[sel] + 1 < n_rel[sel]
+            right = np.zeros((sel.size, 2048), np.int64)
+            right[has_right] = res["q32"][rows[sel][has_right] + 1]
+            mu = O.codec_means_odd(cod, toks, left, right)
+        ora_c = O.centres(mu)[:, keep]
+        gpu_c = res["cen"][rows[sel]].astype(np.int64)
+        bad = ora_c != gpu_c
+        if bad.any():
+            assert np.all(np.abs(ora_c[bad] - gpu_c[bad]) == 1)
+            assert np.all(near_half(mu[:, keep][bad], CENTRE_WINDOW)), "centre differs away from a boundary"
+        mism += int(bad.sum())
+    assert mism <= 1e-4 * max(1, rows.size * int(keep.sum()))
+    # decoded rows
+    xh = O.reconstruct(q_gpu, cod)
+    want = O.output_rows(xh, 4 + rel)
+    want = O.bf16_to_f64(O.f64_to_bf16(want)).reshape(-1, 6, 2, 2, 256)
+    want = np.concatenate([want[:, :, 0].reshape(rows.size, -1), want[:, :, 1].reshape(rows.size, -1)], axis=1)
+    frob, worst = row_errors(token_rows(bits(k), bits(v), tok_rows), want)
+    assert frob <= ROW_TOL, frob
+    assert worst <= ROW_TOL, worst
+    return flips, mism, frob, worst
+
+
+def full_size_check(src, cod, lens, seeds, chunk_rows, student_t=0.0, n_random=320):
+    """One full-size configuration: sampled rows against the oracle (check_sampled), the
+    whole blob re-coded by the oracle coder from the GPU's codes and centres, the payload
+    against the model code length, and the exact code round trip through the GPU decoder."""
+    gc = gpu_codec(cod, chunk_rows)
+    x, tok, offs = make_batch(src, cod, lens, seeds, student_t=student_t)
+    res = encode_gpu(gc, x, tok, offs)
+    assert res["status"] == D.DCKV_OK, D.STATUS_NAMES[res["status"]]
+    lay = O.prompt_layout(np.diff(offs))
     G = D.dckv_codec_info(gc.handle)["chunk_rows"]
-    ora_blob = O.assemble_blob(xb, offs, codes, codec_55.laplace_b, codec_55.delta, G, aux=aux)
-    assert ora_blob == res["blob"]
-    payload = res["size"] - 132 * 12288
-    model_bytes = aux["code_bits"] / 8
-    assert payload <= 1.05 * model_bytes, (payload, model_bytes)
-    assert 150 <= payload / n <= 300
-    k, v, st, q16 = decode_gpu(gc, res["blob_dev"], res["size"], tok, offs)
-    assert st == D.DCKV_OK
-    assert np.array_equal(q16, res["q32"].astype(np.float32))
-    # sampled decoded rows against the oracle's reconstruction of the same codes
-    xh = O.reconstruct(res["q32"][rows].astype(np.int64), codec_55)
-    want = O.f64_to_bf16(O.output_rows(xh, 4 + rows)).reshape(-1, 6, 2, 2, 256)
-    kg = bits(k)[:, 4 + rows].transpose(1, 0, 2, 3)
-    vg = bits(v)[:, 4 + rows].transpose(1, 0, 2, 3)
-    assert rel_frob(O.bf16_to_f64(kg), O.bf16_to_f64(want[:, :, 0])) <= ROW_TOL
-    assert rel_frob(O.bf16_to_f64(vg), O.bf16_to_f64(want[:, :, 1])) <= ROW_TOL
+    assert G == (chunk_rows or 16)
+    codes = split_gpu_codes(gc, cod, res, tok, offs)
+    aux = {}
+    ora_blob = O.assemble_blob(bits(x), offs, codes, cod.laplace_b, cod.delta, G, aux=aux)
+    assert len(ora_blob) == res["size"] and ora_blob == res["blob"]
+    kept = sum(L["N"] - L["n"] for L in lay)
+    payload = res["size"] - kept * 12288
+    assert payload <= 1.05 * aux["code_bits"] / 8, (payload, aux["code_bits"] / 8)
+    if student_t > 0:
+        assert aux["n_esc"] > 0  # heavy-tailed rows force escapes
+    k, v, status, q16 = decode_gpu(gc, res["blob_dev"], res["size"], tok, offs)
+    assert status == D.DCKV_OK
+    small = np.abs(res["q32"]) < 2048
+    assert np.array_equal(q16[small], res["q32"][small].astype(np.float32))
+    rows = sample_rows(lay, np.random.default_rng(sum(seeds)), n_random, G)
+    flips, mism, frob, worst = check_sampled(gc, cod, res, x, tok, offs, rows, k, v)
+    n = sum(L["n"] for L in lay)
+    print(f"{len(lens)} x {lens[0]}: {rows.size} sampled rows, {flips} flips, {mism} centre mismatches, "
+          f"rows {frob:.2e} (worst {worst:.2e}), payload {payload / n:.1f} B/row, {aux['n_esc']} escapes")
+    return dict(res=res, aux=aux, payload=payload, n=n, rows=rows)
+
+
+def test_full_size_4k_prompt_sampled(src, codec_55):
+    """4,096-token prompt at about 220 B/token: sampled and boundary rows against the
+    oracle (codes, centres, decoded rows), every chunk re-coded by the oracle coder, and
+    the payload against the model code length."""
+    r = full_size_check(src, codec_55, [4096], [100], 0)
+    assert 150 <= r["payload"] / r["n"] <= 300
 
 
 _FULL_CODECS = {}
 
 
-def _full_codec(src, target):
-    if target not in _FULL_CODECS:
-        _FULL_CODECS[target] = S.codec(src, step_scale=None, target_bytes=target)
-    return _FULL_CODECS[target]
+def _full_codec(src, target, chunk_rows, student_t):
+    key = (target, chunk_rows, student_t)
+    if key not in _FULL_CODECS:
+        _FULL_CODECS[key] = S.calibrated_codec(src, target, chunk_rows, student_t)
+    return _FULL_CODECS[key]
 
 
 # the larger configurations: (prompt lengths, target bytes per coded row, Student-t fraction,
-# rows per rANS chunk).  At ~110 B per row a chunk's fixed 136 bytes need 32 rows to stay
-# within the 5% payload bound.
+# rows per rANS chunk), each with the step scale calibrated for its rate.  At ~110 B per row a
+# chunk's fixed 136 bytes need 32 rows to stay within the 5% payload bound.
 FULL_CONFIGS = {
     "32k_220B": ([32768], 220.0, 0.0, 16),
     "32k_110B": ([32768], 110.0, 0.0, 32),
@@ -404,49 +552,16 @@ FULL_CONFIGS = {
 
 @pytest.mark.parametrize("name", sorted(FULL_CONFIGS))
 def test_full_size_configs_sampled(src, name):
-    """Full-size configurations: sampled rows' codes against the oracle, the whole blob
-    re-coded by the oracle coder from the GPU's codes and centres, the payload against the
-    model code length, exact code round trip through the GPU decoder, and sampled decoded
-    rows against the oracle's reconstruction."""
+    """Full-size configurations: sampled rows plus every prompt's boundary rows and the
+    rows around each 2^16 mark against the oracle (codes, centres, decoded rows), the whole
+    blob re-coded by the oracle coder, the payload against the model code length, and the
+    exact code round trip through the GPU decoder."""
     lens, target, st, chunk_rows = FULL_CONFIGS[name]
-    cod = _full_codec(src, target)
-    gc = gpu_codec(cod, chunk_rows)
+    cod = _full_codec(src, target, chunk_rows, st)
     seeds = [200 + 7 * i for i in range(len(lens))]
-    x, tok, offs = make_batch(src, cod, lens, seeds, student_t=st)
-    res = encode_gpu(gc, x, tok, offs)
-    assert res["status"] == D.DCKV_OK, D.STATUS_NAMES[res["status"]]
-    lay = O.prompt_layout(np.diff(offs))
-    n = sum(L["n"] for L in lay)
-    rng = np.random.default_rng(1)
-    rows = np.sort(rng.choice(n, 48, replace=False))  # coded-row indices over the batch
-    starts = np.array([L["row_base"] for L in lay])
-    pidx = np.searchsorted(starts, rows, side="right") - 1
-    tok_rows = np.array([lay[p]["tok_base"] + 4 + (r - lay[p]["row_base"]) for p, r in zip(pidx, rows)])
-    pos = np.array([4 + (r - lay[p]["row_base"]) for p, r in zip(pidx, rows)])
-    xb = bits(x)
-    keep = O.scale_index(cod.laplace_b, cod.delta)[1]
-    q_o, ratio = O.quantise(O.transform(xb[tok_rows], cod), cod.delta, keep)
-    check_codes(res["q32"][rows].astype(np.int64), dict(q=q_o, ratio=ratio))
-    codes = split_gpu_codes(gc, cod, res, tok, offs)
-    aux = {}
-    G = D.dckv_codec_info(gc.handle)["chunk_rows"]
-    ora_blob = O.assemble_blob(xb, offs, codes, cod.laplace_b, cod.delta, G, aux=aux)
-    assert len(ora_blob) == res["size"] and ora_blob == res["blob"]
-    kept = sum(L["N"] - L["n"] for L in lay)
-    payload = res["size"] - kept * 12288
-    assert payload <= 1.05 * aux["code_bits"] / 8, (payload, aux["code_bits"] / 8)
-    if st > 0:
-        assert aux["n_esc"] > 0  # heavy-tailed rows force escapes
-    k, v, status, q16 = decode_gpu(gc, res["blob_dev"], res["size"], tok, offs)
-    assert status == D.DCKV_OK
-    small = np.abs(res["q32"]) < 2048
-    assert np.array_equal(q16[small], res["q32"][small].astype(np.float32))
-    xh = O.reconstruct(res["q32"][rows].astype(np.int64), cod)
-    want = O.f64_to_bf16(O.output_rows(xh, pos)).reshape(-1, 6, 2, 2, 256)
-    kg = bits(k)[:, tok_rows].transpose(1, 0, 2, 3)
-    vg = bits(v)[:, tok_rows].transpose(1, 0, 2, 3)
-    assert rel_frob(O.bf16_to_f64(kg), O.bf16_to_f64(want[:, :, 0])) <= ROW_TOL
-    assert rel_frob(O.bf16_to_f64(vg), O.bf16_to_f64(want[:, :, 1])) <= ROW_TOL
+    r = full_size_check(src, cod, lens, seeds, chunk_rows, student_t=st)
+    # the calibrated step scale puts the payload near the configuration's rate
+    assert abs(r["payload"] / r["n"] / target - 1.0) <= 0.05, r["payload"] / r["n"]
 
 
 @pytest.mark.parametrize("which", ["literal", "fitted"])
