@@ -17,19 +17,19 @@ extern "C" {
 #endif
 
 /* Byte offsets (from the workspace base) of the intermediates of one call shape.
- * which = 0: encode layout, 1: decode layout.  Code arrays hold the kept components only,
- * in ascending component order (column m is the m-th kept component), code_width columns
- * wide (K_eff rounded up to 64; the columns past K_eff are 0); dropped components have
- * code 0.  After dckv_encode on a stream:
- *   q32  int32 [n_rows][code_width] codes q = round(y / Delta), rows in prompt order,
- *        coded rows only (positions 4 .. N-129 of each prompt);
- *   qe   bf16 [ne_pad][code_width] even-row codes, one extra zero row after each prompt;
+ * which = 0: encode layout, 1: decode layout.  Code arrays have rows of 2048 entries that
+ * hold the kept components only, in ascending component order (column m is the m-th kept
+ * component); code_width columns are in use (K_eff rounded up to 64, zero past K_eff) and
+ * dropped components have code 0.  After dckv_encode on a stream:
+ *   q32  int32 [n_rows][2048] codes q = round(y / Delta), rows in prompt order, coded rows
+ *        only (positions 4 .. N-129 of each prompt);
+ *   qe   bf16 [ne_pad][2048] even-row codes, one extra zero row after each prompt;
  *   cen8 int8 [n_rows][K_eff] centres in slot order: slot row row_slot[r] of coded row r
  *        (chunk order: every even row of every prompt, then every odd row), kept
  *        components in ascending order;
  *   sym16 uint16 [n_rows][K_eff] symbols in the same order;
  *   row_slot int32 [n_rows].
- * After dckv_decode: q16 fp16 [n_rows][code_width] decoded codes (exact below 2048), qe, cen8.
+ * After dckv_decode: q16 fp16 [n_rows][2048] decoded codes (exact below 2048), qe, cen8.
  * Encode recomputes in fp64 every code whose fp32 ratio y / Delta lies in a guard band
  * around a half-step boundary (whole rows when the row's norm is large). */
 typedef struct {

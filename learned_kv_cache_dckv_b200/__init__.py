@@ -393,11 +393,11 @@ class Codec:
         if None)."""
         torch = self.torch
         v = dckv_ws_offsets(self.handle, seq_offsets, which)
-        n, kw, k = v["n_rows"], v["code_width"], self.k_eff
+        n, k = v["n_rows"], self.k_eff
         if which == 0:
-            c = self._ws[v["q32"]: v["q32"] + 4 * n * kw].view(torch.int32).reshape(n, kw)
+            c = self._ws[v["q32"]: v["q32"] + 4 * n * 2048].view(torch.int32).reshape(n, 2048)
         else:
-            c = self._ws[v["q16"]: v["q16"] + 2 * n * kw].view(torch.float16).reshape(n, kw).float()
+            c = self._ws[v["q16"]: v["q16"] + 2 * n * 2048].view(torch.float16).reshape(n, 2048).float()
         if rows is not None:
             c = c[torch.as_tensor(np.asarray(rows, np.int64), device=c.device)]
         c = c[:, :k].cpu().numpy()

@@ -115,11 +115,12 @@ static int map_a(CUtensorMap *m, const void *ptr, bool bf16, uint64_t K, uint64_
 }
 
 // B operand: [rows][K] (K contiguous), box {64, bn}, 128-byte swizzle, zero fill past the end.
-static int map_b(CUtensorMap *m, const void *ptr, bool bf16, uint64_t K, uint64_t rows, int bn) {
+// B operand [rows][K] of 16-bit values, rows ld elements apart (ld = K when 0)
+static int map_b(CUtensorMap *m, const void *ptr, bool bf16, uint64_t K, uint64_t rows, int bn, uint64_t ld = 0) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(DCKV_ECUDA, "cuTensorMapEncodeTiled unavailable");
   cuuint64_t dims[2] = {K, rows};
-  cuuint64_t strides[1] = {K * 2};
+  cuuint64_t strides[1] = {(ld ? ld : K) * 2};
   cuuint32_t box[2] = {(cuuint32_t)GEMM_BK, (cuuint32_t)bn};
   cuuint32_t es[2] = {1, 1};
   CUresult r = fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
@@ -511,7 +512,7 @@ __global__ void k_layout(const PromptInfo *prompts, int32_t *row_tok, int32_t *r
   }
   if (qe_zero_pad)  // the row after a prompt's last even row is its odd rows' zero right neighbour
     for (int k = t0; k < kw; k += ts)
-      qe_zero_pad[(int64_t)(pi.ebase + pi.n_e) * kw + k] = __float2bfloat16_rn(0.f);
+      qe_zero_pad[(int64_t)(pi.ebase + pi.n_e) * CODE_LD + k] = __float2bfloat16_rn(0.f);
 }
 
 __device__ __forceinline__ int find_prompt(const PromptInfo *p, int batch, int64_t tok) {
@@ -699,8 +700,8 @@ __global__ void __launch_bounds__(256) k_fixup(const int32_t *biglist, const uin
   for (uint32_t li = blockIdx.x; li < n; li += gridDim.x) {
     const int64_t r = biglist[li];
     for (int m = threadIdx.x; m < kw; m += blockDim.x) {  // codes of the kept components, compact order
-      float v = __half2float(q16[r * kw + m]);
-      if (fabsf(v) >= (float)BIG_CODE) v = (float)qbig[r * kw + m];
+      float v = __half2float(q16[r * CODE_LD + m]);
+      if (fabsf(v) >= (float)BIG_CODE) v = (float)qbig[r * CODE_LD + m];
       qs[m] = v;
     }
     __syncthreads();
@@ -772,14 +773,14 @@ __device__ __forceinline__ double warp_sum(double v) {
   return v;
 }
 
-// code of compact component m of a row (code arrays kw wide)
+// code of compact component m of a row
 __device__ __forceinline__ void store_code(int64_t row, int m, double ratio, int32_t *q32, __nv_bfloat16 *qe,
-                                           const int32_t *row_edst, int kw) {
+                                           const int32_t *row_edst) {
   const double qd = fmin(fmax(rint(ratio), -2147483648.0), 2147483647.0);
   const int q = (int)qd;
-  q32[row * kw + m] = q;
+  q32[row * CODE_LD + m] = q;
   const int e = row_edst[row];
-  if (e >= 0) qe[(int64_t)e * kw + m] = __float2bfloat16_rn((float)q);
+  if (e >= 0) qe[(int64_t)e * CODE_LD + m] = __float2bfloat16_rn((float)q);
 }
 
 // bf16 bits to fp64, exactly: the sign, exponent and mantissa fields move into place
@@ -856,7 +857,7 @@ constexpr int REFINE_SMEM = ROW_DIM * 8 + (N_COEF + 1) * 4;
 __global__ void __launch_bounds__(REFINE_THREADS) k_refine_codes(
     const uint32_t *el_bins, const uint32_t *bin_count, uint32_t bin_cap, const __nv_bfloat16 *rows,
     const int32_t *row_tok, const double *mub64, const float *bt32, const float *w2t32, const __half *g16,
-    const float *delta, const uint32_t *rowflag, const int16_t *kept_list, int kw, int32_t *q32, __nv_bfloat16 *qe,
+    const float *delta, const uint32_t *rowflag, const int16_t *kept_list, int32_t *q32, __nv_bfloat16 *qe,
     const int32_t *row_edst) {
   extern __shared__ __align__(16) double bs[];
   uint32_t *item0 = reinterpret_cast<uint32_t *>(bs + ROW_DIM);  // [2049] first item of each bin
@@ -927,7 +928,7 @@ __global__ void __launch_bounds__(REFINE_THREADS) k_refine_codes(
           acc += h;
         }
         acc = warp_sum(acc) - mub64[c];
-        if (lane == 0) store_code(row, m, acc / (double)delta[c], q32, qe, row_edst, kw);
+        if (lane == 0) store_code(row, m, acc / (double)delta[c], q32, qe, row_edst);
       }
     }
     __syncthreads();
@@ -969,7 +970,7 @@ __global__ void __launch_bounds__(256) k_refine_rows(const uint32_t *full_list, 
                                                      const __nv_bfloat16 *rows, const int32_t *row_tok,
                                                      const double *mub64, const float *bt32, const float *w2t32,
                                                      const double *g64, const float *delta, const int16_t *kept_list,
-                                                     int k_eff, int kw, int32_t *q32, __nv_bfloat16 *qe,
+                                                     int k_eff, int32_t *q32, __nv_bfloat16 *qe,
                                                      const int32_t *row_edst) {
   extern __shared__ __align__(16) double xs[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -989,7 +990,7 @@ __global__ void __launch_bounds__(256) k_refine_rows(const uint32_t *full_list, 
         for (int h = lane; h < N_HIDDEN; h += 32) acc = fma(g[h], (double)w2t32[c * N_HIDDEN + h], acc);
       }
       acc = warp_sum(acc) - mub64[c];
-      if (lane == 0) store_code(row, m, acc / (double)delta[c], q32, qe, row_edst, kw);
+      if (lane == 0) store_code(row, m, acc / (double)delta[c], q32, qe, row_edst);
     }
     __syncthreads();
   }
@@ -1092,14 +1093,14 @@ static WsPlan plan_ws(const Layout &L, int which /*0 encode, 1 decode*/) {
   w.e_row = take(4ull * L.ne_pad);
   w.escflag = take(4ull * std::max(L.n_chunks, 1));
   w.slot_chunk = take(4ull * L.n_rows);
-  w.qe = take(2ull * L.ne_pad * L.kw);
+  w.qe = take(2ull * L.ne_pad * CODE_LD);
   w.cen8 = take(1ull * L.n_symbols);
   w.counters = take(256);
   if (which == 0) {
     w.x16 = take(2ull * L.n_rows * ROW_DIM);
     w.g16 = take(2ull * L.n_rows * 2 * N_HIDDEN);
     w.hpart = take(4ull * HIDDEN_SPLIT * L.n_rows * N_HIDDEN);
-    w.q32 = take(4ull * L.n_rows * L.kw);
+    w.q32 = take(4ull * L.n_rows * CODE_LD);
     w.sym16 = take(2ull * L.n_symbols);
     w.cf32 = take(8ull * L.n_symbols);
     w.words = take(2ull * L.n_symbols);
@@ -1120,8 +1121,8 @@ static WsPlan plan_ws(const Layout &L, int which /*0 encode, 1 decode*/) {
     w.slots16 = take(2ull * L.n_symbols);
     w.g16 = take(2ull * L.n_rows * 2 * N_HIDDEN);  // synthesis hidden units (hi/lo)
     w.rope = take(8ull * 128 * std::max<int64_t>(L.max_len, 1));
-    w.q16 = take(2ull * L.n_rows * L.kw);
-    w.qbig = take(4ull * L.n_rows * L.kw);
+    w.q16 = take(2ull * L.n_rows * CODE_LD);
+    w.qbig = take(4ull * L.n_rows * CODE_LD);
     w.bigflag = take(4ull * L.n_rows);
     w.biglist = take(4ull * L.n_rows);
   }
@@ -1605,7 +1606,7 @@ static int encode_impl(const dckv_codec *c, const void *rows, const int32_t *tok
     RET(map_b(&mb_xh, x16, false, ROW_DIM, L.n_rows, HIDDEN_SPLIT_BN / 2));
     RET(map_b(&mb_xt, x16, false, ROW_DIM, L.n_rows, TRANSFORM_BN / 2));
     RET(map_b(&mb_gt, g16, false, 2 * N_HIDDEN, L.n_rows, TRANSFORM_BN / 2));
-    RET(map_b(&mb_qe, qe, true, c->kw, L.ne_pad, MEAN_ODD_BN / 2));
+    RET(map_b(&mb_qe, qe, true, c->kw, L.ne_pad, MEAN_ODD_BN / 2, CODE_LD));
     // correction hidden layer: h = x @ w1 - mu @ w1, GELU, fp16 hi/lo
     if (c->has_mlp) {
       GemmProblem pr = make_problem(N_HIDDEN / GEMM_BM, L.n_rows, HIDDEN_SPLIT_BN, false, status_dev);
@@ -1626,7 +1627,7 @@ static int encode_impl(const dckv_codec *c, const void *rows, const int32_t *tok
         add_seg(pr, 1, 0, 2, 0, 1, 0, 0, N_HIDDEN / GEMM_BK);
         add_seg(pr, 1, 0, 2, 0, 1, 0, N_HIDDEN, N_HIDDEN / GEMM_BK);
       }
-      EpiQuantRegs::Params ep{{c->mub_k, c->delta_k, c->k_eff, c->kw, (float)std::ldexp(1.0, -c->p_y), q32, qe,
+      EpiQuantRegs::Params ep{{c->mub_k, c->delta_k, c->k_eff, (float)std::ldexp(1.0, -c->p_y), q32, qe,
                                row_edst},
                               row_norm, rowflag, el_bins, bin_count, full_list, counters, w.bin_cap,
                               c->dbg_ratio, c->kept_list};
@@ -1640,7 +1641,7 @@ static int encode_impl(const dckv_codec *c, const void *rows, const int32_t *tok
     CK(cudaFuncSetAttribute(k_refine_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, REFINE_SMEM));
     { k_refine_codes<<<c->num_sms * 3, REFINE_THREADS, REFINE_SMEM, st>>>(
           el_bins, bin_count, w.bin_cap, (const __nv_bfloat16 *)rows, row_tok, c->mub64, c->bt32,
-          c->has_mlp ? c->w2t32 : nullptr, g16, c->delta, rowflag, c->kept_list, c->kw, q32, qe, row_edst);
+          c->has_mlp ? c->w2t32 : nullptr, g16, c->delta, rowflag, c->kept_list, q32, qe, row_edst);
       ++g_launches; }
     stage_mark(c, st, "refine_codes");
     double *g64 = (double *)(ws + w.g64);
@@ -1650,7 +1651,7 @@ static int encode_impl(const dckv_codec *c, const void *rows, const int32_t *tok
     { k_refine_rows<<<c->num_sms * 4, 256, REFINE_SMEM, st>>>(full_list, counters, (const __nv_bfloat16 *)rows,
                                                             row_tok, c->mub64, c->bt32,
                                                             c->has_mlp ? c->w2t32 : nullptr, g64, c->delta,
-                                                            c->kept_list, c->k_eff, c->kw, q32, qe, row_edst);
+                                                            c->kept_list, c->k_eff, q32, qe, row_edst);
       ++g_launches; }
     CK(cudaGetLastError());
     stage_mark(c, st, "refine_rows");
@@ -1660,7 +1661,7 @@ static int encode_impl(const dckv_codec *c, const void *rows, const int32_t *tok
       GemmProblem pr = make_problem(c->mp / GEMM_BM, L.ne_pad, MEAN_ODD_BN, true, status_dev);
       add_seg(pr, 0, 0, 1, 0, 0, 0, 0, c->kw / GEMM_BK);
       add_seg(pr, 0, 0, 1, c->kw, 0, 1, 0, c->kw / GEMM_BK);
-      EpiMeanOdd<false>::Params ep{c->t_odd, token_ids, e_tok, e_slot, c->kept_list, cen8, c->k_eff, c->kw, c->vocab};
+      EpiMeanOdd<false>::Params ep{c->t_odd, token_ids, e_tok, e_slot, c->kept_list, cen8, c->k_eff, c->vocab};
       RET((run_gemm2<EpiMeanOdd<false>, 6, 1, 8, MEAN_ODD_BN>(c->map_aon1, c->map_aon1, mb_qe, mb_qe, pr, ep, c->num_sms, true, st)));
     }
     stage_mark(c, st, "gemm_mean_odd");
@@ -1669,7 +1670,7 @@ static int encode_impl(const dckv_codec *c, const void *rows, const int32_t *tok
     if (!c->has_means && L.n_symbols > 0)
       CK(cudaMemsetAsync(cen8, 0, (size_t)L.n_symbols, st));  // unconditional tables: every centre 0
     { k_symbols<<<rg, SYM_THREADS, 0, st>>>(L.n_rows, row_slot, slot_chunk, q32, cen8, c->kept_list, c->kept_scale,
-                                          c->cfm_tab, c->k_eff, c->kw, c->has_means ? c->t_even : nullptr, token_ids,
+                                          c->cfm_tab, c->k_eff, c->has_means ? c->t_even : nullptr, token_ids,
                                           row_tok, row_edst, c->vocab, sym16, cfm, nesc_w); ++g_launches; }
     CK(cudaGetLastError());
     stage_mark(c, st, "symbols");
@@ -1690,7 +1691,7 @@ static int encode_impl(const dckv_codec *c, const void *rows, const int32_t *tok
     CK(cudaGetLastError());
   }
   if (L.n_chunks > 0) {
-    CompactArgs a{d_chunks, d_prompts, L.n_chunks, c->k_eff, c->kw, q32, sym16,
+    CompactArgs a{d_chunks, d_prompts, L.n_chunks, c->k_eff, q32, sym16,
                   (const uint16_t *)(ws + w.words), states, nwords, nesc, offs, bl, blob_cap, L.off_streams};
     { compact_kernel<<<L.n_chunks, COMPACT_THREADS, 0, st>>>(a); ++g_launches; }
     CK(cudaGetLastError());
@@ -1745,9 +1746,9 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
   CK(cudaMemsetAsync(status_dev, 0, 4, st));
   CK(cudaMemsetAsync(counters, 0, 256, st));
   RET(upload_tables(c, L, ws, w, st));
-  CK(cudaMemsetAsync(qe, 0, 2ull * L.ne_pad * c->kw, st));
+  CK(cudaMemset2DAsync(qe, 2ull * CODE_LD, 0, 2ull * c->kw, (size_t)L.ne_pad, st));
   if (L.n_rows) {
-    CK(cudaMemsetAsync(q16, 0, 2ull * L.n_rows * c->kw, st));
+    CK(cudaMemset2DAsync(q16, 2ull * CODE_LD, 0, 2ull * c->kw, (size_t)L.n_rows, st));
     CK(cudaMemsetAsync(bigflag, 0, 4ull * L.n_rows, st));
   }
   if (L.n_chunks) CK(cudaMemsetAsync(ws + w.escflag, 0, 4ull * L.n_chunks, st));
@@ -1773,7 +1774,7 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
   RansDecArgs da{d_chunks, 0, L.n_chunks, c->k_eff, c->kept_scale, c->dcdf, c->lut, c->tail, bl, L.off_streams,
                  offs, syms16, valid, status_dev};
   uint32_t *escflag = (uint32_t *)(ws + w.escflag);
-  DecCodesArgs fa{d_chunks, d_prompts, 0, L.n_chunks_e, c->k_eff, c->kw, syms16, bl, L.off_streams,
+  DecCodesArgs fa{d_chunks, d_prompts, 0, L.n_chunks_e, c->k_eff, syms16, bl, L.off_streams,
                   offs, q16, qe, qbig, bigflag, biglist, counters, escflag, valid, status_dev};
   const unsigned rg = (unsigned)std::max<int64_t>(1, std::min<int64_t>(L.n_rows, 65535));
   if (L.n_chunks > 0) {
@@ -1787,7 +1788,7 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
   CK(cudaGetLastError());
   stage_mark(c, st, "rans_loop");
   if (L.n_chunks_e > 0) {
-    { k_codes_elem<<<rg, 256, 0, st>>>(0, L.n_rows, row_edst, row_slot, slot_chunk, syms16, cen8, c->kw,
+    { k_codes_elem<<<rg, 256, 0, st>>>(0, L.n_rows, row_edst, row_slot, slot_chunk, syms16, cen8,
                                        c->k_eff, q16, qe, escflag, valid); ++g_launches; }
     { k_escape_patch<<<(unsigned)L.n_chunks_e, PATCH_THREADS, 0, st>>>(fa); ++g_launches; }
   }
@@ -1795,19 +1796,19 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
   stage_mark(c, st, "codes_even");
   if (L.n_rows > 0 && c->has_means) {
     CUtensorMap mb_qe;
-    RET(map_b(&mb_qe, qe, true, c->kw, L.ne_pad, MEAN_ODD_BN / 2));
+    RET(map_b(&mb_qe, qe, true, c->kw, L.ne_pad, MEAN_ODD_BN / 2, CODE_LD));
     GemmProblem pr = make_problem(c->mp / GEMM_BM, L.ne_pad, MEAN_ODD_BN, true, status_dev);
     add_seg(pr, 0, 0, 1, 0, 0, 0, 0, c->kw / GEMM_BK);
     add_seg(pr, 0, 0, 1, c->kw, 0, 1, 0, c->kw / GEMM_BK);
     // odd centres, and with them the odd codes (ESC symbols are left to the patch)
-    EpiMeanOdd<true>::Params ep{c->t_odd, token_ids, e_tok, e_slot, c->kept_list, cen8, c->k_eff, c->kw, c->vocab,
+    EpiMeanOdd<true>::Params ep{c->t_odd, token_ids, e_tok, e_slot, c->kept_list, cen8, c->k_eff, c->vocab,
                                 syms16, q16, e_row, slot_chunk, escflag};
     RET((run_gemm2<EpiMeanOdd<true>, 6, 1, 8, MEAN_ODD_BN>(c->map_aon1, c->map_aon1, mb_qe, mb_qe, pr, ep, c->num_sms, true, st)));
   }
   stage_mark(c, st, "gemm_mean_odd");
   if (L.n_chunks_o > 0) {
     if (!c->has_means)  // unconditional tables: every odd centre is 0
-      { k_codes_elem<<<rg, 256, 0, st>>>(1, L.n_rows, row_edst, row_slot, slot_chunk, syms16, cen8, c->kw,
+      { k_codes_elem<<<rg, 256, 0, st>>>(1, L.n_rows, row_edst, row_slot, slot_chunk, syms16, cen8,
                                          c->k_eff, q16, qe, escflag, valid); ++g_launches; }
     fa.chunk0 = L.n_chunks_e;
     fa.n_chunks = L.n_chunks_o;
@@ -1818,7 +1819,7 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
   __half *g16d = (__half *)(ws + w.g16);
   if (L.n_rows > 0 && c->has_synth) {  // decoder-side synthesis, hidden layer: GELU((q Delta) V1)
     CUtensorMap mb_qh;
-    RET(map_b(&mb_qh, q16, false, c->kw, L.n_rows, HIDDEN_BN / 2));
+    RET(map_b(&mb_qh, q16, false, c->kw, L.n_rows, HIDDEN_BN / 2, CODE_LD));
     GemmProblem pr = make_problem(N_HIDDEN / GEMM_BM, L.n_rows, HIDDEN_BN, false, status_dev);
     add_seg(pr, 0, 0, 2, 0, 0, 0, 0, c->kw / GEMM_BK);
     EpiGelu::Params ep{c->zero256, (float)std::ldexp(1.0, -c->p_v1), g16d};
@@ -1827,7 +1828,7 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
   }
   if (L.n_rows > 0) {
     CUtensorMap mb_q, mb_g;
-    RET(map_b(&mb_q, q16, false, c->kw, L.n_rows, INVERSE_BN / 2));
+    RET(map_b(&mb_q, q16, false, c->kw, L.n_rows, INVERSE_BN / 2, CODE_LD));
     GemmProblem pr = make_problem(ROW_DIM / GEMM_BM, L.n_rows, INVERSE_BN, false, status_dev);
     add_seg(pr, 0, 0, 2, 0, 0, 0, 0, c->kw / GEMM_BK);
     if (c->has_synth) {  // + g V2 (hi/lo on both sides)

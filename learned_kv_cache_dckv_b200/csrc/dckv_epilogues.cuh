@@ -141,10 +141,9 @@ struct EpiQuant {
     const float *mub;         // [mp] (mu @ basis) of the kept components, compact order
     const float *delta;       // [mp] Delta of the kept components
     int k_eff;                // features m < k_eff are kept components; the rest give 0
-    int kw;                   // width of the code arrays (a multiple of 64, >= k_eff)
     float scale;
-    int32_t *q32;             // [rows][kw]
-    __nv_bfloat16 *qe;        // [ne_pad][kw]
+    int32_t *q32;             // [rows][CODE_LD], compact columns
+    __nv_bfloat16 *qe;        // [ne_pad][CODE_LD], compact columns
     const int32_t *row_edst;  // [rows]: padded even row or -1
   };
 };
@@ -198,8 +197,9 @@ struct EpiQuantRegs {
     const EpiQuant::Params &p = pp.q;
     const int32_t *s_e = reinterpret_cast<const int32_t *>(buf);
     const float *s_w = reinterpret_cast<const float *>(buf + GEMM_MAX_BN * 4);
-    const int c = mt * GEMM_BM + ew * 32 + lane;  // compact component index
-    if (c >= p.kw) return;  // rows of the tile past the code arrays' width (all zero operands)
+    // compact component index; features past k_eff (zero operands) store code 0 into columns
+    // the readers ignore (mp <= CODE_LD)
+    const int c = mt * GEMM_BM + ew * 32 + lane;
     const float mb = p.mub[c];
     const float dl = p.delta[c];
     const bool kp = c < p.k_eff;
@@ -215,9 +215,9 @@ struct EpiQuantRegs {
         const float y = tot[j] * p.scale - mb;
         const float ratio = __fdiv_rn(y, dl);
         const int q = kp ? __float2int_rn(ratio) : 0;
-        p.q32[(int64_t)row * p.kw + c] = q;
+        p.q32[(int64_t)row * CODE_LD + c] = q;
         const int e = s_e[col];
-        if (e >= 0) p.qe[(int64_t)e * p.kw + c] = __float2bfloat16_rn((float)q);
+        if (e >= 0) p.qe[(int64_t)e * CODE_LD + c] = __float2bfloat16_rn((float)q);
         if (pp.dbg_ratio && kp) pp.dbg_ratio[(int64_t)row * N_COEF + pp.kept_list[c]] = ratio;
         const float w = wk * s_w[col] + REFINE_W0;
         if (kp && (0.5f - fabsf(ratio - rintf(ratio)) < w || !(fabsf(ratio) < 1.0e6f))) fm[j >> 5] |= 1u << (j & 31);
@@ -249,12 +249,11 @@ struct EpiMeanOdd {
     const int16_t *kept_list;  // compact index -> component (the GEMM's features are kept components)
     int8_t *cen8;            // [slots][k_eff]  (encoder: the odd centres)
     int k_eff;
-    int kw;                  // width of q16
     int vocab;
     // decoder: the odd codes themselves, code = centre + symbol - 254 (q16 != NULL); an
     // ESC symbol leaves its code to the escape patch and flags its chunk
     const uint16_t *syms;    // [slots][k_eff] decoded symbols
-    __half *q16;             // [rows][kw]
+    __half *q16;             // [rows][CODE_LD], compact columns
     const int32_t *e_row;    // [ne_pad] natural coded row of that odd row
     const int32_t *slot_chunk;
     uint32_t *escflag;       // [chunks]
@@ -305,7 +304,7 @@ struct EpiMeanOdd {
           } else if (sv[j] == ESC_SYM) {
             p.escflag[__ldg(p.slot_chunk + s_slot[c0 + j])] = 1u;
           } else {
-            p.q16[(int64_t)s_nat[c0 + j] * p.kw + kc] = __float2half_rn((float)((int)sv[j] - R_MAX + (int)cen));
+            p.q16[(int64_t)s_nat[c0 + j] * CODE_LD + kc] = __float2half_rn((float)((int)sv[j] - R_MAX + (int)cen));
           }
         }
       }

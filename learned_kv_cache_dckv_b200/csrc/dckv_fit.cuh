@@ -59,9 +59,8 @@ struct FitRegArgs {
   const int32_t *token_ids;
   const uint16_t *embed;     // bf16 [vocab][2048]
   int vocab;
-  const int32_t *q32;        // [n_rows][kw] final codes of the kept components (compact order)
+  const int32_t *q32;        // [n_rows][CODE_LD] final codes of the kept components (compact order)
   const int16_t *kidx;       // [2048] compact index of a component, -1 if dropped (code 0)
-  int kw;
   int64_t slot0, n, kpad;    // first slot row of the parity, its rows, padded columns
   int n_x;                   // regressors: 2048 (even) or 6144 (odd)
   uint16_t *x_t;             // [n_x][kpad]        bf16 regressors, transposed
@@ -71,7 +70,7 @@ struct FitRegArgs {
 // code of component c of coded row r (0 for a dropped component)
 __device__ __forceinline__ int32_t code_of(const FitRegArgs &a, int64_t r, int c) {
   const int m = __ldg(a.kidx + c);
-  return m >= 0 ? __ldg(a.q32 + r * a.kw + m) : 0;
+  return m >= 0 ? __ldg(a.q32 + r * CODE_LD + m) : 0;
 }
 
 __device__ __forceinline__ uint16_t bf16_bits_of_code(int32_t q) {
@@ -413,7 +412,7 @@ __global__ void k_fit_bf16(const double *w, int64_t count, uint16_t *out) {
 // Scale sums: thread k of a block keeps the sum of |q - centre| of kept components
 // k, k + 256, ... over the block's rows; integer sums, so the result is exact.
 __global__ void __launch_bounds__(256) k_fit_absres(int64_t n_rows, const int32_t *row_slot, const int32_t *q32,
-                                                    const int8_t *cen8, const int16_t *kept_list, int k_eff, int kw,
+                                                    const int8_t *cen8, const int16_t *kept_list, int k_eff,
                                                     unsigned long long *abs_sum) {
   constexpr int PER = N_COEF / 256;
   long long acc[PER];
@@ -425,7 +424,7 @@ __global__ void __launch_bounds__(256) k_fit_absres(int64_t n_rows, const int32_
     for (int u = 0; u < PER; ++u) {
       const int k = threadIdx.x + 256 * u;
       if (k < k_eff) {
-        const long long d = (long long)__ldg(q32 + r * kw + k) - (long long)cen8[base + k];
+        const long long d = (long long)__ldg(q32 + r * CODE_LD + k) - (long long)cen8[base + k];
         acc[u] += d < 0 ? -d : d;
       }
     }
@@ -486,7 +485,7 @@ extern "C" int dckv_fit_accumulate(const dckv_codec *c, const uint16_t *embed, i
     for (int par = 0; par < 2; ++par) {
       a[par] = FitRegArgs{(const PromptInfo *)(ws + f.enc.prompts), L.batch, inv,
                           (const int32_t *)(ws + f.enc.row_tok), token_ids, embed, vocab,
-                          (const int32_t *)(ws + f.enc.q32), c->kidx, c->kw, par ? f.n_e : 0, par ? f.n_o : f.n_e,
+                          (const int32_t *)(ws + f.enc.q32), c->kidx, par ? f.n_e : 0, par ? f.n_o : f.n_e,
                           par ? f.ko : f.ke, par ? 3 * N_COEF : N_COEF,
                           (uint16_t *)(ws + (par ? f.xot : f.et)), (uint16_t *)(ws + (par ? f.yot : f.yet))};
       if (a[par].n == 0) continue;
@@ -557,7 +556,7 @@ extern "C" int dckv_fit_scales_accumulate(const dckv_codec *c, const void *rows,
   uint8_t *ws = (uint8_t *)workspace;
   const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(L.n_rows, (int64_t)c->num_sms * 4));
   { k_fit_absres<<<grid, 256, 0, st>>>(L.n_rows, (const int32_t *)(ws + w.row_slot), (const int32_t *)(ws + w.q32),
-                                     (const int8_t *)(ws + w.cen8), c->kept_list, c->k_eff, c->kw,
+                                     (const int8_t *)(ws + w.cen8), c->kept_list, c->k_eff,
                                      (unsigned long long *)abs_sum); ++g_launches; }
   CK(cudaGetLastError());
   return DCKV_OK;

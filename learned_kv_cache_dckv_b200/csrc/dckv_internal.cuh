@@ -32,7 +32,11 @@ constexpr uint32_t MAGIC = 0x564B4344u;   // "DCKV"
 constexpr int VERSION = 1;
 constexpr int HEADER_BYTES = 64;
 constexpr int CHUNK_FIXED_BYTES = 4 * LANES + 4;  // states + escape count
-constexpr int BIG_CODE = 2048;            // |q| >= 2048 is not exact in the fp16 code operand
+constexpr int BIG_CODE = 2048;
+// Row stride (elements) of the per-call code arrays (q32, qe, q16, qbig).  Their columns
+// hold the kept components in compact order (the codec's kw of them are read); the stride
+// stays 2,048 so that the fused epilogues address them with a compile-time constant.
+constexpr int CODE_LD = N_COEF;            // |q| >= 2048 is not exact in the fp16 code operand
 // Guard band of the transform: a code is recomputed in fp64 when its fp32 ratio y / Delta
 // lies within REFINE_KAPPA * |x|_2 / Delta + REFINE_W0 of a half-step boundary (the fp32
 // path's error grows with the row's norm); rows with |x|_2 > REFINE_NORM_FULL are
@@ -84,7 +88,7 @@ struct Layout {
   int64_t max_len = 0;    // longest prompt (RoPE table positions)
   int n_chunks = 0, n_chunks_e = 0, n_chunks_o = 0;
   int64_t n_symbols = 0;  // n_rows * K_eff
-  int kw = 64;            // width of the code arrays (the codec's kw)
+  int kw = 64;            // columns of the code arrays in use (the codec's kw)
   std::vector<PromptInfo> prompts;
   std::vector<ChunkDesc> chunks;
   uint64_t off_kept = 0, off_streams = 0;  // blob offsets

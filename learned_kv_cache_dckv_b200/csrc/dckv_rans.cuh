@@ -96,7 +96,7 @@ __device__ __forceinline__ int even_centre(const float *t_row, int comp) {
 __global__ void __launch_bounds__(SYM_THREADS) k_symbols(int64_t n_rows, const int32_t *row_slot,
                                                          const int32_t *slot_chunk, const int32_t *q32,
                                                          int8_t *cen8, const int16_t *kept_list,
-                                                         const uint8_t *kept_scale, const uint2 *cfm_tab, int k_eff, int kw,
+                                                         const uint8_t *kept_scale, const uint2 *cfm_tab, int k_eff,
                                                          const float *t_even, const int32_t *tok_ids,
                                                          const int32_t *row_tok, const int32_t *row_edst, int vocab,
                                                          uint16_t *sym16, uint2 *cfm, uint32_t *nesc) {
@@ -112,7 +112,7 @@ __global__ void __launch_bounds__(SYM_THREADS) k_symbols(int64_t n_rows, const i
     __syncthreads();
     const int slot = row_slot[row];
     const int64_t base = (int64_t)slot * k_eff;
-    const int32_t *q = q32 + row * kw;  // compact: kept component k at column k
+    const int32_t *q = q32 + row * CODE_LD;  // compact: kept component k at column k
     const bool even = row_edst[row] >= 0;
     const float *t_row = nullptr;
     if (even && t_even) t_row = t_even + (int64_t)min(max(tok_ids[row_tok[row]], 0), vocab - 1) * N_COEF;
@@ -319,8 +319,7 @@ struct CompactArgs {
   const PromptInfo *prompts;
   int n_chunks;
   int k_eff;
-  int kw;                 // width of q32 (kept components, compact order)
-  const int32_t *q32;
+  const int32_t *q32;     // [rows][CODE_LD]: kept components in compact order
   const uint16_t *sym16;
   const uint16_t *words;
   const uint32_t *states, *nwords, *nesc, *offs;
@@ -371,7 +370,7 @@ __global__ void __launch_bounds__(COMPACT_THREADS) compact_kernel(CompactArgs a)
         const int rl = (int)(i / K);
         const int k = (int)(i - (int64_t)rl * K);
         const int64_t row = (int64_t)pi.row_base + 2 * (cd.j0 + rl) + cd.parity;
-        const int64_t v = (int64_t)a.q32[row * a.kw + k];
+        const int64_t v = (int64_t)a.q32[row * CODE_LD + k];
         const uint32_t slot = ep + __popc(m & lt_mask);
         if (slot < ne) {
           ev[2 * slot] = (uint32_t)(uint64_t)v;
@@ -687,7 +686,7 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1) rans_decode_kernel(RansDecA
 __global__ void __launch_bounds__(256) k_codes_elem(int parity, int64_t n_rows, const int32_t *row_edst,
                                                     const int32_t *row_slot, const int32_t *slot_chunk,
                                                     const uint16_t *syms, const int8_t *cen8,
-                                                    int kw, int k_eff, __half *q16,
+                                                    int k_eff, __half *q16,
                                                     __nv_bfloat16 *qe, uint32_t *escflag, const int32_t *valid) {
   if (*valid != 1) return;
   constexpr int PER = N_COEF / 256;  // blockDim.x == 256
@@ -714,8 +713,8 @@ __global__ void __launch_bounds__(256) k_codes_elem(int parity, int64_t n_rows, 
         continue;
       }
       const int q = sv[u] - R_MAX + cv[u];
-      q16[r * kw + k] = __float2half_rn((float)q);
-      if (e >= 0) qe[(int64_t)e * kw + k] = __float2bfloat16_rn((float)q);
+      q16[r * CODE_LD + k] = __float2half_rn((float)q);
+      if (e >= 0) qe[(int64_t)e * CODE_LD + k] = __float2bfloat16_rn((float)q);
     }
     if (__syncthreads_or(esc) && threadIdx.x == 0) escflag[slot_chunk[slot]] = 1u;
   }
@@ -726,8 +725,7 @@ struct DecCodesArgs {
   const PromptInfo *prompts;
   int chunk0, n_chunks;
   int k_eff;
-  int kw;                   // width of q16, qe, qbig (kept components, compact order)
-  const uint16_t *syms;     // slot order
+  const uint16_t *syms;     // slot order (q16, qe, qbig: [rows][CODE_LD], kept components in compact order)
   const uint8_t *blob;
   uint64_t off_streams;
   const uint32_t *offs;
@@ -791,10 +789,10 @@ __global__ void __launch_bounds__(PATCH_THREADS) k_escape_patch(DecCodesArgs a) 
       const int rl = (int)(i / K);
       const int k = (int)(i - (int64_t)rl * K);
       const int64_t row = (int64_t)pi.row_base + 2 * (cd.j0 + rl) + cd.parity;
-      a.q16[row * a.kw + k] = __float2half_rn((float)q);
-      if (cd.parity == 0) a.qe[(int64_t)(pi.ebase + cd.j0 + rl) * a.kw + k] = __float2bfloat16_rn((float)q);
+      a.q16[row * CODE_LD + k] = __float2half_rn((float)q);
+      if (cd.parity == 0) a.qe[(int64_t)(pi.ebase + cd.j0 + rl) * CODE_LD + k] = __float2bfloat16_rn((float)q);
       if (q >= BIG_CODE || q <= -BIG_CODE) {
-        a.qbig[row * a.kw + k] = q;
+        a.qbig[row * CODE_LD + k] = q;
         if (atomicExch(&a.bigflag[row], 1u) == 0u) a.biglist[atomicAdd(a.bigcount, 1u)] = (int32_t)row;
       }
     }

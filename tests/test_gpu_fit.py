@@ -36,10 +36,9 @@ def _codes_from_ws(handle, ws, offs, k_eff, keep):
     """Per prompt: the GPU's final codes (and, after the symbol kernel, centres)."""
     v = D.dckv_ws_offsets(handle, offs, 0)
     n = v["n_rows"]
-    kw = v["code_width"]
     q32 = np.zeros((n, 2048), np.int64)
     if n:
-        qc = ws[v["q32"]: v["q32"] + 4 * n * kw].view(torch.int32).reshape(n, kw).cpu().numpy()
+        qc = ws[v["q32"]: v["q32"] + 4 * n * 2048].view(torch.int32).reshape(n, 2048).cpu().numpy()
         q32[:, keep] = qc[:, :k_eff]  # the library keeps kept components only, compact
     cen8 = ws[v["cen8"]: v["cen8"] + n * k_eff].view(torch.int8).reshape(n, k_eff).cpu().numpy()
     slot = ws[v["row_slot"]: v["row_slot"] + 4 * n].view(torch.int32).cpu().numpy()
