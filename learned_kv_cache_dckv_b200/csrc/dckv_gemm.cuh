@@ -463,7 +463,12 @@ constexpr int gemm2_smem_bytes() {
 // to Epi::finish.  Both P buffers stay free for the MMA while totals are finished.  Per-column
 // metadata of a tile is staged into shared memory (Epi::stage, two buffers by tile parity)
 // before its chunks are drained, so that finish reads it without global-memory latency.
-constexpr int GEMM2C_THREADS = 320;
+// Epilogue: GEMM2C_COL_GROUPS groups of four warps, each group BN / GEMM2C_COL_GROUPS
+// columns of the tile (four groups: 56 columns and totals per thread at BN = 224, so that
+// the quantiser after a tile's last chunk is spread over sixteen warps and finishes within
+// the two chunks the MMA runs ahead).
+constexpr int GEMM2C_COL_GROUPS = 4;
+constexpr int GEMM2C_THREADS = 64 + 128 * GEMM2C_COL_GROUPS;
 
 template <class Epi, int STAGES, int MAX_SLABS, int CHUNK_STEPS, int BN>
 __global__ void __launch_bounds__(GEMM2C_THREADS, 1)
@@ -471,7 +476,8 @@ __global__ void __launch_bounds__(GEMM2C_THREADS, 1)
                          const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
                          const GemmProblem prob, const typename Epi::Params ep) {
   static_assert(BN % 32 == 0 && BN <= GEMM_MAX_BN, "BN / 2 must be a multiple of 16");
-  constexpr int NC = BN / 2;  // columns per epilogue thread
+  static_assert(BN % (8 * GEMM2C_COL_GROUPS) == 0, "column groups of whole 8-column loads");
+  constexpr int NC = BN / GEMM2C_COL_GROUPS;  // columns per epilogue thread
   extern __shared__ __align__(1024) uint8_t dyn_smem[];
   constexpr int STAGE_BYTES = Gemm2Smem<MAX_SLABS, BN>::STAGE_BYTES;
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
@@ -504,7 +510,7 @@ __global__ void __launch_bounds__(GEMM2C_THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&part_full[a], 1);
-      mbar_init(&part_empty[a], 16);
+      mbar_init(&part_empty[a], 2 * 4 * GEMM2C_COL_GROUPS);  // every epilogue warp of both CTAs
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -643,15 +649,23 @@ __global__ void __launch_bounds__(GEMM2C_THREADS, 1)
         }
         tc_fence_after();
         const uint32_t part = tmem_base + lane_base + (uint32_t)(pb * 256 + col0);
+        constexpr int N32 = NC / 32, REM = NC % 32;  // REM is 0, 8, 16 or 24
 #pragma unroll
-        for (int g = 0; g < NC / 16; g += 2) {
+        for (int g = 0; g < N32; ++g) {
           uint32_t r[32];
-          tmem_ld_32x32b_x16(part + (uint32_t)(g * 16), r);
-          if (g + 1 < NC / 16) tmem_ld_32x32b_x16(part + (uint32_t)((g + 1) * 16), r + 16);
+          tmem_ld_32x32b_x16(part + (uint32_t)(g * 32), r);
+          tmem_ld_32x32b_x16(part + (uint32_t)(g * 32 + 16), r + 16);
           tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (g * 16 + j < NC) tot[g * 16 + j] += __uint_as_float(r[j]);
+          for (int j = 0; j < 32; ++j) tot[g * 32 + j] += __uint_as_float(r[j]);
+        }
+        if constexpr (REM > 0) {
+          uint32_t r[24];
+          if constexpr (REM >= 16) tmem_ld_32x32b_x16(part + (uint32_t)(N32 * 32), r);
+          if constexpr (REM % 16 != 0) tmem_ld_32x32b_x8(part + (uint32_t)(N32 * 32 + (REM & 16)), r + (REM & 16));
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < REM; ++j) tot[N32 * 32 + j] += __uint_as_float(r[j]);
         }
         tc_fence_before();
         __syncwarp();
