@@ -456,16 +456,21 @@ def run_gpu(args):
         "dec:gemm_inverse": 2.0 * n_rows * 2048 * 6144,
     }
     pad = lambda n, t: -(-n // t) * t
-    issued_flops = {  # what the tensor pipe executes (split operands, padded tiles)
+    # what the tensor pipe executes: kept components only (M = mp for the transform and the
+    # odd mean model, K = kw for the GEMMs that read codes), split operands (the inverse's
+    # lo half up to its cut), padded tiles
+    shp = D.dckv_codec_gemm_shape(gc.handle)
+    kw, mp, lo_k = shp["kw"], shp["mp"], shp["inv_lo_k"]
+    issued_flops = {
         "enc:gemm_hidden": 2.0 * 2 * pad(n_rows, 256) * 6144 * 256,
-        "enc:gemm_transform": 2.0 * pad(n_rows, 224) * (2 * 6144 * 2048 + 4 * 256 * 2048),
-        "enc:gemm_mean_odd": 2.0 * pad(n_even + len(offs) - 1, 224) * 4096 * 2048,
-        "dec:gemm_mean_odd": 2.0 * pad(n_even + len(offs) - 1, 224) * 4096 * 2048,
-        "dec:gemm_inverse": 2.0 * 2 * pad(n_rows, 224) * 2048 * 6144,
+        "enc:gemm_transform": 2.0 * pad(n_rows, 224) * (2 * 6144 + 4 * 256) * mp,
+        "enc:gemm_mean_odd": 2.0 * pad(n_even + len(offs) - 1, 224) * 2 * kw * mp,
+        "dec:gemm_mean_odd": 2.0 * pad(n_even + len(offs) - 1, 224) * 2 * kw * mp,
+        "dec:gemm_inverse": 2.0 * pad(n_rows, 224) * 6144 * (kw + lo_k),
     }
     if args.config.endswith("syn"):  # decoder-side synthesis: hidden GEMM, and g V2 in the inverse
         algo_flops["dec:gemm_synth_hidden"] = 2.0 * n_rows * 2048 * 256
-        issued_flops["dec:gemm_synth_hidden"] = 2.0 * 2 * pad(n_rows, 64) * 2048 * 256
+        issued_flops["dec:gemm_synth_hidden"] = 2.0 * 2 * pad(n_rows, 64) * kw * 256
         algo_flops["dec:gemm_inverse"] += 2.0 * n_rows * 256 * 6144
         issued_flops["dec:gemm_inverse"] += 2.0 * 4 * pad(n_rows, 224) * 256 * 6144
     # DRAM bytes (read + write) per launch: the committed ncu captures (profiles/) of the
@@ -534,7 +539,7 @@ def run_gpu(args):
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "fp16", "data": "synthetic",
         "config": {"workload": desc, "prompts": len(lens), "seq_len": lens[0], "tokens_per_step": tokens,
-                   "coded_rows": n_rows, "step_scale": cod.step_scale, "k_eff": k_eff,
+                   "coded_rows": n_rows, "step_scale": cod.step_scale, "k_eff": k_eff, "gemm_shape": shp,
                    "l2": "256 MiB buffer written between encode and decode and between steps (outside the events)",
                    "arith": "fp16 split operands, fp32 TMEM accumulation; rANS in u32",
                    "parallelism": f"replicas x{ws}"},

@@ -59,6 +59,18 @@ int dckv_codec_tables(const dckv_codec *codec, const void **t_even, const void *
  * components' tables in bits per coded row (the rate the codec's own model expects). */
 int dckv_codec_info(const dckv_codec *codec, int32_t *chunk_rows, double *model_bits_per_row);
 
+/* Shapes of the codec's compacted GEMMs (kept components only), int32 [4]:
+ *   [0] K_eff, kept components;
+ *   [1] kw, K_eff rounded up to 64: the K extent of the GEMMs that read codes, and the
+ *       code arrays' columns in use;
+ *   [2] mp, K_eff rounded up to 256: the M extent of the GEMMs that produce one value per
+ *       kept component (transform, odd mean model);
+ *   [3] the inverse's lo-half cut: its split operand's lo half is added for the first this
+ *       many compact components only (the rest carry less than 2^-15 of the reconstruction's
+ *       rms under the codec's Laplace model); equal to kw for a codec with decoder-side
+ *       synthesis. */
+int dckv_codec_gemm_shape(const dckv_codec *codec, int32_t *shape);
+
 /* Self-test hook: when ratio_dev (device fp32 [n_rows][2048]) is not NULL, later encodes
  * also write the fp32 transform ratios y / Delta there, before any exact recomputation.
  * Pass NULL to stop.  The buffer must cover the largest call's coded rows. */

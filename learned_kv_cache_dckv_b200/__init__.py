@@ -95,6 +95,7 @@ def lib():
         "dckv_debug_gemm": (I, [I, P, I, P, I, I, I, P, I, I, P]),
         "dckv_debug_ratio": (I, [P, P]),
         "dckv_codec_info": (I, [P, P, P]),
+        "dckv_codec_gemm_shape": (I, [P, P]),
         "dckv_launch_count": (ctypes.c_longlong, []),
         "dckv_fit_workspace_bytes": (Z, [P, P, I]),
         "dckv_fit_accumulate": (I, [P, P, ctypes.c_int32, P, P, P, I, P, P, P, Z, P]),
@@ -254,6 +255,12 @@ def dckv_codec_info(handle):
     bits = ctypes.c_double()
     _check(lib().dckv_codec_info(handle, ctypes.byref(g), ctypes.byref(bits)), "dckv_codec_info")
     return {"chunk_rows": int(g.value), "model_bits_per_row": float(bits.value)}
+
+
+def dckv_codec_gemm_shape(handle):
+    a = (ctypes.c_int32 * 4)()
+    _check(lib().dckv_codec_gemm_shape(handle, a), "dckv_codec_gemm_shape")
+    return {"k_eff": a[0], "kw": a[1], "mp": a[2], "inv_lo_k": a[3]}
 
 
 def dckv_set_timing(handle, enable: bool):

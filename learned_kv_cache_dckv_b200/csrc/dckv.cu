@@ -456,6 +456,34 @@ __global__ void k_gather_on(const uint16_t *w_odd, const int16_t *kept, int k_ef
   }
 }
 
+// Squared column norms of the inverse GEMM's split operand a_inv [2][6144][kw]: per compact
+// component m, sum over rows of lo^2 (out[m]) and of (hi + lo)^2 (out[kw + m]), fp64.
+__global__ void k_inv_colnorms(const __half *a_inv, int kw, double *out) {
+  __shared__ double s_lo[256], s_all[256];
+  const int m = blockIdx.x;
+  const __half *lo = a_inv + (int64_t)ROW_DIM * kw;
+  double l2 = 0.0, a2 = 0.0;
+  for (int p = threadIdx.x; p < ROW_DIM; p += blockDim.x) {
+    const double h = (double)__half2float(a_inv[(int64_t)p * kw + m]), l = (double)__half2float(lo[(int64_t)p * kw + m]);
+    l2 += l * l;
+    a2 += (h + l) * (h + l);
+  }
+  s_lo[threadIdx.x] = l2;
+  s_all[threadIdx.x] = a2;
+  __syncthreads();
+  for (int s = blockDim.x / 2; s > 0; s >>= 1) {
+    if ((int)threadIdx.x < s) {
+      s_lo[threadIdx.x] += s_lo[threadIdx.x + s];
+      s_all[threadIdx.x] += s_all[threadIdx.x + s];
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    out[m] = s_lo[0];
+    out[kw + m] = s_all[0];
+  }
+}
+
 // Per-component constants of the kept components in compact order (pads: Delta 1, mean 0).
 __global__ void k_compact_meta(const float *delta, const float *mub, const int16_t *kept, int k_eff, int mp,
                                float *delta_k, float *mub_k) {
@@ -1244,6 +1272,7 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
   const uint64_t o_zero = take(4ull * N_HIDDEN);
   const uint64_t o_tmp = take(2ull * 2 * N_COEF * N_COEF);  // W_e^T and W_oE^T (setup only)
   const uint64_t o_scr = take(64);
+  const uint64_t o_norms = take(8ull * 2 * N_COEF);  // setup only: column norms of a_inv
   if (cudaMalloc(&c->blk, o) != cudaSuccess) return cleanup(fail(DCKV_ECUDA, "cudaMalloc(%llu) failed", (unsigned long long)o));
   uint8_t *B = (uint8_t *)c->blk;
   c->a_y = (__half *)(B + o_ay);
@@ -1438,10 +1467,43 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
       (r = map_a(&c->map_aw2_1, c->a_w2, false, N_HIDDEN, c->mp, 2, 1)) ||
       (r = map_a(&c->map_ah2, c->a_h, false, ROW_DIM, N_HIDDEN, 2, 2)) ||
       (r = map_a(&c->map_ainv2, c->a_inv, false, c->kw, ROW_DIM, 2, 2)) ||
+      (r = map_a(&c->map_ainv1, c->a_inv, false, c->kw, ROW_DIM, 2, 1)) ||
       (r = map_a(&c->map_aon1, c->a_on, true, 2 * c->kw, c->mp, 1, 1)) ||
       (has_synth && (r = map_a(&c->map_av1, c->a_v1, false, c->kw, N_HIDDEN, 2, 2))) ||
       (has_synth && (r = map_a(&c->map_av2, c->a_v2, false, N_HIDDEN, ROW_DIM, 2, 2))))
     return cleanup(r);
+  // the inverse's lo-half cut: the smallest multiple of 64 such that the lo halves of the
+  // components past it carry at most INV_LO_THETA^2 of the expected signal energy,
+  // E[q_m^2] |A_m|^2 summed over m, with E[q^2] = 2 beta^2 + 1/12 under the component's own
+  // Laplace scale beta (in steps) and A_m = Delta_m basis[:, m].  The decoder-side synthesis
+  // variant keeps the whole split (its extra operand takes the second tensor map).
+  c->inv_lo_k = c->kw;
+  if (!has_synth && c->k_eff > 0) {
+    double *norms = (double *)(B + o_norms);
+    { k_inv_colnorms<<<c->kw, 256, 0, st>>>(c->a_inv, c->kw, norms); ++g_launches; }
+    std::vector<double> nh(2 * (size_t)c->kw);
+    std::vector<float> bh(N_COEF), dh(N_COEF);
+    if (cudaMemcpy(nh.data(), norms, 8ull * 2 * c->kw, cudaMemcpyDeviceToHost) != cudaSuccess ||
+        cudaMemcpy(bh.data(), prm->laplace_b, 4ull * N_COEF, cudaMemcpyDeviceToHost) != cudaSuccess ||
+        cudaMemcpy(dh.data(), prm->delta, 4ull * N_COEF, cudaMemcpyDeviceToHost) != cudaSuccess)
+      return cleanup(fail(DCKV_ECUDA, "setup readback failed"));
+    std::vector<double> lo_e(c->k_eff);
+    double total = 0.0;
+    for (int m = 0; m < c->k_eff; ++m) {
+      const double beta = (double)bh[kl[m]] / (double)dh[kl[m]];
+      const double eq2 = 2.0 * beta * beta + 1.0 / 12.0;
+      lo_e[m] = eq2 * nh[m];
+      total += eq2 * nh[c->kw + m];
+    }
+    double tail = 0.0;
+    int cut = c->k_eff;  // smallest m with sum over m' >= m of lo_e[m'] within the bound
+    for (int m = c->k_eff - 1; m >= 0; --m) {
+      tail += lo_e[m];
+      if (tail > INV_LO_THETA * INV_LO_THETA * total) break;
+      cut = m;
+    }
+    c->inv_lo_k = std::min(c->kw, (cut + 63) / 64 * 64);
+  }
   // per-vocabulary mean tables: t_even = embed @ w_even, t_odd = embed @ w_odd[0:2048]
   if (has_means) {
     CUtensorMap ma_e, ma_o, mb_emb;
@@ -1830,7 +1892,9 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
     CUtensorMap mb_q, mb_g;
     RET(map_b(&mb_q, q16, false, c->kw, L.n_rows, INVERSE_BN / 2, CODE_LD));
     GemmProblem pr = make_problem(ROW_DIM / GEMM_BM, L.n_rows, INVERSE_BN, false, status_dev);
-    add_seg(pr, 0, 0, 2, 0, 0, 0, 0, c->kw / GEMM_BK);
+    // hi and lo halves up to the cut, the hi half alone after it (second A map, one slab)
+    if (c->inv_lo_k > 0) add_seg(pr, 0, 0, 2, 0, 0, 0, 0, c->inv_lo_k / GEMM_BK);
+    if (c->inv_lo_k < c->kw) add_seg(pr, 1, 0, 1, c->inv_lo_k, 0, 0, c->inv_lo_k, (c->kw - c->inv_lo_k) / GEMM_BK);
     if (c->has_synth) {  // + g V2 (hi/lo on both sides)
       RET(map_b(&mb_g, g16d, false, 2 * N_HIDDEN, L.n_rows, INVERSE_BN / 2));
       add_seg(pr, 1, 0, 2, 0, 1, 0, 0, N_HIDDEN / GEMM_BK);
@@ -1840,7 +1904,7 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
     }
     EpiInverse::Params ep{c->mu_perm, (float)std::ldexp(1.0, -c->p_inv), rope, row_tok, row_pos,
                           (__nv_bfloat16 *)k_out, (__nv_bfloat16 *)v_out, L.n_tokens};
-    RET((run_gemm2<EpiInverse, 4, 2, 8>(c->map_ainv2, c->has_synth ? c->map_av2 : c->map_ainv2, mb_q, mb_g, pr, ep,
+    RET((run_gemm2<EpiInverse, 4, 2, 8>(c->map_ainv2, c->has_synth ? c->map_av2 : c->map_ainv1, mb_q, mb_g, pr, ep,
                                         c->num_sms, false, st)));
   }
   stage_mark(c, st, "gemm_inverse");
@@ -1959,6 +2023,15 @@ extern "C" int dckv_codec_info(const dckv_codec *c, int32_t *chunk_rows, double 
   if (!c) return fail(DCKV_EINVAL, "NULL codec");
   if (chunk_rows) *chunk_rows = c->chunk_rows;
   if (model_bits_per_row) *model_bits_per_row = c->model_bits_per_row;
+  return DCKV_OK;
+}
+
+extern "C" int dckv_codec_gemm_shape(const dckv_codec *c, int32_t *shape) {
+  if (!c || !shape) return fail(DCKV_EINVAL, "NULL argument");
+  shape[0] = c->k_eff;
+  shape[1] = c->kw;
+  shape[2] = c->mp;
+  shape[3] = c->inv_lo_k;
   return DCKV_OK;
 }
 

@@ -36,7 +36,12 @@ constexpr int BIG_CODE = 2048;
 // Row stride (elements) of the per-call code arrays (q32, qe, q16, qbig).  Their columns
 // hold the kept components in compact order (the codec's kw of them are read); the stride
 // stays 2,048 so that the fused epilogues address them with a compile-time constant.
-constexpr int CODE_LD = N_COEF;            // |q| >= 2048 is not exact in the fp16 code operand
+constexpr int CODE_LD = N_COEF;
+// Lo-half cut of the inverse GEMM's split operand (see dckv_codec::inv_lo_k): the lo halves
+// of the components past the cut carry at most this fraction of the reconstruction's rms in
+// expectation (about 3e-5; the hi half alone leaves ~2.4e-4 of each term, and bf16 output
+// rounding ~2e-3).
+constexpr double INV_LO_THETA = 1.0 / 32768.0;            // |q| >= 2048 is not exact in the fp16 code operand
 // Guard band of the transform: a code is recomputed in fp64 when its fp32 ratio y / Delta
 // lies within REFINE_KAPPA * |x|_2 / Delta + REFINE_W0 of a half-step boundary (the fp32
 // path's error grows with the row's norm); rows with |x|_2 > REFINE_NORM_FULL are
@@ -171,7 +176,11 @@ struct dckv_codec {
   float *v2_32 = nullptr;    // [256][6144]  V2
   float *zero256 = nullptr;  // [256] zeros (the synthesis hidden layer has no offset)
   int p_y = 0, p_h = 0, p_inv = 0, p_v1 = 0;  // power-of-two operand scales
-  CUtensorMap map_ay2, map_aw2_2, map_aw2_1, map_ah2, map_ainv2, map_aon1, map_av1, map_av2;
+  CUtensorMap map_ay2, map_aw2_2, map_aw2_1, map_ah2, map_ainv2, map_ainv1, map_aon1, map_av1, map_av2;
+  // The inverse GEMM adds the lo half of its split operand for the first inv_lo_k compact
+  // components only (a multiple of 64, at most kw): past them the lo half carries less than
+  // INV_LO_THETA of the signal's rms under the codec's own Laplace model.
+  int inv_lo_k = 0;
   // stage timing (optional; the events live in a per-thread log of the calling thread)
   int timing = 0;
 };

@@ -271,6 +271,34 @@ def test_tables_scale_and_mask_identical(codec_55, codec_literal):
         assert gc.k_eff == int(keep.sum())
 
 
+def test_compacted_gemm_shapes_and_inverse_lo_cut(src, codec_55):
+    """The GEMMs run on kept components only: K_eff rounded up to 64 (code arrays, K of the
+    GEMMs reading codes) and to 256 (M of the transform and the odd mean model).  The
+    inverse adds the lo half of its split operand Delta_c B[:, c] 2^p for the first
+    inv_lo_k kept components only: the smallest multiple of 64 past which the lo halves
+    carry at most 2^-30 of the expected signal energy sum E[q_m^2] |A_m|^2, with
+    E[q^2] = 2 beta^2 + 1/12 under each component's Laplace scale beta (in steps).  The
+    rule is recomputed here from the codec's parameters in fp64."""
+    gc = gpu_codec(codec_55)
+    shp = D.dckv_codec_gemm_shape(gc.handle)
+    k = gc.k_eff
+    assert shp["k_eff"] == k and shp["kw"] == max(64, -(-k // 64) * 64) and shp["mp"] == max(256, -(-k // 256) * 256)
+    keep = O.scale_index(codec_55.laplace_b, codec_55.delta)[1]
+    kl = np.nonzero(keep)[0]
+    p_inv = int(D.dckv_codec_export(gc.handle)[3][2])
+    a = (codec_55.delta.astype(np.float64)[kl, None] * codec_55.basis.astype(np.float64).T[kl]) * 2.0 ** p_inv
+    hi = a.astype(np.float16).astype(np.float64)
+    lo = (a - hi).astype(np.float16).astype(np.float64)
+    beta = (codec_55.laplace_b.astype(np.float64) / codec_55.delta.astype(np.float64))[kl]
+    eq2 = 2.0 * beta ** 2 + 1.0 / 12.0
+    total = np.sum(eq2 * ((hi + lo) ** 2).sum(axis=1))
+    tail = np.cumsum((eq2 * (lo ** 2).sum(axis=1))[::-1])[::-1]
+    ok = np.nonzero(tail <= total / 2.0 ** 30)[0]
+    cut = int(ok[0]) if ok.size else k
+    assert shp["inv_lo_k"] == min(shp["kw"], -(-cut // 64) * 64)
+    assert 0 < shp["inv_lo_k"] < shp["kw"]  # the cut is in use on this codec
+
+
 def test_parity_literal_small_config(src, codec_literal):
     # one prompt of 256 tokens (124 coded rows) plus ragged neighbours and degenerate prompts
     full_check(src, codec_literal, [256, 700, 50, 132, 133, 134], seeds=[0, 1, 2, 3, 4, 5])
