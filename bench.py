@@ -50,10 +50,19 @@ CONFIGS = {
 # the workload the benchmark reports by default: the largest configuration that fits one GPU
 DEFAULT_CONFIG = "c5"
 
-# DRAM read + write bytes per coded row of the dominant kernels, from the ncu captures of
-# the 4,096-token prompt (3,964 coded rows) in profiles/; a kernel changed after its capture
-# has no entry
-TRAFFIC_PER_CODED_ROW = {}
+# DRAM read + write bytes per coded row of the dominant kernels, from the ncu captures of the
+# profiling case (8 x 4,096 tokens, 31,712 coded rows; profiles/*_c5p.md); a kernel changed
+# after its capture has no entry
+TRAFFIC_PER_CODED_ROW = {
+    "enc:gemm_transform": (1.070784e9 + 282.553344e6) / 31712,
+    "dec:gemm_inverse": (161.299968e6 + 355.810816e6) / 31712,
+    "enc:gemm_hidden": (397.652224e6 + 99.875328e6) / 31712,
+    "enc:gemm_mean_odd": (181.498112e6 + 20.099584e6) / 31712,
+    "dec:gemm_mean_odd": (248.8576e6 + 41.697792e6) / 31712,
+    "dec:rans_loop": (7.335936e6 + 47.22176e6) / 31712,
+    "enc:rans_encode": (419.212288e6 + 8.81024e6) / 31712,
+    "enc:symbols": (362.088704e6 + 496.594944e6) / 31712,
+}
 
 GEMM_STAGES = {"gemm_hidden", "gemm_transform", "gemm_mean_odd", "gemm_inverse", "gemm_synth_hidden"}
 
