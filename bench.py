@@ -54,11 +54,7 @@ DEFAULT_CONFIG = "c5"
 # profiling case (8 x 4,096 tokens, 31,712 coded rows; profiles/*_c5p.md); a kernel changed
 # after its capture has no entry
 TRAFFIC_PER_CODED_ROW = {
-    "enc:gemm_transform": (1.070784e9 + 282.553344e6) / 31712,
-    "dec:gemm_inverse": (161.299968e6 + 355.810816e6) / 31712,
     "enc:gemm_hidden": (397.652224e6 + 99.875328e6) / 31712,
-    "enc:gemm_mean_odd": (181.498112e6 + 20.099584e6) / 31712,
-    "dec:gemm_mean_odd": (248.8576e6 + 41.697792e6) / 31712,
     "dec:rans_loop": (7.335936e6 + 47.22176e6) / 31712,
     "enc:rans_encode": (419.212288e6 + 8.81024e6) / 31712,
     "enc:symbols": (362.088704e6 + 496.594944e6) / 31712,
@@ -470,18 +466,18 @@ def run_gpu(args):
     # lo half up to its cut), padded tiles
     shp = D.dckv_codec_gemm_shape(gc.handle)
     kw, mp, lo_k = shp["kw"], shp["mp"], shp["inv_lo_k"]
-    issued_flops = {
+    issued_flops = {  # every pair GEMM runs 256-token tiles
         "enc:gemm_hidden": 2.0 * 2 * pad(n_rows, 256) * 6144 * 256,
-        "enc:gemm_transform": 2.0 * pad(n_rows, 224) * (2 * 6144 + 4 * 256) * mp,
-        "enc:gemm_mean_odd": 2.0 * pad(n_even + len(offs) - 1, 224) * 2 * kw * mp,
-        "dec:gemm_mean_odd": 2.0 * pad(n_even + len(offs) - 1, 224) * 2 * kw * mp,
-        "dec:gemm_inverse": 2.0 * pad(n_rows, 224) * 6144 * (kw + lo_k),
+        "enc:gemm_transform": 2.0 * pad(n_rows, 256) * (2 * 6144 + 4 * 256) * mp,
+        "enc:gemm_mean_odd": 2.0 * pad(n_even + len(offs) - 1, 256) * 2 * kw * mp,
+        "dec:gemm_mean_odd": 2.0 * pad(n_even + len(offs) - 1, 256) * 2 * kw * mp,
+        "dec:gemm_inverse": 2.0 * pad(n_rows, 256) * 6144 * (kw + lo_k),
     }
     if args.config.endswith("syn"):  # decoder-side synthesis: hidden GEMM, and g V2 in the inverse
         algo_flops["dec:gemm_synth_hidden"] = 2.0 * n_rows * 2048 * 256
         issued_flops["dec:gemm_synth_hidden"] = 2.0 * 2 * pad(n_rows, 64) * kw * 256
         algo_flops["dec:gemm_inverse"] += 2.0 * n_rows * 256 * 6144
-        issued_flops["dec:gemm_inverse"] += 2.0 * 4 * pad(n_rows, 224) * 256 * 6144
+        issued_flops["dec:gemm_inverse"] += 2.0 * 4 * pad(n_rows, 256) * 256 * 6144
     # DRAM bytes (read + write) per launch: the committed ncu captures (profiles/) of the
     # 4,096-token prompt, per coded row of that capture, times this workload's coded rows
     # (every such kernel's traffic grows with the rows it codes); kernels changed since
