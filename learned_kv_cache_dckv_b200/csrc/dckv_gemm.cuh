@@ -73,6 +73,57 @@ struct GemmSmem {
   static constexpr int STAGE_BYTES = MAX_SLABS * GEMM_SLAB_BYTES + BN_MAX * GEMM_BK * 2;
 };
 
+// Teardown state, in the barrier area after the stage and accumulator barriers.  A wait that
+// gives up (a timeout) makes the CTA leave its role loop early, possibly with TMA copies into
+// its shared memory and MMAs on its TMEM still in flight; before it leaves, the CTA waits
+// (bounded) for all of them:
+//   - copies: the producer counts the items (K steps) it issued and remembers each stage's
+//     last transaction bytes; every item's copies are counted on a full barrier, so waiting
+//     for the phases of the last STAGES items (earlier ones were consumed, hence complete)
+//     covers every copy still in flight;
+//   - MMAs: the issuer commits once more, to drain_bar, which completes when every MMA it
+//     issued has.
+// In the CTA pair each producer loads its own half of an item into its own shared memory,
+// counted on the leader's full barrier, and either producer may stop first.  The peer
+// therefore hands the leader its item count and bytes; for the items that only one of them
+// issued the leader settles the barrier's count (complete_tx for a half that will not come,
+// arrive with the peer's bytes for an item it never armed), drains the phases, and a last
+// cluster barrier holds the peer until then.  Without a timeout none of this runs.
+template <int STAGES>
+struct GemmTail {
+  uint64_t drain_bar;
+  uint32_t tmem_base;
+  int abort;                   // this CTA's abort flag
+  int peer_abort;              // the other CTA's flag, stored here by it (CTA pair)
+  uint32_t peer_issued;        // the peer producer's item count (leader's copy)
+  uint32_t ring[STAGES];       // transaction bytes of the last item issued into each stage
+  uint32_t peer_ring[STAGES];  // the peer's ring (leader's copy)
+};
+
+// Waits for the copies of the last min(n, STAGES) of n issued items (one thread).
+template <int STAGES>
+__device__ __forceinline__ void drain_issued(uint64_t *full_bar, uint32_t n) {
+  for (uint32_t i = n > (uint32_t)STAGES ? n - STAGES : 0u; i < n; ++i)
+    mbar_drain(&full_bar[i % STAGES], (i / STAGES) & 1u);
+}
+
+// Leader of a CTA pair after an abort: settles the full barriers of the items only one
+// producer issued (l: the leader's count, p: the peer's), then drains them (one thread).
+// Both producers wait on releases of the same items, so |l - p| <= STAGES and each of those
+// items is the last one its producer put into its stage.
+template <int STAGES>
+__device__ __forceinline__ void pair_drain_issued(uint64_t *full_bar, uint32_t l, uint32_t p,
+                                                  const uint32_t *ring, const volatile uint32_t *peer_ring) {
+  for (uint32_t i = l < p ? l : p; i < (l < p ? p : l); ++i) {
+    const int s = (int)(i % STAGES);
+    if (l > p)
+      mbar_complete_tx(&full_bar[s], ring[s]);  // armed for both halves; the peer's never comes
+    else
+      mbar_arrive_expect_tx(&full_bar[s], peer_ring[s]);  // never armed: count the peer's half
+  }
+  drain_issued<STAGES>(full_bar, l < p ? p : l);
+}
+
 // Epi must provide:
 //   struct Params;   static constexpr int SMEM_BYTES;
 //   __device__ static void tile(const Params&, const EpiCtx&)
@@ -91,13 +142,16 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   uint64_t *empty_bar = full_bar + STAGES;
   uint64_t *acc_full = empty_bar + STAGES;
   uint64_t *acc_empty = acc_full + 2;
-  uint32_t *tmem_base_smem = reinterpret_cast<uint32_t *>(acc_empty + 2);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_base_smem + 1);
+  GemmTail<STAGES> *tail = reinterpret_cast<GemmTail<STAGES> *>(acc_empty + 2);
+  static_assert(sizeof(uint64_t) * (2 * STAGES + 4) + sizeof(GemmTail<STAGES>) <= 1024, "barrier area");
+  uint32_t *tmem_base_smem = &tail->tmem_base;
+  volatile int *abort_flag = &tail->abort;
   char *epi_scratch = reinterpret_cast<char *>(base + STAGES * STAGE_BYTES + 1024);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int total_tiles = prob.m_tiles * prob.n_tiles;
+  uint32_t n_issued = 0;  // items the producer (thread 0) issued
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -108,6 +162,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       mbar_init(&acc_full[a], 1);
       mbar_init(&acc_empty[a], 128);
     }
+    mbar_init(&tail->drain_bar, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -147,6 +202,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             mbar_arrive_expect_tx(&full_bar[stage], bytes);
             tma_load_3d(sa, ta, &full_bar[stage], sg.a_k0 + ks * GEMM_BK, mt * GEMM_BM, sg.a_slab0);
             tma_load_2d(sb, tb, &full_bar[stage], sg.b_k0 + ks * GEMM_BK, n0 + sg.b_row_shift);
+            ++n_issued;
             if (++stage == STAGES) {
               stage = 0;
               phase ^= 1u;
@@ -230,7 +286,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   }
 
   __syncthreads();
-  if (*abort_flag && threadIdx.x == 0 && prob.status) atomicExch(prob.status, 5);
+  if (*abort_flag) {  // a wait gave up: the copies and MMAs this CTA issued finish first
+    if (threadIdx.x == 0) drain_issued<STAGES>(full_bar, n_issued);
+    if (warp == 1 && lane == 0) {
+      umma_commit(&tail->drain_bar);
+      mbar_drain(&tail->drain_bar, 0);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && prob.status) atomicExch(prob.status, 5);
+  }
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, 512);
@@ -251,6 +315,34 @@ constexpr int gemm_smem_bytes() {
 // its own TMEM rows (feature tile 2 * pair_tile + r) with the same epilogue as above.
 // prob.m_tiles counts 128-row tiles and must be even; prob.bn <= 256, bn / 2 a multiple of 8.
 constexpr int GEMM_B_HALF_BYTES = (GEMM_MAX_BN / 2) * GEMM_BK * 2;  // 16 KiB
+
+// End of a CTA-pair kernel, after every role loop of this CTA has left (__syncthreads):
+// the CTAs exchange their abort flags (and the peer its item count and ring) and pass a
+// cluster barrier, so that neither leaves while the other may still signal its barriers or
+// read its TMEM; after an abort in either CTA the drain described at GemmTail follows.
+template <int STAGES>
+__device__ __forceinline__ void pair_teardown(GemmTail<STAGES> *tail, uint64_t *full_bar, uint32_t n_issued,
+                                              uint32_t rank, int warp, int lane, int *status) {
+  const volatile GemmTail<STAGES> *vt = tail;
+  if (threadIdx.x == 0) {
+    st_shared_cluster_u32(mapa_shared(smem_u32(&tail->peer_abort), rank ^ 1u), (uint32_t)vt->abort);
+    if (rank == 1) {
+      st_shared_cluster_u32(mapa_shared(smem_u32(&tail->peer_issued), 0), n_issued);
+      for (int s = 0; s < STAGES; ++s)
+        st_shared_cluster_u32(mapa_shared(smem_u32(&tail->peer_ring[s]), 0), tail->ring[s]);
+    }
+  }
+  cluster_sync();
+  if (vt->abort || vt->peer_abort) {
+    if (rank == 0 && warp == 1 && lane == 0) umma_commit_pair(&tail->drain_bar);
+    if (rank == 0 && threadIdx.x == 0)
+      pair_drain_issued<STAGES>(full_bar, n_issued, vt->peer_issued, tail->ring, vt->peer_ring);
+    if (warp == 1 && lane == 0) mbar_drain(&tail->drain_bar, 0);
+    __syncthreads();
+    cluster_sync();
+    if (vt->abort && threadIdx.x == 0 && status) atomicExch(status, 5);
+  }
+}
 
 template <int MAX_SLABS, int BN = GEMM_MAX_BN>
 struct Gemm2Smem {  // one stage: the A slabs, then this CTA's half of the B tile (a multiple of 1 KiB)
@@ -273,8 +365,10 @@ __global__ void __launch_bounds__(64 + 32 * EPI_WARPS, 1)
   uint64_t *empty_bar = full_bar + STAGES;
   uint64_t *acc_full = empty_bar + STAGES;
   uint64_t *acc_empty = acc_full + 2;  // leader's: one arrival per epilogue warp of either CTA
-  uint32_t *tmem_base_smem = reinterpret_cast<uint32_t *>(acc_empty + 2);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_base_smem + 1);
+  GemmTail<STAGES> *tail = reinterpret_cast<GemmTail<STAGES> *>(acc_empty + 2);
+  static_assert(sizeof(uint64_t) * (2 * STAGES + 4) + sizeof(GemmTail<STAGES>) <= 1024, "barrier area");
+  uint32_t *tmem_base_smem = &tail->tmem_base;
+  volatile int *abort_flag = &tail->abort;
   char *epi_scratch = reinterpret_cast<char *>(base + STAGES * STAGE_BYTES + 1024);
 
   const int warp = threadIdx.x >> 5;
@@ -287,6 +381,7 @@ __global__ void __launch_bounds__(64 + 32 * EPI_WARPS, 1)
   const int mn_tiles = m_pairs * prob.n_tiles;
   const int total_tiles = mn_tiles * n_split;
   const int half_bn = prob.bn >> 1;
+  uint32_t n_issued = 0;  // items this CTA's producer (thread 0) issued
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -297,6 +392,7 @@ __global__ void __launch_bounds__(64 + 32 * EPI_WARPS, 1)
       mbar_init(&acc_full[a], 1);
       mbar_init(&acc_empty[a], 2 * EPI_WARPS);
     }
+    mbar_init(&tail->drain_bar, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -344,6 +440,8 @@ __global__ void __launch_bounds__(64 + 32 * EPI_WARPS, 1)
             if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * bytes);
             tma_load_3d_pair(sa, ta, fb, sg.a_k0 + ks * GEMM_BK, (2 * mp + (int)rank) * GEMM_BM, sg.a_slab0);
             tma_load_2d_pair(sb, tb, fb, sg.b_k0 + ks * GEMM_BK, n0 + (int)rank * half_bn + sg.b_row_shift);
+            tail->ring[stage] = bytes;
+            ++n_issued;
             if (++stage == STAGES) {
               stage = 0;
               phase ^= 1u;
@@ -440,8 +538,7 @@ __global__ void __launch_bounds__(64 + 32 * EPI_WARPS, 1)
   }
 
   __syncthreads();
-  cluster_sync();  // no CTA leaves while its peer may still signal its barriers or read TMEM
-  if (*abort_flag && threadIdx.x == 0 && prob.status) atomicExch(prob.status, 5);
+  pair_teardown<STAGES>(tail, full_bar, n_issued, rank, warp, lane, prob.status);
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc_pair(tmem_base, 512);
@@ -486,8 +583,10 @@ __global__ void __launch_bounds__(GEMM2C_THREADS, 1)
   uint64_t *empty_bar = full_bar + STAGES;
   uint64_t *part_full = empty_bar + STAGES;
   uint64_t *part_empty = part_full + 2;  // leader's: one arrival per epilogue warp of either CTA
-  uint32_t *tmem_base_smem = reinterpret_cast<uint32_t *>(part_empty + 2);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_base_smem + 1);
+  GemmTail<STAGES> *tail = reinterpret_cast<GemmTail<STAGES> *>(part_empty + 2);
+  static_assert(sizeof(uint64_t) * (2 * STAGES + 4) + sizeof(GemmTail<STAGES>) <= 1024, "barrier area");
+  uint32_t *tmem_base_smem = &tail->tmem_base;
+  volatile int *abort_flag = &tail->abort;
   constexpr int EPI_BUF = (Epi::SMEM_BYTES + 15) & ~15;
   char *epi_buf = reinterpret_cast<char *>(base + STAGES * STAGE_BYTES + 1024);  // two buffers
 
@@ -499,6 +598,7 @@ __global__ void __launch_bounds__(GEMM2C_THREADS, 1)
   const int m_pairs = prob.m_tiles >> 1;
   const int total_tiles = m_pairs * prob.n_tiles;
   constexpr int half_bn = BN / 2;
+  uint32_t n_issued = 0;  // items this CTA's producer (thread 0) issued
   int ksteps = 0;
   for (int si = 0; si < prob.n_seg; ++si) ksteps += prob.seg[si].k_steps;
   const int n_chunks = (ksteps + CHUNK_STEPS - 1) / CHUNK_STEPS;
@@ -512,6 +612,7 @@ __global__ void __launch_bounds__(GEMM2C_THREADS, 1)
       mbar_init(&part_full[a], 1);
       mbar_init(&part_empty[a], 2 * 4 * GEMM2C_COL_GROUPS);  // every epilogue warp of both CTAs
     }
+    mbar_init(&tail->drain_bar, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -555,6 +656,8 @@ __global__ void __launch_bounds__(GEMM2C_THREADS, 1)
             if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * bytes);
             tma_load_3d_pair(sa, ta, fb, sg.a_k0 + ks * GEMM_BK, (2 * mp + (int)rank) * GEMM_BM, sg.a_slab0);
             tma_load_2d_pair(sb, tb, fb, sg.b_k0 + ks * GEMM_BK, n0 + (int)rank * half_bn + sg.b_row_shift);
+            tail->ring[stage] = bytes;
+            ++n_issued;
             if (++stage == STAGES) {
               stage = 0;
               phase ^= 1u;
@@ -682,8 +785,7 @@ __global__ void __launch_bounds__(GEMM2C_THREADS, 1)
   }
 
   __syncthreads();
-  cluster_sync();
-  if (*abort_flag && threadIdx.x == 0 && prob.status) atomicExch(prob.status, 5);
+  pair_teardown<STAGES>(tail, full_bar, n_issued, rank, warp, lane, prob.status);
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc_pair(tmem_base, 512);

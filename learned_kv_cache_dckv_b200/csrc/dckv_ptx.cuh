@@ -59,6 +59,12 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Completes `bytes` of the current phase's transaction count without a copy: stands in for
+// a copy that was counted but will never be issued (the abort drain of the CTA-pair GEMMs).
+__device__ __forceinline__ void mbar_complete_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.complete_tx.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
 // Bounded wait on phase `parity`.  Returns false (and sets *abort) on timeout or if
 // another thread of the CTA has already set *abort.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
@@ -240,6 +246,12 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
   uint32_t r;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
   return r;
+}
+
+// 32-bit store into shared memory given by its shared::cluster address (own CTA or peer);
+// made visible to the peer by the release/acquire of the next cluster_sync.
+__device__ __forceinline__ void st_shared_cluster_u32(uint32_t cl_addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cl_addr), "r"(v) : "memory");
 }
 
 __device__ __forceinline__ void cluster_sync() {
