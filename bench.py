@@ -301,7 +301,12 @@ def run_gpu(args):
     _, cod, x, tok, offs = make_inputs(args.config, rank, dev)
     n_tok = int(offs[-1])
     n_rows = sum(max(0, int(n) - 132) for n in np.diff(offs))
-    gc = D.Codec(D.upload_params(cod, dev), dev.index, CONFIGS[args.config][3])
+    params = D.upload_params(cod, dev)
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info(dev)[0]
+    gc = D.Codec(params, dev.index, CONFIGS[args.config][3])
+    torch.cuda.synchronize()
+    codec_mib = (free0 - torch.cuda.mem_get_info(dev)[0]) / 2 ** 20  # the codec's own device memory
     stream = torch.cuda.current_stream()
     blob = torch.empty(D.dckv_blob_bound(gc.handle, offs), dtype=torch.uint8, device=dev)
     k_out = torch.empty((6, n_tok, 2, 256), dtype=torch.bfloat16, device=dev)
@@ -557,6 +562,7 @@ def run_gpu(args):
         "escapes": {"count": rd["n_esc"], "rate": rd["n_esc"] / max(1, rd["n_symbols"]),
                     "of_symbols": rd["n_symbols"]},
         "components": {"kept": k_eff, "dropped": 2048 - k_eff},
+        "codec_device_mib": round(codec_mib, 1),
         "rows_per_chunk": G,
         "bytes_vs_model": payload / max(n_rows, 1) / model_bpt if model_bpt else None,
         "compression_vs_bf16": 12288.0 * n_rows / max(payload, 1),

@@ -113,14 +113,16 @@ typedef struct {
  * and scale indices (Laplace scale in steps beta = b/Delta; dropped if beta < 0.05;
  * s = clamp(round(8 log2(beta/0.05)), 0, 63)), the 64 integer Laplace tables (16-bit
  * precision, 509 residuals + ESC), the split fp16 operands of the transform, correction
- * and inverse GEMMs, and the per-vocabulary mean tables embed @ w_even and
- * embed @ w_odd[0:2048] (fp32).  chunk_rows (1..256) is the number of same-parity rows
+ * and inverse GEMMs, and the per-vocabulary mean tables of the kept components: the even
+ * centres clamp(round(embed @ w_even), +-127) (int8) and embed @ w_odd[0:2048] (fp32).
+ * chunk_rows (1..256) is the number of same-parity rows
  * per rANS chunk; 0 selects 16; -1 selects the smallest count whose fixed per-chunk bytes
  * (states, escape count, offset) stay within 3.5% of the tables' own entropy per row.
  * Fewer rows per chunk give more independent streams (faster decode) and more bytes.
- * Allocates device memory (about 2 * vocab * 8 KiB + 192 MiB: split GEMM operands, fp32
- * weight copies for the exact recomputation of near-boundary codes, tables; 16 MiB more
- * with decoder-side synthesis weights).
+ * Allocates device memory: vocab * kw * 5 bytes for the two tables (kw = kept components
+ * rounded up to 64) and about 177 MiB for the split GEMM operands, the fp32 weight copies
+ * for the exact recomputation of near-boundary codes and the coder's tables (16 MiB more
+ * with decoder-side synthesis weights); 16 MiB more during creation only.
  * Synchronises the device.  Returns DCKV_OK or an error; *out is NULL on error. */
 int dckv_codec_create(const dckv_params *params, int device, int chunk_rows, dckv_codec **out);
 void dckv_codec_destroy(dckv_codec *codec);

@@ -51,8 +51,10 @@ int dckv_ws_offsets(const dckv_codec *codec, const int64_t *seq_offsets, int bat
  * Synchronises the device. */
 int dckv_codec_export(const dckv_codec *codec, uint16_t *cdf, uint8_t *scale, uint8_t *keep, int32_t *exps);
 
-/* Device pointers of the per-vocabulary mean tables (fp32 [vocab][2048]):
- * t_even = embed @ w_even, t_odd = embed @ w_odd[0:2048]. */
+/* Device pointers of the per-vocabulary mean tables, kept components only (column kc is
+ * compact index kc, row stride kw from dckv_codec_gemm_shape), built at creation:
+ * t_even: int8 [vocab][kw], the even rows' centres clamp(round(embed @ w_even), +-127);
+ * t_odd:  fp32 [vocab][kw], embed @ w_odd[0:2048].  NULL without mean models. */
 int dckv_codec_tables(const dckv_codec *codec, const void **t_even, const void **t_odd);
 
 /* Chunk rows G in use (chosen at creation when 0 was passed) and the entropy of the kept

@@ -484,6 +484,13 @@ __global__ void k_inv_colnorms(const __half *a_inv, int kw, double *out) {
   }
 }
 
+// Even centres from the fp32 even table: out[i] = clamp(round-half-even(t[i]), +-127), the rule
+// the odd centres follow in their epilogue.
+__global__ void k_round_centres(const float *t, int64_t n, int8_t *out) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+    out[i] = (int8_t)fminf(fmaxf(rintf(t[i]), -(float)ESC_LIMIT), (float)ESC_LIMIT);
+}
+
 // Per-component constants of the kept components in compact order (pads: Delta 1, mean 0).
 __global__ void k_compact_meta(const float *delta, const float *mub, const int16_t *kept, int k_eff, int mp,
                                float *delta_k, float *mub_k) {
@@ -493,13 +500,17 @@ __global__ void k_compact_meta(const float *delta, const float *mub, const int16
   mub_k[m] = m < k_eff ? mub[kept[m]] : 0.f;
 }
 
-__global__ void k_transpose16(const uint16_t *src, int ld, int k_off, int O, int K, uint16_t *out) {
+// out[o][k] = src[k + k_off][col(o)] (16-bit), o < O; col(o) = kept[o] for o < o_valid with
+// a kept list (rows o_valid .. O - 1 zero), else o.
+__global__ void k_transpose16(const uint16_t *src, int ld, int k_off, int O, int K, uint16_t *out,
+                              const int16_t *kept = nullptr, int o_valid = 0) {
   __shared__ uint16_t tile[32][33];
   const int k0 = blockIdx.x * 32, o0 = blockIdx.y * 32;
   const int tx = threadIdx.x, ty = threadIdx.y;
   for (int y = ty; y < 32; y += 8) {
     const int k = k0 + y, o = o0 + tx;
-    tile[y][tx] = (k < K && o < O) ? src[(int64_t)(k + k_off) * ld + o] : 0;
+    const int col = kept ? (o < o_valid ? kept[o] : -1) : o;
+    tile[y][tx] = (k < K && o < O && col >= 0) ? src[(int64_t)(k + k_off) * ld + col] : 0;
   }
   __syncthreads();
   for (int y = ty; y < 32; y += 8) {
@@ -1240,8 +1251,6 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
   const uint64_t o_ah = take(2ull * 2 * N_HIDDEN * ROW_DIM);
   const uint64_t o_ainv = take(2ull * 2 * ROW_DIM * N_COEF);
   const uint64_t o_aon = take(2ull * N_COEF * 2 * N_COEF);
-  const uint64_t o_te = take(4ull * V * N_COEF);
-  const uint64_t o_to = take(4ull * V * N_COEF);
   const uint64_t o_mub = take(4ull * N_COEF);
   const uint64_t o_mubk = take(4ull * N_COEF);
   const uint64_t o_deltak = take(4ull * N_COEF);
@@ -1270,18 +1279,25 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
   const uint64_t o_v1t32 = take(has_synth ? 4ull * N_HIDDEN * N_COEF : 0);
   const uint64_t o_v2_32 = take(has_synth ? 4ull * N_HIDDEN * ROW_DIM : 0);
   const uint64_t o_zero = take(4ull * N_HIDDEN);
-  const uint64_t o_tmp = take(2ull * 2 * N_COEF * N_COEF);  // W_e^T and W_oE^T (setup only)
   const uint64_t o_scr = take(64);
-  const uint64_t o_norms = take(8ull * 2 * N_COEF);  // setup only: column norms of a_inv
   if (cudaMalloc(&c->blk, o) != cudaSuccess) return cleanup(fail(DCKV_ECUDA, "cudaMalloc(%llu) failed", (unsigned long long)o));
   uint8_t *B = (uint8_t *)c->blk;
+  // setup-only scratch, freed when creation ends: the gathered, K-major W_e^T and W_oE^T,
+  // and the inverse operand's column norms
+  struct SetupScratch {
+    void *p = nullptr;
+    ~SetupScratch() {
+      if (p) cudaFree(p);
+    }
+  } setup;
+  const uint64_t s_norms = 2ull * 2 * N_COEF * N_COEF;
+  if (cudaMalloc(&setup.p, s_norms + 8ull * 2 * N_COEF) != cudaSuccess)
+    return cleanup(fail(DCKV_ECUDA, "cudaMalloc of the setup scratch failed"));
   c->a_y = (__half *)(B + o_ay);
   c->a_w2 = (__half *)(B + o_aw2);
   c->a_h = (__half *)(B + o_ah);
   c->a_inv = (__half *)(B + o_ainv);
   c->a_on = (__nv_bfloat16 *)(B + o_aon);
-  c->t_even = (float *)(B + o_te);
-  c->t_odd = (float *)(B + o_to);
   c->mub = (float *)(B + o_mub);
   c->mub_k = (float *)(B + o_mubk);
   c->delta_k = (float *)(B + o_deltak);
@@ -1310,7 +1326,7 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
   c->v1t32 = (float *)(B + o_v1t32);
   c->v2_32 = (float *)(B + o_v2_32);
   c->zero256 = (float *)(B + o_zero);
-  uint16_t *tmp_e = (uint16_t *)(B + o_tmp);
+  uint16_t *tmp_e = (uint16_t *)setup.p;  // [mp][2048] each, kept components
   uint16_t *tmp_oe = tmp_e + (size_t)N_COEF * N_COEF;
   int32_t *scr = (int32_t *)(B + o_scr);
   cudaStream_t st = 0;
@@ -1456,8 +1472,10 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
   if (has_means) {
     { k_gather_on<<<dim3(2 * c->kw / 32, c->mp / 32), tb, 0, st>>>(prm->w_odd, c->kept_list, c->k_eff, c->kw, c->mp,
                                                                   (uint16_t *)c->a_on); ++g_launches; }
-    { k_transpose16<<<dim3(N_COEF / 32, N_COEF / 32), tb, 0, st>>>(prm->w_even, N_COEF, 0, N_COEF, N_COEF, tmp_e); ++g_launches; }
-    { k_transpose16<<<dim3(N_COEF / 32, N_COEF / 32), tb, 0, st>>>(prm->w_odd, N_COEF, 0, N_COEF, N_COEF, tmp_oe); ++g_launches; }
+    { k_transpose16<<<dim3(N_COEF / 32, c->mp / 32), tb, 0, st>>>(prm->w_even, N_COEF, 0, c->mp, N_COEF, tmp_e,
+                                                                 c->kept_list, c->k_eff); ++g_launches; }
+    { k_transpose16<<<dim3(N_COEF / 32, c->mp / 32), tb, 0, st>>>(prm->w_odd, N_COEF, 0, c->mp, N_COEF, tmp_oe,
+                                                                 c->kept_list, c->k_eff); ++g_launches; }
   }
   if (cudaGetLastError() != cudaSuccess) return cleanup(fail(DCKV_ECUDA, "setup kernels failed to launch"));
   // tensor maps of the static operands
@@ -1479,7 +1497,7 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
   // variant keeps the whole split (its extra operand takes the second tensor map).
   c->inv_lo_k = c->kw;
   if (!has_synth && c->k_eff > 0) {
-    double *norms = (double *)(B + o_norms);
+    double *norms = (double *)((uint8_t *)setup.p + s_norms);
     { k_inv_colnorms<<<c->kw, 256, 0, st>>>(c->a_inv, c->kw, norms); ++g_launches; }
     std::vector<double> nh(2 * (size_t)c->kw);
     std::vector<float> bh(N_COEF), dh(N_COEF);
@@ -1504,18 +1522,29 @@ extern "C" int dckv_codec_create(const dckv_params *prm, int device, int chunk_r
     }
     c->inv_lo_k = std::min(c->kw, (cut + 63) / 64 * 64);
   }
-  // per-vocabulary mean tables: t_even = embed @ w_even, t_odd = embed @ w_odd[0:2048]
+  // per-vocabulary mean tables of the kept components (column kc = compact index), row
+  // stride kw: t_odd = embed @ w_odd[0:2048] in fp32 and, since an even row's centre is the
+  // table value itself, the even centres clamp(round(embed @ w_even), +-127) as int8 (the
+  // fp32 even table passes through the odd table's buffer first)
   if (has_means) {
+    if (cudaMalloc(&c->tab_blk, (size_t)V * c->kw * 5) != cudaSuccess)
+      return cleanup(fail(DCKV_ECUDA, "cudaMalloc of the vocabulary tables failed"));
+    c->t_odd = (float *)c->tab_blk;
+    c->t_even8 = (int8_t *)c->tab_blk + (size_t)V * c->kw * 4;
     CUtensorMap ma_e, ma_o, mb_emb;
-    if ((r = map_a(&ma_e, tmp_e, true, N_COEF, N_COEF, 1, 1)) || (r = map_a(&ma_o, tmp_oe, true, N_COEF, N_COEF, 1, 1)) ||
+    if ((r = map_a(&ma_e, tmp_e, true, N_COEF, c->mp, 1, 1)) || (r = map_a(&ma_o, tmp_oe, true, N_COEF, c->mp, 1, 1)) ||
         (r = map_b(&mb_emb, prm->embed, true, N_COEF, V, 256)))
       return cleanup(r);
     for (int which = 0; which < 2; ++which) {
-      GemmProblem pr = make_problem(N_COEF / GEMM_BM, (int64_t)V, 256, true, scr + 5);
+      GemmProblem pr = make_problem(c->mp / GEMM_BM, (int64_t)V, 256, true, scr + 5);
       add_seg(pr, 0, 0, 1, 0, 0, 0, 0, N_COEF / GEMM_BK);
-      EpiStoreF32::Params ep{which ? c->t_odd : c->t_even, N_COEF, 1.0f};
+      EpiStoreF32::Params ep{c->t_odd, c->kw, 1.0f, c->kw};
       if ((r = run_gemm<EpiStoreF32, 4, 1>(which ? ma_o : ma_e, ma_e, mb_emb, mb_emb, pr, ep, c->num_sms, st)))
         return cleanup(r);
+      if (which == 0) {
+        const int64_t n = (int64_t)V * c->kw;
+        { k_round_centres<<<(unsigned)std::min<int64_t>((n + 255) / 256, 65535), 256, 0, st>>>(c->t_odd, n, c->t_even8); ++g_launches; }
+      }
     }
   }
   if (cudaDeviceSynchronize() != cudaSuccess)
@@ -1531,6 +1560,7 @@ extern "C" void dckv_codec_destroy(dckv_codec *c) {
   if (!c) return;
   DeviceScope dev_scope(c->device);
   if (c->blk) cudaFree(c->blk);
+  if (c->tab_blk) cudaFree(c->tab_blk);
   if (t_stages.codec == c) t_stages.codec = nullptr;
   delete c;
 }
@@ -1723,7 +1753,7 @@ static int encode_impl(const dckv_codec *c, const void *rows, const int32_t *tok
       GemmProblem pr = make_problem(c->mp / GEMM_BM, L.ne_pad, MEAN_ODD_BN, true, status_dev);
       add_seg(pr, 0, 0, 1, 0, 0, 0, 0, c->kw / GEMM_BK);
       add_seg(pr, 0, 0, 1, c->kw, 0, 1, 0, c->kw / GEMM_BK);
-      EpiMeanOdd<false>::Params ep{c->t_odd, token_ids, e_tok, e_slot, c->kept_list, cen8, c->k_eff, c->vocab};
+      EpiMeanOdd<false>::Params ep{c->t_odd, token_ids, e_tok, e_slot, c->kw, cen8, c->k_eff, c->vocab};
       RET((run_gemm2<EpiMeanOdd<false>, 6, 1, 8, MEAN_ODD_BN>(c->map_aon1, c->map_aon1, mb_qe, mb_qe, pr, ep, c->num_sms, true, st)));
     }
     stage_mark(c, st, "gemm_mean_odd");
@@ -1731,8 +1761,8 @@ static int encode_impl(const dckv_codec *c, const void *rows, const int32_t *tok
     const unsigned rg = (unsigned)std::min<int64_t>(L.n_rows, 65535);
     if (!c->has_means && L.n_symbols > 0)
       CK(cudaMemsetAsync(cen8, 0, (size_t)L.n_symbols, st));  // unconditional tables: every centre 0
-    { k_symbols<<<rg, SYM_THREADS, 0, st>>>(L.n_rows, row_slot, slot_chunk, q32, cen8, c->kept_list, c->kept_scale,
-                                          c->cfm_tab, c->k_eff, c->has_means ? c->t_even : nullptr, token_ids,
+    { k_symbols<<<rg, SYM_THREADS, 0, st>>>(L.n_rows, row_slot, slot_chunk, q32, cen8, c->kept_scale, c->cfm_tab,
+                                          c->k_eff, c->has_means ? c->t_even8 : nullptr, c->kw, token_ids,
                                           row_tok, row_edst, c->vocab, sym16, cfm, nesc_w); ++g_launches; }
     CK(cudaGetLastError());
     stage_mark(c, st, "symbols");
@@ -1826,7 +1856,7 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
   const uint32_t *offs = (const uint32_t *)(bl + HEADER_BYTES + 4ull * L.batch);
   if (L.n_rows > 0 && c->has_means) {
     k_centres_even<<<(unsigned)std::min<int64_t>(L.n_rows, 65535), 256, 0, st>>>(
-        L.n_rows, row_slot, row_edst, row_tok, token_ids, c->t_even, c->vocab, c->kept_list, c->k_eff, cen8, valid);
+        L.n_rows, row_slot, row_edst, row_tok, token_ids, c->t_even8, c->kw, c->vocab, c->k_eff, cen8, valid);
     ++g_launches;
   } else if (L.n_symbols > 0) {
     CK(cudaMemsetAsync(cen8, 0, (size_t)L.n_symbols, st));  // unconditional tables: every centre 0
@@ -1863,7 +1893,7 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
     add_seg(pr, 0, 0, 1, 0, 0, 0, 0, c->kw / GEMM_BK);
     add_seg(pr, 0, 0, 1, c->kw, 0, 1, 0, c->kw / GEMM_BK);
     // odd centres, and with them the odd codes (ESC symbols are left to the patch)
-    EpiMeanOdd<true>::Params ep{c->t_odd, token_ids, e_tok, e_slot, c->kept_list, cen8, c->k_eff, c->vocab,
+    EpiMeanOdd<true>::Params ep{c->t_odd, token_ids, e_tok, e_slot, c->kw, cen8, c->k_eff, c->vocab,
                                 syms16, q16, e_row, slot_chunk, escflag};
     RET((run_gemm2<EpiMeanOdd<true>, 6, 1, 8, MEAN_ODD_BN>(c->map_aon1, c->map_aon1, mb_qe, mb_qe, pr, ep, c->num_sms, true, st)));
   }
@@ -2037,7 +2067,7 @@ extern "C" int dckv_codec_gemm_shape(const dckv_codec *c, int32_t *shape) {
 
 extern "C" int dckv_codec_tables(const dckv_codec *c, const void **t_even, const void **t_odd) {
   if (!c) return fail(DCKV_EINVAL, "NULL codec");
-  if (t_even) *t_even = c->t_even;
+  if (t_even) *t_even = c->t_even8;
   if (t_odd) *t_odd = c->t_odd;
   return DCKV_OK;
 }

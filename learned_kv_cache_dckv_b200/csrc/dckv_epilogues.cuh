@@ -28,6 +28,7 @@ struct EpiStoreF32 {
     float *out;
     int64_t ld;
     float scale;
+    int m_valid = 1 << 30;  // features m >= m_valid are not stored
   };
   static constexpr int SMEM_BYTES = 0;
   __device__ __forceinline__ static void tile(const Params &p, const EpiCtx &cx) {
@@ -38,7 +39,7 @@ struct EpiStoreF32 {
       tmem_ld_wait();
 #pragma unroll
       for (int j = 0; j < 32; ++j)
-        if (c0 + j < cx.n_valid) p.out[(int64_t)(cx.n0 + c0 + j) * p.ld + m] = u2f(r[j]) * p.scale;
+        if (c0 + j < cx.n_valid && m < p.m_valid) p.out[(int64_t)(cx.n0 + c0 + j) * p.ld + m] = u2f(r[j]) * p.scale;
     }
   }
 };
@@ -236,17 +237,18 @@ struct EpiQuantRegs {
 };
 
 // ------------------------------------------------------------------ odd mean model
-// mu = D + (embed @ w_odd[0:2048])[token][c]  (code units);  centre = clamp(round(mu), +-127)
+// mu = D + (embed @ w_odd[0:2048])[token][c]  (code units);  centre = clamp(round(mu), +-127);
+// the table holds kept components only, compact index kc at column kc
 // Tile columns are padded even rows e; column e is the odd row whose left neighbour is
 // even row e (e_tok[e] = its token's row in the batch, or -1 where there is no odd row).
 template <bool DEC>  // false: the encoder's centres; true: the decoder's odd codes
 struct EpiMeanOdd {
   struct Params {
-    const float *t_odd;      // [vocab][2048]
+    const float *t_odd;      // [vocab][t_ld], kept components (compact)
     const int32_t *tok_ids;  // [tokens]
     const int32_t *e_tok;    // [ne_pad] token row of the odd row, -1 if none
     const int32_t *e_slot;   // [ne_pad] slot row of that odd row
-    const int16_t *kept_list;  // compact index -> component (the GEMM's features are kept components)
+    int t_ld;                // row stride of t_odd (kw)
     int8_t *cen8;            // [slots][k_eff]  (encoder: the odd centres)
     int k_eff;
     int vocab;
@@ -271,7 +273,7 @@ struct EpiMeanOdd {
       int64_t off = -1;
       if (ti >= 0) {
         const int tok = min(max(__ldg(p.tok_ids + ti), 0), p.vocab - 1);
-        off = (int64_t)tok * N_COEF;
+        off = (int64_t)tok * p.t_ld;
       }
       s_row[j] = off;
       s_slot[j] = __ldg(p.e_slot + cx.n0 + j);
@@ -280,7 +282,6 @@ struct EpiMeanOdd {
     named_bar_sync(cx.bar, 128);
     const int kc0 = cx.mt * GEMM_BM + cx.ew * 32 + cx.lane;  // compact index of this thread's feature
     const int kc = kc0 < p.k_eff ? kc0 : -1;
-    const int c = kc >= 0 ? p.kept_list[kc] : 0;  // its component (t_odd column)
     for (int c0 = cx.grp * 32; c0 < n_valid; c0 += 32 * cx.n_grp) {
       uint32_t r[32];
       tmem_ld_32x32b_x32(cx.tacc + (uint32_t)c0, r);
@@ -289,7 +290,7 @@ struct EpiMeanOdd {
 #pragma unroll
       for (int j = 0; j < 32; ++j) {  // independent loads, issued together
         const int64_t off = (kc >= 0 && c0 + j < n_valid) ? s_row[c0 + j] : -1;
-        tv[j] = off >= 0 ? __ldg(p.t_odd + off + c) : 0.f;
+        tv[j] = off >= 0 ? __ldg(p.t_odd + off + kc) : 0.f;
         if constexpr (DEC) sv[j] = off >= 0 ? __ldg(p.syms + (int64_t)s_slot[c0 + j] * p.k_eff + kc) : (uint16_t)0;
       }
       tmem_ld_wait();

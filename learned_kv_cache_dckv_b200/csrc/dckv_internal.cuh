@@ -137,14 +137,15 @@ struct dckv_codec {
   // caller-owned parameter pointers (read at create)
   dckv_params p{};
   // derived, library-owned device buffers
-  void *blk = nullptr;  // one allocation holding everything below
+  void *blk = nullptr;  // one allocation holding everything below but the vocabulary tables
+  void *tab_blk = nullptr;  // the vocabulary tables (sized by kw, known after the keep mask)
   __half *a_y = nullptr;     // [2][mp][6144]  basis^T * 2^p_y, split hi/lo, kept components (zero rows after)
   __half *a_w2 = nullptr;    // [2][mp][256]   w2^T * 2^p_y, split, kept components
   __half *a_h = nullptr;     // [2][256][6144] w1^T * 2^p_h, split
   __half *a_inv = nullptr;   // [2][6144][kw]  (Delta_c basis[d][c]) * 2^p_inv, dims permuted, kept c
   __nv_bfloat16 *a_on = nullptr;  // [mp][2 kw]  odd mean model, neighbour blocks, kept in and out
-  float *t_even = nullptr;   // [vocab][2048]  embed @ w_even
-  float *t_odd = nullptr;    // [vocab][2048]  embed @ w_odd[0:2048]
+  int8_t *t_even8 = nullptr;  // [vocab][kw]  clamp(round(embed @ w_even), +-127), kept components
+  float *t_odd = nullptr;     // [vocab][kw]  embed @ w_odd[0:2048], kept components
   float *mub = nullptr;      // [2048]  mu @ basis
   float *mub_k = nullptr;    // [mp]    mu @ basis of kept components (0 after)
   float *delta_k = nullptr;  // [mp]    Delta of kept components (1 after)

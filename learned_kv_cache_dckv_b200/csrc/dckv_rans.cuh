@@ -51,30 +51,30 @@ __device__ __forceinline__ void copy_smem16(void *dst, const void *src, int byte
 __device__ __forceinline__ uint32_t cdf_at(const uint16_t *tab, int k) { return k < N_SYM ? tab[k] : PREC_TOTAL; }
 
 // ------------------------------------------------------------------------------ symbols
-// Centres of even rows for the decoder, clamp(round(T_even[token][c]), +-127), in slot order.
+// Centres of even rows for the decoder, in slot order: the row of the even-centre table
+// (clamp(round(T_even[token][c]), +-127), kept components, computed at codec creation).
 __global__ void __launch_bounds__(256) k_centres_even(int64_t n_rows, const int32_t *row_slot,
                                                       const int32_t *row_edst, const int32_t *row_tok,
-                                                      const int32_t *tok_ids, const float *t_even, int vocab,
-                                                      const int16_t *kept_list, int k_eff, int8_t *cen8,
-                                                      const int32_t *valid) {
+                                                      const int32_t *tok_ids, const int8_t *t_even8, int t_ld,
+                                                      int vocab, int k_eff, int8_t *cen8, const int32_t *valid) {
   if (valid && *valid != 1) return;
   for (int64_t row = blockIdx.x; row < n_rows; row += gridDim.x) {
     if (row_edst[row] < 0) continue;
     int tok = tok_ids[row_tok[row]];
     tok = min(max(tok, 0), vocab - 1);
-    const float *te = t_even + (int64_t)tok * N_COEF;
+    const int8_t *te = t_even8 + (int64_t)tok * t_ld;
     int8_t *dst = cen8 + (int64_t)row_slot[row] * k_eff;
     constexpr int PER = N_COEF / 256;  // blockDim.x == 256: every load before the stores
-    float mu[PER];
+    int8_t v[PER];
 #pragma unroll
     for (int u = 0; u < PER; ++u) {
       const int k = threadIdx.x + 256 * u;
-      mu[u] = k < k_eff ? __ldg(te + __ldg(kept_list + k)) : 0.f;
+      v[u] = k < k_eff ? te[k] : (int8_t)0;
     }
 #pragma unroll
     for (int u = 0; u < PER; ++u) {
       const int k = threadIdx.x + 256 * u;
-      if (k < k_eff) dst[k] = (int8_t)fminf(fmaxf(rintf(mu[u]), -(float)ESC_LIMIT), (float)ESC_LIMIT);
+      if (k < k_eff) dst[k] = v[u];
     }
   }
 }
@@ -86,27 +86,19 @@ __global__ void __launch_bounds__(256) k_centres_even(int64_t n_rows, const int3
 constexpr int SYM_THREADS = 256;
 constexpr int SYM_UNROLL = 4;
 
-// Even rows take their centres straight from the vocabulary table t_even (and store them
-// in cen8 too, where the odd rows' centres already are); with t_even NULL (no mean models)
-// every centre is 0.
-__device__ __forceinline__ int even_centre(const float *t_row, int comp) {
-  return (int)fminf(fmaxf(rintf(__ldg(t_row + comp)), -(float)ESC_LIMIT), (float)ESC_LIMIT);
-}
+// Even rows take their centres straight from the even-centre table (and store them in
+// cen8 too, where the odd rows' centres already are); with no table (no mean models) every
+// centre is 0.
 
 __global__ void __launch_bounds__(SYM_THREADS) k_symbols(int64_t n_rows, const int32_t *row_slot,
                                                          const int32_t *slot_chunk, const int32_t *q32,
-                                                         int8_t *cen8, const int16_t *kept_list,
-                                                         const uint8_t *kept_scale, const uint2 *cfm_tab, int k_eff,
-                                                         const float *t_even, const int32_t *tok_ids,
+                                                         int8_t *cen8, const uint8_t *kept_scale, const uint2 *cfm_tab, int k_eff,
+                                                         const int8_t *t_even8, int t_ld, const int32_t *tok_ids,
                                                          const int32_t *row_tok, const int32_t *row_edst, int vocab,
                                                          uint16_t *sym16, uint2 *cfm, uint32_t *nesc) {
   __shared__ int esc_count;
-  __shared__ int16_t s_kl[N_COEF];
   __shared__ uint8_t s_ks[N_COEF];
-  for (int k = threadIdx.x; k < k_eff; k += SYM_THREADS) {
-    s_kl[k] = kept_list[k];
-    s_ks[k] = kept_scale[k];
-  }
+  for (int k = threadIdx.x; k < k_eff; k += SYM_THREADS) s_ks[k] = kept_scale[k];
   for (int64_t row = blockIdx.x; row < n_rows; row += gridDim.x) {
     if (threadIdx.x == 0) esc_count = 0;
     __syncthreads();
@@ -114,8 +106,8 @@ __global__ void __launch_bounds__(SYM_THREADS) k_symbols(int64_t n_rows, const i
     const int64_t base = (int64_t)slot * k_eff;
     const int32_t *q = q32 + row * CODE_LD;  // compact: kept component k at column k
     const bool even = row_edst[row] >= 0;
-    const float *t_row = nullptr;
-    if (even && t_even) t_row = t_even + (int64_t)min(max(tok_ids[row_tok[row]], 0), vocab - 1) * N_COEF;
+    const int8_t *t_row = nullptr;
+    if (even && t_even8) t_row = t_even8 + (int64_t)min(max(tok_ids[row_tok[row]], 0), vocab - 1) * t_ld;
     int esc = 0;
     for (int k0 = threadIdx.x; k0 < k_eff; k0 += SYM_UNROLL * SYM_THREADS) {
       int v[SYM_UNROLL], ce[SYM_UNROLL];
@@ -123,7 +115,7 @@ __global__ void __launch_bounds__(SYM_THREADS) k_symbols(int64_t n_rows, const i
       for (int u = 0; u < SYM_UNROLL; ++u) {
         const int k = k0 + u * SYM_THREADS;
         v[u] = k < k_eff ? __ldg(q + k) : 0;
-        ce[u] = k >= k_eff ? 0 : even ? (t_row ? even_centre(t_row, s_kl[k]) : 0) : (int)__ldg(cen8 + base + k);
+        ce[u] = k >= k_eff ? 0 : even ? (t_row ? (int)__ldg(t_row + k) : 0) : (int)__ldg(cen8 + base + k);
       }
 #pragma unroll
       for (int u = 0; u < SYM_UNROLL; ++u) {

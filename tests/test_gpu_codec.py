@@ -299,6 +299,39 @@ def test_compacted_gemm_shapes_and_inverse_lo_cut(src, codec_55):
     assert 0 < shp["inv_lo_k"] < shp["kw"]  # the cut is in use on this codec
 
 
+def test_vocabulary_tables_kept_components(codec_55, codec_centred):
+    """The per-vocabulary tables hold the kept components only, column kc = compact index,
+    row stride kw: the even table is the even rows' centres themselves (int8), equal to
+    the oracle's centres of mu = e(token) W_e except where mu lies within 1e-4 of a
+    half-step boundary (fp32 vs fp64 sums); the odd table is e(token) W_oE within fp32
+    accumulation error (2^-12 of sum |e||W|); pad columns are zero.  Checked on 2,048
+    sampled vocabulary rows plus the first and last."""
+    for cod in (codec_55, codec_centred):
+        gc = gpu_codec(cod)
+        shp = D.dckv_codec_gemm_shape(gc.handle)
+        k, kw = shp["k_eff"], shp["kw"]
+        V = cod.embed.shape[0]
+        te_p, to_p = D.dckv_codec_tables(gc.handle)
+        te = torch.as_tensor(_CAI(te_p, (V, kw), "|i1"), device="cuda").cpu().numpy()
+        to = torch.as_tensor(_CAI(to_p, (V, kw), "<f4"), device="cuda").cpu().numpy()
+        kl = np.nonzero(O.scale_index(cod.laplace_b, cod.delta)[1])[0]
+        rows = np.unique(np.concatenate([[0, V - 1], np.random.default_rng(7).choice(V, 2048, replace=False)]))
+        e = O.bf16_to_f64(cod.embed[rows])
+        w_e = O.bf16_to_f64(cod.w_even)[:, kl]
+        w_o = O.bf16_to_f64(cod.w_odd[:2048])[:, kl]
+        mu_e = e @ w_e
+        near = np.abs(np.abs(mu_e - np.floor(mu_e)) - 0.5) < CENTRE_WINDOW
+        ce = O.centres(mu_e)
+        got = te[rows, :k].astype(np.int64)
+        assert np.array_equal(got[~near], ce[~near])
+        assert np.all(np.abs(got[near] - ce[near]) <= 1)
+        assert np.all(te[:, k:] == 0) and np.all(to[:, k:] == 0)
+        mu_o = e @ w_o
+        bound = 2.0 ** -12 * (np.abs(e) @ np.abs(w_o)) + 1e-30
+        assert np.all(np.abs(to[rows, :k].astype(np.float64) - mu_o) <= bound)
+    assert np.count_nonzero(got) > got.size // 4  # codec_centred: the even centres are not all 0
+
+
 def test_parity_literal_small_config(src, codec_literal):
     # one prompt of 256 tokens (124 coded rows) plus ragged neighbours and degenerate prompts
     full_check(src, codec_literal, [256, 700, 50, 132, 133, 134], seeds=[0, 1, 2, 3, 4, 5])
