@@ -1700,7 +1700,15 @@ static int encode_impl(const dckv_codec *c, const void *rows, const int32_t *tok
     RET(map_b(&mb_gt, g16, false, 2 * N_HIDDEN, L.n_rows, TRANSFORM_BN / 2));
     RET(map_b(&mb_qe, qe, true, c->kw, L.ne_pad, MEAN_ODD_BN / 2, CODE_LD));
     // correction hidden layer: h = x @ w1 - mu @ w1, GELU, fp16 hi/lo
-    if (c->has_mlp) {
+    if (c->has_mlp && (L.n_rows + HIDDEN_SPLIT_BN - 1) / HIDDEN_SPLIT_BN >= c->num_sms) {
+      // enough token tiles for two per CTA pair: the K parts are summed in registers by the
+      // chunk-accumulated kernel, whose epilogue applies GELU (no fp32 parts in memory)
+      GemmProblem pr = make_problem(N_HIDDEN / GEMM_BM, L.n_rows, HIDDEN_SPLIT_BN, false, status_dev);
+      add_seg(pr, 0, 0, 2, 0, 0, 0, 0, ROW_DIM / GEMM_BK);
+      EpiGeluRegs::Params ep{c->muw1, (float)std::ldexp(1.0, -c->p_h), g16};
+      RET((run_gemm2_chunked<EpiGeluRegs, 4, 2, ROW_DIM / GEMM_BK / HIDDEN_SPLIT, HIDDEN_SPLIT_BN>(
+          c->map_ah2, c->map_ah2, mb_xh, mb_xh, pr, ep, c->num_sms, false, st)));
+    } else if (c->has_mlp) {
       GemmProblem pr = make_problem(N_HIDDEN / GEMM_BM, L.n_rows, HIDDEN_SPLIT_BN, false, status_dev);
       add_seg(pr, 0, 0, 2, 0, 0, 0, 0, ROW_DIM / GEMM_BK);
       pr.k_split = HIDDEN_SPLIT;

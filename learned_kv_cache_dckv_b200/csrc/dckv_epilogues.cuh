@@ -133,6 +133,34 @@ struct EpiGelu {
   }
 };
 
+// The same layer on the chunk-accumulated CTA-pair kernel: the totals it hands over are the
+// fp32 sums, in order, of the TMEM partials of consecutive K parts, the very sums that
+// k_gelu_parts forms from the split-K kernel's parts, so G is bit-identical either way.
+struct EpiGeluRegs {
+  using Params = EpiGelu::Params;
+  static constexpr int SMEM_BYTES = 16;
+  __device__ __forceinline__ static void stage(const Params &, char *, int, int, int, int) {}
+  template <int NC>
+  __device__ __forceinline__ static void finish(const Params &p, const char *, const float (&tot)[NC], int mt, int n0,
+                                                int n_valid, int col0, int ew, int lane) {
+    const int m = mt * GEMM_BM + ew * 32 + lane;
+    const float mw = p.muw1[m];
+#pragma unroll
+    for (int j = 0; j < NC; ++j) {
+      const int col = col0 + j;
+      if (col < n_valid) {
+        const float h = tot[j] * p.scale - mw;
+        const float g = 0.5f * h * (1.0f + erff(h * 0.70710678118654752f));
+        const __half hi = __float2half_rn(g);
+        const __half lo = __float2half_rn(g - __half2float(hi));
+        __half *row = p.g + (int64_t)(n0 + col) * (2 * N_HIDDEN);
+        row[m] = hi;
+        row[N_HIDDEN + m] = lo;
+      }
+    }
+  }
+};
+
 // ------------------------------------------------------------------ transform + quantiser
 // y = D * 2^-p_y - (mu @ basis)[c];  q = round_half_even(y / Delta_c), 0 if dropped;
 // q32[row][c] = q; even rows also write bf16(q) to their padded even row (the odd mean

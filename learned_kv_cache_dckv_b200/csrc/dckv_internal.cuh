@@ -58,8 +58,11 @@ constexpr int MEAN_ODD_BN = 256;
 constexpr int INVERSE_BN = 256;
 // Hidden layers (256 rows of M, one pair tile): the decoder's synthesis layer runs narrow
 // 64-token tiles (62 pairs for a 4K-token prompt); the encoder's correction layer, K = 6,144,
-// runs 256-token tiles with K cut into HIDDEN_SPLIT parts (64 pairs), each tile then reading
-// its A slice once per 256 tokens instead of once per 64, and sums the parts afterwards.
+// runs 256-token tiles with K cut into HIDDEN_SPLIT parts.  A batch with fewer token tiles
+// than SMs runs every part as its own tile (64 pairs for a 4K-token prompt: each tile reads
+// its A slice once per 256 tokens instead of once per 64) and sums the parts afterwards; a
+// larger batch runs each tile's parts as consecutive TMEM partials summed in registers, in
+// the same order, so the hidden units are bit-identical on both paths.
 constexpr int HIDDEN_BN = 64;
 constexpr int HIDDEN_SPLIT_BN = 256;
 constexpr int HIDDEN_SPLIT = 4;

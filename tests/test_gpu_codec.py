@@ -332,6 +332,32 @@ def test_vocabulary_tables_kept_components(codec_55, codec_centred):
     assert np.count_nonzero(got) > got.size // 4  # codec_centred: the even centres are not all 0
 
 
+def test_hidden_layer_identical_across_batch_sizes(src, codec_55):
+    """A batch with at least as many 256-token tiles as SMs sums the correction layer's four
+    K parts in registers; a small batch writes the parts and sums them in a second kernel.
+    Both add the same fp32 partials in the same order, so the hidden units (hi/lo fp16) and
+    the codes of a prompt are bit-identical whichever batch it is coded in."""
+    gc = gpu_codec(codec_55)
+    n_sm = torch.cuda.get_device_properties(0).multi_processor_count
+    n_big = -(-n_sm * 256 // (4096 - 132)) + 1  # prompts of 4,096 tokens: tiles >= SMs
+    got = {}
+    for lens in ([4096], [4096] * n_big):
+        x, tok, offs = S.batch(src, lens, list(range(100, 100 + len(lens))), device="cuda")
+        gc.encode(x, tok, offs)
+        torch.cuda.synchronize()
+        assert int(gc.status.item()) == 0
+        v = D.dckv_ws_offsets(gc.handle, offs, 0)
+        assert -(-v["n_rows"] // 256) >= n_sm or len(lens) == 1
+        n0 = 4096 - 132  # the first prompt's coded rows come first in either batch
+        g = gc._ws[v["g16"]: v["g16"] + 2 * 512 * n0].view(torch.int16).cpu().numpy()
+        got[len(lens)] = (g, gc.workspace_codes(offs, 0, rows=np.arange(n0)))
+        del x
+    (g1, q1), (g2, q2) = got[1], got[n_big]
+    assert np.array_equal(g1, g2)
+    assert np.array_equal(q1, q2)
+    assert np.count_nonzero(g1) > g1.size // 2
+
+
 def test_parity_literal_small_config(src, codec_literal):
     # one prompt of 256 tokens (124 coded rows) plus ragged neighbours and degenerate prompts
     full_check(src, codec_literal, [256, 700, 50, 132, 133, 134], seeds=[0, 1, 2, 3, 4, 5])
