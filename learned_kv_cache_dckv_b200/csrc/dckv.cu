@@ -1762,7 +1762,7 @@ static int encode_impl(const dckv_codec *c, const void *rows, const int32_t *tok
       add_seg(pr, 0, 0, 1, 0, 0, 0, 0, c->kw / GEMM_BK);
       add_seg(pr, 0, 0, 1, c->kw, 0, 1, 0, c->kw / GEMM_BK);
       EpiMeanOdd<false>::Params ep{c->t_odd, token_ids, e_tok, e_slot, c->kw, cen8, c->k_eff, c->vocab};
-      RET((run_gemm2<EpiMeanOdd<false>, 6, 1, 8, MEAN_ODD_BN>(c->map_aon1, c->map_aon1, mb_qe, mb_qe, pr, ep, c->num_sms, true, st)));
+      RET((run_gemm2<EpiMeanOdd<false>, 6, 1, 16, MEAN_ODD_BN>(c->map_aon1, c->map_aon1, mb_qe, mb_qe, pr, ep, c->num_sms, true, st)));
     }
     stage_mark(c, st, "gemm_mean_odd");
     // even centres from the vocabulary table, then every symbol, in slot order
@@ -1903,7 +1903,7 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
     // odd centres, and with them the odd codes (ESC symbols are left to the patch)
     EpiMeanOdd<true>::Params ep{c->t_odd, token_ids, e_tok, e_slot, c->kw, cen8, c->k_eff, c->vocab,
                                 syms16, q16, e_row, slot_chunk, escflag};
-    RET((run_gemm2<EpiMeanOdd<true>, 6, 1, 8, MEAN_ODD_BN>(c->map_aon1, c->map_aon1, mb_qe, mb_qe, pr, ep, c->num_sms, true, st)));
+    RET((run_gemm2<EpiMeanOdd<true>, 6, 1, 16, MEAN_ODD_BN>(c->map_aon1, c->map_aon1, mb_qe, mb_qe, pr, ep, c->num_sms, true, st)));
   }
   stage_mark(c, st, "gemm_mean_odd");
   if (L.n_chunks_o > 0) {

@@ -290,6 +290,9 @@ struct EpiMeanOdd {
   };
   // per tile column: t_odd row offset (or -1), slot row and natural row (each group its own)
   static constexpr int SMEM_BYTES = 256 * 16;
+  // columns per accumulator load: groups take 16-column chunks in turn (four groups of four
+  // warps at 256-column tiles: four chunks per warp and tile)
+  static constexpr int CW = 16;
   __device__ __forceinline__ static void tile(const Params &p, const EpiCtx &cx) {
     int64_t *s_row = reinterpret_cast<int64_t *>(cx.scratch);
     int32_t *s_slot = reinterpret_cast<int32_t *>(cx.scratch + 256 * 8);
@@ -310,13 +313,13 @@ struct EpiMeanOdd {
     named_bar_sync(cx.bar, 128);
     const int kc0 = cx.mt * GEMM_BM + cx.ew * 32 + cx.lane;  // compact index of this thread's feature
     const int kc = kc0 < p.k_eff ? kc0 : -1;
-    for (int c0 = cx.grp * 32; c0 < n_valid; c0 += 32 * cx.n_grp) {
-      uint32_t r[32];
-      tmem_ld_32x32b_x32(cx.tacc + (uint32_t)c0, r);
-      float tv[32];
-      uint16_t sv[DEC ? 32 : 1];
+    for (int c0 = cx.grp * CW; c0 < n_valid; c0 += CW * cx.n_grp) {
+      uint32_t r[CW];
+      tmem_ld_32x32b_x16(cx.tacc + (uint32_t)c0, r);
+      float tv[CW];
+      uint16_t sv[DEC ? CW : 1];
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {  // independent loads, issued together
+      for (int j = 0; j < CW; ++j) {  // independent loads, issued together
         const int64_t off = (kc >= 0 && c0 + j < n_valid) ? s_row[c0 + j] : -1;
         tv[j] = off >= 0 ? __ldg(p.t_odd + off + kc) : 0.f;
         if constexpr (DEC) sv[j] = off >= 0 ? __ldg(p.syms + (int64_t)s_slot[c0 + j] * p.k_eff + kc) : (uint16_t)0;
@@ -324,7 +327,7 @@ struct EpiMeanOdd {
       tmem_ld_wait();
       if (kc < 0) continue;
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
+      for (int j = 0; j < CW; ++j) {
         if (c0 + j < n_valid && s_row[c0 + j] >= 0) {
           const float mu = u2f(r[j]) + tv[j];
           const float cen = fminf(fmaxf(rintf(mu), -(float)ESC_LIMIT), (float)ESC_LIMIT);
