@@ -837,35 +837,6 @@ __device__ __forceinline__ double bf16_bits_to_f64(uint32_t w) {
 // b sits in shared memory as fp64, element 8 v + j at b[j * 768 + v], so that the lanes of
 // a warp read consecutive words (no bank conflicts).  Products of a bf16 and an fp32 value
 // are exact in fp64.
-constexpr int DOT_GROUPS = ROW_DIM / 8;  // 768
-
-__device__ __forceinline__ double row_dot_smem(const uint4 *xr, const double *b, int lane) {
-  constexpr int R = ROW_DIM / 8 / 32;  // 24 groups per lane
-  constexpr int H = R / 2;
-  double part[8];
-#pragma unroll
-  for (int u = 0; u < 8; ++u) part[u] = 0.0;
-#pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    uint4 xv[H];
-#pragma unroll
-    for (int r = 0; r < H; ++r) xv[r] = __ldg(xr + (half * H + r) * 32 + lane);
-#pragma unroll
-    for (int r = 0; r < H; ++r) {
-      const double *bb = b + (half * H + r) * 32 + lane;
-      part[0] = fma(bf16_bits_to_f64(xv[r].x & 0xFFFFu), bb[0 * DOT_GROUPS], part[0]);
-      part[1] = fma(bf16_bits_to_f64(xv[r].x >> 16), bb[1 * DOT_GROUPS], part[1]);
-      part[2] = fma(bf16_bits_to_f64(xv[r].y & 0xFFFFu), bb[2 * DOT_GROUPS], part[2]);
-      part[3] = fma(bf16_bits_to_f64(xv[r].y >> 16), bb[3 * DOT_GROUPS], part[3]);
-      part[4] = fma(bf16_bits_to_f64(xv[r].z & 0xFFFFu), bb[4 * DOT_GROUPS], part[4]);
-      part[5] = fma(bf16_bits_to_f64(xv[r].z >> 16), bb[5 * DOT_GROUPS], part[5]);
-      part[6] = fma(bf16_bits_to_f64(xv[r].w & 0xFFFFu), bb[6 * DOT_GROUPS], part[6]);
-      part[7] = fma(bf16_bits_to_f64(xv[r].w >> 16), bb[7 * DOT_GROUPS], part[7]);
-    }
-  }
-  return ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
-}
-
 // x . w over a 6,144-dim row in fp64 by one warp, x (fp64) in shared memory and w fp32 in
 // global memory, lanes strided.
 __device__ __forceinline__ double smem_dot_lane(const double *xs, const float *w, int lane) {
@@ -880,36 +851,69 @@ __device__ __forceinline__ double smem_dot_lane(const double *xs, const float *w
   return (part[0] + part[1]) + (part[2] + part[3]);
 }
 
+// x . b over a 6,144-dim row in fp64 by one warp, x the caller's bf16 row and b an fp32
+// column, both read from global memory: lane l takes the 16-byte groups l, l + 32, ... of x
+// (8 elements) and the two float4 of b under each; the products are exact in fp64 and go
+// into eight partial sums (one per element of a group), added in a fixed order.
+__device__ __forceinline__ double row_dot_glb(const uint4 *xr, const float4 *b, int lane) {
+  constexpr int R = ROW_DIM / 8 / 32;  // 24 groups per lane
+  constexpr int Q = 6;                 // groups loaded together
+  double part[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) part[u] = 0.0;
+#pragma unroll
+  for (int q0 = 0; q0 < R; q0 += Q) {
+    uint4 xv[Q];
+    float4 b0[Q], b1[Q];
+#pragma unroll
+    for (int r = 0; r < Q; ++r) {
+      const int g = (q0 + r) * 32 + lane;
+      xv[r] = __ldg(xr + g);
+      b0[r] = __ldg(b + 2 * g);
+      b1[r] = __ldg(b + 2 * g + 1);
+    }
+#pragma unroll
+    for (int r = 0; r < Q; ++r) {
+      part[0] = fma(bf16_bits_to_f64(xv[r].x & 0xFFFFu), (double)b0[r].x, part[0]);
+      part[1] = fma(bf16_bits_to_f64(xv[r].x >> 16), (double)b0[r].y, part[1]);
+      part[2] = fma(bf16_bits_to_f64(xv[r].y & 0xFFFFu), (double)b0[r].z, part[2]);
+      part[3] = fma(bf16_bits_to_f64(xv[r].y >> 16), (double)b0[r].w, part[3]);
+      part[4] = fma(bf16_bits_to_f64(xv[r].z & 0xFFFFu), (double)b1[r].x, part[4]);
+      part[5] = fma(bf16_bits_to_f64(xv[r].z >> 16), (double)b1[r].y, part[5]);
+      part[6] = fma(bf16_bits_to_f64(xv[r].w & 0xFFFFu), (double)b1[r].z, part[6]);
+      part[7] = fma(bf16_bits_to_f64(xv[r].w >> 16), (double)b1[r].w, part[7]);
+    }
+  }
+  return ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
+}
+
 // Exact recomputation of codes near a half-step boundary.  The transform's epilogue bins
-// them by component.  A work item is up to eight rows of one component's bin: the block
-// puts basis[:, c] into shared memory as fp64 and each warp takes one row:
+// them by component; codes are numbered by a prefix sum over the bins (each block computes
+// it for itself) and every warp takes one code at a time:
 // y = x . basis[:, c] - (mu basis)[c] + g . w2[:, c] in fp64 (x the caller's bf16 row, the
-// mean term fp64-accumulated at codec creation, g the correction's hidden units as their
-// fp16 hi/lo pair), q = round(y / Delta_c).  Items are numbered by a prefix sum over the
-// bins (each block computes it for itself) and spread over the grid, so a crowded bin is
-// shared by many blocks.  Lane partial sums are added by a butterfly in a fixed order, so
-// the result is deterministic.
-constexpr int REFINE_THREADS = 256;
-constexpr int REFINE_ITEM_ROWS = REFINE_THREADS / 32;
-constexpr int REFINE_SMEM = ROW_DIM * 8 + (N_COEF + 1) * 4;
+// basis column fp32, the mean term fp64-accumulated at codec creation, g the correction's
+// hidden units as their fp16 hi/lo pair), q = round(y / Delta_c).  Consecutive codes share
+// their component, so the warps of a block read the same basis column, mostly from L1.
+// Lane partial sums are added by a butterfly in a fixed order, so the result is
+// deterministic.
+constexpr int REFINE_THREADS = 512;
+constexpr int REFINE_SMEM = ROW_DIM * 8 + (N_COEF + 1) * 4;  // the whole-row kernels' shared memory
 
 __global__ void __launch_bounds__(REFINE_THREADS) k_refine_codes(
     const uint32_t *el_bins, const uint32_t *bin_count, uint32_t bin_cap, const __nv_bfloat16 *rows,
     const int32_t *row_tok, const double *mub64, const float *bt32, const float *w2t32, const __half *g16,
     const float *delta, const uint32_t *rowflag, const int16_t *kept_list, int32_t *q32, __nv_bfloat16 *qe,
     const int32_t *row_edst) {
-  extern __shared__ __align__(16) double bs[];
-  uint32_t *item0 = reinterpret_cast<uint32_t *>(bs + ROW_DIM);  // [2049] first item of each bin
+  __shared__ uint32_t code0[N_COEF + 1];  // first code of each bin
   __shared__ uint32_t warp_tot[REFINE_THREADS / 32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  // items per bin, exclusive prefix sum: thread t owns bins 8t .. 8t + 7
+  // codes per bin, exclusive prefix sum: thread t owns bins PER t .. PER t + PER - 1
   {
     constexpr int PER = N_COEF / REFINE_THREADS;
     uint32_t cnt[PER], run = 0;
 #pragma unroll
     for (int u = 0; u < PER; ++u) {
-      const uint32_t n = min(bin_count[threadIdx.x * PER + u], bin_cap);
-      cnt[u] = (n + REFINE_ITEM_ROWS - 1) / REFINE_ITEM_ROWS;
+      cnt[u] = min(bin_count[threadIdx.x * PER + u], bin_cap);
       run += cnt[u];
     }
     uint32_t incl = run;
@@ -924,53 +928,39 @@ __global__ void __launch_bounds__(REFINE_THREADS) k_refine_codes(
     for (int w = 0; w < warp; ++w) base += warp_tot[w];
 #pragma unroll
     for (int u = 0; u < PER; ++u) {
-      item0[threadIdx.x * PER + u] = base;
+      code0[threadIdx.x * PER + u] = base;
       base += cnt[u];
     }
-    if (threadIdx.x == REFINE_THREADS - 1) item0[N_COEF] = base;
+    if (threadIdx.x == REFINE_THREADS - 1) code0[N_COEF] = base;
     __syncthreads();
   }
-  const uint32_t n_items = item0[N_COEF];
-  for (uint32_t item = blockIdx.x; item < n_items; item += gridDim.x) {
-    int lo = 0, hi = N_COEF;  // the bin holding this item: item0[lo] <= item < item0[lo + 1]
+  const uint32_t n_codes = code0[N_COEF];
+  const uint32_t n_warps = gridDim.x * (REFINE_THREADS / 32);
+  for (uint32_t t = blockIdx.x * (REFINE_THREADS / 32) + warp; t < n_codes; t += n_warps) {
+    int lo = 0, hi = N_COEF;  // the bin holding this code: code0[lo] <= t < code0[lo + 1]
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;
-      if (item0[mid] <= item) lo = mid; else hi = mid;
+      if (code0[mid] <= t) lo = mid; else hi = mid;
     }
-    const int m = lo;               // compact component index of the bin
-    const int c = kept_list[m];     // the component
-    const uint32_t n = min(bin_count[m], bin_cap);
-    const float4 *bt = reinterpret_cast<const float4 *>(bt32 + (int64_t)c * ROW_DIM);
-    for (int i = threadIdx.x; i < ROW_DIM / 4; i += blockDim.x) {  // elements 4 i .. 4 i + 3
-      const float4 v = __ldg(bt + i);
-      double *d = bs + (i & 1) * 4 * DOT_GROUPS + (i >> 1);  // group i / 2, j = 4 (i % 2) + t
-      d[0] = v.x;
-      d[DOT_GROUPS] = v.y;
-      d[2 * DOT_GROUPS] = v.z;
-      d[3 * DOT_GROUPS] = v.w;
-    }
-    __syncthreads();
-    const uint32_t k = (item - item0[m]) * REFINE_ITEM_ROWS + warp;
-    if (k < n) {
-      const int64_t row = el_bins[(int64_t)m * bin_cap + k];
-      if (!rowflag[row]) {  // rows listed for whole-row recomputation are left to k_refine_rows
-        double acc = row_dot_smem(reinterpret_cast<const uint4 *>(rows + (int64_t)row_tok[row] * ROW_DIM), bs, lane);
-        if (w2t32) {  // the correction (absent in a linear codec): eight hidden units per lane
-          const __half *g = g16 + row * (2 * N_HIDDEN);
-          const float *w = w2t32 + (int64_t)c * N_HIDDEN;
-          double h = 0.0;
+    const int m = lo;  // compact component index of the bin
+    const int64_t row = el_bins[(int64_t)m * bin_cap + (t - code0[m])];
+    if (rowflag[row]) continue;  // rows listed for whole-row recomputation are left to k_refine_rows
+    const int c = kept_list[m];
+    double acc = row_dot_glb(reinterpret_cast<const uint4 *>(rows + (int64_t)row_tok[row] * ROW_DIM),
+                             reinterpret_cast<const float4 *>(bt32 + (int64_t)c * ROW_DIM), lane);
+    if (w2t32) {  // the correction (absent in a linear codec): eight hidden units per lane
+      const __half *g = g16 + row * (2 * N_HIDDEN);
+      const float *w = w2t32 + (int64_t)c * N_HIDDEN;
+      double h = 0.0;
 #pragma unroll
-          for (int u = 0; u < N_HIDDEN / 32; ++u) {
-            const int j = u * 32 + lane;
-            h += ((double)__half2float(g[j]) + (double)__half2float(g[N_HIDDEN + j])) * (double)w[j];
-          }
-          acc += h;
-        }
-        acc = warp_sum(acc) - mub64[c];
-        if (lane == 0) store_code(row, m, acc / (double)delta[c], q32, qe, row_edst);
+      for (int u = 0; u < N_HIDDEN / 32; ++u) {
+        const int j = u * 32 + lane;
+        h += ((double)__half2float(g[j]) + (double)__half2float(g[N_HIDDEN + j])) * (double)w[j];
       }
+      acc += h;
     }
-    __syncthreads();
+    acc = warp_sum(acc) - mub64[c];
+    if (lane == 0) store_code(row, m, acc / (double)delta[c], q32, qe, row_edst);
   }
 }
 
@@ -1736,10 +1726,9 @@ static int encode_impl(const dckv_codec *c, const void *rows, const int32_t *tok
     }
     stage_mark(c, st, "gemm_transform");
     // codes whose fp32 ratio lies in the guard band around a half step: exact fp64 values
-    CK(cudaFuncSetAttribute(k_refine_codes, cudaFuncAttributeMaxDynamicSharedMemorySize, REFINE_SMEM));
     CK(cudaFuncSetAttribute(k_refine_hidden, cudaFuncAttributeMaxDynamicSharedMemorySize, REFINE_SMEM));
     CK(cudaFuncSetAttribute(k_refine_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, REFINE_SMEM));
-    { k_refine_codes<<<c->num_sms * 3, REFINE_THREADS, REFINE_SMEM, st>>>(
+    { k_refine_codes<<<c->num_sms * 2, REFINE_THREADS, 0, st>>>(
           el_bins, bin_count, w.bin_cap, (const __nv_bfloat16 *)rows, row_tok, c->mub64, c->bt32,
           c->has_mlp ? c->w2t32 : nullptr, g16, c->delta, rowflag, c->kept_list, q32, qe, row_edst);
       ++g_launches; }
