@@ -1,7 +1,7 @@
 """DCKV codec benchmark on B200: encode + decode throughput of the codec hot path.
 
 python bench.py [--gpus N] [--steps K] [--warmup W] [--impl dckv|reference]
-                [--config c5|c1|c2|c3|c3b|c4|c5p|c2lin|c2syn] [--profile] [--fit]
+                [--config c5|c1|c2|c3|c3b|c4|c5p|c5h|c2lin|c2syn] [--profile] [--fit]
 
 A step is one pass of the whole codec hot path over one batch: encode (transform GEMMs,
 quantiser, mean models, rANS, compaction) then decode (two rANS passes, odd mean model,
@@ -42,6 +42,9 @@ CONFIGS = {
                                          "rows, ~220 B/token"),
     "c5p": ([4096] * 8, 220.0, 0.01, 16, "8 x 4096-token prompts, 1% Student-t (nu=2) rows, ~220 B/token "
                                          "(an eighth of the 64-prompt batch, rows above L2: the profiling case)"),
+    "c5h": ([4096] * 16, 220.0, 0.01, 16, "16 x 4096-token prompts, 1% Student-t (nu=2) rows, ~220 B/token "
+                                          "(a quarter of the 64-prompt batch: profiling case of the kernels "
+                                          "that large batches take)"),
     "c2lin": ([4096], 220.0, 0.0, 16, "1 x 4096-token prompt, linear codec (no correction, unconditional "
                                       "zero-mean tables), ~220 B/token"),
     "c2syn": ([4096], 220.0, 0.0, 16, "1 x 4096-token prompt, ~220 B/token, decoder-side synthesis MLP "
