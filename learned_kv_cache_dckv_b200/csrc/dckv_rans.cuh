@@ -549,6 +549,7 @@ struct DecLane {
   uint32_t w0, w1, w2;  // word ring: lane j holds words wb + j, wb + 32 + j, wb + 64 + j
   uint32_t wb, wp;      // ring base, words consumed
   int k;                // kept component of this lane's next symbol
+  int s;                // its scale, loaded a step ahead (off the state's dependency chain)
 };
 
 // One decode step of all 32 lanes: symbol i = 32 t + lane.  CHECK: some lanes may lie
@@ -563,7 +564,7 @@ __device__ __forceinline__ void dec_step(DecLane &d, uint32_t i, uint32_t S, int
   if (valid) {
     const uint32_t slot = d.x & 0xFFFFu;
     uint32_t c, f;
-    const int sym = find_symbol(slot, s_scale[d.k], s_cdf, s_lut, s_tail, c, f);
+    const int sym = find_symbol(slot, d.s, s_cdf, s_lut, s_tail, c, f);
     d.x = f * (d.x >> 16) + slot - c;
     need = d.x < RANS_L;
     out[i] = (uint16_t)sym;
@@ -588,6 +589,7 @@ __device__ __forceinline__ void dec_step(DecLane &d, uint32_t i, uint32_t S, int
     d.k += 32;
     while (d.k >= K) d.k -= K;
   }
+  d.s = s_scale[d.k];
 }
 
 // One warp decodes chunk ci: states, escape count and word stream from its section.
@@ -619,6 +621,7 @@ __device__ __forceinline__ void decode_chunk(const RansDecArgs &a, int ci, int l
   d.w1 = 32u + lane < n_wd ? wd[32 + lane] : 0u;
   d.w2 = 64u + lane < n_wd ? wd[64 + lane] : 0u;
   d.k = K > 0 ? lane % K : 0;
+  d.s = s_scale[d.k];
   bool bad = d.x < RANS_L;
   int t = 0;
   for (; t + 16 <= T_full && !bad; t += 16) {
