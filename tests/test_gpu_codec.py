@@ -51,6 +51,9 @@ def gpu_codec(np_codec, chunk_rows=0):
 
 def make_batch(src, cod, lens, seeds, boost=(), boost_gain=60.0, student_t=0.0):
     x, tok, offs = S.batch(src, lens, seeds, student_t_frac=student_t, device="cuda")
+    vocab = cod.embed.shape[0] if cod.embed is not None else 0
+    if vocab > S.VOCAB:  # every third token from the rows past the synthetic vocabulary
+        tok[::3] = S.VOCAB + tok[::3] % (vocab - S.VOCAB)
     if boost:
         mu = torch.from_numpy(cod.mu).cuda()
         idx = torch.tensor(list(boost), device="cuda")
@@ -372,6 +375,19 @@ def test_parity_centres_escapes_and_big_codes(src, codec_centred):
     # rows pushed far out: escapes beyond +-127 and codes beyond the fp16-exact 2048
     full_check(src, codec_centred, [132 + 90, 132 + 41, 140], seeds=[11, 12, 13], chunk_rows=8,
                boost=(4, 9, 30, 60, 223 + 4, 223 + 50), boost_gain=400.0, expect_escapes=True, expect_big=True)
+
+
+def test_parity_token_ids_past_2_16(src, codec_centred):
+    """A vocabulary of 70,000 rows, every third token id at or above 2^16: the even-centre
+    and odd tables are indexed by token id times their row stride, so these ids take the
+    tables' upper rows (and 64-bit offsets at the largest vocabularies)."""
+    import copy
+
+    cod = copy.copy(codec_centred)
+    extra = np.random.default_rng(99).standard_normal((70000 - S.VOCAB, cod.embed.shape[1])).astype(np.float32)
+    cod.embed = np.concatenate([cod.embed, S.f32_to_bf16_bits(extra)], axis=0)
+    r = full_check(src, cod, [132 + 300, 132 + 77], seeds=[21, 22], chunk_rows=8)
+    assert (r["tok"].cpu().numpy() >= 1 << 16).sum() > 100
 
 
 def test_parity_student_t_rows(src, codec_55):
