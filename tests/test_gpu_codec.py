@@ -52,8 +52,8 @@ def gpu_codec(np_codec, chunk_rows=0):
 def make_batch(src, cod, lens, seeds, boost=(), boost_gain=60.0, student_t=0.0):
     x, tok, offs = S.batch(src, lens, seeds, student_t_frac=student_t, device="cuda")
     vocab = cod.embed.shape[0] if cod.embed is not None else 0
-    if vocab > S.VOCAB:  # every third token from the rows past the synthetic vocabulary
-        tok[::3] = S.VOCAB + tok[::3] % (vocab - S.VOCAB)
+    if vocab > 1 << 16:  # every third token id from the vocabulary's rows at and past 2^16
+        tok[::3] = (1 << 16) + tok[::3] % (vocab - (1 << 16))
     if boost:
         mu = torch.from_numpy(cod.mu).cuda()
         idx = torch.tensor(list(boost), device="cuda")
