@@ -1835,14 +1835,18 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
   CK(cudaMemsetAsync(status_dev, 0, 4, st));
   CK(cudaMemsetAsync(counters, 0, 256, st));
   RET(upload_tables(c, L, ws, w, st));
-  CK(cudaMemset2DAsync(qe, 2ull * CODE_LD, 0, 2ull * c->kw, (size_t)L.ne_pad, st));
-  if (L.n_rows) {
-    CK(cudaMemset2DAsync(q16, 2ull * CODE_LD, 0, 2ull * c->kw, (size_t)L.n_rows, st));
-    CK(cudaMemsetAsync(bigflag, 0, 4ull * L.n_rows, st));
+  // every kept code of every row is written below (escapes by the patch); only the pad
+  // columns K_eff .. kw - 1, which the GEMMs read against zero operands, and each prompt's
+  // zero right-neighbour row (by k_layout) are cleared here
+  if (c->kw > c->k_eff) {
+    CK(cudaMemset2DAsync(qe + c->k_eff, 2ull * CODE_LD, 0, 2ull * (c->kw - c->k_eff), (size_t)L.ne_pad, st));
+    if (L.n_rows)
+      CK(cudaMemset2DAsync(q16 + c->k_eff, 2ull * CODE_LD, 0, 2ull * (c->kw - c->k_eff), (size_t)L.n_rows, st));
   }
+  if (L.n_rows) CK(cudaMemsetAsync(bigflag, 0, 4ull * L.n_rows, st));
   if (L.n_chunks) CK(cudaMemsetAsync(ws + w.escflag, 0, 4ull * L.n_chunks, st));
   { k_layout<<<dim3(L.batch, LAYOUT_SPLIT), 256, 0, st>>>(d_prompts, row_tok, row_pos, row_edst, row_slot, e_tok, e_slot, e_row, slot_chunk,
-                                    c->chunk_rows, nullptr, c->kw); ++g_launches; }
+                                    c->chunk_rows, qe, c->kw); ++g_launches; }
   HeaderCheck hc{bl, blob_bytes, d_prompts, L.batch, c->chunk_rows, c->k_eff, L.n_chunks_e, L.n_chunks_o,
                  L.n_kept, L.off_kept, L.off_streams, valid, status_dev};
   { k_check_header<<<1, 256, 0, st>>>(hc); ++g_launches; }
