@@ -211,6 +211,20 @@ static int run_gemm2_chunked(const CUtensorMap &a0, const CUtensorMap &a1, const
 }
 
 
+// Token-tile width of a CTA-pair GEMM with m_pairs feature tiles of 256: 256 tokens, unless
+// 192-token tiles fill the last wave of pairs so much better that it pays for their smaller
+// MMA work per staged byte (measured: 25-30% more time per token than 256-token tiles).
+// The transform of a single 4,096-token prompt (16 token tiles x 7 feature tiles = 112
+// tiles on 74 pairs, against 21 x 7 = 147) takes 192: 193 -> 183 us.
+static int pick_pair_bn(int64_t n_rows, int m_pairs, int num_sms) {
+  const int64_t pairs = std::max(1, num_sms / 2);
+  auto cost = [&](int64_t bn, double per_token) {
+    const int64_t tiles = (n_rows + bn - 1) / bn * m_pairs;
+    return (double)((tiles + pairs - 1) / pairs) * (double)bn * per_token;
+  };
+  return cost(192, 1.28) < cost(256, 1.0) ? 192 : 256;
+}
+
 static GemmProblem make_problem(int m_tiles, int64_t n_rows, int bn, bool bf16, int32_t *status) {
   GemmProblem p;
   memset(&p, 0, sizeof(p));
@@ -1686,8 +1700,9 @@ static int encode_impl(const dckv_codec *c, const void *rows, const int32_t *tok
   if (L.n_rows > 0) {
     CUtensorMap mb_xh, mb_xt, mb_gt, mb_qe;
     RET(map_b(&mb_xh, x16, false, ROW_DIM, L.n_rows, HIDDEN_SPLIT_BN / 2));
-    RET(map_b(&mb_xt, x16, false, ROW_DIM, L.n_rows, TRANSFORM_BN / 2));
-    RET(map_b(&mb_gt, g16, false, 2 * N_HIDDEN, L.n_rows, TRANSFORM_BN / 2));
+    const int bn_t = pick_pair_bn(L.n_rows, c->mp / 256, c->num_sms);  // transform token tile
+    RET(map_b(&mb_xt, x16, false, ROW_DIM, L.n_rows, bn_t / 2));
+    RET(map_b(&mb_gt, g16, false, 2 * N_HIDDEN, L.n_rows, bn_t / 2));
     RET(map_b(&mb_qe, qe, true, c->kw, L.ne_pad, MEAN_ODD_BN / 2, CODE_LD));
     // correction hidden layer: h = x @ w1 - mu @ w1, GELU, fp16 hi/lo
     if (c->has_mlp && (L.n_rows + HIDDEN_SPLIT_BN - 1) / HIDDEN_SPLIT_BN >= c->num_sms) {
@@ -1711,7 +1726,7 @@ static int encode_impl(const dckv_codec *c, const void *rows, const int32_t *tok
     stage_mark(c, st, "gemm_hidden");
     // transform + quantiser: y = x @ B + g @ w2 - mu @ B
     {
-      GemmProblem pr = make_problem(c->mp / GEMM_BM, L.n_rows, TRANSFORM_BN, false, status_dev);
+      GemmProblem pr = make_problem(c->mp / GEMM_BM, L.n_rows, bn_t, false, status_dev);
       add_seg(pr, 0, 0, 2, 0, 0, 0, 0, ROW_DIM / GEMM_BK);
       if (c->has_mlp) {  // + g @ w2 (hi/lo on both sides)
         add_seg(pr, 1, 0, 2, 0, 1, 0, 0, N_HIDDEN / GEMM_BK);
@@ -1721,8 +1736,12 @@ static int encode_impl(const dckv_codec *c, const void *rows, const int32_t *tok
                                row_edst},
                               row_norm, rowflag, el_bins, bin_count, full_list, counters, w.bin_cap,
                               c->dbg_ratio, c->kept_list};
-      RET((run_gemm2_chunked<EpiQuantRegs, 4, 2, TRANSFORM_CHUNK_STEPS, TRANSFORM_BN>(c->map_ay2, c->map_aw2_2, mb_xt, mb_gt, pr, ep,
-                                                                   c->num_sms, false, st)));
+      if (bn_t == TRANSFORM_BN)
+        RET((run_gemm2_chunked<EpiQuantRegs, 4, 2, TRANSFORM_CHUNK_STEPS, TRANSFORM_BN>(
+            c->map_ay2, c->map_aw2_2, mb_xt, mb_gt, pr, ep, c->num_sms, false, st)));
+      else
+        RET((run_gemm2_chunked<EpiQuantRegs, 4, 2, TRANSFORM_CHUNK_STEPS, 192>(
+            c->map_ay2, c->map_aw2_2, mb_xt, mb_gt, pr, ep, c->num_sms, false, st)));
     }
     stage_mark(c, st, "gemm_transform");
     // codes whose fp32 ratio lies in the guard band around a half step: exact fp64 values
@@ -1921,13 +1940,14 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
   }
   if (L.n_rows > 0) {
     CUtensorMap mb_q, mb_g;
-    RET(map_b(&mb_q, q16, false, c->kw, L.n_rows, INVERSE_BN / 2, CODE_LD));
-    GemmProblem pr = make_problem(ROW_DIM / GEMM_BM, L.n_rows, INVERSE_BN, false, status_dev);
+    const int bn_i = pick_pair_bn(L.n_rows, ROW_DIM / 256, c->num_sms);  // inverse token tile
+    RET(map_b(&mb_q, q16, false, c->kw, L.n_rows, bn_i / 2, CODE_LD));
+    GemmProblem pr = make_problem(ROW_DIM / GEMM_BM, L.n_rows, bn_i, false, status_dev);
     // hi and lo halves up to the cut, the hi half alone after it (second A map, one slab)
     if (c->inv_lo_k > 0) add_seg(pr, 0, 0, 2, 0, 0, 0, 0, c->inv_lo_k / GEMM_BK);
     if (c->inv_lo_k < c->kw) add_seg(pr, 1, 0, 1, c->inv_lo_k, 0, 0, c->inv_lo_k, (c->kw - c->inv_lo_k) / GEMM_BK);
     if (c->has_synth) {  // + g V2 (hi/lo on both sides)
-      RET(map_b(&mb_g, g16d, false, 2 * N_HIDDEN, L.n_rows, INVERSE_BN / 2));
+      RET(map_b(&mb_g, g16d, false, 2 * N_HIDDEN, L.n_rows, bn_i / 2));
       add_seg(pr, 1, 0, 2, 0, 1, 0, 0, N_HIDDEN / GEMM_BK);
       add_seg(pr, 1, 0, 2, 0, 1, 0, N_HIDDEN, N_HIDDEN / GEMM_BK);
     } else {

@@ -53,9 +53,10 @@ constexpr float REFINE_NORM_FULL = 32.0f;
 // a wider B tile carries more MMA work per byte moved into shared memory, which is what
 // keeps the tensor pipe fed (measured against 224: transform -8%, inverse and odd mean
 // model -12% on 64 x 4,096 tokens).
+// (The transform and the inverse take 192-token tiles instead where these fill the last
+// wave of pairs better: pick_pair_bn.)
 constexpr int TRANSFORM_BN = 256;
 constexpr int MEAN_ODD_BN = 256;
-constexpr int INVERSE_BN = 256;
 // Hidden layers (256 rows of M, one pair tile): the decoder's synthesis layer runs narrow
 // 64-token tiles (62 pairs for a 4K-token prompt); the encoder's correction layer, K = 6,144,
 // runs 256-token tiles with K cut into HIDDEN_SPLIT parts.  A batch with fewer token tiles
