@@ -49,6 +49,8 @@ struct GemmProblem {
   int *status;  // device int32; DCKV_ETIMEOUT (5) is written on a timed-out wait
   int k_split;  // CTA-pair kernel, one segment: K cut into k_split parts, each its own tile
                 // (the epilogue writes part ks of the sum; 0 or 1: no split)
+  int first_chunk;  // chunk-accumulated kernel: K steps of a tile's first TMEM partial (0: the
+                    // kernel's CHUNK_STEPS, like every later partial)
 };
 
 // What an epilogue sees of one output tile.  The epilogue threads form groups of 128 (four
@@ -601,7 +603,11 @@ __global__ void __launch_bounds__(GEMM2C_THREADS, 1)
   uint32_t n_issued = 0;  // items this CTA's producer (thread 0) issued
   int ksteps = 0;
   for (int si = 0; si < prob.n_seg; ++si) ksteps += prob.seg[si].k_steps;
-  const int n_chunks = (ksteps + CHUNK_STEPS - 1) / CHUNK_STEPS;
+  // a tile's partials: the first takes first_steps K steps, every later one CHUNK_STEPS.  The
+  // MMA can run as far ahead of the epilogue as the first two partials reach, so a longer
+  // first partial hides more of the previous tile's finishing epilogue.
+  const int first_steps = min(ksteps, prob.first_chunk > 0 ? prob.first_chunk : CHUNK_STEPS);
+  const int n_chunks = ksteps > 0 ? 1 + (ksteps - first_steps + CHUNK_STEPS - 1) / CHUNK_STEPS : 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -681,7 +687,7 @@ __global__ void __launch_bounds__(GEMM2C_THREADS, 1)
       uint32_t pph = 0;
       bool ok = true;
       for (int t = pair; t < total_tiles && ok; t += n_pairs) {
-        int in_chunk = 0, done = 0;
+        int in_chunk = 0, done = 0, chunk_len = first_steps;
         uint32_t d_tmem = 0, accumulate = 0;
         for (int si = 0; si < prob.n_seg && ok; ++si) {
           const GemmSeg sg = prob.seg[si];
@@ -716,9 +722,10 @@ __global__ void __launch_bounds__(GEMM2C_THREADS, 1)
               phase ^= 1u;
             }
             ++done;
-            if (++in_chunk == CHUNK_STEPS || done == ksteps) {
+            if (++in_chunk == chunk_len || done == ksteps) {
               umma_commit_pair(&part_full[pb]);
               in_chunk = 0;
+              chunk_len = CHUNK_STEPS;
               if (++pb == 2) {
                 pb = 0;
                 pph ^= 1u;
