@@ -42,12 +42,6 @@ constexpr uint16_t LUT_SINGLE = 0x4000;       // the bucket lies inside one symb
 constexpr uint16_t LUT_MULTI = 0x8000;        // two or more symbol boundaries in the bucket
 constexpr uint16_t LUT_SYM = 0x03FF;
 
-__device__ __forceinline__ void copy_smem16(void *dst, const void *src, int bytes) {
-  const uint4 *s = reinterpret_cast<const uint4 *>(src);
-  uint4 *d = reinterpret_cast<uint4 *>(dst);
-  for (int i = threadIdx.x; i < bytes / 16; i += blockDim.x) d[i] = s[i];
-}
-
 __device__ __forceinline__ uint32_t cdf_at(const uint16_t *tab, int k) { return k < N_SYM ? tab[k] : PREC_TOTAL; }
 
 // ------------------------------------------------------------------------------ symbols
@@ -534,13 +528,6 @@ __device__ __forceinline__ bool bulk_load_tables(uint8_t *sm, const uint16_t *dc
     }
   }
   return mbar_wait(bar, 0, abort_flag);
-}
-
-__device__ __forceinline__ void load_tables(uint8_t *sm, const uint16_t *dcdf, const uint16_t *lut,
-                                            const uint32_t *tail) {
-  copy_smem16(sm, dcdf, CDF_SMEM_BYTES);
-  copy_smem16(sm + CDF_SMEM_BYTES, lut, LUT_SMEM_BYTES);
-  copy_smem16(sm + CDF_SMEM_BYTES + LUT_SMEM_BYTES, tail, TAIL_SMEM_BYTES);
 }
 
 // State of one warp decoding one chunk.
