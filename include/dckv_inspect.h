@@ -29,7 +29,7 @@ extern "C" {
  *        components in ascending order;
  *   sym16 uint16 [n_rows][K_eff] symbols in the same order;
  *   row_slot int32 [n_rows].
- * After dckv_decode: q16 fp16 [n_rows][2048] decoded codes (exact below 2048), qe, cen8.
+ * After dckv_decode: q16 fp16 [n_rows][2048] decoded codes (exact below 2048), qe.
  * Encode recomputes in fp64 every code whose fp32 ratio y / Delta lies in a guard band
  * around a half-step boundary (whole rows when the row's norm is large). */
 typedef struct {

@@ -1878,13 +1878,6 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
   CK(cudaGetLastError());
   stage_mark(c, st, "layout+check");
   const uint32_t *offs = (const uint32_t *)(bl + HEADER_BYTES + 4ull * L.batch);
-  if (L.n_rows > 0 && c->has_means) {
-    k_centres_even<<<(unsigned)std::min<int64_t>(L.n_rows, 65535), 256, 0, st>>>(
-        L.n_rows, row_slot, row_edst, row_tok, token_ids, c->t_even8, c->kw, c->vocab, c->k_eff, cen8, valid);
-    ++g_launches;
-  } else if (L.n_symbols > 0) {
-    CK(cudaMemsetAsync(cen8, 0, (size_t)L.n_symbols, st));  // unconditional tables: every centre 0
-  }
   CK(cudaFuncSetAttribute(rans_decode_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, RANS_DEC_SMEM));
   CK(cudaFuncSetAttribute(rans_decode_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, RANS_DEC_SMEM));
   RansDecArgs da{d_chunks, 0, L.n_chunks, c->k_eff, c->kept_scale, c->dcdf, c->lut, c->tail, bl, L.off_streams,
@@ -1904,7 +1897,8 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
   CK(cudaGetLastError());
   stage_mark(c, st, "rans_loop");
   if (L.n_chunks_e > 0) {
-    { k_codes_elem<<<rg, 256, 0, st>>>(0, L.n_rows, row_edst, row_slot, slot_chunk, syms16, cen8,
+    { k_codes_elem<<<rg, 256, 0, st>>>(0, L.n_rows, row_edst, row_slot, slot_chunk, syms16,
+                                       c->has_means ? c->t_even8 : nullptr, c->kw, token_ids, row_tok, c->vocab,
                                        c->k_eff, q16, qe, escflag, valid); ++g_launches; }
     { k_escape_patch<<<(unsigned)L.n_chunks_e, PATCH_THREADS, 0, st>>>(fa); ++g_launches; }
   }
@@ -1924,7 +1918,8 @@ extern "C" int dckv_decode(const dckv_codec *c, const void *blob, size_t blob_by
   stage_mark(c, st, "gemm_mean_odd");
   if (L.n_chunks_o > 0) {
     if (!c->has_means)  // unconditional tables: every odd centre is 0
-      { k_codes_elem<<<rg, 256, 0, st>>>(1, L.n_rows, row_edst, row_slot, slot_chunk, syms16, cen8,
+      { k_codes_elem<<<rg, 256, 0, st>>>(1, L.n_rows, row_edst, row_slot, slot_chunk, syms16, nullptr, c->kw,
+                                         token_ids, row_tok, c->vocab,
                                          c->k_eff, q16, qe, escflag, valid); ++g_launches; }
     fa.chunk0 = L.n_chunks_e;
     fa.n_chunks = L.n_chunks_o;

@@ -45,34 +45,6 @@ constexpr uint16_t LUT_SYM = 0x03FF;
 __device__ __forceinline__ uint32_t cdf_at(const uint16_t *tab, int k) { return k < N_SYM ? tab[k] : PREC_TOTAL; }
 
 // ------------------------------------------------------------------------------ symbols
-// Centres of even rows for the decoder, in slot order: the row of the even-centre table
-// (clamp(round(T_even[token][c]), +-127), kept components, computed at codec creation).
-__global__ void __launch_bounds__(256) k_centres_even(int64_t n_rows, const int32_t *row_slot,
-                                                      const int32_t *row_edst, const int32_t *row_tok,
-                                                      const int32_t *tok_ids, const int8_t *t_even8, int t_ld,
-                                                      int vocab, int k_eff, int8_t *cen8, const int32_t *valid) {
-  if (valid && *valid != 1) return;
-  for (int64_t row = blockIdx.x; row < n_rows; row += gridDim.x) {
-    if (row_edst[row] < 0) continue;
-    int tok = tok_ids[row_tok[row]];
-    tok = min(max(tok, 0), vocab - 1);
-    const int8_t *te = t_even8 + (int64_t)tok * t_ld;
-    int8_t *dst = cen8 + (int64_t)row_slot[row] * k_eff;
-    constexpr int PER = N_COEF / 256;  // blockDim.x == 256: every load before the stores
-    int8_t v[PER];
-#pragma unroll
-    for (int u = 0; u < PER; ++u) {
-      const int k = threadIdx.x + 256 * u;
-      v[u] = k < k_eff ? te[k] : (int8_t)0;
-    }
-#pragma unroll
-    for (int u = 0; u < PER; ++u) {
-      const int k = threadIdx.x + 256 * u;
-      if (k < k_eff) dst[k] = v[u];
-    }
-  }
-}
-
 // Encoder inputs in slot order: the symbol (ESC if |q| > 127 else q - centre + 254), its
 // table entry {cdf | (freq - 1) << 16, division multiplier of freq} (from the codec's
 // packed per-(scale, symbol) table), and the escape count of each chunk.  Four positions
@@ -659,7 +631,9 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1) rans_decode_kernel(RansDecA
 
 // Finishing a decoded pass in two steps.  k_codes_elem writes code = centre + symbol - 254
 // for every symbol of the pass's rows, fully parallel (fp16 to q16; even rows also bf16 to
-// qe, the odd mean model's input); an ESC symbol only flags its chunk.  (The odd pass of a
+// qe, the odd mean model's input); an ESC symbol only flags its chunk.  An even row's
+// centres are its token's row of the even-centre table (kept components, read in place);
+// without mean models every centre is 0.  (The odd pass of a
 // codec with mean models gets the same from the odd mean GEMM's epilogue.)  k_escape_patch
 // then visits the chunks that store escape values or hold a flagged ESC, ranks the ESC
 // symbols in symbol order (escape values are stored in that order), writes those codes,
@@ -667,7 +641,8 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 1) rans_decode_kernel(RansDecA
 // lies within 127 + 254), and checks that every escape value is used exactly once.
 __global__ void __launch_bounds__(256) k_codes_elem(int parity, int64_t n_rows, const int32_t *row_edst,
                                                     const int32_t *row_slot, const int32_t *slot_chunk,
-                                                    const uint16_t *syms, const int8_t *cen8,
+                                                    const uint16_t *syms, const int8_t *t_even8, int t_ld,
+                                                    const int32_t *tok_ids, const int32_t *row_tok, int vocab,
                                                     int k_eff, __half *q16,
                                                     __nv_bfloat16 *qe, uint32_t *escflag, const int32_t *valid) {
   if (*valid != 1) return;
@@ -677,13 +652,14 @@ __global__ void __launch_bounds__(256) k_codes_elem(int parity, int64_t n_rows, 
     if ((e >= 0) != (parity == 0)) continue;  // block-uniform
     const int64_t slot = row_slot[r];
     const uint16_t *sy = syms + slot * k_eff;
-    const int8_t *ce = cen8 + slot * k_eff;
+    const int8_t *ce = (e >= 0 && t_even8) ? t_even8 + (int64_t)min(max(tok_ids[row_tok[r]], 0), vocab - 1) * t_ld
+                                           : nullptr;
     int sv[PER], cv[PER];
 #pragma unroll
     for (int u = 0; u < PER; ++u) {  // every load before the stores
       const int k = threadIdx.x + 256 * u;
       sv[u] = k < k_eff ? (int)__ldg(sy + k) : 0;
-      cv[u] = k < k_eff ? (int)__ldg(ce + k) : 0;
+      cv[u] = (k < k_eff && ce) ? (int)__ldg(ce + k) : 0;
     }
     bool esc = false;
 #pragma unroll
