@@ -647,34 +647,52 @@ __global__ void __launch_bounds__(256) k_codes_elem(int parity, int64_t n_rows, 
                                                     __nv_bfloat16 *qe, uint32_t *escflag, const int32_t *valid) {
   if (*valid != 1) return;
   constexpr int PER = N_COEF / 256;  // blockDim.x == 256
-  for (int64_t r = blockIdx.x; r < n_rows; r += gridDim.x) {
-    const int e = row_edst[r];
-    if ((e >= 0) != (parity == 0)) continue;  // block-uniform
-    const int64_t slot = row_slot[r];
-    const uint16_t *sy = syms + slot * k_eff;
-    const int8_t *ce = (e >= 0 && t_even8) ? t_even8 + (int64_t)min(max(tok_ids[row_tok[r]], 0), vocab - 1) * t_ld
-                                           : nullptr;
+  // a block's rows are r, r + grid, ...: the next row's metadata (its even index, slot and,
+  // for an even row, its token's table row) is fetched while this row's symbols load
+  auto tab_row = [&](int64_t r, int e) -> const int8_t * {
+    return (e >= 0 && t_even8) ? t_even8 + (int64_t)min(max(tok_ids[row_tok[r]], 0), vocab - 1) * t_ld : nullptr;
+  };
+  int64_t r = blockIdx.x;
+  int e = r < n_rows ? row_edst[r] : -1;
+  int64_t slot = r < n_rows ? row_slot[r] : 0;
+  const int8_t *ce = r < n_rows ? tab_row(r, e) : nullptr;
+  while (r < n_rows) {
+    const int64_t rn = r + gridDim.x;
+    const bool has_next = rn < n_rows;
+    const int e_n = has_next ? row_edst[rn] : -1;
+    const int64_t slot_n = has_next ? row_slot[rn] : 0;
+    const bool mine = (e >= 0) == (parity == 0);  // block-uniform
     int sv[PER], cv[PER];
+    if (mine) {
+      const uint16_t *sy = syms + slot * k_eff;
 #pragma unroll
-    for (int u = 0; u < PER; ++u) {  // every load before the stores
-      const int k = threadIdx.x + 256 * u;
-      sv[u] = k < k_eff ? (int)__ldg(sy + k) : 0;
-      cv[u] = (k < k_eff && ce) ? (int)__ldg(ce + k) : 0;
-    }
-    bool esc = false;
-#pragma unroll
-    for (int u = 0; u < PER; ++u) {
-      const int k = threadIdx.x + 256 * u;
-      if (k >= k_eff) continue;
-      if (sv[u] == ESC_SYM) {
-        esc = true;
-        continue;
+      for (int u = 0; u < PER; ++u) {  // every load before the stores
+        const int k = threadIdx.x + 256 * u;
+        sv[u] = k < k_eff ? (int)__ldg(sy + k) : 0;
+        cv[u] = (k < k_eff && ce) ? (int)__ldg(ce + k) : 0;
       }
-      const int q = sv[u] - R_MAX + cv[u];
-      q16[r * CODE_LD + k] = __float2half_rn((float)q);
-      if (e >= 0) qe[(int64_t)e * CODE_LD + k] = __float2bfloat16_rn((float)q);
     }
-    if (__syncthreads_or(esc) && threadIdx.x == 0) escflag[slot_chunk[slot]] = 1u;
+    const int8_t *ce_n = has_next && (e_n >= 0) == (parity == 0) ? tab_row(rn, e_n) : nullptr;
+    if (mine) {
+      bool esc = false;
+#pragma unroll
+      for (int u = 0; u < PER; ++u) {
+        const int k = threadIdx.x + 256 * u;
+        if (k >= k_eff) continue;
+        if (sv[u] == ESC_SYM) {
+          esc = true;
+          continue;
+        }
+        const int q = sv[u] - R_MAX + cv[u];
+        q16[r * CODE_LD + k] = __float2half_rn((float)q);
+        if (e >= 0) qe[(int64_t)e * CODE_LD + k] = __float2bfloat16_rn((float)q);
+      }
+      if (__syncthreads_or(esc) && threadIdx.x == 0) escflag[slot_chunk[slot]] = 1u;
+    }
+    r = rn;
+    e = e_n;
+    slot = slot_n;
+    ce = ce_n;
   }
 }
 
